@@ -1,0 +1,354 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself -- a hand-worked example, a closed form, a library routine, brute force
+or an invariant -- chosen so that a dropped term, a wrong sign or index, or a
+transposed operand in the oracle fails at least one of them.
+
+Passages: CLSA article, sections 研究の背景と課題 (top-k keeps the k
+highest-scoring tokens; sparse attention attends only to them) and CLSAの仕組み
+(one index set, computed once, reused by every cross-decoder layer); Louver
+summary, sections 問題定義 and 1. 半空間範囲検索への帰着 (keep every key with
+<q,k> >= tau, with no false negatives)."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+# --------------------------------------------------------------------------
+# Hand-worked example (tests/golden/hand_worked_tiny.json)
+# --------------------------------------------------------------------------
+
+@pytest.fixture(scope="module")
+def hand():
+    with open(os.path.join(GOLDEN, "hand_worked_tiny.json")) as f:
+        return json.load(f)
+
+
+def test_hand_worked_scores_topk_threshold(hand):
+    q = np.array(hand["q_route"], np.float32)
+    K = np.array(hand["K"], np.float32)
+    S = oracle.scores(q, K)
+    np.testing.assert_array_equal(S, np.array(hand["expected_scores"], np.float32))
+    for k, want in hand["expected_topk"].items():
+        np.testing.assert_array_equal(oracle.topk(S, int(k)), np.array(want))
+    for case in hand["expected_threshold"]:
+        idx, cnt = oracle.threshold(S, np.array([[case["tau"]]], np.float32), cap=5)
+        assert int(cnt[0, 0]) == len(case["idx"])
+        assert list(idx[0, 0, :cnt[0, 0]]) == case["idx"]
+
+
+def test_hand_worked_attention(hand):
+    K = np.array(hand["K"], np.float32)
+    V = np.array(hand["V"], np.float32)
+    ql = np.zeros((1, 1, 2, 4), np.float32)
+    ql[0, 0, 0, 0] = np.float32(2 * math.log(2))
+    idx = np.array(hand["expected_topk"]["2"], np.int32)
+    out, lse = oracle.attn(ql, K, V, idx)
+    exp = hand["expected_attn_top2"]
+    np.testing.assert_allclose(out[0, 0], np.array(exp["out"]), atol=exp["tol"])
+    np.testing.assert_allclose(lse[0, 0], [math.log(12), math.log(2)], atol=exp["tol"])
+
+
+# --------------------------------------------------------------------------
+# Scores
+# --------------------------------------------------------------------------
+
+def _einsum_scores_f64(q, K, G):
+    """Group-summed scores by library einsum in fp64 with the key heads
+    repeated over their query groups (torch/numpy GQA convention)."""
+    Krep = np.repeat(K.astype(np.float64), G, axis=1)          # [B,Hq,N,d]
+    per_head = np.einsum("bgd,bgnd->bgn", q.astype(np.float64), Krep)
+    B, Hq, N = per_head.shape
+    return per_head.reshape(B, Hq // G, G, N).sum(axis=2) / math.sqrt(q.shape[-1])
+
+
+@pytest.mark.parametrize("B,N,Hq,Hkv,d", [(2, 37, 6, 2, 16), (1, 200, 8, 2, 64),
+                                          (3, 19, 4, 4, 8), (1, 50, 8, 1, 128)])
+def test_scores_vs_library_einsum(B, N, Hq, Hkv, d):
+    r = _rng(B * 1000 + N)
+    q = r.standard_normal((B, Hq, d), dtype=np.float32)
+    K = r.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    ref = _einsum_scores_f64(q, K, Hq // Hkv)
+    S64 = oracle.scores(q, K, np.float64)
+    np.testing.assert_allclose(S64, ref, rtol=1e-12, atol=1e-12)
+    # fp32 summation error bound: n * u * sum|terms| with n = G*d + 2.
+    Krep = np.repeat(np.abs(K.astype(np.float64)), Hq // Hkv, axis=1)
+    mag = np.einsum("bgd,bgnd->bgn", np.abs(q.astype(np.float64)), Krep)
+    mag = mag.reshape(B, Hkv, Hq // Hkv, N).sum(axis=2) / math.sqrt(d)
+    bound = ((Hq // Hkv) * d + 2) * 2.0 ** -24 * mag + 1e-30
+    S32 = oracle.scores(q, K)
+    assert np.all(np.abs(S32 - ref) <= bound)
+
+
+def test_scores_integer_inputs_exact():
+    """Small integers: every product and partial sum is exact in fp32 and
+    the scale 1/sqrt(64) = 1/8 is a power of two, so the result is exact."""
+    r = _rng(7)
+    q = r.integers(-3, 4, size=(2, 8, 64)).astype(np.float32)
+    K = r.integers(-3, 4, size=(2, 2, 33, 64)).astype(np.float32)
+    G = 4
+    exact = np.einsum("bgd,bgnd->bgn", q.astype(np.int64),
+                      np.repeat(K.astype(np.int64), G, axis=1))
+    exact = exact.reshape(2, 2, G, 33).sum(axis=2)
+    np.testing.assert_array_equal(oracle.scores(q, K), (exact / 8.0).astype(np.float32))
+
+
+def test_scores_head_mapping_contiguous_groups():
+    """Only query head 5 is non-zero; with G=4 it belongs to KV head 1, whose
+    keys are one-hot, so S[:,1,j] = q[5, c_j] / sqrt(d) and KV head 0 is 0."""
+    d, N = 16, 10
+    q = np.zeros((1, 8, d), np.float32)
+    q[0, 5] = np.arange(1, d + 1, dtype=np.float32)
+    K = np.zeros((1, 2, N, d), np.float32)
+    cols = (np.arange(N) * 3) % d
+    K[0, 1, np.arange(N), cols] = 1.0
+    K[0, 0] = 1.0
+    S = oracle.scores(q, K)
+    np.testing.assert_array_equal(S[0, 0], np.zeros(N, np.float32))
+    np.testing.assert_array_equal(S[0, 1], ((cols + 1) / 4.0).astype(np.float32))
+
+
+def test_scores_power_of_two_scaling_and_key_permutation():
+    r = _rng(3)
+    q = r.standard_normal((1, 4, 32), dtype=np.float32)
+    K = r.standard_normal((1, 1, 64, 32), dtype=np.float32)
+    S = oracle.scores(q, K)
+    np.testing.assert_array_equal(oracle.scores(2 * q, K), 2 * S)
+    perm = r.permutation(64)
+    np.testing.assert_array_equal(oracle.scores(q, K[:, :, perm]), S[:, :, perm])
+
+
+# --------------------------------------------------------------------------
+# Top-k
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,k,levels", [(64, 7, None), (1000, 100, 17),
+                                        (500, 499, 3), (300, 1, None)])
+def test_topk_vs_stable_argsort(N, k, levels):
+    r = _rng(N + k)
+    S = r.standard_normal((3, N)).astype(np.float32)
+    if levels:  # force many exact ties
+        S = np.round(S * levels / 4).astype(np.float32)
+    got = oracle.topk(S, k)
+    for row in range(3):
+        want = np.sort(np.argsort(-S[row], kind="stable")[:k])
+        np.testing.assert_array_equal(got[row], want)
+
+
+def test_topk_bruteforce_all_subsets():
+    """Integer scores with ties, N <= 10: the set with the largest sum,
+    ties between sets broken by the lexicographically smallest index tuple
+    (which is the lower-index tie rule at the k-th score)."""
+    r = _rng(11)
+    for trial in range(30):
+        N = int(r.integers(1, 11))
+        S = r.integers(-2, 3, size=(1, N)).astype(np.float32)
+        for k in range(1, N + 1):
+            best = max(itertools.combinations(range(N), k),
+                       key=lambda c: (S[0, list(c)].sum(), [-i for i in c]))
+            np.testing.assert_array_equal(oracle.topk(S, k)[0], np.array(best))
+
+
+def test_topk_special_cases():
+    S = np.full((2, 50), 0.25, np.float32)
+    np.testing.assert_array_equal(oracle.topk(S, 9), np.tile(np.arange(9), (2, 1)))
+    r = _rng(5)
+    S = r.standard_normal((2, 40)).astype(np.float32)
+    np.testing.assert_array_equal(oracle.topk(S, 40), np.tile(np.arange(40), (2, 1)))
+    # -0.0 and +0.0 are the same score: the lower index wins
+    S = np.array([[-1.0, 0.0, -0.0, -0.0, 0.0]], np.float32)
+    S[0, 2] = -0.0
+    np.testing.assert_array_equal(oracle.topk(S, 2), [[1, 2]])
+    # permutation of distinct scores permutes the set
+    S = r.permutation(1000).astype(np.float32)[None]
+    perm = r.permutation(1000)
+    base = set(oracle.topk(S, 30)[0])
+    got = set(oracle.topk(S[:, perm], 30)[0])
+    assert {int(perm[j]) for j in got} == base
+
+
+# --------------------------------------------------------------------------
+# Threshold
+# --------------------------------------------------------------------------
+
+def test_threshold_special_cases():
+    r = _rng(9)
+    S = r.standard_normal((2, 300)).astype(np.float32)
+    tau = S.max(axis=1) + 1
+    idx, cnt = oracle.threshold(S, tau, cap=300)
+    assert cnt.tolist() == [0, 0]
+    idx, cnt = oracle.threshold(S, S.min(axis=1), cap=300)
+    assert cnt.tolist() == [300, 300]
+    np.testing.assert_array_equal(idx, np.tile(np.arange(300), (2, 1)))
+    # tau = k-th largest of distinct scores -> exactly the top-k set
+    k = 37
+    kth = -np.sort(-S, axis=1)[:, k - 1]
+    idx, cnt = oracle.threshold(S, kth, cap=300)
+    assert cnt.tolist() == [k, k]
+    np.testing.assert_array_equal(idx[:, :k], oracle.topk(S, k))
+    # capacity overflow: true count, lowest indices written
+    idx, cnt = oracle.threshold(S, S.min(axis=1), cap=10)
+    assert cnt.tolist() == [300, 300]
+    np.testing.assert_array_equal(idx, np.tile(np.arange(10), (2, 1)))
+
+
+def test_threshold_no_false_negatives_against_fp64():
+    r = _rng(21)
+    q = r.standard_normal((1, 8, 64), dtype=np.float32)
+    K = r.standard_normal((1, 2, 5000, 64), dtype=np.float32)
+    S = oracle.scores(q, K)
+    S64 = oracle.scores(q, K, np.float64)
+    tau = oracle.percentile_tau(S, 97, 100)
+    idx, cnt = oracle.threshold(S, tau, cap=5000)
+    for h in range(2):
+        band = 1e-4 * abs(float(tau[0, h])) + 1e-6
+        sel = set(idx[0, h, :cnt[0, h]].tolist())
+        must = set(np.nonzero(S64[0, h] >= tau[0, h] + band)[0].tolist())
+        never = set(np.nonzero(S64[0, h] < tau[0, h] - band)[0].tolist())
+        assert must <= sel and not (never & sel)
+
+
+def test_percentile_tau_matches_numpy_inverted_cdf():
+    r = _rng(4)
+    S = r.standard_normal((3, 131)).astype(np.float32)
+    tau = oracle.percentile_tau(S, 97, 100)
+    for row in range(3):
+        want = np.percentile(S[row], 97, method="inverted_cdf")
+        assert tau[row] == np.float32(want)
+    # nearest rank at the headline length: ceil(0.97 * 131072) = 127140, so
+    # 131072 - 127139 = 3933 distinct scores are >= tau
+    S = r.permutation(131072).astype(np.float32)[None]
+    tau = oracle.percentile_tau(S, 97, 100)
+    assert float(tau[0]) == 127139.0
+    assert int(oracle.threshold(S, tau, cap=131072)[1][0]) == 3933
+
+
+# --------------------------------------------------------------------------
+# Attention over the selected set
+# --------------------------------------------------------------------------
+
+def _sdpa_f64(q, K, V):
+    """torch scaled_dot_product_attention in fp64 with GQA repetition.
+    q [B,Hq,d] (one query per head), K,V [B,Hkv,n,d]."""
+    qt = torch.from_numpy(q.astype(np.float64))[:, :, None, :]
+    Kt = torch.from_numpy(K.astype(np.float64))
+    Vt = torch.from_numpy(V.astype(np.float64))
+    G = q.shape[1] // K.shape[1]
+    Kt = Kt.repeat_interleave(G, dim=1)
+    Vt = Vt.repeat_interleave(G, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt)
+    logits = (qt @ Kt.transpose(-1, -2))[:, :, 0, :] / math.sqrt(q.shape[-1])
+    return o[:, :, 0, :].numpy(), torch.logsumexp(logits, dim=-1).numpy()
+
+
+@pytest.mark.parametrize("B,N,Hq,Hkv,d", [(1, 300, 8, 2, 64), (2, 57, 4, 1, 32),
+                                          (1, 129, 32, 8, 128)])
+def test_attn_all_selected_equals_dense_sdpa(B, N, Hq, Hkv, d):
+    r = _rng(N)
+    q = r.standard_normal((B, Hq, d), dtype=np.float32)
+    K = r.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    V = r.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    idx = np.tile(np.arange(N, dtype=np.int32), (B, Hkv, 1))
+    out, lse = oracle.attn(q, K, V, idx)
+    o_ref, lse_ref = _sdpa_f64(q, K, V)
+    np.testing.assert_allclose(out, o_ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_attn_subset_equals_dense_on_gathered_rows():
+    r = _rng(77)
+    B, Hq, Hkv, N, d, c = 2, 8, 2, 400, 64, 33
+    q = r.standard_normal((B, Hq, d), dtype=np.float32)
+    K = r.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    V = r.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    idx = np.stack([np.stack([np.sort(r.choice(N, c, replace=False))
+                              for _ in range(Hkv)]) for _ in range(B)]).astype(np.int32)
+    out, lse = oracle.attn(q, K, V, idx)
+    Kg = np.take_along_axis(K, idx[..., None].astype(np.int64), axis=2)
+    Vg = np.take_along_axis(V, idx[..., None].astype(np.int64), axis=2)
+    o_ref, lse_ref = _sdpa_f64(q, Kg, Vg)
+    np.testing.assert_allclose(out, o_ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_attn_single_key_and_constant_values():
+    r = _rng(8)
+    q = r.standard_normal((1, 4, 16), dtype=np.float32)
+    K = r.standard_normal((1, 1, 20, 16), dtype=np.float32)
+    V = r.standard_normal((1, 1, 20, 16), dtype=np.float32)
+    out, _ = oracle.attn(q, K, V, np.array([[[13]]], np.int32))
+    np.testing.assert_array_equal(out[0], np.tile(V[0, 0, 13].astype(np.float64), (4, 1)))
+    Vc = np.tile(np.linspace(-2, 2, 16, dtype=np.float32), (1, 1, 20, 1))
+    idx = np.array([[[1, 4, 9, 16]]], np.int32)
+    out, _ = oracle.attn(q, K, Vc, idx)
+    np.testing.assert_allclose(out[0], np.tile(Vc[0, 0, 0], (4, 1)), atol=1e-14)
+
+
+def test_attn_weights_are_softmax_and_sum_to_one():
+    """V rows are one-hot (row t of the selection -> e_t), so o equals the
+    softmax weights; compared with scipy's softmax of the logits."""
+    r = _rng(12)
+    d, c, N = 32, 20, 60
+    q = r.standard_normal((1, 2, d), dtype=np.float32)
+    K = r.standard_normal((1, 1, N, d), dtype=np.float32)
+    sel = np.sort(r.choice(N, c, replace=False)).astype(np.int32)
+    V = np.zeros((1, 1, N, d), np.float32)
+    V[0, 0, sel, np.arange(c)] = 1.0
+    out, lse = oracle.attn(q, K, V, sel[None, None])
+    logits = (q[0].astype(np.float64) @ K[0, 0, sel].astype(np.float64).T) / math.sqrt(d)
+    np.testing.assert_allclose(out[0][:, :c], scipy.special.softmax(logits, axis=1),
+                               rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(out[0].sum(axis=1), 1.0, atol=1e-12)
+    np.testing.assert_allclose(lse[0], scipy.special.logsumexp(logits, axis=1), atol=1e-12)
+
+
+def test_attn_empty_and_partial_counts():
+    r = _rng(13)
+    q = r.standard_normal((1, 4, 8), dtype=np.float32)
+    K = r.standard_normal((1, 2, 10, 8), dtype=np.float32)
+    V = r.standard_normal((1, 2, 10, 8), dtype=np.float32)
+    idx = np.array([[[0, 1, 2, 3], [5, 6, 7, 8]]], np.int32)
+    out, lse = oracle.attn(q, K, V, idx, count=np.array([[0, 2]], np.int32))
+    assert np.all(out[0, :2] == 0) and np.all(np.isneginf(lse[0, :2]))
+    o2, l2 = oracle.attn(q[:, 2:], K[:, 1:], V[:, 1:], idx[:, 1:, :2])
+    np.testing.assert_array_equal(out[0, 2:], o2[0])
+    np.testing.assert_array_equal(lse[0, 2:], l2[0])
+
+
+# --------------------------------------------------------------------------
+# The decode step: one routing set shared by every layer
+# --------------------------------------------------------------------------
+
+def test_decode_step_routes_once_and_shares_the_set():
+    r = _rng(31)
+    B, N, Hq, Hkv, d, L, k = 1, 700, 8, 2, 64, 3, 50
+    qr = r.standard_normal((B, Hq, d), dtype=np.float32)
+    ql = r.standard_normal((L, B, Hq, d), dtype=np.float32)
+    K = r.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    V = r.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    res = oracle.decode_step(qr, ql, K, V, k=k)
+    np.testing.assert_array_equal(res["idx"], oracle.topk(oracle.scores(qr, K), k))
+    for layer in range(L):
+        Kg = np.take_along_axis(K, res["idx"][..., None].astype(np.int64), axis=2)
+        Vg = np.take_along_axis(V, res["idx"][..., None].astype(np.int64), axis=2)
+        o_ref, lse_ref = _sdpa_f64(ql[layer], Kg, Vg)
+        np.testing.assert_allclose(res["out"][layer], o_ref, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(res["lse"][layer], lse_ref, atol=1e-12)
+    # nearest rank: tau is the ceil(0.9 * 700) = 630th smallest score, so
+    # 700 - 630 + 1 = 71 distinct scores are kept per head
+    tau = oracle.percentile_tau(res["S"], 90, 100)
+    th = oracle.decode_step(qr, ql, K, V, tau=tau, cap=N)
+    assert th["count"].tolist() == [[71, 71]]

@@ -1,0 +1,58 @@
+"""Host checks of the seeded input generator (no method arithmetic in it)."""
+import numpy as np
+import torch
+
+from token_sparse_attention_sm_b200 import synth
+
+
+def test_deterministic_and_subset_consistent():
+    w = synth.custom(B=3, N=300, Hq=8, Hkv=2, d=64, L=2, k=8, heavy=5,
+                     outlier=True, seed=4)
+    a = synth.generate(w)
+    b = synth.generate(w)
+    for key in a:
+        assert torch.equal(a[key], b[key])
+    sub = synth.generate(w, batches=[2])
+    for key in ("q_route", "K", "V", "outlier", "heavy_pos"):
+        assert torch.equal(sub[key][0], a[key][2])
+    assert torch.equal(sub["q_layers"][:, 0], a["q_layers"][:, 2])
+
+
+def test_heavy_hitters_and_outlier_channel():
+    w = synth.custom(B=1, N=500, Hq=8, Hkv=2, d=64, L=1, k=8, heavy=7,
+                     outlier=True, seed=0)
+    x = synth.generate(w)
+    qf = x["q_route"].float().numpy()[0]
+    for h in range(2):
+        pos = x["heavy_pos"][0, h].numpy()
+        assert len(set(pos.tolist())) == 7 and pos.min() >= 0 and pos.max() < 500
+        qbar = qf[4 * h:4 * h + 4].mean(axis=0)
+        unit = 4 * qbar / np.linalg.norm(qbar)
+        rows = x["K"][0, h, pos].float().numpy()
+        assert np.abs(rows - unit).max() < 0.6          # 0.1-sigma noise
+        c = int(x["outlier"][0, h])
+        others = np.delete(np.arange(500), pos)
+        kc = x["K"][0, h, others, c].float().numpy()
+        assert 6 < kc.std() < 10                          # x8 channel
+        assert 0.8 < np.delete(x["K"][0, h, others].float().numpy(), c, axis=1).std() < 1.2
+
+
+def test_dtypes_and_rounding():
+    w = synth.custom(B=1, N=64, Hq=4, Hkv=1, d=64, L=1, k=4, dtype="bf16")
+    x = synth.generate(w)
+    assert x["K"].dtype == torch.bfloat16
+    f = synth.f32(x["K"])
+    assert f.dtype == np.float32
+    assert np.array_equal(torch.from_numpy(f).to(torch.bfloat16).float().numpy(), f)
+    w32 = w.with_(dtype="f32")
+    assert synth.generate(w32)["K"].dtype == torch.float32
+
+
+def test_named_workloads_shapes():
+    w = synth.WORKLOADS["decode_128k"]
+    assert (w.B, w.N, w.Hq, w.Hkv, w.d, w.L, w.k) == (1, 131072, 32, 8, 128, 16, 2048)
+    assert w.outlier and w.heavy == 256
+    t = synth.WORKLOADS["threshold_128k"]
+    assert t.mode == "threshold" and t.cap == 8192 and t.stride == 8192
+    bt = synth.WORKLOADS["batched_16x64k"]
+    assert bt.seeds == tuple(range(1, 17))
