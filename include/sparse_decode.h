@@ -1,0 +1,192 @@
+/*
+ * sparse_decode.h -- C ABI of the shared-routing token-sparse decode
+ * attention library for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (page title, section):
+ *  - CLSA article "CLSAとは？ルーティング共有で128Kコンテキスト推論を17倍高速化する
+ *    スパースアテンション", section 研究の背景と課題: token-level sparse
+ *    attention attends only to the k highest-scoring cached tokens;
+ *  - same page, section CLSAの仕組み: the top-k routing set is computed once
+ *    per query token over the one shared (YOCO) KV cache, and every
+ *    cross-decoder layer reuses that set unchanged;
+ *  - same page, section 計算コストの削減効果: routing costs one pass over the
+ *    context per step instead of one per layer;
+ *  - Louver summary "技術サマリー：スパースアテンションを範囲検索問題として捉える",
+ *    sections 問題定義 and 1. 半空間範囲検索への帰着: the threshold variant keeps
+ *    every key whose score is >= tau (the halfspace {p : <q,p> >= tau}),
+ *    with no false negatives and a set size that varies per query.
+ *
+ * Definitions used by every entry point:
+ *  - G = Hq / Hkv query heads share one KV head; query head hq reads KV head
+ *    hq / G (contiguous groups).
+ *  - Routing score of key j for KV head h of sequence b:
+ *        S[b,h,j] = (sum over the G query heads g of h: <q[b,g,:], K[b,h,j,:]>)
+ *                   / sqrt(d), accumulated in fp32.
+ *  - Top-k set: the k keys with the largest S; at equal S the lower key
+ *    index wins; -0.0 and +0.0 are equal.  Threshold set: every j with
+ *    S[b,h,j] >= tau[b,h] (inclusive, tau in the units of S).  Sets are
+ *    returned in ascending key order.
+ *  - Attention of query vector x over a set I of keys of head h:
+ *        z_j = <x, K[b,h,j,:]> / sqrt(d),  o = sum_j softmax(z)_j V[b,h,j,:],
+ *        lse = log sum_j exp(z_j); fp32 softmax and accumulation; o is
+ *    written in the input dtype (round to nearest even).  An empty set gives
+ *    o = 0 and lse = -inf.
+ *
+ * Layouts: every tensor is dense and row-major in the order shown.
+ *    q, q_route [B,Hq,d]      q_layers [L,B,Hq,d]      K, V [B,Hkv,N,d]
+ *    S [B,Hkv,N] fp32         tau [B,Hkv] fp32         count [B,Hkv] int32
+ *    idx [B,Hkv,stride] int32 out [L,B,Hq,d]           lse [L,B,Hq] fp32
+ * q/K/V/out share one dtype (fp32 or bf16).  All pointers are device
+ * pointers owned by the caller; the library allocates nothing and keeps no
+ * per-call state.  q, K, V, S and out must be 16-byte aligned.
+ *
+ * Supported: d in {64, 128}; dtype fp32 or bf16; 1 <= G <= 16; N >= 1;
+ * B*Hkv <= 65535; L*G <= 1024.
+ *
+ * Errors: argument problems are returned synchronously, before anything is
+ * enqueued.  Conditions only the device can see (a non-finite score, a
+ * threshold set larger than its capacity, an index outside [0,N), a bounded
+ * wait that expired) are OR-ed into a status word kept in the workspace and
+ * read back with sparse_read_device_status().  Kernels never trap.
+ *
+ * Workspace: every compute entry point takes (ws, ws_bytes); ws_bytes must
+ * be at least sparse_workspace_size() for the same arguments.  The
+ * workspace must be zero-filled once before its first use (for example with
+ * sparse_workspace_init); the library leaves it reusable afterwards.  Calls
+ * that share a workspace must be ordered (same stream, or synchronised).
+ *
+ * Asynchrony: every compute entry point enqueues its kernels on `stream`
+ * and returns without synchronising.
+ */
+#ifndef SPARSE_DECODE_H_
+#define SPARSE_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPARSE_OK = 0,
+  SPARSE_ERR_INVALID_ARG = 1, /* null pointer, bad size, misalignment */
+  SPARSE_ERR_UNSUPPORTED = 2, /* d, dtype or G outside the supported set */
+  SPARSE_ERR_WORKSPACE = 3,   /* ws_bytes smaller than required */
+  SPARSE_ERR_CAPACITY = 4,    /* device: a threshold set exceeded cap */
+  SPARSE_ERR_NONFINITE = 5,   /* device: a score (or tau) was NaN/Inf */
+  SPARSE_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
+  SPARSE_ERR_TIMEOUT = 7,     /* device: a bounded wait expired */
+  SPARSE_ERR_INDEX = 8,       /* device: an idx entry was outside [0,N) */
+  SPARSE_ERR_INTERNAL = 9     /* device: an internal consistency check failed */
+} sparse_status_t;
+
+typedef enum { SPARSE_DTYPE_F32 = 0, SPARSE_DTYPE_BF16 = 1 } sparse_dtype_t;
+
+typedef struct {
+  int32_t B;     /* sequences */
+  int32_t N;     /* cached tokens per sequence */
+  int32_t Hq;    /* query heads */
+  int32_t Hkv;   /* KV heads; Hq % Hkv == 0 */
+  int32_t d;     /* head dimension */
+  int32_t dtype; /* sparse_dtype_t of q, K, V and out */
+} sparse_shape_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *sparse_status_string(sparse_status_t status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t sparse_version(void);
+
+/* Bytes of workspace needed by every entry point for this shape, where
+ * k_or_cap is the top-k size or threshold capacity (the idx stride) and L
+ * the number of query sets (layers) attended per call.  Synchronous. */
+sparse_status_t sparse_workspace_size(const sparse_shape_t *shape,
+                                      int32_t k_or_cap, int32_t L,
+                                      size_t *bytes);
+
+/* Zero-fill the workspace (enqueued on stream). */
+sparse_status_t sparse_workspace_init(void *ws, size_t ws_bytes,
+                                      void *stream);
+
+/* Routing scores only: S[b,h,j] as defined above, for every cached key
+ * (CLSA article, section 研究の背景と課題: the score that decides which
+ * tokens matter).  One streaming pass over K. */
+sparse_status_t sparse_score(const sparse_shape_t *shape, const void *q,
+                             const void *K, float *S, void *ws,
+                             size_t ws_bytes, void *stream);
+
+/* Top-k selection from given scores S [B,Hkv,N] (shape->Hq, d and dtype are
+ * ignored): idx [B,Hkv,k] ascending, ties to the lower index (CLSA
+ * article, section 研究の背景と課題).  1 <= k <= N. */
+sparse_status_t sparse_select_topk(const sparse_shape_t *shape,
+                                   const float *S, int32_t k, int32_t *idx,
+                                   void *ws, size_t ws_bytes, void *stream);
+
+/* Threshold selection from given scores: every j with S >= tau[b,h]
+ * (Louver summary, section 1. 半空間範囲検索への帰着).  count[b,h] receives
+ * the true set size; the lowest min(count, cap) indices are written to
+ * idx [B,Hkv,cap] in ascending order.  A set larger than cap raises
+ * SPARSE_ERR_CAPACITY in the device status. */
+sparse_status_t sparse_select_threshold(const sparse_shape_t *shape,
+                                        const float *S, const float *tau,
+                                        int32_t cap, int32_t *idx,
+                                        int32_t *count, void *ws,
+                                        size_t ws_bytes, void *stream);
+
+/* Shared routing, top-k form: scores of q [B,Hq,d] against every key of K,
+ * then the top-k set per (b, KV head) into idx [B,Hkv,k] (CLSA article,
+ * section CLSAの仕組み: computed once, reused by all layers). */
+sparse_status_t sparse_route_topk(const sparse_shape_t *shape, const void *q,
+                                  const void *K, int32_t k, int32_t *idx,
+                                  void *ws, size_t ws_bytes, void *stream);
+
+/* Shared routing, threshold form (Louver summary, sections 問題定義 and
+ * 1. 半空間範囲検索への帰着): as sparse_select_threshold on the scores of q. */
+sparse_status_t sparse_route_threshold(const sparse_shape_t *shape,
+                                       const void *q, const void *K,
+                                       const float *tau, int32_t cap,
+                                       int32_t *idx, int32_t *count, void *ws,
+                                       size_t ws_bytes, void *stream);
+
+/* Sparse attention over a given index set (CLSA article, section
+ * 研究の背景と課題: attention restricted to the selected tokens).
+ * q holds L query sets [L,B,Hq,d] (L = 1 for one layer); every set attends
+ * over the same idx rows [B,Hkv,stride]; count [B,Hkv] gives the valid
+ * prefix of each row (NULL: all stride entries; counts above stride are
+ * clamped to stride).  Writes out [L,B,Hq,d] (dtype) and, if lse is not
+ * NULL, lse [L,B,Hq]. */
+sparse_status_t sparse_attn_gather(const sparse_shape_t *shape, int32_t L,
+                                   const void *q, const void *K,
+                                   const void *V, const int32_t *idx,
+                                   int32_t stride, const int32_t *count,
+                                   void *out, float *lse, void *ws,
+                                   size_t ws_bytes, void *stream);
+
+/* One fused decode step (CLSA article, sections CLSAの仕組み and
+ * 計算コストの削減効果): route once with q_route [B,Hq,d], then run the
+ * attention of all L layers' queries q_layers [L,B,Hq,d] over that one set.
+ *   top-k mode:     k >= 1, tau == NULL, count may be NULL; idx [B,Hkv,k].
+ *   threshold mode: k == 0, tau [B,Hkv] and count [B,Hkv] given, cap >= 1;
+ *                   idx [B,Hkv,cap]; each layer uses min(count, cap) keys.
+ * out [L,B,Hq,d]; lse [L,B,Hq] or NULL. */
+sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
+                                   const void *q_route, const void *q_layers,
+                                   const void *K, const void *V, int32_t k,
+                                   const float *tau, int32_t cap,
+                                   int32_t *idx, int32_t *count, void *out,
+                                   float *lse, void *ws, size_t ws_bytes,
+                                   void *stream);
+
+/* Synchronise `stream`, read the device status word of ws, reset it to
+ * zero, and return the most severe condition recorded since the last read
+ * (TIMEOUT > INTERNAL > INDEX > NONFINITE > CAPACITY > OK).  *flags (if not NULL)
+ * receives the raw bit set. */
+sparse_status_t sparse_read_device_status(void *ws, void *stream,
+                                          uint32_t *flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_DECODE_H_ */

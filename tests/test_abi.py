@@ -1,0 +1,118 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol
+the header declares, and rejects bad arguments on the host before any device
+work (so these checks need no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import token_sparse_attention_sm_b200 as sd
+from token_sparse_attention_sm_b200 import build as sd_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sparse_decode.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sd_build.build()
+    return sd.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(sparse_[a-z_]+)\s*\(", text)))
+
+
+def test_header_symbols_are_exported(lib):
+    declared = _declared()
+    assert set(declared) == set(sd.EXPORTED_SYMBOLS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in sd.STATUS_NAMES.items():
+        assert lib.sparse_status_string(code).decode().startswith(name)
+    assert lib.sparse_version() >= 100
+
+
+def _shape(**kw):
+    base = dict(B=1, N=4096, Hq=8, Hkv=2, d=64, dtype=1)
+    base.update(kw)
+    return sd._Shape(**base)
+
+
+def _ws_size(lib, sh, k=16, L=2):
+    n = ctypes.c_size_t(0)
+    rc = lib.sparse_workspace_size(ctypes.byref(sh), k, L, ctypes.byref(n))
+    return rc, n.value
+
+
+def test_workspace_size_validation(lib):
+    rc, n = _ws_size(lib, _shape())
+    assert rc == 0 and n >= 256 + 2 * 4096 * 4
+    assert _ws_size(lib, _shape(Hq=7))[0] == 1          # Hq % Hkv
+    assert _ws_size(lib, _shape(d=96))[0] == 2          # unsupported d
+    assert _ws_size(lib, _shape(dtype=7))[0] == 2
+    assert _ws_size(lib, _shape(Hq=34, Hkv=2))[0] == 2  # G = 17 > 16
+    assert _ws_size(lib, _shape(N=0))[0] == 1
+    assert _ws_size(lib, _shape(), k=0)[0] == 1
+    assert _ws_size(lib, _shape(), L=0)[0] == 1
+    assert _ws_size(lib, _shape(Hq=16, Hkv=1), L=65)[0] == 2  # L*G > 1024
+
+
+def test_bad_arguments_rejected_before_device_work(lib):
+    sh = _shape()
+    fake = ctypes.c_void_p(0x10000)      # never dereferenced: checks come first
+    odd = ctypes.c_void_p(0x10008)       # not 16-byte aligned
+    ws_ok = ctypes.c_void_p(0x100000)
+    rc, need = _ws_size(lib, sh, k=16, L=1)
+    # null pointers
+    assert lib.sparse_route_topk(ctypes.byref(sh), None, fake, 16, fake, ws_ok,
+                                 need, None) == 1
+    # k out of range
+    assert lib.sparse_route_topk(ctypes.byref(sh), fake, fake, 0, fake, ws_ok,
+                                 need, None) == 1
+    assert lib.sparse_route_topk(ctypes.byref(sh), fake, fake, 4097, fake, ws_ok,
+                                 need, None) == 1
+    # misaligned K
+    assert lib.sparse_route_topk(ctypes.byref(sh), fake, odd, 16, fake, ws_ok,
+                                 need, None) == 1
+    # workspace too small
+    assert lib.sparse_route_topk(ctypes.byref(sh), fake, fake, 16, fake, ws_ok,
+                                 need - 1, None) == 3
+    # unsupported head dim
+    sh96 = _shape(d=96)
+    assert lib.sparse_score(ctypes.byref(sh96), fake, fake, fake, ws_ok, 1 << 30,
+                            None) == 2
+    # decode step: both k and tau, or neither
+    rc, need = _ws_size(lib, sh, k=16, L=2)
+    assert lib.sparse_decode_step(ctypes.byref(sh), 2, fake, fake, fake, fake, 16,
+                                  fake, 0, fake, fake, fake, None, ws_ok, need,
+                                  None) == 1
+    assert lib.sparse_decode_step(ctypes.byref(sh), 2, fake, fake, fake, fake, 0,
+                                  None, 16, fake, fake, fake, None, ws_ok, need,
+                                  None) == 1
+    # threshold needs count and cap >= 1
+    assert lib.sparse_route_threshold(ctypes.byref(sh), fake, fake, fake, 0, fake,
+                                      fake, ws_ok, need, None) == 1
+    assert lib.sparse_attn_gather(ctypes.byref(sh), 1, fake, fake, fake, fake, 0,
+                                  None, fake, None, ws_ok, need, None) == 1
+    assert lib.sparse_read_device_status(None, None, None) == 1
+
+
+def test_python_binding_refuses_cpu_tensors(lib):
+    q = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
+    K = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        sd.route_topk(q, K, 8)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(sd, "_LIB_FILE", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(sd, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        sd.load()

@@ -1,0 +1,345 @@
+"""Parity of the CUDA library (through its C ABI) with the CPU oracle.
+
+Comparison rules (fixed before any kernel ran):
+* Scores: |S_gpu - S_exact| within the fp32 summation bound
+  (G*d + 2) * 2^-24 * sum|q_i k_i| / sqrt(d), with S_exact in fp64.
+* Selection on the SAME fp32 scores (the GPU's own, fed to the oracle):
+  bit-exact index sets, ties included (the decision is taken in the same
+  precision on both sides).
+* Routing end to end (GPU scores vs oracle scores): the sets may differ only
+  in keys whose oracle score lies within 1e-4*|s_k| + 1e-6 of the k-th score
+  (or of tau); top-k sets keep exactly k members; threshold sets miss no key
+  whose fp64 score is >= tau + band.
+* Attention on the oracle's own index set: max |out - oracle| <= 1e-4 for
+  fp32 and <= 2e-2 for bf16; lse within 1e-4 (fp32) / 1e-3 (bf16).
+Passages: CLSA article, sections 研究の背景と課題 and CLSAの仕組み; Louver
+summary, sections 問題定義 and 1. 半空間範囲検索への帰着."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import token_sparse_attention_sm_b200 as sd
+from token_sparse_attention_sm_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = {"f32": 1e-4, "bf16": 2e-2}
+LSE_TOL = {"f32": 1e-4, "bf16": 1e-3}
+
+
+@pytest.fixture(scope="module")
+def dev():
+    from token_sparse_attention_sm_b200 import build
+    build.build()
+    sd.load()
+    return torch.device("cuda", 0)
+
+
+def _to(dev, x, names=("q_route", "q_layers", "K", "V")):
+    return {n: x[n].to(dev) for n in names}
+
+
+def _f(x):
+    return synth.f32(x)
+
+
+def _band(s):
+    return 1e-4 * abs(float(s)) + 1e-6
+
+
+def assert_topk_within_band(gidx, S_oracle, k):
+    """gidx [B,Hkv,k] from the GPU; S_oracle [B,Hkv,N] fp32 oracle scores."""
+    B, Hkv, _ = gidx.shape
+    ref = oracle.topk(S_oracle, k)
+    for b in range(B):
+        for h in range(Hkv):
+            g = gidx[b, h]
+            assert len(set(g.tolist())) == k, "duplicate indices"
+            assert np.all(np.diff(g) > 0), "not ascending"
+            kth = np.sort(S_oracle[b, h])[-k]
+            diff = set(g.tolist()) ^ set(ref[b, h].tolist())
+            bad = [j for j in diff if abs(S_oracle[b, h, j] - kth) > _band(kth)]
+            assert not bad, f"(b={b},h={h}) {len(bad)} indices outside the band"
+
+
+def assert_attn_close(out_gpu, lse_gpu, out_ref, lse_ref, dtype):
+    o = out_gpu.float().cpu().numpy()
+    err = np.abs(o - out_ref).max()
+    assert err <= OUT_TOL[dtype], f"max |out - oracle| = {err}"
+    lg = lse_gpu.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lg), fin)
+    if fin.any():
+        lerr = np.abs(lg[fin] - lse_ref[fin]).max()
+        assert lerr <= LSE_TOL[dtype], f"max |lse - oracle| = {lerr}"
+
+
+# ---------------------------------------------------------------------------
+# A1: scores
+# ---------------------------------------------------------------------------
+
+SCORE_CASES = [
+    dict(B=1, N=4096, Hq=8, Hkv=2, d=64, dtype="f32"),
+    dict(B=2, N=1000, Hq=8, Hkv=2, d=128, dtype="f32"),
+    dict(B=1, N=4099, Hq=32, Hkv=8, d=128, dtype="bf16"),
+    dict(B=3, N=777, Hq=8, Hkv=8, d=64, dtype="bf16"),
+    dict(B=1, N=5, Hq=16, Hkv=1, d=128, dtype="bf16"),
+    dict(B=2, N=300, Hq=16, Hkv=2, d=64, dtype="f32"),
+]
+
+
+@pytest.mark.parametrize("c", SCORE_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_scores_match_oracle(dev, c):
+    w = synth.custom(L=1, k=1, heavy=0, seed=c["N"], **c)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    S = sd.score(t["q_route"], t["K"]).cpu().numpy()
+    q, K = _f(x["q_route"]), _f(x["K"])
+    S64 = oracle.scores(q, K, np.float64)
+    G = w.G
+    Krep = np.repeat(np.abs(K.astype(np.float64)), G, axis=1)
+    mag = np.einsum("bgd,bgnd->bgn", np.abs(q.astype(np.float64)), Krep)
+    mag = mag.reshape(w.B, w.Hkv, G, w.N).sum(axis=2) / np.sqrt(w.d)
+    bound = (G * w.d + 2) * 2.0 ** -24 * mag * 2 + 1e-30
+    assert np.all(np.abs(S - S64) <= bound)
+
+
+# ---------------------------------------------------------------------------
+# A2 / A2': selection on identical scores -> bit-exact
+# ---------------------------------------------------------------------------
+
+SEL_CASES = [(1, 4096, 256), (2, 32768, 2048), (1, 131072, 2048), (3, 1000, 1),
+             (1, 1000, 1000), (2, 5, 3), (1, 70000, 4097), (4, 2048, 2047)]
+
+
+@pytest.mark.parametrize("B,N,k", SEL_CASES)
+def test_select_topk_bit_exact(dev, B, N, k):
+    r = np.random.default_rng(N + k)
+    S = (r.standard_normal((B, 2, N)) * 2).astype(np.float32)
+    idx = sd.select_topk(torch.from_numpy(S).to(dev), k).cpu().numpy()
+    np.testing.assert_array_equal(idx, oracle.topk(S, k))
+
+
+@pytest.mark.parametrize("levels", [1, 3, 50, 4000])
+def test_select_topk_ties_bit_exact(dev, levels):
+    """Few distinct score values: the k-th value is shared by many keys and
+    the lower indices must win; -0.0 and +0.0 are the same score."""
+    r = np.random.default_rng(levels)
+    N, k = 20000, 1500
+    S = r.integers(0, levels, size=(2, 3, N)).astype(np.float32) - levels // 2
+    S[0, 0, ::7] = -0.0
+    idx = sd.select_topk(torch.from_numpy(S).to(dev), k).cpu().numpy()
+    np.testing.assert_array_equal(idx, oracle.topk(S, k))
+
+
+def test_select_topk_all_equal(dev):
+    S = np.full((1, 2, 5000), 0.5, np.float32)
+    idx = sd.select_topk(torch.from_numpy(S).to(dev), 100).cpu().numpy()
+    np.testing.assert_array_equal(idx, np.tile(np.arange(100), (1, 2, 1)))
+
+
+@pytest.mark.parametrize("B,N,cap,pct", [(1, 131072, 8192, 97), (2, 4096, 300, 90),
+                                         (1, 1000, 1000, 0), (3, 77, 5, 50)])
+def test_select_threshold_bit_exact(dev, B, N, cap, pct):
+    r = np.random.default_rng(N)
+    S = (r.standard_normal((B, 2, N)) * 2).astype(np.float32)
+    tau = oracle.percentile_tau(S, pct, 100) if pct else S.min(axis=2)
+    ws = sd.Workspace(dev)
+    gidx, gcnt = sd.select_threshold(torch.from_numpy(S).to(dev),
+                                     torch.from_numpy(tau).to(dev), cap, ws=ws,
+                                     check=False)
+    st = sd.read_device_status(ws, raise_on_error=False)
+    ridx, rcnt = oracle.threshold(S, tau, cap)
+    gcnt = gcnt.cpu().numpy()
+    np.testing.assert_array_equal(gcnt, rcnt)
+    gidx = gidx.cpu().numpy()
+    for b in range(B):
+        for h in range(2):
+            n = min(rcnt[b, h], cap)
+            np.testing.assert_array_equal(gidx[b, h, :n], ridx[b, h, :n])
+    assert st == (4 if (rcnt > cap).any() else 0)
+
+
+def test_select_threshold_empty_and_capacity(dev):
+    S = np.random.default_rng(1).standard_normal((1, 2, 3000)).astype(np.float32)
+    ws = sd.Workspace(dev)
+    tau = np.array([[100.0, -100.0]], np.float32)
+    gidx, gcnt = sd.select_threshold(torch.from_numpy(S).to(dev),
+                                     torch.from_numpy(tau).to(dev), 64, ws=ws,
+                                     check=False)
+    assert sd.read_device_status(ws, raise_on_error=False) == 4   # capacity
+    assert gcnt.cpu().tolist() == [[0, 3000]]
+    assert gidx[0, 1].cpu().tolist() == list(range(64))
+    sd.select_threshold(torch.from_numpy(S).to(dev),
+                        torch.from_numpy(np.full((1, 2), 100.0, np.float32)).to(dev),
+                        64, ws=ws, check=False)
+    assert sd.read_device_status(ws, raise_on_error=False) == 0   # status was reset
+
+
+# ---------------------------------------------------------------------------
+# A3 / A4: attention on the oracle's index set
+# ---------------------------------------------------------------------------
+
+ATTN_CASES = [
+    dict(B=1, N=4096, Hq=8, Hkv=2, d=64, L=2, k=256, dtype="f32"),
+    dict(B=2, N=3000, Hq=32, Hkv=8, d=128, L=16, k=2048, dtype="bf16"),
+    dict(B=1, N=999, Hq=8, Hkv=1, d=128, L=3, k=77, dtype="bf16"),
+    dict(B=2, N=500, Hq=4, Hkv=4, d=64, L=1, k=1, dtype="bf16"),
+    dict(B=1, N=700, Hq=16, Hkv=1, d=64, L=5, k=700, dtype="f32"),
+    dict(B=1, N=129, Hq=32, Hkv=8, d=128, L=40, k=129, dtype="bf16"),
+]
+
+
+@pytest.mark.parametrize("c", ATTN_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_attn_gather_matches_oracle(dev, c):
+    w = synth.custom(heavy=0, seed=c["N"] + c["L"], **c)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
+    idx = oracle.topk(S, w.k)
+    out, lse = sd.attn_gather(t["q_layers"], t["K"], t["V"], torch.from_numpy(idx).to(dev))
+    o_ref, l_ref = oracle.attn(_f(x["q_layers"]), _f(x["K"]), _f(x["V"]), idx)
+    assert_attn_close(out, lse, o_ref, l_ref, w.dtype)
+    # a single layer through the 3-D form gives the same numbers
+    o1, l1 = sd.attn_gather(t["q_layers"][0], t["K"], t["V"], torch.from_numpy(idx).to(dev))
+    assert_attn_close(o1, l1, o_ref[0], l_ref[0], w.dtype)
+
+
+def test_attn_gather_counts_and_empty_sets(dev):
+    w = synth.custom(B=2, N=2000, Hq=8, Hkv=2, d=128, L=2, k=512, dtype="bf16", seed=3)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    r = np.random.default_rng(0)
+    idx = np.stack([np.stack([np.sort(r.choice(2000, 512, replace=False))
+                              for _ in range(2)]) for _ in range(2)]).astype(np.int32)
+    count = np.array([[0, 5], [512, 300]], np.int32)
+    out, lse = sd.attn_gather(t["q_layers"], t["K"], t["V"], torch.from_numpy(idx).to(dev),
+                              count=torch.from_numpy(count).to(dev))
+    o_ref, l_ref = oracle.attn(_f(x["q_layers"]), _f(x["K"]), _f(x["V"]), idx, count)
+    assert_attn_close(out, lse, o_ref, l_ref, "bf16")
+    assert torch.all(out[:, 0, :4] == 0)
+    assert torch.all(torch.isneginf(lse[:, 0, :4]))
+
+
+def test_attn_gather_bad_index_flags_without_fault(dev):
+    w = synth.custom(B=1, N=100, Hq=4, Hkv=1, d=64, L=1, k=8, dtype="bf16", seed=1)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    idx = torch.tensor([[[0, 1, 2, 3, 4, 5, 6, 100]]], dtype=torch.int32, device=dev)
+    ws = sd.Workspace(dev)
+    sd.attn_gather(t["q_layers"], t["K"], t["V"], idx, ws=ws, check=False)
+    assert sd.read_device_status(ws, raise_on_error=False) == 8   # SPARSE_ERR_INDEX
+
+
+# ---------------------------------------------------------------------------
+# Routing end to end and the fused step
+# ---------------------------------------------------------------------------
+
+ROUTE_CASES = [
+    dict(B=1, N=4096, Hq=8, Hkv=2, d=64, k=256, dtype="f32"),
+    dict(B=2, N=10007, Hq=32, Hkv=8, d=128, k=333, dtype="bf16", heavy=16),
+    dict(B=1, N=1, Hq=4, Hkv=1, d=128, k=1, dtype="bf16"),
+    dict(B=1, N=6000, Hq=16, Hkv=1, d=64, k=6000, dtype="bf16"),
+]
+
+
+@pytest.mark.parametrize("c", ROUTE_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_route_topk_matches_oracle(dev, c):
+    w = synth.custom(L=1, seed=c["N"], **c)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    gidx = sd.route_topk(t["q_route"], t["K"], w.k).cpu().numpy()
+    S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
+    assert_topk_within_band(gidx, S, w.k)
+    again = sd.route_topk(t["q_route"], t["K"], w.k).cpu().numpy()
+    np.testing.assert_array_equal(gidx, again)   # deterministic
+
+
+def test_nonfinite_key_is_flagged(dev):
+    w = synth.custom(B=1, N=1000, Hq=8, Hkv=2, d=64, L=1, k=10, dtype="bf16", seed=2)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    t["K"][0, 1, 17, 3] = float("nan")
+    ws = sd.Workspace(dev)
+    sd.route_topk(t["q_route"], t["K"], 10, ws=ws, check=False)
+    assert sd.read_device_status(ws, raise_on_error=False) == 5   # NONFINITE
+
+
+def _check_decode(dev, w, x, batches_checked=None):
+    t = _to(dev, x)
+    res = sd.decode_step(t["q_route"], t["q_layers"], t["K"], t["V"], k=w.k)
+    gidx = res["idx"].cpu().numpy()
+    bsel = list(range(w.B)) if batches_checked is None else list(batches_checked)
+    q = _f(x["q_route"][bsel])
+    K = _f(x["K"][bsel])
+    S = oracle.scores(q, K)
+    assert_topk_within_band(gidx[bsel], S, w.k)
+    # shared routing: the fused step's set is the routing call's set, bitwise
+    np.testing.assert_array_equal(gidx, sd.route_topk(t["q_route"], t["K"], w.k).cpu().numpy())
+    # every layer's output equals the gather call on that set, and matches the
+    # oracle on the oracle's own set
+    out2, lse2 = sd.attn_gather(t["q_layers"], t["K"], t["V"], res["idx"])
+    assert torch.equal(out2, res["out"]) and torch.equal(lse2, res["lse"])
+    ridx = oracle.topk(S, w.k)
+    o_gpu, l_gpu = sd.attn_gather(t["q_layers"][:, bsel].contiguous(), t["K"][bsel].contiguous(),
+                                  t["V"][bsel].contiguous(), torch.from_numpy(ridx).to(dev))
+    o_ref, l_ref = oracle.attn(_f(x["q_layers"][:, bsel]), K, _f(x["V"][bsel]), ridx)
+    assert_attn_close(o_gpu, l_gpu, o_ref, l_ref, w.dtype)
+    return res
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "decode_32k", "decode_128k"])
+def test_decode_step_named_workloads(dev, name):
+    w = synth.WORKLOADS[name]
+    x = synth.generate(w)
+    _check_decode(dev, w, x)
+
+
+def test_decode_step_batched_16x64k_sampled(dev):
+    w = synth.WORKLOADS["batched_16x64k"]
+    x = synth.generate(w)
+    _check_decode(dev, w, x, batches_checked=[0, 7, 15])
+
+
+@pytest.mark.parametrize("name,cap", [("threshold_128k", 8192), ("threshold_128k", 2000)])
+def test_decode_step_threshold(dev, name, cap):
+    w = synth.WORKLOADS[name]
+    x = synth.generate(w)
+    t = _to(dev, x)
+    q, K = _f(x["q_route"]), _f(x["K"])
+    S = oracle.scores(q, K)
+    S64 = oracle.scores(q, K, np.float64)
+    tau = oracle.percentile_tau(S, *w.tau_pct)
+    ws = sd.Workspace(dev)
+    res = sd.decode_step(t["q_route"], t["q_layers"], t["K"], t["V"],
+                         tau=torch.from_numpy(tau).to(dev), cap=cap, ws=ws, check=False)
+    st = sd.read_device_status(ws, raise_on_error=False)
+    gidx, gcnt = res["idx"].cpu().numpy(), res["count"].cpu().numpy()
+    ridx, rcnt = oracle.threshold(S, tau, cap)
+    assert st == (4 if (rcnt > cap).any() else 0)
+    for h in range(w.Hkv):
+        band = _band(tau[0, h])
+        g = set(gidx[0, h, :min(gcnt[0, h], cap)].tolist())
+        if gcnt[0, h] <= cap:
+            must = set(np.nonzero(S64[0, h] >= tau[0, h] + band)[0].tolist())
+            never = set(np.nonzero(S64[0, h] < tau[0, h] - band)[0].tolist())
+            assert must <= g and not (g & never), "false negative or positive"
+        assert abs(int(gcnt[0, h]) - int(rcnt[0, h])) <= \
+            int(np.sum(np.abs(S[0, h] - tau[0, h]) <= band))
+    # attention with the oracle's set and counts
+    o_gpu, l_gpu = sd.attn_gather(t["q_layers"], t["K"], t["V"], torch.from_numpy(ridx).to(dev),
+                                  count=torch.from_numpy(np.minimum(rcnt, cap)).to(dev))
+    o_ref, l_ref = oracle.attn(_f(x["q_layers"]), K, _f(x["V"]), ridx, np.minimum(rcnt, cap))
+    assert_attn_close(o_gpu, l_gpu, o_ref, l_ref, w.dtype)
+
+
+def test_decode_step_threshold_empty_set(dev):
+    w = synth.custom(B=1, N=3000, Hq=8, Hkv=2, d=128, L=2, dtype="bf16", seed=9,
+                     mode="threshold", cap=64)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    tau = torch.full((1, 2), 1e9, device=dev)
+    res = sd.decode_step(t["q_route"], t["q_layers"], t["K"], t["V"], tau=tau, cap=64)
+    assert res["count"].cpu().tolist() == [[0, 0]]
+    assert torch.all(res["out"] == 0) and torch.all(torch.isneginf(res["lse"]))

@@ -1,2 +1,348 @@
 """token_sparse_attention_sm_b200: shared-routing token-sparse decode
-attention for NVIDIA B200 (sm_100a)."""
+attention for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libsparse_decode.so`` (declared in
+``include/sparse_decode.h``).  It only marshals arguments: every step of the
+path -- scoring, selection, gather attention, split merge -- runs in the
+library's CUDA kernels.  PyTorch provides device memory and the current
+stream.  There is no CPU or PyTorch fallback: if the library is missing,
+every call raises.
+
+What is computed (CLSA article, sections 研究の背景と課題 and CLSAの仕組み;
+Louver summary, sections 問題定義 and 1. 半空間範囲検索への帰着): one routing
+pass scores every cached key with the GQA-group-summed q.k/sqrt(d), keeps the
+top-k (ties to the lower index) or every key with score >= tau, and every
+layer then attends over only that one shared set.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = ["SparseDecodeError", "lib_path", "load", "score", "select_topk",
+           "select_threshold", "route_topk", "route_threshold", "attn_gather",
+           "decode_step", "read_device_status", "workspace_bytes",
+           "Workspace", "STATUS_NAMES", "EXPORTED_SYMBOLS"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_FILE = os.path.join(_PKG, "libsparse_decode.so")
+
+STATUS_NAMES = {
+    0: "SPARSE_OK", 1: "SPARSE_ERR_INVALID_ARG", 2: "SPARSE_ERR_UNSUPPORTED",
+    3: "SPARSE_ERR_WORKSPACE", 4: "SPARSE_ERR_CAPACITY",
+    5: "SPARSE_ERR_NONFINITE", 6: "SPARSE_ERR_CUDA", 7: "SPARSE_ERR_TIMEOUT",
+    8: "SPARSE_ERR_INDEX", 9: "SPARSE_ERR_INTERNAL",
+}
+
+EXPORTED_SYMBOLS = (
+    "sparse_status_string", "sparse_version", "sparse_workspace_size",
+    "sparse_workspace_init", "sparse_score", "sparse_select_topk",
+    "sparse_select_threshold", "sparse_route_topk", "sparse_route_threshold",
+    "sparse_attn_gather", "sparse_decode_step", "sparse_read_device_status",
+)
+
+DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
+
+
+class SparseDecodeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib_path() -> str:
+    return _LIB_FILE
+
+
+def load():
+    """Load libsparse_decode.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_FILE):
+            raise RuntimeError(
+                f"CUDA library not built: {_LIB_FILE} is missing "
+                "(run `python -m token_sparse_attention_sm_b200.build`)")
+        lib = ctypes.CDLL(_LIB_FILE)
+        P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        SH = ctypes.POINTER(_Shape)
+        sigs = {
+            "sparse_status_string": (ctypes.c_char_p, [I32]),
+            "sparse_version": (I32, []),
+            "sparse_workspace_size": (I32, [SH, I32, I32, ctypes.POINTER(SZ)]),
+            "sparse_workspace_init": (I32, [P, SZ, P]),
+            "sparse_score": (I32, [SH, P, P, P, P, SZ, P]),
+            "sparse_select_topk": (I32, [SH, P, I32, P, P, SZ, P]),
+            "sparse_select_threshold": (I32, [SH, P, P, I32, P, P, P, SZ, P]),
+            "sparse_route_topk": (I32, [SH, P, P, I32, P, P, SZ, P]),
+            "sparse_route_threshold": (I32, [SH, P, P, P, I32, P, P, P, SZ, P]),
+            "sparse_attn_gather": (I32, [SH, I32, P, P, P, P, I32, P, P, P, P,
+                                         SZ, P]),
+            "sparse_decode_step": (I32, [SH, I32, P, P, P, P, I32, P, I32, P, P,
+                                         P, P, P, SZ, P]),
+            "sparse_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise SparseDecodeError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _shape(B, N, Hq, Hkv, d, dtype) -> _Shape:
+    if dtype not in DTYPE_CODES:
+        raise TypeError(f"unsupported dtype {dtype}")
+    return _Shape(B, N, Hq, Hkv, d, DTYPE_CODES[dtype])
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+
+
+def workspace_bytes(B, N, Hq, Hkv, d, dtype, k_or_cap: int, L: int) -> int:
+    n = ctypes.c_size_t(0)
+    sh = _shape(B, N, Hq, Hkv, d, dtype)
+    _check(load().sparse_workspace_size(ctypes.byref(sh), int(k_or_cap), int(L),
+                                        ctypes.byref(n)), "workspace_size")
+    return int(n.value)
+
+
+class Workspace:
+    """A zero-initialised device workspace that grows on demand.  Calls that
+    share one must be ordered on the same stream."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device) if device is not None else torch.device(
+            "cuda", torch.cuda.current_device())
+        self.buf = None
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8,
+                                   device=self.device)
+        return self.buf
+
+
+_default_ws = {}
+
+
+def _ws(ws: Workspace | None, device) -> Workspace:
+    if ws is not None:
+        return ws
+    key = torch.device(device).index
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+def read_device_status(ws: Workspace, raise_on_error: bool = True) -> int:
+    """Synchronise the current stream and read (and reset) the device status
+    word of ``ws``; raises SparseDecodeError unless it is SPARSE_OK."""
+    flags = ctypes.c_uint32(0)
+    rc = load().sparse_read_device_status(_ptr(ws.buf), _stream(), ctypes.byref(flags))
+    if raise_on_error:
+        _check(rc, f"device status (flags=0x{flags.value:x})")
+    return rc
+
+
+def _dims_qk(q, K):
+    if q.dim() != 3 or K.dim() != 4:
+        raise ValueError("q must be [B,Hq,d] and K [B,Hkv,N,d]")
+    B, Hq, d = q.shape
+    Bk, Hkv, N, dk = K.shape
+    if Bk != B or dk != d:
+        raise ValueError("q and K disagree on B or d")
+    if q.dtype != K.dtype:
+        raise ValueError("q and K must share a dtype")
+    return B, N, Hq, Hkv, d
+
+
+def score(q, K, ws: Workspace | None = None, check: bool = True):
+    """Routing scores S [B,Hkv,N] fp32."""
+    _need_cuda(q, K)
+    B, N, Hq, Hkv, d = _dims_qk(q, K)
+    w = _ws(ws, q.device)
+    sh = _shape(B, N, Hq, Hkv, d, q.dtype)
+    buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, 1, 1))
+    S = torch.empty((B, Hkv, N), dtype=torch.float32, device=q.device)
+    _check(load().sparse_score(ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(S),
+                               _ptr(buf), buf.numel(), _stream()), "score")
+    if check:
+        read_device_status(w)
+    return S
+
+
+def select_topk(S, k: int, ws: Workspace | None = None, check: bool = True):
+    """Top-k of S [B,Hkv,N] fp32 -> idx [B,Hkv,k] int32 ascending."""
+    _need_cuda(S)
+    B, Hkv, N = S.shape
+    w = _ws(ws, S.device)
+    sh = _shape(B, N, Hkv, Hkv, 64, torch.float32)
+    buf = w.get(workspace_bytes(B, N, Hkv, Hkv, 64, torch.float32, k, 1))
+    idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=S.device)
+    _check(load().sparse_select_topk(ctypes.byref(sh), _ptr(S), int(k), _ptr(idx),
+                                     _ptr(buf), buf.numel(), _stream()),
+           "select_topk")
+    if check:
+        read_device_status(w)
+    return idx
+
+
+def select_threshold(S, tau, cap: int, ws: Workspace | None = None,
+                     check: bool = True):
+    """Threshold sets of S: (idx [B,Hkv,cap], count [B,Hkv])."""
+    _need_cuda(S, tau)
+    B, Hkv, N = S.shape
+    w = _ws(ws, S.device)
+    sh = _shape(B, N, Hkv, Hkv, 64, torch.float32)
+    buf = w.get(workspace_bytes(B, N, Hkv, Hkv, 64, torch.float32, cap, 1))
+    idx = torch.empty((B, Hkv, cap), dtype=torch.int32, device=S.device)
+    count = torch.empty((B, Hkv), dtype=torch.int32, device=S.device)
+    _check(load().sparse_select_threshold(
+        ctypes.byref(sh), _ptr(S), _ptr(tau.float().contiguous()), int(cap),
+        _ptr(idx), _ptr(count), _ptr(buf), buf.numel(), _stream()),
+        "select_threshold")
+    if check:
+        read_device_status(w)
+    return idx, count
+
+
+def route_topk(q, K, k: int, ws: Workspace | None = None, check: bool = True):
+    """Shared routing (top-k): idx [B,Hkv,k] int32 ascending."""
+    _need_cuda(q, K)
+    B, N, Hq, Hkv, d = _dims_qk(q, K)
+    w = _ws(ws, q.device)
+    sh = _shape(B, N, Hq, Hkv, d, q.dtype)
+    buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, k, 1))
+    idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=q.device)
+    _check(load().sparse_route_topk(ctypes.byref(sh), _ptr(q), _ptr(K), int(k),
+                                    _ptr(idx), _ptr(buf), buf.numel(), _stream()),
+           "route_topk")
+    if check:
+        read_device_status(w)
+    return idx
+
+
+def route_threshold(q, K, tau, cap: int, ws: Workspace | None = None,
+                    check: bool = True):
+    """Shared routing (threshold): (idx [B,Hkv,cap], count [B,Hkv])."""
+    _need_cuda(q, K, tau)
+    B, N, Hq, Hkv, d = _dims_qk(q, K)
+    w = _ws(ws, q.device)
+    sh = _shape(B, N, Hq, Hkv, d, q.dtype)
+    buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, cap, 1))
+    idx = torch.empty((B, Hkv, cap), dtype=torch.int32, device=q.device)
+    count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    tau = tau.float().contiguous()
+    _check(load().sparse_route_threshold(
+        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(tau), int(cap), _ptr(idx),
+        _ptr(count), _ptr(buf), buf.numel(), _stream()), "route_threshold")
+    if check:
+        read_device_status(w)
+    return idx, count
+
+
+def attn_gather(q, K, V, idx, count=None, ws: Workspace | None = None,
+                check: bool = True, return_lse: bool = True):
+    """Attention of q ([B,Hq,d] or [L,B,Hq,d]) over the idx rows
+    [B,Hkv,stride] (first count[b,h] of each row if count is given).
+    Returns (out, lse) with out shaped like q."""
+    _need_cuda(q, K, V, idx, count)
+    single = q.dim() == 3
+    q4 = q.unsqueeze(0) if single else q
+    L, B, Hq, d = q4.shape
+    Bk, Hkv, N, dk = K.shape
+    if V.shape != K.shape or Bk != B or dk != d:
+        raise ValueError("shape mismatch between q, K and V")
+    if idx.dtype != torch.int32 or idx.dim() != 3 or idx.shape[:2] != (B, Hkv):
+        raise ValueError("idx must be int32 [B,Hkv,stride]")
+    stride = idx.shape[2]
+    w = _ws(ws, q.device)
+    sh = _shape(B, N, Hq, Hkv, d, q.dtype)
+    buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, stride, L))
+    out = torch.empty_like(q4)
+    lse = torch.empty((L, B, Hq), dtype=torch.float32, device=q.device) if return_lse else None
+    _check(load().sparse_attn_gather(
+        ctypes.byref(sh), L, _ptr(q4), _ptr(K), _ptr(V), _ptr(idx), stride,
+        _ptr(count), _ptr(out), _ptr(lse), _ptr(buf), buf.numel(), _stream()),
+        "attn_gather")
+    if check:
+        read_device_status(w)
+    if single:
+        return out[0], (lse[0] if lse is not None else None)
+    return out, lse
+
+
+def decode_step(q_route, q_layers, K, V, k: int | None = None, tau=None,
+                cap: int | None = None, ws: Workspace | None = None,
+                check: bool = True, out=None, idx=None, count=None, lse=None,
+                return_lse: bool = True):
+    """One fused decode step: route once, attend L layers over that set.
+
+    Top-k mode with ``k``; threshold mode with ``tau`` [B,Hkv] and ``cap``.
+    Returns dict(idx, count, out, lse).  Preallocated outputs may be passed
+    to keep a timing loop free of allocations."""
+    _need_cuda(q_route, q_layers, K, V, tau)
+    B, N, Hq, Hkv, d = _dims_qk(q_route, K)
+    L = q_layers.shape[0]
+    if q_layers.shape != (L, B, Hq, d) or V.shape != K.shape:
+        raise ValueError("q_layers must be [L,B,Hq,d] and V like K")
+    topk = k is not None
+    if topk == (tau is not None):
+        raise ValueError("give exactly one of k or tau")
+    stride = int(k) if topk else int(cap)
+    dev = q_route.device
+    w = _ws(ws, dev)
+    sh = _shape(B, N, Hq, Hkv, d, q_route.dtype)
+    buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q_route.dtype, stride, L))
+    if idx is None:
+        idx = torch.empty((B, Hkv, stride), dtype=torch.int32, device=dev)
+    if count is None and not topk:
+        count = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty_like(q_layers)
+    if lse is None and return_lse:
+        lse = torch.empty((L, B, Hq), dtype=torch.float32, device=dev)
+    tau_t = None if topk else tau.float().contiguous()
+    _check(load().sparse_decode_step(
+        ctypes.byref(sh), L, _ptr(q_route), _ptr(q_layers), _ptr(K), _ptr(V),
+        int(k) if topk else 0, _ptr(tau_t), 0 if topk else int(cap), _ptr(idx),
+        _ptr(count), _ptr(out), _ptr(lse), _ptr(buf), buf.numel(), _stream()),
+        "decode_step")
+    if check:
+        read_device_status(w)
+    return {"idx": idx, "count": count, "out": out, "lse": lse}

@@ -1,0 +1,322 @@
+// api.cu -- the C ABI of libsparse_decode (declared in sparse_decode.h).
+//
+// Every entry point validates its arguments on the host and returns an error
+// before anything is enqueued; then it enqueues the kernels on the caller's
+// stream and returns.  The library allocates nothing: scratch lives in the
+// caller's workspace, whose layout is
+//   [0, 256)              header: device status word (uint32) at offset 0
+//   [256, 256 + S bytes)  fp32 scores S [B,Hkv,N]
+//   [.., ..)              attention split partials
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sparse_decode.h"
+
+namespace sd {
+
+cudaError_t select_cluster_size(int sm_count, int smem_optin, int *out);
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::once_flag g_once[kMaxDevices];
+DeviceInfo g_info[kMaxDevices];
+cudaError_t g_info_err[kMaxDevices];
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+constexpr size_t kHeader = 256;
+
+struct Layout {
+  size_t scores_off, scores_bytes, attn_off, attn_bytes, total;
+};
+
+Layout layout(const Shape &s, int stride, int L) {
+  Layout l;
+  l.scores_off = kHeader;
+  l.scores_bytes = align_up((size_t)s.BH() * s.N * sizeof(float), 256);
+  l.attn_off = l.scores_off + l.scores_bytes;
+  l.attn_bytes = align_up(attn_workspace_bytes(s, L, stride), 256);
+  l.total = l.attn_off + l.attn_bytes;
+  return l;
+}
+
+bool aligned(const void *p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+sparse_status_t check_shape(const sparse_shape_t *shape, Shape *s) {
+  if (!shape) return SPARSE_ERR_INVALID_ARG;
+  s->B = shape->B;
+  s->N = shape->N;
+  s->Hq = shape->Hq;
+  s->Hkv = shape->Hkv;
+  s->d = shape->d;
+  s->dtype = shape->dtype;
+  if (s->B < 1 || s->N < 1 || s->Hq < 1 || s->Hkv < 1 || s->d < 1)
+    return SPARSE_ERR_INVALID_ARG;
+  if (s->Hq % s->Hkv != 0) return SPARSE_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return SPARSE_ERR_UNSUPPORTED;
+  if (s->dtype != SPARSE_DTYPE_F32 && s->dtype != SPARSE_DTYPE_BF16)
+    return SPARSE_ERR_UNSUPPORTED;
+  if (s->G() > 16) return SPARSE_ERR_UNSUPPORTED;
+  if ((long long)s->B * s->Hkv > 65535) return SPARSE_ERR_UNSUPPORTED;
+  return SPARSE_OK;
+}
+
+sparse_status_t check_ws(const Shape &s, int stride, int L, void *ws,
+                         size_t ws_bytes) {
+  if (!ws || !aligned(ws, 256)) return SPARSE_ERR_INVALID_ARG;
+  if (ws_bytes < layout(s, stride, L).total) return SPARSE_ERR_WORKSPACE;
+  return SPARSE_OK;
+}
+
+sparse_status_t from_cuda(cudaError_t e) {
+  return e == cudaSuccess ? SPARSE_OK : SPARSE_ERR_CUDA;
+}
+
+uint32_t *status_word(void *ws) { return static_cast<uint32_t *>(ws); }
+float *scores_ptr(void *ws, const Layout &l) {
+  return reinterpret_cast<float *>(static_cast<char *>(ws) + l.scores_off);
+}
+void *attn_ptr(void *ws, const Layout &l) {
+  return static_cast<char *>(ws) + l.attn_off;
+}
+
+}  // namespace
+
+cudaError_t device_info(DeviceInfo *out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_once[dev], [dev]() {
+    DeviceInfo di;
+    cudaError_t err =
+        cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (err == cudaSuccess)
+      err = cudaDeviceGetAttribute(&di.max_smem_optin,
+                                   cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (err == cudaSuccess)
+      err = select_cluster_size(di.sm_count, di.max_smem_optin,
+                                &di.select_cluster);
+    g_info[dev] = di;
+    g_info_err[dev] = err;
+  });
+  *out = g_info[dev];
+  return g_info_err[dev];
+}
+
+}  // namespace sd
+
+using sd::Shape;
+
+extern "C" {
+
+const char *sparse_status_string(sparse_status_t status) {
+  switch (status) {
+    case SPARSE_OK: return "SPARSE_OK";
+    case SPARSE_ERR_INVALID_ARG: return "SPARSE_ERR_INVALID_ARG: invalid argument";
+    case SPARSE_ERR_UNSUPPORTED: return "SPARSE_ERR_UNSUPPORTED: unsupported shape or dtype";
+    case SPARSE_ERR_WORKSPACE: return "SPARSE_ERR_WORKSPACE: workspace too small";
+    case SPARSE_ERR_CAPACITY: return "SPARSE_ERR_CAPACITY: threshold set larger than cap";
+    case SPARSE_ERR_NONFINITE: return "SPARSE_ERR_NONFINITE: non-finite score or tau";
+    case SPARSE_ERR_CUDA: return "SPARSE_ERR_CUDA: CUDA runtime error";
+    case SPARSE_ERR_TIMEOUT: return "SPARSE_ERR_TIMEOUT: bounded device wait expired";
+    case SPARSE_ERR_INDEX: return "SPARSE_ERR_INDEX: index outside [0, N)";
+    case SPARSE_ERR_INTERNAL: return "SPARSE_ERR_INTERNAL: internal consistency check failed";
+  }
+  return "SPARSE_ERR_UNKNOWN";
+}
+
+int32_t sparse_version(void) { return 100; }
+
+sparse_status_t sparse_workspace_size(const sparse_shape_t *shape,
+                                      int32_t k_or_cap, int32_t L,
+                                      size_t *bytes) {
+  Shape s;
+  sparse_status_t r = sd::check_shape(shape, &s);
+  if (r != SPARSE_OK) return r;
+  if (!bytes || k_or_cap < 1 || L < 1) return SPARSE_ERR_INVALID_ARG;
+  if ((long long)L * s.G() > 1024) return SPARSE_ERR_UNSUPPORTED;
+  *bytes = sd::layout(s, k_or_cap, L).total;
+  return SPARSE_OK;
+}
+
+sparse_status_t sparse_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+  if (!ws || ws_bytes < 256) return SPARSE_ERR_INVALID_ARG;
+  return sd::from_cuda(
+      cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+sparse_status_t sparse_score(const sparse_shape_t *shape, const void *q,
+                             const void *K, float *S, void *ws,
+                             size_t ws_bytes, void *stream) {
+  Shape s;
+  sparse_status_t r = sd::check_shape(shape, &s);
+  if (r != SPARSE_OK) return r;
+  if (!q || !K || !S) return SPARSE_ERR_INVALID_ARG;
+  if (!sd::aligned(q, 16) || !sd::aligned(K, 16) || !sd::aligned(S, 16))
+    return SPARSE_ERR_INVALID_ARG;
+  if ((r = sd::check_ws(s, 1, 1, ws, ws_bytes)) != SPARSE_OK) return r;
+  return sd::from_cuda(sd::launch_score(s, q, K, S, sd::status_word(ws),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+sparse_status_t sparse_select_topk(const sparse_shape_t *shape,
+                                   const float *S, int32_t k, int32_t *idx,
+                                   void *ws, size_t ws_bytes, void *stream) {
+  Shape s;
+  sparse_status_t r = sd::check_shape(shape, &s);
+  if (r != SPARSE_OK) return r;
+  if (!S || !idx || k < 1 || k > s.N) return SPARSE_ERR_INVALID_ARG;
+  if (!sd::aligned(S, 16) || !sd::aligned(idx, 4)) return SPARSE_ERR_INVALID_ARG;
+  if ((r = sd::check_ws(s, k, 1, ws, ws_bytes)) != SPARSE_OK) return r;
+  return sd::from_cuda(sd::launch_select(s, S, k, nullptr, 0, idx, nullptr, k,
+                                         sd::status_word(ws),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+sparse_status_t sparse_select_threshold(const sparse_shape_t *shape,
+                                        const float *S, const float *tau,
+                                        int32_t cap, int32_t *idx,
+                                        int32_t *count, void *ws,
+                                        size_t ws_bytes, void *stream) {
+  Shape s;
+  sparse_status_t r = sd::check_shape(shape, &s);
+  if (r != SPARSE_OK) return r;
+  if (!S || !tau || !idx || !count || cap < 1) return SPARSE_ERR_INVALID_ARG;
+  if (!sd::aligned(S, 16) || !sd::aligned(tau, 4) || !sd::aligned(idx, 4) ||
+      !sd::aligned(count, 4))
+    return SPARSE_ERR_INVALID_ARG;
+  if ((r = sd::check_ws(s, cap, 1, ws, ws_bytes)) != SPARSE_OK) return r;
+  return sd::from_cuda(sd::launch_select(s, S, 0, tau, cap, idx, count, cap,
+                                         sd::status_word(ws),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+sparse_status_t sparse_route_topk(const sparse_shape_t *shape, const void *q,
+                                  const void *K, int32_t k, int32_t *idx,
+                                  void *ws, size_t ws_bytes, void *stream) {
+  Shape s;
+  sparse_status_t r = sd::check_shape(shape, &s);
+  if (r != SPARSE_OK) return r;
+  if (!q || !K || !idx || k < 1 || k > s.N) return SPARSE_ERR_INVALID_ARG;
+  if (!sd::aligned(q, 16) || !sd::aligned(K, 16) || !sd::aligned(idx, 4))
+    return SPARSE_ERR_INVALID_ARG;
+  if ((r = sd::check_ws(s, k, 1, ws, ws_bytes)) != SPARSE_OK) return r;
+  const sd::Layout l = sd::layout(s, k, 1);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float *S = sd::scores_ptr(ws, l);
+  cudaError_t e = sd::launch_score(s, q, K, S, sd::status_word(ws), st);
+  if (e == cudaSuccess)
+    e = sd::launch_select(s, S, k, nullptr, 0, idx, nullptr, k,
+                          sd::status_word(ws), st);
+  return sd::from_cuda(e);
+}
+
+sparse_status_t sparse_route_threshold(const sparse_shape_t *shape,
+                                       const void *q, const void *K,
+                                       const float *tau, int32_t cap,
+                                       int32_t *idx, int32_t *count, void *ws,
+                                       size_t ws_bytes, void *stream) {
+  Shape s;
+  sparse_status_t r = sd::check_shape(shape, &s);
+  if (r != SPARSE_OK) return r;
+  if (!q || !K || !tau || !idx || !count || cap < 1) return SPARSE_ERR_INVALID_ARG;
+  if (!sd::aligned(q, 16) || !sd::aligned(K, 16) || !sd::aligned(tau, 4) ||
+      !sd::aligned(idx, 4) || !sd::aligned(count, 4))
+    return SPARSE_ERR_INVALID_ARG;
+  if ((r = sd::check_ws(s, cap, 1, ws, ws_bytes)) != SPARSE_OK) return r;
+  const sd::Layout l = sd::layout(s, cap, 1);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float *S = sd::scores_ptr(ws, l);
+  cudaError_t e = sd::launch_score(s, q, K, S, sd::status_word(ws), st);
+  if (e == cudaSuccess)
+    e = sd::launch_select(s, S, 0, tau, cap, idx, count, cap,
+                          sd::status_word(ws), st);
+  return sd::from_cuda(e);
+}
+
+sparse_status_t sparse_attn_gather(const sparse_shape_t *shape, int32_t L,
+                                   const void *q, const void *K,
+                                   const void *V, const int32_t *idx,
+                                   int32_t stride, const int32_t *count,
+                                   void *out, float *lse, void *ws,
+                                   size_t ws_bytes, void *stream) {
+  Shape s;
+  sparse_status_t r = sd::check_shape(shape, &s);
+  if (r != SPARSE_OK) return r;
+  if (L < 1 || !q || !K || !V || !idx || stride < 1 || !out)
+    return SPARSE_ERR_INVALID_ARG;
+  if ((long long)L * s.G() > 1024) return SPARSE_ERR_UNSUPPORTED;
+  if (!sd::aligned(q, 16) || !sd::aligned(K, 16) || !sd::aligned(V, 16) ||
+      !sd::aligned(out, 16) || !sd::aligned(idx, 4) ||
+      (count && !sd::aligned(count, 4)) || (lse && !sd::aligned(lse, 4)))
+    return SPARSE_ERR_INVALID_ARG;
+  if ((r = sd::check_ws(s, stride, L, ws, ws_bytes)) != SPARSE_OK) return r;
+  const sd::Layout l = sd::layout(s, stride, L);
+  return sd::from_cuda(sd::launch_attn(
+      s, L, q, K, V, idx, stride, count, stride, out, lse, sd::attn_ptr(ws, l),
+      sd::status_word(ws), static_cast<cudaStream_t>(stream)));
+}
+
+sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
+                                   const void *q_route, const void *q_layers,
+                                   const void *K, const void *V, int32_t k,
+                                   const float *tau, int32_t cap,
+                                   int32_t *idx, int32_t *count, void *out,
+                                   float *lse, void *ws, size_t ws_bytes,
+                                   void *stream) {
+  Shape s;
+  sparse_status_t r = sd::check_shape(shape, &s);
+  if (r != SPARSE_OK) return r;
+  if (L < 1 || !q_route || !q_layers || !K || !V || !idx || !out)
+    return SPARSE_ERR_INVALID_ARG;
+  if ((long long)L * s.G() > 1024) return SPARSE_ERR_UNSUPPORTED;
+  const bool topk = k > 0;
+  if (topk) {
+    if (k > s.N || tau) return SPARSE_ERR_INVALID_ARG;
+  } else {
+    if (k < 0 || !tau || !count || cap < 1) return SPARSE_ERR_INVALID_ARG;
+  }
+  if (!sd::aligned(q_route, 16) || !sd::aligned(q_layers, 16) ||
+      !sd::aligned(K, 16) || !sd::aligned(V, 16) || !sd::aligned(out, 16) ||
+      !sd::aligned(idx, 4) || (count && !sd::aligned(count, 4)) ||
+      (tau && !sd::aligned(tau, 4)) || (lse && !sd::aligned(lse, 4)))
+    return SPARSE_ERR_INVALID_ARG;
+  const int stride = topk ? k : cap;
+  if ((r = sd::check_ws(s, stride, L, ws, ws_bytes)) != SPARSE_OK) return r;
+  const sd::Layout l = sd::layout(s, stride, L);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *status = sd::status_word(ws);
+  float *S = sd::scores_ptr(ws, l);
+  cudaError_t e = sd::launch_score(s, q_route, K, S, status, st);
+  if (e == cudaSuccess)
+    e = topk ? sd::launch_select(s, S, k, nullptr, 0, idx, nullptr, k, status, st)
+             : sd::launch_select(s, S, 0, tau, cap, idx, count, cap, status, st);
+  if (e == cudaSuccess)
+    e = sd::launch_attn(s, L, q_layers, K, V, idx, stride, topk ? nullptr : count,
+                        stride, out, lse, sd::attn_ptr(ws, l), status, st);
+  return sd::from_cuda(e);
+}
+
+sparse_status_t sparse_read_device_status(void *ws, void *stream,
+                                          uint32_t *flags) {
+  if (!ws) return SPARSE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t f = 0;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(&f, ws, sizeof(f), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(f), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return SPARSE_ERR_CUDA;
+  if (flags) *flags = f;
+  if (f & sd::FLAG_TIMEOUT) return SPARSE_ERR_TIMEOUT;
+  if (f & sd::FLAG_INTERNAL) return SPARSE_ERR_INTERNAL;
+  if (f & sd::FLAG_INDEX) return SPARSE_ERR_INDEX;
+  if (f & sd::FLAG_NONFINITE) return SPARSE_ERR_NONFINITE;
+  if (f & sd::FLAG_CAPACITY) return SPARSE_ERR_CAPACITY;
+  return SPARSE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,44 @@
+// internal.h -- launchers shared between the translation units of
+// libsparse_decode.  Host-side only; no torch types anywhere.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sd {
+
+struct Shape {
+  int B, N, Hq, Hkv, d, dtype;  // dtype: 0 = fp32, 1 = bf16
+  int G() const { return Hq / Hkv; }
+  int BH() const { return B * Hkv; }
+  int esize() const { return dtype == 0 ? 4 : 2; }
+};
+
+// Device properties cached per device (SM count, cluster support).
+struct DeviceInfo {
+  int sm_count = 0;
+  int max_smem_optin = 0;
+  int select_cluster = 0;  // cluster size the select kernel uses
+};
+cudaError_t device_info(DeviceInfo *out);
+
+// A1: S[b,h,j] for every key; one streaming pass over K.
+cudaError_t launch_score(const Shape &s, const void *q, const void *K,
+                         float *S, uint32_t *status, cudaStream_t st);
+
+// A2 / A2': selection from S.  k >= 1: top-k (tau ignored); k == 0:
+// threshold with tau and cap, count written.  idx rows have `stride`
+// entries.
+cudaError_t launch_select(const Shape &s, const float *S, int k,
+                          const float *tau, int cap, int *idx, int *count,
+                          int stride, uint32_t *status, cudaStream_t st);
+
+// A3 + A4: L query sets over the same index rows.
+size_t attn_workspace_bytes(const Shape &s, int L, int stride);
+cudaError_t launch_attn(const Shape &s, int L, const void *q, const void *K,
+                        const void *V, const int *idx, int stride,
+                        const int *count, int count_cap, void *out, float *lse,
+                        void *ws, uint32_t *status, cudaStream_t st);
+
+}  // namespace sd
