@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Decode-step throughput of shared-routing token-sparse attention on B200.
+
+One step = one fused decode call over the whole batch: the routing score
+scan over the K cache, the top-k select per (sequence, KV head), and the
+gather attention of all L layers over that one set (CLSA article, sections
+CLSAの仕組み and 計算コストの削減効果).  The default workload is the 128K-token
+headline: B=1, N=131072, Hq=32, Hkv=8, d=128, k=2048, L=16, bf16.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Rank 0 prints one JSON line.  With N > 1 (torchrun, one process per GPU)
+every rank runs its own replica on its own sequences: the path shards into
+independent sequences with no exchange step, so the scaling is weak and the
+only collectives are the barrier and the max-over-ranks of the timed region.
+
+``--impl reference`` times the CPU oracle (the plain C reference under
+oracle/) on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from token_sparse_attention_sm_b200 import dist as sdist  # noqa: E402
+from token_sparse_attention_sm_b200 import synth  # noqa: E402
+
+METRIC = ("128K-context sparse decode steps/s (16 layers, k=2048); "
+          "HBM GB/s vs roofline")
+FALLBACK_HBM_GBS = 6650.0
+QUERY_SETS = 8
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, burst copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s pool measurement)"
+
+
+def algorithmic_bytes(w):
+    """Bytes the method must move per step: the K cache once for routing plus
+    the selected K and V rows once (the set and the cache are shared by all
+    layers).  q, idx and out are < 0.3 MB and not counted."""
+    scan = w.B * w.Hkv * w.N * w.d * w.esize
+    gathered = 2 * w.B * w.Hkv * w.k * w.d * w.esize
+    return scan, gathered
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+_SMI_FIELDS = ["timestamp", "clocks.sm", "clocks.max.sm", "power.draw",
+               "clocks_event_reasons.active",
+               "clocks_event_reasons.hw_slowdown",
+               "clocks_event_reasons.hw_thermal_slowdown",
+               "clocks_event_reasons.sw_thermal_slowdown",
+               "clocks_event_reasons.sw_power_cap"]
+
+
+def _smi_id(local_rank: int) -> str:
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(local_rank).uuid)
+    except Exception:
+        return str(local_rank)
+
+
+def _smi_time(s: str) -> float:
+    from datetime import datetime
+    return datetime.strptime(s.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+
+
+class ClockSampler:
+    """nvidia-smi sampling in the background; only samples taken between
+    mark_start() and mark_stop() (the timed region) are summarised."""
+
+    def __init__(self, local_rank: int, interval_ms: int = 50):
+        self.dev = _smi_id(local_rank)
+        self.interval = interval_ms
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_stop(self):
+        self.t1 = time.time()
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}",
+                 "--query-gpu=" + ",".join(_SMI_FIELDS),
+                 "--format=csv,noheader,nounits", f"-lms", str(self.interval)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        time.sleep(0.15)
+
+    def result(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) == len(_SMI_FIELDS)]
+        try:
+            if self.t0 is not None and self.t1 is not None:
+                rows = [r for r in rows if self.t0 - 0.05 <= _smi_time(r[0]) <= self.t1 + 0.05]
+        except Exception:
+            pass
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def time_graphs(graphs, steps: int, warmup: int, stream, sampler=None) -> float:
+    """Replay graphs[i % len] for warmup + steps iterations; return the
+    CUDA-event time (ms) of the last `steps` replays, bracketed by a barrier
+    and device synchronisation."""
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    sdist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.mark_start()
+    start.record(stream)
+    for i in range(steps):
+        graphs[i % len(graphs)].replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark_stop()
+    sdist.barrier()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
+
+
+def capture(fn_list, stream):
+    graphs = []
+    for fn in fn_list:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        graphs.append(g)
+    return graphs
+
+
+def traffic_record(kernel_file: str):
+    """ncu DRAM bytes per launch of the dominant kernel, valid only while the
+    kernel source is unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "score_kernel_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        with open(kernel_file, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        if rec.get("source_sha256") == sha:
+            return rec
+    except Exception:
+        pass
+    return None
+
+
+def run_native(args, rank, world, local_rank):
+    import token_sparse_attention_sm_b200 as sd
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    base = synth.WORKLOADS[args.workload]
+    # each rank decodes its own sequences (independent seeds)
+    w = base.with_(seeds=tuple(s + 1000 * rank for s in base.seeds))
+    x = synth.generate(w)
+    variants = synth.query_variants(w, x, QUERY_SETS, seed=2000 + 1000 * rank)
+    K = x["K"].to(dev)
+    V = x["V"].to(dev)
+    qs = [(qr.to(dev), ql.to(dev)) for qr, ql in variants]
+    stream = torch.cuda.Stream(device=dev)
+    ws = sd.Workspace(dev)
+    # one workspace, sized up front for every op timed below, so that no
+    # captured graph refers to a buffer that is later replaced
+    ws.get(max(sd.workspace_bytes(w.B, w.N, w.Hq, w.Hkv, w.d, w.torch_dtype, w.k, w.L),
+               sd.workspace_bytes(w.B, w.N, w.Hkv, w.Hkv, 64, torch.float32, w.k, 1)))
+    outs = [dict(out=torch.empty_like(ql), idx=torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device=dev),
+                 lse=torch.empty((w.L, w.B, w.Hq), dtype=torch.float32, device=dev)) for _, ql in qs]
+
+    def step_fn(i):
+        qr, ql = qs[i]
+        o = outs[i]
+        return lambda: sd.decode_step(qr, ql, K, V, k=w.k, ws=ws, check=False,
+                                      out=o["out"], idx=o["idx"], lse=o["lse"])
+
+    with torch.cuda.stream(stream):
+        for i in range(len(qs)):          # warm the workspace and the library
+            step_fn(i)()
+        sd.read_device_status(ws)
+        graphs = capture([step_fn(i) for i in range(len(qs))], stream)
+        with ClockSampler(local_rank) as cs:
+            ms = time_graphs(graphs, args.steps, args.warmup, stream, cs)
+        clocks = cs.result()
+        sd.read_device_status(ws)         # no device-side condition in the run
+
+        # per-kernel durations, each kernel alone in a graph of back-to-back
+        # launches over the rotating queries (CUDA events on this stream)
+        S_buf = torch.empty((w.B, w.Hkv, w.N), dtype=torch.float32, device=dev)
+        idx0 = outs[0]["idx"]
+        # size the workspace for every op before any capture
+        sd.score(qs[0][0], K, ws=ws, check=False, out=S_buf)
+        sd.select_topk(S_buf, w.k, ws=ws, check=False, idx=idx0)
+        sd.attn_gather(qs[0][1], K, V, idx0, ws=ws, check=False, out=outs[0]["out"],
+                       lse=outs[0]["lse"])
+        torch.cuda.synchronize()
+        score_graphs = capture([lambda qr=qr: sd.score(qr, K, ws=ws, check=False, out=S_buf)
+                                for qr, _ in qs], stream)
+        n_k = max(args.steps // 4, 64)
+        t_score = time_graphs(score_graphs, n_k, max(args.warmup, 3), stream) / n_k
+        sel_graphs = capture([lambda: sd.select_topk(S_buf, w.k, ws=ws, check=False, idx=idx0)],
+                             stream)
+        t_sel = time_graphs(sel_graphs, n_k, max(args.warmup, 3), stream) / n_k
+        attn_graphs = capture([lambda qi=qi: sd.attn_gather(qs[qi][1], K, V, outs[qi]["idx"], ws=ws,
+                                                            check=False, out=outs[qi]["out"],
+                                                            lse=outs[qi]["lse"])
+                               for qi in range(len(qs))], stream)
+        t_attn = time_graphs(attn_graphs, n_k, max(args.warmup, 3), stream) / n_k
+        sd.read_device_status(ws)
+
+    ms_max = sdist.max_over_ranks(ms)
+    t_score_max = sdist.max_over_ranks(t_score)
+    ms_per_step = ms_max / args.steps
+    value = world * args.steps / (ms_max / 1e3)
+
+    # end to end through the public API: pinned host queries in, results out
+    e2e = run_e2e(sd, w, variants, K, V, ws, stream, dev, args, world)
+
+    peak, peak_src = load_peaks()
+    scan_b, gath_b = algorithmic_bytes(w)
+    achieved = scan_b / (t_score_max * 1e-3) / 1e9
+    trec = traffic_record(os.path.join(ROOT, "token_sparse_attention_sm_b200", "csrc", "score.cu"))
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded Gaussian K/V/q, planted heavy hitters, x8 outlier channel)",
+        "config": {
+            "workload": w.name, "B": w.B, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv,
+            "d": w.d, "k": w.k, "L": w.L, "parallelism": f"replicas x{world}",
+            "query_sets": QUERY_SETS,
+            "l2": "inputs larger than L2 (K+V = %.0f MB per replica); the query "
+                  "rotates over %d sets so the selected rows change every step"
+                  % (2 * scan_b / 1e6, QUERY_SETS),
+            "timing": "one CUDA graph per decode step (4 kernels), replayed; "
+                      "CUDA events on the launch stream; max over ranks",
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "score_kernel (routing scan)",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": trec.get("traffic_bytes_per_launch") if trec else None,
+            "algorithmic_bytes_per_launch": scan_b,
+            "avg_launch_us": round(t_score_max * 1e3, 2),
+            "peak_source": peak_src,
+        },
+        "step_roofline": {
+            "unique_bytes_per_step": scan_b + gath_b,
+            "achieved_gbs": round((scan_b + gath_b) / (ms_per_step * 1e-3) / 1e9, 1),
+            "frac_of_measured_peak": round((scan_b + gath_b) / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+        },
+        "kernels_us": {"score": round(t_score * 1e3, 2), "select": round(t_sel * 1e3, 2),
+                       "attn_gather_all_layers": round(t_attn * 1e3, 2),
+                       "note": "each kernel timed alone in back-to-back graph launches; "
+                               "attention alone may find its rows in L2"},
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_full(w, x)
+    return line
+
+
+def run_e2e(sd, w, variants, K, V, ws, stream, dev, args, world):
+    """Same metric through the public Python API with host buffers: every
+    step copies its queries from pinned host memory to the device, runs the
+    decode step, and reads the outputs and index set back to pinned host
+    memory (synchronised), all inside the timed region."""
+    hq = [(qr.pin_memory(), ql.pin_memory()) for qr, ql in variants]
+    dq = [(torch.empty_like(qr, device=dev), torch.empty_like(ql, device=dev)) for qr, ql in variants]
+    out_h = torch.empty(tuple(variants[0][1].shape), dtype=variants[0][1].dtype).pin_memory()
+    idx_h = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32).pin_memory()
+    out_d = torch.empty(tuple(variants[0][1].shape), dtype=variants[0][1].dtype, device=dev)
+    idx_d = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device=dev)
+    steps = min(args.steps, 2000)
+    h2d = hq[0][0].numel() * hq[0][0].element_size() + hq[0][1].numel() * hq[0][1].element_size()
+    d2h = out_h.numel() * out_h.element_size() + idx_h.numel() * idx_h.element_size()
+
+    def one(i):
+        hqr, hql = hq[i % len(hq)]
+        dqr, dql = dq[i % len(dq)]
+        dqr.copy_(hqr, non_blocking=True)
+        dql.copy_(hql, non_blocking=True)
+        sd.decode_step(dqr, dql, K, V, k=w.k, ws=ws, check=False, out=out_d, idx=idx_d,
+                       return_lse=False)
+        out_h.copy_(out_d, non_blocking=True)
+        idx_h.copy_(idx_d, non_blocking=True)
+        stream.synchronize()
+
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            one(i)
+        torch.cuda.synchronize()
+        sdist.barrier()
+        t0 = time.perf_counter()
+        for i in range(steps):
+            one(i)
+        t1 = time.perf_counter()
+        sdist.barrier()
+    sec = sdist.max_over_ranks(t1 - t0)
+    return {"value": round(world * steps / sec, 2), "unit": "steps/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "api": "token_sparse_attention_sm_b200.decode_step (eager, per-step sync)"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs
+# ---------------------------------------------------------------------------
+
+def cpu_baseline_full(w, x, budget_s: float = 10.0):
+    """The C oracle, as it stands, on full decode steps of the same workload,
+    repeated until about `budget_s` seconds of CPU work."""
+    import oracle
+    qr, ql = synth.f32(x["q_route"]), synth.f32(x["q_layers"])
+    Kf, Vf = synth.f32(x["K"]), synth.f32(x["V"])
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode_step(qr, ql, Kf, Vf, k=w.k)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    sec = time.perf_counter() - t0
+    return {"value": round(n / sec, 4), "unit": "steps/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n} full decode steps of {w.name} (all {w.B * w.Hkv} KV heads, "
+                      f"{w.L} layers) by the plain C oracle with OpenMP, {sec:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the CPU oracle timed on bounded samples of the workload.
+    A sample is one KV head's sub-problem (its G query heads) over the first
+    n keys of the cache with k scaled in proportion, sized so the whole run
+    takes about a minute; steps/s is scaled to full steps by the fraction of
+    the step's keys the sample covers."""
+    import oracle
+    w = synth.WORKLOADS[args.workload]
+    x = synth.generate(w.with_(N=min(w.N, 131072)))
+    G = w.G
+    qr = synth.f32(x["q_route"][:1, :G])
+    ql = synth.f32(x["q_layers"][:, :1, :G])
+    K_all = synth.f32(x["K"][:1, :1])
+    V_all = synth.f32(x["V"][:1, :1])
+
+    def sample(n):
+        kk = max(1, round(w.k * n / w.N))
+        t0 = time.perf_counter()
+        oracle.decode_step(qr, ql, K_all[:, :, :n], V_all[:, :, :n], k=kk)
+        return time.perf_counter() - t0
+
+    t_full_head = sample(w.N)                       # calibration, untimed
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    n = int(min(w.N, max(1024, w.N * budget / max(t_full_head, 1e-6))))
+    for _ in range(args.warmup):
+        sample(n)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        sample(n)
+    sec = time.perf_counter() - t0
+    frac = (n / w.N) / (w.B * w.Hkv)                # share of one full step
+    value = args.steps * frac / sec
+    desc = (f"{args.steps} samples, each the oracle decode step of one KV head "
+            f"(G={G} query heads, L={w.L}) over the first {n} of {w.N} keys with "
+            f"k={max(1, round(w.k * n / w.N))}; value scaled by {frac:.3g} step per sample")
+    return {
+        "metric": METRIC, "value": round(value, 5), "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 / value, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 attention / f32 scores (CPU oracle)", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv,
+                   "d": w.d, "k": w.k, "L": w.L, "parallelism": "host cores"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 5), "unit": "steps/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 5), "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="decode_128k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local_rank = sdist.env_rank_world()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+    sdist.init("nccl")
+    try:
+        line = run_native(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        sdist.finalize()
+
+
+if __name__ == "__main__":
+    main()

@@ -343,3 +343,32 @@ def test_decode_step_threshold_empty_set(dev):
     res = sd.decode_step(t["q_route"], t["q_layers"], t["K"], t["V"], tau=tau, cap=64)
     assert res["count"].cpu().tolist() == [[0, 0]]
     assert torch.all(res["out"] == 0) and torch.all(torch.isneginf(res["lse"]))
+
+
+def test_route_topk_all_equal_keys_takes_lowest_indices(dev):
+    """Every score equal: the boundary bin holds all N keys, more than the
+    candidate buffers, so the select takes its general path."""
+    w = synth.custom(B=1, N=20000, Hq=8, Hkv=2, d=128, L=1, k=300, dtype="bf16", seed=4)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    K = t["K"].clone()
+    K[:] = K[:, :, :1, :]
+    idx = sd.route_topk(t["q_route"], K, 300).cpu().numpy()
+    np.testing.assert_array_equal(idx, np.tile(np.arange(300), (1, 2, 1)))
+
+
+def test_route_topk_recovers_from_dirty_workspace(dev):
+    """A workspace whose histogram area holds garbage (not zero-filled) is
+    detected (the counts do not sum to N) and the result is still exact; the
+    call leaves the workspace clean for the next one."""
+    w = synth.custom(B=2, N=5000, Hq=8, Hkv=2, d=128, L=1, k=100, dtype="bf16", seed=6)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
+    ws = sd.Workspace(dev)
+    ws.get(sd.workspace_bytes(2, 5000, 8, 2, 128, torch.bfloat16, 100, 1))
+    ws.buf[256:256 + 4 * 2048 * 4] = 7
+    for _ in range(2):
+        gidx = sd.route_topk(t["q_route"], t["K"], 100, ws=ws).cpu().numpy()
+        assert_topk_within_band(gidx, S, 100)
+    assert int(ws.buf[256:256 + 4 * 2048 * 4].sum()) == 0

@@ -191,14 +191,14 @@ def _dims_qk(q, K):
     return B, N, Hq, Hkv, d
 
 
-def score(q, K, ws: Workspace | None = None, check: bool = True):
-    """Routing scores S [B,Hkv,N] fp32."""
-    _need_cuda(q, K)
+def score(q, K, ws: Workspace | None = None, check: bool = True, out=None):
+    """Routing scores S [B,Hkv,N] fp32 (written into ``out`` if given)."""
+    _need_cuda(q, K, out)
     B, N, Hq, Hkv, d = _dims_qk(q, K)
     w = _ws(ws, q.device)
     sh = _shape(B, N, Hq, Hkv, d, q.dtype)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, 1, 1))
-    S = torch.empty((B, Hkv, N), dtype=torch.float32, device=q.device)
+    S = torch.empty((B, Hkv, N), dtype=torch.float32, device=q.device) if out is None else out
     _check(load().sparse_score(ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(S),
                                _ptr(buf), buf.numel(), _stream()), "score")
     if check:
@@ -206,14 +206,16 @@ def score(q, K, ws: Workspace | None = None, check: bool = True):
     return S
 
 
-def select_topk(S, k: int, ws: Workspace | None = None, check: bool = True):
+def select_topk(S, k: int, ws: Workspace | None = None, check: bool = True,
+                idx=None):
     """Top-k of S [B,Hkv,N] fp32 -> idx [B,Hkv,k] int32 ascending."""
-    _need_cuda(S)
+    _need_cuda(S, idx)
     B, Hkv, N = S.shape
     w = _ws(ws, S.device)
     sh = _shape(B, N, Hkv, Hkv, 64, torch.float32)
     buf = w.get(workspace_bytes(B, N, Hkv, Hkv, 64, torch.float32, k, 1))
-    idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=S.device)
+    if idx is None:
+        idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=S.device)
     _check(load().sparse_select_topk(ctypes.byref(sh), _ptr(S), int(k), _ptr(idx),
                                      _ptr(buf), buf.numel(), _stream()),
            "select_topk")
@@ -277,7 +279,7 @@ def route_threshold(q, K, tau, cap: int, ws: Workspace | None = None,
 
 
 def attn_gather(q, K, V, idx, count=None, ws: Workspace | None = None,
-                check: bool = True, return_lse: bool = True):
+                check: bool = True, return_lse: bool = True, out=None, lse=None):
     """Attention of q ([B,Hq,d] or [L,B,Hq,d]) over the idx rows
     [B,Hkv,stride] (first count[b,h] of each row if count is given).
     Returns (out, lse) with out shaped like q."""
@@ -294,8 +296,14 @@ def attn_gather(q, K, V, idx, count=None, ws: Workspace | None = None,
     w = _ws(ws, q.device)
     sh = _shape(B, N, Hq, Hkv, d, q.dtype)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, stride, L))
-    out = torch.empty_like(q4)
-    lse = torch.empty((L, B, Hq), dtype=torch.float32, device=q.device) if return_lse else None
+    if out is None:
+        out = torch.empty_like(q4)
+    elif single:
+        out = out.unsqueeze(0)
+    if lse is None and return_lse:
+        lse = torch.empty((L, B, Hq), dtype=torch.float32, device=q.device)
+    elif lse is not None and single:
+        lse = lse.unsqueeze(0)
     _check(load().sparse_attn_gather(
         ctypes.byref(sh), L, _ptr(q4), _ptr(K), _ptr(V), _ptr(idx), stride,
         _ptr(count), _ptr(out), _ptr(lse), _ptr(buf), buf.numel(), _stream()),

@@ -5,8 +5,10 @@
 // stream and returns.  The library allocates nothing: scratch lives in the
 // caller's workspace, whose layout is
 //   [0, 256)              header: device status word (uint32) at offset 0
-//   [256, 256 + S bytes)  fp32 scores S [B,Hkv,N]
-//   [.., ..)              attention split partials
+//   [256, ..)             radix histogram [B*Hkv][2048] uint32 (scan -> select;
+//                         the select kernel clears it after use)
+//   [.., ..)              fp32 scores S [B,Hkv,N]
+//   [.., ..)              attention split partials (fp32 inputs only)
 #include <mutex>
 
 #include "common.cuh"
@@ -27,12 +29,15 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 constexpr size_t kHeader = 256;
 
 struct Layout {
-  size_t scores_off, scores_bytes, attn_off, attn_bytes, total;
+  size_t hist_off, hist_bytes, scores_off, scores_bytes, attn_off, attn_bytes,
+      total;
 };
 
 Layout layout(const Shape &s, int stride, int L) {
   Layout l;
-  l.scores_off = kHeader;
+  l.hist_off = kHeader;
+  l.hist_bytes = align_up((size_t)s.BH() * 2048 * sizeof(uint32_t), 256);
+  l.scores_off = l.hist_off + l.hist_bytes;
   l.scores_bytes = align_up((size_t)s.BH() * s.N * sizeof(float), 256);
   l.attn_off = l.scores_off + l.scores_bytes;
   l.attn_bytes = align_up(attn_workspace_bytes(s, L, stride), 256);
@@ -75,6 +80,9 @@ sparse_status_t from_cuda(cudaError_t e) {
 }
 
 uint32_t *status_word(void *ws) { return static_cast<uint32_t *>(ws); }
+uint32_t *hist_ptr(void *ws, const Layout &l) {
+  return reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + l.hist_off);
+}
 float *scores_ptr(void *ws, const Layout &l) {
   return reinterpret_cast<float *>(static_cast<char *>(ws) + l.scores_off);
 }
@@ -158,7 +166,7 @@ sparse_status_t sparse_score(const sparse_shape_t *shape, const void *q,
   if (!sd::aligned(q, 16) || !sd::aligned(K, 16) || !sd::aligned(S, 16))
     return SPARSE_ERR_INVALID_ARG;
   if ((r = sd::check_ws(s, 1, 1, ws, ws_bytes)) != SPARSE_OK) return r;
-  return sd::from_cuda(sd::launch_score(s, q, K, S, sd::status_word(ws),
+  return sd::from_cuda(sd::launch_score(s, q, K, S, nullptr, sd::status_word(ws),
                                         static_cast<cudaStream_t>(stream)));
 }
 
@@ -172,7 +180,7 @@ sparse_status_t sparse_select_topk(const sparse_shape_t *shape,
   if (!sd::aligned(S, 16) || !sd::aligned(idx, 4)) return SPARSE_ERR_INVALID_ARG;
   if ((r = sd::check_ws(s, k, 1, ws, ws_bytes)) != SPARSE_OK) return r;
   return sd::from_cuda(sd::launch_select(s, S, k, nullptr, 0, idx, nullptr, k,
-                                         sd::status_word(ws),
+                                         nullptr, sd::status_word(ws),
                                          static_cast<cudaStream_t>(stream)));
 }
 
@@ -190,7 +198,7 @@ sparse_status_t sparse_select_threshold(const sparse_shape_t *shape,
     return SPARSE_ERR_INVALID_ARG;
   if ((r = sd::check_ws(s, cap, 1, ws, ws_bytes)) != SPARSE_OK) return r;
   return sd::from_cuda(sd::launch_select(s, S, 0, tau, cap, idx, count, cap,
-                                         sd::status_word(ws),
+                                         nullptr, sd::status_word(ws),
                                          static_cast<cudaStream_t>(stream)));
 }
 
@@ -207,9 +215,10 @@ sparse_status_t sparse_route_topk(const sparse_shape_t *shape, const void *q,
   const sd::Layout l = sd::layout(s, k, 1);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float *S = sd::scores_ptr(ws, l);
-  cudaError_t e = sd::launch_score(s, q, K, S, sd::status_word(ws), st);
+  uint32_t *hist = sd::hist_ptr(ws, l);
+  cudaError_t e = sd::launch_score(s, q, K, S, hist, sd::status_word(ws), st);
   if (e == cudaSuccess)
-    e = sd::launch_select(s, S, k, nullptr, 0, idx, nullptr, k,
+    e = sd::launch_select(s, S, k, nullptr, 0, idx, nullptr, k, hist,
                           sd::status_word(ws), st);
   return sd::from_cuda(e);
 }
@@ -230,9 +239,9 @@ sparse_status_t sparse_route_threshold(const sparse_shape_t *shape,
   const sd::Layout l = sd::layout(s, cap, 1);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float *S = sd::scores_ptr(ws, l);
-  cudaError_t e = sd::launch_score(s, q, K, S, sd::status_word(ws), st);
+  cudaError_t e = sd::launch_score(s, q, K, S, nullptr, sd::status_word(ws), st);
   if (e == cudaSuccess)
-    e = sd::launch_select(s, S, 0, tau, cap, idx, count, cap,
+    e = sd::launch_select(s, S, 0, tau, cap, idx, count, cap, nullptr,
                           sd::status_word(ws), st);
   return sd::from_cuda(e);
 }
@@ -290,10 +299,11 @@ sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t *status = sd::status_word(ws);
   float *S = sd::scores_ptr(ws, l);
-  cudaError_t e = sd::launch_score(s, q_route, K, S, status, st);
+  uint32_t *hist = topk ? sd::hist_ptr(ws, l) : nullptr;
+  cudaError_t e = sd::launch_score(s, q_route, K, S, hist, status, st);
   if (e == cudaSuccess)
-    e = topk ? sd::launch_select(s, S, k, nullptr, 0, idx, nullptr, k, status, st)
-             : sd::launch_select(s, S, 0, tau, cap, idx, count, cap, status, st);
+    e = topk ? sd::launch_select(s, S, k, nullptr, 0, idx, nullptr, k, hist, status, st)
+             : sd::launch_select(s, S, 0, tau, cap, idx, count, cap, nullptr, status, st);
   if (e == cudaSuccess)
     e = sd::launch_attn(s, L, q_layers, K, V, idx, stride, topk ? nullptr : count,
                         stride, out, lse, sd::attn_ptr(ws, l), status, st);

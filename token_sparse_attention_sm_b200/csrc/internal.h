@@ -19,23 +19,33 @@ struct Shape {
 struct DeviceInfo {
   int sm_count = 0;
   int max_smem_optin = 0;
-  int select_cluster = 0;  // cluster size the select kernel uses
+  int select_cluster = 0;  // largest cluster size the library launches
 };
 cudaError_t device_info(DeviceInfo *out);
 
-// A1: S[b,h,j] for every key; one streaming pass over K.
+// A1: S[b,h,j] for every key; one streaming pass over K.  hist (nullable):
+// [B*Hkv][2048] counts of the top 11 key bits, accumulated (must start zero).
 cudaError_t launch_score(const Shape &s, const void *q, const void *K,
-                         float *S, uint32_t *status, cudaStream_t st);
+                         float *S, uint32_t *hist, uint32_t *status,
+                         cudaStream_t st);
 
 // A2 / A2': selection from S.  k >= 1: top-k (tau ignored); k == 0:
 // threshold with tau and cap, count written.  idx rows have `stride`
 // entries.
+// hist (top-k, nullable): the scan's histogram; consumed and cleared.
 cudaError_t launch_select(const Shape &s, const float *S, int k,
                           const float *tau, int cap, int *idx, int *count,
-                          int stride, uint32_t *status, cudaStream_t st);
+                          int stride, uint32_t *hist, uint32_t *status,
+                          cudaStream_t st);
 
-// A3 + A4: L query sets over the same index rows.
+// A3 + A4: L query sets over the same index rows.  bf16 runs on the tensor
+// cores with the split merge in distributed shared memory (no workspace);
+// fp32 runs on the CUDA cores with split partials in the workspace.
 size_t attn_workspace_bytes(const Shape &s, int L, int stride);
+cudaError_t launch_attn_mma(const Shape &s, int L, const void *q, const void *K,
+                            const void *V, const int *idx, int stride,
+                            const int *count, void *out, float *lse,
+                            uint32_t *status, cudaStream_t st);
 cudaError_t launch_attn(const Shape &s, int L, const void *q, const void *K,
                         const void *V, const int *idx, int stride,
                         const int *count, int count_cap, void *out, float *lse,

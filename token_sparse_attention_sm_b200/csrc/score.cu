@@ -22,6 +22,11 @@
 //    round (rows are split over LPK lanes), keeps one partial dot per round,
 //    and a transposing shuffle reduction (LPK-1 shuffles for 32 keys) leaves
 //    one finished score per lane, stored as one coalesced 128-byte write.
+//  * Optionally (hist != nullptr) the scan also counts, per (sequence, KV
+//    head), the scores by the top 11 bits of their order-preserving key --
+//    the first level of the radix top-k -- in shared memory, and adds the
+//    non-zero bins to the global histogram at the end.  This costs nothing
+//    in a memory-bound scan and saves the select kernel a pass.
 #include "common.cuh"
 #include "internal.h"
 
@@ -32,7 +37,10 @@ constexpr int kConsumerWarps = 4;
 constexpr int kStages = 5;
 constexpr int kStageBytes = 32768;
 constexpr int kScoreThreads = (kConsumerWarps + 1) * 32;
-constexpr int kScoreSmem = kStages * kStageBytes + 2 * kStages * 8;
+constexpr int kHistBins = 2048;
+constexpr int kHistSlots = 4;  // heads a CTA can count in shared memory
+constexpr int kScoreSmem =
+    kStages * kStageBytes + kHistSlots * kHistBins * 4 + 2 * kStages * 8;
 
 template <typename T, int D>
 struct ScoreCfg {
@@ -72,17 +80,24 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const T *__restrict__ q, const T *__restrict__ K,
                  float *__restrict__ S, int N, int Hq, int Hkv,
                  int tiles_per_head, long long total_tiles, float scale,
-                 uint32_t *status) {
+                 uint32_t *__restrict__ hist, uint32_t *status) {
   using C = ScoreCfg<T, D>;
   extern __shared__ __align__(128) unsigned char smem[];
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
+  uint32_t *shist = reinterpret_cast<uint32_t *>(smem + kStages * kStageBytes);
+  uint64_t *full = reinterpret_cast<uint64_t *>(
+      smem + kStages * kStageBytes + kHistSlots * kHistBins * 4);
   uint64_t *empty = full + kStages;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long t_begin = (long long)blockIdx.x * total_tiles / gridDim.x;
   const long long t_end = (long long)(blockIdx.x + 1) * total_tiles / gridDim.x;
   const int ntiles = (int)(t_end - t_begin);
+  const int bh_first = (int)(t_begin / tiles_per_head);
 
+  if (hist) {
+    for (int i = threadIdx.x; i < kHistSlots * kHistBins; i += kScoreThreads)
+      shist[i] = 0u;
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -162,18 +177,39 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       TReduce<C::kLpk, C::kLpk / 2>::run(v, lane);
       const int kk = key0 + sub * C::kKpr + lane / C::kLpk;
       const bool valid = kk < nk;
-      if (valid) Srow[kk] = v[0];
+      if (valid) {
+        Srow[kk] = v[0];
+        if (hist) {
+          const uint32_t bin = order_key(v[0]) >> 21;
+          const int slot = bh - bh_first;
+          if (slot < kHistSlots)
+            atomicAdd(&shist[slot * kHistBins + bin], 1u);
+          else
+            atomicAdd(&hist[(size_t)bh * kHistBins + bin], 1u);
+        }
+      }
       if (__any_sync(0xffffffffu, valid && !isfinite(v[0])) && lane == 0)
         raise_flag(status, FLAG_NONFINITE);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
+  if (hist) {
+    // consumer warps only (named barrier 1): every count is in shared memory
+    asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
+    const int bh_last = ntiles > 0 ? (int)((t_end - 1) / tiles_per_head) : bh_first - 1;
+    const int nslots = min(kHistSlots, bh_last - bh_first + 1);
+    for (int i = threadIdx.x; i < nslots * kHistBins; i += kConsumerWarps * 32) {
+      const uint32_t c = shist[i];
+      if (c) atomicAdd(&hist[(size_t)(bh_first + i / kHistBins) * kHistBins + (i % kHistBins)], c);
+    }
+  }
 }
 
 template <typename T, int D>
 cudaError_t launch_score_t(const Shape &s, const void *q, const void *K,
-                           float *S, uint32_t *status, cudaStream_t st) {
+                           float *S, uint32_t *hist, uint32_t *status,
+                           cudaStream_t st) {
   using C = ScoreCfg<T, D>;
   DeviceInfo di;
   cudaError_t e = device_info(&di);
@@ -188,21 +224,22 @@ cudaError_t launch_score_t(const Shape &s, const void *q, const void *K,
   const float scale = (float)(1.0 / __builtin_sqrt((double)D));
   kern<<<grid, kScoreThreads, kScoreSmem, st>>>(
       static_cast<const T *>(q), static_cast<const T *>(K), S, s.N, s.Hq,
-      s.Hkv, tiles_per_head, total, scale, status);
+      s.Hkv, tiles_per_head, total, scale, hist, status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_score(const Shape &s, const void *q, const void *K,
-                         float *S, uint32_t *status, cudaStream_t st) {
+                         float *S, uint32_t *hist, uint32_t *status,
+                         cudaStream_t st) {
   if (s.dtype == 1) {
     if (s.d == 128)
-      return launch_score_t<__nv_bfloat16, 128>(s, q, K, S, status, st);
-    return launch_score_t<__nv_bfloat16, 64>(s, q, K, S, status, st);
+      return launch_score_t<__nv_bfloat16, 128>(s, q, K, S, hist, status, st);
+    return launch_score_t<__nv_bfloat16, 64>(s, q, K, S, hist, status, st);
   }
-  if (s.d == 128) return launch_score_t<float, 128>(s, q, K, S, status, st);
-  return launch_score_t<float, 64>(s, q, K, S, status, st);
+  if (s.d == 128) return launch_score_t<float, 128>(s, q, K, S, hist, status, st);
+  return launch_score_t<float, 64>(s, q, K, S, hist, status, st);
 }
 
 }  // namespace sd

@@ -13,18 +13,25 @@
 // needed).
 //  * Top-k is a radix select without any sort: an 11-bit histogram of the top
 //    key bits, then (only if the boundary bin still holds more keys than
-//    needed) 11 more bits, then the last 10 bits.  Each level builds a
-//    shared-memory histogram per CTA, one cluster barrier, and every CTA sums
-//    the C histograms through distributed shared memory and finds the bin in
-//    which the descending cumulative count reaches k (block-wide scan).  The
-//    result is either a key threshold T (take every key >= T) or the exact
-//    k-th key value v plus the number t of keys equal to v to take, which go
-//    to the lowest indices.
-//  * Compaction is order preserving: each thread owns a contiguous run of its
-//    CTA's slice; block scans give per-thread offsets, one more cluster
-//    barrier exchanges the per-CTA totals, and every selected index is
-//    written straight to its final position.  The output is therefore
-//    deterministic and ascending.
+//    needed) 11 more bits, then the last 10 bits.  The result is either a key
+//    threshold T (take every key >= T) or the exact k-th key value v plus the
+//    number t of keys equal to v to take, which go to the lowest indices.
+//  * Fast path: the score scan has already counted the top 11 bits per head
+//    (global histogram).  Every CTA reads it and finds the boundary bin; the
+//    few keys inside that bin (about k/... of N, a couple of thousand) are
+//    gathered from all CTAs of the cluster through distributed shared memory
+//    after one cluster barrier, and each CTA finishes the remaining 21 bits
+//    on that small candidate list locally, with no further cluster barrier.
+//    Rank 0 then clears the head's histogram for the next call.
+//  * General path (no histogram, a histogram that does not sum to N, or more
+//    candidates than fit): each level builds a shared-memory histogram per
+//    CTA, one cluster barrier, and every CTA sums the C histograms through
+//    distributed shared memory.
+//  * Compaction is order preserving: each warp owns a contiguous run of its
+//    CTA's slice and walks it 32 keys at a time; warp ballots and popcounts
+//    give positions, one more cluster barrier exchanges the per-CTA totals,
+//    and every selected index is written straight to its final position.
+//    The output is therefore deterministic and ascending.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -39,14 +46,22 @@ constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kBinsPerThread = kBins / kSelThreads;
-constexpr int kSelFixedSmem = 2 * kBins * 4 + 256;
+constexpr int kCandLocal = 2048;  // boundary-bin keys one CTA may hold
+constexpr int kCandAll = 8192;    // boundary-bin keys of a whole head
+constexpr int kSelFixedSmem = 2 * kBins * 4 + (kCandLocal + kCandAll) * 4 + 384;
 
 struct SelShared {
   uint32_t hist[2][kBins];
+  uint32_t cand_local[kCandLocal];  // read remotely by the other CTAs
+  uint32_t cand_all[kCandAll];
   uint32_t warp_buf[33];
   uint32_t pub[2];        // this CTA's (>= T count, == v count), read remotely
   uint32_t bnd[3];        // boundary bin, count above it, count in it
-  uint32_t pad[24];
+  uint32_t ncand;         // candidates in cand_local (may exceed kCandLocal)
+  uint32_t cinfo[2];      // total candidates, overflow flag
+  uint32_t wge[kSelWarps];  // per-warp counts of keys >= threshold
+  uint32_t weq[kSelWarps];  // per-warp counts of keys == tie value
+  uint32_t pad[2];
 };
 static_assert(sizeof(SelShared) <= kSelFixedSmem, "fixed select smem");
 
@@ -93,6 +108,7 @@ __device__ void find_boundary(cg::cluster_group &cluster, uint32_t *h,
   for (int e = 0; e < kBinsPerThread; ++e) {
     const int b = kBins - 1 - (kBinsPerThread * t + e);
     uint32_t acc = 0;
+#pragma unroll 4
     for (int r = 0; r < csize; ++r) acc += cluster.map_shared_rank(h, r)[b];
     c[e] = acc;
     sum += acc;
@@ -114,12 +130,42 @@ __device__ void find_boundary(cg::cluster_group &cluster, uint32_t *h,
   __syncthreads();
 }
 
-// k >= 1: top-k; k == 0: threshold (tau, cap, count).
+// As find_boundary, for a histogram held by this CTA alone.
+__device__ void find_boundary_local(const uint32_t *h, uint32_t need,
+                                    SelShared *sh) {
+  const int t = threadIdx.x;
+  uint32_t c[kBinsPerThread];
+  uint32_t sum = 0;
+#pragma unroll
+  for (int e = 0; e < kBinsPerThread; ++e) {
+    c[e] = h[kBins - 1 - (kBinsPerThread * t + e)];
+    sum += c[e];
+  }
+  uint32_t tot;
+  uint32_t above = block_excl_scan(sum, sh->warp_buf, &tot);
+  if (above < need && above + sum >= need) {
+#pragma unroll
+    for (int e = 0; e < kBinsPerThread; ++e) {
+      if (above + c[e] >= need) {
+        sh->bnd[0] = (uint32_t)(kBins - 1 - (kBinsPerThread * t + e));
+        sh->bnd[1] = above;
+        sh->bnd[2] = c[e];
+        break;
+      }
+      above += c[e];
+    }
+  }
+  __syncthreads();
+}
+
+// k >= 1: top-k; k == 0: threshold (tau, cap, count).  hist (top-k only,
+// may be null): per-head counts of the top 11 key bits from the score scan.
 template <bool IN_SMEM>
 __global__ void __launch_bounds__(kSelThreads)
     select_kernel(const float *__restrict__ S, int N, int k,
                   const float *__restrict__ tau, int cap, int *__restrict__ idx,
-                  int *__restrict__ count, int stride, uint32_t *status) {
+                  int *__restrict__ count, int stride,
+                  uint32_t *__restrict__ hist, uint32_t *status) {
   cg::cluster_group cluster = cg::this_cluster();
   const int csize = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
@@ -134,15 +180,24 @@ __global__ void __launch_bounds__(kSelThreads)
   const int n = hi - lo;
   const float *Sh = S + (size_t)bh * N + lo;
 
+  // Load the slice (8 independent loads in flight per thread) and keep it as
+  // order-preserving keys.
   bool bad = false;
-  if (IN_SMEM) {
-    for (int t = tid; t < n; t += kSelThreads) {
-      const float f = Sh[t];
-      bad |= !isfinite(f);
-      keys[t] = order_key(f);
+  for (int t0 = 0; t0 < n; t0 += kSelThreads * 8) {
+    float f[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int t = t0 + u * kSelThreads + tid;
+      f[u] = t < n ? Sh[t] : 0.f;
     }
-  } else {
-    for (int t = tid; t < n; t += kSelThreads) bad |= !isfinite(Sh[t]);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int t = t0 + u * kSelThreads + tid;
+      if (t < n) {
+        bad |= !isfinite(f[u]);
+        if (IN_SMEM) keys[t] = order_key(f[u]);
+      }
+    }
   }
   if (__syncthreads_or(bad) && tid == 0) raise_flag(status, FLAG_NONFINITE);
   auto key_at = [&](int t) -> uint32_t {
@@ -151,15 +206,128 @@ __global__ void __launch_bounds__(kSelThreads)
 
   // Selection rule: key >= t_ge, or (key == tie_val and its rank among the
   // keys equal to tie_val, in index order, is < n_ties).
-  uint64_t t_ge;
+  uint64_t t_ge = 0;
   uint32_t tie_val = 0, n_ties = 0;
   const uint32_t limit = k > 0 ? (uint32_t)k : (uint32_t)cap;
-  if (k > 0) {
+  bool fast = false;
+  bool hist_cleared = hist == nullptr;
+  if (k > 0 && hist) {
+    // ---- fast path: level 1 from the scan's histogram ----------------------
+    uint32_t *gh = hist + (size_t)bh * kBins;
+    uint32_t c[kBinsPerThread], sum = 0;
+#pragma unroll
+    for (int e = 0; e < kBinsPerThread; ++e) {
+      c[e] = gh[kBins - 1 - (kBinsPerThread * tid + e)];
+      sum += c[e];
+    }
+    uint32_t tot;
+    uint32_t above = block_excl_scan(sum, sh->warp_buf, &tot);
+    if (tid == 0) sh->ncand = 0;
+    if (tot == (uint32_t)N) {  // block-uniform: a clean, complete histogram
+      if (above < (uint32_t)k && above + sum >= (uint32_t)k) {
+#pragma unroll
+        for (int e = 0; e < kBinsPerThread; ++e) {
+          if (above + c[e] >= (uint32_t)k) {
+            sh->bnd[0] = (uint32_t)(kBins - 1 - (kBinsPerThread * tid + e));
+            sh->bnd[1] = above;
+            sh->bnd[2] = c[e];
+            break;
+          }
+          above += c[e];
+        }
+      }
+      fast = true;
+    }
+    __syncthreads();
+    uint32_t b1 = sh->bnd[0];
+    if (fast) {
+      const int lane = tid & 31;
+      for (int t0 = 0; t0 < n; t0 += kSelThreads) {
+        const int t = t0 + tid;
+        const uint32_t key = t < n ? key_at(t) : 0u;
+        const bool hit = t < n && (key >> 21) == b1;
+        const uint32_t m = __ballot_sync(0xffffffffu, hit);
+        if (m) {  // warp-aggregated slot reservation
+          uint32_t base = 0;
+          if (lane == 0) base = atomicAdd(&sh->ncand, (uint32_t)__popc(m));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          const uint32_t slot = base + __popc(m & ((1u << lane) - 1u));
+          if (hit && slot < (uint32_t)kCandLocal) sh->cand_local[slot] = key;
+        }
+      }
+    }
+    cluster.sync();  // candidates published; everyone has read the histogram
+    if (rank == 0)
+      for (int b = tid; b < kBins; b += kSelThreads) gh[b] = 0u;
+    hist_cleared = true;
+    if (fast) {
+      if (tid == 0) {
+        uint32_t total = 0, over = 0;
+        for (int r = 0; r < csize; ++r) {
+          const uint32_t nr = *cluster.map_shared_rank(&sh->ncand, r);
+          over |= nr > (uint32_t)kCandLocal;
+          total += nr;
+        }
+        sh->cinfo[0] = total;
+        sh->cinfo[1] = over | (total > (uint32_t)kCandAll);
+      }
+      __syncthreads();
+      if (sh->cinfo[1] == 0u) {
+        uint32_t off = 0;
+        for (int r = 0; r < csize; ++r) {
+          const uint32_t nr = *cluster.map_shared_rank(&sh->ncand, r);
+          const uint32_t *src = cluster.map_shared_rank(sh->cand_local, r);
+          for (uint32_t i = tid; i < nr; i += kSelThreads) sh->cand_all[off + i] = src[i];
+          off += nr;
+        }
+        const uint32_t ncand = sh->cinfo[0];
+        uint32_t need = (uint32_t)k - sh->bnd[1];
+        __syncthreads();
+        // level 2 on the candidates only (bits 20..10)
+        for (int b = tid; b < kBins; b += kSelThreads) sh->hist[1][b] = 0;
+        __syncthreads();
+        for (uint32_t i = tid; i < ncand; i += kSelThreads)
+          atomicAdd(&sh->hist[1][(sh->cand_all[i] >> 10) & 2047u], 1u);
+        __syncthreads();
+        find_boundary_local(sh->hist[1], need, sh);
+        const uint32_t b2 = sh->bnd[0];
+        need -= sh->bnd[1];
+        const uint32_t p2 = (b1 << 11) | b2;
+        if (sh->bnd[2] == need) {
+          t_ge = (uint64_t)p2 << 10;
+        } else {
+          for (int b = tid; b < kBins; b += kSelThreads) sh->hist[0][b] = 0;
+          __syncthreads();
+          for (uint32_t i = tid; i < ncand; i += kSelThreads) {
+            const uint32_t key = sh->cand_all[i];
+            if ((key >> 10) == p2) atomicAdd(&sh->hist[0][key & 1023u], 1u);
+          }
+          __syncthreads();
+          find_boundary_local(sh->hist[0], need, sh);
+          const uint32_t v = (p2 << 10) | sh->bnd[0];
+          need -= sh->bnd[1];
+          if (sh->bnd[2] == need) {
+            t_ge = v;
+          } else {
+            t_ge = (uint64_t)v + 1;
+            tie_val = v;
+            n_ties = need;
+          }
+        }
+      } else {
+        fast = false;  // uniform: every CTA saw the same counts
+      }
+    }
+  }
+  if (k > 0 && !fast) {
+    // ---- general path ------------------------------------------------------
     for (int b = tid; b < kBins; b += kSelThreads) sh->hist[0][b] = 0;
     __syncthreads();
     for (int t = tid; t < n; t += kSelThreads)
       atomicAdd(&sh->hist[0][key_at(t) >> 21], 1u);
     cluster.sync();
+    if (!hist_cleared && rank == 0)
+      for (int b = tid; b < kBins; b += kSelThreads) hist[(size_t)bh * kBins + b] = 0u;
     find_boundary(cluster, sh->hist[0], csize, (uint32_t)k, sh);
     const uint32_t b1 = sh->bnd[0];
     uint32_t need = (uint32_t)k - sh->bnd[1];
@@ -199,25 +367,37 @@ __global__ void __launch_bounds__(kSelThreads)
         }
       }
     }
-  } else {
+  } else if (k == 0) {
     const float tv = tau[bh];
     if (!isfinite(tv) && tid == 0 && rank == 0) raise_flag(status, FLAG_NONFINITE);
     t_ge = order_key(tv);
   }
 
   // ---- order-preserving compaction -----------------------------------------
-  const int per = (n + kSelThreads - 1) / kSelThreads;
-  const int c0 = min(n, tid * per), c1 = min(n, c0 + per);
-  uint32_t n_ge = 0, n_eq = 0;
-  for (int t = c0; t < c1; ++t) {
-    const uint32_t key = key_at(t);
-    n_ge += (uint64_t)key >= t_ge;
-    n_eq += (n_ties != 0u) & (key == tie_val);
+  // Warp w owns the contiguous segment [s0, s1) of this CTA's slice and walks
+  // it 32 keys at a time (conflict-free reads); ballots keep index order.
+  const int lane = tid & 31, wid = tid >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int s0 = (int)((long long)n * wid / kSelWarps);
+  const int s1 = (int)((long long)n * (wid + 1) / kSelWarps);
+  uint32_t w_ge = 0, w_eq = 0;
+  for (int t0 = s0; t0 < s1; t0 += 32) {
+    const int t = t0 + lane;
+    const bool in = t < s1;
+    const uint32_t key = in ? key_at(t) : 0u;
+    w_ge += __popc(__ballot_sync(0xffffffffu, in && (uint64_t)key >= t_ge));
+    if (n_ties) w_eq += __popc(__ballot_sync(0xffffffffu, in && key == tie_val));
   }
-  uint32_t cta_ge, cta_eq;
-  const uint32_t ex_ge = block_excl_scan(n_ge, sh->warp_buf, &cta_ge);
-  const uint32_t ex_eq = block_excl_scan(n_eq, sh->warp_buf, &cta_eq);
-  (void)ex_ge;
+  if (lane == 0) {
+    sh->wge[wid] = w_ge;
+    sh->weq[wid] = w_eq;
+  }
+  __syncthreads();
+  uint32_t cta_ge = 0, cta_eq = 0;
+  for (int i = 0; i < kSelWarps; ++i) {
+    cta_ge += sh->wge[i];
+    cta_eq += sh->weq[i];
+  }
   if (tid == 0) {
     sh->pub[0] = cta_ge;
     sh->pub[1] = cta_eq;
@@ -233,21 +413,31 @@ __global__ void __launch_bounds__(kSelThreads)
     total_sel += ge_r + ties_r;
     eq_pre += eq_r;
   }
-  const uint32_t tie0 = base_eq + ex_eq;
-  const uint32_t my_ties = n_ties > tie0 ? min(n_eq, n_ties - tie0) : 0u;
-  uint32_t cta_sel;
-  const uint32_t ex_sel = block_excl_scan(n_ge + my_ties, sh->warp_buf, &cta_sel);
-  uint32_t pos = base_sel + ex_sel;
-  uint32_t tie_rank = tie0;
+  // keys taken by the warps before this one, and this warp's first tie rank
+  uint32_t pos = base_sel, tie_rank = base_eq;
+  for (int i = 0; i < wid; ++i) {
+    const uint32_t ties_i = n_ties > tie_rank ? min(sh->weq[i], n_ties - tie_rank) : 0u;
+    pos += sh->wge[i] + ties_i;
+    tie_rank += sh->weq[i];
+  }
   int *out = idx + (size_t)bh * stride;
-  for (int t = c0; t < c1; ++t) {
-    const uint32_t key = key_at(t);
-    bool take = (uint64_t)key >= t_ge;
-    if (!take && n_ties != 0u && key == tie_val) take = tie_rank++ < n_ties;
-    if (take) {
-      if (pos < limit) out[pos] = lo + t;
-      ++pos;
+  for (int t0 = s0; t0 < s1; t0 += 32) {
+    const int t = t0 + lane;
+    const bool in = t < s1;
+    const uint32_t key = in ? key_at(t) : 0u;
+    const uint32_t ge = __ballot_sync(0xffffffffu, in && (uint64_t)key >= t_ge);
+    uint32_t take = ge;
+    if (n_ties) {
+      const uint32_t eq = __ballot_sync(0xffffffffu, in && key == tie_val);
+      const bool mine = ((eq >> lane) & 1u) && tie_rank + __popc(eq & lt_mask) < n_ties;
+      take |= __ballot_sync(0xffffffffu, mine);
+      tie_rank += __popc(eq);
     }
+    if ((take >> lane) & 1u) {
+      const uint32_t p = pos + __popc(take & lt_mask);
+      if (p < limit) out[p] = lo + t;
+    }
+    pos += __popc(take);
   }
   if (rank == 0 && tid == 0) {
     if (k > 0) {
@@ -285,7 +475,8 @@ cudaError_t select_cluster_size(int sm_count, int smem_optin, int *out);
 
 cudaError_t launch_select(const Shape &s, const float *S, int k,
                           const float *tau, int cap, int *idx, int *count,
-                          int stride, uint32_t *status, cudaStream_t st) {
+                          int stride, uint32_t *hist, uint32_t *status,
+                          cudaStream_t st) {
   SelectPlan plan;
   cudaError_t e = plan_select(s, &plan);
   if (e != cudaSuccess) return e;
@@ -308,7 +499,7 @@ cudaError_t launch_select(const Shape &s, const float *S, int k,
     if (e == cudaSuccess && plan.csize > 8)
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, kern, S, s.N, k, tau, cap, idx, count, stride, status);
+    e = cudaLaunchKernelEx(&cfg, kern, S, s.N, k, tau, cap, idx, count, stride, hist, status);
   } else {
     auto kern = select_kernel<false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -316,7 +507,7 @@ cudaError_t launch_select(const Shape &s, const float *S, int k,
     if (e == cudaSuccess && plan.csize > 8)
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, kern, S, s.N, k, tau, cap, idx, count, stride, status);
+    e = cudaLaunchKernelEx(&cfg, kern, S, s.N, k, tau, cap, idx, count, stride, hist, status);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -1,0 +1,49 @@
+"""Run a few launches of one entry point on a named workload, for profilers.
+
+    python -m token_sparse_attention_sm_b200.profile_case \
+        --workload decode_128k --op decode --reps 3
+
+--op is one of: score, route, attn, decode.  Inputs come from the seeded
+generator; nothing is checked or timed here (use bench.py for timing and the
+tests for parity).  The process exits non-zero if the device reports any
+condition."""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+import token_sparse_attention_sm_b200 as sd
+from token_sparse_attention_sm_b200 import synth
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="decode_128k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--op", default="decode", choices=["score", "route", "attn", "decode"])
+    ap.add_argument("--reps", type=int, default=3)
+    a = ap.parse_args()
+    w = synth.WORKLOADS[a.workload]
+    x = synth.generate(w)
+    dev = torch.device("cuda", 0)
+    t = {n: x[n].to(dev) for n in ("q_route", "q_layers", "K", "V")}
+    ws = sd.Workspace(dev)
+    k = w.k if w.mode == "topk" else w.cap
+    idx = sd.route_topk(t["q_route"], t["K"], k, ws=ws) if a.op == "attn" else None
+    for _ in range(a.reps):
+        if a.op == "score":
+            sd.score(t["q_route"], t["K"], ws=ws, check=False)
+        elif a.op == "route":
+            sd.route_topk(t["q_route"], t["K"], k, ws=ws, check=False)
+        elif a.op == "attn":
+            sd.attn_gather(t["q_layers"], t["K"], t["V"], idx, ws=ws, check=False)
+        else:
+            sd.decode_step(t["q_route"], t["q_layers"], t["K"], t["V"], k=k, ws=ws,
+                           check=False)
+    torch.cuda.synchronize()
+    sd.read_device_status(ws)
+    print(f"{a.op} x{a.reps} on {w.name}: ok")
+
+
+if __name__ == "__main__":
+    main()

@@ -175,3 +175,23 @@ def generate(w: Workload, batches=None) -> dict:
 def f32(t: torch.Tensor) -> np.ndarray:
     """Exact float32 numpy view of a workload tensor (bf16 widens exactly)."""
     return np.ascontiguousarray(t.float().numpy())
+
+
+def query_variants(w: Workload, x: dict, n: int, seed: int = 1000) -> list:
+    """``n`` further decode queries for the same cache, for benchmarks that
+    rotate queries so the selected rows change from step to step.
+
+    Variant r (r >= 1) draws, per sequence, with default_rng(seed + r):
+    q_route = x's q_route + 0.5 * N(0,1) (so the planted keys stay relevant)
+    and fresh N(0,1) q_layers; both rounded to the dtype.  Variant 0 is x's
+    own pair."""
+    out = [(x["q_route"], x["q_layers"])]
+    for r in range(1, n):
+        rng = np.random.default_rng(seed + r)
+        qr = x["q_route"].float().numpy()
+        noise = rng.standard_normal(qr.shape, dtype=np.float32)
+        q_route = _round(qr + 0.5 * noise, w.dtype)
+        q_layers = _round(rng.standard_normal(tuple(x["q_layers"].shape),
+                                              dtype=np.float32), w.dtype)
+        out.append((q_route, q_layers))
+    return out
