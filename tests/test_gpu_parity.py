@@ -372,3 +372,32 @@ def test_route_topk_recovers_from_dirty_workspace(dev):
         gidx = sd.route_topk(t["q_route"], t["K"], 100, ws=ws).cpu().numpy()
         assert_topk_within_band(gidx, S, 100)
     assert int(ws.buf[256:256 + 4 * 2048 * 4].sum()) == 0
+
+
+@pytest.mark.parametrize("k,count", [(4096, None), (8192, [3933, 4100, 100, 0, 8192, 2, 3000, 7000])])
+def test_attn_gather_many_keys_per_cta(dev, k, count):
+    """More selected keys than one on-chip chunk per CTA: the running max is
+    carried across chunks and the tensor-memory accumulator is rescaled."""
+    w = synth.custom(B=1, N=30000, Hq=32, Hkv=8, d=128, L=16, k=k, dtype="bf16", seed=k)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
+    idx = oracle.topk(S, k)
+    c = None if count is None else np.array([count], np.int32)
+    out, lse = sd.attn_gather(t["q_layers"], t["K"], t["V"], torch.from_numpy(idx).to(dev),
+                              count=None if c is None else torch.from_numpy(c).to(dev))
+    o_ref, l_ref = oracle.attn(_f(x["q_layers"]), _f(x["K"]), _f(x["V"]), idx, c)
+    assert_attn_close(out, lse, o_ref, l_ref, "bf16")
+
+
+def test_attn_gather_mma_sync_variant_matches(dev, monkeypatch):
+    """The warp-level mma.sync kernel (kept for comparison) agrees too."""
+    monkeypatch.setenv("SPARSE_DECODE_ATTN", "mma")
+    w = synth.custom(B=2, N=3000, Hq=32, Hkv=8, d=128, L=16, k=2048, dtype="bf16", seed=77)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
+    idx = oracle.topk(S, w.k)
+    out, lse = sd.attn_gather(t["q_layers"], t["K"], t["V"], torch.from_numpy(idx).to(dev))
+    o_ref, l_ref = oracle.attn(_f(x["q_layers"]), _f(x["K"]), _f(x["V"]), idx)
+    assert_attn_close(out, lse, o_ref, l_ref, "bf16")

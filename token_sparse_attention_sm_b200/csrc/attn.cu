@@ -12,6 +12,9 @@
 // online softmax (running max, rescaled sum) per query and writes a partial
 // (max, sum, unnormalised output).  A merge kernel combines the partials of
 // the splits by log-sum-exp rescaling and writes out and lse.
+#include <stdlib.h>
+#include <string.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -248,8 +251,14 @@ cudaError_t launch_attn(const Shape &s, int L, const void *q, const void *K,
                         const void *V, const int *idx, int stride,
                         const int *count, int count_cap, void *out, float *lse,
                         void *ws, uint32_t *status, cudaStream_t st) {
-  if (s.dtype == 1)
-    return launch_attn_mma(s, L, q, K, V, idx, stride, count, out, lse, status, st);
+  if (s.dtype == 1) {
+    // bf16: tcgen05 tensor cores by default; SPARSE_DECODE_ATTN=mma selects
+    // the warp-level mma.sync kernel instead (kept for comparison).
+    const char *impl = getenv("SPARSE_DECODE_ATTN");
+    if (impl && strcmp(impl, "mma") == 0)
+      return launch_attn_mma(s, L, q, K, V, idx, stride, count, out, lse, status, st);
+    return launch_attn_tc(s, L, q, K, V, idx, stride, count, out, lse, status, st);
+  }
   if (s.d == 128)
     return launch_attn_t<float, 128>(s, L, q, K, V, idx, stride, count, count_cap,
                                      out, lse, ws, status, st);

@@ -1,0 +1,556 @@
+// attn_tc.cu -- A3 + A4 for bf16 on the 5th-generation tensor cores
+// (tcgen05): gather attention with the accumulators in tensor memory and the
+// split-k merge in distributed shared memory.
+//
+// Every cross-decoder layer attends over the one shared index set (CLSA
+// article, section CLSAの仕組み), so for one (sequence, KV head) the M = L*G
+// query vectors of all layers and query heads form a dense block against the
+// same gathered keys: S = Q K^T and O = P V are real dense contractions.
+//
+// One thread-block cluster of C CTAs per (sequence, KV head, block of 128
+// query vectors); CTA r owns a contiguous share of the selected keys and
+// works through it in chunks of up to 256 keys:
+//  1. 16-byte async copies gather the chunk's K and V rows straight into
+//     128-byte-swizzled shared-memory tiles (the canonical K-major layout
+//     for K, the MN-major layout for V -- the same bytes, read two ways).
+//  2. One thread issues tcgen05.mma (kind::f16, bf16 in, fp32 accumulate,
+//     M=128 query rows, N=64 keys per tile) for S into tensor memory.
+//  3. Query row i lives in tensor-memory lane i; the two warps that share a
+//     lane quadrant split every 64-key tile in halves.  They read S with
+//     tcgen05.ld, take the exact row maximum of the chunk (joined through
+//     shared memory), and write P = exp2(S*scale*log2e - max) as two bf16
+//     parts (P = P_hi + P_lo, ~16 significant bits) into swizzled shared
+//     memory that reuses the K tiles.
+//  4. One thread issues O += P_hi V + P_lo V (M=128, N=d, K=64 per tile)
+//     into tensor memory, double-buffered against step 3.
+// A running max carried between chunks rescales O in tensor memory (only
+// when a CTA holds more than 256 keys).  Each CTA finally leaves its
+// partial (max, sum, O) in shared memory; after a cluster barrier every CTA
+// merges a slice of the rows by log-sum-exp rescaling through distributed
+// shared memory and writes out and lse.
+//
+// Every wait is bounded; on expiry the kernel raises the TIMEOUT flag, keeps
+// the cluster barriers in step, frees its tensor memory and returns.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace sd {
+namespace {
+
+constexpr int kTcThreads = 256;     // two warps per tensor-memory lane quadrant
+constexpr int kTcRows = 128;        // MMA M
+constexpr int kTileN = 64;          // keys per S tile (MMA N of QK^T, K of PV)
+constexpr int kChunkTiles = 4;      // tiles per chunk (S uses 256 TMEM columns)
+constexpr int kChunkKeys = kTileN * kChunkTiles;
+constexpr int kTmemCols = 512;
+constexpr int kTcMaxCluster = 16;
+
+template <int D>
+struct TcCfg {
+  static constexpr int kQBytes = kTcRows * D * 2;               // 32 KB at d=128
+  static constexpr int kKTile = kTileN * D * 2;                 // 16 KB
+  static constexpr int kPBuf = kTcRows * kTileN * 2;            // 16 KB (hi or lo)
+  static constexpr int kKPBytes =
+      (kChunkTiles * kKTile > 4 * kPBuf) ? kChunkTiles * kKTile : 4 * kPBuf;
+  static constexpr int kVBytes = kChunkTiles * kKTile;
+  static constexpr int kQOff = 0;
+  static constexpr int kKPOff = kQOff + kQBytes;
+  static constexpr int kVOff = kKPOff + kKPBytes;
+  static constexpr int kSmallOff = kVOff + kVBytes;
+  static constexpr int kSmallBytes = 4096;
+  static constexpr int kSmem = kSmallOff + kSmallBytes + 1024;  // + alignment slack
+  static_assert(kTcRows * D * 4 <= kKPBytes + kVBytes, "merge area fits");
+};
+
+// ---- tcgen05 helpers --------------------------------------------------------
+// Shared-memory matrix descriptor: 128-byte swizzle, version 1 (sm_100).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo,
+                                               uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+      ::"r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+               : "memory");
+}
+
+
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void *gmem, bool pred) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr),
+               "l"(gmem), "r"(pred ? 16u : 0u)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Byte offset of 16-byte chunk c (0..7) of row r inside a 128B-swizzled
+// block of 128-byte rows.
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+  return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_tc_kernel(const __nv_bfloat16 *__restrict__ q,
+                   const __nv_bfloat16 *__restrict__ K,
+                   const __nv_bfloat16 *__restrict__ V,
+                   const int *__restrict__ idx, int stride,
+                   const int *__restrict__ count, int N, int B, int Hq, int Hkv,
+                   int L, float scale_log2, __nv_bfloat16 *__restrict__ out,
+                   float *__restrict__ lse, uint32_t *status) {
+  using C = TcCfg<D>;
+  constexpr int KSTEPS = D / 16;  // MMA k-steps of S = Q K^T
+  constexpr int CPR = D / 8;      // 16-byte chunks per K/V row
+  cg::cluster_group cluster = cg::this_cluster();
+  const int csize = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int qb = blockIdx.y, bh = blockIdx.z;
+  const int b = bh / Hkv, h = bh % Hkv, G = Hq / Hkv;
+  const int M = L * G;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // Warps w and w+4 share tensor-memory lane quadrant w%4 (query rows
+  // 32*(w%4) .. +31); they split every 64-key tile into halves.
+  const int quad = warp & 3, hf = warp >> 2;
+  const int row = quad * 32 + lane;
+
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t base_s = (raw_s + 1023u) & ~1023u;  // swizzle atoms need 1 KB alignment
+  unsigned char *base = smem_raw + (base_s - raw_s);
+  const uint32_t q_s = base_s + C::kQOff;
+  const uint32_t kp_s = base_s + C::kKPOff;
+  const uint32_t v_s = base_s + C::kVOff;
+  unsigned char *small = base + C::kSmallOff;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(small);        // s, pv0, pv1, done
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(small + 64);
+  int *sidx = reinterpret_cast<int *>(small + 128);            // [256] chunk indices
+  unsigned char *kval = small + 128 + 4 * kChunkKeys;          // [256] valid flags
+  float *xred = reinterpret_cast<float *>(small + 128 + 5 * kChunkKeys);  // [2][128]
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_S = tmem;                          // columns [0, 256)
+  const uint32_t t_O = tmem + kChunkKeys;             // columns [256, 256 + D)
+  const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+
+  int cnt = stride;
+  if (count) cnt = min(max(count[bh], 0), stride);
+  const int per = (cnt + csize - 1) / csize;
+  const int k0 = min(cnt, rank * per), k1 = min(cnt, k0 + per);
+  const int *rowidx = idx + (size_t)bh * stride;
+  const size_t head_off = (size_t)bh * N * D;
+
+  // ---- Q block (rows beyond M are zero): thread = (row, half of the row) ----
+  {
+    const int r = tid & (kTcRows - 1), part = tid >> 7;
+    const int m = qb * kTcRows + r;
+    const __nv_bfloat16 *qr = nullptr;
+    if (m < M) qr = q + (((size_t)(m / G) * B + b) * Hq + (size_t)h * G + m % G) * D;
+#pragma unroll
+    for (int cc = 0; cc < CPR / 2; ++cc) {
+      const int c = part * (CPR / 2) + cc;
+      const uint32_t dst = q_s + (c >> 3) * (kTcRows * 128) + swz(r, c & 7);
+      cp_async16(dst, qr ? qr + c * 8 : q, qr != nullptr);
+    }
+    cp_async_commit();
+  }
+
+  bool failed = false;
+  float mrun = -INFINITY, lsum = 0.f;
+  uint32_t phase_s = 0, phase_done = 0, pv_uses[2] = {0u, 0u};
+  bool first_pv = true;
+  const uint32_t idS = idesc_bf16(kTcRows, kTileN, false);
+  const uint32_t idPV = idesc_bf16(kTcRows, D, true);
+
+  for (int c0 = k0; c0 < k1 && !failed; c0 += kChunkKeys) {
+    const int nk = min(kChunkKeys, k1 - c0);
+    const int ntile = (nk + kTileN - 1) / kTileN;
+    // indices of the chunk
+    sidx[tid] = tid < nk ? rowidx[c0 + tid] : -1;
+    __syncthreads();
+    // gather the chunk's K rows, then its V rows (two async-copy groups)
+    for (int p = tid; p < ntile * kTileN * CPR; p += kTcThreads) {
+      const int r = p / CPR, c = p % CPR;
+      const int j = sidx[r];
+      const bool ok = r < nk && j >= 0 && j < N;
+      if (r < nk && !ok && c == 0) raise_flag(status, FLAG_INDEX);
+      if (c == 0) kval[r] = ok;
+      const uint32_t dst = kp_s + (r >> 6) * C::kKTile + (c >> 3) * (kTileN * 128) +
+                           swz(r & 63, c & 7);
+      cp_async16(dst, K + head_off + (size_t)(ok ? j : 0) * D + c * 8, ok);
+    }
+    cp_async_commit();
+    for (int p = tid; p < ntile * kTileN * CPR; p += kTcThreads) {
+      const int r = p / CPR, c = p % CPR;
+      const int j = sidx[r];
+      const bool ok = r < nk && j >= 0 && j < N;
+      const uint32_t dst = v_s + (r >> 6) * C::kKTile + (c >> 3) * (kTileN * 128) +
+                           swz(r & 63, c & 7);
+      cp_async16(dst, V + head_off + (size_t)(ok ? j : 0) * D + c * 8, ok);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();      // Q and K have landed (this thread's copies)
+    fence_async_smem();      // make them visible to the tensor-core proxy
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- S = Q K^T for every tile of the chunk, one issuing thread ----------
+    if (tid == 0) {
+      for (int t = 0; t < ntile; ++t) {
+#pragma unroll
+        for (int s = 0; s < KSTEPS; ++s) {
+          const uint64_t a = sw128_desc(q_s + (s >> 2) * (kTcRows * 128) + (s & 3) * 32, 16, 1024);
+          const uint64_t bk = sw128_desc(kp_s + t * C::kKTile + (s >> 2) * (kTileN * 128) + (s & 3) * 32,
+                                         16, 1024);
+          mma_f16(t_S + t * kTileN, a, bk, idS, s > 0 ? 1u : 0u);
+        }
+      }
+      mma_commit(&bars[0]);
+    }
+    // validity of this warp's 32 keys of each tile, as bit masks (ballots over
+    // the flags written by the gather; identical in every warp)
+    uint32_t vmask[kChunkTiles];
+#pragma unroll
+    for (int t = 0; t < kChunkTiles; ++t) {
+      const int key = t * kTileN + hf * 32 + lane;
+      vmask[t] = __ballot_sync(0xffffffffu, key < nk && kval[key] != 0);
+    }
+    if (!mbar_wait(&bars[0], phase_s & 1u, status)) failed = true;
+    ++phase_s;
+    tc_fence_after();
+    if (__syncthreads_or(failed)) {
+      failed = true;
+      break;
+    }
+
+    // ---- row maximum over the chunk (two warps per row, joined in smem) -------
+    float cmax = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < kChunkTiles; ++t) {
+      if (t < ntile) {
+        uint32_t r[32];
+        tmem_ld32(t_S + lane_off + t * kTileN + hf * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if ((vmask[t] >> i) & 1u) cmax = fmaxf(cmax, __uint_as_float(r[i]));
+      }
+    }
+    xred[hf * kTcRows + row] = cmax;
+    __syncthreads();
+    cmax = fmaxf(xred[row], xred[kTcRows + row]) * scale_log2;  // scale > 0
+    const float mnew = fmaxf(mrun, cmax);
+    const float muse = mnew == -INFINITY ? 0.f : mnew;
+    const bool rescale = !first_pv && mnew != mrun;
+    if (__any_sync(0xffffffffu, rescale)) {
+      // a later chunk raised some row's max: rescale O (this warp's half of
+      // the columns); tcgen05.ld/st are warp-collective, so the whole warp
+      // takes this path
+      const float corr = rescale ? exp2f(mrun - muse) : 1.f;
+      lsum *= corr;
+#pragma unroll
+      for (int cb = 0; cb < D / 64; ++cb) {
+        uint32_t r[32];
+        const uint32_t col = t_O + lane_off + hf * (D / 2) + cb * 32;
+        tmem_ld32(col, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
+        tmem_st32(col, r);
+      }
+      tmem_wait_st();
+    }
+    mrun = mnew;
+
+    // ---- P tiles and O += P V ---------------------------------------------------
+    for (int t = 0; t < ntile; ++t) {
+      const int buf = t & 1;
+      if (pv_uses[buf] > 0) {  // PV of tile t-2 must be done with this buffer
+        if (!mbar_wait(&bars[1 + buf], (pv_uses[buf] - 1) & 1u, status)) failed = true;
+        tc_fence_after();
+      }
+      const uint32_t ph = kp_s + buf * 2 * C::kPBuf;  // hi, then lo
+      const uint32_t pl = ph + C::kPBuf;
+      uint32_t vm = 0;
+#pragma unroll
+      for (int u = 0; u < kChunkTiles; ++u)
+        if (u == t) vm = vmask[u];
+      uint32_t r[32];
+      tmem_ld32(t_S + lane_off + t * kTileN + hf * 32, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {  // four 16-byte chunks of 8 keys
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = c * 8 + e * 2;
+          const float p0 = ((vm >> i) & 1u) ? exp2f(fmaf(__uint_as_float(r[i]), scale_log2, -muse)) : 0.f;
+          const float p1 = ((vm >> (i + 1)) & 1u) ? exp2f(fmaf(__uint_as_float(r[i + 1]), scale_log2, -muse)) : 0.f;
+          lsum += p0 + p1;
+          hi[e] = pack_bf16x2(p0, p1);
+          const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162 *>(&hi[e]);
+          lo[e] = pack_bf16x2(p0 - __low2float(hb), p1 - __high2float(hb));
+        }
+        const uint32_t off = swz(row, hf * 4 + c);
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(ph + off), "r"(hi[0]),
+                     "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(pl + off), "r"(lo[0]),
+                     "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
+                     : "memory");
+      }
+      if (t == 0) cp_async_wait<0>();  // V tiles have landed (this thread's copies)
+      fence_async_smem();
+      tc_fence_before();
+      if (__syncthreads_or(failed)) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      if (tid == 0) {
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 16; ++kk) {
+          const uint64_t bv = sw128_desc(v_s + t * C::kKTile + kk * 2048, kTileN * 128, 1024);
+          mma_f16(t_O, sw128_desc(ph + kk * 32, 16, 1024), bv, idPV,
+                  (first_pv && kk == 0) ? 0u : 1u);
+          mma_f16(t_O, sw128_desc(pl + kk * 32, 16, 1024), bv, idPV, 1u);
+        }
+        mma_commit(&bars[1 + buf]);
+      }
+      first_pv = false;
+      ++pv_uses[buf];
+    }
+    // every MMA of this chunk done before its shared memory is reused
+    if (!failed) {
+      if (tid == 0) mma_commit(&bars[3]);
+      if (!mbar_wait(&bars[3], phase_done & 1u, status)) failed = true;
+      ++phase_done;
+      tc_fence_after();
+    }
+    if (__syncthreads_or(failed)) failed = true;
+  }
+  cp_async_wait<0>();
+
+  // ---- this CTA's partial -------------------------------------------------------
+  __syncthreads();
+  // Op: [D/4][128] float4 (chunk-major, so consecutive rows are consecutive
+  // 16-byte slots and the stores below are conflict-free)
+  float4 *Op = reinterpret_cast<float4 *>(base + C::kKPOff);
+  float *ML = reinterpret_cast<float *>(base + C::kVOff);  // [128][2]
+  {
+    const bool have = !first_pv && !failed;
+#pragma unroll
+    for (int cb = 0; cb < D / 64; ++cb) {
+      uint32_t r[32];
+      if (have) {
+        tmem_ld32(t_O + lane_off + hf * (D / 2) + cb * 32, r);
+        tmem_wait_ld();
+      }
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        const int chunk = (hf * (D / 2) + cb * 32 + i) >> 2;
+        Op[chunk * kTcRows + row] =
+            have ? make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                               __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    xred[hf * kTcRows + row] = have ? lsum : 0.f;
+    __syncthreads();
+    if (hf == 0) {
+      ML[row * 2] = have ? mrun : -INFINITY;
+      ML[row * 2 + 1] = xred[row] + xred[kTcRows + row];
+    }
+  }
+  tc_fence_before();
+  cluster.sync();
+
+  // ---- merge the cluster's partials ---------------------------------------------
+  constexpr int CH = D / 4;             // float4 chunks per row
+  constexpr int RPP = kTcThreads / CH;  // rows per pass
+  const int nmine = (kTcRows - rank + csize - 1) / csize;
+  for (int i = tid / CH; i < nmine; i += RPP) {
+    const int lr = rank + i * csize;
+    const int m = qb * kTcRows + lr;
+    if (m >= M) continue;
+    const int ch = tid % CH;
+    float mr[kTcMaxCluster], lr_[kTcMaxCluster];
+    float4 vr[kTcMaxCluster];
+#pragma unroll
+    for (int r = 0; r < kTcMaxCluster; ++r) {
+      if (r < csize) {
+        const float2 ml = *reinterpret_cast<const float2 *>(cluster.map_shared_rank(ML, r) + lr * 2);
+        mr[r] = ml.x;
+        lr_[r] = ml.y;
+        vr[r] = cluster.map_shared_rank(Op, r)[ch * kTcRows + lr];
+      } else {
+        mr[r] = -INFINITY;
+        lr_[r] = 0.f;
+        vr[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < kTcMaxCluster; ++r) mx = fmaxf(mx, mr[r]);
+    float ls = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (mx != -INFINITY) {
+#pragma unroll
+      for (int r = 0; r < kTcMaxCluster; ++r) {
+        const float w = mr[r] == -INFINITY ? 0.f : exp2f(mr[r] - mx);
+        ls += lr_[r] * w;
+        acc.x += w * vr[r].x;
+        acc.y += w * vr[r].y;
+        acc.z += w * vr[r].z;
+        acc.w += w * vr[r].w;
+      }
+    }
+    const float inv = ls > 0.f ? 1.f / ls : 0.f;
+    const size_t orow = ((size_t)(m / G) * B + b) * Hq + (size_t)h * G + m % G;
+    uint2 pk;
+    pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2 *>(out + orow * D + ch * 4) = pk;
+    if (lse && ch == 0)
+      lse[orow] = ls > 0.f ? (mx + log2f(ls)) * 0.69314718055994531f : -INFINITY;
+  }
+  cluster.sync();  // partials stay alive until every CTA has merged
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+}
+
+template <int D>
+cudaError_t launch_tc_t(const Shape &s, int L, const void *q, const void *K,
+                        const void *V, const int *idx, int stride, const int *count,
+                        void *out, float *lse, uint32_t *status, cudaStream_t st) {
+  using C = TcCfg<D>;
+  DeviceInfo di;
+  cudaError_t e = device_info(&di);
+  if (e != cudaSuccess) return e;
+  const int M = L * s.G();
+  const int qblocks = (M + kTcRows - 1) / kTcRows;
+  int csize = (stride + kChunkKeys - 1) / kChunkKeys;  // at least a chunk each
+  csize = csize < 2 ? 2 : csize;                       // keep the gather parallel
+  csize = csize > di.select_cluster ? di.select_cluster : csize;
+  csize = csize > kTcMaxCluster ? kTcMaxCluster : csize;
+  auto kern = attn_tc_kernel<D>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e == cudaSuccess && csize > 8)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)csize, (unsigned)qblocks, (unsigned)s.BH());
+  cfg.blockDim = dim3(kTcThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
+  e = cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16 *>(q),
+                         static_cast<const __nv_bfloat16 *>(K),
+                         static_cast<const __nv_bfloat16 *>(V), idx, stride, count, s.N,
+                         s.B, s.Hq, s.Hkv, L, scale_log2, static_cast<__nv_bfloat16 *>(out),
+                         lse, status);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_tc(const Shape &s, int L, const void *q, const void *K,
+                           const void *V, const int *idx, int stride,
+                           const int *count, void *out, float *lse,
+                           uint32_t *status, cudaStream_t st) {
+  if (s.d == 128)
+    return launch_tc_t<128>(s, L, q, K, V, idx, stride, count, out, lse, status, st);
+  return launch_tc_t<64>(s, L, q, K, V, idx, stride, count, out, lse, status, st);
+}
+
+}  // namespace sd

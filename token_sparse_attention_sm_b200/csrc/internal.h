@@ -46,6 +46,10 @@ cudaError_t launch_attn_mma(const Shape &s, int L, const void *q, const void *K,
                             const void *V, const int *idx, int stride,
                             const int *count, void *out, float *lse,
                             uint32_t *status, cudaStream_t st);
+cudaError_t launch_attn_tc(const Shape &s, int L, const void *q, const void *K,
+                           const void *V, const int *idx, int stride,
+                           const int *count, void *out, float *lse,
+                           uint32_t *status, cudaStream_t st);
 cudaError_t launch_attn(const Shape &s, int L, const void *q, const void *K,
                         const void *V, const int *idx, int stride,
                         const int *count, int count_cap, void *out, float *lse,

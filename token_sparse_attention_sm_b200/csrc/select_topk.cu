@@ -1,0 +1,325 @@
+// select_topk.cu -- A2 fast path: exact top-k of each (sequence, KV head)
+// when the score scan has already counted the top 11 key bits per head.
+//
+// Same contract as the general select kernel (select.cu): the k highest
+// scores, ties to the lower key index (CLSA article, section 研究の背景と課題),
+// written in ascending key order.
+//
+// One thread-block cluster per head; CTA r owns a contiguous slice of the
+// head's scores and each warp owns a contiguous segment of that slice, which
+// it walks one float4 (four keys) per lane at a time.
+//  1. Every CTA reads the head's global histogram and finds the boundary bin
+//     b1 where the descending count reaches k: keys above b1 are in, keys
+//     below are out, and only the keys inside b1 (a couple of thousand at the
+//     headline sizes) need the remaining 21 bits.
+//  2. One pass loads the slice, keeps it on chip as order-preserving keys,
+//     counts per warp the keys above b1, and appends the keys inside b1
+//     (with their slice index) to a shared-memory candidate list.
+//  3. Each CTA pushes its candidate keys into every CTA's shared memory
+//     (distributed shared-memory stores); after one cluster barrier every CTA
+//     finishes the selection on that small list locally (two more 11- and
+//     10-bit histogram levels).  Rank 0 clears the head's histogram for the
+//     next call.
+//  4. Per-warp counts (keys above b1 plus own candidates that pass) are
+//     pushed the same way; one more cluster barrier gives every warp its
+//     output offset, and a last pass writes the indices in ascending order.
+//     All exchanges are pushes, so no CTA reads another's shared memory
+//     after the last barrier and no trailing barrier is needed.
+// Falls back to the general multi-level cluster path when the histogram is
+// not complete (the counts do not sum to N), the candidates overflow the
+// on-chip lists, or the k-th score is shared by several keys (ties).
+#include "internal.h"
+#include "select_common.cuh"
+
+namespace sd {
+namespace {
+
+__global__ void __launch_bounds__(kSelThreads)
+    select_topk_fast_kernel(const float *__restrict__ S, int N, int k,
+                            int *__restrict__ idx, uint32_t *__restrict__ hist,
+                            uint32_t *status) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int csize = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int bh = blockIdx.x / csize;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SelShared *sh = reinterpret_cast<SelShared *>(smem_raw);
+  uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + kSelFixedSmem);
+  uint4 *keys4 = reinterpret_cast<uint4 *>(keys);
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int per_rank = kCandAll / csize;  // receive slots per source CTA
+
+  const int N4 = N >> 2;  // N % 4 == 0 on this path
+  const int lo4 = (int)((long long)N4 * rank / csize);
+  const int n4 = (int)((long long)N4 * (rank + 1) / csize) - lo4;
+  const int lo = lo4 * 4, n = n4 * 4;
+  const float4 *S4 = reinterpret_cast<const float4 *>(S + (size_t)bh * N) + lo4;
+  uint32_t *gh = hist + (size_t)bh * kBins;
+
+  // ---- 1. boundary bin from the scan's histogram ------------------------------
+  uint32_t c[kBinsPerThread], sum = 0;
+#pragma unroll
+  for (int e = 0; e < kBinsPerThread; ++e) {
+    c[e] = gh[kBins - 1 - (kBinsPerThread * tid + e)];
+    sum += c[e];
+  }
+  uint32_t tot;
+  uint32_t above = block_excl_scan(sum, sh->warp_buf, &tot);
+  const bool fast = tot == (uint32_t)N;  // block-uniform: a complete histogram
+  if (fast && above < (uint32_t)k && above + sum >= (uint32_t)k) {
+#pragma unroll
+    for (int e = 0; e < kBinsPerThread; ++e) {
+      if (above + c[e] >= (uint32_t)k) {
+        sh->bnd[0] = (uint32_t)(kBins - 1 - (kBinsPerThread * tid + e));
+        sh->bnd[1] = above;
+        sh->bnd[2] = c[e];
+        break;
+      }
+      above += c[e];
+    }
+  }
+  if (tid == 0) sh->ncand = 0;
+  if (tid < kSelWarps) sh->wpass[tid] = 0;
+  if (tid <= kSelWarps) sh->seg4[tid] = (int)((long long)n4 * tid / kSelWarps);
+  __syncthreads();
+  const uint32_t b1 = sh->bnd[0];
+  const uint32_t above1 = sh->bnd[1];
+
+  // ---- 2. load (a whole warp segment in flight), keep as keys, classify ------
+  const int sg0 = (int)((long long)n4 * wid / kSelWarps);
+  const int sg1 = (int)((long long)n4 * (wid + 1) / kSelWarps);
+  constexpr int U = 8;  // float4 per lane per batch
+  uint32_t wdef = 0;
+  bool bad = false;
+  for (int b4 = sg0; b4 < sg1; b4 += U * 32) {
+    float4 f[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i4 = b4 + u * 32 + lane;
+      f[u] = i4 < sg1 ? S4[i4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    uint32_t cand[U];  // 4 candidate bits per float4
+    uint32_t nc = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i4 = b4 + u * 32 + lane;
+      const bool in = i4 < sg1;
+      const uint4 kk = make_uint4(order_key(f[u].x), order_key(f[u].y),
+                                  order_key(f[u].z), order_key(f[u].w));
+      if (in) {
+        keys4[i4] = kk;
+        bad |= !isfinite(f[u].x) | !isfinite(f[u].y) | !isfinite(f[u].z) |
+               !isfinite(f[u].w);
+      }
+      const uint32_t kv[4] = {kk.x, kk.y, kk.z, kk.w};
+      uint32_t cm = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t top = kv[e] >> 21;
+        wdef += (in && top > b1) ? 1u : 0u;
+        cm |= (in && top == b1) ? (1u << e) : 0u;
+      }
+      cand[u] = cm;
+      nc += __popc(cm);
+    }
+    if (fast && __any_sync(0xffffffffu, nc != 0)) {
+      uint32_t inc = nc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      const uint32_t wtot = __shfl_sync(0xffffffffu, inc, 31);
+      uint32_t base = 0;
+      if (lane == 31) base = atomicAdd(&sh->ncand, wtot);
+      base = __shfl_sync(0xffffffffu, base, 31) + inc - nc;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (cand[u]) {
+          const int i4 = b4 + u * 32 + lane;
+          const uint4 kk = keys4[i4];
+          const uint32_t kv[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if ((cand[u] >> e) & 1u) {
+              if (base < (uint32_t)kCandLocal)
+                sh->cand_local[base] = make_uint2(kv[e], (uint32_t)(4 * i4 + e));
+              ++base;
+            }
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wdef += __shfl_xor_sync(0xffffffffu, wdef, o);
+  if (lane == 0) sh->wdef[wid] = wdef;
+  if (__syncthreads_or(bad) && tid == 0) raise_flag(status, FLAG_NONFINITE);
+  auto key_at = [&](int t) -> uint32_t { return keys[t]; };
+
+  // push this CTA's candidate count and keys into every CTA of the cluster
+  // (remote stores; the barrier below makes them visible)
+  const uint32_t my_cand = sh->ncand;
+  if (fast) {
+    if (tid < csize) cluster.map_shared_rank(sh->rcnt, tid)[rank] = my_cand;
+    const uint32_t npush = min(my_cand, (uint32_t)per_rank);
+    for (uint32_t i = tid; i < npush; i += kSelThreads) {
+      const uint32_t key = sh->cand_local[i].x;
+      for (int r = 0; r < csize; ++r)
+        cluster.map_shared_rank(sh->cand_all, r)[rank * per_rank + i] = key;
+    }
+  }
+  cluster.sync();  // candidates delivered; every CTA has read the histogram
+  if (rank == 0)
+    for (int b = tid; b < kBins; b += kSelThreads) gh[b] = 0u;
+
+  // ---- 3. refine the boundary bin on the candidate keys, locally ---------------
+  uint64_t t_ge = 0;
+  uint32_t tie_val = 0, n_ties = 0;
+  bool fast_ok = fast;
+  if (fast) {
+    uint32_t over = 0;
+    for (int r = 0; r < csize; ++r) over |= sh->rcnt[r] > (uint32_t)per_rank;
+    fast_ok = over == 0u;  // uniform: every CTA received the same counts
+    if (fast_ok) {
+      for (int b = tid; b < kBins; b += kSelThreads) sh->hist[1][b] = 0;
+      __syncthreads();
+      for (int r = 0; r < csize; ++r) {
+        const uint32_t nr = sh->rcnt[r];
+        for (uint32_t i = tid; i < nr; i += kSelThreads)
+          atomicAdd(&sh->hist[1][(sh->cand_all[r * per_rank + i] >> 10) & 2047u], 1u);
+      }
+      __syncthreads();
+      uint32_t need = (uint32_t)k - above1;
+      find_boundary_local(sh->hist[1], need, sh);
+      const uint32_t b2 = sh->bnd[0];
+      need -= sh->bnd[1];
+      const uint32_t p2 = (b1 << 11) | b2;
+      if (sh->bnd[2] == need) {
+        t_ge = (uint64_t)p2 << 10;
+      } else {
+        for (int b = tid; b < kBins; b += kSelThreads) sh->hist[0][b] = 0;
+        __syncthreads();
+        for (int r = 0; r < csize; ++r) {
+          const uint32_t nr = sh->rcnt[r];
+          for (uint32_t i = tid; i < nr; i += kSelThreads) {
+            const uint32_t key = sh->cand_all[r * per_rank + i];
+            if ((key >> 10) == p2) atomicAdd(&sh->hist[0][key & 1023u], 1u);
+          }
+        }
+        __syncthreads();
+        find_boundary_local(sh->hist[0], need, sh);
+        const uint32_t v = (p2 << 10) | sh->bnd[0];
+        need -= sh->bnd[1];
+        if (sh->bnd[2] == need) {
+          t_ge = v;
+        } else {
+          t_ge = (uint64_t)v + 1;
+          tie_val = v;
+          n_ties = need;
+        }
+      }
+    }
+  }
+
+  int *out = idx + (size_t)bh * k;
+  if (!fast_ok || n_ties) {
+    // general path (pulls from remote shared memory, so it ends with a
+    // cluster barrier that keeps every CTA's shared memory alive)
+    if (!fast_ok)
+      radix_general(cluster, sh, key_at, n, (uint32_t)k, csize, rank, nullptr, t_ge,
+                    tie_val, n_ties);
+    const uint32_t total_sel = compact_general(cluster, sh, key_at, n, lo, csize, rank,
+                                               t_ge, tie_val, n_ties, out, (uint32_t)k);
+    if (rank == 0 && tid == 0 && total_sel != (uint32_t)k) raise_flag(status, FLAG_INTERNAL);
+    cluster.sync();
+    return;
+  }
+
+  // ---- 4. per-warp counts, pushed offsets, ordered write --------------------
+  const uint32_t nloc = min(my_cand, (uint32_t)kCandLocal);
+  for (uint32_t i = tid; i < nloc; i += kSelThreads) {
+    const uint2 cd = sh->cand_local[i];
+    if ((uint64_t)cd.x >= t_ge) {
+      const int q4 = (int)(cd.y >> 2);
+      int w = 0;
+#pragma unroll
+      for (int s = 1; s < kSelWarps; ++s) w += q4 >= sh->seg4[s];
+      atomicAdd(&sh->wpass[w], 1u);
+    }
+  }
+  __syncthreads();
+  uint32_t before = 0, cta_sel = 0;
+#pragma unroll
+  for (int i = 0; i < kSelWarps; ++i) {
+    const uint32_t sel = sh->wdef[i] + sh->wpass[i];
+    before += i < wid ? sel : 0u;
+    cta_sel += sel;
+  }
+  if (tid < csize) cluster.map_shared_rank(sh->rge, tid)[rank] = cta_sel;
+  cluster.sync();  // last barrier: no remote access after it
+  uint32_t pos = before, total_sel = 0;
+  for (int r = 0; r < csize; ++r) {
+    pos += r < rank ? sh->rge[r] : 0u;
+    total_sel += sh->rge[r];
+  }
+  for (int b4 = sg0; b4 < sg1; b4 += 32) {
+    const int i4 = b4 + lane;
+    const bool in = i4 < sg1;
+    const uint4 kk = in ? keys4[i4] : make_uint4(0u, 0u, 0u, 0u);
+    const bool s0 = in && (uint64_t)kk.x >= t_ge, s1 = in && (uint64_t)kk.y >= t_ge;
+    const bool s2 = in && (uint64_t)kk.z >= t_ge, s3 = in && (uint64_t)kk.w >= t_ge;
+    const uint32_t q0 = __ballot_sync(0xffffffffu, s0), q1 = __ballot_sync(0xffffffffu, s1);
+    const uint32_t q2 = __ballot_sync(0xffffffffu, s2), q3 = __ballot_sync(0xffffffffu, s3);
+    const uint32_t wsel = __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
+    if (wsel == 0) continue;
+    uint32_t p = pos + __popc(q0 & lt_mask) + __popc(q1 & lt_mask) + __popc(q2 & lt_mask) +
+                 __popc(q3 & lt_mask);
+    const int j = lo + 4 * i4;
+    if (s0) { if (p < (uint32_t)k) out[p] = j; ++p; }
+    if (s1) { if (p < (uint32_t)k) out[p] = j + 1; ++p; }
+    if (s2) { if (p < (uint32_t)k) out[p] = j + 2; ++p; }
+    if (s3) { if (p < (uint32_t)k) out[p] = j + 3; ++p; }
+    pos += wsel;
+  }
+  if (rank == 0 && tid == 0 && total_sel != (uint32_t)k) raise_flag(status, FLAG_INTERNAL);
+}
+
+}  // namespace
+
+// Launch the fast top-k kernel if its preconditions hold; returns
+// cudaErrorNotSupported (nothing launched) otherwise.
+cudaError_t launch_select_topk_fast(const Shape &s, const float *S, int k, int *idx,
+                                    uint32_t *hist, uint32_t *status, cudaStream_t st) {
+  DeviceInfo di;
+  cudaError_t e = device_info(&di);
+  if (e != cudaSuccess) return e;
+  const int csize = di.select_cluster;
+  if (!hist || (s.N & 3) != 0) return cudaErrorNotSupported;
+  const size_t keys_bytes = (size_t)((s.N / 4 + csize - 1) / csize) * 16;
+  const size_t smem = kSelFixedSmem + keys_bytes;
+  if (smem > (size_t)di.max_smem_optin) return cudaErrorNotSupported;
+  auto kern = select_topk_fast_kernel;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess && csize > 8)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(s.BH() * csize), 1, 1);
+  cfg.blockDim = dim3(kSelThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, S, s.N, k, idx, hist, status);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace sd
