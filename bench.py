@@ -188,7 +188,7 @@ def capture(fn_list, stream):
 def traffic_record(kernel_file: str):
     """ncu DRAM bytes per launch of the dominant kernel, valid only while the
     kernel source is unchanged since the capture."""
-    path = os.path.join(ROOT, "profiles", "score_kernel_traffic.json")
+    path = os.path.join(ROOT, "profiles", "score_kernel_traffic.txt")
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -218,8 +218,7 @@ def run_native(args, rank, world, local_rank):
     ws = sd.Workspace(dev)
     # one workspace, sized up front for every op timed below, so that no
     # captured graph refers to a buffer that is later replaced
-    ws.get(max(sd.workspace_bytes(w.B, w.N, w.Hq, w.Hkv, w.d, w.torch_dtype, w.k, w.L),
-               sd.workspace_bytes(w.B, w.N, w.Hkv, w.Hkv, 64, torch.float32, w.k, 1)))
+    ws.get(sd.workspace_bytes(w.B, w.N, w.Hq, w.Hkv, w.d, w.torch_dtype, w.k, w.L))
     outs = [dict(out=torch.empty_like(ql), idx=torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device=dev),
                  lse=torch.empty((w.L, w.B, w.Hq), dtype=torch.float32, device=dev)) for _, ql in qs]
 
@@ -245,7 +244,7 @@ def run_native(args, rank, world, local_rank):
         idx0 = outs[0]["idx"]
         # size the workspace for every op before any capture
         sd.score(qs[0][0], K, ws=ws, check=False, out=S_buf)
-        sd.select_topk(S_buf, w.k, ws=ws, check=False, idx=idx0)
+        sd.route_topk(qs[0][0], K, w.k, ws=ws, check=False, idx=idx0)
         sd.attn_gather(qs[0][1], K, V, idx0, ws=ws, check=False, out=outs[0]["out"],
                        lse=outs[0]["lse"])
         torch.cuda.synchronize()
@@ -253,9 +252,11 @@ def run_native(args, rank, world, local_rank):
                                 for qr, _ in qs], stream)
         n_k = max(args.steps // 4, 64)
         t_score = time_graphs(score_graphs, n_k, max(args.warmup, 3), stream) / n_k
-        sel_graphs = capture([lambda: sd.select_topk(S_buf, w.k, ws=ws, check=False, idx=idx0)],
-                             stream)
-        t_sel = time_graphs(sel_graphs, n_k, max(args.warmup, 3), stream) / n_k
+        # the select kernel consumes the scan's histogram, so it is timed as
+        # route (scan + select) minus the scan alone
+        route_graphs = capture([lambda qr=qr: sd.route_topk(qr, K, w.k, ws=ws, check=False, idx=idx0)
+                                for qr, _ in qs], stream)
+        t_sel = time_graphs(route_graphs, n_k, max(args.warmup, 3), stream) / n_k - t_score
         attn_graphs = capture([lambda qi=qi: sd.attn_gather(qs[qi][1], K, V, outs[qi]["idx"], ws=ws,
                                                             check=False, out=outs[qi]["out"],
                                                             lse=outs[qi]["lse"])
@@ -314,8 +315,9 @@ def run_native(args, rank, world, local_rank):
         },
         "kernels_us": {"score": round(t_score * 1e3, 2), "select": round(t_sel * 1e3, 2),
                        "attn_gather_all_layers": round(t_attn * 1e3, 2),
-                       "note": "each kernel timed alone in back-to-back graph launches; "
-                               "attention alone may find its rows in L2"},
+                       "note": "score and attention timed alone in back-to-back graph "
+                               "launches (attention alone may find its rows in L2); select "
+                               "= route (score + select) minus score"},
         "e2e": e2e,
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,

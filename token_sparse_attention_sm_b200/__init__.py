@@ -243,14 +243,16 @@ def select_threshold(S, tau, cap: int, ws: Workspace | None = None,
     return idx, count
 
 
-def route_topk(q, K, k: int, ws: Workspace | None = None, check: bool = True):
+def route_topk(q, K, k: int, ws: Workspace | None = None, check: bool = True,
+               idx=None):
     """Shared routing (top-k): idx [B,Hkv,k] int32 ascending."""
-    _need_cuda(q, K)
+    _need_cuda(q, K, idx)
     B, N, Hq, Hkv, d = _dims_qk(q, K)
     w = _ws(ws, q.device)
     sh = _shape(B, N, Hq, Hkv, d, q.dtype)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, k, 1))
-    idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=q.device)
+    if idx is None:
+        idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=q.device)
     _check(load().sparse_route_topk(ctypes.byref(sh), _ptr(q), _ptr(K), int(k),
                                     _ptr(idx), _ptr(buf), buf.numel(), _stream()),
            "route_topk")
