@@ -178,6 +178,32 @@ sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
                                    float *lse, void *ws, size_t ws_bytes,
                                    void *stream);
 
+/* Shared routing, top-k form (as sparse_route_topk) for callers that cannot
+ * allocate device memory: a plugin inside a host framework that owns every
+ * device allocation, or code that must not call cudaMalloc once it is
+ * running (an allocation can synchronise the device and is not allowed while
+ * a stream is being captured).  It takes no workspace: its scratch (status
+ * word, radix histogram, fp32 scores) is a fixed array of about 4.5 MB built
+ * into the library, so every GPU that loads the library holds it until the
+ * process exits.  No page counterpart: this is a packaging variant, not part
+ * of the method the pages describe.
+ *   - Limit: B*Hkv <= 64 and B*Hkv*N <= 1048576 (the 128K-token, 8-head
+ *     headline fits exactly); larger shapes return SPARSE_ERR_WORKSPACE.
+ *   - The first call made with a given device current looks up the array's
+ *     device address (cudaGetSymbolAddress); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array; the call clears the parts that must
+ *     start at zero (status word, its histogram rows) on `stream` before
+ *     using them.  Calls that overlap on the GPU (different streams without
+ *     ordering) race on the array.
+ *   - Device-detected conditions are not reported (the status word lives in
+ *     the shared array); use sparse_route_topk with a workspace to read them.
+ *   - Calls no cudaMalloc, cudaFree or allocating library routine. */
+sparse_status_t sparse_route_topk_static(const sparse_shape_t *shape,
+                                         const void *q, const void *K,
+                                         int32_t k, int32_t *idx,
+                                         void *stream);
+
 /* Synchronise `stream`, read the device status word of ws, reset it to
  * zero, and return the most severe condition recorded since the last read
  * (TIMEOUT > INTERNAL > INDEX > NONFINITE > CAPACITY > OK).  *flags (if not NULL)

@@ -42,6 +42,7 @@ EXPORTED_SYMBOLS = (
     "sparse_workspace_init", "sparse_score", "sparse_select_topk",
     "sparse_select_threshold", "sparse_route_topk", "sparse_route_threshold",
     "sparse_attn_gather", "sparse_decode_step", "sparse_read_device_status",
+    "sparse_route_topk_static",
 )
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
@@ -95,6 +96,7 @@ def load():
             "sparse_decode_step": (I32, [SH, I32, P, P, P, P, I32, P, I32, P, P,
                                          P, P, P, SZ, P]),
             "sparse_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
+            "sparse_route_topk_static": (I32, [SH, P, P, I32, P, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
