@@ -367,11 +367,11 @@ def test_route_topk_recovers_from_dirty_workspace(dev):
     S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
     ws = sd.Workspace(dev)
     ws.get(sd.workspace_bytes(2, 5000, 8, 2, 128, torch.bfloat16, 100, 1))
-    ws.buf[256:256 + 4 * 2048 * 4] = 7
+    ws.buf[1024:1024 + 4 * 2048 * 4] = 7  # the histogram area (after the 1 KB header)
     for _ in range(2):
         gidx = sd.route_topk(t["q_route"], t["K"], 100, ws=ws).cpu().numpy()
         assert_topk_within_band(gidx, S, 100)
-    assert int(ws.buf[256:256 + 4 * 2048 * 4].sum()) == 0
+    assert int(ws.buf[1024:1024 + 4 * 2048 * 4].sum()) == 0
 
 
 @pytest.mark.parametrize("k,count", [(4096, None), (8192, [3933, 4100, 100, 0, 8192, 2, 3000, 7000])])

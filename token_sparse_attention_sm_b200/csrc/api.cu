@@ -4,8 +4,10 @@
 // before anything is enqueued; then it enqueues the kernels on the caller's
 // stream and returns.  The library allocates nothing: scratch lives in the
 // caller's workspace, whose layout is
-//   [0, 256)              header: device status word (uint32) at offset 0
-//   [256, ..)             radix histogram [B*Hkv][2048] uint32 (scan -> select;
+//   [0, 1024)             header: device status word (uint32) at offset 0;
+//                         [256, 1024) attention split-merge counters (a fixed,
+//                         shape-independent area, zero between calls)
+//   [1024, ..)            radix histogram [B*Hkv][2048] uint32 (scan -> select;
 //                         the select kernel clears it after use)
 //   [.., ..)              fp32 scores S [B,Hkv,N]
 //   [.., ..)              attention split partials (fp32 inputs only)
@@ -26,7 +28,8 @@ DeviceInfo g_info[kMaxDevices];
 cudaError_t g_info_err[kMaxDevices];
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-constexpr size_t kHeader = 256;
+constexpr size_t kHeader = 1024;
+constexpr size_t kCountersOff = 256;
 
 struct Layout {
   size_t hist_off, hist_bytes, scores_off, scores_bytes, attn_off, attn_bytes,
@@ -80,6 +83,11 @@ sparse_status_t from_cuda(cudaError_t e) {
 }
 
 uint32_t *status_word(void *ws) { return static_cast<uint32_t *>(ws); }
+uint32_t *attn_counters(void *ws) {
+  return reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + kCountersOff);
+}
+static_assert(kCountersOff + 2 * sizeof(uint32_t) * kAttnMaxCounterBlocks <= kHeader,
+              "counter area fits in the header");
 uint32_t *hist_ptr(void *ws, const Layout &l) {
   return reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + l.hist_off);
 }
@@ -266,7 +274,7 @@ sparse_status_t sparse_attn_gather(const sparse_shape_t *shape, int32_t L,
   const sd::Layout l = sd::layout(s, stride, L);
   return sd::from_cuda(sd::launch_attn(
       s, L, q, K, V, idx, stride, count, stride, out, lse, sd::attn_ptr(ws, l),
-      sd::status_word(ws), static_cast<cudaStream_t>(stream)));
+      sd::attn_counters(ws), sd::status_word(ws), static_cast<cudaStream_t>(stream)));
 }
 
 sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
@@ -306,7 +314,8 @@ sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
              : sd::launch_select(s, S, 0, tau, cap, idx, count, cap, nullptr, status, st);
   if (e == cudaSuccess)
     e = sd::launch_attn(s, L, q_layers, K, V, idx, stride, topk ? nullptr : count,
-                        stride, out, lse, sd::attn_ptr(ws, l), status, st);
+                        stride, out, lse, sd::attn_ptr(ws, l), sd::attn_counters(ws), status,
+                        st);
   return sd::from_cuda(e);
 }
 

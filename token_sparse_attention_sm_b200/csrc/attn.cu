@@ -240,7 +240,7 @@ cudaError_t launch_attn_t(const Shape &s, int L, const void *q, const void *K,
 }  // namespace
 
 size_t attn_workspace_bytes(const Shape &s, int L, int stride) {
-  if (s.dtype == 1) return 0;  // tensor-core path merges on chip
+  if (s.dtype == 1) return attn_tc_workspace_bytes(s, L);
   const int Mtot = L * s.G();
   const int qblocks = (Mtot + kQPerCta - 1) / kQPerCta;
   const int nsplit = num_splits(s.BH(), qblocks, stride);
@@ -250,14 +250,16 @@ size_t attn_workspace_bytes(const Shape &s, int L, int stride) {
 cudaError_t launch_attn(const Shape &s, int L, const void *q, const void *K,
                         const void *V, const int *idx, int stride,
                         const int *count, int count_cap, void *out, float *lse,
-                        void *ws, uint32_t *status, cudaStream_t st) {
+                        void *ws, uint32_t *counters, uint32_t *status,
+                        cudaStream_t st) {
   if (s.dtype == 1) {
     // bf16: tcgen05 tensor cores by default; SPARSE_DECODE_ATTN=mma selects
     // the warp-level mma.sync kernel instead (kept for comparison).
     const char *impl = getenv("SPARSE_DECODE_ATTN");
     if (impl && strcmp(impl, "mma") == 0)
       return launch_attn_mma(s, L, q, K, V, idx, stride, count, out, lse, status, st);
-    return launch_attn_tc(s, L, q, K, V, idx, stride, count, out, lse, status, st);
+    return launch_attn_tc(s, L, q, K, V, idx, stride, count, out, lse, ws, counters,
+                          status, st);
   }
   if (s.d == 128)
     return launch_attn_t<float, 128>(s, L, q, K, V, idx, stride, count, count_cap,

@@ -1,15 +1,15 @@
 // attn_tc.cu -- A3 + A4 for bf16 on the 5th-generation tensor cores
-// (tcgen05): gather attention with the accumulators in tensor memory and the
-// split-k merge in distributed shared memory.
+// (tcgen05): gather attention with the accumulators in tensor memory.
 //
 // Every cross-decoder layer attends over the one shared index set (CLSA
 // article, section CLSAの仕組み), so for one (sequence, KV head) the M = L*G
 // query vectors of all layers and query heads form a dense block against the
 // same gathered keys: S = Q K^T and O = P V are real dense contractions.
 //
-// One thread-block cluster of C CTAs per (sequence, KV head, block of 128
-// query vectors); CTA r owns a contiguous share of the selected keys and
-// works through it in chunks of up to 256 keys:
+// Grid: (key splits, blocks of 128 query vectors, sequence x KV head), one CTA
+// per SM (tile buffers and 512 tensor-memory columns).  CTA r owns a
+// contiguous share of the head's selected keys and works through it in
+// chunks of up to 256 keys:
 //  1. 16-byte async copies gather the chunk's K and V rows straight into
 //     128-byte-swizzled shared-memory tiles (the canonical K-major layout
 //     for K, the MN-major layout for V -- the same bytes, read two ways).
@@ -24,19 +24,17 @@
 //  4. One thread issues O += P_hi V + P_lo V (M=128, N=d, K=64 per tile)
 //     into tensor memory, double-buffered against step 3.
 // A running max carried between chunks rescales O in tensor memory (only
-// when a CTA holds more than 256 keys).  Each CTA finally leaves its
-// partial (max, sum, O) in shared memory; after a cluster barrier every CTA
-// merges a slice of the rows by log-sum-exp rescaling through distributed
-// shared memory and writes out and lse.
+// when a CTA holds more than 256 keys).  With one split the CTA normalises O
+// and writes out directly.  With several, each writes its partial (O, max,
+// sum) for the real query rows to the workspace, arrives on a per-head
+// counter and waits (bounded) for the other splits -- the launch is
+// cooperative, so all of them are resident -- then merges its share of the
+// rows by log-sum-exp rescaling; the last split to leave resets the counters.
 //
-// Every wait is bounded; on expiry the kernel raises the TIMEOUT flag, keeps
-// the cluster barriers in step, frees its tensor memory and returns.
-#include <cooperative_groups.h>
-
+// Every wait is bounded; on expiry the kernel raises the TIMEOUT flag, stops
+// issuing work, frees its tensor memory and returns.
 #include "common.cuh"
 #include "internal.h"
-
-namespace cg = cooperative_groups;
 
 namespace sd {
 namespace {
@@ -47,7 +45,7 @@ constexpr int kTileN = 64;          // keys per S tile (MMA N of QK^T, K of PV)
 constexpr int kChunkTiles = 4;      // tiles per chunk (S uses 256 TMEM columns)
 constexpr int kChunkKeys = kTileN * kChunkTiles;
 constexpr int kTmemCols = 512;
-constexpr int kTcMaxCluster = 16;
+constexpr int kTcMaxSplits = 16;
 
 template <int D>
 struct TcCfg {
@@ -163,13 +161,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    const int *__restrict__ idx, int stride,
                    const int *__restrict__ count, int N, int B, int Hq, int Hkv,
                    int L, float scale_log2, __nv_bfloat16 *__restrict__ out,
-                   float *__restrict__ lse, uint32_t *status) {
+                   float *__restrict__ lse, float *__restrict__ part,
+                   uint32_t *__restrict__ counters, uint32_t *status) {
   using C = TcCfg<D>;
   constexpr int KSTEPS = D / 16;  // MMA k-steps of S = Q K^T
   constexpr int CPR = D / 8;      // 16-byte chunks per K/V row
-  cg::cluster_group cluster = cg::this_cluster();
-  const int csize = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
+  const int csize = (int)gridDim.x;   // key splits of this head
+  const int rank = (int)blockIdx.x;
   const int qb = blockIdx.y, bh = blockIdx.z;
   const int b = bh / Hkv, h = bh % Hkv, G = Hq / Hkv;
   const int M = L * G;
@@ -411,13 +409,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   cp_async_wait<0>();
 
   // ---- this CTA's partial -------------------------------------------------------
+  const int mrows = min(kTcRows, M - qb * kTcRows);  // real query rows of the block
+  const bool have = !first_pv && !failed;
   __syncthreads();
-  // Op: [D/4][128] float4 (chunk-major, so consecutive rows are consecutive
-  // 16-byte slots and the stores below are conflict-free)
-  float4 *Op = reinterpret_cast<float4 *>(base + C::kKPOff);
-  float *ML = reinterpret_cast<float *>(base + C::kVOff);  // [128][2]
-  {
-    const bool have = !first_pv && !failed;
+  float *xsum = xred;  // [2][128]: the two warps' halves of each row's sum
+  xsum[hf * kTcRows + row] = have ? lsum : 0.f;
+  if (csize == 1) {
+    // one split: normalise straight from tensor memory
+    __syncthreads();
+    const float ls = xsum[row] + xsum[kTcRows + row];
+    const float inv = (have && ls > 0.f) ? 1.f / ls : 0.f;
+    const int m = qb * kTcRows + row;
+    const size_t orow = m < M ? ((size_t)(m / G) * B + b) * Hq + (size_t)h * G + m % G : 0;
 #pragma unroll
     for (int cb = 0; cb < D / 64; ++cb) {
       uint32_t r[32];
@@ -425,132 +428,206 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_ld32(t_O + lane_off + hf * (D / 2) + cb * 32, r);
         tmem_wait_ld();
       }
+      if (row < mrows) {
 #pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        const int chunk = (hf * (D / 2) + cb * 32 + i) >> 2;
-        Op[chunk * kTcRows + row] =
-            have ? make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                               __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]))
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < 32; i += 8) {
+          uint4 pk;
+          pk.x = pack_bf16x2(have ? __uint_as_float(r[i]) * inv : 0.f, have ? __uint_as_float(r[i + 1]) * inv : 0.f);
+          pk.y = pack_bf16x2(have ? __uint_as_float(r[i + 2]) * inv : 0.f, have ? __uint_as_float(r[i + 3]) * inv : 0.f);
+          pk.z = pack_bf16x2(have ? __uint_as_float(r[i + 4]) * inv : 0.f, have ? __uint_as_float(r[i + 5]) * inv : 0.f);
+          pk.w = pack_bf16x2(have ? __uint_as_float(r[i + 6]) * inv : 0.f, have ? __uint_as_float(r[i + 7]) * inv : 0.f);
+          *reinterpret_cast<uint4 *>(out + orow * D + hf * (D / 2) + cb * 32 + i) = pk;
+        }
       }
     }
-    xred[hf * kTcRows + row] = have ? lsum : 0.f;
+    if (lse && hf == 0 && row < mrows)
+      lse[orow] = (have && ls > 0.f) ? (mrun + log2f(ls)) * 0.69314718055994531f : -INFINITY;
+    tc_fence_before();
     __syncthreads();
-    if (hf == 0) {
-      ML[row * 2] = have ? mrun : -INFINITY;
-      ML[row * 2 + 1] = xred[row] + xred[kTcRows + row];
-    }
+    tc_fence_after();
+    if (warp == 0)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(kTmemCols)
+                   : "memory");
+    return;
   }
-  tc_fence_before();
-  cluster.sync();
 
-  // ---- merge the cluster's partials ---------------------------------------------
-  constexpr int CH = D / 4;             // float4 chunks per row
-  constexpr int RPP = kTcThreads / CH;  // rows per pass
-  const int nmine = (kTcRows - rank + csize - 1) / csize;
-  for (int i = tid / CH; i < nmine; i += RPP) {
-    const int lr = rank + i * csize;
-    const int m = qb * kTcRows + lr;
-    if (m >= M) continue;
-    const int ch = tid % CH;
-    float mr[kTcMaxCluster], lr_[kTcMaxCluster];
-    float4 vr[kTcMaxCluster];
+  // Several splits: write (O, max, sum) of the real rows to the partials,
+  // [head][qblock][split][row][D + 2] fp32, then merge a share of the rows.
+  float *mypart = part + (((size_t)bh * gridDim.y + qb) * csize + rank) * kTcRows * (D + 2);
 #pragma unroll
-    for (int r = 0; r < kTcMaxCluster; ++r) {
-      if (r < csize) {
-        const float2 ml = *reinterpret_cast<const float2 *>(cluster.map_shared_rank(ML, r) + lr * 2);
-        mr[r] = ml.x;
-        lr_[r] = ml.y;
-        vr[r] = cluster.map_shared_rank(Op, r)[ch * kTcRows + lr];
-      } else {
-        mr[r] = -INFINITY;
-        lr_[r] = 0.f;
-        vr[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+  for (int cb = 0; cb < D / 64; ++cb) {
+    uint32_t r[32];
+    if (have) {
+      tmem_ld32(t_O + lane_off + hf * (D / 2) + cb * 32, r);
+      tmem_wait_ld();
     }
-    float mx = -INFINITY;
+    if (row < mrows) {
+      float *dst = mypart + (size_t)row * (D + 2) + hf * (D / 2) + cb * 32;
 #pragma unroll
-    for (int r = 0; r < kTcMaxCluster; ++r) mx = fmaxf(mx, mr[r]);
-    float ls = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (mx != -INFINITY) {
-#pragma unroll
-      for (int r = 0; r < kTcMaxCluster; ++r) {
-        const float w = mr[r] == -INFINITY ? 0.f : exp2f(mr[r] - mx);
-        ls += lr_[r] * w;
-        acc.x += w * vr[r].x;
-        acc.y += w * vr[r].y;
-        acc.z += w * vr[r].z;
-        acc.w += w * vr[r].w;
-      }
+      for (int i = 0; i < 32; i += 2)
+        *reinterpret_cast<float2 *>(dst + i) =
+            have ? make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]))
+                 : make_float2(0.f, 0.f);
     }
-    const float inv = ls > 0.f ? 1.f / ls : 0.f;
-    const size_t orow = ((size_t)(m / G) * B + b) * Hq + (size_t)h * G + m % G;
-    uint2 pk;
-    pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2 *>(out + orow * D + ch * 4) = pk;
-    if (lse && ch == 0)
-      lse[orow] = ls > 0.f ? (mx + log2f(ls)) * 0.69314718055994531f : -INFINITY;
   }
-  cluster.sync();  // partials stay alive until every CTA has merged
+  __syncthreads();
+  if (hf == 0 && row < mrows) {
+    float *dst = mypart + (size_t)row * (D + 2) + D;
+    *reinterpret_cast<float2 *>(dst) =
+        make_float2(have ? mrun : -INFINITY, xsum[row] + xsum[kTcRows + row]);
+  }
+  // tensor memory is no longer needed
+  tc_fence_before();
+  __syncthreads();
   tc_fence_after();
   if (warp == 0)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)
                  : "memory");
+  // arrive, then wait (bounded) until every split of this head block arrived;
+  // the launch is cooperative, so all of them are resident
+  uint32_t *arrive = counters + 2 * ((size_t)bh * gridDim.y + qb);
+  uint32_t *depart = arrive + 1;
+  __shared__ int ready;
+  if (tid == 0) {
+    __threadfence();
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(arrive) : "memory");
+    bool ok = true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+      uint32_t v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(arrive) : "memory");
+      if (v >= (uint32_t)csize) break;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        raise_flag(status, FLAG_TIMEOUT);
+        ok = false;
+        break;
+      }
+      __nanosleep(64);
+    }
+    ready = ok;
+  }
+  __syncthreads();
+  if (ready) {
+    // merge rows lr = rank, rank + csize, ...: thread = (row slot, float4 chunk)
+    constexpr int CH = D / 4;
+    constexpr int RPP = kTcThreads / CH;  // rows per pass
+    const float *hp = part + ((size_t)bh * gridDim.y + qb) * csize * kTcRows * (D + 2);
+    const int nmine = (mrows - rank + csize - 1) / csize;
+    for (int i = tid / CH; i < nmine; i += RPP) {
+      const int lr = rank + i * csize;
+      const int ch = tid % CH;
+      float mx = -INFINITY;
+      for (int r = 0; r < csize; ++r)
+        mx = fmaxf(mx, hp[((size_t)r * kTcRows + lr) * (D + 2) + D]);
+      float ls = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (mx != -INFINITY) {
+#pragma unroll 4
+        for (int r = 0; r < csize; ++r) {
+          const float *pr = hp + ((size_t)r * kTcRows + lr) * (D + 2);
+          const float2 ml = *reinterpret_cast<const float2 *>(pr + D);
+          const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - mx);
+          ls += ml.y * w;
+          const float2 v0 = *reinterpret_cast<const float2 *>(pr + ch * 4);
+          const float2 v1 = *reinterpret_cast<const float2 *>(pr + ch * 4 + 2);
+          acc.x += w * v0.x;
+          acc.y += w * v0.y;
+          acc.z += w * v1.x;
+          acc.w += w * v1.y;
+        }
+      }
+      const float inv = ls > 0.f ? 1.f / ls : 0.f;
+      const int m = qb * kTcRows + lr;
+      const size_t orow = ((size_t)(m / G) * B + b) * Hq + (size_t)h * G + m % G;
+      uint2 pk;
+      pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+      pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2 *>(out + orow * D + ch * 4) = pk;
+      if (lse && ch == 0)
+        lse[orow] = ls > 0.f ? (mx + log2f(ls)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+  // the last split to leave resets both counters for the next call
+  __syncthreads();
+  if (tid == 0) {
+    const uint32_t old = atomicAdd(depart, 1u);
+    if (old == (uint32_t)csize - 1) {
+      *arrive = 0u;
+      *depart = 0u;
+      __threadfence();
+    }
+  }
+}
+
+template <int D>
+size_t tc_part_bytes(const Shape &s, int L) {
+  const int M = L * s.G();
+  const int qblocks = (M + kTcRows - 1) / kTcRows;
+  return (size_t)s.BH() * qblocks * kTcMaxSplits * kTcRows * (D + 2) * sizeof(float);
 }
 
 template <int D>
 cudaError_t launch_tc_t(const Shape &s, int L, const void *q, const void *K,
                         const void *V, const int *idx, int stride, const int *count,
-                        void *out, float *lse, uint32_t *status, cudaStream_t st) {
+                        void *out, float *lse, void *ws, uint32_t *counters,
+                        uint32_t *status, cudaStream_t st) {
   using C = TcCfg<D>;
   DeviceInfo di;
   cudaError_t e = device_info(&di);
   if (e != cudaSuccess) return e;
   const int M = L * s.G();
   const int qblocks = (M + kTcRows - 1) / kTcRows;
-  int csize = (stride + kChunkKeys - 1) / kChunkKeys;  // at least a chunk each
-  csize = csize < 2 ? 2 : csize;                       // keep the gather parallel
-  csize = csize > di.select_cluster ? di.select_cluster : csize;
-  csize = csize > kTcMaxCluster ? kTcMaxCluster : csize;
+  // key splits per head block: enough CTAs to cover the SMs (one CTA per SM:
+  // the tile buffers and 512 tensor-memory columns), every split at least one
+  // 64-key tile, all CTAs resident at once when there is more than one split
+  const long long blocks = (long long)s.BH() * qblocks;
+  int nsplit = (int)(di.sm_count / blocks);
+  const int by_keys = (stride + kTileN - 1) / kTileN;
+  nsplit = nsplit > by_keys ? by_keys : nsplit;
+  nsplit = nsplit > kTcMaxSplits ? kTcMaxSplits : nsplit;
+  nsplit = nsplit < 1 ? 1 : nsplit;
+  if (blocks > kAttnMaxCounterBlocks) nsplit = 1;  // counters live in a fixed area
   auto kern = attn_tc_kernel<D>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-  if (e == cudaSuccess && csize > 8)
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
+  float *part = static_cast<float *>(ws);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)csize, (unsigned)qblocks, (unsigned)s.BH());
+  cfg.gridDim = dim3((unsigned)nsplit, (unsigned)qblocks, (unsigned)s.BH());
   cfg.blockDim = dim3(kTcThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)csize;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = nsplit > 1 ? 1 : 0;
   const float scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16 *>(q),
                          static_cast<const __nv_bfloat16 *>(K),
                          static_cast<const __nv_bfloat16 *>(V), idx, stride, count, s.N,
                          s.B, s.Hq, s.Hkv, L, scale_log2, static_cast<__nv_bfloat16 *>(out),
-                         lse, status);
+                         lse, part, counters, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 }  // namespace
 
+size_t attn_tc_workspace_bytes(const Shape &s, int L) {
+  return s.d == 128 ? tc_part_bytes<128>(s, L) : tc_part_bytes<64>(s, L);
+}
+
 cudaError_t launch_attn_tc(const Shape &s, int L, const void *q, const void *K,
                            const void *V, const int *idx, int stride,
-                           const int *count, void *out, float *lse,
-                           uint32_t *status, cudaStream_t st) {
+                           const int *count, void *out, float *lse, void *ws,
+                           uint32_t *counters, uint32_t *status, cudaStream_t st) {
   if (s.d == 128)
-    return launch_tc_t<128>(s, L, q, K, V, idx, stride, count, out, lse, status, st);
-  return launch_tc_t<64>(s, L, q, K, V, idx, stride, count, out, lse, status, st);
+    return launch_tc_t<128>(s, L, q, K, V, idx, stride, count, out, lse, ws, counters,
+                            status, st);
+  return launch_tc_t<64>(s, L, q, K, V, idx, stride, count, out, lse, ws, counters, status,
+                         st);
 }
 
 }  // namespace sd

@@ -38,21 +38,28 @@ cudaError_t launch_select(const Shape &s, const float *S, int k,
                           int stride, uint32_t *hist, uint32_t *status,
                           cudaStream_t st);
 
-// A3 + A4: L query sets over the same index rows.  bf16 runs on the tensor
-// cores with the split merge in distributed shared memory (no workspace);
-// fp32 runs on the CUDA cores with split partials in the workspace.
+// A3 + A4: L query sets over the same index rows.  bf16 runs on the tcgen05
+// tensor cores (split partials in the workspace) or, on request, the mma.sync
+// kernel (split merge in distributed shared memory); fp32 runs on the CUDA
+// cores with split partials in the workspace.
 size_t attn_workspace_bytes(const Shape &s, int L, int stride);
 cudaError_t launch_attn_mma(const Shape &s, int L, const void *q, const void *K,
                             const void *V, const int *idx, int stride,
                             const int *count, void *out, float *lse,
                             uint32_t *status, cudaStream_t st);
+size_t attn_tc_workspace_bytes(const Shape &s, int L);
+// Split-merge counters of the tcgen05 attention: two per (head, query block)
+// in a fixed, shape-independent area of the workspace header (zero between
+// calls: the kernel resets them).  More blocks than this run unsplit.
+constexpr int kAttnMaxCounterBlocks = 96;
 cudaError_t launch_attn_tc(const Shape &s, int L, const void *q, const void *K,
                            const void *V, const int *idx, int stride,
-                           const int *count, void *out, float *lse,
-                           uint32_t *status, cudaStream_t st);
+                           const int *count, void *out, float *lse, void *ws,
+                           uint32_t *counters, uint32_t *status, cudaStream_t st);
 cudaError_t launch_attn(const Shape &s, int L, const void *q, const void *K,
                         const void *V, const int *idx, int stride,
                         const int *count, int count_cap, void *out, float *lse,
-                        void *ws, uint32_t *status, cudaStream_t st);
+                        void *ws, uint32_t *counters, uint32_t *status,
+                        cudaStream_t st);
 
 }  // namespace sd
