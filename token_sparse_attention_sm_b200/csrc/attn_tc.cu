@@ -61,7 +61,7 @@ struct TcCfg {
   static constexpr int kSmallOff = kVOff + kVBytes;
   static constexpr int kSmallBytes = 4096;
   static constexpr int kSmem = kSmallOff + kSmallBytes + 1024;  // + alignment slack
-  static_assert(kTcRows * D * 4 <= kKPBytes + kVBytes, "merge area fits");
+  static_assert(kTcRows * (D + 4) * 4 <= kKPBytes + kVBytes, "staging area fits");
 };
 
 // ---- tcgen05 helpers --------------------------------------------------------
@@ -453,8 +453,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 
   // Several splits: write (O, max, sum) of the real rows to the partials,
-  // [head][qblock][split][row][D + 2] fp32, then merge a share of the rows.
-  float *mypart = part + (((size_t)bh * gridDim.y + qb) * csize + rank) * kTcRows * (D + 2);
+  // [head][qblock][split][row][D + 4] fp32 (O, max, sum, pad), staged through
+  // shared memory (the tile buffers are free now) so the global stores are
+  // coalesced.
+  constexpr int PR = D + 4;  // partial row stride in floats (16-byte aligned)
+  float *stage = reinterpret_cast<float *>(base + C::kKPOff);  // [128][PR]
+  float *mypart = part + (((size_t)bh * gridDim.y + qb) * csize + rank) * kTcRows * PR;
 #pragma unroll
   for (int cb = 0; cb < D / 64; ++cb) {
     uint32_t r[32];
@@ -463,19 +467,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tmem_wait_ld();
     }
     if (row < mrows) {
-      float *dst = mypart + (size_t)row * (D + 2) + hf * (D / 2) + cb * 32;
+      float *dst = stage + row * PR + hf * (D / 2) + cb * 32;
 #pragma unroll
-      for (int i = 0; i < 32; i += 2)
-        *reinterpret_cast<float2 *>(dst + i) =
-            have ? make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]))
-                 : make_float2(0.f, 0.f);
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4 *>(dst + i) =
+            have ? make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                               __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
   __syncthreads();
-  if (hf == 0 && row < mrows) {
-    float *dst = mypart + (size_t)row * (D + 2) + D;
-    *reinterpret_cast<float2 *>(dst) =
-        make_float2(have ? mrun : -INFINITY, xsum[row] + xsum[kTcRows + row]);
+  if (hf == 0 && row < mrows)
+    *reinterpret_cast<float4 *>(stage + row * PR + D) =
+        make_float4(have ? mrun : -INFINITY, xsum[row] + xsum[kTcRows + row], 0.f, 0.f);
+  __syncthreads();
+  {
+    const int n4 = mrows * PR / 4;
+    const float4 *src = reinterpret_cast<const float4 *>(stage);
+    float4 *dst = reinterpret_cast<float4 *>(mypart);
+    for (int i = tid; i < n4; i += kTcThreads) dst[i] = src[i];
   }
   // tensor memory is no longer needed
   tc_fence_before();
@@ -510,32 +520,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   __syncthreads();
   if (ready) {
-    // merge rows lr = rank, rank + csize, ...: thread = (row slot, float4 chunk)
+    // merge rows lr = rank, rank + csize, ...: thread = (row slot, float4
+    // chunk); every split's values are loaded before any is used
     constexpr int CH = D / 4;
     constexpr int RPP = kTcThreads / CH;  // rows per pass
-    const float *hp = part + ((size_t)bh * gridDim.y + qb) * csize * kTcRows * (D + 2);
+    const float *hp = part + ((size_t)bh * gridDim.y + qb) * csize * kTcRows * PR;
     const int nmine = (mrows - rank + csize - 1) / csize;
     for (int i = tid / CH; i < nmine; i += RPP) {
       const int lr = rank + i * csize;
       const int ch = tid % CH;
+      float2 ml[kTcMaxSplits];
+      float4 v[kTcMaxSplits];
+#pragma unroll
+      for (int r = 0; r < kTcMaxSplits; ++r) {
+        if (r < csize) {
+          const float *pr = hp + ((size_t)r * kTcRows + lr) * PR;
+          ml[r] = *reinterpret_cast<const float2 *>(pr + D);
+          v[r] = *reinterpret_cast<const float4 *>(pr + ch * 4);
+        } else {
+          ml[r] = make_float2(-INFINITY, 0.f);
+          v[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
       float mx = -INFINITY;
-      for (int r = 0; r < csize; ++r)
-        mx = fmaxf(mx, hp[((size_t)r * kTcRows + lr) * (D + 2) + D]);
+#pragma unroll
+      for (int r = 0; r < kTcMaxSplits; ++r) mx = fmaxf(mx, ml[r].x);
       float ls = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       if (mx != -INFINITY) {
-#pragma unroll 4
-        for (int r = 0; r < csize; ++r) {
-          const float *pr = hp + ((size_t)r * kTcRows + lr) * (D + 2);
-          const float2 ml = *reinterpret_cast<const float2 *>(pr + D);
-          const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - mx);
-          ls += ml.y * w;
-          const float2 v0 = *reinterpret_cast<const float2 *>(pr + ch * 4);
-          const float2 v1 = *reinterpret_cast<const float2 *>(pr + ch * 4 + 2);
-          acc.x += w * v0.x;
-          acc.y += w * v0.y;
-          acc.z += w * v1.x;
-          acc.w += w * v1.y;
+#pragma unroll
+        for (int r = 0; r < kTcMaxSplits; ++r) {
+          const float w = ml[r].x == -INFINITY ? 0.f : exp2f(ml[r].x - mx);
+          ls += ml[r].y * w;
+          acc.x += w * v[r].x;
+          acc.y += w * v[r].y;
+          acc.z += w * v[r].z;
+          acc.w += w * v[r].w;
         }
       }
       const float inv = ls > 0.f ? 1.f / ls : 0.f;
@@ -565,7 +585,7 @@ template <int D>
 size_t tc_part_bytes(const Shape &s, int L) {
   const int M = L * s.G();
   const int qblocks = (M + kTcRows - 1) / kTcRows;
-  return (size_t)s.BH() * qblocks * kTcMaxSplits * kTcRows * (D + 2) * sizeof(float);
+  return (size_t)s.BH() * qblocks * kTcMaxSplits * kTcRows * (D + 4) * sizeof(float);
 }
 
 template <int D>
