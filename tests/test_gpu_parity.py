@@ -401,3 +401,25 @@ def test_attn_gather_mma_sync_variant_matches(dev, monkeypatch):
     out, lse = sd.attn_gather(t["q_layers"], t["K"], t["V"], torch.from_numpy(idx).to(dev))
     o_ref, l_ref = oracle.attn(_f(x["q_layers"]), _f(x["K"]), _f(x["V"]), idx)
     assert_attn_close(out, lse, o_ref, l_ref, "bf16")
+
+
+@pytest.mark.parametrize("kind", ["random", "duplicated_rows", "few_values", "heavy"])
+def test_route_topk_bit_exact_on_its_own_scores(dev, kind):
+    """Routing (scan + histogram fast-path select) against the oracle's top-k
+    of the very scores the scan produced: identical fp32 scores, so the index
+    sets must be identical, ties included."""
+    w = synth.custom(B=2, N=40000, Hq=32, Hkv=8, d=128, L=1, k=2048, dtype="bf16",
+                     heavy=64 if kind == "heavy" else 0, seed=17)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    K = t["K"]
+    if kind == "duplicated_rows":       # groups of 3 identical rows: exact score ties
+        K = K.clone()
+        K[:, :, 1::3] = K[:, :, 0:-1:3][:, :, :K[:, :, 1::3].shape[2]]
+        K[:, :, 2::3] = K[:, :, 0:-2:3][:, :, :K[:, :, 2::3].shape[2]]
+    elif kind == "few_values":          # small integers: many exact ties
+        K = torch.randint(-2, 3, K.shape, device=dev).to(K.dtype)
+    ws = sd.Workspace(dev)
+    S = sd.score(t["q_route"], K, ws=ws).cpu().numpy()
+    idx = sd.route_topk(t["q_route"], K, w.k, ws=ws).cpu().numpy()
+    np.testing.assert_array_equal(idx, oracle.topk(S, w.k))

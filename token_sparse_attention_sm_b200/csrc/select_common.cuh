@@ -17,6 +17,7 @@ constexpr int kBinsPerThread = kBins / kSelThreads;
 constexpr int kCandLocal = 2048;  // boundary-bin keys one CTA may hold
 constexpr int kCandAll = 8192;    // boundary-bin keys of a whole head
 constexpr int kMaxCluster = 16;
+constexpr int kFinMax = 64;       // keys ranked pairwise after two levels
 constexpr int kSelFixedSmem = 2 * kBins * 4 + kCandLocal * 8 + kCandAll * 4 + 1024;
 
 struct SelShared {
@@ -36,6 +37,8 @@ struct SelShared {
   uint32_t wdef[kSelWarps];    // fast path: keys above the boundary bin, per warp
   uint32_t wpass[kSelWarps];   // fast path: boundary-bin keys that pass, per warp
   int seg4[kSelWarps + 1];     // fast path: warp segment bounds in float4 units
+  uint32_t nfin;               // fast path: keys left after two levels
+  uint32_t fin[kFinMax];
 };
 static_assert(sizeof(SelShared) <= kSelFixedSmem, "fixed select smem");
 

@@ -17,8 +17,10 @@
 //     (with their slice index) to a shared-memory candidate list.
 //  3. Each CTA pushes its candidate keys into every CTA's shared memory
 //     (distributed shared-memory stores); after one cluster barrier every CTA
-//     finishes the selection on that small list locally (two more 11- and
-//     10-bit histogram levels).  Rank 0 clears the head's histogram for the
+//     finishes the selection on that small list locally: one more 11-bit
+//     histogram level, then the few keys left in its boundary bin are ranked
+//     exactly by pairwise counts within one warp (a 10-bit histogram level
+//     only if more than 64 remain).  Rank 0 clears the head's histogram for the
 //     next call.
 //  4. Per-warp counts (keys above b1 plus own candidates that pass) are
 //     pushed the same way; one more cluster barrier gives every warp its
@@ -196,8 +198,64 @@ __global__ void __launch_bounds__(kSelThreads)
       const uint32_t b2 = sh->bnd[0];
       need -= sh->bnd[1];
       const uint32_t p2 = (b1 << 11) | b2;
-      if (sh->bnd[2] == need) {
+      const uint32_t cnt2 = sh->bnd[2];
+      if (cnt2 == need) {
         t_ge = (uint64_t)p2 << 10;
+      } else if (cnt2 <= (uint32_t)kFinMax) {
+        // few keys left in the level-2 boundary bin: rank them exactly within
+        // one warp (pairwise counts) instead of another histogram level
+        if (tid == 0) sh->nfin = 0;
+        __syncthreads();
+        for (int r = 0; r < csize; ++r) {
+          const uint32_t nr = sh->rcnt[r];
+          for (uint32_t i = tid; i < nr; i += kSelThreads) {
+            const uint32_t key = sh->cand_all[r * per_rank + i];
+            if ((key >> 10) == p2) sh->fin[atomicAdd(&sh->nfin, 1u)] = key;
+          }
+        }
+        __syncthreads();
+        if (wid == 0) {
+          const uint32_t nf = sh->nfin;  // == cnt2
+          uint32_t best_v = 0, best_gt = 0, best_eq = 0;
+          bool found = false;
+          for (uint32_t a = lane; a < nf; a += 32) {
+            const uint32_t v = sh->fin[a];
+            uint32_t gt = 0, eq = 0;
+            for (uint32_t c2 = 0; c2 < nf; ++c2) {
+              const uint32_t u = sh->fin[c2];
+              gt += u > v;
+              eq += u == v;
+            }
+            if (gt < need && need <= gt + eq) {
+              found = true;
+              best_v = v;
+              best_gt = gt;
+              best_eq = eq;
+            }
+          }
+          // every lane that found it holds the same value; take the lowest
+          const uint32_t m = __ballot_sync(0xffffffffu, found);
+          const int src = m ? __ffs(m) - 1 : 0;
+          best_v = __shfl_sync(0xffffffffu, best_v, src);
+          best_gt = __shfl_sync(0xffffffffu, best_gt, src);
+          best_eq = __shfl_sync(0xffffffffu, best_eq, src);
+          if (lane == 0) {
+            sh->bnd[0] = best_v;
+            sh->bnd[1] = best_gt;
+            sh->bnd[2] = best_eq;
+            if (!m) raise_flag(status, FLAG_INTERNAL);
+          }
+        }
+        __syncthreads();
+        const uint32_t v = sh->bnd[0];
+        const uint32_t rest = need - sh->bnd[1];  // keys equal to v still needed
+        if (sh->bnd[2] == rest) {
+          t_ge = v;
+        } else {
+          t_ge = (uint64_t)v + 1;
+          tie_val = v;
+          n_ties = rest;
+        }
       } else {
         for (int b = tid; b < kBins; b += kSelThreads) sh->hist[0][b] = 0;
         __syncthreads();
@@ -264,12 +322,15 @@ __global__ void __launch_bounds__(kSelThreads)
     pos += r < rank ? sh->rge[r] : 0u;
     total_sel += sh->rge[r];
   }
+  // t_ge <= 2^32 here; keep the compares 32-bit
+  const bool none = t_ge > 0xFFFFFFFFull;
+  const uint32_t t32 = (uint32_t)t_ge;
   for (int b4 = sg0; b4 < sg1; b4 += 32) {
     const int i4 = b4 + lane;
-    const bool in = i4 < sg1;
+    const bool in = i4 < sg1 && !none;
     const uint4 kk = in ? keys4[i4] : make_uint4(0u, 0u, 0u, 0u);
-    const bool s0 = in && (uint64_t)kk.x >= t_ge, s1 = in && (uint64_t)kk.y >= t_ge;
-    const bool s2 = in && (uint64_t)kk.z >= t_ge, s3 = in && (uint64_t)kk.w >= t_ge;
+    const bool s0 = in && kk.x >= t32, s1 = in && kk.y >= t32;
+    const bool s2 = in && kk.z >= t32, s3 = in && kk.w >= t32;
     const uint32_t q0 = __ballot_sync(0xffffffffu, s0), q1 = __ballot_sync(0xffffffffu, s1);
     const uint32_t q2 = __ballot_sync(0xffffffffu, s2), q3 = __ballot_sync(0xffffffffu, s3);
     const uint32_t wsel = __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
