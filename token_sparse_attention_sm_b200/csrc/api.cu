@@ -11,6 +11,8 @@
 //                         the select kernel clears it after use)
 //   [.., ..)              fp32 scores S [B,Hkv,N]
 //   [.., ..)              attention split partials (fp32 inputs only)
+#include <stdlib.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -99,6 +101,14 @@ void *attn_ptr(void *ws, const Layout &l) {
 }
 
 }  // namespace
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char *v = getenv("SPARSE_DECODE_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
 
 cudaError_t device_info(DeviceInfo *out) {
   int dev = 0;

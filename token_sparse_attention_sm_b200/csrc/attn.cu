@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(kAttnThreads)
                         int nsplit, float scale, float *__restrict__ part,
                         uint32_t *status) {
   constexpr int EPL = D / 32;  // fp32 elements per lane
+  grid_dep_wait();
+  grid_dep_launch();
   __shared__ __align__(16) float Ks[kChunk][D];
   __shared__ __align__(16) float Vs[kChunk][D];
   __shared__ int valid[kChunk];
@@ -180,6 +182,8 @@ __global__ void __launch_bounds__(256)
                       int Mtot, int B, int Hq, int Hkv, T *__restrict__ out,
                       float *__restrict__ lse) {
   constexpr int EPL = D / 32;
+  grid_dep_wait();
+  grid_dep_launch();
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= BHM) return;

@@ -116,6 +116,8 @@ __global__ void __launch_bounds__(kThreads)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t4 = lane & 3;
 
+  grid_dep_wait();
+  grid_dep_launch();
   extern __shared__ __align__(128) unsigned char smem[];
   __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(smem);
   __nv_bfloat16 *Vs = Ks + 2 * kTileKeys * D;

@@ -204,6 +204,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_dep_wait();  // the index set and queries may come from earlier kernels
+  grid_dep_launch();
   const uint32_t tmem = *tmem_slot;
   const uint32_t t_S = tmem;                          // columns [0, 256)
   const uint32_t t_O = tmem + kChunkKeys;             // columns [256, 256 + D)
@@ -618,11 +620,12 @@ cudaError_t launch_tc_t(const Shape &s, int L, const void *q, const void *K,
   cfg.blockDim = dim3(kTcThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = nsplit > 1 ? 1 : 0;
+  add_pdl_attr(cfg, attr);
   const float scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16 *>(q),
                          static_cast<const __nv_bfloat16 *>(K),

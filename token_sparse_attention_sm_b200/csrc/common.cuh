@@ -31,6 +31,17 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// ---- programmatic dependent launch ----------------------------------------
+// Every kernel waits here before touching memory that an earlier kernel on
+// the stream may still be writing (a no-op unless launched with programmatic
+// stream serialisation), then lets its own dependents start launching.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- mbarrier -------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -23,6 +23,17 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo *out);
 
+// Programmatic dependent launch: a kernel may be scheduled while the previous
+// kernel on the stream drains; it waits (griddepcontrol.wait) before using
+// that kernel's results.  On unless SPARSE_DECODE_PDL=0.
+bool pdl_enabled();
+inline void add_pdl_attr(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attrs) {
+  if (!pdl_enabled()) return;
+  attrs[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+  ++cfg.numAttrs;
+}
+
 // A1: S[b,h,j] for every key; one streaming pass over K.  hist (nullable):
 // [B*Hkv][2048] counts of the top 11 key bits, accumulated (must start zero).
 cudaError_t launch_score(const Shape &s, const void *q, const void *K,

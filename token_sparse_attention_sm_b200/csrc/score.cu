@@ -106,6 +106,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     fence_mbar_init();
   }
   __syncthreads();
+  grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == kConsumerWarps) {
     // ---- producer: one thread issues the bulk copies -----------------------
@@ -222,9 +224,18 @@ cudaError_t launch_score_t(const Shape &s, const void *q, const void *K,
   const long long total = (long long)s.BH() * tiles_per_head;
   const int grid = (int)(total < di.sm_count ? total : di.sm_count);
   const float scale = (float)(1.0 / __builtin_sqrt((double)D));
-  kern<<<grid, kScoreThreads, kScoreSmem, st>>>(
-      static_cast<const T *>(q), static_cast<const T *>(K), S, s.N, s.Hq,
-      s.Hkv, tiles_per_head, total, scale, hist, status);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kScoreThreads, 1, 1);
+  cfg.dynamicSmemBytes = kScoreSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  cfg.attrs = attrs;
+  cfg.numAttrs = 0;
+  add_pdl_attr(cfg, attrs);
+  e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(q), static_cast<const T *>(K), S,
+                         s.N, s.Hq, s.Hkv, tiles_per_head, total, scale, hist, status);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

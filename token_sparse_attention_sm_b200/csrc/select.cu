@@ -53,6 +53,8 @@ __global__ void __launch_bounds__(kSelThreads)
   const int hi = (int)((long long)N * (rank + 1) / csize);
   const int n = hi - lo;
   const float *Sh = S + (size_t)bh * N + lo;
+  grid_dep_wait();
+  grid_dep_launch();
 
   // Load the slice (8 independent loads in flight per thread) and keep it as
   // order-preserving keys.
@@ -145,13 +147,14 @@ cudaError_t launch_select(const Shape &s, const float *S, int k,
   cfg.blockDim = dim3(kSelThreads, 1, 1);
   cfg.dynamicSmemBytes = plan.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)plan.csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  add_pdl_attr(cfg, attr);
   if (plan.in_smem) {
     auto kern = select_kernel<true>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -51,6 +51,8 @@ __global__ void __launch_bounds__(kSelThreads)
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const uint32_t lt_mask = (1u << lane) - 1u;
   const int per_rank = kCandAll / csize;  // receive slots per source CTA
+  grid_dep_wait();
+  grid_dep_launch();
 
   const int N4 = N >> 2;  // N % 4 == 0 on this path
   const int lo4 = (int)((long long)N4 * rank / csize);
@@ -371,13 +373,14 @@ cudaError_t launch_select_topk_fast(const Shape &s, const float *S, int k, int *
   cfg.blockDim = dim3(kSelThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  add_pdl_attr(cfg, attr);
   e = cudaLaunchKernelEx(&cfg, kern, S, s.N, k, idx, hist, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
