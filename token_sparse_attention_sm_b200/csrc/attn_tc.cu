@@ -142,6 +142,14 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// 2^x with the hardware approximation (ex2.approx.ftz: relative error about
+// 2^-22, results below 2^-126 flush to zero -- harmless for softmax weights).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
@@ -363,8 +371,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = c * 8 + e * 2;
-          const float p0 = ((vm >> i) & 1u) ? exp2f(fmaf(__uint_as_float(r[i]), scale_log2, -muse)) : 0.f;
-          const float p1 = ((vm >> (i + 1)) & 1u) ? exp2f(fmaf(__uint_as_float(r[i + 1]), scale_log2, -muse)) : 0.f;
+          const float p0 = ((vm >> i) & 1u) ? fast_exp2(fmaf(__uint_as_float(r[i]), scale_log2, -muse)) : 0.f;
+          const float p1 = ((vm >> (i + 1)) & 1u) ? fast_exp2(fmaf(__uint_as_float(r[i + 1]), scale_log2, -muse)) : 0.f;
           lsum += p0 + p1;
           hi[e] = pack_bf16x2(p0, p1);
           const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162 *>(&hi[e]);
