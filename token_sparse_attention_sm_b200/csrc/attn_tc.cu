@@ -15,8 +15,8 @@
 //     for K, the MN-major layout for V -- the same bytes, read two ways).
 //  2. One thread issues tcgen05.mma (kind::f16, bf16 in, fp32 accumulate,
 //     M=128 query rows, N=64 keys per tile) for S into tensor memory.
-//  3. Query row i lives in tensor-memory lane i; the two warps that share a
-//     lane quadrant split every 64-key tile in halves.  They read S with
+//  3. Query row i lives in tensor-memory lane i; the four warps that share
+//     a lane quadrant split every 64-key tile in quarters.  They read S with
 //     tcgen05.ld, take the exact row maximum of the chunk (joined through
 //     shared memory), and write P = exp2(S*scale*log2e - max) as two bf16
 //     parts (P = P_hi + P_lo, ~16 significant bits) into swizzled shared
@@ -39,7 +39,9 @@
 namespace sd {
 namespace {
 
-constexpr int kTcThreads = 256;     // two warps per tensor-memory lane quadrant
+constexpr int kGroups = 4;          // warps sharing a tensor-memory lane quadrant
+constexpr int kTcThreads = 128 * kGroups;
+constexpr int KPT = 64 / kGroups;    // keys per thread of each 64-key tile
 constexpr int kTcRows = 128;        // MMA M
 constexpr int kTileN = 64;          // keys per S tile (MMA N of QK^T, K of PV)
 constexpr int kChunkTiles = 4;      // tiles per chunk (S uses 256 TMEM columns)
@@ -122,12 +124,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
                : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-               : "memory");
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+               : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+               : "memory");
+}
 
 __device__ __forceinline__ void cp_async16(uint32_t saddr, const void *gmem, bool pred) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr),
@@ -180,9 +187,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int b = bh / Hkv, h = bh % Hkv, G = Hq / Hkv;
   const int M = L * G;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // Warps w and w+4 share tensor-memory lane quadrant w%4 (query rows
-  // 32*(w%4) .. +31); they split every 64-key tile into halves.
-  const int quad = warp & 3, hf = warp >> 2;
+  // Warps w, w+4, ... share tensor-memory lane quadrant w%4 (query rows
+  // 32*(w%4) .. +31); they split every 64-key tile into kGroups parts.
+  const int quad = warp & 3, grp = warp >> 2;
   const int row = quad * 32 + lane;
 
   extern __shared__ unsigned char smem_raw[];
@@ -197,7 +204,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(small + 64);
   int *sidx = reinterpret_cast<int *>(small + 128);            // [256] chunk indices
   unsigned char *kval = small + 128 + 4 * kChunkKeys;          // [256] valid flags
-  float *xred = reinterpret_cast<float *>(small + 128 + 5 * kChunkKeys);  // [2][128]
+  float *xred = reinterpret_cast<float *>(small + 128 + 5 * kChunkKeys);  // [kGroups][128]
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -226,15 +233,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int *rowidx = idx + (size_t)bh * stride;
   const size_t head_off = (size_t)bh * N * D;
 
-  // ---- Q block (rows beyond M are zero): thread = (row, half of the row) ----
+  // ---- Q block (rows beyond M are zero): thread = (row, part of the row) ----
   {
     const int r = tid & (kTcRows - 1), part = tid >> 7;
     const int m = qb * kTcRows + r;
     const __nv_bfloat16 *qr = nullptr;
     if (m < M) qr = q + (((size_t)(m / G) * B + b) * Hq + (size_t)h * G + m % G) * D;
 #pragma unroll
-    for (int cc = 0; cc < CPR / 2; ++cc) {
-      const int c = part * (CPR / 2) + cc;
+    for (int cc = 0; cc < CPR / kGroups; ++cc) {
+      const int c = part * (CPR / kGroups) + cc;
       const uint32_t dst = q_s + (c >> 3) * (kTcRows * 128) + swz(r, c & 7);
       cp_async16(dst, qr ? qr + c * 8 : q, qr != nullptr);
     }
@@ -252,7 +259,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int nk = min(kChunkKeys, k1 - c0);
     const int ntile = (nk + kTileN - 1) / kTileN;
     // indices of the chunk
-    sidx[tid] = tid < nk ? rowidx[c0 + tid] : -1;
+    if (tid < kChunkKeys) sidx[tid] = tid < nk ? rowidx[c0 + tid] : -1;
     __syncthreads();
     // gather the chunk's K rows, then its V rows (two async-copy groups)
     for (int p = tid; p < ntile * kTileN * CPR; p += kTcThreads) {
@@ -296,11 +303,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     // validity of this warp's 32 keys of each tile, as bit masks (ballots over
     // the flags written by the gather; identical in every warp)
-    uint32_t vmask[kChunkTiles];
+    uint32_t vmask[kChunkTiles];  // this thread's KPT keys of each tile
 #pragma unroll
     for (int t = 0; t < kChunkTiles; ++t) {
-      const int key = t * kTileN + hf * 32 + lane;
-      vmask[t] = __ballot_sync(0xffffffffu, key < nk && kval[key] != 0);
+      constexpr int PER32 = 32 / KPT;  // groups covered by one 32-key ballot
+      const int key = t * kTileN + (grp / PER32) * 32 + lane;
+      const uint32_t b = __ballot_sync(0xffffffffu, key < nk && kval[key] != 0);
+      vmask[t] = KPT == 32 ? b : (b >> ((grp % PER32) * KPT)) & ((1u << KPT) - 1u);
     }
     if (!mbar_wait(&bars[0], phase_s & 1u, status)) failed = true;
     ++phase_s;
@@ -315,17 +324,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
     for (int t = 0; t < kChunkTiles; ++t) {
       if (t < ntile) {
-        uint32_t r[32];
-        tmem_ld32(t_S + lane_off + t * kTileN + hf * 32, r);
+        uint32_t r[KPT];
+        if (KPT == 32) tmem_ld32(t_S + lane_off + t * kTileN + grp * KPT, r);
+        else tmem_ld16(t_S + lane_off + t * kTileN + grp * KPT, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < KPT; ++i)
           if ((vmask[t] >> i) & 1u) cmax = fmaxf(cmax, __uint_as_float(r[i]));
       }
     }
-    xred[hf * kTcRows + row] = cmax;
+    xred[grp * kTcRows + row] = cmax;
     __syncthreads();
-    cmax = fmaxf(xred[row], xred[kTcRows + row]) * scale_log2;  // scale > 0
+#pragma unroll
+    for (int g = 0; g < kGroups; ++g) cmax = fmaxf(cmax, xred[g * kTcRows + row]);
+    cmax *= scale_log2;  // scale > 0
     const float mnew = fmaxf(mrun, cmax);
     const float muse = mnew == -INFINITY ? 0.f : mnew;
     const bool rescale = !first_pv && mnew != mrun;
@@ -336,14 +348,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float corr = rescale ? exp2f(mrun - muse) : 1.f;
       lsum *= corr;
 #pragma unroll
-      for (int cb = 0; cb < D / 64; ++cb) {
-        uint32_t r[32];
-        const uint32_t col = t_O + lane_off + hf * (D / 2) + cb * 32;
-        tmem_ld32(col, r);
+      for (int cb = 0; cb < D / kGroups / 16; ++cb) {
+        uint32_t r[16];
+        const uint32_t col = t_O + lane_off + grp * (D / kGroups) + cb * 16;
+        tmem_ld16(col, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
-        tmem_st32(col, r);
+        for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
+        tmem_st16(col, r);
       }
       tmem_wait_st();
     }
@@ -362,11 +374,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int u = 0; u < kChunkTiles; ++u)
         if (u == t) vm = vmask[u];
-      uint32_t r[32];
-      tmem_ld32(t_S + lane_off + t * kTileN + hf * 32, r);
+      uint32_t r[KPT];
+      if (KPT == 32) tmem_ld32(t_S + lane_off + t * kTileN + grp * KPT, r);
+      else tmem_ld16(t_S + lane_off + t * kTileN + grp * KPT, r);
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {  // four 16-byte chunks of 8 keys
+      for (int c = 0; c < KPT / 8; ++c) {  // 16-byte chunks of 8 keys
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -378,7 +391,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162 *>(&hi[e]);
           lo[e] = pack_bf16x2(p0 - __low2float(hb), p1 - __high2float(hb));
         }
-        const uint32_t off = swz(row, hf * 4 + c);
+        const uint32_t off = swz(row, grp * (KPT / 8) + c);
         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(ph + off), "r"(hi[0]),
                      "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
                      : "memory");
@@ -422,35 +435,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int mrows = min(kTcRows, M - qb * kTcRows);  // real query rows of the block
   const bool have = !first_pv && !failed;
   __syncthreads();
-  float *xsum = xred;  // [2][128]: the two warps' halves of each row's sum
-  xsum[hf * kTcRows + row] = have ? lsum : 0.f;
+  float *xsum = xred;  // [kGroups][128]: the warps' parts of each row's sum
+  xsum[grp * kTcRows + row] = have ? lsum : 0.f;
   if (csize == 1) {
     // one split: normalise straight from tensor memory
     __syncthreads();
-    const float ls = xsum[row] + xsum[kTcRows + row];
+    float ls = 0.f;
+#pragma unroll
+    for (int g = 0; g < kGroups; ++g) ls += xsum[g * kTcRows + row];
     const float inv = (have && ls > 0.f) ? 1.f / ls : 0.f;
     const int m = qb * kTcRows + row;
     const size_t orow = m < M ? ((size_t)(m / G) * B + b) * Hq + (size_t)h * G + m % G : 0;
 #pragma unroll
-    for (int cb = 0; cb < D / 64; ++cb) {
-      uint32_t r[32];
+    for (int cb = 0; cb < D / kGroups / 16; ++cb) {
+      uint32_t r[16];
       if (have) {
-        tmem_ld32(t_O + lane_off + hf * (D / 2) + cb * 32, r);
+        tmem_ld16(t_O + lane_off + grp * (D / kGroups) + cb * 16, r);
         tmem_wait_ld();
       }
       if (row < mrows) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
+        for (int i = 0; i < 16; i += 8) {
           uint4 pk;
           pk.x = pack_bf16x2(have ? __uint_as_float(r[i]) * inv : 0.f, have ? __uint_as_float(r[i + 1]) * inv : 0.f);
           pk.y = pack_bf16x2(have ? __uint_as_float(r[i + 2]) * inv : 0.f, have ? __uint_as_float(r[i + 3]) * inv : 0.f);
           pk.z = pack_bf16x2(have ? __uint_as_float(r[i + 4]) * inv : 0.f, have ? __uint_as_float(r[i + 5]) * inv : 0.f);
           pk.w = pack_bf16x2(have ? __uint_as_float(r[i + 6]) * inv : 0.f, have ? __uint_as_float(r[i + 7]) * inv : 0.f);
-          *reinterpret_cast<uint4 *>(out + orow * D + hf * (D / 2) + cb * 32 + i) = pk;
+          *reinterpret_cast<uint4 *>(out + orow * D + grp * (D / kGroups) + cb * 16 + i) = pk;
         }
       }
     }
-    if (lse && hf == 0 && row < mrows)
+    if (lse && grp == 0 && row < mrows)
       lse[orow] = (have && ls > 0.f) ? (mrun + log2f(ls)) * 0.69314718055994531f : -INFINITY;
     tc_fence_before();
     __syncthreads();
@@ -470,16 +485,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float *stage = reinterpret_cast<float *>(base + C::kKPOff);  // [128][PR]
   float *mypart = part + (((size_t)bh * gridDim.y + qb) * csize + rank) * kTcRows * PR;
 #pragma unroll
-  for (int cb = 0; cb < D / 64; ++cb) {
-    uint32_t r[32];
+  for (int cb = 0; cb < D / kGroups / 16; ++cb) {
+    uint32_t r[16];
     if (have) {
-      tmem_ld32(t_O + lane_off + hf * (D / 2) + cb * 32, r);
+      tmem_ld16(t_O + lane_off + grp * (D / kGroups) + cb * 16, r);
       tmem_wait_ld();
     }
     if (row < mrows) {
-      float *dst = stage + row * PR + hf * (D / 2) + cb * 32;
+      float *dst = stage + row * PR + grp * (D / kGroups) + cb * 16;
 #pragma unroll
-      for (int i = 0; i < 32; i += 4)
+      for (int i = 0; i < 16; i += 4)
         *reinterpret_cast<float4 *>(dst + i) =
             have ? make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
                                __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]))
@@ -487,9 +502,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
   __syncthreads();
-  if (hf == 0 && row < mrows)
+  if (grp == 0 && row < mrows) {
+    float ls = 0.f;
+#pragma unroll
+    for (int g = 0; g < kGroups; ++g) ls += xsum[g * kTcRows + row];
     *reinterpret_cast<float4 *>(stage + row * PR + D) =
-        make_float4(have ? mrun : -INFINITY, xsum[row] + xsum[kTcRows + row], 0.f, 0.f);
+        make_float4(have ? mrun : -INFINITY, ls, 0.f, 0.f);
+  }
   __syncthreads();
   {
     const int n4 = mrows * PR / 4;
