@@ -18,7 +18,9 @@ constexpr int kCandLocal = 2048;  // boundary-bin keys one CTA may hold
 constexpr int kCandAll = 8192;    // boundary-bin keys of a whole head
 constexpr int kMaxCluster = 16;
 constexpr int kFinMax = 64;       // keys ranked pairwise after two levels
-constexpr int kSelFixedSmem = 2 * kBins * 4 + kCandLocal * 8 + kCandAll * 4 + 1024;
+constexpr int kWarpList = 128;    // fast path: keys >= the boundary bin per warp
+constexpr int kSelFixedSmem =
+    2 * kBins * 4 + kCandLocal * 8 + kCandAll * 4 + 2 * kSelWarps * kWarpList * 4 + 1024;
 
 struct SelShared {
   uint32_t hist[2][kBins];
@@ -39,6 +41,8 @@ struct SelShared {
   int seg4[kSelWarps + 1];     // fast path: warp segment bounds in float4 units
   uint32_t nfin;               // fast path: keys left after two levels
   uint32_t fin[kFinMax];
+  uint32_t wl_key[kSelWarps][kWarpList];  // fast path: per-warp key lists
+  uint32_t wl_idx[kSelWarps][kWarpList];
 };
 static_assert(sizeof(SelShared) <= kSelFixedSmem, "fixed select smem");
 

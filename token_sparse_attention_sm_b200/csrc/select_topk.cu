@@ -13,8 +13,8 @@
 //     below are out, and only the keys inside b1 (a couple of thousand at the
 //     headline sizes) need the remaining 21 bits.
 //  2. One pass loads the slice, keeps it on chip as order-preserving keys,
-//     counts per warp the keys above b1, and appends the keys inside b1
-//     (with their slice index) to a shared-memory candidate list.
+//     and appends every key at or above b1 (with its slice index) to its
+//     warp's list, in index order (a warp scan per float4 column).
 //  3. Each CTA pushes its candidate keys into every CTA's shared memory
 //     (distributed shared-memory stores); after one cluster barrier every CTA
 //     finishes the selection on that small list locally: one more 11-bit
@@ -22,9 +22,10 @@
 //     exactly by pairwise counts within one warp (a 10-bit histogram level
 //     only if more than 64 remain).  Rank 0 clears the head's histogram for the
 //     next call.
-//  4. Per-warp counts (keys above b1 plus own candidates that pass) are
-//     pushed the same way; one more cluster barrier gives every warp its
-//     output offset, and a last pass writes the indices in ascending order.
+//  4. Each warp counts the entries of its list that pass; the per-CTA
+//     totals are pushed the same way; one more cluster barrier gives every
+//     warp its output offset, and the warp writes its passing entries in
+//     list (= ascending index) order -- no second pass over the slice.
 //     All exchanges are pushes, so no CTA reads another's shared memory
 //     after the last barrier and no trailing barrier is needed.
 // Falls back to the general multi-level cluster path when the histogram is
@@ -36,7 +37,7 @@
 namespace sd {
 namespace {
 
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __launch_bounds__(kSelThreads, 1)
     select_topk_fast_kernel(const float *__restrict__ S, int N, int k,
                             int *__restrict__ idx, uint32_t *__restrict__ hist,
                             uint32_t *status) {
@@ -94,7 +95,12 @@ __global__ void __launch_bounds__(kSelThreads)
   const int sg0 = (int)((long long)n4 * wid / kSelWarps);
   const int sg1 = (int)((long long)n4 * (wid + 1) / kSelWarps);
   constexpr int U = 8;  // float4 per lane per batch
-  uint32_t wdef = 0;
+  // Per-warp list, in index order, of the keys whose top 11 bits are >= b1
+  // (every key that can be selected); a few dozen per warp in practice.
+  uint32_t *wl_key = sh->wl_key[wid];
+  uint32_t *wl_idx = sh->wl_idx[wid];
+  uint32_t wn = 0, wcand = 0;  // list length, boundary-bin keys in it
+  bool wover = false;
   bool bad = false;
   for (int b4 = sg0; b4 < sg1; b4 += U * 32) {
     float4 f[U];
@@ -103,8 +109,6 @@ __global__ void __launch_bounds__(kSelThreads)
       const int i4 = b4 + u * 32 + lane;
       f[u] = i4 < sg1 ? S4[i4] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    uint32_t cand[U];  // 4 candidate bits per float4
-    uint32_t nc = 0;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int i4 = b4 + u * 32 + lane;
@@ -116,62 +120,77 @@ __global__ void __launch_bounds__(kSelThreads)
         bad |= !isfinite(f[u].x) | !isfinite(f[u].y) | !isfinite(f[u].z) |
                !isfinite(f[u].w);
       }
+      if (!fast) continue;
       const uint32_t kv[4] = {kk.x, kk.y, kk.z, kk.w};
-      uint32_t cm = 0;
+      uint32_t qm = 0, cm = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const uint32_t top = kv[e] >> 21;
-        wdef += (in && top > b1) ? 1u : 0u;
+        qm |= (in && top >= b1) ? (1u << e) : 0u;
         cm |= (in && top == b1) ? (1u << e) : 0u;
       }
-      cand[u] = cm;
-      nc += __popc(cm);
-    }
-    if (fast && __any_sync(0xffffffffu, nc != 0)) {
-      uint32_t inc = nc;
+      const uint32_t c = __popc(qm);
+      if (!__any_sync(0xffffffffu, c != 0)) continue;
+      uint32_t inc = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
         if (lane >= o) inc += y;
       }
-      const uint32_t wtot = __shfl_sync(0xffffffffu, inc, 31);
-      uint32_t base = 0;
-      if (lane == 31) base = atomicAdd(&sh->ncand, wtot);
-      base = __shfl_sync(0xffffffffu, base, 31) + inc - nc;
+      uint32_t slot = wn + inc - c;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (cand[u]) {
-          const int i4 = b4 + u * 32 + lane;
-          const uint4 kk = keys4[i4];
-          const uint32_t kv[4] = {kk.x, kk.y, kk.z, kk.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if ((cand[u] >> e) & 1u) {
-              if (base < (uint32_t)kCandLocal)
-                sh->cand_local[base] = make_uint2(kv[e], (uint32_t)(4 * i4 + e));
-              ++base;
-            }
+      for (int e = 0; e < 4; ++e) {
+        if ((qm >> e) & 1u) {
+          if (slot < (uint32_t)kWarpList) {
+            wl_key[slot] = kv[e];
+            wl_idx[slot] = (uint32_t)(4 * i4 + e);
           }
+          ++slot;
         }
       }
+      wn += __shfl_sync(0xffffffffu, inc, 31);
+      wcand += __popc(__ballot_sync(0xffffffffu, cm & 1u)) +
+               __popc(__ballot_sync(0xffffffffu, cm & 2u)) +
+               __popc(__ballot_sync(0xffffffffu, cm & 4u)) +
+               __popc(__ballot_sync(0xffffffffu, cm & 8u));
     }
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) wdef += __shfl_xor_sync(0xffffffffu, wdef, o);
-  if (lane == 0) sh->wdef[wid] = wdef;
+  wover = wn > (uint32_t)kWarpList;
+  if (lane == 0) {
+    sh->wdef[wid] = wcand;          // this warp's boundary-bin keys
+    sh->wpass[wid] = wover ? 1u : 0u;
+  }
   if (__syncthreads_or(bad) && tid == 0) raise_flag(status, FLAG_NONFINITE);
   auto key_at = [&](int t) -> uint32_t { return keys[t]; };
+  // candidates of this CTA = boundary-bin entries of every warp list, in
+  // warp order; any list overflow turns the fast path off cluster-wide
+  uint32_t cand_off = 0, my_cand = 0, my_over = 0;
+#pragma unroll
+  for (int i = 0; i < kSelWarps; ++i) {
+    cand_off += i < wid ? sh->wdef[i] : 0u;
+    my_cand += sh->wdef[i];
+    my_over |= sh->wpass[i];
+  }
 
-  // push this CTA's candidate count and keys into every CTA of the cluster
-  // (remote stores; the barrier below makes them visible)
-  const uint32_t my_cand = sh->ncand;
+  // push this CTA's candidate count (with the overflow flag in bit 31) and
+  // keys into every CTA of the cluster (remote stores; the barrier below makes
+  // them visible)
   if (fast) {
-    if (tid < csize) cluster.map_shared_rank(sh->rcnt, tid)[rank] = my_cand;
-    const uint32_t npush = min(my_cand, (uint32_t)per_rank);
-    for (uint32_t i = tid; i < npush; i += kSelThreads) {
-      const uint32_t key = sh->cand_local[i].x;
-      for (int r = 0; r < csize; ++r)
-        cluster.map_shared_rank(sh->cand_all, r)[rank * per_rank + i] = key;
+    if (tid < csize)
+      cluster.map_shared_rank(sh->rcnt, tid)[rank] = my_cand | (my_over << 31);
+    if (!wover) {
+      uint32_t o = cand_off;
+      for (uint32_t i0 = 0; i0 < wn; i0 += 32) {
+        const uint32_t i = i0 + lane;
+        const uint32_t key = i < wn ? wl_key[i] : 0u;
+        const bool c = i < wn && (key >> 21) == b1;
+        const uint32_t m = __ballot_sync(0xffffffffu, c);
+        const uint32_t slot = o + __popc(m & lt_mask);
+        if (c && slot < (uint32_t)per_rank)
+          for (int r = 0; r < csize; ++r)
+            cluster.map_shared_rank(sh->cand_all, r)[rank * per_rank + slot] = key;
+        o += __popc(m);
+      }
     }
   }
   cluster.sync();  // candidates delivered; every CTA has read the histogram
@@ -184,7 +203,10 @@ __global__ void __launch_bounds__(kSelThreads)
   bool fast_ok = fast;
   if (fast) {
     uint32_t over = 0;
-    for (int r = 0; r < csize; ++r) over |= sh->rcnt[r] > (uint32_t)per_rank;
+    for (int r = 0; r < csize; ++r) {
+      over |= sh->rcnt[r] >> 31;
+      over |= (sh->rcnt[r] & 0x7FFFFFFFu) > (uint32_t)per_rank;
+    }
     fast_ok = over == 0u;  // uniform: every CTA received the same counts
     if (fast_ok) {
       for (int b = tid; b < kBins; b += kSelThreads) sh->hist[1][b] = 0;
@@ -297,23 +319,22 @@ __global__ void __launch_bounds__(kSelThreads)
     return;
   }
 
-  // ---- 4. per-warp counts, pushed offsets, ordered write --------------------
-  const uint32_t nloc = min(my_cand, (uint32_t)kCandLocal);
-  for (uint32_t i = tid; i < nloc; i += kSelThreads) {
-    const uint2 cd = sh->cand_local[i];
-    if ((uint64_t)cd.x >= t_ge) {
-      const int q4 = (int)(cd.y >> 2);
-      int w = 0;
-#pragma unroll
-      for (int s = 1; s < kSelWarps; ++s) w += q4 >= sh->seg4[s];
-      atomicAdd(&sh->wpass[w], 1u);
-    }
+  // ---- 4. per-warp counts from the lists, pushed offsets, ordered write ------
+  // t_ge <= 2^32 here; keep the compares 32-bit
+  const bool none = t_ge > 0xFFFFFFFFull;
+  const uint32_t t32 = (uint32_t)t_ge;
+  uint32_t wsel = 0;
+  for (uint32_t i0 = 0; i0 < wn; i0 += 32) {
+    const uint32_t i = i0 + lane;
+    wsel += __popc(__ballot_sync(0xffffffffu, i < wn && !none && wl_key[i] >= t32));
   }
+  __syncthreads();  // every warp has read wdef / wpass above
+  if (lane == 0) sh->wge[wid] = wsel;
   __syncthreads();
   uint32_t before = 0, cta_sel = 0;
 #pragma unroll
   for (int i = 0; i < kSelWarps; ++i) {
-    const uint32_t sel = sh->wdef[i] + sh->wpass[i];
+    const uint32_t sel = sh->wge[i];
     before += i < wid ? sel : 0u;
     cta_sel += sel;
   }
@@ -324,27 +345,13 @@ __global__ void __launch_bounds__(kSelThreads)
     pos += r < rank ? sh->rge[r] : 0u;
     total_sel += sh->rge[r];
   }
-  // t_ge <= 2^32 here; keep the compares 32-bit
-  const bool none = t_ge > 0xFFFFFFFFull;
-  const uint32_t t32 = (uint32_t)t_ge;
-  for (int b4 = sg0; b4 < sg1; b4 += 32) {
-    const int i4 = b4 + lane;
-    const bool in = i4 < sg1 && !none;
-    const uint4 kk = in ? keys4[i4] : make_uint4(0u, 0u, 0u, 0u);
-    const bool s0 = in && kk.x >= t32, s1 = in && kk.y >= t32;
-    const bool s2 = in && kk.z >= t32, s3 = in && kk.w >= t32;
-    const uint32_t q0 = __ballot_sync(0xffffffffu, s0), q1 = __ballot_sync(0xffffffffu, s1);
-    const uint32_t q2 = __ballot_sync(0xffffffffu, s2), q3 = __ballot_sync(0xffffffffu, s3);
-    const uint32_t wsel = __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
-    if (wsel == 0) continue;
-    uint32_t p = pos + __popc(q0 & lt_mask) + __popc(q1 & lt_mask) + __popc(q2 & lt_mask) +
-                 __popc(q3 & lt_mask);
-    const int j = lo + 4 * i4;
-    if (s0) { if (p < (uint32_t)k) out[p] = j; ++p; }
-    if (s1) { if (p < (uint32_t)k) out[p] = j + 1; ++p; }
-    if (s2) { if (p < (uint32_t)k) out[p] = j + 2; ++p; }
-    if (s3) { if (p < (uint32_t)k) out[p] = j + 3; ++p; }
-    pos += wsel;
+  for (uint32_t i0 = 0; i0 < wn; i0 += 32) {
+    const uint32_t i = i0 + lane;
+    const bool take = i < wn && !none && wl_key[i] >= t32;
+    const uint32_t m = __ballot_sync(0xffffffffu, take);
+    const uint32_t p = pos + __popc(m & lt_mask);
+    if (take && p < (uint32_t)k) out[p] = lo + (int)wl_idx[i];
+    pos += __popc(m);
   }
   if (rank == 0 && tid == 0 && total_sel != (uint32_t)k) raise_flag(status, FLAG_INTERNAL);
 }
