@@ -57,6 +57,22 @@
  *
  * Asynchrony: every compute entry point enqueues its kernels on `stream`
  * and returns without synchronising.
+ *
+ * Co-residency: the bf16 attention kernel (and the optional fused routing
+ * kernel) split one head's work over several CTAs that wait for one another
+ * (bounded waits).  Their grid is at most one CTA per SM, so it is resident
+ * as a whole while the device runs nothing else; they are launched as
+ * ordinary kernels so that each can start while its predecessor drains.  A
+ * caller that runs other kernels on the same device at the same time (other
+ * streams, other processes) sets SPARSE_DECODE_COOPERATIVE=1: they are then
+ * launched cooperatively and the driver guarantees co-residency.
+ *
+ * Environment variables read by the library:
+ *   SPARSE_DECODE_PDL=0           no programmatic dependent launch
+ *   SPARSE_DECODE_COOPERATIVE=1   cooperative launches (see Co-residency)
+ *   SPARSE_DECODE_FUSED_ROUTE=1   top-k routing as one fused scan+select kernel
+ *                                 where the shape allows (results identical)
+ *   SPARSE_DECODE_ATTN=mma        bf16 attention on the mma.sync kernel
  */
 #ifndef SPARSE_DECODE_H_
 #define SPARSE_DECODE_H_

@@ -236,6 +236,15 @@ def test_attn_gather_bad_index_flags_without_fault(dev):
 # Routing end to end and the fused step
 # ---------------------------------------------------------------------------
 
+@pytest.fixture(params=["fused", "scan_then_select"])
+def route_path(request, monkeypatch):
+    """Routing runs as one fused scan+select kernel when the shape allows it,
+    else as the scan kernel followed by the select kernel; every routing test
+    runs both ways."""
+    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "1" if request.param == "fused" else "0")
+    return request.param
+
+
 ROUTE_CASES = [
     dict(B=1, N=4096, Hq=8, Hkv=2, d=64, k=256, dtype="f32"),
     dict(B=2, N=10007, Hq=32, Hkv=8, d=128, k=333, dtype="bf16", heavy=16),
@@ -245,7 +254,7 @@ ROUTE_CASES = [
 
 
 @pytest.mark.parametrize("c", ROUTE_CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
-def test_route_topk_matches_oracle(dev, c):
+def test_route_topk_matches_oracle(dev, c, route_path):
     w = synth.custom(L=1, seed=c["N"], **c)
     x = synth.generate(w)
     t = _to(dev, x)
@@ -290,7 +299,7 @@ def _check_decode(dev, w, x, batches_checked=None):
 
 
 @pytest.mark.parametrize("name", ["tiny_f32", "decode_32k", "decode_128k"])
-def test_decode_step_named_workloads(dev, name):
+def test_decode_step_named_workloads(dev, name, route_path):
     w = synth.WORKLOADS[name]
     x = synth.generate(w)
     _check_decode(dev, w, x)
@@ -345,7 +354,7 @@ def test_decode_step_threshold_empty_set(dev):
     assert torch.all(res["out"] == 0) and torch.all(torch.isneginf(res["lse"]))
 
 
-def test_route_topk_all_equal_keys_takes_lowest_indices(dev):
+def test_route_topk_all_equal_keys_takes_lowest_indices(dev, route_path):
     """Every score equal: the boundary bin holds all N keys, more than the
     candidate buffers, so the select takes its general path."""
     w = synth.custom(B=1, N=20000, Hq=8, Hkv=2, d=128, L=1, k=300, dtype="bf16", seed=4)
@@ -357,7 +366,7 @@ def test_route_topk_all_equal_keys_takes_lowest_indices(dev):
     np.testing.assert_array_equal(idx, np.tile(np.arange(300), (1, 2, 1)))
 
 
-def test_route_topk_recovers_from_dirty_workspace(dev):
+def test_route_topk_recovers_from_dirty_workspace(dev, route_path):
     """A workspace whose histogram area holds garbage (not zero-filled) is
     detected (the counts do not sum to N) and the result is still exact; the
     call leaves the workspace clean for the next one."""
@@ -367,11 +376,11 @@ def test_route_topk_recovers_from_dirty_workspace(dev):
     S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
     ws = sd.Workspace(dev)
     ws.get(sd.workspace_bytes(2, 5000, 8, 2, 128, torch.bfloat16, 100, 1))
-    ws.buf[1024:1024 + 4 * 2048 * 4] = 7  # the histogram area (after the 1 KB header)
+    ws.buf[4096:4096 + 4 * 2048 * 4] = 7  # the histogram area (after the 4 KB header)
     for _ in range(2):
         gidx = sd.route_topk(t["q_route"], t["K"], 100, ws=ws).cpu().numpy()
         assert_topk_within_band(gidx, S, 100)
-    assert int(ws.buf[1024:1024 + 4 * 2048 * 4].sum()) == 0
+    assert int(ws.buf[4096:4096 + 4 * 2048 * 4].sum()) == 0
 
 
 @pytest.mark.parametrize("k,count", [(4096, None), (8192, [3933, 4100, 100, 0, 8192, 2, 3000, 7000])])
@@ -404,7 +413,7 @@ def test_attn_gather_mma_sync_variant_matches(dev, monkeypatch):
 
 
 @pytest.mark.parametrize("kind", ["random", "duplicated_rows", "few_values", "heavy"])
-def test_route_topk_bit_exact_on_its_own_scores(dev, kind):
+def test_route_topk_bit_exact_on_its_own_scores(dev, kind, route_path):
     """Routing (scan + histogram fast-path select) against the oracle's top-k
     of the very scores the scan produced: identical fp32 scores, so the index
     sets must be identical, ties included."""
@@ -423,3 +432,22 @@ def test_route_topk_bit_exact_on_its_own_scores(dev, kind):
     S = sd.score(t["q_route"], K, ws=ws).cpu().numpy()
     idx = sd.route_topk(t["q_route"], K, w.k, ws=ws).cpu().numpy()
     np.testing.assert_array_equal(idx, oracle.topk(S, w.k))
+
+
+@pytest.mark.parametrize("B,N,Hkv,k", [(1, 131072, 8, 2048), (3, 20000, 2, 1), (4, 8192, 4, 8000),
+                                       (1, 65536, 1, 700), (2, 2048, 8, 64)])
+def test_fused_route_equals_scan_then_select(dev, monkeypatch, B, N, Hkv, k):
+    """The fused scan+select kernel and the two-kernel path give the same
+    index sets, bit for bit (same scan arithmetic, exact selection), over
+    shapes where CTAs span two heads, a head spans one CTA or many, k = 1 and
+    k close to N."""
+    w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=1, k=k, dtype="bf16", seed=N + k)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "1")
+    a = sd.route_topk(t["q_route"], t["K"], k).cpu().numpy()
+    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "0")
+    b = sd.route_topk(t["q_route"], t["K"], k).cpu().numpy()
+    np.testing.assert_array_equal(a, b)
+    S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
+    assert_topk_within_band(a, S, k)

@@ -4,13 +4,18 @@
 // before anything is enqueued; then it enqueues the kernels on the caller's
 // stream and returns.  The library allocates nothing: scratch lives in the
 // caller's workspace, whose layout is
-//   [0, 1024)             header: device status word (uint32) at offset 0;
-//                         [256, 1024) attention split-merge counters (a fixed,
-//                         shape-independent area, zero between calls)
-//   [1024, ..)            radix histogram [B*Hkv][2048] uint32 (scan -> select;
-//                         the select kernel clears it after use)
+//   [0, 4096)             header: device status word (uint32) at offset 0;
+//                         [256, 1024) attention split-merge counters;
+//                         [1024, 4096) fused-routing barrier counters, one
+//                         per head (fixed, shape-independent areas, zero
+//                         between calls: the kernels reset them)
+//   [4096, ..)            radix histogram [max(B*Hkv, 256)][2048] uint32 (scan ->
+//                         select; cleared after use).  At least 256 rows, so
+//                         that calls of different shapes (up to 256 heads)
+//                         sharing one workspace never put other data there.
 //   [.., ..)              fp32 scores S [B,Hkv,N]
-//   [.., ..)              attention split partials (fp32 inputs only)
+//   [.., ..)              fused routing: published boundary-bin keys
+//   [.., ..)              attention split partials
 #include <stdlib.h>
 
 #include <mutex>
@@ -30,21 +35,25 @@ DeviceInfo g_info[kMaxDevices];
 cudaError_t g_info_err[kMaxDevices];
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-constexpr size_t kHeader = 1024;
+constexpr size_t kHeader = 4096;
 constexpr size_t kCountersOff = 256;
+constexpr size_t kRouteCountersOff = 1024;
+constexpr int kHistMinRows = 256;
 
 struct Layout {
-  size_t hist_off, hist_bytes, scores_off, scores_bytes, attn_off, attn_bytes,
-      total;
+  size_t hist_off, hist_bytes, scores_off, scores_bytes, seg_off, seg_bytes, attn_off,
+      attn_bytes, total;
 };
 
 Layout layout(const Shape &s, int stride, int L) {
   Layout l;
   l.hist_off = kHeader;
-  l.hist_bytes = align_up((size_t)s.BH() * 2048 * sizeof(uint32_t), 256);
+  l.hist_bytes = (size_t)(s.BH() > kHistMinRows ? s.BH() : kHistMinRows) * 2048 * sizeof(uint32_t);
   l.scores_off = l.hist_off + l.hist_bytes;
   l.scores_bytes = align_up((size_t)s.BH() * s.N * sizeof(float), 256);
-  l.attn_off = l.scores_off + l.scores_bytes;
+  l.seg_off = l.scores_off + l.scores_bytes;
+  l.seg_bytes = align_up(kFusedSegAreaBytes, 256);
+  l.attn_off = l.seg_off + l.seg_bytes;
   l.attn_bytes = align_up(attn_workspace_bytes(s, L, stride), 256);
   l.total = l.attn_off + l.attn_bytes;
   return l;
@@ -88,8 +97,15 @@ uint32_t *status_word(void *ws) { return static_cast<uint32_t *>(ws); }
 uint32_t *attn_counters(void *ws) {
   return reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + kCountersOff);
 }
-static_assert(kCountersOff + 2 * sizeof(uint32_t) * kAttnMaxCounterBlocks <= kHeader,
-              "counter area fits in the header");
+static_assert(kCountersOff + 2 * sizeof(uint32_t) * kAttnMaxCounterBlocks <= kRouteCountersOff,
+              "attention counters fit in their area");
+static_assert(kRouteCountersOff + sizeof(uint32_t) * kFusedMaxHeads <= kHeader,
+              "routing counters fit in the header");
+uint32_t *route_counters(void *ws) {
+  return reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + kRouteCountersOff);
+}
+void *seg_ptr(void *ws, const Layout &l) { return static_cast<char *>(ws) + l.seg_off; }
+
 uint32_t *hist_ptr(void *ws, const Layout &l) {
   return reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + l.hist_off);
 }
@@ -100,7 +116,31 @@ void *attn_ptr(void *ws, const Layout &l) {
   return static_cast<char *>(ws) + l.attn_off;
 }
 
+// A1 + A2 (top-k): the fused kernel when the shape allows it, else the scan
+// followed by the select kernel.
+cudaError_t route_topk_any(const Shape &s, const void *q, const void *K, int k, int *idx,
+                           void *ws, const Layout &l, cudaStream_t st) {
+  float *S = scores_ptr(ws, l);
+  uint32_t *hist = hist_ptr(ws, l);
+  cudaError_t e = launch_route_topk_fused(s, q, K, k, S, hist, route_counters(ws),
+                                          seg_ptr(ws, l), idx, status_word(ws), st);
+  if (e != cudaErrorNotSupported) return e;
+  cudaGetLastError();
+  e = launch_score(s, q, K, S, hist, status_word(ws), st);
+  if (e == cudaSuccess)
+    e = launch_select(s, S, k, nullptr, 0, idx, nullptr, k, hist, status_word(ws), st);
+  return e;
+}
+
 }  // namespace
+
+bool cooperative_forced() {
+  static const bool on = [] {
+    const char *v = getenv("SPARSE_DECODE_COOPERATIVE");
+    return v && v[0] == '1';
+  }();
+  return on;
+}
 
 bool pdl_enabled() {
   static const bool on = [] {
@@ -231,13 +271,8 @@ sparse_status_t sparse_route_topk(const sparse_shape_t *shape, const void *q,
     return SPARSE_ERR_INVALID_ARG;
   if ((r = sd::check_ws(s, k, 1, ws, ws_bytes)) != SPARSE_OK) return r;
   const sd::Layout l = sd::layout(s, k, 1);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float *S = sd::scores_ptr(ws, l);
-  uint32_t *hist = sd::hist_ptr(ws, l);
-  cudaError_t e = sd::launch_score(s, q, K, S, hist, sd::status_word(ws), st);
-  if (e == cudaSuccess)
-    e = sd::launch_select(s, S, k, nullptr, 0, idx, nullptr, k, hist,
-                          sd::status_word(ws), st);
+  cudaError_t e =
+      sd::route_topk_any(s, q, K, k, idx, ws, l, static_cast<cudaStream_t>(stream));
   return sd::from_cuda(e);
 }
 
@@ -316,12 +351,15 @@ sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
   const sd::Layout l = sd::layout(s, stride, L);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t *status = sd::status_word(ws);
-  float *S = sd::scores_ptr(ws, l);
-  uint32_t *hist = topk ? sd::hist_ptr(ws, l) : nullptr;
-  cudaError_t e = sd::launch_score(s, q_route, K, S, hist, status, st);
-  if (e == cudaSuccess)
-    e = topk ? sd::launch_select(s, S, k, nullptr, 0, idx, nullptr, k, hist, status, st)
-             : sd::launch_select(s, S, 0, tau, cap, idx, count, cap, nullptr, status, st);
+  cudaError_t e;
+  if (topk) {
+    e = sd::route_topk_any(s, q_route, K, k, idx, ws, l, st);
+  } else {
+    float *S = sd::scores_ptr(ws, l);
+    e = sd::launch_score(s, q_route, K, S, nullptr, status, st);
+    if (e == cudaSuccess)
+      e = sd::launch_select(s, S, 0, tau, cap, idx, count, cap, nullptr, status, st);
+  }
   if (e == cudaSuccess)
     e = sd::launch_attn(s, L, q_layers, K, V, idx, stride, topk ? nullptr : count,
                         stride, out, lse, sd::attn_ptr(ws, l), sd::attn_counters(ws), status,

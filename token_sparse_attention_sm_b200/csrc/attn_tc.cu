@@ -27,8 +27,8 @@
 // when a CTA holds more than 256 keys).  With one split the CTA normalises O
 // and writes out directly.  With several, each writes its partial (O, max,
 // sum) for the real query rows to the workspace, arrives on a per-head
-// counter and waits (bounded) for the other splits -- the launch is
-// cooperative, so all of them are resident -- then merges its share of the
+// counter and waits (bounded) for the other splits -- the grid is at most
+// one CTA per SM, so all of them are resident -- then merges its share of the
 // rows by log-sum-exp rescaling; the last split to leave resets the counters.
 //
 // Every wait is bounded; on expiry the kernel raises the TIMEOUT flag, stops
@@ -525,7 +525,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                  "r"(kTmemCols)
                  : "memory");
   // arrive, then wait (bounded) until every split of this head block arrived;
-  // the launch is cooperative, so all of them are resident
+  // the grid (at most one CTA per SM) is resident as a whole
   uint32_t *arrive = counters + 2 * ((size_t)bh * gridDim.y + qb);
   uint32_t *depart = arrive + 1;
   __shared__ int ready;
@@ -651,7 +651,7 @@ cudaError_t launch_tc_t(const Shape &s, int L, const void *q, const void *K,
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = nsplit > 1 ? 1 : 0;
+  cfg.numAttrs = (nsplit > 1 && cooperative_forced()) ? 1 : 0;
   add_pdl_attr(cfg, attr);
   const float scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16 *>(q),

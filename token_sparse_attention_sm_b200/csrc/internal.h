@@ -40,6 +40,34 @@ cudaError_t launch_score(const Shape &s, const void *q, const void *K,
                          float *S, uint32_t *hist, uint32_t *status,
                          cudaStream_t st);
 
+// A1 + A2 fused (route_fused.cu): the scan and the exact top-k in one
+// persistent kernel whose CTAs synchronise per head through counters in
+// global memory.  ctr: one uint32 per head, zero between calls (the kernel
+// resets them); seg_area: kFusedSegAreaBytes of scratch.  Returns
+// cudaErrorNotSupported, launching nothing, when the shape does not fit (a
+// CTA's keys must fit on chip) or unless SPARSE_DECODE_FUSED_ROUTE=1 (the
+// scan followed by the select kernel is the default: at the 128K decode
+// shapes the two are on par and the two-kernel path leaves SMs free for the
+// attention kernel to start early).
+constexpr int kFusedMaxCtas = 256;
+constexpr int kFusedMaxHeads = 768;
+constexpr int kFusedSegCap = 1024;  // boundary-bin keys a CTA publishes per head
+constexpr size_t kFusedMetaBytes = (size_t)kFusedMaxCtas * 2 * 8;
+constexpr size_t kFusedSegAreaBytes =
+    kFusedMetaBytes + (size_t)kFusedMaxCtas * 2 * kFusedSegCap * sizeof(uint32_t);
+bool fused_route_enabled();
+cudaError_t launch_route_topk_fused(const Shape &s, const void *q, const void *K, int k,
+                                    float *S, uint32_t *hist, uint32_t *ctr, void *seg_area,
+                                    int *idx, uint32_t *status, cudaStream_t st);
+
+// Kernels whose CTAs wait for one another (the fused routing kernel, the
+// split merge of the tcgen05 attention) rely on the whole grid being resident
+// at once -- at most one CTA per SM.  They are launched as ordinary kernels so
+// that programmatic dependent launch can overlap them with their predecessor;
+// SPARSE_DECODE_COOPERATIVE=1 launches them cooperatively instead (the driver
+// then guarantees co-residency even next to other work on the device).
+bool cooperative_forced();
+
 // A2 / A2': selection from S.  k >= 1: top-k (tau ignored); k == 0:
 // threshold with tau and cap, count written.  idx rows have `stride`
 // entries.

@@ -1,0 +1,184 @@
+// scan.cuh -- the streaming q.K scan shared by the score kernel (score.cu)
+// and the fused routing kernel (route_fused.cu).
+//
+// S[b,h,j] = (sum over the G query heads of KV head h: <q_g, K[b,h,j]>)/sqrt(d)
+// (CLSA article, section CLSAの仕組み).  A CTA owns a contiguous run of 32 KB
+// key tiles (tiles never straddle heads).  One producer thread streams them
+// into a shared-memory ring with 1-D bulk copies (cp.async.bulk + mbarrier
+// transaction counts, L2 evict-first: K is read once); four consumer warps
+// read them back with conflict-free 128-bit shared loads.  A warp handles 32
+// keys at a time: each lane loads 16 bytes of a row per round (rows are split
+// over LPK lanes), keeps one partial dot per round, and a transposing shuffle
+// reduction leaves one finished score per lane, stored as one coalesced
+// 128-byte write.  The G query rows are summed once into qbar (fp32) and
+// pre-scaled by 1/sqrt(d); by linearity this is the group sum, only the fp32
+// rounding order differs.
+#pragma once
+
+#include "common.cuh"
+
+namespace sd {
+namespace {
+
+constexpr int kScanConsumerWarps = 4;
+constexpr int kScanStages = 5;
+constexpr int kScanStageBytes = 32768;
+constexpr int kScanThreads = (kScanConsumerWarps + 1) * 32;
+constexpr int kScanBins = 2048;  // top 11 bits of the order-preserving key
+
+template <typename T, int D>
+struct ScoreCfg {
+  static constexpr int kRowBytes = D * (int)sizeof(T);
+  static constexpr int kEpl = 16 / (int)sizeof(T);  // elements per 16 B
+  static constexpr int kLpk = D / kEpl;              // lanes per key row
+  static constexpr int kKpr = 32 / kLpk;             // keys per round
+  static constexpr int kStageKeys = kScanStageBytes / kRowBytes;
+  static constexpr int kWarpTiles = kStageKeys / 32;
+  static_assert(kKpr * kRowBytes == 512, "a round covers 512 contiguous bytes");
+  static_assert(kWarpTiles >= 1, "stage holds at least one warp tile");
+};
+
+// Transposing reduction: on entry v[0..R) are per-lane partial sums of R
+// different keys; partners `O` lanes apart exchange halves.  On exit v[0]
+// holds the finished sum of key (lane % (2*O_top)).
+template <int R, int O>
+struct TReduce {
+  static __device__ __forceinline__ void run(float *v, int lane) {
+    const bool upper = (lane & O) != 0;
+#pragma unroll
+    for (int i = 0; i < R / 2; ++i) {
+      const float send = upper ? v[i] : v[i + R / 2];
+      const float keep = upper ? v[i + R / 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+    }
+    TReduce<R / 2, O / 2>::run(v, lane);
+  }
+};
+template <int R>
+struct TReduce<R, 0> {
+  static __device__ __forceinline__ void run(float *, int) {}
+};
+
+// Where the scan puts its by-products.  shist: kSlots per-head shared-memory
+// histograms (heads bh_first .. bh_first + kSlots - 1; later heads go to the
+// global histogram directly); hist == nullptr disables counting.  keys
+// (nullable): order-preserving keys kept on chip, key j of head bh_first at
+// keys[key_off + j].  (Plain scalars, not an array: an array indexed by a
+// run-time value would be placed in local memory and reloaded in the loop.)
+struct ScanOut {
+  float *S;
+  uint32_t *hist;
+  uint32_t *shist;
+  uint32_t *keys;
+  int key_off;
+};
+
+// One CTA's share of the scan: tiles [t_begin, t_begin + ntiles).  Warps
+// 0..3 consume, warp 4 produces: its lane 0 issues the copies and waits for
+// the last ones to land, its other lanes (and any further warps) return at
+// once.  Barriers full/empty
+// must be initialised (count 1 / kScanConsumerWarps).
+template <typename T, int D, int kSlots>
+__device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__restrict__ K,
+                                           int N, int Hq, int Hkv, int tiles_per_head,
+                                           long long t_begin, int ntiles, int bh_first,
+                                           float scale, unsigned char *ring, uint64_t *full,
+                                           uint64_t *empty, ScanOut o,
+                                           uint32_t *status) {
+  using C = ScoreCfg<T, D>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp > kScanConsumerWarps) return;  // extra warps of a larger CTA idle here
+  if (warp == kScanConsumerWarps) {
+    // ---- producer: one thread issues the bulk copies -------------------------
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % kScanStages;
+        if (i >= kScanStages &&
+            !mbar_wait(&empty[s], ((i / kScanStages) - 1) & 1, status))
+          break;
+        const long long t = t_begin + i;
+        const int bh = (int)(t / tiles_per_head);
+        const int j0 = (int)(t % tiles_per_head) * C::kStageKeys;
+        const int nk = min(C::kStageKeys, N - j0);
+        const uint32_t bytes = (uint32_t)nk * C::kRowBytes;
+        mbar_arrive_expect_tx(&full[s], bytes);
+        bulk_g2s(ring + (size_t)s * kScanStageBytes, K + ((size_t)bh * N + j0) * D,
+                 bytes, &full[s], pol);
+        ++issued;
+      }
+      // Do not leave while copies may still be landing in shared memory.
+      for (int i = max(0, issued - kScanStages); i < issued; ++i)
+        mbar_wait(&full[i % kScanStages], (i / kScanStages) & 1, status);
+    }
+    return;
+  }
+
+  // ---- consumers ------------------------------------------------------------
+  const int sub = lane % C::kLpk;  // which 16-byte slice of the row
+  int cur_bh = -1;
+  float qs[C::kEpl];
+  for (int i = 0; i < ntiles; ++i) {
+    const int s = i % kScanStages;
+    const long long t = t_begin + i;
+    const int bh = (int)(t / tiles_per_head);
+    const int j0 = (int)(t % tiles_per_head) * C::kStageKeys;
+    const int nk = min(C::kStageKeys, N - j0);
+    if (bh != cur_bh) {
+      cur_bh = bh;
+      const int b = bh / Hkv, h = bh % Hkv, G = Hq / Hkv;
+#pragma unroll
+      for (int e = 0; e < C::kEpl; ++e) qs[e] = 0.f;
+      for (int g = 0; g < G; ++g) {
+        const T *qp = q + ((size_t)b * Hq + (size_t)h * G + g) * D + sub * C::kEpl;
+#pragma unroll
+        for (int e = 0; e < C::kEpl; ++e) qs[e] += DT<T>::to_f(qp[e]);
+      }
+#pragma unroll
+      for (int e = 0; e < C::kEpl; ++e) qs[e] *= scale;
+    }
+    if (!mbar_wait(&full[s], (i / kScanStages) & 1, status)) break;
+    const unsigned char *stage = ring + (size_t)s * kScanStageBytes;
+    float *Srow = o.S + (size_t)bh * N + j0;
+    const int slot = bh - bh_first;
+    uint32_t *krow = (o.keys && slot == 0) ? o.keys + o.key_off + j0 : nullptr;
+    for (int wt = warp; wt < C::kWarpTiles; wt += kScanConsumerWarps) {
+      const int key0 = wt * 32;
+      if (key0 >= nk) break;
+      const unsigned char *base = stage + (size_t)key0 * C::kRowBytes + lane * 16;
+      float v[C::kLpk];
+#pragma unroll
+      for (int r = 0; r < C::kLpk; ++r) {
+        float f[C::kEpl];
+        unpack16<T>(lds128(base + r * 512), f);
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < C::kEpl; ++e) acc = fmaf(qs[e], f[e], acc);
+        v[r] = acc;
+      }
+      TReduce<C::kLpk, C::kLpk / 2>::run(v, lane);
+      const int kk = key0 + sub * C::kKpr + lane / C::kLpk;
+      const bool valid = kk < nk;
+      if (valid) {
+        Srow[kk] = v[0];
+        const uint32_t key = order_key(v[0]);
+        if (krow) krow[kk] = key;
+        if (o.hist) {
+          const uint32_t bin = key >> 21;
+          if (slot < kSlots)
+            atomicAdd(&o.shist[slot * kScanBins + bin], 1u);
+          else
+            atomicAdd(&o.hist[(size_t)bh * kScanBins + bin], 1u);
+        }
+      }
+      if (__any_sync(0xffffffffu, valid && !isfinite(v[0])) && lane == 0)
+        raise_flag(status, FLAG_NONFINITE);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+}
+
+}  // namespace
+}  // namespace sd
