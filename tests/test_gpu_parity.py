@@ -451,3 +451,25 @@ def test_fused_route_equals_scan_then_select(dev, monkeypatch, B, N, Hkv, k):
     np.testing.assert_array_equal(a, b)
     S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
     assert_topk_within_band(a, S, k)
+
+
+@pytest.mark.parametrize("B,N,Hkv,hot", [(1, 65536, 1, 4096), (2, 131072, 2, 20000)])
+def test_fused_route_concentrated_top_k(dev, monkeypatch, B, N, Hkv, hot):
+    """Most of the top k lies in the first `hot` keys of each head, far more
+    than any CTA's proportional share: the fused kernel's local threshold
+    estimate is too high there and its second (histogram) round must give
+    the same exact sets as the two-kernel path."""
+    k = 2048
+    w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=1, k=k, dtype="bf16", seed=hot)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    K = t["K"].clone()
+    K[:, :, :hot] *= 4
+    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "1")
+    a = sd.route_topk(t["q_route"], K, k).cpu().numpy()
+    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "0")
+    b = sd.route_topk(t["q_route"], K, k).cpu().numpy()
+    np.testing.assert_array_equal(a, b)
+    S = oracle.scores(_f(x["q_route"]), _f(K.cpu()))
+    assert_topk_within_band(a, S, k)
+    assert (a < hot).mean() > 0.3   # far above the hot keys' proportional share
