@@ -71,6 +71,8 @@ def _load():
                 "oracle_attn": [I, I, I, I, I, I, P, P, P, P, I, P, P, P],
                 "oracle_decode_step": [I, I, I, I, I, I, P, P, P, P, I, P, I,
                                        P, P, P, P, P],
+                "oracle_decode_step_grouped": [I, I, I, I, I, I, I, P, P, P, P, I, P,
+                                               I, P, P, P, P, P],
                 "oracle_num_threads": [],
             }
             for name, argtypes in sigs.items():
@@ -210,4 +212,36 @@ def decode_step(q_route, q_layers, K, V, k: int | None = None, tau=None,
                                     _p(q_layers), _p(K), _p(V), kk, tau_p, capv,
                                     _p(S), _p(idx), _p(count), _p(out), _p(lse))
     _check(rc, "decode_step")
+    return {"S": S, "idx": idx, "count": count, "out": out, "lse": lse}
+
+
+def decode_step_grouped(q_routes, q_layers, K, V, R: int, k: int | None = None,
+                        tau=None, cap: int | None = None):
+    """Decode step re-routing every R layers (``oracle_decode_step_grouped``).
+
+    q_routes [ngroups,B,Hq,d] with ngroups = ceil(L/R); tau [ngroups,B,Hkv]
+    in threshold mode.  Returns dict(S [ngroups,B,Hkv,N], idx [ngroups,B,Hkv,
+    stride], count [ngroups,B,Hkv], out [L,B,Hq,d], lse [L,B,Hq])."""
+    q_routes, q_layers, K, V = _f32(q_routes), _f32(q_layers), _f32(K), _f32(V)
+    L, B, Hq, d = q_layers.shape
+    _, Hkv, N, _ = K.shape
+    ng = (L + R - 1) // R
+    if q_routes.shape != (ng, B, Hq, d):
+        raise OracleError("decode_step_grouped: q_routes must be [ceil(L/R),B,Hq,d]")
+    if k is not None:
+        stride, kk, tau_p, capv = int(k), int(k), None, 0
+    else:
+        if tau is None or cap is None:
+            raise OracleError("decode_step_grouped: give k, or tau and cap")
+        tau = _f32(tau).reshape(ng * B * Hkv)
+        stride, kk, tau_p, capv = int(cap), 0, _p(tau), int(cap)
+    S = np.empty((ng, B, Hkv, N), np.float32)
+    idx = np.full((ng, B, Hkv, stride), -1, np.int32)
+    count = np.full((ng, B, Hkv), stride, np.int32)
+    out = np.empty((L, B, Hq, d), np.float64)
+    lse = np.empty((L, B, Hq), np.float64)
+    rc = _load().oracle_decode_step_grouped(L, int(R), B, Hq, Hkv, d, N, _p(q_routes),
+                                            _p(q_layers), _p(K), _p(V), kk, tau_p, capv,
+                                            _p(S), _p(idx), _p(count), _p(out), _p(lse))
+    _check(rc, "decode_step_grouped")
     return {"S": S, "idx": idx, "count": count, "out": out, "lse": lse}

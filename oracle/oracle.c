@@ -305,6 +305,37 @@ int oracle_decode_step(int L, int B, int Hq, int Hkv, int d, int N,
   return st;
 }
 
+/* Decode step with the routing set recomputed every R layers.  CLSA article,
+ * section 計算コストの削減効果: per-layer routing (DSA) scores the context once
+ * per layer, CLSA once per step; section 推論速度の改善結果: IndexCache shares
+ * an index set across only some layers.  Reading: the L layers form groups
+ * of R consecutive layers (the last group may be shorter); group g routes
+ * with its own query q_routes[g] and its layers attend over that group's set.
+ * R >= L is the shared-routing step above, R = 1 per-layer routing.
+ * Layouts: q_routes [ngroups,B,Hq,d], tau [ngroups,B,Hkv] (threshold mode),
+ * S [ngroups,B,Hkv,N], idx [ngroups,B,Hkv,stride], count [ngroups,B,Hkv],
+ * out [L,B,Hq,d], lse [L,B,Hq]; ngroups = ceil(L/R). */
+int oracle_decode_step_grouped(int L, int R, int B, int Hq, int Hkv, int d, int N,
+                               const float *q_routes, const float *q_layers,
+                               const float *K, const float *V, int k, const float *tau,
+                               int cap, float *S, int *idx, int *count, double *out,
+                               double *lse) {
+  if (L < 1 || R < 1) return ORACLE_BAD_ARG;
+  const int stride = k > 0 ? k : cap;
+  const int ngroups = (L + R - 1) / R;
+  for (int g = 0; g < ngroups; ++g) {
+    const int l0 = g * R, lg = (L - l0) < R ? (L - l0) : R;
+    const int st = oracle_decode_step(
+        lg, B, Hq, Hkv, d, N, q_routes + (size_t)g * B * Hq * d,
+        q_layers + (size_t)l0 * B * Hq * d, K, V, k,
+        tau ? tau + (size_t)g * B * Hkv : NULL, cap, S + (size_t)g * B * Hkv * N,
+        idx + (size_t)g * B * Hkv * stride, count + (size_t)g * B * Hkv,
+        out + (size_t)l0 * B * Hq * d, lse + (size_t)l0 * B * Hq);
+    if (st != ORACLE_OK) return st;
+  }
+  return ORACLE_OK;
+}
+
 #ifdef _OPENMP
 #include <omp.h>
 #endif

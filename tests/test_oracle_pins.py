@@ -352,3 +352,67 @@ def test_decode_step_routes_once_and_shares_the_set():
     tau = oracle.percentile_tau(res["S"], 90, 100)
     th = oracle.decode_step(qr, ql, K, V, tau=tau, cap=N)
     assert th["count"].tolist() == [[71, 71]]
+
+
+# --------------------------------------------------------------------------
+# Routing recomputed every R layers (CLSA article, sections 計算コストの削減効果
+# and 推論速度の改善結果: per-layer routing vs one shared set vs sharing across
+# a few layers)
+# --------------------------------------------------------------------------
+
+def test_grouped_step_per_layer_routing_vs_library():
+    """R = 1: every layer routes with its own query.  Integer inputs make the
+    scores exact, so each layer's set equals a stable argsort of the fp64
+    library scores, and each layer's output equals dense attention over the
+    gathered rows."""
+    r = _rng(41)
+    B, N, Hq, Hkv, d, L, k = 2, 90, 8, 2, 16, 3, 7
+    G = Hq // Hkv
+    qrs = r.integers(-3, 4, (L, B, Hq, d)).astype(np.float32)
+    ql = r.standard_normal((L, B, Hq, d), dtype=np.float32)
+    K = r.integers(-3, 4, (B, Hkv, N, d)).astype(np.float32)
+    V = r.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    res = oracle.decode_step_grouped(qrs, ql, K, V, 1, k=k)
+    for layer in range(L):
+        qsum = qrs[layer].astype(np.float64).reshape(B, Hkv, G, d).sum(2)
+        S64 = np.einsum("bhd,bhnd->bhn", qsum, K.astype(np.float64)) / math.sqrt(d)
+        for b in range(B):
+            for h in range(Hkv):
+                ref = np.sort(np.argsort(-S64[b, h], kind="stable")[:k])
+                np.testing.assert_array_equal(res["idx"][layer, b, h], ref)
+        Kg = np.take_along_axis(K, res["idx"][layer][..., None].astype(np.int64), axis=2)
+        Vg = np.take_along_axis(V, res["idx"][layer][..., None].astype(np.int64), axis=2)
+        o_ref, lse_ref = _sdpa_f64(ql[layer], Kg, Vg)
+        np.testing.assert_allclose(res["out"][layer], o_ref, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(res["lse"][layer], lse_ref, atol=1e-12)
+
+
+def test_grouped_step_group_boundaries_and_invariants():
+    """Groups are R consecutive layers, the last one shorter when R does not
+    divide L; R >= L is the shared-routing step; equal routing queries give
+    equal sets in every group; threshold mode counts per group."""
+    r = _rng(43)
+    B, N, Hq, Hkv, d, L, k = 1, 300, 8, 2, 32, 5, 20
+    ql = r.standard_normal((L, B, Hq, d), dtype=np.float32)
+    K = r.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    V = r.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    qrs = r.standard_normal((3, B, Hq, d), dtype=np.float32)
+    res = oracle.decode_step_grouped(qrs, ql, K, V, 2, k=k)       # layers {0,1} {2,3} {4}
+    for g, layers in enumerate([[0, 1], [2, 3], [4]]):
+        one = oracle.decode_step(qrs[g], ql[layers], K, V, k=k)
+        np.testing.assert_array_equal(res["idx"][g], one["idx"])
+        np.testing.assert_array_equal(res["out"][layers], one["out"])
+    assert not np.array_equal(res["idx"][0], res["idx"][1])   # distinct queries route apart
+    shared = oracle.decode_step_grouped(qrs[:1], ql, K, V, L, k=k)
+    ref = oracle.decode_step(qrs[0], ql, K, V, k=k)
+    np.testing.assert_array_equal(shared["idx"][0], ref["idx"])
+    np.testing.assert_array_equal(shared["out"], ref["out"])
+    same = oracle.decode_step_grouped(np.repeat(qrs[:1], 3, 0), ql, K, V, 2, k=k)
+    for g in range(3):
+        np.testing.assert_array_equal(same["idx"][g], ref["idx"])
+    np.testing.assert_allclose(same["out"], ref["out"], rtol=0, atol=0)
+    tau = np.stack([oracle.percentile_tau(res["S"][g], 95, 100) for g in range(3)])
+    th = oracle.decode_step_grouped(qrs, ql, K, V, 2, tau=tau, cap=N)
+    for g in range(3):
+        S = oracle.scores(qrs[g], K)
+        np.testing.assert_array_equal(th["count"][g], (S >= tau[g][..., None]).sum(-1))
