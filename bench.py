@@ -218,13 +218,15 @@ def capture_loop(fn_list, stream):
     return g
 
 
-def kernels_per_step(w) -> int:
+def kernels_per_step(w, reroute: int = 0) -> int:
     """Kernels one decode step launches: the routing scan and the select (one
     fused kernel when SPARSE_DECODE_FUSED_ROUTE=1 applies), then the
-    attention (one kernel for bf16, a partial and a merge kernel for fp32)."""
+    attention (one kernel for bf16, a partial and a merge kernel for fp32);
+    once per group of `reroute` layers when routing is re-computed."""
     route = 1 if os.environ.get("SPARSE_DECODE_FUSED_ROUTE") == "1" and w.mode == "topk" else 2
     attn = 1 if w.dtype == "bf16" else 2
-    return route + attn
+    groups = -(-w.L // reroute) if reroute else 1
+    return (route + attn) * groups
 
 
 def capture(fn_list, stream):
@@ -285,9 +287,22 @@ def run_native(args, rank, world, local_rank):
     outs = [dict(out=torch.empty_like(ql), idx=torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device=dev),
                  lse=torch.empty((w.L, w.B, w.Hq), dtype=torch.float32, device=dev)) for _, ql in qs]
 
+    R = args.reroute
+    if R:
+        # routing re-computed every R layers: group g routes with the query
+        # of its first layer (R = 1: every layer routes with its own query)
+        ng = -(-w.L // R)
+        qrs = [ql[::R].contiguous() for _, ql in qs]
+        ws.get(sd.workspace_bytes(w.B, w.N, w.Hq, w.Hkv, w.d, w.torch_dtype, w.k, min(R, w.L)))
+        for o in outs:
+            o["idx"] = torch.empty((ng, w.B, w.Hkv, w.k), dtype=torch.int32, device=dev)
+
     def step_fn(i):
         qr, ql = qs[i]
         o = outs[i]
+        if R:
+            return lambda: sd.decode_step_grouped(qrs[i], ql, K, V, R, k=w.k, ws=ws, check=False,
+                                                  out=o["out"], idx=o["idx"], lse=o["lse"])
         return lambda: sd.decode_step(qr, ql, K, V, k=w.k, ws=ws, check=False,
                                       out=o["out"], idx=o["idx"], lse=o["lse"])
 
@@ -305,10 +320,13 @@ def run_native(args, rank, world, local_rank):
         # per-kernel durations, each kernel alone in a graph of back-to-back
         # launches over the rotating queries (CUDA events on this stream)
         S_buf = torch.empty((w.B, w.Hkv, w.N), dtype=torch.float32, device=dev)
-        idx0 = outs[0]["idx"]
+        # one routing set per query set (computed here, outside any graph)
+        sets = [torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device=dev) for _ in qs]
+        idx0 = sets[0]
         # size the workspace for every op before any capture
         sd.score(qs[0][0], K, ws=ws, check=False, out=S_buf)
-        sd.route_topk(qs[0][0], K, w.k, ws=ws, check=False, idx=idx0)
+        for qi in range(len(qs)):
+            sd.route_topk(qs[qi][0], K, w.k, ws=ws, check=False, idx=sets[qi])
         sd.attn_gather(qs[0][1], K, V, idx0, ws=ws, check=False, out=outs[0]["out"],
                        lse=outs[0]["lse"])
         torch.cuda.synchronize()
@@ -321,7 +339,7 @@ def run_native(args, rank, world, local_rank):
         route_graphs = capture([lambda qr=qr: sd.route_topk(qr, K, w.k, ws=ws, check=False, idx=idx0)
                                 for qr, _ in qs], stream)
         t_sel = time_graphs(route_graphs, n_k, max(args.warmup, 3), stream) / n_k - t_score
-        attn_graphs = capture([lambda qi=qi: sd.attn_gather(qs[qi][1], K, V, outs[qi]["idx"], ws=ws,
+        attn_graphs = capture([lambda qi=qi: sd.attn_gather(qs[qi][1], K, V, sets[qi], ws=ws,
                                                             check=False, out=outs[qi]["out"],
                                                             lse=outs[qi]["lse"])
                                for qi in range(len(qs))], stream)
@@ -364,7 +382,10 @@ def run_native(args, rank, world, local_rank):
                       "(query set i at step i; %d kernels per step, programmatic "
                       "dependent launch between them), single-step graphs for a "
                       "remainder; CUDA events on the launch stream; max over ranks"
-                      % (QUERY_SETS, kernels_per_step(w)),
+                      % (QUERY_SETS, kernels_per_step(w, args.reroute)),
+            **({"reroute": args.reroute,
+                "routing": "re-computed every %d layers (group g routes with its first "
+                           "layer's query)" % args.reroute} if args.reroute else {}),
         },
         "roofline": {
             "bound": "hbm", "kernel": "score_kernel (routing scan)",
@@ -386,7 +407,7 @@ def run_native(args, rank, world, local_rank):
                                "launches (attention alone may find its rows in L2); select "
                                "= route (score + select) minus score"},
         "e2e": e2e,
-        "gpu_launches": kernels_per_step(w) * args.steps,
+        "gpu_launches": kernels_per_step(w, args.reroute) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -518,6 +539,9 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="decode_128k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reroute", type=int, default=0,
+                    help="re-route every R layers (1: per-layer routing); default: route "
+                         "once per step, the method's shared routing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

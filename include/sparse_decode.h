@@ -194,6 +194,30 @@ sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
                                    float *lse, void *ws, size_t ws_bytes,
                                    void *stream);
 
+/* Decode step that re-routes every R layers (CLSA article, section
+ * 計算コストの削減効果: token-sparse attention with per-layer routing (DSA)
+ * scores the context once per layer, CLSA once per step; section
+ * 推論速度の改善結果: IndexCache shares an index set across only some layers).
+ * The L layers form ngroups = ceil(L/R) groups of R consecutive layers (the
+ * last one shorter when R does not divide L); group g routes with its own
+ * query q_routes[g] and its layers attend over that group's set.  R >= L is
+ * sparse_decode_step (one shared set); R = 1 is per-layer routing.
+ *   q_routes [ngroups,B,Hq,d]; q_layers [L,B,Hq,d]; out [L,B,Hq,d];
+ *   lse [L,B,Hq] or NULL;
+ *   top-k mode:     k >= 1, tau == NULL; idx [ngroups,B,Hkv,k];
+ *   threshold mode: k == 0, tau [ngroups,B,Hkv], count [ngroups,B,Hkv],
+ *                   cap >= 1; idx [ngroups,B,Hkv,cap].
+ * The workspace is sized for the layers of one group: ws_bytes >=
+ * sparse_workspace_size(shape, k or cap, min(R, L)).  The groups run one after
+ * another on `stream`, reusing the workspace. */
+sparse_status_t sparse_decode_step_grouped(const sparse_shape_t *shape, int32_t L,
+                                           int32_t R, const void *q_routes,
+                                           const void *q_layers, const void *K,
+                                           const void *V, int32_t k, const float *tau,
+                                           int32_t cap, int32_t *idx, int32_t *count,
+                                           void *out, float *lse, void *ws,
+                                           size_t ws_bytes, void *stream);
+
 /* Shared routing, top-k form (as sparse_route_topk) for callers that cannot
  * allocate device memory: a plugin inside a host framework that owns every
  * device allocation, or code that must not call cudaMalloc once it is

@@ -473,3 +473,75 @@ def test_fused_route_concentrated_top_k(dev, monkeypatch, B, N, Hkv, hot):
     S = oracle.scores(_f(x["q_route"]), _f(K.cpu()))
     assert_topk_within_band(a, S, k)
     assert (a < hot).mean() > 0.3   # far above the hot keys' proportional share
+
+
+# ---------------------------------------------------------------------------
+# Routing recomputed every R layers (per-layer routing at R = 1, partial
+# sharing in between, shared routing at R >= L)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("L,R", [(7, 3), (16, 1), (16, 4), (4, 9)])
+def test_decode_step_grouped_topk(dev, L, R):
+    """Every group's set matches the oracle's top-k of that group's routing
+    scores (within the rounding band) and equals the routing call on that
+    query bitwise; every layer's output equals the gather call on its group's
+    set and matches the oracle on the oracle's sets."""
+    w = synth.custom(B=1, N=6000, Hq=16, Hkv=4, d=128, L=L, k=300, dtype="bf16", seed=10 * L + R)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    ng = -(-L // R)
+    g = torch.Generator().manual_seed(R)
+    qrs = torch.randn((ng, w.B, w.Hq, w.d), generator=g).to(torch.bfloat16)
+    qrs_d = qrs.to(dev)
+    res = sd.decode_step_grouped(qrs_d, t["q_layers"], t["K"], t["V"], R, k=w.k)
+    ref = oracle.decode_step_grouped(_f(qrs), _f(x["q_layers"]), _f(x["K"]), _f(x["V"]), R,
+                                     k=w.k)
+    gidx = res["idx"].cpu().numpy()
+    for grp in range(ng):
+        layers = list(range(grp * R, min(L, (grp + 1) * R)))
+        assert_topk_within_band(gidx[grp], ref["S"][grp], w.k)
+        np.testing.assert_array_equal(
+            gidx[grp], sd.route_topk(qrs_d[grp], t["K"], w.k).cpu().numpy())
+        out2, lse2 = sd.attn_gather(t["q_layers"][layers].contiguous(), t["K"], t["V"],
+                                    res["idx"][grp].contiguous())
+        assert torch.equal(out2, res["out"][layers]) and torch.equal(lse2, res["lse"][layers])
+    o_gpu = torch.empty_like(res["out"])
+    l_gpu = torch.empty_like(res["lse"])
+    for grp in range(ng):
+        layers = list(range(grp * R, min(L, (grp + 1) * R)))
+        o, l = sd.attn_gather(t["q_layers"][layers].contiguous(), t["K"], t["V"],
+                              torch.from_numpy(ref["idx"][grp]).to(dev))
+        o_gpu[layers], l_gpu[layers] = o, l
+    assert_attn_close(o_gpu, l_gpu, ref["out"], ref["lse"], "bf16")
+
+
+def test_decode_step_grouped_threshold(dev):
+    """Threshold mode: each group keeps every key at or above its own tau
+    (no false negatives against fp64 scores) and each layer attends over its
+    group's set."""
+    L, R = 5, 2
+    w = synth.custom(B=1, N=8000, Hq=8, Hkv=2, d=128, L=L, k=1, dtype="bf16", seed=5)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    ng = -(-L // R)
+    g = torch.Generator().manual_seed(99)
+    qrs = torch.randn((ng, w.B, w.Hq, w.d), generator=g).to(torch.bfloat16)
+    S = np.stack([oracle.scores(_f(qrs[i]), _f(x["K"])) for i in range(ng)])
+    S64 = np.stack([oracle.scores(_f(qrs[i]), _f(x["K"]), np.float64) for i in range(ng)])
+    tau = np.stack([oracle.percentile_tau(S[i], 97, 100) for i in range(ng)])
+    cap = 512
+    res = sd.decode_step_grouped(qrs.to(dev), t["q_layers"], t["K"], t["V"], R,
+                                 tau=torch.from_numpy(tau).to(dev), cap=cap)
+    gidx, gcnt = res["idx"].cpu().numpy(), res["count"].cpu().numpy()
+    for grp in range(ng):
+        for h in range(w.Hkv):
+            band = _band(tau[grp, 0, h])
+            got = set(gidx[grp, 0, h, :gcnt[grp, 0, h]].tolist())
+            must = set(np.nonzero(S64[grp, 0, h] >= tau[grp, 0, h] + band)[0].tolist())
+            never = set(np.nonzero(S64[grp, 0, h] < tau[grp, 0, h] - band)[0].tolist())
+            assert must <= got and not (got & never)
+        layers = list(range(grp * R, min(L, (grp + 1) * R)))
+        out2, lse2 = sd.attn_gather(t["q_layers"][layers].contiguous(), t["K"], t["V"],
+                                    res["idx"][grp].contiguous(),
+                                    count=res["count"][grp].contiguous())
+        assert torch.equal(out2, res["out"][layers]) and torch.equal(lse2, res["lse"][layers])

@@ -25,7 +25,7 @@ import torch
 __all__ = ["SparseDecodeError", "lib_path", "load", "score", "select_topk",
            "select_threshold", "route_topk", "route_threshold", "attn_gather",
            "decode_step", "read_device_status", "workspace_bytes",
-           "Workspace", "STATUS_NAMES", "EXPORTED_SYMBOLS"]
+           "Workspace", "STATUS_NAMES", "EXPORTED_SYMBOLS", "decode_step_grouped"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_PKG, "libsparse_decode.so")
@@ -42,7 +42,7 @@ EXPORTED_SYMBOLS = (
     "sparse_workspace_init", "sparse_score", "sparse_select_topk",
     "sparse_select_threshold", "sparse_route_topk", "sparse_route_threshold",
     "sparse_attn_gather", "sparse_decode_step", "sparse_read_device_status",
-    "sparse_route_topk_static",
+    "sparse_route_topk_static", "sparse_decode_step_grouped",
 )
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
@@ -97,6 +97,8 @@ def load():
                                          P, P, P, SZ, P]),
             "sparse_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
             "sparse_route_topk_static": (I32, [SH, P, P, I32, P, P]),
+            "sparse_decode_step_grouped": (I32, [SH, I32, I32, P, P, P, P, I32, P, I32,
+                                                 P, P, P, P, P, SZ, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -355,6 +357,54 @@ def decode_step(q_route, q_layers, K, V, k: int | None = None, tau=None,
         int(k) if topk else 0, _ptr(tau_t), 0 if topk else int(cap), _ptr(idx),
         _ptr(count), _ptr(out), _ptr(lse), _ptr(buf), buf.numel(), _stream()),
         "decode_step")
+    if check:
+        read_device_status(w)
+    return {"idx": idx, "count": count, "out": out, "lse": lse}
+
+
+def decode_step_grouped(q_routes, q_layers, K, V, R: int, k: int | None = None, tau=None,
+                        cap: int | None = None, ws: Workspace | None = None,
+                        check: bool = True, out=None, idx=None, count=None, lse=None,
+                        return_lse: bool = True):
+    """Decode step re-routing every R layers (sparse_decode_step_grouped).
+
+    q_routes [ceil(L/R),B,Hq,d]: group g of R consecutive layers routes with
+    q_routes[g].  Top-k mode with ``k``; threshold mode with ``tau``
+    [ceil(L/R),B,Hkv] and ``cap``.  Returns dict(idx [ngroups,B,Hkv,stride],
+    count, out [L,B,Hq,d], lse [L,B,Hq])."""
+    _need_cuda(q_routes, q_layers, K, V, tau)
+    if q_routes.dim() != 4 or K.dim() != 4:
+        raise ValueError("q_routes must be [ngroups,B,Hq,d] and K [B,Hkv,N,d]")
+    B, N, Hq, Hkv, d = _dims_qk(q_routes[0], K)
+    L = q_layers.shape[0]
+    R = int(R)
+    if R < 1:
+        raise ValueError("R must be >= 1")
+    ng = (L + R - 1) // R
+    if q_routes.shape[0] != ng or q_layers.shape != (L, B, Hq, d) or V.shape != K.shape:
+        raise ValueError("q_routes must be [ceil(L/R),B,Hq,d], q_layers [L,B,Hq,d], V like K")
+    topk = k is not None
+    if topk == (tau is not None):
+        raise ValueError("give exactly one of k or tau")
+    stride = int(k) if topk else int(cap)
+    dev = q_routes.device
+    w = _ws(ws, dev)
+    sh = _shape(B, N, Hq, Hkv, d, q_routes.dtype)
+    buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q_routes.dtype, stride, min(R, L)))
+    if idx is None:
+        idx = torch.empty((ng, B, Hkv, stride), dtype=torch.int32, device=dev)
+    if count is None and not topk:
+        count = torch.empty((ng, B, Hkv), dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty_like(q_layers)
+    if lse is None and return_lse:
+        lse = torch.empty((L, B, Hq), dtype=torch.float32, device=dev)
+    tau_t = None if topk else tau.float().contiguous()
+    _check(load().sparse_decode_step_grouped(
+        ctypes.byref(sh), L, R, _ptr(q_routes), _ptr(q_layers), _ptr(K), _ptr(V),
+        int(k) if topk else 0, _ptr(tau_t), 0 if topk else int(cap), _ptr(idx),
+        _ptr(count), _ptr(out), _ptr(lse), _ptr(buf), buf.numel(), _stream()),
+        "decode_step_grouped")
     if check:
         read_device_status(w)
     return {"idx": idx, "count": count, "out": out, "lse": lse}

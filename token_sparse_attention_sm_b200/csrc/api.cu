@@ -172,6 +172,51 @@ cudaError_t device_info(DeviceInfo *out) {
   return g_info_err[dev];
 }
 
+// Checks shared by the decode-step entry points (L layers per routing set).
+sparse_status_t check_decode_args(const Shape &s, int32_t L, const void *q_route,
+                                  const void *q_layers, const void *K, const void *V,
+                                  int32_t k, const float *tau, int32_t cap, int32_t *idx,
+                                  int32_t *count, void *out, float *lse) {
+  if (L < 1 || !q_route || !q_layers || !K || !V || !idx || !out)
+    return SPARSE_ERR_INVALID_ARG;
+  if ((long long)L * s.G() > 1024) return SPARSE_ERR_UNSUPPORTED;
+  if (k > 0) {
+    if (k > s.N || tau) return SPARSE_ERR_INVALID_ARG;
+  } else {
+    if (k < 0 || !tau || !count || cap < 1) return SPARSE_ERR_INVALID_ARG;
+  }
+  if (!aligned(q_route, 16) || !aligned(q_layers, 16) || !aligned(K, 16) ||
+      !aligned(V, 16) || !aligned(out, 16) || !aligned(idx, 4) ||
+      (count && !aligned(count, 4)) || (tau && !aligned(tau, 4)) ||
+      (lse && !aligned(lse, 4)))
+    return SPARSE_ERR_INVALID_ARG;
+  return SPARSE_OK;
+}
+
+// Route once with q_route, then attend L layers over that set (arguments
+// checked by the caller; the workspace layout l fits L layers).
+cudaError_t decode_step_enqueue(const Shape &s, int L, const void *q_route,
+                                const void *q_layers, const void *K, const void *V, int k,
+                                const float *tau, int cap, int *idx, int *count, void *out,
+                                float *lse, void *ws, const Layout &l, cudaStream_t st) {
+  const bool topk = k > 0;
+  const int stride = topk ? k : cap;
+  uint32_t *status = status_word(ws);
+  cudaError_t e;
+  if (topk) {
+    e = route_topk_any(s, q_route, K, k, idx, ws, l, st);
+  } else {
+    float *S = scores_ptr(ws, l);
+    e = launch_score(s, q_route, K, S, nullptr, status, st);
+    if (e == cudaSuccess)
+      e = launch_select(s, S, 0, tau, cap, idx, count, cap, nullptr, status, st);
+  }
+  if (e == cudaSuccess)
+    e = launch_attn(s, L, q_layers, K, V, idx, stride, topk ? nullptr : count, stride, out,
+                    lse, attn_ptr(ws, l), attn_counters(ws), status, st);
+  return e;
+}
+
 }  // namespace sd
 
 using sd::Shape;
@@ -332,38 +377,47 @@ sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
   Shape s;
   sparse_status_t r = sd::check_shape(shape, &s);
   if (r != SPARSE_OK) return r;
-  if (L < 1 || !q_route || !q_layers || !K || !V || !idx || !out)
-    return SPARSE_ERR_INVALID_ARG;
-  if ((long long)L * s.G() > 1024) return SPARSE_ERR_UNSUPPORTED;
-  const bool topk = k > 0;
-  if (topk) {
-    if (k > s.N || tau) return SPARSE_ERR_INVALID_ARG;
-  } else {
-    if (k < 0 || !tau || !count || cap < 1) return SPARSE_ERR_INVALID_ARG;
-  }
-  if (!sd::aligned(q_route, 16) || !sd::aligned(q_layers, 16) ||
-      !sd::aligned(K, 16) || !sd::aligned(V, 16) || !sd::aligned(out, 16) ||
-      !sd::aligned(idx, 4) || (count && !sd::aligned(count, 4)) ||
-      (tau && !sd::aligned(tau, 4)) || (lse && !sd::aligned(lse, 4)))
-    return SPARSE_ERR_INVALID_ARG;
-  const int stride = topk ? k : cap;
+  if ((r = sd::check_decode_args(s, L, q_route, q_layers, K, V, k, tau, cap, idx, count, out,
+                                 lse)) != SPARSE_OK)
+    return r;
+  const int stride = k > 0 ? k : cap;
   if ((r = sd::check_ws(s, stride, L, ws, ws_bytes)) != SPARSE_OK) return r;
-  const sd::Layout l = sd::layout(s, stride, L);
+  return sd::from_cuda(sd::decode_step_enqueue(s, L, q_route, q_layers, K, V, k, tau, cap, idx,
+                                               count, out, lse, ws, sd::layout(s, stride, L),
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+sparse_status_t sparse_decode_step_grouped(const sparse_shape_t *shape, int32_t L, int32_t R,
+                                           const void *q_routes, const void *q_layers,
+                                           const void *K, const void *V, int32_t k,
+                                           const float *tau, int32_t cap, int32_t *idx,
+                                           int32_t *count, void *out, float *lse, void *ws,
+                                           size_t ws_bytes, void *stream) {
+  Shape s;
+  sparse_status_t r = sd::check_shape(shape, &s);
+  if (r != SPARSE_OK) return r;
+  if (R < 1) return SPARSE_ERR_INVALID_ARG;
+  const int Lg = R < L ? R : L;  // layers per routing group
+  if ((r = sd::check_decode_args(s, Lg, q_routes, q_layers, K, V, k, tau, cap, idx, count, out,
+                                 lse)) != SPARSE_OK)
+    return r;
+  if (L < 1) return SPARSE_ERR_INVALID_ARG;
+  const int stride = k > 0 ? k : cap;
+  if ((r = sd::check_ws(s, stride, Lg, ws, ws_bytes)) != SPARSE_OK) return r;
+  const sd::Layout l = sd::layout(s, stride, Lg);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t *status = sd::status_word(ws);
-  cudaError_t e;
-  if (topk) {
-    e = sd::route_topk_any(s, q_route, K, k, idx, ws, l, st);
-  } else {
-    float *S = sd::scores_ptr(ws, l);
-    e = sd::launch_score(s, q_route, K, S, nullptr, status, st);
-    if (e == cudaSuccess)
-      e = sd::launch_select(s, S, 0, tau, cap, idx, count, cap, nullptr, status, st);
+  const size_t qsz = (size_t)s.B * s.Hq * s.d * s.esize();  // one [B,Hq,d] query set
+  const int ngroups = (L + R - 1) / R;
+  cudaError_t e = cudaSuccess;
+  for (int g = 0; g < ngroups && e == cudaSuccess; ++g) {
+    const int l0 = g * R, lg = L - l0 < R ? L - l0 : R;
+    e = sd::decode_step_enqueue(
+        s, lg, static_cast<const char *>(q_routes) + g * qsz,
+        static_cast<const char *>(q_layers) + (size_t)l0 * qsz, K, V, k,
+        tau ? tau + (size_t)g * s.BH() : nullptr, cap, idx + (size_t)g * s.BH() * stride,
+        count ? count + (size_t)g * s.BH() : nullptr, static_cast<char *>(out) + (size_t)l0 * qsz,
+        lse ? lse + (size_t)l0 * s.B * s.Hq : nullptr, ws, l, st);
   }
-  if (e == cudaSuccess)
-    e = sd::launch_attn(s, L, q_layers, K, V, idx, stride, topk ? nullptr : count,
-                        stride, out, lse, sd::attn_ptr(ws, l), sd::attn_counters(ws), status,
-                        st);
   return sd::from_cuda(e);
 }
 
