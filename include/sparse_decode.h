@@ -101,11 +101,14 @@ typedef enum { SPARSE_DTYPE_F32 = 0, SPARSE_DTYPE_BF16 = 1 } sparse_dtype_t;
 
 typedef struct {
   int32_t B;     /* sequences */
-  int32_t N;     /* cached tokens per sequence */
+  int32_t N;     /* cached tokens per sequence (the current length) */
   int32_t Hq;    /* query heads */
   int32_t Hkv;   /* KV heads; Hq % Hkv == 0 */
   int32_t d;     /* head dimension */
   int32_t dtype; /* sparse_dtype_t of q, K, V and out */
+  int32_t n_cap; /* rows allocated per (sequence, KV head) in K and V: K and V
+                    are [B,Hkv,n_cap,d] and rows 0..N-1 are the cache; 0 means
+                    n_cap = N (a dense cache); otherwise n_cap >= N */
 } sparse_shape_t;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -217,6 +220,17 @@ sparse_status_t sparse_decode_step_grouped(const sparse_shape_t *shape, int32_t 
                                            int32_t cap, int32_t *idx, int32_t *count,
                                            void *out, float *lse, void *ws,
                                            size_t ws_bytes, void *stream);
+
+/* The self-decoder's cache write for one decode step (CLSA article, section
+ * CLSAの仕組み: the self-decoder generates the shared KV cache once; routing
+ * and every cross-decoder layer read it, the new token included): copies
+ * k_new[b,h,:] and v_new[b,h,:] ([B,Hkv,d], dtype of the cache, 16-byte
+ * aligned) into row N-1 of K and V ([B,Hkv,n_cap,d]) for every (b, h), where
+ * N = shape->N is the cache length counting the new token (N <= n_cap).  A
+ * model's step is then this call followed by sparse_decode_step with the same
+ * shape.  Hq is not used.  Asynchronous on `stream`; no workspace. */
+sparse_status_t sparse_kv_append(const sparse_shape_t *shape, void *K, void *V,
+                                 const void *k_new, const void *v_new, void *stream);
 
 /* Shared routing, top-k form (as sparse_route_topk) for callers that cannot
  * allocate device memory: a plugin inside a host framework that owns every

@@ -102,6 +102,19 @@ def test_bad_arguments_rejected_before_device_work(lib):
     assert lib.sparse_attn_gather(ctypes.byref(sh), 1, fake, fake, fake, fake, 0,
                                   None, fake, None, ws_ok, need, None) == 1
     assert lib.sparse_read_device_status(None, None, None) == 1
+    # cache capacity below the cache length
+    short = _shape(n_cap=100)
+    assert lib.sparse_route_topk(ctypes.byref(short), fake, fake, 16, fake, ws_ok,
+                                 1 << 30, None) == 1
+    assert lib.sparse_kv_append(ctypes.byref(short), fake, fake, fake, fake, None) == 1
+    # append: null or misaligned rows
+    assert lib.sparse_kv_append(ctypes.byref(sh), fake, fake, None, fake, None) == 1
+    assert lib.sparse_kv_append(ctypes.byref(sh), fake, fake, odd, fake, None) == 1
+    # grouped step: R < 1
+    rc, need = _ws_size(lib, sh, k=16, L=2)
+    assert lib.sparse_decode_step_grouped(ctypes.byref(sh), 4, 0, fake, fake, fake, fake, 16,
+                                          None, 0, fake, None, fake, None, ws_ok, need,
+                                          None) == 1
 
 
 def test_python_binding_refuses_cpu_tensors(lib):

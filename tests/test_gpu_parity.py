@@ -545,3 +545,43 @@ def test_decode_step_grouped_threshold(dev):
                                     res["idx"][grp].contiguous(),
                                     count=res["count"][grp].contiguous())
         assert torch.equal(out2, res["out"][layers]) and torch.equal(lse2, res["lse"][layers])
+
+
+# ---------------------------------------------------------------------------
+# Decode steps as a model runs them: append the new token's K/V row, then route
+# and attend over a cache whose allocation is longer than its length
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_kv_append_then_decode(dev, dtype, d):
+    """Three steps on a cache allocated for n_cap rows: each appends a row at
+    the current length and decodes over exactly the first n rows.  Rows past n
+    hold huge values that would dominate any score if read.  Results equal a
+    dense copy of the first n rows bitwise, and the oracle on that cache."""
+    B, n_cap, n0, Hq, Hkv, L, k = 1, 3000, 2500, 8, 2, 2, 100
+    w = synth.custom(B=B, N=n_cap, Hq=Hq, Hkv=Hkv, d=d, L=L, k=k, dtype=dtype, seed=d)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    K, V = t["K"].clone(), t["V"].clone()
+    K[:, :, n0:] = 100
+    V[:, :, n0:] = 100
+    g = torch.Generator().manual_seed(7)
+    for step in range(3):
+        n = n0 + 1 + step
+        k_new = torch.randn((B, Hkv, d), generator=g).to(K.dtype).to(dev)
+        v_new = torch.randn((B, Hkv, d), generator=g).to(K.dtype).to(dev)
+        sd.kv_append(K, V, k_new, v_new, n)
+        assert torch.equal(K[:, :, n - 1], k_new) and torch.equal(V[:, :, n - 1], v_new)
+        assert torch.all(K[:, :, n:] == 100)
+        res = sd.decode_step(t["q_route"], t["q_layers"], K, V, k=k, n=n)
+        Kd, Vd = K[:, :, :n].contiguous(), V[:, :, :n].contiguous()
+        dense = sd.decode_step(t["q_route"], t["q_layers"], Kd, Vd, k=k)
+        np.testing.assert_array_equal(res["idx"].cpu().numpy(), dense["idx"].cpu().numpy())
+        assert torch.equal(res["out"], dense["out"]) and torch.equal(res["lse"], dense["lse"])
+        Kh, Vh = _f(Kd.cpu()), _f(Vd.cpu())
+        S = oracle.scores(_f(x["q_route"]), Kh)
+        assert_topk_within_band(res["idx"].cpu().numpy(), S, k)
+        ridx = oracle.topk(S, k)
+        o_gpu, l_gpu = sd.attn_gather(t["q_layers"], K, V, torch.from_numpy(ridx).to(dev), n=n)
+        o_ref, l_ref = oracle.attn(_f(x["q_layers"]), Kh, Vh, ridx)
+        assert_attn_close(o_gpu, l_gpu, o_ref, l_ref, dtype)

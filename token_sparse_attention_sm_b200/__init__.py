@@ -25,7 +25,8 @@ import torch
 __all__ = ["SparseDecodeError", "lib_path", "load", "score", "select_topk",
            "select_threshold", "route_topk", "route_threshold", "attn_gather",
            "decode_step", "read_device_status", "workspace_bytes",
-           "Workspace", "STATUS_NAMES", "EXPORTED_SYMBOLS", "decode_step_grouped"]
+           "Workspace", "STATUS_NAMES", "EXPORTED_SYMBOLS", "decode_step_grouped",
+           "kv_append"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_PKG, "libsparse_decode.so")
@@ -42,7 +43,7 @@ EXPORTED_SYMBOLS = (
     "sparse_workspace_init", "sparse_score", "sparse_select_topk",
     "sparse_select_threshold", "sparse_route_topk", "sparse_route_threshold",
     "sparse_attn_gather", "sparse_decode_step", "sparse_read_device_status",
-    "sparse_route_topk_static", "sparse_decode_step_grouped",
+    "sparse_route_topk_static", "sparse_decode_step_grouped", "sparse_kv_append",
 )
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
@@ -57,7 +58,8 @@ class SparseDecodeError(RuntimeError):
 class _Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("N", ctypes.c_int32),
                 ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
-                ("d", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+                ("d", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("n_cap", ctypes.c_int32)]
 
 
 _lock = threading.Lock()
@@ -99,6 +101,7 @@ def load():
             "sparse_route_topk_static": (I32, [SH, P, P, I32, P, P]),
             "sparse_decode_step_grouped": (I32, [SH, I32, I32, P, P, P, P, I32, P, I32,
                                                  P, P, P, P, P, SZ, P]),
+            "sparse_kv_append": (I32, [SH, P, P, P, P, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -121,10 +124,20 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def _shape(B, N, Hq, Hkv, d, dtype) -> _Shape:
+def _shape(B, N, Hq, Hkv, d, dtype, n_cap: int = 0) -> _Shape:
     if dtype not in DTYPE_CODES:
         raise TypeError(f"unsupported dtype {dtype}")
-    return _Shape(B, N, Hq, Hkv, d, DTYPE_CODES[dtype])
+    return _Shape(B, N, Hq, Hkv, d, DTYPE_CODES[dtype], int(n_cap))
+
+
+def _length(n_cap: int, n: int | None) -> int:
+    """Cache length in use: n (1 <= n <= rows allocated) or all rows."""
+    if n is None:
+        return n_cap
+    n = int(n)
+    if not 1 <= n <= n_cap:
+        raise ValueError(f"cache length n={n} outside [1, {n_cap}]")
+    return n
 
 
 def _need_cuda(*ts):
@@ -195,12 +208,15 @@ def _dims_qk(q, K):
     return B, N, Hq, Hkv, d
 
 
-def score(q, K, ws: Workspace | None = None, check: bool = True, out=None):
-    """Routing scores S [B,Hkv,N] fp32 (written into ``out`` if given)."""
+def score(q, K, ws: Workspace | None = None, check: bool = True, out=None,
+          n: int | None = None):
+    """Routing scores S [B,Hkv,N] fp32 (written into ``out`` if given).  K may
+    hold more rows than the cache length n (default: all rows)."""
     _need_cuda(q, K, out)
-    B, N, Hq, Hkv, d = _dims_qk(q, K)
+    B, Ncap, Hq, Hkv, d = _dims_qk(q, K)
+    N = _length(Ncap, n)
     w = _ws(ws, q.device)
-    sh = _shape(B, N, Hq, Hkv, d, q.dtype)
+    sh = _shape(B, N, Hq, Hkv, d, q.dtype, Ncap)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, 1, 1))
     S = torch.empty((B, Hkv, N), dtype=torch.float32, device=q.device) if out is None else out
     _check(load().sparse_score(ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(S),
@@ -248,12 +264,14 @@ def select_threshold(S, tau, cap: int, ws: Workspace | None = None,
 
 
 def route_topk(q, K, k: int, ws: Workspace | None = None, check: bool = True,
-               idx=None):
-    """Shared routing (top-k): idx [B,Hkv,k] int32 ascending."""
+               idx=None, n: int | None = None):
+    """Shared routing (top-k): idx [B,Hkv,k] int32 ascending, over the first n
+    cache rows (default: all rows of K)."""
     _need_cuda(q, K, idx)
-    B, N, Hq, Hkv, d = _dims_qk(q, K)
+    B, Ncap, Hq, Hkv, d = _dims_qk(q, K)
+    N = _length(Ncap, n)
     w = _ws(ws, q.device)
-    sh = _shape(B, N, Hq, Hkv, d, q.dtype)
+    sh = _shape(B, N, Hq, Hkv, d, q.dtype, Ncap)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, k, 1))
     if idx is None:
         idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=q.device)
@@ -266,12 +284,14 @@ def route_topk(q, K, k: int, ws: Workspace | None = None, check: bool = True,
 
 
 def route_threshold(q, K, tau, cap: int, ws: Workspace | None = None,
-                    check: bool = True):
-    """Shared routing (threshold): (idx [B,Hkv,cap], count [B,Hkv])."""
+                    check: bool = True, n: int | None = None):
+    """Shared routing (threshold): (idx [B,Hkv,cap], count [B,Hkv]), over the
+    first n cache rows (default: all rows of K)."""
     _need_cuda(q, K, tau)
-    B, N, Hq, Hkv, d = _dims_qk(q, K)
+    B, Ncap, Hq, Hkv, d = _dims_qk(q, K)
+    N = _length(Ncap, n)
     w = _ws(ws, q.device)
-    sh = _shape(B, N, Hq, Hkv, d, q.dtype)
+    sh = _shape(B, N, Hq, Hkv, d, q.dtype, Ncap)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, cap, 1))
     idx = torch.empty((B, Hkv, cap), dtype=torch.int32, device=q.device)
     count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
@@ -285,7 +305,8 @@ def route_threshold(q, K, tau, cap: int, ws: Workspace | None = None,
 
 
 def attn_gather(q, K, V, idx, count=None, ws: Workspace | None = None,
-                check: bool = True, return_lse: bool = True, out=None, lse=None):
+                check: bool = True, return_lse: bool = True, out=None, lse=None,
+                n: int | None = None):
     """Attention of q ([B,Hq,d] or [L,B,Hq,d]) over the idx rows
     [B,Hkv,stride] (first count[b,h] of each row if count is given).
     Returns (out, lse) with out shaped like q."""
@@ -293,14 +314,15 @@ def attn_gather(q, K, V, idx, count=None, ws: Workspace | None = None,
     single = q.dim() == 3
     q4 = q.unsqueeze(0) if single else q
     L, B, Hq, d = q4.shape
-    Bk, Hkv, N, dk = K.shape
+    Bk, Hkv, Ncap, dk = K.shape
+    N = _length(Ncap, n)
     if V.shape != K.shape or Bk != B or dk != d:
         raise ValueError("shape mismatch between q, K and V")
     if idx.dtype != torch.int32 or idx.dim() != 3 or idx.shape[:2] != (B, Hkv):
         raise ValueError("idx must be int32 [B,Hkv,stride]")
     stride = idx.shape[2]
     w = _ws(ws, q.device)
-    sh = _shape(B, N, Hq, Hkv, d, q.dtype)
+    sh = _shape(B, N, Hq, Hkv, d, q.dtype, Ncap)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, stride, L))
     if out is None:
         out = torch.empty_like(q4)
@@ -324,14 +346,16 @@ def attn_gather(q, K, V, idx, count=None, ws: Workspace | None = None,
 def decode_step(q_route, q_layers, K, V, k: int | None = None, tau=None,
                 cap: int | None = None, ws: Workspace | None = None,
                 check: bool = True, out=None, idx=None, count=None, lse=None,
-                return_lse: bool = True):
+                return_lse: bool = True, n: int | None = None):
     """One fused decode step: route once, attend L layers over that set.
 
     Top-k mode with ``k``; threshold mode with ``tau`` [B,Hkv] and ``cap``.
+    The cache is the first n rows of K and V (default: all rows).
     Returns dict(idx, count, out, lse).  Preallocated outputs may be passed
     to keep a timing loop free of allocations."""
     _need_cuda(q_route, q_layers, K, V, tau)
-    B, N, Hq, Hkv, d = _dims_qk(q_route, K)
+    B, Ncap, Hq, Hkv, d = _dims_qk(q_route, K)
+    N = _length(Ncap, n)
     L = q_layers.shape[0]
     if q_layers.shape != (L, B, Hq, d) or V.shape != K.shape:
         raise ValueError("q_layers must be [L,B,Hq,d] and V like K")
@@ -341,7 +365,7 @@ def decode_step(q_route, q_layers, K, V, k: int | None = None, tau=None,
     stride = int(k) if topk else int(cap)
     dev = q_route.device
     w = _ws(ws, dev)
-    sh = _shape(B, N, Hq, Hkv, d, q_route.dtype)
+    sh = _shape(B, N, Hq, Hkv, d, q_route.dtype, Ncap)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q_route.dtype, stride, L))
     if idx is None:
         idx = torch.empty((B, Hkv, stride), dtype=torch.int32, device=dev)
@@ -365,7 +389,7 @@ def decode_step(q_route, q_layers, K, V, k: int | None = None, tau=None,
 def decode_step_grouped(q_routes, q_layers, K, V, R: int, k: int | None = None, tau=None,
                         cap: int | None = None, ws: Workspace | None = None,
                         check: bool = True, out=None, idx=None, count=None, lse=None,
-                        return_lse: bool = True):
+                        return_lse: bool = True, n: int | None = None):
     """Decode step re-routing every R layers (sparse_decode_step_grouped).
 
     q_routes [ceil(L/R),B,Hq,d]: group g of R consecutive layers routes with
@@ -375,7 +399,8 @@ def decode_step_grouped(q_routes, q_layers, K, V, R: int, k: int | None = None, 
     _need_cuda(q_routes, q_layers, K, V, tau)
     if q_routes.dim() != 4 or K.dim() != 4:
         raise ValueError("q_routes must be [ngroups,B,Hq,d] and K [B,Hkv,N,d]")
-    B, N, Hq, Hkv, d = _dims_qk(q_routes[0], K)
+    B, Ncap, Hq, Hkv, d = _dims_qk(q_routes[0], K)
+    N = _length(Ncap, n)
     L = q_layers.shape[0]
     R = int(R)
     if R < 1:
@@ -389,7 +414,7 @@ def decode_step_grouped(q_routes, q_layers, K, V, R: int, k: int | None = None, 
     stride = int(k) if topk else int(cap)
     dev = q_routes.device
     w = _ws(ws, dev)
-    sh = _shape(B, N, Hq, Hkv, d, q_routes.dtype)
+    sh = _shape(B, N, Hq, Hkv, d, q_routes.dtype, Ncap)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q_routes.dtype, stride, min(R, L)))
     if idx is None:
         idx = torch.empty((ng, B, Hkv, stride), dtype=torch.int32, device=dev)
@@ -408,3 +433,21 @@ def decode_step_grouped(q_routes, q_layers, K, V, R: int, k: int | None = None, 
     if check:
         read_device_status(w)
     return {"idx": idx, "count": count, "out": out, "lse": lse}
+
+
+def kv_append(K, V, k_new, v_new, n: int):
+    """Write the new token's key and value rows k_new, v_new [B,Hkv,d] as row
+    n-1 of every (sequence, KV head) of K and V [B,Hkv,n_cap,d] (n <= n_cap:
+    the cache length including the new token), on the current stream."""
+    _need_cuda(K, V, k_new, v_new)
+    if K.dim() != 4 or V.shape != K.shape:
+        raise ValueError("K and V must be [B,Hkv,n_cap,d] of one shape")
+    B, Hkv, Ncap, d = K.shape
+    N = _length(Ncap, n)
+    if k_new.shape != (B, Hkv, d) or v_new.shape != (B, Hkv, d):
+        raise ValueError("k_new and v_new must be [B,Hkv,d]")
+    if not (k_new.dtype == v_new.dtype == K.dtype == V.dtype):
+        raise ValueError("K, V, k_new and v_new must share a dtype")
+    sh = _shape(B, N, Hkv, Hkv, d, K.dtype, Ncap)
+    _check(load().sparse_kv_append(ctypes.byref(sh), _ptr(K), _ptr(V), _ptr(k_new),
+                                   _ptr(v_new), _stream()), "kv_append")

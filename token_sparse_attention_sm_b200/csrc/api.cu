@@ -71,8 +71,10 @@ sparse_status_t check_shape(const sparse_shape_t *shape, Shape *s) {
   s->Hkv = shape->Hkv;
   s->d = shape->d;
   s->dtype = shape->dtype;
+  s->Ncap = shape->n_cap == 0 ? shape->N : shape->n_cap;
   if (s->B < 1 || s->N < 1 || s->Hq < 1 || s->Hkv < 1 || s->d < 1)
     return SPARSE_ERR_INVALID_ARG;
+  if (s->Ncap < s->N) return SPARSE_ERR_INVALID_ARG;
   if (s->Hq % s->Hkv != 0) return SPARSE_ERR_INVALID_ARG;
   if (s->d != 64 && s->d != 128) return SPARSE_ERR_UNSUPPORTED;
   if (s->dtype != SPARSE_DTYPE_F32 && s->dtype != SPARSE_DTYPE_BF16)

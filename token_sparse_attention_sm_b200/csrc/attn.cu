@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kAttnThreads)
     attn_partial_kernel(const T *__restrict__ q, const T *__restrict__ K,
                         const T *__restrict__ V, const int *__restrict__ idx,
                         int stride, const int *__restrict__ count,
-                        int count_cap, int N, int B, int Hq, int Hkv, int L,
+                        int count_cap, int N, int kv_rows, int B, int Hq, int Hkv, int L,
                         int nsplit, float scale, float *__restrict__ part,
                         uint32_t *status) {
   constexpr int EPL = D / 32;  // fp32 elements per lane
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kAttnThreads)
       if (r < nc && !ok && c == 0) raise_flag(status, FLAG_INDEX);
       float fk[EV], fv[EV];
       if (ok) {
-        const size_t off = ((size_t)bh * N + j) * D + c;
+        const size_t off = ((size_t)bh * kv_rows + j) * D + c;
         unpack16<T>(*reinterpret_cast<const uint4 *>(K + off), fk);
         unpack16<T>(*reinterpret_cast<const uint4 *>(V + off), fv);
       } else {
@@ -231,7 +231,7 @@ cudaError_t launch_attn_t(const Shape &s, int L, const void *q, const void *K,
   dim3 grid(nsplit, s.BH(), qblocks);
   attn_partial_kernel<T, D><<<grid, kAttnThreads, 0, st>>>(
       static_cast<const T *>(q), static_cast<const T *>(K),
-      static_cast<const T *>(V), idx, stride, count, count_cap, s.N, s.B,
+      static_cast<const T *>(V), idx, stride, count, count_cap, s.N, s.Ncap, s.B,
       s.Hq, s.Hkv, L, nsplit, scale, part, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kThreads)
                     const __nv_bfloat16 *__restrict__ K,
                     const __nv_bfloat16 *__restrict__ V,
                     const int *__restrict__ idx, int stride,
-                    const int *__restrict__ count, int N, int B, int Hq,
+                    const int *__restrict__ count, int N, int kv_rows, int B, int Hq,
                     int Hkv, int L, float scale_log2,
                     __nv_bfloat16 *__restrict__ out, float *__restrict__ lse,
                     uint32_t *status) {
@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(kThreads)
   const int per = (cnt + csize - 1) / csize;
   const int k0 = min(cnt, rank * per), k1 = min(cnt, k0 + per);
   const int *row = idx + (size_t)bh * stride;
-  const size_t head_off = (size_t)bh * N * D;
+  const size_t head_off = (size_t)bh * kv_rows * D;
 
   auto load_tile = [&](int buf, int t0) {
     __nv_bfloat16 *kt = Ks + buf * kTileKeys * D;
@@ -401,7 +401,7 @@ cudaError_t launch_mma_t(const Shape &s, int L, const void *q, const void *K,
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16 *>(q),
                          static_cast<const __nv_bfloat16 *>(K),
                          static_cast<const __nv_bfloat16 *>(V), idx, stride, count,
-                         s.N, s.B, s.Hq, s.Hkv, L, scale_log2,
+                         s.N, s.Ncap, s.B, s.Hq, s.Hkv, L, scale_log2,
                          static_cast<__nv_bfloat16 *>(out), lse, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

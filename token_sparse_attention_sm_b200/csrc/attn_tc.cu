@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    const __nv_bfloat16 *__restrict__ K,
                    const __nv_bfloat16 *__restrict__ V,
                    const int *__restrict__ idx, int stride,
-                   const int *__restrict__ count, int N, int B, int Hq, int Hkv,
+                   const int *__restrict__ count, int N, int kv_rows, int B, int Hq, int Hkv,
                    int L, float scale_log2, __nv_bfloat16 *__restrict__ out,
                    float *__restrict__ lse, float *__restrict__ part,
                    uint32_t *__restrict__ counters, uint32_t *status) {
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int per = (cnt + csize - 1) / csize;
   const int k0 = min(cnt, rank * per), k1 = min(cnt, k0 + per);
   const int *rowidx = idx + (size_t)bh * stride;
-  const size_t head_off = (size_t)bh * N * D;
+  const size_t head_off = (size_t)bh * kv_rows * D;
 
   // ---- Q block (rows beyond M are zero): thread = (row, part of the row) ----
   {
@@ -656,7 +656,7 @@ cudaError_t launch_tc_t(const Shape &s, int L, const void *q, const void *K,
   const float scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16 *>(q),
                          static_cast<const __nv_bfloat16 *>(K),
-                         static_cast<const __nv_bfloat16 *>(V), idx, stride, count, s.N,
+                         static_cast<const __nv_bfloat16 *>(V), idx, stride, count, s.N, s.Ncap,
                          s.B, s.Hq, s.Hkv, L, scale_log2, static_cast<__nv_bfloat16 *>(out),
                          lse, part, counters, status);
   if (e != cudaSuccess) return e;

@@ -10,6 +10,7 @@ namespace sd {
 
 struct Shape {
   int B, N, Hq, Hkv, d, dtype;  // dtype: 0 = fp32, 1 = bf16
+  int Ncap;                     // rows allocated per (sequence, KV head) in K, V (>= N)
   int G() const { return Hq / Hkv; }
   int BH() const { return B * Hkv; }
   int esize() const { return dtype == 0 ? 4 : 2; }

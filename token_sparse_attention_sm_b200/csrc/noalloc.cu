@@ -42,7 +42,9 @@ extern "C" sparse_status_t sparse_route_topk_static(const sparse_shape_t *shape,
                                                     int32_t k, int32_t *idx,
                                                     void *stream) {
   if (!shape) return SPARSE_ERR_INVALID_ARG;
-  sd::Shape s{shape->B, shape->N, shape->Hq, shape->Hkv, shape->d, shape->dtype};
+  sd::Shape s{shape->B, shape->N, shape->Hq, shape->Hkv, shape->d, shape->dtype,
+              shape->n_cap == 0 ? shape->N : shape->n_cap};
+  if (s.Ncap < s.N) return SPARSE_ERR_INVALID_ARG;
   if (s.B < 1 || s.N < 1 || s.Hq < 1 || s.Hkv < 1 || s.Hq % s.Hkv != 0)
     return SPARSE_ERR_INVALID_ARG;
   if ((s.d != 64 && s.d != 128) || (s.dtype != 0 && s.dtype != 1) || s.G() > 16)

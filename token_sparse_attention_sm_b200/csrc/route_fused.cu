@@ -316,7 +316,8 @@ __device__ void cta_select_full(const float *__restrict__ Srow, int N, int k,
 template <typename T, int D>
 __global__ void __launch_bounds__(kFThreads, 1)
     route_topk_fused_kernel(const T *__restrict__ q, const T *__restrict__ K,
-                            float *__restrict__ S, int N, int Hq, int Hkv, int tph, int cpp,
+                            float *__restrict__ S, int N, int kv_rows, int Hq, int Hkv,
+                            int tph, int cpp,
                             float scale, int k, uint32_t *__restrict__ hist,
                             uint32_t *__restrict__ ctr, uint2 *__restrict__ meta,
                             uint32_t *__restrict__ gcand, int *__restrict__ idx,
@@ -366,7 +367,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
     o.shist = shist;
     o.keys = keys;
     o.key_off = -jlo;
-    scan_tiles<T, D, 1>(q, K, N, Hq, Hkv, tph, (long long)bh * tph + tl, th - tl, bh, scale,
+    scan_tiles<T, D, 1>(q, K, N, kv_rows, Hq, Hkv, tph, (long long)bh * tph + tl, th - tl, bh,
+                        scale,
                         smem, full, empty, o, status);
   }
   __syncthreads();  // the ring is free and every count is in shared memory
@@ -767,7 +769,8 @@ cudaError_t launch_fused_t(const Shape &s, const void *q, const void *K, int k, 
   }
   add_pdl_attr(cfg, attrs);
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(q), static_cast<const T *>(K), S,
-                         s.N, s.Hq, s.Hkv, tph, cpp, scale, k, hist, ctr, meta, gcand, idx,
+                         s.N, s.Ncap, s.Hq, s.Hkv, tph, cpp, scale, k, hist, ctr, meta, gcand,
+                         idx,
                          status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -73,14 +73,16 @@ struct ScanOut {
   int key_off;
 };
 
-// One CTA's share of the scan: tiles [t_begin, t_begin + ntiles).  Warps
+// One CTA's share of the scan: tiles [t_begin, t_begin + ntiles).  K holds
+// kv_rows rows per (sequence, KV head), the first N of them scanned.  Warps
 // 0..3 consume, warp 4 produces: its lane 0 issues the copies and waits for
 // the last ones to land, its other lanes (and any further warps) return at
 // once.  Barriers full/empty
 // must be initialised (count 1 / kScanConsumerWarps).
 template <typename T, int D, int kSlots>
 __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__restrict__ K,
-                                           int N, int Hq, int Hkv, int tiles_per_head,
+                                           int N, int kv_rows, int Hq, int Hkv,
+                                           int tiles_per_head,
                                            long long t_begin, int ntiles, int bh_first,
                                            float scale, unsigned char *ring, uint64_t *full,
                                            uint64_t *empty, ScanOut o,
@@ -104,7 +106,7 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
         const int nk = min(C::kStageKeys, N - j0);
         const uint32_t bytes = (uint32_t)nk * C::kRowBytes;
         mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_g2s(ring + (size_t)s * kScanStageBytes, K + ((size_t)bh * N + j0) * D,
+        bulk_g2s(ring + (size_t)s * kScanStageBytes, K + ((size_t)bh * kv_rows + j0) * D,
                  bytes, &full[s], pol);
         ++issued;
       }

@@ -41,7 +41,7 @@ constexpr int kScoreSmem = kScanStages * kScanStageBytes + kHistSlots * kScanBin
 template <typename T, int D>
 __global__ void __launch_bounds__(kScanThreads, 1)
     score_kernel(const T *__restrict__ q, const T *__restrict__ K,
-                 float *__restrict__ S, int N, int Hq, int Hkv,
+                 float *__restrict__ S, int N, int kv_rows, int Hq, int Hkv,
                  int tiles_per_head, long long total_tiles, float scale,
                  uint32_t *__restrict__ hist, uint32_t *status) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -76,7 +76,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   o.shist = shist;
   o.keys = nullptr;
   o.key_off = 0;
-  scan_tiles<T, D, kHistSlots>(q, K, N, Hq, Hkv, tiles_per_head, t_begin, ntiles, bh_first,
+  scan_tiles<T, D, kHistSlots>(q, K, N, kv_rows, Hq, Hkv, tiles_per_head, t_begin, ntiles,
+                               bh_first,
                                scale, smem, full, empty, o, status);
   if (threadIdx.x >= kScanConsumerWarps * 32) return;  // producer warp
   if (hist) {
@@ -117,7 +118,7 @@ cudaError_t launch_score_t(const Shape &s, const void *q, const void *K,
   cfg.numAttrs = 0;
   add_pdl_attr(cfg, attrs);
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(q), static_cast<const T *>(K), S,
-                         s.N, s.Hq, s.Hkv, tiles_per_head, total, scale, hist, status);
+                         s.N, s.Ncap, s.Hq, s.Hkv, tiles_per_head, total, scale, hist, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
