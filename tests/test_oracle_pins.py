@@ -416,3 +416,72 @@ def test_grouped_step_group_boundaries_and_invariants():
     for g in range(3):
         S = oracle.scores(qrs[g], K)
         np.testing.assert_array_equal(th["count"][g], (S >= tau[g][..., None]).sum(-1))
+
+
+# --------------------------------------------------------------------------
+# Louver index, one subspace (Louver summary, section 2. Louver インデックス):
+# balanced PCA tree clusters, bounding balls, ball test then exact check
+# --------------------------------------------------------------------------
+
+def _blobs(r, B, Hkv, N, d, nblob=16, spread=0.05):
+    """Keys drawn around a few centres (low intrinsic dimension, like real
+    attention keys), the structure the index prunes on."""
+    centres = r.standard_normal((B, Hkv, nblob, d)).astype(np.float32) * 2
+    which = r.integers(0, nblob, (B, Hkv, N))
+    K = np.take_along_axis(centres, which[..., None], axis=2)
+    return (K + spread * r.standard_normal((B, Hkv, N, d))).astype(np.float32)
+
+
+def test_louver_tree_closed_form_split_and_balls():
+    """Keys spread along one axis u (plus tiny noise): the root split of the
+    balanced PCA tree puts the N/2 keys with the smallest coordinate along u
+    on one side; clusters partition the keys; every ball holds its keys."""
+    from oracle import louver
+    r = _rng(51)
+    N, d, rc = 256, 16, 16
+    u = r.standard_normal(d)
+    u /= np.linalg.norm(u)
+    t = r.permutation(N).astype(np.float64)          # distinct coordinates
+    Kh = (t[:, None] * u[None, :] + 1e-3 * r.standard_normal((N, d))).astype(np.float32)
+    ix = louver.build_index(Kh, rc)
+    perm = ix["perm"]
+    assert sorted(perm.tolist()) == list(range(N))
+    low = set(np.argsort(t)[:N // 2].tolist())
+    halves = [set(perm[:N // 2].tolist()), set(perm[N // 2:].tolist())]
+    assert low in halves
+    X = Kh.astype(np.float64)[perm].reshape(N // rc, rc, d)
+    dist = np.sqrt(((X - ix["centres"][:, None, :]) ** 2).sum(-1))
+    assert np.all(dist <= ix["radii"][:, None] + 1e-12)
+    np.testing.assert_allclose(ix["centres"], X.mean(1), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", ["gaussian", "blobs"])
+def test_louver_query_equals_full_scan_and_prunes_soundly(kind):
+    """The index's threshold set equals the full-scan threshold set exactly
+    (no false negatives, no extras) at several tau; every pruned cluster
+    holds only keys scoring below tau; on clustered keys most clusters are
+    pruned."""
+    from oracle import louver
+    r = _rng(53)
+    B, Hq, Hkv, N, d, rc = 1, 8, 2, 1024, 32, 16
+    q = r.standard_normal((B, Hq, d), dtype=np.float32)
+    K = (r.standard_normal((B, Hkv, N, d), dtype=np.float32) if kind == "gaussian"
+         else _blobs(r, B, Hkv, N, d))
+    S = oracle.scores(q, K)
+    S64 = oracle.scores(q, K, np.float64)
+    for pct in (50, 97, 100):
+        tau = oracle.percentile_tau(S, pct, 100)
+        idx, cnt, surv = louver.route_threshold(q, K, tau, N, rc)
+        ridx, rcnt = louver.full_scan_threshold(q, K, tau, N)
+        np.testing.assert_array_equal(cnt, rcnt)
+        np.testing.assert_array_equal(idx, ridx)
+        G = Hq // Hkv
+        for h in range(Hkv):
+            ix = louver.build_index(K[0, h], rc)
+            qbar = q[0, h * G:(h + 1) * G].astype(np.float64).sum(0) / math.sqrt(d)
+            t = float(tau[0, h])
+            pruned = louver.ball_bounds(ix, qbar) < t - louver.band(t)
+            keys = ix["perm"].reshape(-1, rc)[pruned].ravel()
+            assert np.all(S64[0, h, keys] < t)
+        if kind == "blobs" and pct == 97:
+            assert surv.sum() < 0.5 * Hkv * (N // rc)
