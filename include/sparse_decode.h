@@ -232,6 +232,59 @@ sparse_status_t sparse_decode_step_grouped(const sparse_shape_t *shape, int32_t 
 sparse_status_t sparse_kv_append(const sparse_shape_t *shape, void *K, void *V,
                                  const void *k_new, const void *v_new, void *stream);
 
+/* ---- Louver index (threshold routing with cluster pruning) ----------------
+ * Louver summary, section 2. Louver インデックス: the keys of every (sequence,
+ * KV head) are grouped into clusters of r keys by a balanced PCA tree and each
+ * cluster is enclosed in a bounding ball; a threshold query (section 1.
+ * 半空間範囲検索への帰着: keep every key in the halfspace {p : <qbar,p> >= tau},
+ * no false negatives) skips the clusters whose ball misses the halfspace and
+ * checks the keys of the others exactly.  One subspace (the page's S = 1).
+ * Requirements: r a power of two in [32, 256], N a multiple of r, N / r a
+ * power of two and N <= 1048576; the usual shape limits.
+ *
+ * Index buffer (device, caller-owned, index_bytes, 256-byte aligned):
+ *   perm [B*Hkv][N] int32 (key ids in cluster order: cluster c of head bh is
+ *   perm[bh][c*r .. c*r+r)), centres [B*Hkv][N/r][d] fp32, radii [B*Hkv][N/r]
+ *   fp32, at the offsets 0, align256(B*Hkv*N*4), and after the centres.
+ * The index describes K's first N rows; it must be rebuilt (or the keys
+ * re-indexed) when those rows change.
+ * Workspace: ws_bytes from sparse_louver_sizes, zero-filled once before first
+ * use like the other workspaces.  Build and query calls may share one
+ * (ordered), but it must not be shared with the other entry points: their
+ * scratch areas overlap and each side keeps parts of its own zero between
+ * calls. */
+
+/* Sizes of the index buffer and of the workspace for this shape and r. */
+sparse_status_t sparse_louver_sizes(const sparse_shape_t *shape, int32_t r,
+                                    size_t *index_bytes, size_t *ws_bytes);
+
+/* Builds the index of K [B,Hkv,n_cap,d] (first N rows) into `index`.
+ * Each tree level splits every node at the median of its keys' projections
+ * on the node's principal direction (8 power-iteration passes); leaves get
+ * their mean as centre and the largest distance to it (inflated by 1e-5
+ * relative) as radius.  fp32 atomic sums make the directions depend on
+ * summation order: two builds may differ, every build is a valid index and
+ * query results do not depend on it.  Asynchronous on `stream`. */
+sparse_status_t sparse_louver_build(const sparse_shape_t *shape, const void *K, int32_t r,
+                                    void *index, size_t index_bytes, void *ws,
+                                    size_t ws_bytes, void *stream);
+
+/* Threshold routing through the index: the same set as
+ * sparse_route_threshold (identical scores, keys with S >= tau[b,h]) in
+ * ascending order in idx [B,Hkv,cap], its size in count [B,Hkv]
+ * (SPARSE_ERR_CAPACITY is reported through the status word when a count
+ * exceeds cap, as there).  A cluster is skipped only when its ball bound
+ * <qbar,c> + |qbar| rho is below tau - (1e-4 |tau| + 1e-6) - 1e-5 |qbar|
+ * (|c| + rho), a margin above the fp32 rounding of any member's score, so
+ * rounding cannot drop a key.  survivors (nullable) [B,Hkv] int32: clusters that
+ * passed the ball test.  q [B,Hq,d] and K of the shape's dtype. */
+sparse_status_t sparse_louver_route_threshold(const sparse_shape_t *shape, const void *q,
+                                              const void *K, const void *index,
+                                              size_t index_bytes, int32_t r,
+                                              const float *tau, int32_t cap, int32_t *idx,
+                                              int32_t *count, int32_t *survivors, void *ws,
+                                              size_t ws_bytes, void *stream);
+
 /* Shared routing, top-k form (as sparse_route_topk) for callers that cannot
  * allocate device memory: a plugin inside a host framework that owns every
  * device allocation, or code that must not call cudaMalloc once it is

@@ -29,9 +29,12 @@ Readings (where the page is silent):
 * The query vector is the routing query of the scores, qbar = (sum over the
   G query heads of the KV head) / sqrt(d), so <qbar, k_j> is the score S_j.
   A ball meets the halfspace iff <qbar, c> + |qbar| rho >= tau; a cluster is
-  pruned only when that bound is below tau by more than the comparison band
-  (1e-4 |tau| + 1e-6), so fp32 rounding of the exact check cannot make a
-  pruned key pass.
+  pruned only when that bound is below tau by more than a margin: the
+  comparison band (1e-4 |tau| + 1e-6) plus 1e-5 |qbar| (|c| + rho).  The
+  second term bounds the fp32 rounding of a member's score (at most a few
+  1e-7 of |qbar| |k| for d <= 128, and |k| <= |c| + rho), which does not
+  shrink with tau, so no fp32 rounding of the exact check can make a pruned
+  key pass even when tau is near zero.
 """
 from __future__ import annotations
 
@@ -84,6 +87,15 @@ def band(tau: float) -> float:
     return 1e-4 * abs(tau) + 1e-6
 
 
+def keep_clusters(index: dict, qbar, tau: float) -> np.ndarray:
+    """The ball test: True for every cluster that may hold a key with score
+    >= tau (its bound is not below tau by more than the margin)."""
+    q = np.asarray(qbar, np.float64)
+    qn = np.linalg.norm(q)
+    slack = 1e-5 * qn * (np.linalg.norm(index["centres"], axis=1) + index["radii"])
+    return ball_bounds(index, q) >= tau - band(tau) - slack
+
+
 def route_threshold(q, K, tau, cap: int, r: int):
     """Threshold routing through the index, every (b, h).
 
@@ -106,7 +118,7 @@ def route_threshold(q, K, tau, cap: int, r: int):
             index = build_index(K[b, h], r)
             qbar = q[b, h * G:(h + 1) * G].astype(np.float64).sum(0) / math.sqrt(d)
             t = float(tau[b, h])
-            keep = ball_bounds(index, qbar) >= t - band(t)
+            keep = keep_clusters(index, qbar, t)
             surv[b, h] = int(keep.sum())
             cand = index["perm"].reshape(-1, r)[keep].ravel()
             sel = np.sort(cand[S[b, h, cand] >= tau[b, h]])

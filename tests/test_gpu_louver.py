@@ -1,0 +1,226 @@
+"""GPU parity of the Louver index (Louver summary, section 2. Louver インデックス;
+section 1. 半空間範囲検索への帰着 for the set it must return).
+
+The index itself is not unique (the tree's directions come from fp32 power
+iteration on the device, the oracle's from an exact eigendecomposition), so
+the tests check what makes any index valid -- the permutation, the clusters'
+balanced sizes, ball containment in fp64, centres equal to member means --
+and what is unique: the returned set, which must equal the full-scan
+threshold set on the same scores bit for bit (GPU route_threshold) and the
+oracle's set within the comparison band; and zero false negatives.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import louver as olouver
+import token_sparse_attention_sm_b200 as sd
+from token_sparse_attention_sm_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    from token_sparse_attention_sm_b200 import build
+    build.build()
+    sd.load()
+    return torch.device("cuda", 0)
+
+
+def _band(s):
+    return 1e-4 * abs(float(s)) + 1e-6
+
+
+def _f(x):
+    return synth.f32(x)
+
+
+def _assert_same_set(a, b, cap):
+    """(idx, count) pairs equal: the counts, and the first min(count, cap)
+    entries of every row (entries beyond them are not written)."""
+    ai, ac = a[0].cpu().numpy(), a[1].cpu().numpy()
+    bi, bc = b[0].cpu().numpy(), b[1].cpu().numpy()
+    np.testing.assert_array_equal(ac, bc)
+    for bh in np.ndindex(ac.shape):
+        n = min(int(ac[bh]), cap)
+        np.testing.assert_array_equal(ai[bh][:n], bi[bh][:n])
+
+
+def _check_index(ix, K32, r):
+    """K32 [B,Hkv,N,d] fp32 (the keys the index covers)."""
+    B, Hkv, N, d = K32.shape
+    perm = ix.perm().cpu().numpy()
+    cen = ix.centres().cpu().numpy().astype(np.float64)
+    rad = ix.radii().cpu().numpy().astype(np.float64)
+    for b in range(B):
+        for h in range(Hkv):
+            p = perm[b, h]
+            assert np.array_equal(np.sort(p), np.arange(N)), "not a permutation"
+            members = K32[b, h][p].astype(np.float64).reshape(N // r, r, d)
+            mean = members.mean(axis=1)
+            np.testing.assert_allclose(cen[b, h], mean, rtol=1e-4, atol=1e-4)
+            dist = np.sqrt(((members - cen[b, h][:, None, :]) ** 2).sum(-1)).max(axis=1)
+            assert np.all(dist <= rad[b, h]), "a key lies outside its cluster's ball"
+
+
+def _check_set(gidx, gcnt, q32, K32, tau, cap):
+    """The GPU set against the oracle: equal to the fp32 threshold set except
+    for keys within the band of tau; every key >= tau + band present."""
+    S = oracle.scores(q32, K32)
+    S64 = oracle.scores(q32, K32, np.float64)
+    ridx, rcnt = oracle.threshold(S, tau, cap)
+    B, Hkv = gcnt.shape
+    for b in range(B):
+        for h in range(Hkv):
+            t = tau[b, h]
+            band = _band(t)
+            g = set(gidx[b, h, :min(gcnt[b, h], cap)].tolist())
+            if gcnt[b, h] <= cap:
+                must = set(np.nonzero(S64[b, h] >= t + band)[0].tolist())
+                never = set(np.nonzero(S64[b, h] < t - band)[0].tolist())
+                assert must <= g, "false negative"
+                assert not (g & never), "false positive"
+            assert abs(int(gcnt[b, h]) - int(rcnt[b, h])) <= \
+                int(np.sum(np.abs(S[b, h] - t) <= band))
+    return rcnt
+
+
+CASES = [
+    dict(B=1, N=8192, Hq=8, Hkv=2, d=128, dtype="bf16", r=128, blobs=16, pct=97),
+    dict(B=2, N=4096, Hq=4, Hkv=2, d=64, dtype="f32", r=64, blobs=8, pct=90),
+    dict(B=1, N=16384, Hq=16, Hkv=4, d=128, dtype="bf16", r=256, blobs=0, pct=99),
+    dict(B=1, N=2048, Hq=2, Hkv=1, d=64, dtype="bf16", r=32, blobs=4, pct=50),
+]
+
+
+@pytest.mark.parametrize("c", CASES, ids=lambda c: "-".join(f"{k}{v}" for k, v in c.items()))
+def test_louver_index_and_set(dev, c):
+    w = synth.custom(B=c["B"], N=c["N"], Hq=c["Hq"], Hkv=c["Hkv"], d=c["d"], L=1,
+                     dtype=c["dtype"], seed=11, mode="threshold", cap=c["N"],
+                     blobs=c["blobs"], blob_spread=0.1)
+    x = synth.generate(w)
+    q32, K32 = _f(x["q_route"]), _f(x["K"])
+    qd, Kd = x["q_route"].to(dev), x["K"].to(dev)
+    ix = sd.louver_build(Kd, c["r"])
+    _check_index(ix, K32, c["r"])
+    S = oracle.scores(q32, K32)
+    tau = oracle.percentile_tau(S, c["pct"], 100)
+    taud = torch.from_numpy(tau).to(dev)
+    cap = c["N"]
+    gidx, gcnt, surv = sd.louver_route_threshold(qd, Kd, ix, taud, cap, return_survivors=True)
+    # bit-identical to the full-scan threshold routing on the GPU
+    _assert_same_set((gidx, gcnt), sd.route_threshold(qd, Kd, taud, cap), cap)
+    gidx, gcnt = gidx.cpu().numpy(), gcnt.cpu().numpy()
+    _check_set(gidx, gcnt, q32, K32, tau, cap)
+    # every cluster holding a selected key passed the ball test
+    perm = ix.perm().cpu().numpy()
+    surv = surv.cpu().numpy()
+    nc = c["N"] // c["r"]
+    for b in range(c["B"]):
+        for h in range(c["Hkv"]):
+            cl = np.empty(c["N"], np.int64)
+            cl[perm[b, h]] = np.arange(c["N"]) // c["r"]
+            held = len(set(cl[gidx[b, h, :gcnt[b, h]]].tolist()))
+            assert held <= surv[b, h] <= nc
+
+
+def test_louver_matches_oracle_louver(dev):
+    """The oracle's own Louver route (its own index) returns the same set on
+    the oracle's scores; the GPU set agrees with it within the band."""
+    w = synth.custom(B=1, N=4096, Hq=8, Hkv=2, d=64, L=1, dtype="f32", seed=5,
+                     mode="threshold", cap=4096, blobs=16, blob_spread=0.05)
+    x = synth.generate(w)
+    q32, K32 = _f(x["q_route"]), _f(x["K"])
+    tau = oracle.percentile_tau(oracle.scores(q32, K32), 97, 100)
+    oidx, ocnt, osurv = olouver.route_threshold(q32, K32, tau, 4096, 64)
+    ix = sd.louver_build(x["K"].to(dev), 64)
+    gidx, gcnt, gsurv = sd.louver_route_threshold(x["q_route"].to(dev), x["K"].to(dev), ix,
+                                                  torch.from_numpy(tau).to(dev), 4096,
+                                                  return_survivors=True)
+    gidx, gcnt = gidx.cpu().numpy(), gcnt.cpu().numpy()
+    rcnt = _check_set(gidx, gcnt, q32, K32, tau, 4096)
+    np.testing.assert_array_equal(ocnt, rcnt)
+    # both indexes prune most clusters on tightly clustered keys
+    assert osurv.max() < 0.5 * (4096 // 64)
+    assert gsurv.cpu().numpy().max() < 0.5 * (4096 // 64)
+
+
+def test_louver_prunes_clustered_128k(dev):
+    """The clustered 128K workload: zero false negatives and most clusters
+    pruned, at the size the benchmark measures."""
+    w = synth.WORKLOADS["louver_128k"]
+    x = synth.generate(w)
+    q32, K32 = _f(x["q_route"]), _f(x["K"])
+    qd, Kd = x["q_route"].to(dev), x["K"].to(dev)
+    tau = oracle.percentile_tau(oracle.scores(q32, K32), *w.tau_pct)
+    taud = torch.from_numpy(tau).to(dev)
+    ix = sd.louver_build(Kd, 128)
+    gidx, gcnt, surv = sd.louver_route_threshold(qd, Kd, ix, taud, w.cap, return_survivors=True)
+    _assert_same_set((gidx, gcnt), sd.route_threshold(qd, Kd, taud, w.cap), w.cap)
+    _check_set(gidx.cpu().numpy(), gcnt.cpu().numpy(), q32, K32, tau, w.cap)
+    assert surv.cpu().numpy().max() < 0.5 * (w.N // 128)
+
+
+def test_louver_cache_longer_than_length_and_rebuild(dev):
+    """n < n_cap: the index covers the first n rows only; keys beyond are
+    never returned.  A second build over the same keys gives a valid index
+    and the same set."""
+    w = synth.custom(B=1, N=6144, Hq=8, Hkv=2, d=128, L=1, dtype="bf16", seed=3,
+                     mode="threshold", cap=4096, blobs=8)
+    x = synth.generate(w)
+    n = 4096
+    Kd = x["K"].to(dev)
+    qd = x["q_route"].to(dev)
+    K32 = _f(x["K"])[:, :, :n]
+    q32 = _f(x["q_route"])
+    tau = oracle.percentile_tau(oracle.scores(q32, K32), 90, 100)
+    taud = torch.from_numpy(tau).to(dev)
+    ix = sd.louver_build(Kd, 64, n=n)
+    _check_index(ix, K32, 64)
+    a = sd.louver_route_threshold(qd, Kd, ix, taud, 4096)
+    ix2 = sd.louver_build(Kd, 64, n=n)
+    _check_index(ix2, K32, 64)
+    b = sd.louver_route_threshold(qd, Kd, ix2, taud, 4096)
+    f = sd.route_threshold(qd, Kd, taud, 4096, n=n)
+    _assert_same_set(a, f, 4096)
+    _assert_same_set(b, f, 4096)
+    _check_set(a[0].cpu().numpy(), a[1].cpu().numpy(), q32, K32, tau, 4096)
+
+
+def test_louver_empty_set_capacity_and_status_reset(dev):
+    w = synth.custom(B=1, N=2048, Hq=4, Hkv=2, d=64, L=1, dtype="bf16", seed=8,
+                     mode="threshold", cap=64, blobs=4)
+    x = synth.generate(w)
+    qd, Kd = x["q_route"].to(dev), x["K"].to(dev)
+    ix = sd.louver_build(Kd, 64)
+    tau = torch.tensor([[1e9, -1e9]], device=dev)
+    gidx, gcnt = sd.louver_route_threshold(qd, Kd, ix, tau, 64, check=False)
+    assert sd.read_device_status(ix.ws, raise_on_error=False) == 4   # capacity
+    assert gcnt.cpu().tolist() == [[0, 2048]]
+    assert gidx[0, 1].cpu().tolist() == list(range(64))
+    tau = torch.full((1, 2), 1e9, device=dev)
+    _, gcnt = sd.louver_route_threshold(qd, Kd, ix, tau, 64, check=False)
+    assert sd.read_device_status(ix.ws, raise_on_error=False) == 0   # reset
+    assert gcnt.cpu().tolist() == [[0, 0]]
+
+
+def test_louver_repeated_queries_keep_workspace_clean(dev):
+    """Many queries through one index: the bitmap and survivor counters the
+    kernels keep zero between calls stay zero (every call equals the full
+    scan)."""
+    w = synth.custom(B=2, N=4096, Hq=8, Hkv=2, d=128, L=1, dtype="bf16", seed=21,
+                     mode="threshold", cap=4096, blobs=16)
+    x = synth.generate(w)
+    Kd = x["K"].to(dev)
+    ix = sd.louver_build(Kd, 128)
+    variants = synth.query_variants(w, x, 6, seed=77)
+    for i, (qr, _) in enumerate(variants):
+        qd = qr.to(dev)
+        S = oracle.scores(_f(qr), _f(x["K"]))
+        tau = torch.from_numpy(oracle.percentile_tau(S, 80 + 3 * i, 100)).to(dev)
+        a = sd.louver_route_threshold(qd, Kd, ix, tau, 4096)
+        _assert_same_set(a, sd.route_threshold(qd, Kd, tau, 4096), 4096)

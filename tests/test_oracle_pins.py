@@ -480,7 +480,7 @@ def test_louver_query_equals_full_scan_and_prunes_soundly(kind):
             ix = louver.build_index(K[0, h], rc)
             qbar = q[0, h * G:(h + 1) * G].astype(np.float64).sum(0) / math.sqrt(d)
             t = float(tau[0, h])
-            pruned = louver.ball_bounds(ix, qbar) < t - louver.band(t)
+            pruned = ~louver.keep_clusters(ix, qbar, t)
             keys = ix["perm"].reshape(-1, rc)[pruned].ravel()
             assert np.all(S64[0, h, keys] < t)
         if kind == "blobs" and pct == 97:

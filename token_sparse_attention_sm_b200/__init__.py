@@ -26,7 +26,7 @@ __all__ = ["SparseDecodeError", "lib_path", "load", "score", "select_topk",
            "select_threshold", "route_topk", "route_threshold", "attn_gather",
            "decode_step", "read_device_status", "workspace_bytes",
            "Workspace", "STATUS_NAMES", "EXPORTED_SYMBOLS", "decode_step_grouped",
-           "kv_append"]
+           "kv_append", "LouverIndex", "louver_build", "louver_route_threshold"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_PKG, "libsparse_decode.so")
@@ -44,6 +44,7 @@ EXPORTED_SYMBOLS = (
     "sparse_select_threshold", "sparse_route_topk", "sparse_route_threshold",
     "sparse_attn_gather", "sparse_decode_step", "sparse_read_device_status",
     "sparse_route_topk_static", "sparse_decode_step_grouped", "sparse_kv_append",
+    "sparse_louver_sizes", "sparse_louver_build", "sparse_louver_route_threshold",
 )
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
@@ -102,6 +103,10 @@ def load():
             "sparse_decode_step_grouped": (I32, [SH, I32, I32, P, P, P, P, I32, P, I32,
                                                  P, P, P, P, P, SZ, P]),
             "sparse_kv_append": (I32, [SH, P, P, P, P, P]),
+            "sparse_louver_sizes": (I32, [SH, I32, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
+            "sparse_louver_build": (I32, [SH, P, I32, P, SZ, P, SZ, P]),
+            "sparse_louver_route_threshold": (I32, [SH, P, P, P, SZ, I32, P, I32, P, P, P, P,
+                                                    SZ, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -451,3 +456,92 @@ def kv_append(K, V, k_new, v_new, n: int):
     sh = _shape(B, N, Hkv, Hkv, d, K.dtype, Ncap)
     _check(load().sparse_kv_append(ctypes.byref(sh), _ptr(K), _ptr(V), _ptr(k_new),
                                    _ptr(v_new), _stream()), "kv_append")
+
+
+class LouverIndex:
+    """A Louver index over the first n rows of one K cache [B,Hkv,n_cap,d]:
+    the device index buffer and the index's own workspace (which no other
+    call may share)."""
+
+    def __init__(self, K, r: int, n: int):
+        B, Hkv, Ncap, d = K.shape
+        self.B, self.Hkv, self.N, self.Ncap, self.d = B, Hkv, n, Ncap, d
+        self.dtype, self.r, self.device = K.dtype, int(r), K.device
+        ib, wb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        sh = _shape(B, n, Hkv, Hkv, d, K.dtype, Ncap)
+        _check(load().sparse_louver_sizes(ctypes.byref(sh), self.r, ctypes.byref(ib),
+                                          ctypes.byref(wb)), "louver_sizes")
+        self.index = torch.empty(int(ib.value), dtype=torch.uint8, device=K.device)
+        self.ws = Workspace(K.device)
+        self.ws_bytes = int(wb.value)
+        self.ws.get(self.ws_bytes)
+
+    def perm(self):
+        """Key ids in cluster order, [B,Hkv,N] int32."""
+        n = self.B * self.Hkv * self.N
+        return self.index[:4 * n].view(torch.int32).view(self.B, self.Hkv, self.N)
+
+    def _offsets(self):
+        al = lambda x: (x + 255) // 256 * 256
+        BH, nc = self.B * self.Hkv, self.N // self.r
+        c0 = al(BH * self.N * 4)
+        r0 = c0 + al(BH * nc * self.d * 4)
+        return c0, r0
+
+    def centres(self):
+        """Cluster centres, [B,Hkv,N/r,d] fp32."""
+        c0, _ = self._offsets()
+        nc = self.N // self.r
+        n = self.B * self.Hkv * nc * self.d
+        return self.index[c0:c0 + 4 * n].view(torch.float32).view(self.B, self.Hkv, nc, self.d)
+
+    def radii(self):
+        """Cluster radii, [B,Hkv,N/r] fp32."""
+        _, r0 = self._offsets()
+        nc = self.N // self.r
+        n = self.B * self.Hkv * nc
+        return self.index[r0:r0 + 4 * n].view(torch.float32).view(self.B, self.Hkv, nc)
+
+
+def louver_build(K, r: int, n: int | None = None, check: bool = True) -> LouverIndex:
+    """Build the Louver index (balanced PCA tree, clusters of r keys, bounding
+    balls) over the first n rows of K [B,Hkv,n_cap,d] on the current stream."""
+    _need_cuda(K)
+    if K.dim() != 4:
+        raise ValueError("K must be [B,Hkv,n_cap,d]")
+    N = _length(K.shape[2], n)
+    ix = LouverIndex(K, r, N)
+    sh = _shape(ix.B, N, ix.Hkv, ix.Hkv, ix.d, K.dtype, ix.Ncap)
+    buf = ix.ws.get(ix.ws_bytes)
+    _check(load().sparse_louver_build(ctypes.byref(sh), _ptr(K), ix.r, _ptr(ix.index),
+                                      ix.index.numel(), _ptr(buf), buf.numel(), _stream()),
+           "louver_build")
+    if check:
+        read_device_status(ix.ws)
+    return ix
+
+
+def louver_route_threshold(q, K, index: LouverIndex, tau, cap: int, check: bool = True,
+                           return_survivors: bool = False):
+    """Threshold routing through a Louver index: (idx [B,Hkv,cap], count [B,Hkv])
+    -- the set route_threshold returns -- plus, if asked, survivors [B,Hkv]
+    (clusters that passed the ball test)."""
+    _need_cuda(q, K, tau)
+    B, Ncap, Hq, Hkv, d = _dims_qk(q, K)
+    if (B, Hkv, Ncap, d, K.dtype) != (index.B, index.Hkv, index.Ncap, index.d, index.dtype):
+        raise ValueError("the index was built for another K")
+    sh = _shape(B, index.N, Hq, Hkv, d, q.dtype, Ncap)
+    idx = torch.empty((B, Hkv, cap), dtype=torch.int32, device=q.device)
+    count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    surv = torch.empty((B, Hkv), dtype=torch.int32, device=q.device) if return_survivors else None
+    tau = tau.float().contiguous()
+    buf = index.ws.get(index.ws_bytes)
+    _check(load().sparse_louver_route_threshold(
+        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(index.index), index.index.numel(), index.r,
+        _ptr(tau), int(cap), _ptr(idx), _ptr(count), _ptr(surv), _ptr(buf), buf.numel(),
+        _stream()), "louver_route_threshold")
+    if check:
+        read_device_status(index.ws)
+    if return_survivors:
+        return idx, count, surv
+    return idx, count

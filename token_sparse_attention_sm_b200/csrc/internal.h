@@ -102,4 +102,13 @@ cudaError_t launch_attn(const Shape &s, int L, const void *q, const void *K,
                         void *ws, uint32_t *counters, uint32_t *status,
                         cudaStream_t st);
 
+// Louver index (louver.cu).  louver_shape_ok: r and N fit the balanced tree.
+bool louver_shape_ok(const Shape &s, int r);
+void louver_sizes(const Shape &s, int r, size_t *index_bytes, size_t *ws_bytes);
+cudaError_t louver_build(const Shape &s, const void *K, int r, void *index, void *ws,
+                         cudaStream_t st);
+cudaError_t louver_query(const Shape &s, const void *q, const void *K, int r, const void *index,
+                         const float *tau, int cap, int *idx, int *count, int *survivors,
+                         void *ws, cudaStream_t st);
+
 }  // namespace sd

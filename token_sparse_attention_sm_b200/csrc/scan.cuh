@@ -59,6 +59,50 @@ struct TReduce<R, 0> {
   static __device__ __forceinline__ void run(float *, int) {}
 };
 
+// This lane's slice of qbar (the group's query rows summed in fp32, then
+// scaled): lane `sub` of a row holds elements sub*kEpl .. sub*kEpl+kEpl-1.
+template <typename T, int D>
+__device__ __forceinline__ void load_qbar(const T *__restrict__ q, int bh, int Hq, int Hkv,
+                                          int sub, float scale,
+                                          float (&qs)[ScoreCfg<T, D>::kEpl]) {
+  using C = ScoreCfg<T, D>;
+  const int b = bh / Hkv, h = bh % Hkv, G = Hq / Hkv;
+#pragma unroll
+  for (int e = 0; e < C::kEpl; ++e) qs[e] = 0.f;
+  for (int g = 0; g < G; ++g) {
+    const T *qp = q + ((size_t)b * Hq + (size_t)h * G + g) * D + sub * C::kEpl;
+#pragma unroll
+    for (int e = 0; e < C::kEpl; ++e) qs[e] += DT<T>::to_f(qp[e]);
+  }
+#pragma unroll
+  for (int e = 0; e < C::kEpl; ++e) qs[e] *= scale;
+}
+
+// Scores of the 32 keys of one warp tile: rows key0 .. key0+31 of a block of
+// contiguous rows in shared memory (kRowBytes each).  Returns, in every lane,
+// the score of key key0 + (lane % kLpk) * kKpr + lane / kLpk.  The one place
+// that fixes the scan's fp32 arithmetic (used by every kernel whose scores
+// must agree bit for bit).
+template <typename T, int D>
+__device__ __forceinline__ float warp_tile_scores(const unsigned char *rows, int key0,
+                                                  const float (&qs)[ScoreCfg<T, D>::kEpl],
+                                                  int lane) {
+  using C = ScoreCfg<T, D>;
+  const unsigned char *base = rows + (size_t)key0 * C::kRowBytes + lane * 16;
+  float v[C::kLpk];
+#pragma unroll
+  for (int r = 0; r < C::kLpk; ++r) {
+    float f[C::kEpl];
+    unpack16<T>(lds128(base + r * 512), f);
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < C::kEpl; ++e) acc = fmaf(qs[e], f[e], acc);
+    v[r] = acc;
+  }
+  TReduce<C::kLpk, C::kLpk / 2>::run(v, lane);
+  return v[0];
+}
+
 // Where the scan puts its by-products.  shist: kSlots per-head shared-memory
 // histograms (heads bh_first .. bh_first + kSlots - 1; later heads go to the
 // global histogram directly); hist == nullptr disables counting.  keys
@@ -129,16 +173,7 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
     const int nk = min(C::kStageKeys, N - j0);
     if (bh != cur_bh) {
       cur_bh = bh;
-      const int b = bh / Hkv, h = bh % Hkv, G = Hq / Hkv;
-#pragma unroll
-      for (int e = 0; e < C::kEpl; ++e) qs[e] = 0.f;
-      for (int g = 0; g < G; ++g) {
-        const T *qp = q + ((size_t)b * Hq + (size_t)h * G + g) * D + sub * C::kEpl;
-#pragma unroll
-        for (int e = 0; e < C::kEpl; ++e) qs[e] += DT<T>::to_f(qp[e]);
-      }
-#pragma unroll
-      for (int e = 0; e < C::kEpl; ++e) qs[e] *= scale;
+      load_qbar<T, D>(q, bh, Hq, Hkv, sub, scale, qs);
     }
     if (!mbar_wait(&full[s], (i / kScanStages) & 1, status)) break;
     const unsigned char *stage = ring + (size_t)s * kScanStageBytes;
@@ -148,23 +183,12 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
     for (int wt = warp; wt < C::kWarpTiles; wt += kScanConsumerWarps) {
       const int key0 = wt * 32;
       if (key0 >= nk) break;
-      const unsigned char *base = stage + (size_t)key0 * C::kRowBytes + lane * 16;
-      float v[C::kLpk];
-#pragma unroll
-      for (int r = 0; r < C::kLpk; ++r) {
-        float f[C::kEpl];
-        unpack16<T>(lds128(base + r * 512), f);
-        float acc = 0.f;
-#pragma unroll
-        for (int e = 0; e < C::kEpl; ++e) acc = fmaf(qs[e], f[e], acc);
-        v[r] = acc;
-      }
-      TReduce<C::kLpk, C::kLpk / 2>::run(v, lane);
+      const float score = warp_tile_scores<T, D>(stage, key0, qs, lane);
       const int kk = key0 + sub * C::kKpr + lane / C::kLpk;
       const bool valid = kk < nk;
       if (valid) {
-        Srow[kk] = v[0];
-        const uint32_t key = order_key(v[0]);
+        Srow[kk] = score;
+        const uint32_t key = order_key(score);
         if (krow) krow[kk] = key;
         if (o.hist) {
           const uint32_t bin = key >> 21;
@@ -174,7 +198,7 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
             atomicAdd(&o.hist[(size_t)bh * kScanBins + bin], 1u);
         }
       }
-      if (__any_sync(0xffffffffu, valid && !isfinite(v[0])) && lane == 0)
+      if (__any_sync(0xffffffffu, valid && !isfinite(score)) && lane == 0)
         raise_flag(status, FLAG_NONFINITE);
     }
     __syncwarp();

@@ -12,13 +12,19 @@ routing set; and, for the threshold variant, the Louver summary
 ("技術サマリー：スパースアテンションを範囲検索問題として捉える", section 問題定義),
 where the kept set size varies per query.  No dataset or trained weights are
 used: q, K and V are Gaussian, with optional planted heavy-hitter keys and one
-amplified outlier channel per head.
+amplified outlier channel per head.  The Louver workload draws its keys
+around a few centres instead (a low intrinsic dimension, the structure its
+index prunes on; the summary's section 2. Louver インデックス groups keys
+into compact clusters for that reason).
 
 Draw order, per sequence b with ``numpy.random.default_rng(seeds[b])``, all as
 float32 standard normals unless stated:
   1. q_route[b]             [Hq, d]
   2. q_layers[:, b]         [L, Hq, d]
-  3. K[b, h] for h ascending [N, d] each
+  3. K[b, h] for h ascending [N, d] each; with ``blobs`` > 0 (clustered
+     keys) instead, per h: centres 2 * N(0,1) [blobs, d], each key's centre
+     as integers in [0, blobs) [N], then N(0,1) [N, d] noise scaled by
+     ``blob_spread`` and added to the key's centre
   4. V[b, h] for h ascending [N, d] each
   5. outlier channel per h  integers in [0, d)        (only if ``outlier``)
   6. heavy-hitter positions per h, uniform without replacement (``heavy`` > 0)
@@ -57,6 +63,8 @@ class Workload:
     mode: str = "topk"         # "topk" or "threshold"
     cap: int = 0               # threshold capacity per head
     tau_pct: tuple = (97, 100)  # threshold: nearest-rank percentile of scores
+    blobs: int = 0             # clustered keys: centres per KV head (0: i.i.d.)
+    blob_spread: float = 0.1   # clustered keys: noise scale around a centre
     description: str = field(default="", compare=False)
 
     @property
@@ -107,17 +115,25 @@ WORKLOADS = {
         description="threshold bf16: B=1, N=131072, Hq=32, Hkv=8, d=128, "
                     "L=16; tau per head = nearest-rank 97th percentile score; "
                     "cap 8192; 64 planted heavy hitters per head"),
+    "louver_128k": Workload(
+        "louver_128k", B=1, N=131072, Hq=32, Hkv=8, d=128, L=16,
+        mode="threshold", cap=8192, blobs=64, blob_spread=0.1, seeds=(0,),
+        description="threshold bf16 over clustered keys: B=1, N=131072, Hq=32, "
+                    "Hkv=8, d=128, L=16; keys = one of 64 centres 2*N(0,1) per "
+                    "head + 0.1*N(0,1); tau per head = nearest-rank 97th "
+                    "percentile score; cap 8192"),
 }
 
 
 def custom(B=1, N=1000, Hq=8, Hkv=2, d=64, L=2, k=16, dtype="bf16", heavy=0,
-           outlier=False, seed=0, mode="topk", cap=0) -> Workload:
+           outlier=False, seed=0, mode="topk", cap=0, blobs=0,
+           blob_spread=0.1) -> Workload:
     """A small workload for tests; sequence b uses seed + b."""
     return Workload(f"custom_B{B}_N{N}_Hq{Hq}_Hkv{Hkv}_d{d}_L{L}_{dtype}",
                     B=B, N=N, Hq=Hq, Hkv=Hkv, d=d, L=L, k=k, dtype=dtype,
                     heavy=heavy, outlier=outlier,
                     seeds=tuple(seed + b for b in range(B)), mode=mode,
-                    cap=cap)
+                    cap=cap, blobs=blobs, blob_spread=blob_spread)
 
 
 def _round(a: np.ndarray, dtype: str) -> torch.Tensor:
@@ -147,7 +163,13 @@ def generate(w: Workload, batches=None) -> dict:
         q_route[bi] = _round(rng.standard_normal((Hq, d), dtype=np.float32), w.dtype)
         q_layers[:, bi] = _round(rng.standard_normal((L, Hq, d), dtype=np.float32), w.dtype)
         for h in range(Hkv):
-            K[bi, h] = _round(rng.standard_normal((N, d), dtype=np.float32), w.dtype)
+            if w.blobs > 0:
+                cen = 2.0 * rng.standard_normal((w.blobs, d), dtype=np.float32)
+                which = rng.integers(0, w.blobs, size=N)
+                noise = rng.standard_normal((N, d), dtype=np.float32)
+                K[bi, h] = _round(cen[which] + np.float32(w.blob_spread) * noise, w.dtype)
+            else:
+                K[bi, h] = _round(rng.standard_normal((N, d), dtype=np.float32), w.dtype)
         for h in range(Hkv):
             V[bi, h] = _round(rng.standard_normal((N, d), dtype=np.float32), w.dtype)
         if w.outlier:
