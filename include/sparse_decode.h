@@ -242,12 +242,15 @@ sparse_status_t sparse_kv_append(const sparse_shape_t *shape, void *K, void *V,
  * Requirements: r a power of two in [32, 256], N a multiple of r, N / r a
  * power of two and N <= 1048576; the usual shape limits.
  *
- * Index buffer (device, caller-owned, index_bytes, 256-byte aligned):
- *   perm [B*Hkv][N] int32 (key ids in cluster order: cluster c of head bh is
- *   perm[bh][c*r .. c*r+r)), centres [B*Hkv][N/r][d] fp32, radii [B*Hkv][N/r]
- *   fp32, at the offsets 0, align256(B*Hkv*N*4), and after the centres.
- * The index describes K's first N rows; it must be rebuilt (or the keys
- * re-indexed) when those rows change.
+ * Index buffer (device, caller-owned, index_bytes, 256-byte aligned), each
+ * part at the next 256-byte boundary after the one before:
+ *   perm [B*Hkv][N] int32: key ids in cluster order (cluster c of head bh is
+ *        perm[bh][c*r .. c*r+r));
+ *   centres [B*Hkv][N/r][d] fp32;  radii [B*Hkv][N/r] fp32;
+ *   keys [B*Hkv][N][d] of the cache's dtype: row p of head bh is key
+ *        perm[bh][p], so that each cluster's keys are contiguous.
+ * The index describes K's first N rows and holds a copy of them; it must be
+ * rebuilt when those rows change.
  * Workspace: ws_bytes from sparse_louver_sizes, zero-filled once before first
  * use like the other workspaces.  Build and query calls may share one
  * (ordered), but it must not be shared with the other entry points: their
@@ -269,18 +272,19 @@ sparse_status_t sparse_louver_build(const sparse_shape_t *shape, const void *K, 
                                     void *index, size_t index_bytes, void *ws,
                                     size_t ws_bytes, void *stream);
 
-/* Threshold routing through the index: the same set as
- * sparse_route_threshold (identical scores, keys with S >= tau[b,h]) in
+/* Threshold routing through the index (which holds the keys; K is not
+ * read): the same set as sparse_route_threshold on the indexed keys
+ * (identical scores, keys with S >= tau[b,h]) in
  * ascending order in idx [B,Hkv,cap], its size in count [B,Hkv]
  * (SPARSE_ERR_CAPACITY is reported through the status word when a count
  * exceeds cap, as there).  A cluster is skipped only when its ball bound
  * <qbar,c> + |qbar| rho is below tau - (1e-4 |tau| + 1e-6) - 1e-5 |qbar|
  * (|c| + rho), a margin above the fp32 rounding of any member's score, so
  * rounding cannot drop a key.  survivors (nullable) [B,Hkv] int32: clusters that
- * passed the ball test.  q [B,Hq,d] and K of the shape's dtype. */
+ * passed the ball test.  q [B,Hq,d] of the shape's dtype; the shape is the
+ * one the index was built for (Hq may differ; n_cap is not used). */
 sparse_status_t sparse_louver_route_threshold(const sparse_shape_t *shape, const void *q,
-                                              const void *K, const void *index,
-                                              size_t index_bytes, int32_t r,
+                                              const void *index, size_t index_bytes, int32_t r,
                                               const float *tau, int32_t cap, int32_t *idx,
                                               int32_t *count, int32_t *survivors, void *ws,
                                               size_t ws_bytes, void *stream);

@@ -129,3 +129,44 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(sd, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         sd.load()
+
+
+def test_louver_arguments_rejected_before_device_work(lib):
+    """Louver index: r and N must give a balanced tree (r a power of two in
+    [32, 256], N / r a power of two); undersized buffers, null or misaligned
+    pointers are refused before any device work."""
+    P = ctypes.c_size_t
+    ib, wb = P(0), P(0)
+    ok = _shape(N=8192)
+    assert lib.sparse_louver_sizes(ctypes.byref(ok), 128, ctypes.byref(ib), ctypes.byref(wb)) == 0
+    # the index holds perm, centres, radii and a copy of the keys
+    BH, N, d, es = ok.B * ok.Hkv, ok.N, ok.d, 2 if ok.dtype == 1 else 4
+    assert ib.value >= BH * N * 4 + BH * (N // 128) * (d + 1) * 4 + BH * N * d * es
+    for r in (16, 48, 512):
+        assert lib.sparse_louver_sizes(ctypes.byref(ok), r, ctypes.byref(ib),
+                                       ctypes.byref(wb)) == 2
+    for n in (8192 + 128, 96 * 128):           # N not a multiple / N/r not a power of two
+        sh = _shape(N=n)
+        assert lib.sparse_louver_sizes(ctypes.byref(sh), 128, ctypes.byref(ib),
+                                       ctypes.byref(wb)) == 2
+    assert lib.sparse_louver_sizes(ctypes.byref(ok), 128, None, ctypes.byref(wb)) == 1
+    lib.sparse_louver_sizes(ctypes.byref(ok), 128, ctypes.byref(ib), ctypes.byref(wb))
+    fake = ctypes.c_void_p(0x10000)
+    big = ctypes.c_void_p(0x100000)
+    odd = ctypes.c_void_p(0x10010)              # 16- but not 256-byte aligned
+    # build: null K, misaligned index, index or workspace too small
+    assert lib.sparse_louver_build(ctypes.byref(ok), None, 128, big, ib.value, big, wb.value,
+                                   None) == 1
+    assert lib.sparse_louver_build(ctypes.byref(ok), fake, 128, odd, ib.value, big, wb.value,
+                                   None) == 1
+    assert lib.sparse_louver_build(ctypes.byref(ok), fake, 128, big, ib.value - 1, big,
+                                   wb.value, None) == 3
+    assert lib.sparse_louver_build(ctypes.byref(ok), fake, 128, big, ib.value, big,
+                                   wb.value - 1, None) == 3
+    # query: cap < 1, null tau, unsupported r
+    assert lib.sparse_louver_route_threshold(ctypes.byref(ok), fake, big, ib.value, 128, fake,
+                                             0, fake, fake, None, big, wb.value, None) == 1
+    assert lib.sparse_louver_route_threshold(ctypes.byref(ok), fake, big, ib.value, 128, None,
+                                             8, fake, fake, None, big, wb.value, None) == 1
+    assert lib.sparse_louver_route_threshold(ctypes.byref(ok), fake, big, ib.value, 100, fake,
+                                             8, fake, fake, None, big, wb.value, None) == 2

@@ -54,12 +54,14 @@ def _check_index(ix, K32, r):
     """K32 [B,Hkv,N,d] fp32 (the keys the index covers)."""
     B, Hkv, N, d = K32.shape
     perm = ix.perm().cpu().numpy()
+    keys = ix.keys().float().cpu().numpy()
     cen = ix.centres().cpu().numpy().astype(np.float64)
     rad = ix.radii().cpu().numpy().astype(np.float64)
     for b in range(B):
         for h in range(Hkv):
             p = perm[b, h]
             assert np.array_equal(np.sort(p), np.arange(N)), "not a permutation"
+            np.testing.assert_array_equal(keys[b, h], K32[b, h][p])  # cluster-ordered copy
             members = K32[b, h][p].astype(np.float64).reshape(N // r, r, d)
             mean = members.mean(axis=1)
             np.testing.assert_allclose(cen[b, h], mean, rtol=1e-4, atol=1e-4)
@@ -94,6 +96,9 @@ CASES = [
     dict(B=2, N=4096, Hq=4, Hkv=2, d=64, dtype="f32", r=64, blobs=8, pct=90),
     dict(B=1, N=16384, Hq=16, Hkv=4, d=128, dtype="bf16", r=256, blobs=0, pct=99),
     dict(B=1, N=2048, Hq=2, Hkv=1, d=64, dtype="bf16", r=32, blobs=4, pct=50),
+    # more than 16 heads: each head's clusters owned by CTAs of that head only
+    dict(B=3, N=2048, Hq=8, Hkv=8, d=64, dtype="bf16", r=64, blobs=4, pct=90),
+    dict(B=5, N=4096, Hq=16, Hkv=4, d=128, dtype="f32", r=128, blobs=8, pct=97),
 ]
 
 

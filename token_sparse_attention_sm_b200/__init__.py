@@ -105,7 +105,7 @@ def load():
             "sparse_kv_append": (I32, [SH, P, P, P, P, P]),
             "sparse_louver_sizes": (I32, [SH, I32, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
             "sparse_louver_build": (I32, [SH, P, I32, P, SZ, P, SZ, P]),
-            "sparse_louver_route_threshold": (I32, [SH, P, P, P, SZ, I32, P, I32, P, P, P, P,
+            "sparse_louver_route_threshold": (I32, [SH, P, P, SZ, I32, P, I32, P, P, P, P,
                                                     SZ, P]),
         }
         for name, (res, args) in sigs.items():
@@ -495,6 +495,16 @@ class LouverIndex:
         n = self.B * self.Hkv * nc * self.d
         return self.index[c0:c0 + 4 * n].view(torch.float32).view(self.B, self.Hkv, nc, self.d)
 
+    def keys(self):
+        """Cluster-ordered key rows, [B,Hkv,N,d] (row p of head bh is key
+        perm[bh][p])."""
+        _, r0 = self._offsets()
+        al = lambda x: (x + 255) // 256 * 256
+        k0 = r0 + al(self.B * self.Hkv * (self.N // self.r) * 4)
+        es = 4 if self.dtype == torch.float32 else 2
+        n = self.B * self.Hkv * self.N * self.d
+        return self.index[k0:k0 + es * n].view(self.dtype).view(self.B, self.Hkv, self.N, self.d)
+
     def radii(self):
         """Cluster radii, [B,Hkv,N/r] fp32."""
         _, r0 = self._offsets()
@@ -525,7 +535,8 @@ def louver_route_threshold(q, K, index: LouverIndex, tau, cap: int, check: bool 
                            return_survivors: bool = False):
     """Threshold routing through a Louver index: (idx [B,Hkv,cap], count [B,Hkv])
     -- the set route_threshold returns -- plus, if asked, survivors [B,Hkv]
-    (clusters that passed the ball test)."""
+    (clusters that passed the ball test).  K only checks that the index was
+    built for this cache: the index holds its own copy of the keys."""
     _need_cuda(q, K, tau)
     B, Ncap, Hq, Hkv, d = _dims_qk(q, K)
     if (B, Hkv, Ncap, d, K.dtype) != (index.B, index.Hkv, index.Ncap, index.d, index.dtype):
@@ -537,7 +548,7 @@ def louver_route_threshold(q, K, index: LouverIndex, tau, cap: int, check: bool 
     tau = tau.float().contiguous()
     buf = index.ws.get(index.ws_bytes)
     _check(load().sparse_louver_route_threshold(
-        ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(index.index), index.index.numel(), index.r,
+        ctypes.byref(sh), _ptr(q), _ptr(index.index), index.index.numel(), index.r,
         _ptr(tau), int(cap), _ptr(idx), _ptr(count), _ptr(surv), _ptr(buf), buf.numel(),
         _stream()), "louver_route_threshold")
     if check:

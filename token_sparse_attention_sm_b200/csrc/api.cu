@@ -451,17 +451,15 @@ sparse_status_t sparse_louver_build(const sparse_shape_t *shape, const void *K, 
 }
 
 sparse_status_t sparse_louver_route_threshold(const sparse_shape_t *shape, const void *q,
-                                              const void *K, const void *index,
-                                              size_t index_bytes, int32_t r,
+                                              const void *index, size_t index_bytes, int32_t r,
                                               const float *tau, int32_t cap, int32_t *idx,
                                               int32_t *count, int32_t *survivors, void *ws,
                                               size_t ws_bytes, void *stream) {
   Shape s;
   sparse_status_t rc = sd::check_shape(shape, &s);
   if (rc != SPARSE_OK) return rc;
-  if (!q || !K || !index || !tau || !idx || !count || !ws || cap < 1)
-    return SPARSE_ERR_INVALID_ARG;
-  if (!sd::aligned(q, 16) || !sd::aligned(K, 16) || !sd::aligned(index, 256) ||
+  if (!q || !index || !tau || !idx || !count || !ws || cap < 1) return SPARSE_ERR_INVALID_ARG;
+  if (!sd::aligned(q, 16) || !sd::aligned(index, 256) ||
       !sd::aligned(tau, 4) || !sd::aligned(idx, 4) || !sd::aligned(count, 4) ||
       !sd::aligned(survivors, 4) || !sd::aligned(ws, 256))
     return SPARSE_ERR_INVALID_ARG;
@@ -469,7 +467,7 @@ sparse_status_t sparse_louver_route_threshold(const sparse_shape_t *shape, const
   size_t ib = 0, wb = 0;
   sd::louver_sizes(s, r, &ib, &wb);
   if (index_bytes < ib || ws_bytes < wb) return SPARSE_ERR_WORKSPACE;
-  return sd::from_cuda(sd::louver_query(s, q, K, r, index, tau, cap, idx, count, survivors, ws,
+  return sd::from_cuda(sd::louver_query(s, q, r, index, tau, cap, idx, count, survivors, ws,
                                         static_cast<cudaStream_t>(stream)));
 }
 

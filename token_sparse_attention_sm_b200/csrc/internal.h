@@ -107,7 +107,7 @@ bool louver_shape_ok(const Shape &s, int r);
 void louver_sizes(const Shape &s, int r, size_t *index_bytes, size_t *ws_bytes);
 cudaError_t louver_build(const Shape &s, const void *K, int r, void *index, void *ws,
                          cudaStream_t st);
-cudaError_t louver_query(const Shape &s, const void *q, const void *K, int r, const void *index,
+cudaError_t louver_query(const Shape &s, const void *q, int r, const void *index,
                          const float *tau, int cap, int *idx, int *count, int *survivors,
                          void *ws, cudaStream_t st);
 

@@ -39,6 +39,9 @@
 #include "scan.cuh"
 #include "sparse_decode.h"
 
+#include <cooperative_groups.h>
+namespace cg = cooperative_groups;
+
 namespace sd {
 namespace {
 
@@ -47,9 +50,6 @@ constexpr int kChunk = 256;       // keys per CTA in the per-node passes
 constexpr int kLvThreads = 512;   // partition / compaction / filter CTAs
 constexpr size_t kLvHeader = 4096;
 
-__device__ __forceinline__ void cp_async16(uint32_t saddr, const void *gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(gmem) : "memory");
-}
 
 template <typename T, int EPL>
 __device__ __forceinline__ void load_elems(const T *p, float (&x)[EPL]) {
@@ -57,7 +57,8 @@ __device__ __forceinline__ void load_elems(const T *p, float (&x)[EPL]) {
   for (int e = 0; e < EPL; ++e) x[e] = DT<T>::to_f(p[e]);
 }
 
-// Exclusive prefix sum over a kLvThreads block; *total = block sum.
+// Exclusive prefix sum over a block of NT threads; *total = block sum.
+template <int NT>
 __device__ uint32_t lv_block_scan(uint32_t x, uint32_t *wbuf, uint32_t *total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t inc = x;
@@ -70,7 +71,7 @@ __device__ uint32_t lv_block_scan(uint32_t x, uint32_t *wbuf, uint32_t *total) {
   if (lane == 31) wbuf[warp] = inc;
   __syncthreads();
   uint32_t pre = 0, tot = 0;
-  for (int w = 0; w < kLvThreads / 32; ++w) {
+  for (int w = 0; w < NT / 32; ++w) {
     pre += w < warp ? wbuf[w] : 0u;
     tot += wbuf[w];
   }
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(kLvThreads)
   uint32_t cnt = 0;
   for (int w = w0; w < w1; ++w) cnt += __popc(~bits[w]);
   uint32_t total;
-  uint32_t pos = lv_block_scan(cnt, wbuf, &total);
+  uint32_t pos = lv_block_scan<kLvThreads>(cnt, wbuf, &total);
   for (int w = w0; w < w1; ++w) {
     uint32_t m = ~bits[w];
     while (m) {
@@ -194,6 +195,21 @@ __global__ void __launch_bounds__(kLvThreads)
       perm_out[base + pos++] = perm[base + w * 32 + b];
     }
   }
+}
+
+// The index's cluster-ordered copy of the keys: row p of head bh is key
+// perm[bh][p]; one thread per 16-byte piece.
+template <typename T, int D>
+__global__ void gather_keys_kernel(const T *__restrict__ K, const int *__restrict__ perm, int N,
+                                   int rows, long long total_rows, T *__restrict__ keys) {
+  constexpr int CPR = D * (int)sizeof(T) / 16;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= total_rows * CPR) return;
+  const long long row = i / CPR;
+  const int part = (int)(i % CPR);
+  const long long bh = row / N;
+  const uint4 *src = reinterpret_cast<const uint4 *>(K + ((size_t)bh * rows + perm[row]) * D);
+  reinterpret_cast<uint4 *>(keys + (size_t)row * D)[part] = src[part];
 }
 
 // Centre (mean) and radius (largest distance from it, inflated) of each leaf
@@ -233,160 +249,250 @@ __global__ void __launch_bounds__(128)
   if (lane == 0) radii[cl] = sqrtf(dmax) * (1.f + 1e-5f) + 1e-6f;
 }
 
-// Ball test of every cluster of a head against its halfspace; the survivors'
-// cluster ids are appended to surv[bh][..] (any order), their number counted
-// in nsurv[bh] (zero on entry; the compaction kernel resets it).  Grid
-// (splits, heads), a warp per cluster.
+// The query's first kernel: ball tests and exact checks, results as bits in
+// the heads' bitmaps.  Grid (splits, heads), kQThreads threads, one CTA per
+// SM; CTA x of head bh owns the head's clusters x, x + splits, ...
+//  1. ball test of the owned clusters, eight lanes per cluster (64 clusters
+//     per round with all their loads in flight; the first round's before
+//     q's); survivors listed in shared memory;
+//  2. exact check of the survivors' keys in items of 32 keys, each warp
+//     taking every kQWarps-th item through its own ring of nb shared-memory
+//     slots: an item's rows are contiguous in the index's cluster-ordered key
+//     copy, so one bulk copy (TMA, completion on the slot's mbarrier) brings
+//     them in, nb - 1 items ahead of the one being scored; the rows' key ids
+//     are read one item ahead of their copy.  Scores come from the scan's
+//     warp routine with qbar formed as the scan forms it; keys >= tau are
+//     marked in the head's bitmap.
+// The compaction kernel below then turns the bitmaps into the ordered sets.
+constexpr int kQWarps = 8;
+constexpr int kQThreads = kQWarps * 32;
+constexpr int kQGroupsPerRound = kQThreads / 8;   // clusters tested at once
+constexpr int kQMaxSlots = 4;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(kLvThreads)
-    louver_filter_kernel(const T *__restrict__ q, int Hq, int Hkv, float scale,
-                         const float *__restrict__ centres, const float *__restrict__ radii,
-                         int nc, const float *__restrict__ tau, int *__restrict__ surv,
-                         int *__restrict__ nsurv, uint32_t *status) {
-  constexpr int EPL = D / 32;
-  __shared__ float qb[D];
-  __shared__ float qn;
+__global__ void __launch_bounds__(kQThreads)
+    louver_query_kernel(const T *__restrict__ q, int Hq, int Hkv, int N, float scale,
+                        const int *__restrict__ perm, const float *__restrict__ centres,
+                        const float *__restrict__ radii, const T *__restrict__ keys, int r,
+                        int nc, const float *__restrict__ tau, int nb,
+                        uint32_t *__restrict__ bitmap, int *__restrict__ nsurv,
+                        uint32_t *status) {
+  using C = ScoreCfg<T, D>;
+  constexpr int EPG = D / 8;                  // centre elements per lane of a group
+  constexpr int kItemBytes = 32 * C::kRowBytes;
+  constexpr int kSlotBytes = kItemBytes + 32 * 4;  // rows + their key ids
+  extern __shared__ __align__(128) unsigned char lv_smem[];
+  __shared__ __align__(16) float qb[D];
+  __shared__ __align__(8) uint64_t bars[kQWarps][kQMaxSlots];
+  __shared__ float qn_s;
+  __shared__ int nlist;
   const int bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int b = bh / Hkv, h = bh % Hkv, G = Hq / Hkv;
+  const int splits = gridDim.x;
+  const int mc = (nc - (int)blockIdx.x + splits - 1) / splits;  // clusters owned
+  int *list = reinterpret_cast<int *>(lv_smem + (size_t)kQWarps * nb * kSlotBytes);
+  if (lane == 0)
+    for (int i = 0; i < nb; ++i) mbar_init(&bars[warp][i], 1);
+  fence_mbar_init();
   grid_dep_wait();
   grid_dep_launch();
-  if (tid < D) {
-    float s = 0.f;
-    for (int g = 0; g < G; ++g) s += DT<T>::to_f(q[((size_t)b * Hq + (size_t)h * G + g) * D + tid]);
-    qb[tid] = s * scale;
-  }
+
+  // ---- 1. ball test
+  const int grp = tid >> 3, gl = tid & 7;
+  float4 cv[2][EPG / 4];
+  float rho[2];
+  int ci[2];
+  auto load_round = [&](int m0) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int m = m0 + u * kQGroupsPerRound + grp;
+      ci[u] = m < mc ? (int)blockIdx.x + m * splits : -1;
+      const float4 *c = reinterpret_cast<const float4 *>(
+          centres + ((size_t)bh * nc + (ci[u] < 0 ? 0 : ci[u])) * D + gl * EPG);
+#pragma unroll
+      for (int v = 0; v < EPG / 4; ++v)
+        cv[u][v] = ci[u] < 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(c + v);
+      rho[u] = ci[u] < 0 ? 0.f : __ldg(radii + (size_t)bh * nc + ci[u]);
+    }
+  };
+  load_round(0);
+  if (tid < D) qb[tid] = qbar_elem<T, D>(q, bh, Hq, Hkv, tid, scale);
+  if (tid == 0) nlist = 0;
   __syncthreads();
   if (tid < 32) {
     float s = 0.f;
     for (int i = tid; i < D; i += 32) s += qb[i] * qb[i];
     s = warp_sum(s);
-    if (tid == 0) qn = sqrtf(s);
+    if (tid == 0) qn_s = sqrtf(s);
   }
   __syncthreads();
+  const float qn = qn_s;
   const float t = tau[bh];
   if (!isfinite(t) && tid == 0 && blockIdx.x == 0) raise_flag(status, FLAG_NONFINITE);
   const float lim = t - (1e-4f * fabsf(t) + 1e-6f);
-  float qv[EPL];
+  {
+    float qv[EPG];
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) qv[e] = qb[lane * EPL + e];
-  const int nwarps = gridDim.x * (kLvThreads / 32);
-  for (int i = blockIdx.x * (kLvThreads / 32) + warp; i < nc; i += nwarps) {
-    const float *c = centres + ((size_t)bh * nc + i) * D + lane * EPL;
-    float dot = 0.f, cc = 0.f;
+    for (int e = 0; e < EPG; ++e) qv[e] = qb[gl * EPG + e];
+    for (int m0 = 0; m0 < mc; m0 += 2 * kQGroupsPerRound) {
+      if (m0 > 0) load_round(m0);
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      dot = fmaf(qv[e], c[e], dot);
-      cc = fmaf(c[e], c[e], cc);
-    }
-    dot = warp_sum(dot);
-    cc = warp_sum(cc);
-    const float rho = radii[(size_t)bh * nc + i];
-    const float ub = dot + qn * rho;
-    const float slack = 1e-5f * qn * (sqrtf(cc) + rho);
-    if (lane == 0 && (ub >= lim - slack || !(ub == ub))) {
-      const int slot = atomicAdd(&nsurv[bh], 1);
-      if (slot < nc)
-        surv[(size_t)bh * nc + slot] = i;
-      else  // the count did not start at zero (workspace not initialised)
-        raise_flag(status, FLAG_INTERNAL);
+      for (int u = 0; u < 2; ++u) {
+        float dot = 0.f, cc = 0.f;
+#pragma unroll
+        for (int v = 0; v < EPG / 4; ++v) {
+          const float4 c4 = cv[u][v];
+          dot = fmaf(qv[4 * v + 0], c4.x, dot);
+          dot = fmaf(qv[4 * v + 1], c4.y, dot);
+          dot = fmaf(qv[4 * v + 2], c4.z, dot);
+          dot = fmaf(qv[4 * v + 3], c4.w, dot);
+          cc = fmaf(c4.x, c4.x, fmaf(c4.y, c4.y, fmaf(c4.z, c4.z, fmaf(c4.w, c4.w, cc))));
+        }
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) {
+          dot += __shfl_xor_sync(0xffffffffu, dot, o);
+          cc += __shfl_xor_sync(0xffffffffu, cc, o);
+        }
+        const float ub = dot + qn * rho[u];
+        const float slack = 1e-5f * qn * (sqrtf(cc) + rho[u]);
+        if (gl == 0 && ci[u] >= 0 && (ub >= lim - slack || !(ub == ub)))
+          list[atomicAdd(&nlist, 1)] = ci[u];
+      }
     }
   }
-}
+  __syncthreads();
+  const int ns = nlist;
+  if (tid == 0 && ns) atomicAdd(&nsurv[bh], ns);
 
-// Exact check of the surviving clusters: their rows are gathered into shared
-// memory as one scan tile and scored by the scan's warp routine (the same
-// per-key arithmetic, so the same bits); keys at or above tau are marked in
-// the head's bitmap.  Grid (splits, heads); four warps per CTA.
-template <typename T, int D>
-__global__ void __launch_bounds__(128)
-    louver_exact_kernel(const T *__restrict__ q, const T *__restrict__ K, int Hq, int Hkv,
-                        int N, int rows, float scale, const int *__restrict__ perm, int r,
-                        const int *__restrict__ surv, const int *__restrict__ nsurv, int nc,
-                        const float *__restrict__ tau, uint32_t *__restrict__ bitmap,
-                        uint32_t *status) {
-  using C = ScoreCfg<T, D>;
-  constexpr int CPR = C::kRowBytes / 16;  // 16-byte pieces per row
-  extern __shared__ __align__(128) unsigned char tile[];
-  const int bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int sub = lane % C::kLpk;
-  grid_dep_wait();
-  grid_dep_launch();
+  // ---- 2. exact check, 32 keys per item, a private ring of slots per warp
   float qs[C::kEpl];
-  load_qbar<T, D>(q, bh, Hq, Hkv, sub, scale, qs);
-  const uint32_t tkey = order_key(tau[bh]);
-  const int ns = min(nsurv[bh], nc);
-  const int *pbase = perm + (size_t)bh * N;
+#pragma unroll
+  for (int e = 0; e < C::kEpl; ++e) qs[e] = qb[(lane % C::kLpk) * C::kEpl + e];
+  const uint32_t tkey = order_key(t);
+  const int ipc = r / 32;  // items per cluster
+  const int nitems = ns * ipc;
+  unsigned char *wb = lv_smem + (size_t)warp * nb * kSlotBytes;
+  const size_t head0 = (size_t)bh * nc * r;  // the head's first cluster-ordered row
   uint32_t *bm = bitmap + (size_t)bh * (N / 32);
-  const uint32_t tile_s = smem_u32(tile);
-  for (int i = blockIdx.x; i < ns; i += gridDim.x) {
-    const int cl = surv[(size_t)bh * nc + i];
-    if ((unsigned)cl >= (unsigned)nc) {  // uniform across the CTA
-      if (tid == 0) raise_flag(status, FLAG_INTERNAL);
-      continue;
+  // cluster-ordered row of row 0 of item it
+  auto item_row = [&](int it) -> size_t {
+    return head0 + (size_t)list[it / ipc] * r + (it % ipc) * 32;
+  };
+  // key id of row `lane` of item it (0 past the end)
+  auto load_id = [&](int it) -> int { return it < nitems ? __ldg(perm + item_row(it) + lane) : 0; };
+  // item it's rows into slot `slot` (its key ids j, one per lane)
+  auto issue = [&](int it, int slot, int j) {
+    if (it < nitems) {
+      unsigned char *dst = wb + slot * kSlotBytes;
+      reinterpret_cast<int *>(dst + kItemBytes)[lane] = j;
+      if (lane == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // slot reuse
+        mbar_arrive_expect_tx(&bars[warp][slot], kItemBytes);
+        bulk_g2s(dst, keys + item_row(it) * D, kItemBytes, &bars[warp][slot]);
+      }
     }
-    const int *cp = pbase + (size_t)cl * r;
-    for (int c = tid; c < r * CPR; c += 128) {
-      const int row = c / CPR, part = c % CPR;
-      cp_async16(tile_s + row * C::kRowBytes + part * 16,
-                 reinterpret_cast<const unsigned char *>(K + ((size_t)bh * rows + cp[row]) * D) +
-                     part * 16);
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncthreads();
-    for (int wt = warp; wt < r / 32; wt += 4) {
-      const float score = warp_tile_scores<T, D>(tile, wt * 32, qs, lane);
-      const int kk = wt * 32 + sub * C::kKpr + lane / C::kLpk;
-      const int j = cp[kk];
-      if (order_key(score) >= tkey) atomicOr(&bm[j >> 5], 1u << (j & 31));
-      if (__any_sync(0xffffffffu, !isfinite(score)) && lane == 0)
-        raise_flag(status, FLAG_NONFINITE);
-    }
-    __syncthreads();  // the tile is read before the next gather
+  };
+  __syncwarp();
+  int jn = load_id(warp);
+  for (int p = 0; p < nb - 1; ++p) {
+    const int j = jn;
+    jn = load_id(warp + (p + 1) * kQWarps);
+    issue(warp + p * kQWarps, p, j);
   }
+  int kfail = -1;
+  for (int k = 0, it = warp; it < nitems; ++k, it += kQWarps) {
+    const int itn = it + (nb - 1) * kQWarps;
+    const int j = jn;
+    jn = load_id(itn + kQWarps);
+    issue(itn, (k + nb - 1) % nb, j);
+    const int slot = k % nb;
+    const bool ok = mbar_wait(&bars[warp][slot], (uint32_t)((k / nb) & 1), status);
+    if (!__all_sync(0xffffffffu, ok)) {  // expired wait (flagged): stop
+      kfail = k;
+      break;
+    }
+    __syncwarp();
+    const unsigned char *sp = wb + slot * kSlotBytes;
+    const float score = warp_tile_scores<T, D>(sp, 0, qs, lane);
+    const int row = (lane % C::kLpk) * C::kKpr + lane / C::kLpk;
+    const int jk = reinterpret_cast<const int *>(sp + kItemBytes)[row];
+    if (order_key(score) >= tkey) atomicOr(&bm[jk >> 5], 1u << (jk & 31));
+    if (__any_sync(0xffffffffu, !isfinite(score)) && lane == 0)
+      raise_flag(status, FLAG_NONFINITE);
+    __syncwarp();  // the slot is read before it is refilled
+  }
+  // after an expired wait, the copies issued and not consumed (items kfail
+  // .. kfail + nb - 1) are waited for, again with a limit, before exit
+  if (kfail >= 0)
+    for (int k2 = kfail; k2 < kfail + nb && warp + k2 * kQWarps < nitems; ++k2)
+      mbar_wait(&bars[warp][k2 % nb], (uint32_t)((k2 / nb) & 1), status);
 }
 
-// Bitmap -> ascending indices (the first cap), count; clears the bitmap and
-// the survivor count for the next query.
-__global__ void __launch_bounds__(kLvThreads)
+// Bitmap -> ascending indices.  One thread-block cluster of kCSlices CTAs
+// per head; CTA c owns the c-th contiguous slice of the head's bitmap words.
+// Each CTA counts its slice's set bits, the counts are exchanged through
+// distributed shared memory after a cluster barrier (so no CTA reads another
+// slice's words, and each may clear its own), and each CTA then writes its
+// slice's indices from its base (the first cap of the head).  The last CTA
+// writes the head's count and survivor count and resets the latter.
+constexpr int kCSlices = 8;
+constexpr int kCThreads = 256;
+
+__global__ void __launch_bounds__(kCThreads)
     louver_compact_kernel(uint32_t *__restrict__ bitmap, int N, int cap, int *__restrict__ idx,
                           int *__restrict__ count, int *__restrict__ nsurv,
                           int *__restrict__ survivors_out, uint32_t *status) {
-  __shared__ uint32_t wbuf[kLvThreads / 32];
-  const int bh = blockIdx.x, tid = threadIdx.x, nw = N / 32;
+  cg::cluster_group cluster = cg::this_cluster();
+  __shared__ uint32_t wbuf[kCThreads / 32];
+  __shared__ uint32_t slice_total;
+  const int rank = (int)cluster.block_rank();
+  const int bh = blockIdx.y, tid = threadIdx.x;
+  const int nw = N / 32;
+  const int per_slice = (nw + kCSlices - 1) / kCSlices;
+  const int s0 = min(nw, rank * per_slice), s1 = min(nw, s0 + per_slice);
+  const int wpt = (s1 - s0 + kCThreads - 1) / kCThreads;
+  const int r0 = min(s1, s0 + tid * wpt), r1 = min(s1, r0 + wpt);
   grid_dep_wait();
   grid_dep_launch();
   uint32_t *bm = bitmap + (size_t)bh * nw;
-  const int per = (nw + kLvThreads - 1) / kLvThreads;
-  const int w0 = min(nw, tid * per), w1 = min(nw, w0 + per);
   uint32_t cnt = 0;
-  for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+  for (int wi = r0; wi < r1; ++wi) cnt += __popc(__ldcg(bm + wi));
   uint32_t total;
-  uint32_t pos = lv_block_scan(cnt, wbuf, &total);
+  const uint32_t off = lv_block_scan<kCThreads>(cnt, wbuf, &total);
+  if (tid == 0) slice_total = total;
+  cluster.sync();
+  uint32_t base = 0, head_total = 0;
+  for (int c = 0; c < kCSlices; ++c) {
+    const uint32_t v = *cluster.map_shared_rank(&slice_total, c);
+    base += c < rank ? v : 0u;
+    head_total += v;
+  }
+  uint32_t pos = base + off;
   int *out = idx + (size_t)bh * cap;
-  for (int w = w0; w < w1; ++w) {
-    uint32_t m = bm[w];
-    bm[w] = 0u;
+  for (int wi = r0; wi < r1; ++wi) {
+    uint32_t m = __ldcg(bm + wi);
+    if (m) bm[wi] = 0u;
     while (m) {
-      const int b = __ffs(m) - 1;
+      const int bit = __ffs(m) - 1;
       m &= m - 1u;
-      if (pos < (uint32_t)cap) out[pos] = w * 32 + b;
+      if (pos < (uint32_t)cap) out[pos] = wi * 32 + bit;
       ++pos;
     }
   }
-  if (tid == 0) {
-    count[bh] = (int)total;
-    if (total > (uint32_t)cap) raise_flag(status, FLAG_CAPACITY);
-    if (survivors_out) survivors_out[bh] = nsurv[bh];
+  if (rank == kCSlices - 1 && tid == 0) {
+    count[bh] = (int)head_total;
+    if (head_total > (uint32_t)cap) raise_flag(status, FLAG_CAPACITY);
+    const int sv = __ldcg(nsurv + bh);
+    if (survivors_out) survivors_out[bh] = sv;
     nsurv[bh] = 0;
   }
+  cluster.sync();  // no CTA leaves while another may read its shared memory
 }
 
 // ---- host side ----------------------------------------------------------------
 
 struct LvLayout {
-  size_t perm, centres, radii, index_total;                            // index
-  size_t sums, va, vb, proj, perm2, sel, bitmap, surv, nsurv, ws_total;  // workspace
+  size_t perm, centres, radii, keys, index_total;                      // index
+  size_t sums, va, vb, proj, perm2, sel, bitmap, nsurv, ws_total;  // workspace
 };
 
 size_t lv_align(size_t x) { return (x + 255) / 256 * 256; }
@@ -404,7 +510,8 @@ LvLayout lv_layout(const Shape &s, int r) {
   l.perm = 0;
   l.centres = lv_align(BH * N * 4);
   l.radii = l.centres + lv_align(BH * nc * d * 4);
-  l.index_total = l.radii + lv_align(BH * nc * 4);
+  l.keys = l.radii + lv_align(BH * nc * 4);
+  l.index_total = l.keys + lv_align(BH * N * d * (size_t)s.esize());
   const size_t nseg = BH * N / r;  // bound on the segments of any level
   l.sums = kLvHeader;
   l.va = l.sums + lv_align(nseg * d * 4);
@@ -413,8 +520,7 @@ LvLayout lv_layout(const Shape &s, int r) {
   l.perm2 = l.proj + lv_align(BH * N * 4);
   l.sel = l.perm2 + lv_align(BH * N * 4);
   l.bitmap = l.sel + lv_align(BH * N / 2 * 4 + 4);
-  l.surv = l.bitmap + lv_align(BH * N / 32 * 4);
-  l.nsurv = l.surv + lv_align(BH * nc * 4);
+  l.nsurv = l.bitmap + lv_align(BH * N / 32 * 4);
   l.ws_total = l.nsurv + lv_align(BH * 4);
   return l;
 }
@@ -476,6 +582,11 @@ cudaError_t lv_build_t(const Shape &s, const void *Kv, int r, char *index, char 
   if (e == cudaSuccess && cur != perm)
     e = cudaMemcpyAsync(perm, cur, (size_t)total * 4, cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return e;
+  constexpr int CPR = D * (int)sizeof(T) / 16;
+  gather_keys_kernel<T, D><<<(unsigned)((total * CPR + 255) / 256), 256, 0, st>>>(
+      K, perm, s.N, s.Ncap, total, reinterpret_cast<T *>(index + l.keys));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   const long long ncl = total / r;
   bounds_kernel<T, D><<<(unsigned)((ncl + 3) / 4), 128, 0, st>>>(
       K, perm, r, s.N, s.Ncap, ncl, reinterpret_cast<float *>(index + l.centres),
@@ -484,65 +595,62 @@ cudaError_t lv_build_t(const Shape &s, const void *Kv, int r, char *index, char 
 }
 
 template <typename T, int D>
-cudaError_t lv_query_t(const Shape &s, const void *qv, const void *Kv, int r, const char *index,
-                       const float *tau, int cap, int *idx, int *count, int *survivors,
-                       char *ws, cudaStream_t st) {
+cudaError_t lv_query_t(const Shape &s, const void *qv, int r, const char *index, const float *tau,
+                       int cap, int *idx, int *count, int *survivors, char *ws, cudaStream_t st) {
   using C = ScoreCfg<T, D>;
-  const T *q = static_cast<const T *>(qv);
-  const T *K = static_cast<const T *>(Kv);
   const LvLayout l = lv_layout(s, r);
   const int nc = s.N / r;
   const float scale = (float)(1.0 / __builtin_sqrt((double)D));
-  uint32_t *status = reinterpret_cast<uint32_t *>(ws);
-  int *surv = reinterpret_cast<int *>(ws + l.surv);
-  int *nsurv = reinterpret_cast<int *>(ws + l.nsurv);
-  uint32_t *bitmap = reinterpret_cast<uint32_t *>(ws + l.bitmap);
-  const int *perm = reinterpret_cast<const int *>(index + l.perm);
+  DeviceInfo di;
+  cudaError_t e = device_info(&di);
+  if (e != cudaSuccess) return e;
+  // one CTA per SM over all heads (one wave); clusters dealt round-robin to
+  // a head's CTAs
+  int splits = di.sm_count / s.BH();
+  splits = splits < 1 ? 1 : (splits > nc ? nc : splits);
+  const int mc = (nc + splits - 1) / splits;
+  const size_t slot = 32 * (size_t)C::kRowBytes + 32 * 4;
+  const size_t list_bytes = (size_t)mc * sizeof(int);
+  // as many slots per warp as fit next to the static shared memory, up to 4
+  const size_t static_smem = 2048;
+  int nb = (int)(((size_t)di.max_smem_optin - static_smem - list_bytes) / (kQWarps * slot));
+  nb = nb > kQMaxSlots ? kQMaxSlots : nb;
+  if (nb < 1) return cudaErrorNotSupported;
+  const size_t smem = kQWarps * nb * slot + list_bytes;
+  auto kern = louver_query_kernel<T, D>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attrs[1];
   cfg.attrs = attrs;
   cfg.stream = st;
-  DeviceInfo di;
-  cudaError_t e = device_info(&di);
-  if (e != cudaSuccess) return e;
-  // ball test
-  int fsplit = (di.sm_count + s.BH() - 1) / s.BH();
-  const int fmax = (nc + kLvThreads / 32 - 1) / (kLvThreads / 32);
-  fsplit = fsplit < 1 ? 1 : (fsplit > fmax ? fmax : fsplit);
-  cfg.gridDim = dim3((unsigned)fsplit, (unsigned)s.BH(), 1);
-  cfg.blockDim = dim3(kLvThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.numAttrs = 0;
-  add_pdl_attr(cfg, attrs);
-  e = cudaLaunchKernelEx(&cfg, louver_filter_kernel<T, D>, q, s.Hq, s.Hkv, scale,
-                         reinterpret_cast<const float *>(index + l.centres),
-                         reinterpret_cast<const float *>(index + l.radii), nc, tau, surv, nsurv,
-                         status);
-  if (e != cudaSuccess) return e;
-  // exact check of the survivors
-  const int smem = r * C::kRowBytes;
-  auto kx = louver_exact_kernel<T, D>;
-  e = cudaFuncSetAttribute(kx, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  int splits = (4 * di.sm_count + s.BH() - 1) / s.BH();
-  splits = splits < 1 ? 1 : (splits > nc ? nc : splits);
   cfg.gridDim = dim3((unsigned)splits, (unsigned)s.BH(), 1);
-  cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.blockDim = dim3(kQThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
   cfg.numAttrs = 0;
   add_pdl_attr(cfg, attrs);
-  e = cudaLaunchKernelEx(&cfg, kx, q, K, s.Hq, s.Hkv, s.N, s.Ncap, scale, perm, r,
-                         static_cast<const int *>(surv), static_cast<const int *>(nsurv), nc,
-                         tau, bitmap, status);
+  e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(qv), s.Hq, s.Hkv, s.N, scale,
+                         reinterpret_cast<const int *>(index + l.perm),
+                         reinterpret_cast<const float *>(index + l.centres),
+                         reinterpret_cast<const float *>(index + l.radii),
+                         reinterpret_cast<const T *>(index + l.keys), r, nc, tau, nb,
+                         reinterpret_cast<uint32_t *>(ws + l.bitmap),
+                         reinterpret_cast<int *>(ws + l.nsurv), reinterpret_cast<uint32_t *>(ws));
   if (e != cudaSuccess) return e;
-  // ordered compaction
-  cfg.gridDim = dim3((unsigned)s.BH(), 1, 1);
-  cfg.blockDim = dim3(kLvThreads, 1, 1);
+  cudaLaunchAttribute cattrs[2];
+  cattrs[0].id = cudaLaunchAttributeClusterDimension;
+  cattrs[0].val.clusterDim.x = kCSlices;
+  cattrs[0].val.clusterDim.y = 1;
+  cattrs[0].val.clusterDim.z = 1;
+  cfg.attrs = cattrs;
+  cfg.gridDim = dim3((unsigned)kCSlices, (unsigned)s.BH(), 1);
+  cfg.blockDim = dim3(kCThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
-  cfg.numAttrs = 0;
-  add_pdl_attr(cfg, attrs);
-  e = cudaLaunchKernelEx(&cfg, louver_compact_kernel, bitmap, s.N, cap, idx, count, nsurv,
-                         survivors, status);
+  cfg.numAttrs = 1;
+  add_pdl_attr(cfg, cattrs);
+  e = cudaLaunchKernelEx(&cfg, louver_compact_kernel, reinterpret_cast<uint32_t *>(ws + l.bitmap),
+                         s.N, cap, idx, count, reinterpret_cast<int *>(ws + l.nsurv), survivors,
+                         reinterpret_cast<uint32_t *>(ws));
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -568,19 +676,17 @@ cudaError_t louver_build(const Shape &s, const void *K, int r, void *index, void
                     : lv_build_t<float, 64>(s, K, r, ix, w, st);
 }
 
-cudaError_t louver_query(const Shape &s, const void *q, const void *K, int r, const void *index,
+cudaError_t louver_query(const Shape &s, const void *q, int r, const void *index,
                          const float *tau, int cap, int *idx, int *count, int *survivors,
                          void *ws, cudaStream_t st) {
   const char *ix = static_cast<const char *>(index);
   char *w = static_cast<char *>(ws);
   if (s.dtype == 1)
-    return s.d == 128 ? lv_query_t<__nv_bfloat16, 128>(s, q, K, r, ix, tau, cap, idx, count,
-                                                       survivors, w, st)
-                      : lv_query_t<__nv_bfloat16, 64>(s, q, K, r, ix, tau, cap, idx, count,
-                                                      survivors, w, st);
-  return s.d == 128 ? lv_query_t<float, 128>(s, q, K, r, ix, tau, cap, idx, count, survivors, w, st)
-                    : lv_query_t<float, 64>(s, q, K, r, ix, tau, cap, idx, count, survivors, w,
-                                            st);
+    return s.d == 128
+               ? lv_query_t<__nv_bfloat16, 128>(s, q, r, ix, tau, cap, idx, count, survivors, w, st)
+               : lv_query_t<__nv_bfloat16, 64>(s, q, r, ix, tau, cap, idx, count, survivors, w, st);
+  return s.d == 128 ? lv_query_t<float, 128>(s, q, r, ix, tau, cap, idx, count, survivors, w, st)
+                    : lv_query_t<float, 64>(s, q, r, ix, tau, cap, idx, count, survivors, w, st);
 }
 
 }  // namespace sd

@@ -59,8 +59,20 @@ struct TReduce<R, 0> {
   static __device__ __forceinline__ void run(float *, int) {}
 };
 
-// This lane's slice of qbar (the group's query rows summed in fp32, then
-// scaled): lane `sub` of a row holds elements sub*kEpl .. sub*kEpl+kEpl-1.
+// Element i of qbar for head bh: the group's query rows summed in fp32 in
+// head order, then scaled.  Every kernel whose scores must agree bit for bit
+// with the scan forms qbar this way.
+template <typename T, int D>
+__device__ __forceinline__ float qbar_elem(const T *__restrict__ q, int bh, int Hq, int Hkv,
+                                           int i, float scale) {
+  const int b = bh / Hkv, h = bh % Hkv, G = Hq / Hkv;
+  float s = 0.f;
+  for (int g = 0; g < G; ++g) s += DT<T>::to_f(q[((size_t)b * Hq + (size_t)h * G + g) * D + i]);
+  return s * scale;
+}
+
+// This lane's slice of qbar: lane `sub` of a row holds elements
+// sub*kEpl .. sub*kEpl+kEpl-1 (the same arithmetic as qbar_elem).
 template <typename T, int D>
 __device__ __forceinline__ void load_qbar(const T *__restrict__ q, int bh, int Hq, int Hkv,
                                           int sub, float scale,
