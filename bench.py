@@ -495,10 +495,18 @@ def run_reference(args, rank, world):
     K_all = synth.f32(x["K"][:1, :1])
     V_all = synth.f32(x["V"][:1, :1])
 
+    threshold = w.mode == "threshold"
+
     def sample(n):
         kk = max(1, round(w.k * n / w.N))
+        if threshold:  # tau of the sample's own scores (untimed set-up)
+            tau = oracle.percentile_tau(oracle.scores(qr, K_all[:, :, :n]), *w.tau_pct)
+            capn = max(1, round(w.cap * n / w.N))
         t0 = time.perf_counter()
-        oracle.decode_step(qr, ql, K_all[:, :, :n], V_all[:, :, :n], k=kk)
+        if threshold:
+            oracle.decode_step(qr, ql, K_all[:, :, :n], V_all[:, :, :n], tau=tau, cap=capn)
+        else:
+            oracle.decode_step(qr, ql, K_all[:, :, :n], V_all[:, :, :n], k=kk)
         return time.perf_counter() - t0
 
     t_full_head = sample(w.N)                       # calibration, untimed
@@ -512,11 +520,14 @@ def run_reference(args, rank, world):
     sec = time.perf_counter() - t0
     frac = (n / w.N) / (w.B * w.Hkv)                # share of one full step
     value = args.steps * frac / sec
+    sel = (f"tau = {w.tau_pct[0]}th-percentile score, cap {max(1, round(w.cap * n / w.N))}"
+           if threshold else f"k={max(1, round(w.k * n / w.N))}")
     desc = (f"{args.steps} samples, each the oracle decode step of one KV head "
             f"(G={G} query heads, L={w.L}) over the first {n} of {w.N} keys with "
-            f"k={max(1, round(w.k * n / w.N))}; value scaled by {frac:.3g} step per sample")
+            f"{sel}; value scaled by {frac:.3g} step per sample")
     return {
-        "metric": METRIC, "value": round(value, 5), "unit": "steps/s", "n_gpus": world,
+        "metric": LOUVER_METRIC if args.louver else METRIC, "value": round(value, 5),
+        "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 / value, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
@@ -531,6 +542,249 @@ def run_reference(args, rank, world):
     }
 
 
+# ---------------------------------------------------------------------------
+# Louver-index threshold step
+# ---------------------------------------------------------------------------
+
+LOUVER_METRIC = ("128K-context threshold sparse decode steps/s through the Louver index "
+                 "(16 layers, tau = 97th-percentile score per head)")
+
+
+def percentile_tau_device(sd, q_route, K, ws, num=97, den=100):
+    """tau per (sequence, KV head): the nearest-rank num/den percentile of the
+    head's routing scores (the library's scores; workload set-up, untimed)."""
+    S = sd.score(q_route, K, ws=ws)
+    N = S.shape[-1]
+    rank = -(-num * N // den)
+    return torch.kthvalue(S, rank, dim=-1).values.contiguous()
+
+
+def run_native_louver(args, rank, world, local_rank):
+    """One step = threshold routing through the Louver index (ball tests,
+    exact checks of the surviving clusters, ordered compaction) and the
+    attention of all L layers over that set.  The full-scan threshold step
+    (score scan, threshold select, attention) is timed beside it."""
+    import token_sparse_attention_sm_b200 as sd
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    base = synth.WORKLOADS[args.workload]
+    w = base.with_(seeds=tuple(s + 1000 * rank for s in base.seeds))
+    r = args.louver
+    x = synth.generate(w)
+    variants = synth.query_variants(w, x, QUERY_SETS, seed=2000 + 1000 * rank)
+    K = x["K"].to(dev)
+    V = x["V"].to(dev)
+    qs = [(qr.to(dev), ql.to(dev)) for qr, ql in variants]
+    stream = torch.cuda.Stream(device=dev)
+    ws = sd.Workspace(dev)
+    ws.get(sd.workspace_bytes(w.B, w.N, w.Hq, w.Hkv, w.d, w.torch_dtype, w.cap, w.L))
+    cap = w.cap
+    with torch.cuda.stream(stream):
+        taus = [percentile_tau_device(sd, qr, K, ws, *w.tau_pct) for qr, _ in qs]
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        ix = sd.louver_build(K, r)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        build_ms = ev0.elapsed_time(ev1)
+        outs = [dict(out=torch.empty_like(ql),
+                     idx=torch.empty((w.B, w.Hkv, cap), dtype=torch.int32, device=dev),
+                     count=torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev),
+                     surv=torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev),
+                     lse=torch.empty((w.L, w.B, w.Hq), dtype=torch.float32, device=dev))
+                for _, ql in qs]
+
+        def route_fn(i):
+            o = outs[i]
+            return lambda: sd.louver_route_threshold(qs[i][0], K, ix, taus[i], cap, check=False,
+                                                     idx=o["idx"], count=o["count"])
+
+        def attn_fn(i):
+            o = outs[i]
+            return lambda: sd.attn_gather(qs[i][1], K, V, o["idx"], count=o["count"], ws=ws,
+                                          check=False, out=o["out"], lse=o["lse"])
+
+        def step_fn(i):
+            a, b = route_fn(i), attn_fn(i)
+            return lambda: (a(), b())
+
+        def full_fn(i):
+            o = outs[i]
+            return lambda: sd.decode_step(qs[i][0], qs[i][1], K, V, tau=taus[i], cap=cap, ws=ws,
+                                          check=False, out=o["out"], idx=o["idx"],
+                                          count=o["count"], lse=o["lse"])
+
+        # survivors and set sizes per query set (untimed); equality with the
+        # full-scan set is the tests' business, the sizes are reported here
+        surv, counts = [], []
+        for i in range(len(qs)):
+            sd.louver_route_threshold(qs[i][0], K, ix, taus[i], cap, check=True,
+                                      return_survivors=True, idx=outs[i]["idx"],
+                                      count=outs[i]["count"], survivors=outs[i]["surv"])
+            surv.append(outs[i]["surv"].cpu())
+            counts.append(outs[i]["count"].cpu())
+            step_fn(i)()
+            full_fn(i)()
+        sd.read_device_status(ws)
+        sd.read_device_status(ix.ws)
+        graphs = capture([step_fn(i) for i in range(len(qs))], stream)
+        loop = capture_loop([step_fn(i) for i in range(len(qs))], stream)
+        with ClockSampler(local_rank) as cs:
+            ms = time_steps(loop, graphs, args.steps, args.warmup, stream, cs)
+        clocks = cs.result()
+        sd.read_device_status(ws)
+        sd.read_device_status(ix.ws)
+        n_k = max(args.steps // 4, 64)
+        wk = max(args.warmup, 3)
+        t_route = time_graphs(capture([route_fn(i) for i in range(len(qs))], stream), n_k, wk,
+                              stream) / n_k
+        t_attn = time_graphs(capture([attn_fn(i) for i in range(len(qs))], stream), n_k, wk,
+                             stream) / n_k
+        full_one = capture([full_fn(i) for i in range(len(qs))], stream)
+        full_loop = capture_loop([full_fn(i) for i in range(len(qs))], stream)
+        ms_full = time_steps(full_loop, full_one, n_k, wk, stream) / n_k
+        full_route = capture([lambda i=i: sd.route_threshold(qs[i][0], K, taus[i], cap, ws=ws,
+                                                             check=False)
+                              for i in range(len(qs))], stream)
+        t_full_route = time_graphs(full_route, n_k, wk, stream) / n_k
+        sd.read_device_status(ws)
+        sd.read_device_status(ix.ws)
+
+    ms_max = sdist.max_over_ranks(ms)
+    t_route_max = sdist.max_over_ranks(t_route)
+    ms_per_step = ms_max / args.steps
+    value = world * args.steps / (ms_max / 1e3)
+    e2e = run_e2e_louver(sd, w, variants, K, V, ix, taus, ws, stream, dev, args, world)
+
+    peak, peak_src = load_peaks()
+    nc = w.N // r
+    BH = w.B * w.Hkv
+    mean_surv = float(np.mean([s.sum().item() for s in surv]))
+    mean_count = float(np.mean([np.minimum(c.numpy(), cap).sum() for c in counts]))
+    route_b = (BH * nc * (w.d + 1) * 4 + mean_surv * r * (w.d * w.esize + 4) + mean_count * 4)
+    attn_b = 2 * mean_count * w.d * w.esize
+    achieved = route_b / (t_route_max * 1e-3) / 1e9
+    line = {
+        "metric": LOUVER_METRIC,
+        "value": round(value, 2),
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded clustered keys: 64 centres per head plus noise; Gaussian q, V)",
+        "config": {
+            "workload": w.name, "B": w.B, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+            "L": w.L, "cap": cap, "tau": "nearest-rank 97th percentile score per head",
+            "louver_r": r, "parallelism": f"replicas x{world}", "query_sets": QUERY_SETS,
+            "l2": "inputs larger than L2 (K+V = %.0f MB, index keys %.0f MB per replica); the "
+                  "query rotates over %d sets" % (2 * BH * w.N * w.d * w.esize / 1e6,
+                                                    BH * w.N * w.d * w.esize / 1e6, QUERY_SETS),
+            "timing": "steps replayed as CUDA graphs of %d consecutive steps; CUDA events on "
+                      "the launch stream; max over ranks" % QUERY_SETS,
+            "index_build_ms": round(build_ms, 3),
+            "surviving_clusters_per_query": round(mean_surv, 1),
+            "clusters_per_query": BH * nc,
+            "mean_set_size_per_query": round(mean_count, 1),
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "louver_query_kernel + louver_compact_kernel (routing)",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": None,
+            "algorithmic_bytes_per_launch": int(route_b),
+            "avg_launch_us": round(t_route_max * 1e3, 2),
+            "peak_source": peak_src,
+        },
+        "step_roofline": {
+            "unique_bytes_per_step": int(route_b + attn_b),
+            "achieved_gbs": round((route_b + attn_b) / (ms_per_step * 1e-3) / 1e9, 1),
+            "frac_of_measured_peak": round((route_b + attn_b) / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+        },
+        "kernels_us": {"louver_route": round(t_route * 1e3, 2),
+                       "attn_gather_all_layers": round(t_attn * 1e3, 2),
+                       "full_scan_route_threshold": round(t_full_route * 1e3, 2),
+                       "full_scan_threshold_step": round(ms_full * 1e3, 2)},
+        "e2e": e2e,
+        "gpu_launches": (2 + (1 if w.dtype == "bf16" else 2)) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_threshold(w, x)
+    return line
+
+
+def run_e2e_louver(sd, w, variants, K, V, ix, taus, ws, stream, dev, args, world):
+    """The Louver step through the public Python API with host buffers:
+    queries copied in from pinned host memory, the outputs, the set and its
+    counts read back, all inside the timed region (per-step sync)."""
+    hq = [(qr.pin_memory(), ql.pin_memory()) for qr, ql in variants]
+    dq = [(torch.empty_like(qr, device=dev), torch.empty_like(ql, device=dev)) for qr, ql in variants]
+    out_h = torch.empty(tuple(variants[0][1].shape), dtype=variants[0][1].dtype).pin_memory()
+    idx_h = torch.empty((w.B, w.Hkv, w.cap), dtype=torch.int32).pin_memory()
+    cnt_h = torch.empty((w.B, w.Hkv), dtype=torch.int32).pin_memory()
+    out_d = torch.empty(tuple(variants[0][1].shape), dtype=variants[0][1].dtype, device=dev)
+    idx_d = torch.empty((w.B, w.Hkv, w.cap), dtype=torch.int32, device=dev)
+    cnt_d = torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev)
+    steps = min(args.steps, 2000)
+    h2d = hq[0][0].numel() * hq[0][0].element_size() + hq[0][1].numel() * hq[0][1].element_size()
+    d2h = (out_h.numel() * out_h.element_size() + idx_h.numel() * 4 + cnt_h.numel() * 4)
+
+    def one(i):
+        j = i % len(hq)
+        (hqr, hql), (dqr, dql) = hq[j], dq[j]
+        dqr.copy_(hqr, non_blocking=True)
+        dql.copy_(hql, non_blocking=True)
+        sd.louver_route_threshold(dqr, K, ix, taus[j], w.cap, check=False, idx=idx_d, count=cnt_d)
+        sd.attn_gather(dql, K, V, idx_d, count=cnt_d, ws=ws, check=False, out=out_d,
+                       return_lse=False)
+        out_h.copy_(out_d, non_blocking=True)
+        idx_h.copy_(idx_d, non_blocking=True)
+        cnt_h.copy_(cnt_d, non_blocking=True)
+        stream.synchronize()
+
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            one(i)
+        torch.cuda.synchronize()
+        sdist.barrier()
+        t0 = time.perf_counter()
+        for i in range(steps):
+            one(i)
+        t1 = time.perf_counter()
+        sdist.barrier()
+    sec = sdist.max_over_ranks(t1 - t0)
+    return {"value": round(world * steps / sec, 2), "unit": "steps/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "api": "token_sparse_attention_sm_b200.louver_route_threshold + attn_gather "
+                   "(eager, per-step sync)"}
+
+
+def cpu_baseline_threshold(w, x, budget_s: float = 10.0):
+    """The C oracle, as it stands, on full threshold decode steps of the same
+    workload (its set is the one the Louver index returns), repeated for
+    about `budget_s` seconds."""
+    import oracle
+    qr, ql = synth.f32(x["q_route"]), synth.f32(x["q_layers"])
+    Kf, Vf = synth.f32(x["K"]), synth.f32(x["V"])
+    tau = oracle.percentile_tau(oracle.scores(qr, Kf), *w.tau_pct)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode_step(qr, ql, Kf, Vf, tau=tau, cap=w.cap)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    sec = time.perf_counter() - t0
+    return {"value": round(n / sec, 4), "unit": "steps/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n} full threshold decode steps of {w.name} (all {w.B * w.Hkv} KV "
+                      f"heads, {w.L} layers, full scan) by the plain C oracle, {sec:.1f} s"}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -542,7 +796,13 @@ def main():
     ap.add_argument("--reroute", type=int, default=0,
                     help="re-route every R layers (1: per-layer routing); default: route "
                          "once per step, the method's shared routing")
+    ap.add_argument("--louver", type=int, default=0, metavar="R",
+                    help="threshold steps routed through the Louver index with clusters of "
+                         "R keys (workload louver_128k unless --workload names another "
+                         "threshold workload)")
     args = ap.parse_args()
+    if args.louver and synth.WORKLOADS[args.workload].mode != "threshold":
+        args.workload = "louver_128k"
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank, world, local_rank = sdist.env_rank_world()
@@ -552,7 +812,10 @@ def main():
         return
     sdist.init("nccl")
     try:
-        line = run_native(args, rank, world, local_rank)
+        if args.louver:
+            line = run_native_louver(args, rank, world, local_rank)
+        else:
+            line = run_native(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -532,7 +532,8 @@ def louver_build(K, r: int, n: int | None = None, check: bool = True) -> LouverI
 
 
 def louver_route_threshold(q, K, index: LouverIndex, tau, cap: int, check: bool = True,
-                           return_survivors: bool = False):
+                           return_survivors: bool = False, idx=None, count=None,
+                           survivors=None):
     """Threshold routing through a Louver index: (idx [B,Hkv,cap], count [B,Hkv])
     -- the set route_threshold returns -- plus, if asked, survivors [B,Hkv]
     (clusters that passed the ball test).  K only checks that the index was
@@ -542,9 +543,15 @@ def louver_route_threshold(q, K, index: LouverIndex, tau, cap: int, check: bool 
     if (B, Hkv, Ncap, d, K.dtype) != (index.B, index.Hkv, index.Ncap, index.d, index.dtype):
         raise ValueError("the index was built for another K")
     sh = _shape(B, index.N, Hq, Hkv, d, q.dtype, Ncap)
-    idx = torch.empty((B, Hkv, cap), dtype=torch.int32, device=q.device)
-    count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
-    surv = torch.empty((B, Hkv), dtype=torch.int32, device=q.device) if return_survivors else None
+    if idx is None:
+        idx = torch.empty((B, Hkv, cap), dtype=torch.int32, device=q.device)
+    if count is None:
+        count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    surv = survivors
+    if return_survivors and surv is None:
+        surv = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    if idx.shape != (B, Hkv, cap) or count.shape != (B, Hkv):
+        raise ValueError("idx must be [B,Hkv,cap] and count [B,Hkv]")
     tau = tau.float().contiguous()
     buf = index.ws.get(index.ws_bytes)
     _check(load().sparse_louver_route_threshold(

@@ -3,7 +3,9 @@
     python -m token_sparse_attention_sm_b200.profile_case \
         --workload decode_128k --op decode --reps 3
 
---op is one of: score, route, attn, decode.  Inputs come from the seeded
+--op is one of: score, route, attn, decode, louver (threshold routing
+through a Louver index with clusters of --r keys, tau the 97th-percentile
+score of each head).  Inputs come from the seeded
 generator; nothing is checked or timed here (use bench.py for timing and the
 tests for parity).  The process exits non-zero if the device reports any
 condition."""
@@ -20,7 +22,9 @@ from token_sparse_attention_sm_b200 import synth
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="decode_128k", choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--op", default="decode", choices=["score", "route", "attn", "decode"])
+    ap.add_argument("--op", default="decode",
+                    choices=["score", "route", "attn", "decode", "louver"])
+    ap.add_argument("--r", type=int, default=128)
     ap.add_argument("--reps", type=int, default=3)
     a = ap.parse_args()
     w = synth.WORKLOADS[a.workload]
@@ -30,7 +34,14 @@ def main():
     ws = sd.Workspace(dev)
     k = w.k if w.mode == "topk" else w.cap
     idx = sd.route_topk(t["q_route"], t["K"], k, ws=ws) if a.op == "attn" else None
+    if a.op == "louver":
+        S = sd.score(t["q_route"], t["K"], ws=ws)
+        tau = torch.kthvalue(S, -(-97 * w.N // 100), dim=-1).values.contiguous()
+        ix = sd.louver_build(t["K"], a.r)
     for _ in range(a.reps):
+        if a.op == "louver":
+            sd.louver_route_threshold(t["q_route"], t["K"], ix, tau, w.cap or w.N, check=False)
+            continue
         if a.op == "score":
             sd.score(t["q_route"], t["K"], ws=ws, check=False)
         elif a.op == "route":
@@ -42,6 +53,8 @@ def main():
                            check=False)
     torch.cuda.synchronize()
     sd.read_device_status(ws)
+    if a.op == "louver":
+        sd.read_device_status(ix.ws)
     print(f"{a.op} x{a.reps} on {w.name}: ok")
 
 
