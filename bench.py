@@ -693,7 +693,7 @@ def run_native_louver(args, rank, world, local_rank):
             "mean_set_size_per_query": round(mean_count, 1),
         },
         "roofline": {
-            "bound": "hbm", "kernel": "louver_query_kernel + louver_compact_kernel (routing)",
+            "bound": "hbm", "kernel": "louver_query_kernel (routing: ball tests, exact checks, ordered set)",
             "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": None,
             "algorithmic_bytes_per_launch": int(route_b),
@@ -710,7 +710,7 @@ def run_native_louver(args, rank, world, local_rank):
                        "full_scan_route_threshold": round(t_full_route * 1e3, 2),
                        "full_scan_threshold_step": round(ms_full * 1e3, 2)},
         "e2e": e2e,
-        "gpu_launches": (2 + (1 if w.dtype == "bf16" else 2)) * args.steps,
+        "gpu_launches": (1 + (1 if w.dtype == "bf16" else 2)) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

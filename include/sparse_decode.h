@@ -58,9 +58,9 @@
  * Asynchrony: every compute entry point enqueues its kernels on `stream`
  * and returns without synchronising.
  *
- * Co-residency: the bf16 attention kernel (and the optional fused routing
- * kernel) split one head's work over several CTAs that wait for one another
- * (bounded waits).  Their grid is at most one CTA per SM, so it is resident
+ * Co-residency: the bf16 attention kernel, the Louver query kernel (and the
+ * optional fused routing kernel) split one head's work over several CTAs
+ * that wait for one another (bounded waits).  Their grid is at most one CTA per SM, so it is resident
  * as a whole while the device runs nothing else; they are launched as
  * ordinary kernels so that each can start while its predecessor drains.  A
  * caller that runs other kernels on the same device at the same time (other
@@ -282,7 +282,10 @@ sparse_status_t sparse_louver_build(const sparse_shape_t *shape, const void *K, 
  * (|c| + rho), a margin above the fp32 rounding of any member's score, so
  * rounding cannot drop a key.  survivors (nullable) [B,Hkv] int32: clusters that
  * passed the ball test.  q [B,Hq,d] of the shape's dtype; the shape is the
- * one the index was built for (Hq may differ; n_cap is not used). */
+ * one the index was built for (Hq may differ; n_cap is not used).  One
+ * kernel: its CTAs of a head meet at a bounded wait before writing the set
+ * (see Co-residency); a wait that expires reports SPARSE_ERR_TIMEOUT and
+ * leaves the workspace to be zero-filled again before the next query. */
 sparse_status_t sparse_louver_route_threshold(const sparse_shape_t *shape, const void *q,
                                               const void *index, size_t index_bytes, int32_t r,
                                               const float *tau, int32_t cap, int32_t *idx,

@@ -229,3 +229,27 @@ def test_louver_repeated_queries_keep_workspace_clean(dev):
         tau = torch.from_numpy(oracle.percentile_tau(S, 80 + 3 * i, 100)).to(dev)
         a = sd.louver_route_threshold(qd, Kd, ix, tau, 4096)
         _assert_same_set(a, sd.route_threshold(qd, Kd, tau, 4096), 4096)
+
+
+@pytest.mark.parametrize("cap", [262144, 100000])
+def test_louver_large_sets_several_compaction_passes(dev, cap):
+    """Half of 262,144 keys selected: the head's bitmap takes two compaction
+    passes and each pass selects more indices than the staging buffer in
+    shared memory holds (the rest go straight to memory); with cap below the
+    count the first cap indices are kept and capacity is flagged."""
+    w = synth.custom(B=1, N=262144, Hq=4, Hkv=1, d=64, L=1, dtype="bf16", seed=13,
+                     mode="threshold", cap=cap)
+    x = synth.generate(w)
+    qd, Kd = x["q_route"].to(dev), x["K"].to(dev)
+    q32, K32 = _f(x["q_route"]), _f(x["K"])
+    tau = oracle.percentile_tau(oracle.scores(q32, K32), 50, 100)
+    taud = torch.from_numpy(tau).to(dev)
+    ix = sd.louver_build(Kd, 64)
+    a = sd.louver_route_threshold(qd, Kd, ix, taud, cap, check=False)
+    st_a = sd.read_device_status(ix.ws, raise_on_error=False)
+    ws = sd.Workspace(dev)
+    f = sd.route_threshold(qd, Kd, taud, cap, ws=ws, check=False)
+    st_f = sd.read_device_status(ws, raise_on_error=False)
+    _assert_same_set(a, f, cap)
+    assert st_a == st_f == (4 if int(a[1][0, 0]) > cap else 0)
+    assert int(a[1][0, 0]) > 65536

@@ -263,20 +263,84 @@ __global__ void __launch_bounds__(128)
 //     are read one item ahead of their copy.  Scores come from the scan's
 //     warp routine with qbar formed as the scan forms it; keys >= tau are
 //     marked in the head's bitmap.
-// The compaction kernel below then turns the bitmaps into the ordered sets.
+//  3. once every CTA of the head has marked its keys (a per-head arrival
+//     counter, bounded wait), each CTA writes a slice of the ordered set
+//     (compact_slice).  The bitmaps are double-buffered per head: a query
+//     marks one and clears the other (the previous query's), and the last
+//     CTA of the head to leave flips the head's parity and resets its
+//     counters.
 constexpr int kQWarps = 8;
 constexpr int kQThreads = kQWarps * 32;
 constexpr int kQGroupsPerRound = kQThreads / 8;   // clusters tested at once
 constexpr int kQMaxSlots = 4;
+
+// One CTA's share of turning a head's bitmap (nw words) into its ascending
+// indices: the words [s0, s1).  The CTA counts the set bits before s0 (its
+// base) and in its slice; thread t owns a contiguous run of the slice, so a
+// block scan orders the threads.  The indices are staged in shared memory
+// (stage_cap entries; a direct store per index would cost one memory sector
+// each) and written out with coalesced stores; only the first cap are kept.
+// Returns base + the slice's count (the head's total for the last slice).
+__device__ uint32_t compact_slice(const uint32_t *__restrict__ bm, int s0, int s1, int cap,
+                                  int *__restrict__ out, int *stage, int stage_cap,
+                                  uint32_t *wbuf) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // base: set bits in words [0, s0), coalesced, 8 loads in flight per thread
+  uint32_t pre = 0;
+  for (int w0 = 0; w0 < s0; w0 += 8 * kQThreads) {
+    uint32_t v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int wi = w0 + u * kQThreads + tid;
+      v[u] = wi < s0 ? __ldcg(bm + wi) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) pre += __popc(v[u]);
+  }
+  pre = __reduce_add_sync(0xffffffffu, pre);
+  __syncthreads();
+  if (lane == 0) wbuf[warp] = pre;
+  __syncthreads();
+  uint32_t base = 0;
+  for (int w = 0; w < kQWarps; ++w) base += wbuf[w];
+  // the slice: thread tid owns words [r0, r1)
+  const int wpt = (s1 - s0 + kQThreads - 1) / kQThreads;
+  const int r0 = min(s1, s0 + tid * wpt), r1 = min(s1, r0 + wpt);
+  uint32_t cnt = 0;
+  for (int wi = r0; wi < r1; ++wi) cnt += __popc(__ldcg(bm + wi));
+  uint32_t total;
+  uint32_t pos = base + lv_block_scan<kQThreads>(cnt, wbuf, &total);
+  const uint32_t lim = (uint32_t)(cap < stage_cap ? cap : stage_cap);
+  for (int wi = r0; wi < r1; ++wi) {
+    uint32_t m = __ldcg(bm + wi);
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      m &= m - 1u;
+      if (pos < (uint32_t)cap) {
+        const uint32_t sp = pos - base;
+        if (sp < lim) stage[sp] = wi * 32 + bit;
+        else out[pos] = wi * 32 + bit;
+      }
+      ++pos;
+    }
+  }
+  __syncthreads();
+  const uint32_t hi = base + total < (uint32_t)cap ? base + total : (uint32_t)cap;
+  const uint32_t nst = hi > base ? min(hi - base, lim) : 0u;
+  for (uint32_t i = tid; i < nst; i += kQThreads) out[base + i] = stage[i];
+  return base + total;
+}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kQThreads)
     louver_query_kernel(const T *__restrict__ q, int Hq, int Hkv, int N, float scale,
                         const int *__restrict__ perm, const float *__restrict__ centres,
                         const float *__restrict__ radii, const T *__restrict__ keys, int r,
-                        int nc, const float *__restrict__ tau, int nb,
-                        uint32_t *__restrict__ bitmap, int *__restrict__ nsurv,
-                        uint32_t *status) {
+                        int nc, const float *__restrict__ tau, int nb, int cap,
+                        uint32_t *__restrict__ bitmap, uint32_t *__restrict__ parity,
+                        int *__restrict__ nsurv, uint32_t *__restrict__ done,
+                        int *__restrict__ idx, int *__restrict__ count,
+                        int *__restrict__ survivors_out, uint32_t *status) {
   using C = ScoreCfg<T, D>;
   constexpr int EPG = D / 8;                  // centre elements per lane of a group
   constexpr int kItemBytes = 32 * C::kRowBytes;
@@ -285,7 +349,8 @@ __global__ void __launch_bounds__(kQThreads)
   __shared__ __align__(16) float qb[D];
   __shared__ __align__(8) uint64_t bars[kQWarps][kQMaxSlots];
   __shared__ float qn_s;
-  __shared__ int nlist;
+  __shared__ int nlist, ready;
+  __shared__ uint32_t wbuf[kQWarps];
   const int bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int splits = gridDim.x;
   const int mc = (nc - (int)blockIdx.x + splits - 1) / splits;  // clusters owned
@@ -295,6 +360,17 @@ __global__ void __launch_bounds__(kQThreads)
   fence_mbar_init();
   grid_dep_wait();
   grid_dep_launch();
+  // this query marks bitmap `par` of the head and clears (its share of) the
+  // other one, which the previous query used and the next one will mark
+  const int nw = N / 32, BH = gridDim.y;
+  const uint32_t par = __ldcg(parity + bh) & 1u;
+  uint32_t *bm = bitmap + ((size_t)par * BH + bh) * nw;
+  {
+    uint32_t *old = bitmap + ((size_t)(par ^ 1u) * BH + bh) * nw;
+    const int c0 = (int)((long long)nw * blockIdx.x / splits);
+    const int c1 = (int)((long long)nw * (blockIdx.x + 1) / splits);
+    for (int wi = c0 + tid; wi < c1; wi += kQThreads) old[wi] = 0u;
+  }
 
   // ---- 1. ball test
   const int grp = tid >> 3, gl = tid & 7;
@@ -372,7 +448,6 @@ __global__ void __launch_bounds__(kQThreads)
   const int nitems = ns * ipc;
   unsigned char *wb = lv_smem + (size_t)warp * nb * kSlotBytes;
   const size_t head0 = (size_t)bh * nc * r;  // the head's first cluster-ordered row
-  uint32_t *bm = bitmap + (size_t)bh * (N / 32);
   // cluster-ordered row of row 0 of item it
   auto item_row = [&](int it) -> size_t {
     return head0 + (size_t)list[it / ipc] * r + (it % ipc) * 32;
@@ -421,78 +496,66 @@ __global__ void __launch_bounds__(kQThreads)
     __syncwarp();  // the slot is read before it is refilled
   }
   // after an expired wait, the copies issued and not consumed (items kfail
-  // .. kfail + nb - 1) are waited for, again with a limit, before exit
+  // .. kfail + nb - 1) are waited for, again with a limit, before going on
   if (kfail >= 0)
     for (int k2 = kfail; k2 < kfail + nb && warp + k2 * kQWarps < nitems; ++k2)
       mbar_wait(&bars[warp][k2 % nb], (uint32_t)((k2 / nb) & 1), status);
-}
 
-// Bitmap -> ascending indices.  One thread-block cluster of kCSlices CTAs
-// per head; CTA c owns the c-th contiguous slice of the head's bitmap words.
-// Each CTA counts its slice's set bits, the counts are exchanged through
-// distributed shared memory after a cluster barrier (so no CTA reads another
-// slice's words, and each may clear its own), and each CTA then writes its
-// slice's indices from its base (the first cap of the head).  The last CTA
-// writes the head's count and survivor count and resets the latter.
-constexpr int kCSlices = 8;
-constexpr int kCThreads = 256;
-
-__global__ void __launch_bounds__(kCThreads)
-    louver_compact_kernel(uint32_t *__restrict__ bitmap, int N, int cap, int *__restrict__ idx,
-                          int *__restrict__ count, int *__restrict__ nsurv,
-                          int *__restrict__ survivors_out, uint32_t *status) {
-  cg::cluster_group cluster = cg::this_cluster();
-  __shared__ uint32_t wbuf[kCThreads / 32];
-  __shared__ uint32_t slice_total;
-  const int rank = (int)cluster.block_rank();
-  const int bh = blockIdx.y, tid = threadIdx.x;
-  const int nw = N / 32;
-  const int per_slice = (nw + kCSlices - 1) / kCSlices;
-  const int s0 = min(nw, rank * per_slice), s1 = min(nw, s0 + per_slice);
-  const int wpt = (s1 - s0 + kCThreads - 1) / kCThreads;
-  const int r0 = min(s1, s0 + tid * wpt), r1 = min(s1, r0 + wpt);
-  grid_dep_wait();
-  grid_dep_launch();
-  uint32_t *bm = bitmap + (size_t)bh * nw;
-  uint32_t cnt = 0;
-  for (int wi = r0; wi < r1; ++wi) cnt += __popc(__ldcg(bm + wi));
-  uint32_t total;
-  const uint32_t off = lv_block_scan<kCThreads>(cnt, wbuf, &total);
-  if (tid == 0) slice_total = total;
-  cluster.sync();
-  uint32_t base = 0, head_total = 0;
-  for (int c = 0; c < kCSlices; ++c) {
-    const uint32_t v = *cluster.map_shared_rank(&slice_total, c);
-    base += c < rank ? v : 0u;
-    head_total += v;
+  // ---- 3. the head's CTAs turn the bitmap into the ordered set, a slice
+  // each, once all of them have marked their keys: an arrival counter per
+  // head (bounded wait; the grid is one wave, one CTA per SM).  The barrier
+  // orders each CTA's bitmap updates before thread 0's release; thread 0's
+  // acquire and the barrier after it order every CTA's updates before the
+  // reads below.
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t *arrive = done + 2 * bh;
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(arrive) : "memory");
+    bool ok = true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+      uint32_t v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(arrive) : "memory");
+      if (v >= (uint32_t)splits) break;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        raise_flag(status, FLAG_TIMEOUT);
+        ok = false;
+        break;
+      }
+      __nanosleep(32);
+    }
+    ready = ok;
   }
-  uint32_t pos = base + off;
-  int *out = idx + (size_t)bh * cap;
-  for (int wi = r0; wi < r1; ++wi) {
-    uint32_t m = __ldcg(bm + wi);
-    if (m) bm[wi] = 0u;
-    while (m) {
-      const int bit = __ffs(m) - 1;
-      m &= m - 1u;
-      if (pos < (uint32_t)cap) out[pos] = wi * 32 + bit;
-      ++pos;
+  __syncthreads();
+  if (!ready) return;
+  const int s0 = (int)((long long)nw * blockIdx.x / splits);
+  const int s1 = (int)((long long)nw * (blockIdx.x + 1) / splits);
+  const uint32_t end = compact_slice(bm, s0, s1, cap, idx + (size_t)bh * cap,
+                                     reinterpret_cast<int *>(lv_smem),
+                                     (int)(((size_t)kQWarps * nb * kSlotBytes) / sizeof(int)),
+                                     wbuf);
+  if (tid == 0) {
+    if (blockIdx.x == splits - 1) {  // the last slice ends at the head's total
+      count[bh] = (int)end;
+      if (end > (uint32_t)cap) raise_flag(status, FLAG_CAPACITY);
+    }
+    // the last CTA to leave resets the head's counters and flips its bitmaps
+    if (atomicAdd(done + 2 * bh + 1, 1u) == (uint32_t)splits - 1) {
+      const int sv = __ldcg(nsurv + bh);
+      if (survivors_out) survivors_out[bh] = sv;
+      nsurv[bh] = 0;
+      parity[bh] = par ^ 1u;
+      done[2 * bh] = 0u;
+      done[2 * bh + 1] = 0u;
     }
   }
-  if (rank == kCSlices - 1 && tid == 0) {
-    count[bh] = (int)head_total;
-    if (head_total > (uint32_t)cap) raise_flag(status, FLAG_CAPACITY);
-    const int sv = __ldcg(nsurv + bh);
-    if (survivors_out) survivors_out[bh] = sv;
-    nsurv[bh] = 0;
-  }
-  cluster.sync();  // no CTA leaves while another may read its shared memory
 }
 
 // ---- host side ----------------------------------------------------------------
 
 struct LvLayout {
   size_t perm, centres, radii, keys, index_total;                      // index
-  size_t sums, va, vb, proj, perm2, sel, bitmap, nsurv, ws_total;  // workspace
+  size_t sums, va, vb, proj, perm2, sel, bitmap, parity, nsurv, done, ws_total;  // workspace
 };
 
 size_t lv_align(size_t x) { return (x + 255) / 256 * 256; }
@@ -519,9 +582,11 @@ LvLayout lv_layout(const Shape &s, int r) {
   l.proj = l.vb + lv_align(nseg * d * 4);
   l.perm2 = l.proj + lv_align(BH * N * 4);
   l.sel = l.perm2 + lv_align(BH * N * 4);
-  l.bitmap = l.sel + lv_align(BH * N / 2 * 4 + 4);
-  l.nsurv = l.bitmap + lv_align(BH * N / 32 * 4);
-  l.ws_total = l.nsurv + lv_align(BH * 4);
+  l.bitmap = l.sel + lv_align(BH * N / 2 * 4 + 4);  // two per head (double-buffered)
+  l.parity = l.bitmap + lv_align(2 * BH * N / 32 * 4);
+  l.nsurv = l.parity + lv_align(BH * 4);
+  l.done = l.nsurv + lv_align(BH * 4);
+  l.ws_total = l.done + lv_align(2 * BH * 4);
   return l;
 }
 
@@ -621,35 +686,25 @@ cudaError_t lv_query_t(const Shape &s, const void *qv, int r, const char *index,
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attrs[1];
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeCooperative;
+  attrs[0].val.cooperative = 1;
   cfg.attrs = attrs;
   cfg.stream = st;
   cfg.gridDim = dim3((unsigned)splits, (unsigned)s.BH(), 1);
   cfg.blockDim = dim3(kQThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
-  cfg.numAttrs = 0;
+  cfg.numAttrs = (splits > 1 && cooperative_forced()) ? 1 : 0;
   add_pdl_attr(cfg, attrs);
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(qv), s.Hq, s.Hkv, s.N, scale,
                          reinterpret_cast<const int *>(index + l.perm),
                          reinterpret_cast<const float *>(index + l.centres),
                          reinterpret_cast<const float *>(index + l.radii),
-                         reinterpret_cast<const T *>(index + l.keys), r, nc, tau, nb,
+                         reinterpret_cast<const T *>(index + l.keys), r, nc, tau, nb, cap,
                          reinterpret_cast<uint32_t *>(ws + l.bitmap),
-                         reinterpret_cast<int *>(ws + l.nsurv), reinterpret_cast<uint32_t *>(ws));
-  if (e != cudaSuccess) return e;
-  cudaLaunchAttribute cattrs[2];
-  cattrs[0].id = cudaLaunchAttributeClusterDimension;
-  cattrs[0].val.clusterDim.x = kCSlices;
-  cattrs[0].val.clusterDim.y = 1;
-  cattrs[0].val.clusterDim.z = 1;
-  cfg.attrs = cattrs;
-  cfg.gridDim = dim3((unsigned)kCSlices, (unsigned)s.BH(), 1);
-  cfg.blockDim = dim3(kCThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.numAttrs = 1;
-  add_pdl_attr(cfg, cattrs);
-  e = cudaLaunchKernelEx(&cfg, louver_compact_kernel, reinterpret_cast<uint32_t *>(ws + l.bitmap),
-                         s.N, cap, idx, count, reinterpret_cast<int *>(ws + l.nsurv), survivors,
+                         reinterpret_cast<uint32_t *>(ws + l.parity),
+                         reinterpret_cast<int *>(ws + l.nsurv),
+                         reinterpret_cast<uint32_t *>(ws + l.done), idx, count, survivors,
                          reinterpret_cast<uint32_t *>(ws));
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
