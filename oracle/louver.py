@@ -16,9 +16,15 @@ Louver summary ("技術サマリー：スパースアテンションを範囲検
 
 Readings (where the page is silent):
 
-* One subspace (S = 1): the page splits d into S subspaces with an index each
-  and leaves the per-subspace threshold rule open; with S = 1 its two query
-  algorithms (all-subspace filter and TA filter) are the same ball test.
+* Subspaces: the page splits d into S contiguous subspaces of d/S dimensions
+  with an index each, and its first query algorithm keeps a key only if the
+  key's cluster passes the ball test in every subspace, against a threshold
+  tau_s per subspace whose rule it does not give.  Reading: the plainest rule
+  that keeps every key scoring >= tau.  With U_s the largest ball bound of
+  subspace s over the head's clusters, <q,k> = sum_s <q_s,k_s> >= tau forces
+  <q_s,k_s> >= tau - sum_{s' != s} U_s' for every s, so
+  tau_s = tau - sum_{s' != s} U_s'.  With S = 1 this is the plain ball test
+  (tau_1 = tau), and the page's two query algorithms coincide.
 * Balanced PCA tree: a node's keys are split at the median of their
   projections on the node's principal direction (the top eigenvector of the
   node's covariance) into two halves of equal size, recursively, down to
@@ -34,7 +40,9 @@ Readings (where the page is silent):
   second term bounds the fp32 rounding of a member's score (at most a few
   1e-7 of |qbar| |k| for d <= 128, and |k| <= |c| + rho), which does not
   shrink with tau, so no fp32 rounding of the exact check can make a pruned
-  key pass even when tau is near zero.
+  key pass even when tau is near zero.  With S subspaces the norm bound of a
+  member is (|c_s| + rho_s) + sum_{s' != s} R_s', R_s' the largest
+  |c| + rho of subspace s', and the bound against tau_s uses it.
 """
 from __future__ import annotations
 
@@ -94,6 +102,72 @@ def keep_clusters(index: dict, qbar, tau: float) -> np.ndarray:
     qn = np.linalg.norm(q)
     slack = 1e-5 * qn * (np.linalg.norm(index["centres"], axis=1) + index["radii"])
     return ball_bounds(index, q) >= tau - band(tau) - slack
+
+
+def keep_clusters_subspaces(indexes: list, qbar, tau: float) -> list:
+    """The all-subspace filter: for every subspace s (index s over dimensions
+    s*d/S .. (s+1)*d/S), True for each cluster that passes its ball test
+    against tau_s = tau - sum_{s' != s} U_s'."""
+    q = np.asarray(qbar, np.float64)
+    S = len(indexes)
+    ds = q.shape[0] // S
+    qs = [q[s * ds:(s + 1) * ds] for s in range(S)]
+    bounds = [ball_bounds(ix, qs[s]) for s, ix in enumerate(indexes)]
+    U = [float(b.max()) for b in bounds]
+    R = [float((np.linalg.norm(ix["centres"], axis=1) + ix["radii"]).max()) for ix in indexes]
+    qn = np.linalg.norm(q)
+    keep = []
+    for s, ix in enumerate(indexes):
+        rest_U = sum(U) - U[s]
+        rest_R = sum(R) - R[s]
+        slack = 1e-5 * qn * (np.linalg.norm(ix["centres"], axis=1) + ix["radii"] + rest_R)
+        keep.append(bounds[s] >= tau - rest_U - band(tau) - slack)
+    return keep
+
+
+def candidates(indexes: list, keep: list, N: int) -> np.ndarray:
+    """Keys whose cluster passes in every subspace (bool [N])."""
+    ok = np.ones(N, bool)
+    for ix, kp in zip(indexes, keep):
+        r = N // len(kp)
+        member = np.zeros(N, bool)
+        member[ix["perm"].reshape(-1, r)[kp].ravel()] = True
+        ok &= member
+    return ok
+
+
+def route_threshold_subspaces(q, K, tau, cap: int, r: int, S: int):
+    """Threshold routing through S subspace indexes (the all-subspace
+    filter, then the exact check of the candidates), every (b, h).
+
+    Returns (idx [B,Hkv,cap], count [B,Hkv], candidates [B,Hkv] = keys that
+    passed the filter in every subspace).  The set equals the full-scan
+    threshold set on the oracle's fp32 scores."""
+    q = np.asarray(q, np.float32)
+    K = np.asarray(K, np.float32)
+    tau = np.asarray(tau, np.float32)
+    B, Hq, d = q.shape
+    _, Hkv, N, _ = K.shape
+    if d % S:
+        raise ValueError("S must divide d")
+    ds = d // S
+    G = Hq // Hkv
+    Sc = _scores(q, K)
+    idx = np.full((B, Hkv, cap), -1, np.int32)
+    count = np.zeros((B, Hkv), np.int32)
+    ncand = np.zeros((B, Hkv), np.int64)
+    for b in range(B):
+        for h in range(Hkv):
+            indexes = [build_index(K[b, h][:, s * ds:(s + 1) * ds], r) for s in range(S)]
+            qbar = q[b, h * G:(h + 1) * G].astype(np.float64).sum(0) / math.sqrt(d)
+            keep = keep_clusters_subspaces(indexes, qbar, float(tau[b, h]))
+            cand = np.nonzero(candidates(indexes, keep, N))[0]
+            ncand[b, h] = len(cand)
+            sel = cand[Sc[b, h, cand] >= tau[b, h]]
+            count[b, h] = len(sel)
+            m = min(len(sel), cap)
+            idx[b, h, :m] = sel[:m]
+    return idx, count, ncand
 
 
 def route_threshold(q, K, tau, cap: int, r: int):

@@ -485,3 +485,51 @@ def test_louver_query_equals_full_scan_and_prunes_soundly(kind):
             assert np.all(S64[0, h, keys] < t)
         if kind == "blobs" and pct == 97:
             assert surv.sum() < 0.5 * Hkv * (N // rc)
+
+
+@pytest.mark.parametrize("S", [2, 4])
+@pytest.mark.parametrize("kind", ["gaussian", "blobs"])
+def test_louver_subspaces_equal_full_scan_and_sound(S, kind):
+    """The all-subspace filter with tau_s = tau - sum of the other subspaces'
+    largest bounds: the set equals the full-scan threshold set; every key
+    scoring >= tau in fp64 is a candidate (closed form: the sum of a key's
+    subspace scores is its score, each bounded by its subspace's largest
+    ball bound); with S = 1 the filter is the plain ball test."""
+    from oracle import louver
+    r = _rng(61 + S)
+    B, Hq, Hkv, N, d, rc = 1, 8, 2, 1024, 32, 16
+    q = r.standard_normal((B, Hq, d), dtype=np.float32)
+    K = (r.standard_normal((B, Hkv, N, d), dtype=np.float32) if kind == "gaussian"
+         else _blobs(r, B, Hkv, N, d))
+    S32 = oracle.scores(q, K)
+    S64 = oracle.scores(q, K, np.float64)
+    G = Hq // Hkv
+    for pct in (50, 97, 100):
+        tau = oracle.percentile_tau(S32, pct, 100)
+        idx, cnt, ncand = louver.route_threshold_subspaces(q, K, tau, N, rc, S)
+        ridx, rcnt = louver.full_scan_threshold(q, K, tau, N)
+        np.testing.assert_array_equal(cnt, rcnt)
+        np.testing.assert_array_equal(idx, ridx)
+        assert np.all(ncand >= cnt)
+        ds = d // S
+        for h in range(Hkv):
+            Kh = K[0, h]
+            indexes = [louver.build_index(Kh[:, s * ds:(s + 1) * ds], rc) for s in range(S)]
+            qbar = q[0, h * G:(h + 1) * G].astype(np.float64).sum(0) / math.sqrt(d)
+            t = float(tau[0, h])
+            keep = louver.keep_clusters_subspaces(indexes, qbar, t)
+            cand = louver.candidates(indexes, keep, N)
+            assert np.all(cand[S64[0, h] >= t]), "a key scoring >= tau was filtered out"
+            # the subspace scores of every key add up to its score
+            part = sum(Kh[:, s * ds:(s + 1) * ds].astype(np.float64) @ qbar[s * ds:(s + 1) * ds]
+                       for s in range(S))
+            np.testing.assert_allclose(part, S64[0, h], rtol=1e-12, atol=1e-12)
+    # S = 1 reduces to the plain ball test
+    tau = oracle.percentile_tau(S32, 97, 100)
+    for h in range(Hkv):
+        ix = louver.build_index(K[0, h], rc)
+        qbar = q[0, h * G:(h + 1) * G].astype(np.float64).sum(0) / math.sqrt(d)
+        t = float(tau[0, h])
+        np.testing.assert_array_equal(louver.keep_clusters_subspaces([ix], qbar, t)[0],
+                                      louver.keep_clusters(ix, qbar, t))
+
