@@ -26,7 +26,8 @@ __all__ = ["SparseDecodeError", "lib_path", "load", "score", "select_topk",
            "select_threshold", "route_topk", "route_threshold", "attn_gather",
            "decode_step", "read_device_status", "workspace_bytes",
            "Workspace", "STATUS_NAMES", "EXPORTED_SYMBOLS", "decode_step_grouped",
-           "kv_append", "LouverIndex", "louver_build", "louver_route_threshold"]
+           "kv_append", "LouverIndex", "louver_build", "louver_route_threshold",
+           "DecodeStepGraph"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_PKG, "libsparse_decode.so")
@@ -563,3 +564,84 @@ def louver_route_threshold(q, K, index: LouverIndex, tau, cap: int, check: bool 
     if return_survivors:
         return idx, count, surv
     return idx, count
+
+
+class DecodeStepGraph:
+    """A decode step with its host transfers, captured once as a CUDA graph.
+
+    Each replay copies q_route and q_layers from the given pinned host
+    tensors to the device, runs one fused decode step (top-k with ``k``, or
+    threshold with a device ``tau`` and ``cap``) over the cache K, V, and
+    copies out and idx (and count in threshold mode) back into pinned host
+    tensors -- one graph launch instead of a Python call and four copy
+    launches per step.  The host tensors are bound at capture time: write
+    the next step's queries into them (or keep one graph per buffer set) and
+    call ``replay()``; ``synchronize()`` waits for the results.  The graph
+    runs on ``stream`` (a new one by default); graphs that share a workspace
+    must run on one stream.  The device status is checked once after the
+    warm-up step (use ``read_device_status(self.ws)`` to check later ones)."""
+
+    def __init__(self, q_route_host, q_layers_host, K, V, k: int | None = None, tau=None,
+                 cap: int | None = None, ws: Workspace | None = None, out_host=None,
+                 idx_host=None, count_host=None, n: int | None = None, stream=None):
+        for t in (q_route_host, q_layers_host):
+            if t.is_cuda or not t.is_pinned():
+                raise ValueError("host queries must be pinned CPU tensors")
+        _need_cuda(K, V, tau)
+        dev = K.device
+        self.ws = _ws(ws, dev)
+        self.stream = stream if stream is not None else torch.cuda.Stream(device=dev)
+        self.q_route_host, self.q_layers_host = q_route_host, q_layers_host
+        self.q_route = torch.empty(q_route_host.shape, dtype=q_route_host.dtype, device=dev)
+        self.q_layers = torch.empty(q_layers_host.shape, dtype=q_layers_host.dtype, device=dev)
+        L, B, Hq, d = q_layers_host.shape
+        Hkv = K.shape[1]
+        topk = k is not None
+        stride = int(k) if topk else int(cap)
+        self.out = torch.empty_like(self.q_layers)
+        self.idx = torch.empty((B, Hkv, stride), dtype=torch.int32, device=dev)
+        self.count = None if topk else torch.empty((B, Hkv), dtype=torch.int32, device=dev)
+        self.out_host = out_host if out_host is not None else torch.empty(
+            self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.idx_host = idx_host if idx_host is not None else torch.empty(
+            self.idx.shape, dtype=torch.int32).pin_memory()
+        self.count_host = None
+        if not topk:
+            self.count_host = count_host if count_host is not None else torch.empty(
+                (B, Hkv), dtype=torch.int32).pin_memory()
+        args = dict(k=k, tau=tau, cap=cap, ws=self.ws, check=False, out=self.out, idx=self.idx,
+                    count=self.count, return_lse=False, n=n)
+
+        def body():
+            self.q_route.copy_(self.q_route_host, non_blocking=True)
+            self.q_layers.copy_(self.q_layers_host, non_blocking=True)
+            decode_step(self.q_route, self.q_layers, K, V, **args)
+            self.out_host.copy_(self.out, non_blocking=True)
+            self.idx_host.copy_(self.idx, non_blocking=True)
+            if self.count is not None:
+                self.count_host.copy_(self.count, non_blocking=True)
+
+        with torch.cuda.stream(self.stream):
+            body()                       # warm-up: sizes the workspace, loads the library
+            self.stream.synchronize()
+            read_device_status(self.ws)
+            self.graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.graph, stream=self.stream):
+                body()
+
+    def replay(self):
+        """Enqueue one step (inputs from, results to, the bound host tensors)."""
+        with torch.cuda.stream(self.stream):
+            self.graph.replay()
+
+    def synchronize(self):
+        self.stream.synchronize()
+
+    def __call__(self):
+        """One step, synchronised: returns (out_host, idx_host[, count_host])."""
+        self.replay()
+        self.synchronize()
+        if self.count_host is None:
+            return self.out_host, self.idx_host
+        return self.out_host, self.idx_host, self.count_host
+
