@@ -345,6 +345,40 @@ def run_native(args, rank, world, local_rank):
                                for qi in range(len(qs))], stream)
         t_attn = time_graphs(attn_graphs, n_k, max(args.warmup, 3), stream) / n_k
         sd.read_device_status(ws)
+        dense = None
+        if args.dense:
+            # dense attention: every key selected (k = N), all L layers over one
+            # read of K and V, and layer by layer (L reads)
+            all_idx = torch.arange(w.N, dtype=torch.int32, device=dev).repeat(w.B, w.Hkv, 1)
+            dense_out = torch.empty_like(qs[0][1])
+            dense_lse = torch.empty((w.L, w.B, w.Hq), dtype=torch.float32, device=dev)
+            ws.get(sd.workspace_bytes(w.B, w.N, w.Hq, w.Hkv, w.d, w.torch_dtype, w.N, w.L))
+            sd.attn_gather(qs[0][1], K, V, all_idx, ws=ws, check=True, out=dense_out,
+                           lse=dense_lse)
+            n_d = max(args.steps // 64, 16)
+            g_all = capture([lambda qi=qi: sd.attn_gather(qs[qi][1], K, V, all_idx, ws=ws,
+                                                          check=False, out=dense_out,
+                                                          lse=dense_lse)
+                             for qi in range(len(qs))], stream)
+            t_dense_all = time_graphs(g_all, n_d, max(args.warmup, 3), stream) / n_d
+
+            def per_layer(qi):
+                def run():
+                    for l in range(w.L):
+                        sd.attn_gather(qs[qi][1][l:l + 1], K, V, all_idx, ws=ws, check=False,
+                                       out=dense_out[l:l + 1], lse=dense_lse[l:l + 1])
+                return run
+            g_pl = capture([per_layer(qi) for qi in range(len(qs))], stream)
+            t_dense_pl = time_graphs(g_pl, n_d, max(args.warmup, 3), stream) / n_d
+            sd.read_device_status(ws)
+            kv_b = 2 * w.B * w.Hkv * w.N * w.d * w.esize
+            dense = {"all_layers_one_pass_us": round(t_dense_all * 1e3, 2),
+                     "all_layers_one_pass_gbs": round(kv_b / (t_dense_all * 1e-3) / 1e9, 1),
+                     "layer_by_layer_us": round(t_dense_pl * 1e3, 2),
+                     "layer_by_layer_gbs": round(w.L * kv_b / (t_dense_pl * 1e-3) / 1e9, 1),
+                     "note": "attn_gather with every key selected; the one-pass form reads K "
+                             "and V once for all layers (the shared cache), the layer-by-layer "
+                             "form L times"}
 
     ms_max = sdist.max_over_ranks(ms)
     t_score_max = sdist.max_over_ranks(t_score)
@@ -406,6 +440,7 @@ def run_native(args, rank, world, local_rank):
                        "note": "score and attention timed alone in back-to-back graph "
                                "launches (attention alone may find its rows in L2); select "
                                "= route (score + select) minus score"},
+        **({"dense_attention": dense} if dense else {}),
         "e2e": e2e,
         "gpu_launches": kernels_per_step(w, args.reroute) * args.steps,
         "clocks": clocks,
@@ -796,6 +831,9 @@ def main():
     ap.add_argument("--reroute", type=int, default=0,
                     help="re-route every R layers (1: per-layer routing); default: route "
                          "once per step, the method's shared routing")
+    ap.add_argument("--dense", action="store_true",
+                    help="also time dense attention over all N keys (k = N), all layers in "
+                         "one pass and layer by layer, as the comparison for per-layer routing")
     ap.add_argument("--louver", type=int, default=0, metavar="R",
                     help="threshold steps routed through the Louver index with clusters of "
                          "R keys (workload louver_128k unless --workload names another "

@@ -399,6 +399,20 @@ def test_attn_gather_many_keys_per_cta(dev, k, count):
     assert_attn_close(out, lse, o_ref, l_ref, "bf16")
 
 
+@pytest.mark.parametrize("dtype,N", [("bf16", 20011), ("f32", 3001)])
+def test_dense_attention_all_keys(dev, dtype, N):
+    """k = N: the gather attention over every cached key is dense attention
+    (the comparison the per-layer routing measurement uses), against the
+    oracle on all keys."""
+    w = synth.custom(B=1, N=N, Hq=8, Hkv=2, d=128, L=4, k=N, dtype=dtype, seed=29)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    idx = np.tile(np.arange(N, dtype=np.int32), (1, w.Hkv, 1))
+    out, lse = sd.attn_gather(t["q_layers"], t["K"], t["V"], torch.from_numpy(idx).to(dev))
+    o_ref, l_ref = oracle.attn(_f(x["q_layers"]), _f(x["K"]), _f(x["V"]), idx)
+    assert_attn_close(out, lse, o_ref, l_ref, dtype)
+
+
 def test_attn_gather_mma_sync_variant_matches(dev, monkeypatch):
     """The warp-level mma.sync kernel (kept for comparison) agrees too."""
     monkeypatch.setenv("SPARSE_DECODE_ATTN", "mma")
