@@ -21,35 +21,32 @@
 //  4. the n/2 largest projections by the library's exact radix select (ties
 //     to the lower position), then a stable partition: the other half first,
 //     the selected half second;
-// and at the leaves one warp per cluster computes the centre (mean) and the
-// radius (largest distance, inflated by 1e-5 relative to cover fp32
-// rounding).  The fp32 atomic sums make the build's directions depend on
-// summation order, so two builds can differ; every build is a valid index
-// and query results do not depend on it.
+// then the cluster-ordered copy of the keys, and at the leaves one warp per
+// cluster computes the centre (mean) and the radius (largest distance,
+// inflated by 1e-5 relative to cover fp32 rounding).  The fp32 atomic sums
+// make the build's directions depend on summation order, so two builds can
+// differ; every build is a valid index and query results do not depend on
+// it.
 //
-// Query: a ball test per cluster (bound <qbar, c> + |qbar| rho against
-// tau - band - slack, band = 1e-4 |tau| + 1e-6 and slack = 1e-5 |qbar|
-// (|c| + rho), which bounds the fp32 rounding of a member's score, so no
-// rounding can prune a key that scores >= tau), an exact check of the survivors' keys with the scan's own
+// Query (one kernel, louver_query_kernel below): a ball test per cluster
+// (bound <qbar, c> + |qbar| rho against tau - band - slack, band =
+// 1e-4 |tau| + 1e-6 and slack = 1e-5 |qbar| (|c| + rho), which bounds the
+// fp32 rounding of a member's score, so no rounding can prune a key that
+// scores >= tau), an exact check of the survivors' keys with the scan's own
 // per-key arithmetic (bit-identical to sparse_route_threshold's scores), a
-// bitmap of the passing keys and an ordered compaction into ascending
-// indices.
+// bitmap of the passing keys and the ordered set written from it.
 #include "common.cuh"
 #include "internal.h"
 #include "scan.cuh"
 #include "sparse_decode.h"
-
-#include <cooperative_groups.h>
-namespace cg = cooperative_groups;
 
 namespace sd {
 namespace {
 
 constexpr int kPowerIters = 8;
 constexpr int kChunk = 256;       // keys per CTA in the per-node passes
-constexpr int kLvThreads = 512;   // partition / compaction / filter CTAs
+constexpr int kLvThreads = 512;   // partition CTAs
 constexpr size_t kLvHeader = 4096;
-
 
 template <typename T, int EPL>
 __device__ __forceinline__ void load_elems(const T *p, float (&x)[EPL]) {
