@@ -517,48 +517,52 @@ def cpu_baseline_full(w, x, budget_s: float = 10.0):
 
 def run_reference(args, rank, world):
     """Reference arm: the CPU oracle timed on bounded samples of the workload.
-    A sample is one KV head's sub-problem (its G query heads) over the first
-    n keys of the cache with k scaled in proportion, sized so the whole run
-    takes about a minute; steps/s is scaled to full steps by the fraction of
-    the step's keys the sample covers."""
+    A sample is the whole step (every sequence and KV head, so the oracle's
+    parallel loops see the same work split as on a full step) over the first
+    n keys of the cache with k (or cap) scaled in proportion, sized so the
+    whole run takes about a minute; steps/s is scaled to full steps by the
+    fraction n / N of the keys the sample covers."""
     import oracle
     w = synth.WORKLOADS[args.workload]
-    x = synth.generate(w.with_(N=min(w.N, 131072)))
+    x = synth.generate(w)
     G = w.G
-    qr = synth.f32(x["q_route"][:1, :G])
-    ql = synth.f32(x["q_layers"][:, :1, :G])
-    K_all = synth.f32(x["K"][:1, :1])
-    V_all = synth.f32(x["V"][:1, :1])
+    qr = synth.f32(x["q_route"])
+    ql = synth.f32(x["q_layers"])
+    K_all = synth.f32(x["K"])
+    V_all = synth.f32(x["V"])
 
     threshold = w.mode == "threshold"
 
-    def sample(n):
-        kk = max(1, round(w.k * n / w.N))
-        if threshold:  # tau of the sample's own scores (untimed set-up)
-            tau = oracle.percentile_tau(oracle.scores(qr, K_all[:, :, :n]), *w.tau_pct)
-            capn = max(1, round(w.cap * n / w.N))
+    def prepare(n):
+        """Contiguous inputs of the n-key sample and its k or tau (untimed)."""
+        Kn = np.ascontiguousarray(K_all[:, :, :n])
+        Vn = np.ascontiguousarray(V_all[:, :, :n])
+        if threshold:  # tau of the sample's own scores
+            tau = oracle.percentile_tau(oracle.scores(qr, Kn), *w.tau_pct)
+            return Kn, Vn, dict(tau=tau, cap=max(1, round(w.cap * n / w.N)))
+        return Kn, Vn, dict(k=max(1, round(w.k * n / w.N)))
+
+    def sample(inputs):
+        Kn, Vn, sel = inputs
         t0 = time.perf_counter()
-        if threshold:
-            oracle.decode_step(qr, ql, K_all[:, :, :n], V_all[:, :, :n], tau=tau, cap=capn)
-        else:
-            oracle.decode_step(qr, ql, K_all[:, :, :n], V_all[:, :, :n], k=kk)
+        oracle.decode_step(qr, ql, Kn, Vn, **sel)
         return time.perf_counter() - t0
 
-    t_full_head = sample(w.N)                       # calibration, untimed
+    t_full = sample(prepare(w.N))                   # calibration, untimed
     budget = 60.0 / max(1, args.steps + args.warmup)
-    n = int(min(w.N, max(1024, w.N * budget / max(t_full_head, 1e-6))))
+    n = int(min(w.N, max(1024, w.N * budget / max(t_full, 1e-6))))
+    inputs = prepare(n)
     for _ in range(args.warmup):
-        sample(n)
-    t0 = time.perf_counter()
+        sample(inputs)
+    sec = 0.0
     for _ in range(args.steps):
-        sample(n)
-    sec = time.perf_counter() - t0
-    frac = (n / w.N) / (w.B * w.Hkv)                # share of one full step
+        sec += sample(inputs)
+    frac = n / w.N                                  # share of one full step
     value = args.steps * frac / sec
     sel = (f"tau = {w.tau_pct[0]}th-percentile score, cap {max(1, round(w.cap * n / w.N))}"
            if threshold else f"k={max(1, round(w.k * n / w.N))}")
-    desc = (f"{args.steps} samples, each the oracle decode step of one KV head "
-            f"(G={G} query heads, L={w.L}) over the first {n} of {w.N} keys with "
+    desc = (f"{args.steps} samples, each the oracle decode step of all {w.B * w.Hkv} KV "
+            f"heads (G={G}, L={w.L}) over the first {n} of {w.N} keys with "
             f"{sel}; value scaled by {frac:.3g} step per sample")
     return {
         "metric": LOUVER_METRIC if args.louver else METRIC, "value": round(value, 5),
