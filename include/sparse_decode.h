@@ -292,6 +292,18 @@ sparse_status_t sparse_louver_route_threshold(const sparse_shape_t *shape, const
                                               int32_t *count, int32_t *survivors, void *ws,
                                               size_t ws_bytes, void *stream);
 
+/* Self-test of failure detection, with no fault: one device thread waits,
+ * through the bounded wait that every counter barrier of the library uses
+ * (the split attention's merge, the Louver query's per-head barrier, the
+ * fused routing kernel), on a workspace word that nothing ever increments.
+ * After limit_ns of the GPU's global timer (capped at the library's own 2 s
+ * limit) the wait gives up and raises the TIMEOUT flag in the status word,
+ * so sparse_read_device_status then returns SPARSE_ERR_TIMEOUT and the
+ * context stays usable.  ws: any library workspace (>= 4096 bytes, 256-byte
+ * aligned); the word waited on is not used by any other call. */
+sparse_status_t sparse_selftest_bounded_wait(void *ws, size_t ws_bytes, uint64_t limit_ns,
+                                             void *stream);
+
 /* Shared routing, top-k form (as sparse_route_topk) for callers that cannot
  * allocate device memory: a plugin inside a host framework that owns every
  * device allocation, or code that must not call cudaMalloc once it is

@@ -170,3 +170,11 @@ def test_louver_arguments_rejected_before_device_work(lib):
                                              8, fake, fake, None, big, wb.value, None) == 1
     assert lib.sparse_louver_route_threshold(ctypes.byref(ok), fake, big, ib.value, 100, fake,
                                              8, fake, fake, None, big, wb.value, None) == 2
+
+
+def test_selftest_arguments_rejected(lib):
+    fake = ctypes.c_void_p(0x100000)
+    assert lib.sparse_selftest_bounded_wait(None, 1 << 20, 1000, None) == 1
+    assert lib.sparse_selftest_bounded_wait(ctypes.c_void_p(0x100010), 1 << 20, 1000, None) == 1
+    assert lib.sparse_selftest_bounded_wait(fake, 1024, 1000, None) == 1
+

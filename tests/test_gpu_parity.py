@@ -633,3 +633,22 @@ def test_decode_step_graph_equals_eager_step(dev, mode):
                     assert torch.equal(res[1][b, h, :n], ref["idx"][b, h, :n].cpu())
     sd.read_device_status(g.ws)
 
+
+def test_bounded_wait_expires_and_context_stays_usable(dev):
+    """Failure detection without a fault: the library's bounded wait, on a
+    counter nothing increments, gives up after its limit, reports
+    SPARSE_ERR_TIMEOUT through the status word, and the next calls on the
+    same workspace and stream run normally."""
+    import time
+    ws = sd.Workspace(dev)
+    t0 = time.perf_counter()
+    assert sd.selftest_bounded_wait(ws, limit_ns=100_000_000) == 7   # TIMEOUT
+    assert time.perf_counter() - t0 >= 0.09
+    assert sd.read_device_status(ws, raise_on_error=False) == 0       # status was reset
+    w = synth.custom(B=1, N=4096, Hq=8, Hkv=2, d=128, L=2, k=64, dtype="bf16", seed=3)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    res = sd.decode_step(t["q_route"], t["q_layers"], t["K"], t["V"], k=w.k, ws=ws)
+    ref = oracle.decode_step(_f(x["q_route"]), _f(x["q_layers"]), _f(x["K"]), _f(x["V"]), k=w.k)
+    assert_topk_within_band(res["idx"].cpu().numpy(), ref["S"], w.k)
+

@@ -27,7 +27,7 @@ __all__ = ["SparseDecodeError", "lib_path", "load", "score", "select_topk",
            "decode_step", "read_device_status", "workspace_bytes",
            "Workspace", "STATUS_NAMES", "EXPORTED_SYMBOLS", "decode_step_grouped",
            "kv_append", "LouverIndex", "louver_build", "louver_route_threshold",
-           "DecodeStepGraph"]
+           "DecodeStepGraph", "selftest_bounded_wait"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_PKG, "libsparse_decode.so")
@@ -46,6 +46,7 @@ EXPORTED_SYMBOLS = (
     "sparse_attn_gather", "sparse_decode_step", "sparse_read_device_status",
     "sparse_route_topk_static", "sparse_decode_step_grouped", "sparse_kv_append",
     "sparse_louver_sizes", "sparse_louver_build", "sparse_louver_route_threshold",
+    "sparse_selftest_bounded_wait",
 )
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
@@ -105,6 +106,7 @@ def load():
                                                  P, P, P, P, P, SZ, P]),
             "sparse_kv_append": (I32, [SH, P, P, P, P, P]),
             "sparse_louver_sizes": (I32, [SH, I32, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
+            "sparse_selftest_bounded_wait": (I32, [P, SZ, ctypes.c_uint64, P]),
             "sparse_louver_build": (I32, [SH, P, I32, P, SZ, P, SZ, P]),
             "sparse_louver_route_threshold": (I32, [SH, P, P, SZ, I32, P, I32, P, P, P, P,
                                                     SZ, P]),
@@ -200,6 +202,16 @@ def read_device_status(ws: Workspace, raise_on_error: bool = True) -> int:
     if raise_on_error:
         _check(rc, f"device status (flags=0x{flags.value:x})")
     return rc
+
+
+def selftest_bounded_wait(ws: Workspace, limit_ns: int = 50_000_000) -> int:
+    """Run the bounded-wait self-test on ws (a wait nothing satisfies, given
+    up after limit_ns) and return the device status it leaves: expected
+    SPARSE_ERR_TIMEOUT (7).  Resets the status word."""
+    buf = ws.get(1 << 20)
+    _check(load().sparse_selftest_bounded_wait(_ptr(buf), buf.numel(), int(limit_ns),
+                                               _stream()), "selftest_bounded_wait")
+    return read_device_status(ws, raise_on_error=False)
 
 
 def _dims_qk(q, K):

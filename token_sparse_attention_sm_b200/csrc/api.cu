@@ -5,6 +5,8 @@
 // stream and returns.  The library allocates nothing: scratch lives in the
 // caller's workspace, whose layout is
 //   [0, 4096)             header: device status word (uint32) at offset 0;
+//                         offset 64: a word no kernel writes (the bounded
+//                         wait self-test waits on it);
 //                         [256, 1024) attention split-merge counters;
 //                         [1024, 4096) fused-routing barrier counters, one
 //                         per head (fixed, shape-independent areas, zero
@@ -37,6 +39,7 @@ cudaError_t g_info_err[kMaxDevices];
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 constexpr size_t kHeader = 4096;
 constexpr size_t kCountersOff = 256;
+constexpr size_t kSelftestOff = 64;  // a header word no kernel writes
 constexpr size_t kRouteCountersOff = 1024;
 constexpr int kHistMinRows = 256;
 
@@ -469,6 +472,15 @@ sparse_status_t sparse_louver_route_threshold(const sparse_shape_t *shape, const
   if (index_bytes < ib || ws_bytes < wb) return SPARSE_ERR_WORKSPACE;
   return sd::from_cuda(sd::louver_query(s, q, r, index, tau, cap, idx, count, survivors, ws,
                                         static_cast<cudaStream_t>(stream)));
+}
+
+sparse_status_t sparse_selftest_bounded_wait(void *ws, size_t ws_bytes, uint64_t limit_ns,
+                                             void *stream) {
+  if (!ws || !sd::aligned(ws, 256) || ws_bytes < sd::kHeader) return SPARSE_ERR_INVALID_ARG;
+  // a header word that no kernel writes: the wait cannot be satisfied
+  uint32_t *ctr = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + sd::kSelftestOff);
+  return sd::from_cuda(sd::launch_selftest_wait(ctr, limit_ns, sd::status_word(ws),
+                                                static_cast<cudaStream_t>(stream)));
 }
 
 sparse_status_t sparse_read_device_status(void *ws, void *stream,

@@ -532,20 +532,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     __threadfence();
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(arrive) : "memory");
-    bool ok = true;
-    const uint64_t t0 = global_ns();
-    while (true) {
-      uint32_t v;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(arrive) : "memory");
-      if (v >= (uint32_t)csize) break;
-      if (global_ns() - t0 > kWaitLimitNs) {
-        raise_flag(status, FLAG_TIMEOUT);
-        ok = false;
-        break;
-      }
-      __nanosleep(64);
-    }
-    ready = ok;
+    ready = wait_counter_geq(arrive, (uint32_t)csize, kWaitLimitNs, status);
   }
   __syncthreads();
   if (ready) {

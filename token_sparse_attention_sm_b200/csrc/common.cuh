@@ -31,6 +31,25 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// Counter barriers in global memory: wait (one thread) until *ctr >= target,
+// with acquire loads and short sleeps; false, and the TIMEOUT flag, if that
+// has not happened within limit_ns of %globaltimer.  Every kernel whose CTAs
+// wait for one another waits here.
+__device__ __forceinline__ bool wait_counter_geq(const uint32_t *ctr, uint32_t target,
+                                                 uint64_t limit_ns, uint32_t *status) {
+  const uint64_t t0 = global_ns();
+  while (true) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if (global_ns() - t0 > limit_ns) {
+      raise_flag(status, FLAG_TIMEOUT);
+      return false;
+    }
+    __nanosleep(32);
+  }
+}
+
 // ---- programmatic dependent launch ----------------------------------------
 // Every kernel waits here before touching memory that an earlier kernel on
 // the stream may still be writing (a no-op unless launched with programmatic

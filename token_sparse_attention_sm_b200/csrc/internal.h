@@ -111,4 +111,9 @@ cudaError_t louver_query(const Shape &s, const void *q, int r, const void *index
                          const float *tau, int cap, int *idx, int *count, int *survivors,
                          void *ws, cudaStream_t st);
 
+// Self-test of the bounded wait (selftest.cu): one thread waits on *ctr >= 1
+// for limit_ns (at most the library's limit); nothing increments ctr.
+cudaError_t launch_selftest_wait(uint32_t *ctr, uint64_t limit_ns, uint32_t *status,
+                                 cudaStream_t st);
+
 }  // namespace sd

@@ -508,20 +508,7 @@ __global__ void __launch_bounds__(kQThreads)
   if (tid == 0) {
     uint32_t *arrive = done + 2 * bh;
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(arrive) : "memory");
-    bool ok = true;
-    const uint64_t t0 = global_ns();
-    while (true) {
-      uint32_t v;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(arrive) : "memory");
-      if (v >= (uint32_t)splits) break;
-      if (global_ns() - t0 > kWaitLimitNs) {
-        raise_flag(status, FLAG_TIMEOUT);
-        ok = false;
-        break;
-      }
-      __nanosleep(32);
-    }
-    ready = ok;
+    ready = wait_counter_geq(arrive, (uint32_t)splits, kWaitLimitNs, status);
   }
   __syncthreads();
   if (!ready) return;

@@ -93,16 +93,7 @@ __device__ __forceinline__ void arrive(uint32_t *ctr) {
 
 // thread 0 only: wait until *ctr >= target (bounded)
 __device__ bool wait_count(const uint32_t *ctr, uint32_t target, uint32_t *status) {
-  const uint64_t t0 = global_ns();
-  while (true) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-    if (v >= target) return true;
-    if (global_ns() - t0 > kWaitLimitNs) {
-      raise_flag(status, FLAG_TIMEOUT);
-      return false;
-    }
-  }
+  return wait_counter_geq(ctr, target, kWaitLimitNs, status);
 }
 
 // Bins taken from the top down: bnd[0] = the bin at which the running count
