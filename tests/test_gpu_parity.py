@@ -652,3 +652,73 @@ def test_bounded_wait_expires_and_context_stays_usable(dev):
     ref = oracle.decode_step(_f(x["q_route"]), _f(x["q_layers"]), _f(x["K"]), _f(x["V"]), k=w.k)
     assert_topk_within_band(res["idx"].cpu().numpy(), ref["S"], w.k)
 
+
+CANARY = -123456789
+
+
+def _fenced(shape, dtype, dev, pad=4096):
+    """A contiguous tensor of `shape` at the front of a larger buffer whose
+    tail holds a canary pattern."""
+    n = int(np.prod(shape))
+    if dtype in (torch.int32,):
+        buf = torch.full((n + pad,), CANARY, dtype=dtype, device=dev)
+    else:
+        buf = torch.full((n + pad,), -7.25, dtype=dtype, device=dev)
+    return buf, buf[:n].view(*shape)
+
+
+def _tail_intact(buf, n):
+    tail = buf[n:]
+    want = CANARY if buf.dtype == torch.int32 else -7.25
+    return bool((tail == want).all())
+
+
+def test_no_call_writes_past_its_outputs(dev):
+    """Canary words after every output buffer (scores, index sets, counts,
+    attention outputs and lse, the Louver set) stay untouched, including a
+    threshold set that overflows its capacity."""
+    w = synth.custom(B=2, N=8192, Hq=8, Hkv=2, d=128, L=3, k=100, dtype="bf16", seed=41,
+                     heavy=4, blobs=0)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    B, Hkv, N, L, Hq, d, k = w.B, w.Hkv, w.N, w.L, w.Hq, w.d, w.k
+    ws = sd.Workspace(dev)
+    bS, S = _fenced((B, Hkv, N), torch.float32, dev)
+    sd.score(t["q_route"], t["K"], ws=ws, out=S)
+    assert _tail_intact(bS, S.numel())
+    bi, idx = _fenced((B, Hkv, k), torch.int32, dev)
+    sd.route_topk(t["q_route"], t["K"], k, ws=ws, idx=idx)
+    assert _tail_intact(bi, idx.numel())
+    bi2, idx2 = _fenced((B, Hkv, k), torch.int32, dev)
+    sd.select_topk(S, k, ws=ws, idx=idx2)
+    assert _tail_intact(bi2, idx2.numel())
+    cap = 64   # far below the set size: capacity overflow
+    tau = torch.zeros((B, Hkv), device=dev)
+    for fn in (lambda i, c: sd.route_threshold(t["q_route"], t["K"], tau, cap, ws=ws,
+                                               check=False, idx=i, count=c),
+               lambda i, c: sd.select_threshold(S, tau, cap, ws=ws, check=False, idx=i,
+                                                count=c)):
+        bti, ti = _fenced((B, Hkv, cap), torch.int32, dev)
+        btc, tc = _fenced((B, Hkv), torch.int32, dev)
+        fn(ti, tc)
+        assert sd.read_device_status(ws, raise_on_error=False) == 4
+        assert _tail_intact(bti, ti.numel()) and _tail_intact(btc, tc.numel())
+        assert int(tc.min()) > cap
+    bo, out = _fenced((L, B, Hq, d), torch.bfloat16, dev)
+    bl, lse = _fenced((L, B, Hq), torch.float32, dev)
+    sd.attn_gather(t["q_layers"], t["K"], t["V"], idx, ws=ws, out=out, lse=lse)
+    assert _tail_intact(bo, out.numel()) and _tail_intact(bl, lse.numel())
+    bo2, out2 = _fenced((L, B, Hq, d), torch.bfloat16, dev)
+    bl2, lse2 = _fenced((L, B, Hq), torch.float32, dev)
+    bi3, idx3 = _fenced((B, Hkv, k), torch.int32, dev)
+    sd.decode_step(t["q_route"], t["q_layers"], t["K"], t["V"], k=k, ws=ws, out=out2,
+                   lse=lse2, idx=idx3)
+    assert _tail_intact(bo2, out2.numel()) and _tail_intact(bl2, lse2.numel())
+    assert _tail_intact(bi3, idx3.numel())
+    ix = sd.louver_build(t["K"], 128)
+    bli, li = _fenced((B, Hkv, cap), torch.int32, dev)
+    blc, lc = _fenced((B, Hkv), torch.int32, dev)
+    sd.louver_route_threshold(t["q_route"], t["K"], ix, tau, cap, check=False, idx=li, count=lc)
+    assert sd.read_device_status(ix.ws, raise_on_error=False) == 4
+    assert _tail_intact(bli, li.numel()) and _tail_intact(blc, lc.numel())
+

@@ -262,16 +262,29 @@ def select_topk(S, k: int, ws: Workspace | None = None, check: bool = True,
     return idx
 
 
+def _threshold_outputs(idx, count, B, Hkv, cap, device):
+    """idx [B,Hkv,cap] and count [B,Hkv] int32: the given ones (checked) or
+    new ones."""
+    if idx is None:
+        idx = torch.empty((B, Hkv, cap), dtype=torch.int32, device=device)
+    if count is None:
+        count = torch.empty((B, Hkv), dtype=torch.int32, device=device)
+    _need_cuda(idx, count)
+    if (idx.shape != (B, Hkv, cap) or count.shape != (B, Hkv) or idx.dtype != torch.int32
+            or count.dtype != torch.int32):
+        raise ValueError("idx must be int32 [B,Hkv,cap] and count int32 [B,Hkv]")
+    return idx, count
+
+
 def select_threshold(S, tau, cap: int, ws: Workspace | None = None,
-                     check: bool = True):
+                     check: bool = True, idx=None, count=None):
     """Threshold sets of S: (idx [B,Hkv,cap], count [B,Hkv])."""
     _need_cuda(S, tau)
     B, Hkv, N = S.shape
     w = _ws(ws, S.device)
     sh = _shape(B, N, Hkv, Hkv, 64, torch.float32)
     buf = w.get(workspace_bytes(B, N, Hkv, Hkv, 64, torch.float32, cap, 1))
-    idx = torch.empty((B, Hkv, cap), dtype=torch.int32, device=S.device)
-    count = torch.empty((B, Hkv), dtype=torch.int32, device=S.device)
+    idx, count = _threshold_outputs(idx, count, B, Hkv, cap, S.device)
     _check(load().sparse_select_threshold(
         ctypes.byref(sh), _ptr(S), _ptr(tau.float().contiguous()), int(cap),
         _ptr(idx), _ptr(count), _ptr(buf), buf.numel(), _stream()),
@@ -302,7 +315,7 @@ def route_topk(q, K, k: int, ws: Workspace | None = None, check: bool = True,
 
 
 def route_threshold(q, K, tau, cap: int, ws: Workspace | None = None,
-                    check: bool = True, n: int | None = None):
+                    check: bool = True, n: int | None = None, idx=None, count=None):
     """Shared routing (threshold): (idx [B,Hkv,cap], count [B,Hkv]), over the
     first n cache rows (default: all rows of K)."""
     _need_cuda(q, K, tau)
@@ -311,8 +324,7 @@ def route_threshold(q, K, tau, cap: int, ws: Workspace | None = None,
     w = _ws(ws, q.device)
     sh = _shape(B, N, Hq, Hkv, d, q.dtype, Ncap)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, cap, 1))
-    idx = torch.empty((B, Hkv, cap), dtype=torch.int32, device=q.device)
-    count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    idx, count = _threshold_outputs(idx, count, B, Hkv, cap, q.device)
     tau = tau.float().contiguous()
     _check(load().sparse_route_threshold(
         ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(tau), int(cap), _ptr(idx),
