@@ -599,10 +599,11 @@ def percentile_tau_device(sd, q_route, K, ws, num=97, den=100):
 
 
 def run_native_louver(args, rank, world, local_rank):
-    """One step = threshold routing through the Louver index (ball tests,
-    exact checks of the surviving clusters, ordered compaction) and the
-    attention of all L layers over that set.  The full-scan threshold step
-    (score scan, threshold select, attention) is timed beside it."""
+    """One step = one sparse_louver_decode_step: threshold routing through the
+    Louver index (ball tests, exact checks of the surviving clusters, the
+    ordered set) and the attention of all L layers over that set.  The
+    full-scan threshold step (score scan, threshold select, attention) is
+    timed beside it."""
     import token_sparse_attention_sm_b200 as sd
 
     torch.cuda.set_device(local_rank)
@@ -645,8 +646,10 @@ def run_native_louver(args, rank, world, local_rank):
                                           check=False, out=o["out"], lse=o["lse"])
 
         def step_fn(i):
-            a, b = route_fn(i), attn_fn(i)
-            return lambda: (a(), b())
+            o = outs[i]
+            return lambda: sd.louver_decode_step(qs[i][0], qs[i][1], K, V, ix, taus[i], cap,
+                                                 ws=ws, check=False, out=o["out"],
+                                                 idx=o["idx"], count=o["count"], lse=o["lse"])
 
         def full_fn(i):
             o = outs[i]
@@ -778,9 +781,8 @@ def run_e2e_louver(sd, w, variants, K, V, ix, taus, ws, stream, dev, args, world
         (hqr, hql), (dqr, dql) = hq[j], dq[j]
         dqr.copy_(hqr, non_blocking=True)
         dql.copy_(hql, non_blocking=True)
-        sd.louver_route_threshold(dqr, K, ix, taus[j], w.cap, check=False, idx=idx_d, count=cnt_d)
-        sd.attn_gather(dql, K, V, idx_d, count=cnt_d, ws=ws, check=False, out=out_d,
-                       return_lse=False)
+        sd.louver_decode_step(dqr, dql, K, V, ix, taus[j], w.cap, ws=ws, check=False,
+                              out=out_d, idx=idx_d, count=cnt_d, return_lse=False)
         out_h.copy_(out_d, non_blocking=True)
         idx_h.copy_(idx_d, non_blocking=True)
         cnt_h.copy_(cnt_d, non_blocking=True)
@@ -799,8 +801,7 @@ def run_e2e_louver(sd, w, variants, K, V, ix, taus, ws, stream, dev, args, world
     sec = sdist.max_over_ranks(t1 - t0)
     return {"value": round(world * steps / sec, 2), "unit": "steps/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "api": "token_sparse_attention_sm_b200.louver_route_threshold + attn_gather "
-                   "(eager, per-step sync)"}
+            "api": "token_sparse_attention_sm_b200.louver_decode_step (eager, per-step sync)"}
 
 
 def cpu_baseline_threshold(w, x, budget_s: float = 10.0):

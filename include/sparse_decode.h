@@ -292,6 +292,23 @@ sparse_status_t sparse_louver_route_threshold(const sparse_shape_t *shape, const
                                               int32_t *count, int32_t *survivors, void *ws,
                                               size_t ws_bytes, void *stream);
 
+/* One decode step with threshold routing through the Louver index: the set
+ * of sparse_louver_route_threshold (q_route, tau [B,Hkv], cap), then every
+ * layer's attention over it, as sparse_decode_step does in threshold mode
+ * (the same outputs as that call on the indexed keys).  Two workspaces:
+ * louver_ws (the index's, sizes from sparse_louver_sizes) and ws
+ * (sparse_workspace_size(shape, cap, L)); device conditions of both parts
+ * are reported in ws's status word.  K, V [B,Hkv,n_cap,d] are the cache the
+ * index was built from (its first N rows); idx [B,Hkv,cap], count [B,Hkv],
+ * out [L,B,Hq,d], lse [L,B,Hq] or NULL. */
+sparse_status_t sparse_louver_decode_step(const sparse_shape_t *shape, int32_t L,
+                                          const void *q_route, const void *q_layers,
+                                          const void *K, const void *V, const void *index,
+                                          size_t index_bytes, int32_t r, const float *tau,
+                                          int32_t cap, int32_t *idx, int32_t *count, void *out,
+                                          float *lse, void *louver_ws, size_t louver_ws_bytes,
+                                          void *ws, size_t ws_bytes, void *stream);
+
 /* Self-test of failure detection, with no fault: one device thread waits,
  * through the bounded wait that every counter barrier of the library uses
  * (the split attention's merge, the Louver query's per-head barrier, the

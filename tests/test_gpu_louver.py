@@ -253,3 +253,32 @@ def test_louver_large_sets_several_compaction_passes(dev, cap):
     _assert_same_set(a, f, cap)
     assert st_a == st_f == (4 if int(a[1][0, 0]) > cap else 0)
     assert int(a[1][0, 0]) > 65536
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_louver_decode_step_equals_route_then_gather(dev, dtype, d):
+    """The fused Louver step returns exactly what routing through the index
+    followed by the gather attention returns, and its attention matches the
+    oracle on the oracle's threshold set."""
+    w = synth.custom(B=1, N=8192, Hq=8, Hkv=2, d=d, L=4, dtype=dtype, seed=23,
+                     mode="threshold", cap=2048, blobs=16)
+    x = synth.generate(w)
+    t = {n: x[n].to(dev) for n in ("q_route", "q_layers", "K", "V")}
+    q32, K32 = _f(x["q_route"]), _f(x["K"])
+    S = oracle.scores(q32, K32)
+    tau = oracle.percentile_tau(S, 95, 100)
+    taud = torch.from_numpy(tau).to(dev)
+    ix = sd.louver_build(t["K"], 128)
+    res = sd.louver_decode_step(t["q_route"], t["q_layers"], t["K"], t["V"], ix, taud, w.cap)
+    gidx, gcnt = sd.louver_route_threshold(t["q_route"], t["K"], ix, taud, w.cap)
+    o, l = sd.attn_gather(t["q_layers"], t["K"], t["V"], gidx, count=gcnt)
+    _assert_same_set((res["idx"], res["count"]), (gidx, gcnt), w.cap)
+    assert torch.equal(res["out"], o) and torch.equal(res["lse"], l)
+    ridx, rcnt = oracle.threshold(S, tau, w.cap)
+    _check_set(res["idx"].cpu().numpy(), res["count"].cpu().numpy(), q32, K32, tau, w.cap)
+    o_ref, l_ref = oracle.attn(_f(x["q_layers"]), K32, _f(x["V"]), ridx, rcnt)
+    o_gpu, l_gpu = sd.attn_gather(t["q_layers"], t["K"], t["V"], torch.from_numpy(ridx).to(dev),
+                                  count=torch.from_numpy(rcnt).to(dev))
+    tol = 2e-2 if dtype == "bf16" else 1e-4
+    assert np.abs(o_gpu.float().cpu().numpy() - o_ref).max() <= tol
+

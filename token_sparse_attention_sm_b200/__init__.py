@@ -27,7 +27,7 @@ __all__ = ["SparseDecodeError", "lib_path", "load", "score", "select_topk",
            "decode_step", "read_device_status", "workspace_bytes",
            "Workspace", "STATUS_NAMES", "EXPORTED_SYMBOLS", "decode_step_grouped",
            "kv_append", "LouverIndex", "louver_build", "louver_route_threshold",
-           "DecodeStepGraph", "selftest_bounded_wait"]
+           "DecodeStepGraph", "selftest_bounded_wait", "louver_decode_step"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_PKG, "libsparse_decode.so")
@@ -46,7 +46,7 @@ EXPORTED_SYMBOLS = (
     "sparse_attn_gather", "sparse_decode_step", "sparse_read_device_status",
     "sparse_route_topk_static", "sparse_decode_step_grouped", "sparse_kv_append",
     "sparse_louver_sizes", "sparse_louver_build", "sparse_louver_route_threshold",
-    "sparse_selftest_bounded_wait",
+    "sparse_selftest_bounded_wait", "sparse_louver_decode_step",
 )
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
@@ -107,6 +107,8 @@ def load():
             "sparse_kv_append": (I32, [SH, P, P, P, P, P]),
             "sparse_louver_sizes": (I32, [SH, I32, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
             "sparse_selftest_bounded_wait": (I32, [P, SZ, ctypes.c_uint64, P]),
+            "sparse_louver_decode_step": (I32, [SH, I32, P, P, P, P, P, SZ, I32, P, I32, P, P,
+                                                P, P, P, SZ, P, SZ, P]),
             "sparse_louver_build": (I32, [SH, P, I32, P, SZ, P, SZ, P]),
             "sparse_louver_route_threshold": (I32, [SH, P, P, SZ, I32, P, I32, P, P, P, P,
                                                     SZ, P]),
@@ -668,4 +670,39 @@ class DecodeStepGraph:
         if self.count_host is None:
             return self.out_host, self.idx_host
         return self.out_host, self.idx_host, self.count_host
+
+
+def louver_decode_step(q_route, q_layers, K, V, index: LouverIndex, tau, cap: int,
+                       ws: Workspace | None = None, check: bool = True, out=None, idx=None,
+                       count=None, lse=None, return_lse: bool = True):
+    """One decode step with threshold routing through a Louver index, then
+    every layer's attention over the set.  Returns dict(idx, count, out, lse)
+    (as decode_step in threshold mode)."""
+    _need_cuda(q_route, q_layers, K, V, tau)
+    B, Ncap, Hq, Hkv, d = _dims_qk(q_route, K)
+    if (B, Hkv, Ncap, d, K.dtype) != (index.B, index.Hkv, index.Ncap, index.d, index.dtype):
+        raise ValueError("the index was built for another K")
+    L = q_layers.shape[0]
+    if q_layers.shape != (L, B, Hq, d) or V.shape != K.shape:
+        raise ValueError("q_layers must be [L,B,Hq,d] and V like K")
+    dev = q_route.device
+    w = _ws(ws, dev)
+    N = index.N
+    sh = _shape(B, N, Hq, Hkv, d, q_route.dtype, Ncap)
+    buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q_route.dtype, cap, L))
+    idx, count = _threshold_outputs(idx, count, B, Hkv, cap, dev)
+    if out is None:
+        out = torch.empty_like(q_layers)
+    if lse is None and return_lse:
+        lse = torch.empty((L, B, Hq), dtype=torch.float32, device=dev)
+    tau = tau.float().contiguous()
+    lbuf = index.ws.get(index.ws_bytes)
+    _check(load().sparse_louver_decode_step(
+        ctypes.byref(sh), L, _ptr(q_route), _ptr(q_layers), _ptr(K), _ptr(V),
+        _ptr(index.index), index.index.numel(), index.r, _ptr(tau), int(cap), _ptr(idx),
+        _ptr(count), _ptr(out), _ptr(lse), _ptr(lbuf), lbuf.numel(), _ptr(buf), buf.numel(),
+        _stream()), "louver_decode_step")
+    if check:
+        read_device_status(w)
+    return {"idx": idx, "count": count, "out": out, "lse": lse}
 

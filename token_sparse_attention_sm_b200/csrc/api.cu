@@ -471,7 +471,38 @@ sparse_status_t sparse_louver_route_threshold(const sparse_shape_t *shape, const
   sd::louver_sizes(s, r, &ib, &wb);
   if (index_bytes < ib || ws_bytes < wb) return SPARSE_ERR_WORKSPACE;
   return sd::from_cuda(sd::louver_query(s, q, r, index, tau, cap, idx, count, survivors, ws,
-                                        static_cast<cudaStream_t>(stream)));
+                                        nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+sparse_status_t sparse_louver_decode_step(const sparse_shape_t *shape, int32_t L,
+                                          const void *q_route, const void *q_layers,
+                                          const void *K, const void *V, const void *index,
+                                          size_t index_bytes, int32_t r, const float *tau,
+                                          int32_t cap, int32_t *idx, int32_t *count, void *out,
+                                          float *lse, void *louver_ws, size_t louver_ws_bytes,
+                                          void *ws, size_t ws_bytes, void *stream) {
+  Shape s;
+  sparse_status_t rc = sd::check_shape(shape, &s);
+  if (rc != SPARSE_OK) return rc;
+  if ((rc = sd::check_decode_args(s, L, q_route, q_layers, K, V, 0, tau, cap, idx, count, out,
+                                  lse)) != SPARSE_OK)
+    return rc;
+  if (!index || !louver_ws || !sd::aligned(index, 256) || !sd::aligned(louver_ws, 256))
+    return SPARSE_ERR_INVALID_ARG;
+  if (!sd::louver_shape_ok(s, r)) return SPARSE_ERR_UNSUPPORTED;
+  size_t ib = 0, wb = 0;
+  sd::louver_sizes(s, r, &ib, &wb);
+  if (index_bytes < ib || louver_ws_bytes < wb) return SPARSE_ERR_WORKSPACE;
+  if ((rc = sd::check_ws(s, cap, L, ws, ws_bytes)) != SPARSE_OK) return rc;
+  const sd::Layout l = sd::layout(s, cap, L);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // one status word for the step: the attention workspace's
+  cudaError_t e = sd::louver_query(s, q_route, r, index, tau, cap, idx, count, nullptr,
+                                   louver_ws, sd::status_word(ws), st);
+  if (e == cudaSuccess)
+    e = sd::launch_attn(s, L, q_layers, K, V, idx, cap, count, cap, out, lse, sd::attn_ptr(ws, l),
+                        sd::attn_counters(ws), sd::status_word(ws), st);
+  return sd::from_cuda(e);
 }
 
 sparse_status_t sparse_selftest_bounded_wait(void *ws, size_t ws_bytes, uint64_t limit_ns,

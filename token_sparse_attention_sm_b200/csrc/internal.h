@@ -107,9 +107,10 @@ bool louver_shape_ok(const Shape &s, int r);
 void louver_sizes(const Shape &s, int r, size_t *index_bytes, size_t *ws_bytes);
 cudaError_t louver_build(const Shape &s, const void *K, int r, void *index, void *ws,
                          cudaStream_t st);
+// status: the status word to raise flags in (nullptr: the Louver workspace's).
 cudaError_t louver_query(const Shape &s, const void *q, int r, const void *index,
                          const float *tau, int cap, int *idx, int *count, int *survivors,
-                         void *ws, cudaStream_t st);
+                         void *ws, uint32_t *status, cudaStream_t st);
 
 // Self-test of the bounded wait (selftest.cu): one thread waits on *ctr >= 1
 // for limit_ns (at most the library's limit); nothing increments ctr.

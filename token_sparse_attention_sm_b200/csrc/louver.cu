@@ -645,7 +645,8 @@ cudaError_t lv_build_t(const Shape &s, const void *Kv, int r, char *index, char 
 
 template <typename T, int D>
 cudaError_t lv_query_t(const Shape &s, const void *qv, int r, const char *index, const float *tau,
-                       int cap, int *idx, int *count, int *survivors, char *ws, cudaStream_t st) {
+                       int cap, int *idx, int *count, int *survivors, char *ws,
+                       uint32_t *status, cudaStream_t st) {
   using C = ScoreCfg<T, D>;
   const LvLayout l = lv_layout(s, r);
   const int nc = s.N / r;
@@ -689,7 +690,7 @@ cudaError_t lv_query_t(const Shape &s, const void *qv, int r, const char *index,
                          reinterpret_cast<uint32_t *>(ws + l.parity),
                          reinterpret_cast<int *>(ws + l.nsurv),
                          reinterpret_cast<uint32_t *>(ws + l.done), idx, count, survivors,
-                         reinterpret_cast<uint32_t *>(ws));
+                         status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -717,15 +718,18 @@ cudaError_t louver_build(const Shape &s, const void *K, int r, void *index, void
 
 cudaError_t louver_query(const Shape &s, const void *q, int r, const void *index,
                          const float *tau, int cap, int *idx, int *count, int *survivors,
-                         void *ws, cudaStream_t st) {
+                         void *ws, uint32_t *status, cudaStream_t st) {
   const char *ix = static_cast<const char *>(index);
   char *w = static_cast<char *>(ws);
+  if (!status) status = reinterpret_cast<uint32_t *>(ws);
   if (s.dtype == 1)
-    return s.d == 128
-               ? lv_query_t<__nv_bfloat16, 128>(s, q, r, ix, tau, cap, idx, count, survivors, w, st)
-               : lv_query_t<__nv_bfloat16, 64>(s, q, r, ix, tau, cap, idx, count, survivors, w, st);
-  return s.d == 128 ? lv_query_t<float, 128>(s, q, r, ix, tau, cap, idx, count, survivors, w, st)
-                    : lv_query_t<float, 64>(s, q, r, ix, tau, cap, idx, count, survivors, w, st);
+    return s.d == 128 ? lv_query_t<__nv_bfloat16, 128>(s, q, r, ix, tau, cap, idx, count,
+                                                       survivors, w, status, st)
+                      : lv_query_t<__nv_bfloat16, 64>(s, q, r, ix, tau, cap, idx, count,
+                                                      survivors, w, status, st);
+  return s.d == 128
+             ? lv_query_t<float, 128>(s, q, r, ix, tau, cap, idx, count, survivors, w, status, st)
+             : lv_query_t<float, 64>(s, q, r, ix, tau, cap, idx, count, survivors, w, status, st);
 }
 
 }  // namespace sd
