@@ -99,6 +99,8 @@ CASES = [
     # more than 16 heads: each head's clusters owned by CTAs of that head only
     dict(B=3, N=2048, Hq=8, Hkv=8, d=64, dtype="bf16", r=64, blobs=4, pct=90),
     dict(B=5, N=4096, Hq=16, Hkv=4, d=128, dtype="f32", r=128, blobs=8, pct=97),
+    # more heads than SMs: one CTA per head, the grid takes more than one wave
+    dict(B=40, N=1024, Hq=8, Hkv=4, d=64, dtype="bf16", r=32, blobs=4, pct=90),
 ]
 
 
