@@ -722,3 +722,46 @@ def test_no_call_writes_past_its_outputs(dev):
     assert sd.read_device_status(ix.ws, raise_on_error=False) == 4
     assert _tail_intact(bli, li.numel()) and _tail_intact(blc, lc.numel())
 
+
+@pytest.mark.parametrize("B,N,Hkv,d,dtype,pct,cap", [(2, 5003, 2, 128, "bf16", 90, 600),
+                                                     (1, 131072, 8, 128, "bf16", 97, 8192),
+                                                     (3, 777, 4, 64, "f32", 50, 200),
+                                                     (1, 4096, 2, 64, "bf16", 99, 5)])
+def test_route_threshold_equals_select_on_its_scores(dev, B, N, Hkv, d, dtype, pct, cap):
+    """The marking scan + bitmap compaction gives exactly the threshold select
+    of the scan's own scores (same fp32 scores, same comparison): counts and
+    index rows bitwise, capacity overflow included; and the oracle's set
+    within the band."""
+    w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=d, L=1, dtype=dtype, seed=N + pct,
+                     mode="threshold", cap=cap)
+    x = synth.generate(w)
+    t = _to(dev, x, ("q_route", "K"))
+    q32, K32 = _f(x["q_route"]), _f(x["K"])
+    S = oracle.scores(q32, K32)
+    tau = oracle.percentile_tau(S, pct, 100)
+    taud = torch.from_numpy(tau).to(dev)
+    ws = sd.Workspace(dev)
+    gi, gc = sd.route_threshold(t["q_route"], t["K"], taud, cap, ws=ws, check=False)
+    st1 = sd.read_device_status(ws, raise_on_error=False)
+    Sg = sd.score(t["q_route"], t["K"], ws=ws)
+    si, sc = sd.select_threshold(Sg, taud, cap, ws=ws, check=False)
+    st2 = sd.read_device_status(ws, raise_on_error=False)
+    assert st1 == st2
+    np.testing.assert_array_equal(gc.cpu().numpy(), sc.cpu().numpy())
+    gi, si, gcn = gi.cpu().numpy(), si.cpu().numpy(), gc.cpu().numpy()
+    for b in range(B):
+        for h in range(Hkv):
+            n = min(int(gcn[b, h]), cap)
+            np.testing.assert_array_equal(gi[b, h, :n], si[b, h, :n])
+    S64 = oracle.scores(q32, K32, np.float64)
+    ridx, rcnt = oracle.threshold(S, tau, cap)
+    for b in range(B):
+        for h in range(Hkv):
+            band = _band(tau[b, h])
+            assert abs(int(gcn[b, h]) - int(rcnt[b, h])) <= int(np.sum(np.abs(S[b, h] - tau[b, h]) <= band))
+            if gcn[b, h] <= cap:
+                g = set(gi[b, h, :gcn[b, h]].tolist())
+                must = set(np.nonzero(S64[b, h] >= tau[b, h] + band)[0].tolist())
+                never = set(np.nonzero(S64[b, h] < tau[b, h] - band)[0].tolist())
+                assert must <= g and not (g & never)
+

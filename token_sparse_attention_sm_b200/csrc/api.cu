@@ -137,6 +137,18 @@ cudaError_t route_topk_any(const Shape &s, const void *q, const void *K, int k, 
   return e;
 }
 
+// A1 + A2' (threshold): the scan marks the keys >= tau in per-head bitmaps
+// (in the scores area, which threshold routing does not need), then one
+// cluster per head writes the ordered sets.
+cudaError_t route_threshold_any(const Shape &s, const void *q, const void *K, const float *tau,
+                                int cap, int *idx, int *count, void *ws, const Layout &l,
+                                cudaStream_t st) {
+  uint32_t *bits = reinterpret_cast<uint32_t *>(scores_ptr(ws, l));
+  cudaError_t e = launch_threshold_mark(s, q, K, tau, bits, status_word(ws), st);
+  if (e == cudaSuccess) e = launch_bitmap_compact(s, bits, cap, idx, count, status_word(ws), st);
+  return e;
+}
+
 }  // namespace
 
 bool cooperative_forced() {
@@ -211,10 +223,7 @@ cudaError_t decode_step_enqueue(const Shape &s, int L, const void *q_route,
   if (topk) {
     e = route_topk_any(s, q_route, K, k, idx, ws, l, st);
   } else {
-    float *S = scores_ptr(ws, l);
-    e = launch_score(s, q_route, K, S, nullptr, status, st);
-    if (e == cudaSuccess)
-      e = launch_select(s, S, 0, tau, cap, idx, count, cap, nullptr, status, st);
+    e = route_threshold_any(s, q_route, K, tau, cap, idx, count, ws, l, st);
   }
   if (e == cudaSuccess)
     e = launch_attn(s, L, q_layers, K, V, idx, stride, topk ? nullptr : count, stride, out,
@@ -341,12 +350,7 @@ sparse_status_t sparse_route_threshold(const sparse_shape_t *shape,
   if ((r = sd::check_ws(s, cap, 1, ws, ws_bytes)) != SPARSE_OK) return r;
   const sd::Layout l = sd::layout(s, cap, 1);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float *S = sd::scores_ptr(ws, l);
-  cudaError_t e = sd::launch_score(s, q, K, S, nullptr, sd::status_word(ws), st);
-  if (e == cudaSuccess)
-    e = sd::launch_select(s, S, 0, tau, cap, idx, count, cap, nullptr,
-                          sd::status_word(ws), st);
-  return sd::from_cuda(e);
+  return sd::from_cuda(sd::route_threshold_any(s, q, K, tau, cap, idx, count, ws, l, st));
 }
 
 sparse_status_t sparse_attn_gather(const sparse_shape_t *shape, int32_t L,

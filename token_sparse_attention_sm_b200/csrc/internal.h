@@ -117,4 +117,13 @@ cudaError_t louver_query(const Shape &s, const void *q, int r, const void *index
 cudaError_t launch_selftest_wait(uint32_t *ctr, uint64_t limit_ns, uint32_t *status,
                                  cudaStream_t st);
 
+// A2' by marking: the scan writes, per 32 keys, the word of bits "score >=
+// tau[head]" into bits [B*Hkv][ceil(N/32)] (score.cu); the compaction turns
+// the words into ascending idx rows (stride cap) and counts (threshold.cu).
+cudaError_t launch_threshold_mark(const Shape &s, const void *q, const void *K,
+                                  const float *tau, uint32_t *bits, uint32_t *status,
+                                  cudaStream_t st);
+cudaError_t launch_bitmap_compact(const Shape &s, const uint32_t *bits, int cap, int *idx,
+                                  int *count, uint32_t *status, cudaStream_t st);
+
 }  // namespace sd

@@ -358,6 +358,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
     o.shist = shist;
     o.keys = keys;
     o.key_off = -jlo;
+    o.bits = nullptr;
+    o.tau = nullptr;
     scan_tiles<T, D, 1>(q, K, N, kv_rows, Hq, Hkv, tph, (long long)bh * tph + tl, th - tl, bh,
                         scale,
                         smem, full, empty, o, status);

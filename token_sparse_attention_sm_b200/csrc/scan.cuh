@@ -127,6 +127,12 @@ struct ScanOut {
   uint32_t *shist;
   uint32_t *keys;
   int key_off;
+  // threshold marking (scan_tiles<..., true>): bits [heads][ceil(N/32)] gets,
+  // for each 32-key word, bit t set iff key 32*word + t scores >= tau[head]
+  // (order-preserving keys compared, as the threshold select compares);
+  // nothing else is written.
+  uint32_t *bits;
+  const float *tau;
 };
 
 // One CTA's share of the scan: tiles [t_begin, t_begin + ntiles).  K holds
@@ -135,7 +141,7 @@ struct ScanOut {
 // the last ones to land, its other lanes (and any further warps) return at
 // once.  Barriers full/empty
 // must be initialised (count 1 / kScanConsumerWarps).
-template <typename T, int D, int kSlots>
+template <typename T, int D, int kSlots, bool kMark = false>
 __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__restrict__ K,
                                            int N, int kv_rows, int Hq, int Hkv,
                                            int tiles_per_head,
@@ -176,6 +182,8 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
   // ---- consumers ------------------------------------------------------------
   const int sub = lane % C::kLpk;  // which 16-byte slice of the row
   int cur_bh = -1;
+  uint32_t tkey = 0;  // threshold marking: order key of the head's tau
+  const int nw = (N + 31) / 32;
   float qs[C::kEpl];
   for (int i = 0; i < ntiles; ++i) {
     const int s = i % kScanStages;
@@ -186,10 +194,15 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
     if (bh != cur_bh) {
       cur_bh = bh;
       load_qbar<T, D>(q, bh, Hq, Hkv, sub, scale, qs);
+      if constexpr (kMark) {
+        const float tv = o.tau[bh];
+        tkey = order_key(tv);
+        if (!isfinite(tv) && lane == 0 && warp == 0) raise_flag(status, FLAG_NONFINITE);
+      }
     }
     if (!mbar_wait(&full[s], (i / kScanStages) & 1, status)) break;
     const unsigned char *stage = ring + (size_t)s * kScanStageBytes;
-    float *Srow = o.S + (size_t)bh * N + j0;
+    float *Srow = kMark ? nullptr : o.S + (size_t)bh * N + j0;
     const int slot = bh - bh_first;
     uint32_t *krow = (o.keys && slot == 0) ? o.keys + o.key_off + j0 : nullptr;
     for (int wt = warp; wt < C::kWarpTiles; wt += kScanConsumerWarps) {
@@ -198,7 +211,12 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
       const float score = warp_tile_scores<T, D>(stage, key0, qs, lane);
       const int kk = key0 + sub * C::kKpr + lane / C::kLpk;
       const bool valid = kk < nk;
-      if (valid) {
+      if constexpr (kMark) {
+        // one word per 32 keys, written whole by this warp (no atomics)
+        const bool pass = valid && order_key(score) >= tkey;
+        const uint32_t word = __reduce_or_sync(0xffffffffu, pass ? 1u << (kk - key0) : 0u);
+        if (lane == 0) o.bits[(size_t)bh * nw + (j0 + key0) / 32] = word;
+      } else if (valid) {
         Srow[kk] = score;
         const uint32_t key = order_key(score);
         if (krow) krow[kk] = key;

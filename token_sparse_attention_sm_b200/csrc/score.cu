@@ -76,6 +76,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   o.shist = shist;
   o.keys = nullptr;
   o.key_off = 0;
+  o.bits = nullptr;
+  o.tau = nullptr;
   scan_tiles<T, D, kHistSlots>(q, K, N, kv_rows, Hq, Hkv, tiles_per_head, t_begin, ntiles,
                                bh_first,
                                scale, smem, full, empty, o, status);
@@ -90,6 +92,75 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       if (c) atomicAdd(&hist[(size_t)(bh_first + i / kScanBins) * kScanBins + (i % kScanBins)], c);
     }
   }
+}
+
+// A1 + A2' for the full-scan threshold routing: the same scan, but instead of
+// the scores it writes, per 32 keys, the word of bits "score >= tau" (one
+// plain store per warp tile: the words are owned by one warp each, every word
+// of a head is rewritten on every call, so nothing needs clearing).
+template <typename T, int D>
+__global__ void __launch_bounds__(kScanThreads, 1)
+    threshold_mark_kernel(const T *__restrict__ q, const T *__restrict__ K,
+                          const float *__restrict__ tau, uint32_t *__restrict__ bits, int N,
+                          int kv_rows, int Hq, int Hkv, int tiles_per_head, long long total_tiles,
+                          float scale, uint32_t *status) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kScanStages * kScanStageBytes);
+  uint64_t *empty = full + kScanStages;
+  const long long t_begin = (long long)blockIdx.x * total_tiles / gridDim.x;
+  const long long t_end = (long long)(blockIdx.x + 1) * total_tiles / gridDim.x;
+  const int ntiles = (int)(t_end - t_begin);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kScanStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kScanConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  grid_dep_wait();
+  grid_dep_launch();
+  ScanOut o;
+  o.S = nullptr;
+  o.hist = nullptr;
+  o.shist = nullptr;
+  o.keys = nullptr;
+  o.key_off = 0;
+  o.bits = bits;
+  o.tau = tau;
+  scan_tiles<T, D, kHistSlots, true>(q, K, N, kv_rows, Hq, Hkv, tiles_per_head, t_begin, ntiles,
+                                     (int)(t_begin / tiles_per_head), scale, smem, full, empty, o,
+                                     status);
+}
+
+template <typename T, int D>
+cudaError_t launch_mark_t(const Shape &s, const void *q, const void *K, const float *tau,
+                          uint32_t *bits, uint32_t *status, cudaStream_t st) {
+  using C = ScoreCfg<T, D>;
+  DeviceInfo di;
+  cudaError_t e = device_info(&di);
+  if (e != cudaSuccess) return e;
+  constexpr int kSmem = kScanStages * kScanStageBytes + 2 * kScanStages * 8;
+  auto kern = threshold_mark_kernel<T, D>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e != cudaSuccess) return e;
+  const int tiles_per_head = (s.N + C::kStageKeys - 1) / C::kStageKeys;
+  const long long total = (long long)s.BH() * tiles_per_head;
+  const int grid = (int)(total < di.sm_count ? total : di.sm_count);
+  const float scale = (float)(1.0 / __builtin_sqrt((double)D));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kScanThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  cfg.attrs = attrs;
+  cfg.numAttrs = 0;
+  add_pdl_attr(cfg, attrs);
+  e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(q), static_cast<const T *>(K), tau,
+                         bits, s.N, s.Ncap, s.Hq, s.Hkv, tiles_per_head, total, scale, status);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 template <typename T, int D>
@@ -124,6 +195,17 @@ cudaError_t launch_score_t(const Shape &s, const void *q, const void *K,
 }
 
 }  // namespace
+
+cudaError_t launch_threshold_mark(const Shape &s, const void *q, const void *K,
+                                  const float *tau, uint32_t *bits, uint32_t *status,
+                                  cudaStream_t st) {
+  if (s.dtype == 1) {
+    if (s.d == 128) return launch_mark_t<__nv_bfloat16, 128>(s, q, K, tau, bits, status, st);
+    return launch_mark_t<__nv_bfloat16, 64>(s, q, K, tau, bits, status, st);
+  }
+  if (s.d == 128) return launch_mark_t<float, 128>(s, q, K, tau, bits, status, st);
+  return launch_mark_t<float, 64>(s, q, K, tau, bits, status, st);
+}
 
 cudaError_t launch_score(const Shape &s, const void *q, const void *K,
                          float *S, uint32_t *hist, uint32_t *status,
