@@ -565,7 +565,8 @@ def run_reference(args, rank, world):
             f"heads (G={G}, L={w.L}) over the first {n} of {w.N} keys with "
             f"{sel}; value scaled by {frac:.3g} step per sample")
     return {
-        "metric": LOUVER_METRIC if args.louver else METRIC, "value": round(value, 5),
+        "metric": (LOUVER_METRIC if args.louver else
+                   THRESHOLD_METRIC if threshold else METRIC), "value": round(value, 5),
         "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 / value, 3), "higher_is_better": True,
@@ -760,6 +761,173 @@ def run_native_louver(args, rank, world, local_rank):
     return line
 
 
+THRESHOLD_METRIC = ("128K-context threshold sparse decode steps/s (16 layers, tau = "
+                    "97th-percentile score per head, full scan)")
+
+
+def run_native_threshold(args, rank, world, local_rank):
+    """One step = one sparse_decode_step in threshold mode: the marking scan
+    over the whole K cache (bits 'score >= tau' per key), the ordered sets
+    written from the bitmaps, and the attention of all L layers over them."""
+    import token_sparse_attention_sm_b200 as sd
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    base = synth.WORKLOADS[args.workload]
+    w = base.with_(seeds=tuple(s + 1000 * rank for s in base.seeds))
+    x = synth.generate(w)
+    variants = synth.query_variants(w, x, QUERY_SETS, seed=2000 + 1000 * rank)
+    K = x["K"].to(dev)
+    V = x["V"].to(dev)
+    qs = [(qr.to(dev), ql.to(dev)) for qr, ql in variants]
+    stream = torch.cuda.Stream(device=dev)
+    ws = sd.Workspace(dev)
+    ws.get(sd.workspace_bytes(w.B, w.N, w.Hq, w.Hkv, w.d, w.torch_dtype, w.cap, w.L))
+    cap = w.cap
+    with torch.cuda.stream(stream):
+        taus = [percentile_tau_device(sd, qr, K, ws, *w.tau_pct) for qr, _ in qs]
+        outs = [dict(out=torch.empty_like(ql),
+                     idx=torch.empty((w.B, w.Hkv, cap), dtype=torch.int32, device=dev),
+                     count=torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev),
+                     lse=torch.empty((w.L, w.B, w.Hq), dtype=torch.float32, device=dev))
+                for _, ql in qs]
+
+        def step_fn(i):
+            o = outs[i]
+            return lambda: sd.decode_step(qs[i][0], qs[i][1], K, V, tau=taus[i], cap=cap, ws=ws,
+                                          check=False, out=o["out"], idx=o["idx"],
+                                          count=o["count"], lse=o["lse"])
+
+        def route_fn(i):
+            o = outs[i]
+            return lambda: sd.route_threshold(qs[i][0], K, taus[i], cap, ws=ws, check=False,
+                                              idx=o["idx"], count=o["count"])
+
+        def attn_fn(i):
+            o = outs[i]
+            return lambda: sd.attn_gather(qs[i][1], K, V, o["idx"], count=o["count"], ws=ws,
+                                          check=False, out=o["out"], lse=o["lse"])
+
+        counts = []
+        for i in range(len(qs)):
+            step_fn(i)()
+            counts.append(outs[i]["count"].cpu())
+        sd.read_device_status(ws)
+        graphs = capture([step_fn(i) for i in range(len(qs))], stream)
+        loop = capture_loop([step_fn(i) for i in range(len(qs))], stream)
+        with ClockSampler(local_rank) as cs:
+            ms = time_steps(loop, graphs, args.steps, args.warmup, stream, cs)
+        clocks = cs.result()
+        sd.read_device_status(ws)
+        n_k = max(args.steps // 4, 64)
+        wk = max(args.warmup, 3)
+        t_route = time_graphs(capture([route_fn(i) for i in range(len(qs))], stream), n_k, wk,
+                              stream) / n_k
+        t_attn = time_graphs(capture([attn_fn(i) for i in range(len(qs))], stream), n_k, wk,
+                             stream) / n_k
+        sd.read_device_status(ws)
+
+    ms_max = sdist.max_over_ranks(ms)
+    t_route_max = sdist.max_over_ranks(t_route)
+    ms_per_step = ms_max / args.steps
+    value = world * args.steps / (ms_max / 1e3)
+    e2e = run_e2e_threshold(sd, w, variants, K, V, taus, ws, stream, dev, args, world)
+    peak, peak_src = load_peaks()
+    scan_b = w.B * w.Hkv * w.N * w.d * w.esize
+    mean_count = float(np.mean([np.minimum(c.numpy(), cap).sum() for c in counts]))
+    gath_b = 2 * mean_count * w.d * w.esize
+    achieved = scan_b / (t_route_max * 1e-3) / 1e9
+    line = {
+        "metric": THRESHOLD_METRIC,
+        "value": round(value, 2),
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded Gaussian K/V/q, planted heavy hitters)",
+        "config": {
+            "workload": w.name, "B": w.B, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+            "L": w.L, "cap": cap, "tau": "nearest-rank 97th percentile score per head",
+            "parallelism": f"replicas x{world}", "query_sets": QUERY_SETS,
+            "l2": "inputs larger than L2 (K+V = %.0f MB per replica); the query rotates over "
+                  "%d sets" % (2 * scan_b / 1e6, QUERY_SETS),
+            "timing": "steps replayed as CUDA graphs of %d consecutive steps; CUDA events on "
+                      "the launch stream; max over ranks" % QUERY_SETS,
+            "mean_set_size_per_query": round(mean_count, 1),
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "threshold_mark_kernel + bitmap_compact_kernel (routing)",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": None,
+            "algorithmic_bytes_per_launch": scan_b,
+            "avg_launch_us": round(t_route_max * 1e3, 2),
+            "peak_source": peak_src,
+        },
+        "step_roofline": {
+            "unique_bytes_per_step": int(scan_b + gath_b),
+            "achieved_gbs": round((scan_b + gath_b) / (ms_per_step * 1e-3) / 1e9, 1),
+            "frac_of_measured_peak": round((scan_b + gath_b) / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+        },
+        "kernels_us": {"route_threshold": round(t_route * 1e3, 2),
+                       "attn_gather_all_layers": round(t_attn * 1e3, 2)},
+        "e2e": e2e,
+        "gpu_launches": (2 + (1 if w.dtype == "bf16" else 2)) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_threshold(w, x)
+    return line
+
+
+def run_e2e_threshold(sd, w, variants, K, V, taus, ws, stream, dev, args, world):
+    """The threshold step through the public API with host buffers (queries in
+    from pinned memory, outputs, set and counts back, per-step sync)."""
+    hq = [(qr.pin_memory(), ql.pin_memory()) for qr, ql in variants]
+    dq = [(torch.empty_like(qr, device=dev), torch.empty_like(ql, device=dev)) for qr, ql in variants]
+    out_h = torch.empty(tuple(variants[0][1].shape), dtype=variants[0][1].dtype).pin_memory()
+    idx_h = torch.empty((w.B, w.Hkv, w.cap), dtype=torch.int32).pin_memory()
+    cnt_h = torch.empty((w.B, w.Hkv), dtype=torch.int32).pin_memory()
+    out_d = torch.empty(tuple(variants[0][1].shape), dtype=variants[0][1].dtype, device=dev)
+    idx_d = torch.empty((w.B, w.Hkv, w.cap), dtype=torch.int32, device=dev)
+    cnt_d = torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev)
+    steps = min(args.steps, 2000)
+    h2d = hq[0][0].numel() * hq[0][0].element_size() + hq[0][1].numel() * hq[0][1].element_size()
+    d2h = out_h.numel() * out_h.element_size() + idx_h.numel() * 4 + cnt_h.numel() * 4
+
+    def one(i):
+        j = i % len(hq)
+        (hqr, hql), (dqr, dql) = hq[j], dq[j]
+        dqr.copy_(hqr, non_blocking=True)
+        dql.copy_(hql, non_blocking=True)
+        sd.decode_step(dqr, dql, K, V, tau=taus[j], cap=w.cap, ws=ws, check=False, out=out_d,
+                       idx=idx_d, count=cnt_d, return_lse=False)
+        out_h.copy_(out_d, non_blocking=True)
+        idx_h.copy_(idx_d, non_blocking=True)
+        cnt_h.copy_(cnt_d, non_blocking=True)
+        stream.synchronize()
+
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            one(i)
+        torch.cuda.synchronize()
+        sdist.barrier()
+        t0 = time.perf_counter()
+        for i in range(steps):
+            one(i)
+        t1 = time.perf_counter()
+        sdist.barrier()
+    sec = sdist.max_over_ranks(t1 - t0)
+    return {"value": round(world * steps / sec, 2), "unit": "steps/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "api": "token_sparse_attention_sm_b200.decode_step threshold mode (eager, "
+                   "per-step sync)"}
+
+
 def run_e2e_louver(sd, w, variants, K, V, ix, taus, ws, stream, dev, args, world):
     """The Louver step through the public Python API with host buffers:
     queries copied in from pinned host memory, the outputs, the set and its
@@ -857,6 +1025,8 @@ def main():
     try:
         if args.louver:
             line = run_native_louver(args, rank, world, local_rank)
+        elif synth.WORKLOADS[args.workload].mode == "threshold":
+            line = run_native_threshold(args, rank, world, local_rank)
         else:
             line = run_native(args, rank, world, local_rank)
         if rank == 0:
