@@ -209,6 +209,34 @@ def time_steps(g_loop, g_one, steps: int, warmup: int, stream, sampler=None) -> 
     return start.elapsed_time(end)
 
 
+def step_distribution(g_loop, n_steps: int, stream, replays: int = 200) -> dict:
+    """Median and p90 of the per-step time: `replays` replays of the
+    n_steps-step graph, each bracketed by its own CUDA events (after the
+    timed region; the per-step figure is a replay's time / n_steps)."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(replays)]
+    for a, b in evs:
+        a.record(stream)
+        g_loop.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    us = sorted(a.elapsed_time(b) * 1e3 / n_steps for a, b in evs)
+    return {"median_us": round(statistics.median(us), 2),
+            "p90_us": round(us[int(0.9 * (len(us) - 1))], 2), "replays": replays,
+            "note": "per-step time of each %d-step graph replay" % n_steps}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def capture_loop(fn_list, stream):
     """One graph running every fn of fn_list in order."""
     g = torch.cuda.CUDAGraph()
@@ -315,6 +343,7 @@ def run_native(args, rank, world, local_rank):
         with ClockSampler(local_rank) as cs:
             ms = time_steps(loop, graphs, args.steps, args.warmup, stream, cs)
         clocks = cs.result()
+        dist = step_distribution(loop, len(qs), stream)
         sd.read_device_status(ws)         # no device-side condition in the run
 
         # per-kernel durations, each kernel alone in a graph of back-to-back
@@ -444,6 +473,7 @@ def run_native(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": kernels_per_step(w, args.reroute) * args.steps,
         "clocks": clocks,
+        "step_time": dist,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_full(w, x)
@@ -510,7 +540,7 @@ def cpu_baseline_full(w, x, budget_s: float = 10.0):
             break
     sec = time.perf_counter() - t0
     return {"value": round(n / sec, 4), "unit": "steps/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
+            "kind": "oracle", "cpu": cpu_model(),
             "sample": f"{n} full decode steps of {w.name} (all {w.B * w.Hkv} KV heads, "
                       f"{w.L} layers) by the plain C oracle with OpenMP, {sec:.1f} s"}
 
@@ -576,7 +606,7 @@ def run_reference(args, rank, world):
                    "d": w.d, "k": w.k, "L": w.L, "parallelism": "host cores"},
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 5), "unit": "steps/s", "cores": oracle.num_threads(),
-                         "kind": "oracle", "sample": desc},
+                         "kind": "oracle", "cpu": cpu_model(), "sample": desc},
         "e2e": {"value": round(value, 5), "unit": "steps/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -676,6 +706,7 @@ def run_native_louver(args, rank, world, local_rank):
         with ClockSampler(local_rank) as cs:
             ms = time_steps(loop, graphs, args.steps, args.warmup, stream, cs)
         clocks = cs.result()
+        dist = step_distribution(loop, len(qs), stream)
         sd.read_device_status(ws)
         sd.read_device_status(ix.ws)
         n_k = max(args.steps // 4, 64)
@@ -755,6 +786,7 @@ def run_native_louver(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": (1 + (1 if w.dtype == "bf16" else 2)) * args.steps,
         "clocks": clocks,
+        "step_time": dist,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_threshold(w, x)
@@ -818,6 +850,7 @@ def run_native_threshold(args, rank, world, local_rank):
         with ClockSampler(local_rank) as cs:
             ms = time_steps(loop, graphs, args.steps, args.warmup, stream, cs)
         clocks = cs.result()
+        dist = step_distribution(loop, len(qs), stream)
         sd.read_device_status(ws)
         n_k = max(args.steps // 4, 64)
         wk = max(args.warmup, 3)
@@ -878,6 +911,7 @@ def run_native_threshold(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": (2 + (1 if w.dtype == "bf16" else 2)) * args.steps,
         "clocks": clocks,
+        "step_time": dist,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_threshold(w, x)
@@ -988,7 +1022,7 @@ def cpu_baseline_threshold(w, x, budget_s: float = 10.0):
             break
     sec = time.perf_counter() - t0
     return {"value": round(n / sec, 4), "unit": "steps/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
+            "kind": "oracle", "cpu": cpu_model(),
             "sample": f"{n} full threshold decode steps of {w.name} (all {w.B * w.Hkv} KV "
                       f"heads, {w.L} layers, full scan) by the plain C oracle, {sec:.1f} s"}
 
