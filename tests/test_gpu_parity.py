@@ -603,23 +603,22 @@ def test_kv_append_then_decode(dev, dtype, d):
 
 @pytest.mark.parametrize("mode", ["topk", "threshold"])
 def test_decode_step_graph_equals_eager_step(dev, mode):
-    """The captured step with its host copies returns, for each new query
-    written into its pinned host buffers, exactly what the eager step
+    """The captured step with its packed host transfers returns, for each new
+    query written into its pinned input views, exactly what the eager step
     returns."""
     w = synth.custom(B=2, N=5000, Hq=8, Hkv=2, d=128, L=3, k=100, dtype="bf16", seed=17,
                      heavy=8, mode=mode, cap=5000)
     x = synth.generate(w)
     K, V = x["K"].to(dev), x["V"].to(dev)
     variants = synth.query_variants(w, x, 3, seed=90)
-    qrh = variants[0][0].clone().pin_memory()
-    qlh = variants[0][1].clone().pin_memory()
     kw = dict(k=w.k) if mode == "topk" else dict(
         tau=torch.from_numpy(oracle.percentile_tau(oracle.scores(_f(x["q_route"]), _f(x["K"])),
                                                    90, 100)).to(dev), cap=w.cap)
-    g = sd.DecodeStepGraph(qrh, qlh, K, V, ws=sd.Workspace(dev), **kw)
+    g = sd.DecodeStepGraph(K, V, w.L, w.Hq, ws=sd.Workspace(dev), **kw)
+    assert g.h2d_bytes >= (w.B * w.Hq * w.d + w.L * w.B * w.Hq * w.d) * 2
     for qr, ql in variants:
-        qrh.copy_(qr)
-        qlh.copy_(ql)
+        g.q_route_host.copy_(qr)
+        g.q_layers_host.copy_(ql)
         res = g()
         ref = sd.decode_step(qr.to(dev), ql.to(dev), K, V, **kw)
         assert torch.equal(res[0], ref["out"].cpu())

@@ -20,6 +20,7 @@ import ctypes
 import os
 import threading
 
+import numpy as np
 import torch
 
 __all__ = ["SparseDecodeError", "lib_path", "load", "score", "select_topk",
@@ -595,58 +596,78 @@ def louver_route_threshold(q, K, index: LouverIndex, tau, cap: int, check: bool 
 class DecodeStepGraph:
     """A decode step with its host transfers, captured once as a CUDA graph.
 
-    Each replay copies q_route and q_layers from the given pinned host
-    tensors to the device, runs one fused decode step (top-k with ``k``, or
-    threshold with a device ``tau`` and ``cap``) over the cache K, V, and
-    copies out and idx (and count in threshold mode) back into pinned host
-    tensors -- one graph launch instead of a Python call and four copy
-    launches per step.  The host tensors are bound at capture time: write
-    the next step's queries into them (or keep one graph per buffer set) and
-    call ``replay()``; ``synchronize()`` waits for the results.  The graph
-    runs on ``stream`` (a new one by default); graphs that share a workspace
-    must run on one stream.  The device status is checked once after the
-    warm-up step (use ``read_device_status(self.ws)`` to check later ones)."""
+    The object owns one pinned host buffer for the step's inputs and one for
+    its results, with tensor views: ``q_route_host`` [B,Hq,d] and
+    ``q_layers_host`` [L,B,Hq,d] (the cache dtype) to write the next step's
+    queries into, ``out_host`` [L,B,Hq,d], ``idx_host`` [B,Hkv,k or cap] and,
+    in threshold mode, ``count_host`` [B,Hkv] to read.  Each replay copies
+    the inputs to the device in one transfer, runs one fused decode step (top-k
+    with ``k``, or threshold with a device ``tau`` [B,Hkv] and ``cap``) over
+    the cache K, V, and copies the results back in one transfer: one graph
+    launch and two copies per step instead of a Python call and four copy
+    launches.  ``replay()`` enqueues a step on ``stream`` (a new stream by
+    default; graphs that share a workspace must use one stream),
+    ``synchronize()`` waits for it, calling the object does both.  The device
+    status is checked once after the warm-up step (use
+    ``read_device_status(self.ws)`` to check later ones)."""
 
-    def __init__(self, q_route_host, q_layers_host, K, V, k: int | None = None, tau=None,
-                 cap: int | None = None, ws: Workspace | None = None, out_host=None,
-                 idx_host=None, count_host=None, n: int | None = None, stream=None):
-        for t in (q_route_host, q_layers_host):
-            if t.is_cuda or not t.is_pinned():
-                raise ValueError("host queries must be pinned CPU tensors")
+    @staticmethod
+    def _layout(parts):
+        """Byte offsets of tensors packed at 256-byte boundaries."""
+        offs, n = [], 0
+        for shape, dtype in parts:
+            offs.append(n)
+            size = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+            n += (size + 255) // 256 * 256
+        return offs, n
+
+    def __init__(self, K, V, L: int, Hq: int, k: int | None = None, tau=None,
+                 cap: int | None = None, ws: Workspace | None = None, n: int | None = None,
+                 stream=None):
         _need_cuda(K, V, tau)
         dev = K.device
-        self.ws = _ws(ws, dev)
-        self.stream = stream if stream is not None else torch.cuda.Stream(device=dev)
-        self.q_route_host, self.q_layers_host = q_route_host, q_layers_host
-        self.q_route = torch.empty(q_route_host.shape, dtype=q_route_host.dtype, device=dev)
-        self.q_layers = torch.empty(q_layers_host.shape, dtype=q_layers_host.dtype, device=dev)
-        L, B, Hq, d = q_layers_host.shape
-        Hkv = K.shape[1]
+        B, Hkv, _, d = K.shape
+        dt = K.dtype
         topk = k is not None
         stride = int(k) if topk else int(cap)
-        self.out = torch.empty_like(self.q_layers)
-        self.idx = torch.empty((B, Hkv, stride), dtype=torch.int32, device=dev)
-        self.count = None if topk else torch.empty((B, Hkv), dtype=torch.int32, device=dev)
-        self.out_host = out_host if out_host is not None else torch.empty(
-            self.out.shape, dtype=self.out.dtype).pin_memory()
-        self.idx_host = idx_host if idx_host is not None else torch.empty(
-            self.idx.shape, dtype=torch.int32).pin_memory()
-        self.count_host = None
+        self.ws = _ws(ws, dev)
+        self.stream = stream if stream is not None else torch.cuda.Stream(device=dev)
+        ins = [((B, Hq, d), dt), ((L, B, Hq, d), dt)]
+        outs = [((L, B, Hq, d), dt), ((B, Hkv, stride), torch.int32)]
         if not topk:
-            self.count_host = count_host if count_host is not None else torch.empty(
-                (B, Hkv), dtype=torch.int32).pin_memory()
-        args = dict(k=k, tau=tau, cap=cap, ws=self.ws, check=False, out=self.out, idx=self.idx,
-                    count=self.count, return_lse=False, n=n)
+            outs.append(((B, Hkv), torch.int32))
+        in_offs, in_n = self._layout(ins)
+        out_offs, out_n = self._layout(outs)
+        self.host_in = torch.empty(in_n, dtype=torch.uint8).pin_memory()
+        self.host_out = torch.empty(out_n, dtype=torch.uint8).pin_memory()
+        self.dev_in = torch.empty(in_n, dtype=torch.uint8, device=dev)
+        self.dev_out = torch.empty(out_n, dtype=torch.uint8, device=dev)
+
+        def views(buf, offs, parts):
+            res = []
+            for o, (shape, dtype) in zip(offs, parts):
+                size = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+                res.append(buf[o:o + size].view(dtype).view(shape))
+            return res
+
+        self.q_route_host, self.q_layers_host = views(self.host_in, in_offs, ins)
+        q_route, q_layers = views(self.dev_in, in_offs, ins)
+        hv = views(self.host_out, out_offs, outs)
+        dv = views(self.dev_out, out_offs, outs)
+        self.out_host, self.idx_host = hv[0], hv[1]
+        self.count_host = None if topk else hv[2]
+        out, idx = dv[0], dv[1]
+        count = None if topk else dv[2]
+        args = dict(k=k, tau=tau, cap=cap, ws=self.ws, check=False, out=out, idx=idx,
+                    count=count, return_lse=False, n=n)
 
         def body():
-            self.q_route.copy_(self.q_route_host, non_blocking=True)
-            self.q_layers.copy_(self.q_layers_host, non_blocking=True)
-            decode_step(self.q_route, self.q_layers, K, V, **args)
-            self.out_host.copy_(self.out, non_blocking=True)
-            self.idx_host.copy_(self.idx, non_blocking=True)
-            if self.count is not None:
-                self.count_host.copy_(self.count, non_blocking=True)
+            self.dev_in.copy_(self.host_in, non_blocking=True)
+            decode_step(q_route, q_layers, K, V, **args)
+            self.host_out.copy_(self.dev_out, non_blocking=True)
 
+        self.q_route_host.zero_()
+        self.q_layers_host.zero_()
         with torch.cuda.stream(self.stream):
             body()                       # warm-up: sizes the workspace, loads the library
             self.stream.synchronize()
@@ -655,10 +676,22 @@ class DecodeStepGraph:
             with torch.cuda.graph(self.graph, stream=self.stream):
                 body()
 
+    @property
+    def h2d_bytes(self) -> int:
+        return self.host_in.numel()
+
+    @property
+    def d2h_bytes(self) -> int:
+        return self.host_out.numel()
+
     def replay(self):
-        """Enqueue one step (inputs from, results to, the bound host tensors)."""
-        with torch.cuda.stream(self.stream):
+        """Enqueue one step (inputs from, results to, the pinned host buffers).
+        Cheapest when called with the graph's stream current."""
+        if torch.cuda.current_stream(self.stream.device).cuda_stream == self.stream.cuda_stream:
             self.graph.replay()
+        else:
+            with torch.cuda.stream(self.stream):
+                self.graph.replay()
 
     def synchronize(self):
         self.stream.synchronize()
