@@ -764,3 +764,69 @@ def test_route_threshold_equals_select_on_its_scores(dev, B, N, Hkv, d, dtype, p
                 never = set(np.nonzero(S64[b, h] < tau[b, h] - band)[0].tolist())
                 assert must <= g and not (g & never)
 
+
+
+def _random_case(seed):
+    r = np.random.default_rng(10_000 + seed)
+    d = int(r.choice([64, 128]))
+    dtype = str(r.choice(["bf16", "f32"]))
+    G = int(r.choice([1, 2, 4, 8, 16]))
+    Hkv = int(r.choice([1, 2, 3, 4, 8]))
+    B = int(r.integers(1, 4))
+    N = int(r.choice([1, 2, 31, 33, 127, 500, 1000, 4097, 12345, 30001]))
+    L = int(r.integers(1, 6))
+    mode = str(r.choice(["topk", "threshold"]))
+    k = int(r.integers(1, N + 1))
+    cap = int(r.integers(1, N + 1))
+    return dict(B=B, N=N, Hq=G * Hkv, Hkv=Hkv, d=d, L=L, k=k, dtype=dtype, mode=mode, cap=cap,
+                heavy=int(min(N, r.integers(0, 5))), seed=seed)
+
+
+@pytest.mark.parametrize("seed", range(64))
+def test_random_shapes_fused_step(dev, seed):
+    """Seeded random shapes (ragged N from 1, any k or cap, G 1..16, d 64/128,
+    fp32/bf16, top-k and threshold with capacity overflow) through the fused
+    step: the set within the band of the oracle's, the shared-routing
+    property, and attention on the oracle's set within tolerance."""
+    c = _random_case(seed)
+    w = synth.custom(B=c["B"], N=c["N"], Hq=c["Hq"], Hkv=c["Hkv"], d=c["d"], L=c["L"],
+                     k=c["k"], dtype=c["dtype"], heavy=c["heavy"], seed=c["seed"],
+                     mode=c["mode"], cap=c["cap"])
+    x = synth.generate(w)
+    t = _to(dev, x)
+    q32, K32, V32 = _f(x["q_route"]), _f(x["K"]), _f(x["V"])
+    S = oracle.scores(q32, K32)
+    ws = sd.Workspace(dev)
+    if c["mode"] == "topk":
+        res = sd.decode_step(t["q_route"], t["q_layers"], t["K"], t["V"], k=c["k"], ws=ws)
+        gidx = res["idx"].cpu().numpy()
+        assert_topk_within_band(gidx, S, c["k"])
+        np.testing.assert_array_equal(gidx, sd.route_topk(t["q_route"], t["K"], c["k"],
+                                                          ws=ws).cpu().numpy())
+        ridx, rcnt = oracle.topk(S, c["k"]), None
+    else:
+        tau = oracle.percentile_tau(S, 90, 100)
+        res = sd.decode_step(t["q_route"], t["q_layers"], t["K"], t["V"],
+                             tau=torch.from_numpy(tau).to(dev), cap=c["cap"], ws=ws, check=False)
+        st = sd.read_device_status(ws, raise_on_error=False)
+        ridx, rcnt = oracle.threshold(S, tau, c["cap"])
+        gcnt = res["count"].cpu().numpy()
+        gidx = res["idx"].cpu().numpy()
+        S64 = oracle.scores(q32, K32, np.float64)
+        for b in range(c["B"]):
+            for h in range(c["Hkv"]):
+                band = _band(tau[b, h])
+                assert abs(int(gcnt[b, h]) - int(rcnt[b, h])) <= \
+                    int(np.sum(np.abs(S[b, h] - tau[b, h]) <= band))
+                if gcnt[b, h] <= c["cap"]:
+                    g = set(gidx[b, h, :gcnt[b, h]].tolist())
+                    must = set(np.nonzero(S64[b, h] >= tau[b, h] + band)[0].tolist())
+                    never = set(np.nonzero(S64[b, h] < tau[b, h] - band)[0].tolist())
+                    assert must <= g and not (g & never)
+        assert (st == 4) == bool((gcnt > c["cap"]).any())
+        rcnt = np.minimum(rcnt, c["cap"]).astype(np.int32)
+    o_gpu, l_gpu = sd.attn_gather(t["q_layers"], t["K"], t["V"], torch.from_numpy(ridx).to(dev),
+                                  count=None if rcnt is None else torch.from_numpy(rcnt).to(dev),
+                                  ws=ws)
+    o_ref, l_ref = oracle.attn(_f(x["q_layers"]), K32, V32, ridx, rcnt)
+    assert_attn_close(o_gpu, l_gpu, o_ref, l_ref, c["dtype"])
