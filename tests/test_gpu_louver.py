@@ -284,3 +284,39 @@ def test_louver_decode_step_equals_route_then_gather(dev, dtype, d):
     tol = 2e-2 if dtype == "bf16" else 1e-4
     assert np.abs(o_gpu.float().cpu().numpy() - o_ref).max() <= tol
 
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_louver_random_shapes(dev, seed):
+    """Seeded random shapes (r 32..256, N = r * 2^j up to 32K, B, Hkv, G,
+    d 64/128, fp32/bf16, clustered or Gaussian keys, tau from the median to
+    beyond the maximum, cap below and above the set size): the set equals the
+    full-scan threshold routing bitwise, with the same status."""
+    rng = np.random.default_rng(20_000 + seed)
+    r = int(rng.choice([32, 64, 128, 256]))
+    N = r * int(2 ** rng.integers(0, 8))
+    N = min(N, 32768)
+    Hkv = int(rng.choice([1, 2, 4, 8]))
+    G = int(rng.choice([1, 2, 4]))
+    B = int(rng.integers(1, 3))
+    d = int(rng.choice([64, 128]))
+    dtype = str(rng.choice(["bf16", "f32"]))
+    blobs = int(rng.choice([0, 4, 16]))
+    pct = int(rng.choice([50, 90, 99, 100]))
+    cap = int(rng.integers(1, N + 1))
+    w = synth.custom(B=B, N=N, Hq=G * Hkv, Hkv=Hkv, d=d, L=1, dtype=dtype, seed=seed,
+                     mode="threshold", cap=cap, blobs=blobs)
+    x = synth.generate(w)
+    qd, Kd = x["q_route"].to(dev), x["K"].to(dev)
+    tau = oracle.percentile_tau(oracle.scores(_f(x["q_route"]), _f(x["K"])), pct, 100)
+    if pct == 100:
+        tau = tau + 1.0  # beyond every score: empty sets
+    taud = torch.from_numpy(tau.astype(np.float32)).to(dev)
+    ix = sd.louver_build(Kd, r)
+    a = sd.louver_route_threshold(qd, Kd, ix, taud, cap, check=False)
+    sa = sd.read_device_status(ix.ws, raise_on_error=False)
+    ws = sd.Workspace(dev)
+    f = sd.route_threshold(qd, Kd, taud, cap, ws=ws, check=False)
+    sf = sd.read_device_status(ws, raise_on_error=False)
+    _assert_same_set(a, f, cap)
+    assert sa == sf
