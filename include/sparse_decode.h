@@ -161,7 +161,11 @@ sparse_status_t sparse_route_topk(const sparse_shape_t *shape, const void *q,
                                   void *ws, size_t ws_bytes, void *stream);
 
 /* Shared routing, threshold form (Louver summary, sections 問題定義 and
- * 1. 半空間範囲検索への帰着): as sparse_select_threshold on the scores of q. */
+ * 1. 半空間範囲検索への帰着): the set sparse_select_threshold returns on the
+ * scores of q (the same fp32 scores, the same comparison), computed without
+ * storing them: the scan marks the keys >= tau[b,h] in per-head bitmaps in
+ * the workspace and one cluster per head writes the ascending idx rows and
+ * count (SPARSE_ERR_CAPACITY through the status word when count > cap). */
 sparse_status_t sparse_route_threshold(const sparse_shape_t *shape,
                                        const void *q, const void *K,
                                        const float *tau, int32_t cap,
