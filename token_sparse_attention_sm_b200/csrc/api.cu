@@ -15,7 +15,8 @@
 //                         select; cleared after use).  At least 256 rows, so
 //                         that calls of different shapes (up to 256 heads)
 //                         sharing one workspace never put other data there.
-//   [.., ..)              fp32 scores S [B,Hkv,N]
+//   [.., ..)              fp32 scores S [B,Hkv,N]; threshold routing keeps
+//                         its per-head bitmaps [B*Hkv][ceil(N/32)] here
 //   [.., ..)              fused routing: published boundary-bin keys
 //   [.., ..)              attention split partials
 #include <stdlib.h>
