@@ -915,90 +915,47 @@ def run_native_threshold(args, rank, world, local_rank):
 
 def run_e2e_threshold(sd, w, variants, K, V, taus, ws, stream, dev, args, world):
     """The threshold step through the public API with host buffers (queries in
-    from pinned memory, outputs, set and counts back, per-step sync)."""
-    hq = [(qr.pin_memory(), ql.pin_memory()) for qr, ql in variants]
-    dq = [(torch.empty_like(qr, device=dev), torch.empty_like(ql, device=dev)) for qr, ql in variants]
-    out_h = torch.empty(tuple(variants[0][1].shape), dtype=variants[0][1].dtype).pin_memory()
-    idx_h = torch.empty((w.B, w.Hkv, w.cap), dtype=torch.int32).pin_memory()
-    cnt_h = torch.empty((w.B, w.Hkv), dtype=torch.int32).pin_memory()
-    out_d = torch.empty(tuple(variants[0][1].shape), dtype=variants[0][1].dtype, device=dev)
-    idx_d = torch.empty((w.B, w.Hkv, w.cap), dtype=torch.int32, device=dev)
-    cnt_d = torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev)
-    steps = min(args.steps, 2000)
-    h2d = hq[0][0].numel() * hq[0][0].element_size() + hq[0][1].numel() * hq[0][1].element_size()
-    d2h = out_h.numel() * out_h.element_size() + idx_h.numel() * 4 + cnt_h.numel() * 4
-
-    def one(i):
-        j = i % len(hq)
-        (hqr, hql), (dqr, dql) = hq[j], dq[j]
-        dqr.copy_(hqr, non_blocking=True)
-        dql.copy_(hql, non_blocking=True)
-        sd.decode_step(dqr, dql, K, V, tau=taus[j], cap=w.cap, ws=ws, check=False, out=out_d,
-                       idx=idx_d, count=cnt_d, return_lse=False)
-        out_h.copy_(out_d, non_blocking=True)
-        idx_h.copy_(idx_d, non_blocking=True)
-        cnt_h.copy_(cnt_d, non_blocking=True)
-        stream.synchronize()
-
-    with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 3)):
-            one(i)
-        torch.cuda.synchronize()
-        sdist.barrier()
-        t0 = time.perf_counter()
-        for i in range(steps):
-            one(i)
-        t1 = time.perf_counter()
-        sdist.barrier()
-    sec = sdist.max_over_ranks(t1 - t0)
-    return {"value": round(world * steps / sec, 2), "unit": "steps/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "api": "token_sparse_attention_sm_b200.decode_step threshold mode (eager, "
-                   "per-step sync)"}
+    from pinned memory, outputs, set and counts back, per-step sync):
+    DecodeStepGraph, one per query set."""
+    return _e2e_graphs(sd, w, variants, K, V, taus, ws, stream, args, world, None,
+                       "decode_step threshold mode")
 
 
 def run_e2e_louver(sd, w, variants, K, V, ix, taus, ws, stream, dev, args, world):
-    """The Louver step through the public Python API with host buffers:
-    queries copied in from pinned host memory, the outputs, the set and its
-    counts read back, all inside the timed region (per-step sync)."""
-    hq = [(qr.pin_memory(), ql.pin_memory()) for qr, ql in variants]
-    dq = [(torch.empty_like(qr, device=dev), torch.empty_like(ql, device=dev)) for qr, ql in variants]
-    out_h = torch.empty(tuple(variants[0][1].shape), dtype=variants[0][1].dtype).pin_memory()
-    idx_h = torch.empty((w.B, w.Hkv, w.cap), dtype=torch.int32).pin_memory()
-    cnt_h = torch.empty((w.B, w.Hkv), dtype=torch.int32).pin_memory()
-    out_d = torch.empty(tuple(variants[0][1].shape), dtype=variants[0][1].dtype, device=dev)
-    idx_d = torch.empty((w.B, w.Hkv, w.cap), dtype=torch.int32, device=dev)
-    cnt_d = torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev)
+    """The Louver step through the public API with host buffers:
+    DecodeStepGraph over the index, one per query set."""
+    return _e2e_graphs(sd, w, variants, K, V, taus, ws, stream, args, world, ix,
+                       "louver_decode_step")
+
+
+def _e2e_graphs(sd, w, variants, K, V, taus, ws, stream, args, world, index, what):
+    graphs = []
+    for (qr, ql), tau in zip(variants, taus):
+        g = sd.DecodeStepGraph(K, V, w.L, w.Hq, tau=tau, cap=w.cap, ws=ws, stream=stream,
+                               index=index)
+        g.q_route_host.copy_(qr)
+        g.q_layers_host.copy_(ql)
+        graphs.append(g)
     steps = min(args.steps, 2000)
-    h2d = hq[0][0].numel() * hq[0][0].element_size() + hq[0][1].numel() * hq[0][1].element_size()
-    d2h = (out_h.numel() * out_h.element_size() + idx_h.numel() * 4 + cnt_h.numel() * 4)
-
-    def one(i):
-        j = i % len(hq)
-        (hqr, hql), (dqr, dql) = hq[j], dq[j]
-        dqr.copy_(hqr, non_blocking=True)
-        dql.copy_(hql, non_blocking=True)
-        sd.louver_decode_step(dqr, dql, K, V, ix, taus[j], w.cap, ws=ws, check=False,
-                              out=out_d, idx=idx_d, count=cnt_d, return_lse=False)
-        out_h.copy_(out_d, non_blocking=True)
-        idx_h.copy_(idx_d, non_blocking=True)
-        cnt_h.copy_(cnt_d, non_blocking=True)
-        stream.synchronize()
-
     with torch.cuda.stream(stream):
         for i in range(max(args.warmup, 3)):
-            one(i)
+            graphs[i % len(graphs)]()
         torch.cuda.synchronize()
         sdist.barrier()
         t0 = time.perf_counter()
         for i in range(steps):
-            one(i)
+            graphs[i % len(graphs)]()
         t1 = time.perf_counter()
         sdist.barrier()
+        sd.read_device_status(ws)
     sec = sdist.max_over_ranks(t1 - t0)
+    g0 = graphs[0]
     return {"value": round(world * steps / sec, 2), "unit": "steps/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "api": "token_sparse_attention_sm_b200.louver_decode_step (eager, per-step sync)"}
+            "h2d_bytes_per_step": g0.h2d_bytes, "d2h_bytes_per_step": g0.d2h_bytes,
+            "steps": steps,
+            "api": "token_sparse_attention_sm_b200.DecodeStepGraph (%s with one packed "
+                   "host-to-device and one device-to-host transfer, one CUDA graph; "
+                   "synchronised every step)" % what}
 
 
 def cpu_baseline_threshold(w, x, budget_s: float = 10.0):

@@ -320,3 +320,23 @@ def test_louver_random_shapes(dev, seed):
     sf = sd.read_device_status(ws, raise_on_error=False)
     _assert_same_set(a, f, cap)
     assert sa == sf
+
+
+def test_louver_step_graph_equals_eager(dev):
+    """DecodeStepGraph routing through a Louver index returns, for each query
+    written into its pinned views, what the eager louver_decode_step returns."""
+    w = synth.custom(B=1, N=8192, Hq=8, Hkv=2, d=128, L=3, dtype="bf16", seed=31,
+                     mode="threshold", cap=2048, blobs=16)
+    x = synth.generate(w)
+    K, V = x["K"].to(dev), x["V"].to(dev)
+    tau = oracle.percentile_tau(oracle.scores(_f(x["q_route"]), _f(x["K"])), 95, 100)
+    taud = torch.from_numpy(tau).to(dev)
+    ix = sd.louver_build(K, 128)
+    g = sd.DecodeStepGraph(K, V, w.L, w.Hq, tau=taud, cap=w.cap, ws=sd.Workspace(dev), index=ix)
+    for qr, ql in synth.query_variants(w, x, 3, seed=5):
+        g.q_route_host.copy_(qr)
+        g.q_layers_host.copy_(ql)
+        out_h, idx_h, cnt_h = g()
+        ref = sd.louver_decode_step(qr.to(dev), ql.to(dev), K, V, ix, taud, w.cap)
+        assert torch.equal(out_h, ref["out"].cpu())
+        _assert_same_set((idx_h, cnt_h), (ref["idx"].cpu(), ref["count"].cpu()), w.cap)

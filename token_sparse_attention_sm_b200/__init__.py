@@ -605,7 +605,8 @@ class DecodeStepGraph:
     with ``k``, or threshold with a device ``tau`` [B,Hkv] and ``cap``) over
     the cache K, V, and copies the results back in one transfer: one graph
     launch and two copies per step instead of a Python call and four copy
-    launches.  ``replay()`` enqueues a step on ``stream`` (a new stream by
+    launches.  With ``index`` (a LouverIndex of K) and threshold mode the
+    step routes through the index (louver_decode_step).  ``replay()`` enqueues a step on ``stream`` (a new stream by
     default; graphs that share a workspace must use one stream),
     ``synchronize()`` waits for it, calling the object does both.  The device
     status is checked once after the warm-up step (use
@@ -623,7 +624,7 @@ class DecodeStepGraph:
 
     def __init__(self, K, V, L: int, Hq: int, k: int | None = None, tau=None,
                  cap: int | None = None, ws: Workspace | None = None, n: int | None = None,
-                 stream=None):
+                 stream=None, index: "LouverIndex | None" = None):
         _need_cuda(K, V, tau)
         dev = K.device
         B, Hkv, _, d = K.shape
@@ -658,12 +659,24 @@ class DecodeStepGraph:
         self.count_host = None if topk else hv[2]
         out, idx = dv[0], dv[1]
         count = None if topk else dv[2]
-        args = dict(k=k, tau=tau, cap=cap, ws=self.ws, check=False, out=out, idx=idx,
-                    count=count, return_lse=False, n=n)
+        if index is not None:
+            if topk:
+                raise ValueError("routing through a Louver index needs tau and cap")
+
+            def run_step():
+                louver_decode_step(q_route, q_layers, K, V, index, tau, cap, ws=self.ws,
+                                   check=False, out=out, idx=idx, count=count,
+                                   return_lse=False)
+        else:
+            args = dict(k=k, tau=tau, cap=cap, ws=self.ws, check=False, out=out, idx=idx,
+                        count=count, return_lse=False, n=n)
+
+            def run_step():
+                decode_step(q_route, q_layers, K, V, **args)
 
         def body():
             self.dev_in.copy_(self.host_in, non_blocking=True)
-            decode_step(q_route, q_layers, K, V, **args)
+            run_step()
             self.host_out.copy_(self.dev_out, non_blocking=True)
 
         self.q_route_host.zero_()
