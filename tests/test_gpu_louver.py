@@ -340,3 +340,27 @@ def test_louver_step_graph_equals_eager(dev):
         ref = sd.louver_decode_step(qr.to(dev), ql.to(dev), K, V, ix, taud, w.cap)
         assert torch.equal(out_h, ref["out"].cpu())
         _assert_same_set((idx_h, cnt_h), (ref["idx"].cpu(), ref["count"].cpu()), w.cap)
+
+
+def test_louver_nonfinite_inputs_are_flagged(dev):
+    """A NaN key makes the index build report SPARSE_ERR_NONFINITE; a NaN tau
+    makes the query report it; neither faults, and a clean build and query on
+    the same workspace afterwards work."""
+    w = synth.custom(B=1, N=2048, Hq=4, Hkv=2, d=64, L=1, dtype="f32", seed=12,
+                     mode="threshold", cap=2048, blobs=4)
+    x = synth.generate(w)
+    K = x["K"].clone()
+    K[0, 1, 77, 5] = float("nan")
+    Kd = K.to(dev)
+    with pytest.raises(sd.SparseDecodeError) as ei:
+        sd.louver_build(Kd, 64)
+    assert ei.value.status == 5
+    Kc = x["K"].to(dev)
+    ix = sd.louver_build(Kc, 64)
+    qd = x["q_route"].to(dev)
+    tau = torch.tensor([[0.5, float("nan")]], device=dev)
+    sd.louver_route_threshold(qd, Kc, ix, tau, 2048, check=False)
+    assert sd.read_device_status(ix.ws, raise_on_error=False) == 5
+    tau = torch.tensor([[0.5, 0.5]], device=dev)
+    a = sd.louver_route_threshold(qd, Kc, ix, tau, 2048)
+    _assert_same_set(a, sd.route_threshold(qd, Kc, tau, 2048), 2048)
