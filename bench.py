@@ -657,7 +657,7 @@ def run_native_louver(args, rank, world, local_rank):
         outs = [dict(out=torch.empty_like(ql),
                      idx=torch.empty((w.B, w.Hkv, cap), dtype=torch.int32, device=dev),
                      count=torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev),
-                     surv=torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev),
+                     surv=torch.empty((w.B, w.Hkv, 2), dtype=torch.int32, device=dev),
                      lse=torch.empty((w.L, w.B, w.Hq), dtype=torch.float32, device=dev))
                 for _, ql in qs]
 
@@ -729,9 +729,13 @@ def run_native_louver(args, rank, world, local_rank):
     peak, peak_src = load_peaks()
     nc = w.N // r
     BH = w.B * w.Hkv
-    mean_surv = float(np.mean([s.sum().item() for s in surv]))
+    mean_surv = float(np.mean([s[..., 0].sum().item() for s in surv]))
+    mean_leaves = float(np.mean([s[..., 1].sum().item() for s in surv]))
     mean_count = float(np.mean([np.minimum(c.numpy(), cap).sum() for c in counts]))
-    route_b = (BH * nc * (w.d + 1) * 4 + mean_surv * r * (w.d * w.esize + 4) + mean_count * 4)
+    # cluster balls, the leaf balls of the surviving clusters, the surviving
+    # leaves' keys and key ids, the set written
+    route_b = (BH * nc * (w.d + 1) * 4 + mean_surv * (r // 32) * (w.d + 1) * 4
+               + mean_leaves * 32 * (w.d * w.esize + 4) + mean_count * 4)
     attn_b = 2 * mean_count * w.d * w.esize
     achieved = route_b / (t_route_max * 1e-3) / 1e9
     line = {
@@ -758,6 +762,7 @@ def run_native_louver(args, rank, world, local_rank):
                       "the launch stream; max over ranks" % QUERY_SETS,
             "index_build_ms": round(build_ms, 3),
             "surviving_clusters_per_query": round(mean_surv, 1),
+            "surviving_leaves_per_query": round(mean_leaves, 1),
             "clusters_per_query": BH * nc,
             "mean_set_size_per_query": round(mean_count, 1),
         },

@@ -252,7 +252,11 @@ sparse_status_t sparse_kv_append(const sparse_shape_t *shape, void *K, void *V,
  *        perm[bh][c*r .. c*r+r));
  *   centres [B*Hkv][N/r][d] fp32;  radii [B*Hkv][N/r] fp32;
  *   keys [B*Hkv][N][d] of the cache's dtype: row p of head bh is key
- *        perm[bh][p], so that each cluster's keys are contiguous.
+ *        perm[bh][p], so that each cluster's keys are contiguous;
+ *   leaf centres [B*Hkv][N/32][d] fp32;  leaf radii [B*Hkv][N/32] fp32: the
+ *        tree continues below the clusters to leaves of 32 keys (cluster c
+ *        is leaves c*r/32 .. (c+1)*r/32 - 1); a query tests the leaves of
+ *        the clusters that pass, with the same rule, before checking keys.
  * The index describes K's first N rows and holds a copy of them; it must be
  * rebuilt when those rows change.
  * Workspace: ws_bytes from sparse_louver_sizes, zero-filled once before first
@@ -284,8 +288,9 @@ sparse_status_t sparse_louver_build(const sparse_shape_t *shape, const void *K, 
  * exceeds cap, as there).  A cluster is skipped only when its ball bound
  * <qbar,c> + |qbar| rho is below tau - (1e-4 |tau| + 1e-6) - 1e-5 |qbar|
  * (|c| + rho), a margin above the fp32 rounding of any member's score, so
- * rounding cannot drop a key.  survivors (nullable) [B,Hkv] int32: clusters that
- * passed the ball test.  q [B,Hq,d] of the shape's dtype; the shape is the
+ * rounding cannot drop a key.  survivors (nullable) [B,Hkv,2] int32: the
+ * clusters that passed the ball test and, of their 32-key leaves, those
+ * that passed theirs (the keys checked exactly are 32 per such leaf).  q [B,Hq,d] of the shape's dtype; the shape is the
  * one the index was built for (Hq may differ; n_cap is not used).  One
  * kernel: its CTAs of a head meet at a bounded wait before writing the set
  * (see Co-residency); a wait that expires reports SPARSE_ERR_TIMEOUT and

@@ -57,6 +57,8 @@ def _check_index(ix, K32, r):
     keys = ix.keys().float().cpu().numpy()
     cen = ix.centres().cpu().numpy().astype(np.float64)
     rad = ix.radii().cpu().numpy().astype(np.float64)
+    lcen = ix.leaf_centres().cpu().numpy().astype(np.float64)
+    lrad = ix.leaf_radii().cpu().numpy().astype(np.float64)
     for b in range(B):
         for h in range(Hkv):
             p = perm[b, h]
@@ -67,6 +69,11 @@ def _check_index(ix, K32, r):
             np.testing.assert_allclose(cen[b, h], mean, rtol=1e-4, atol=1e-4)
             dist = np.sqrt(((members - cen[b, h][:, None, :]) ** 2).sum(-1)).max(axis=1)
             assert np.all(dist <= rad[b, h]), "a key lies outside its cluster's ball"
+            # the 32-key leaves below the clusters
+            leaves = K32[b, h][p].astype(np.float64).reshape(N // 32, 32, d)
+            np.testing.assert_allclose(lcen[b, h], leaves.mean(axis=1), rtol=1e-4, atol=1e-4)
+            ldist = np.sqrt(((leaves - lcen[b, h][:, None, :]) ** 2).sum(-1)).max(axis=1)
+            assert np.all(ldist <= lrad[b, h]), "a key lies outside its leaf's ball"
 
 
 def _check_set(gidx, gcnt, q32, K32, tau, cap):
@@ -123,16 +130,20 @@ def test_louver_index_and_set(dev, c):
     _assert_same_set((gidx, gcnt), sd.route_threshold(qd, Kd, taud, cap), cap)
     gidx, gcnt = gidx.cpu().numpy(), gcnt.cpu().numpy()
     _check_set(gidx, gcnt, q32, K32, tau, cap)
-    # every cluster holding a selected key passed the ball test
+    # every cluster, and every 32-key leaf, holding a selected key passed its
+    # ball test
     perm = ix.perm().cpu().numpy()
     surv = surv.cpu().numpy()
     nc = c["N"] // c["r"]
     for b in range(c["B"]):
         for h in range(c["Hkv"]):
-            cl = np.empty(c["N"], np.int64)
-            cl[perm[b, h]] = np.arange(c["N"]) // c["r"]
-            held = len(set(cl[gidx[b, h, :gcnt[b, h]]].tolist()))
-            assert held <= surv[b, h] <= nc
+            pos = np.empty(c["N"], np.int64)
+            pos[perm[b, h]] = np.arange(c["N"])
+            sel = gidx[b, h, :gcnt[b, h]]
+            held = len(set((pos[sel] // c["r"]).tolist()))
+            held_leaves = len(set((pos[sel] // 32).tolist()))
+            assert held <= surv[b, h, 0] <= nc
+            assert held_leaves <= surv[b, h, 1] <= surv[b, h, 0] * (c["r"] // 32)
 
 
 def test_louver_matches_oracle_louver(dev):
@@ -153,7 +164,7 @@ def test_louver_matches_oracle_louver(dev):
     np.testing.assert_array_equal(ocnt, rcnt)
     # both indexes prune most clusters on tightly clustered keys
     assert osurv.max() < 0.5 * (4096 // 64)
-    assert gsurv.cpu().numpy().max() < 0.5 * (4096 // 64)
+    assert gsurv.cpu().numpy()[..., 0].max() < 0.5 * (4096 // 64)
 
 
 def test_louver_prunes_clustered_128k(dev):
@@ -169,7 +180,9 @@ def test_louver_prunes_clustered_128k(dev):
     gidx, gcnt, surv = sd.louver_route_threshold(qd, Kd, ix, taud, w.cap, return_survivors=True)
     _assert_same_set((gidx, gcnt), sd.route_threshold(qd, Kd, taud, w.cap), w.cap)
     _check_set(gidx.cpu().numpy(), gcnt.cpu().numpy(), q32, K32, tau, w.cap)
-    assert surv.cpu().numpy().max() < 0.5 * (w.N // 128)
+    surv = surv.cpu().numpy()
+    assert surv[..., 0].max() < 0.5 * (w.N // 128)
+    assert np.all(surv[..., 1] < surv[..., 0] * 4)   # the leaf balls prune inside clusters
 
 
 def test_louver_cache_longer_than_length_and_rebuild(dev):

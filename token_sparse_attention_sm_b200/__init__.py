@@ -523,6 +523,27 @@ class LouverIndex:
         n = self.B * self.Hkv * nc * self.d
         return self.index[c0:c0 + 4 * n].view(torch.float32).view(self.B, self.Hkv, nc, self.d)
 
+    def _leaf_offsets(self):
+        al = lambda x: (x + 255) // 256 * 256
+        _, r0 = self._offsets()
+        k0 = r0 + al(self.B * self.Hkv * (self.N // self.r) * 4)
+        es = 4 if self.dtype == torch.float32 else 2
+        c0 = k0 + al(self.B * self.Hkv * self.N * self.d * es)
+        return c0, c0 + al(self.B * self.Hkv * (self.N // 32) * self.d * 4)
+
+    def leaf_centres(self):
+        """Centres of the 32-key leaves, [B,Hkv,N/32,d] fp32."""
+        c0, _ = self._leaf_offsets()
+        n = self.B * self.Hkv * (self.N // 32) * self.d
+        return self.index[c0:c0 + 4 * n].view(torch.float32).view(
+            self.B, self.Hkv, self.N // 32, self.d)
+
+    def leaf_radii(self):
+        """Radii of the 32-key leaves, [B,Hkv,N/32] fp32."""
+        _, r0 = self._leaf_offsets()
+        n = self.B * self.Hkv * (self.N // 32)
+        return self.index[r0:r0 + 4 * n].view(torch.float32).view(self.B, self.Hkv, self.N // 32)
+
     def keys(self):
         """Cluster-ordered key rows, [B,Hkv,N,d] (row p of head bh is key
         perm[bh][p])."""
@@ -563,8 +584,9 @@ def louver_route_threshold(q, K, index: LouverIndex, tau, cap: int, check: bool 
                            return_survivors: bool = False, idx=None, count=None,
                            survivors=None):
     """Threshold routing through a Louver index: (idx [B,Hkv,cap], count [B,Hkv])
-    -- the set route_threshold returns -- plus, if asked, survivors [B,Hkv]
-    (clusters that passed the ball test).  K only checks that the index was
+    -- the set route_threshold returns -- plus, if asked, survivors [B,Hkv,2]
+    (clusters that passed the ball test, and the 32-key leaves of those that
+    passed theirs: the keys checked exactly).  K only checks that the index was
     built for this cache: the index holds its own copy of the keys."""
     _need_cuda(q, K, tau)
     B, Ncap, Hq, Hkv, d = _dims_qk(q, K)
@@ -577,7 +599,7 @@ def louver_route_threshold(q, K, index: LouverIndex, tau, cap: int, check: bool 
         count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
     surv = survivors
     if return_survivors and surv is None:
-        surv = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+        surv = torch.empty((B, Hkv, 2), dtype=torch.int32, device=q.device)
     if idx.shape != (B, Hkv, cap) or count.shape != (B, Hkv):
         raise ValueError("idx must be [B,Hkv,cap] and count [B,Hkv]")
     tau = tau.float().contiguous()

@@ -21,9 +21,10 @@
 //  4. the n/2 largest projections by the library's exact radix select (ties
 //     to the lower position), then a stable partition: the other half first,
 //     the selected half second;
-// then the cluster-ordered copy of the keys, and at the leaves one warp per
-// cluster computes the centre (mean) and the radius (largest distance,
-// inflated by 1e-5 relative to cover fp32 rounding).  The fp32 atomic sums
+// down to leaves of 32 keys (a cluster of r keys is r/32 consecutive
+// leaves); then the cluster-ordered copy of the keys, and one warp per
+// cluster and per leaf computes the centre (mean) and the radius (largest
+// distance, inflated by 1e-5 relative to cover fp32 rounding).  The fp32 atomic sums
 // make the build's directions depend on summation order, so two builds can
 // differ; every build is a valid index and query results do not depend on
 // it.
@@ -52,6 +53,16 @@ template <typename T, int EPL>
 __device__ __forceinline__ void load_elems(const T *p, float (&x)[EPL]) {
 #pragma unroll
   for (int e = 0; e < EPL; ++e) x[e] = DT<T>::to_f(p[e]);
+}
+
+// A key id read from the permutation, checked: an id outside [0, N) (only a
+// corrupted permutation or workspace can produce one) raises INTERNAL and is
+// replaced by 0, so no load or store leaves the head's rows.
+__device__ __forceinline__ int checked_id(const int *perm, long long i, int N, uint32_t *status) {
+  const int j = perm[i];
+  if ((unsigned)j < (unsigned)N) return j;
+  raise_flag(status, FLAG_INTERNAL);
+  return 0;
 }
 
 // Exclusive prefix sum over a block of NT threads; *total = block sum.
@@ -86,13 +97,13 @@ __global__ void identity_perm_kernel(int *perm, int N, long long total) {
 template <typename T, int D>
 __global__ void __launch_bounds__(D)
     seg_sum_kernel(const T *__restrict__ K, const int *__restrict__ perm, int n, int N,
-                   int rows, float *__restrict__ sums) {
+                   int rows, float *__restrict__ sums, uint32_t *status) {
   const long long base = (long long)blockIdx.x * n;
   const int bh = (int)(base / N);
   const int p0 = blockIdx.y * kChunk, p1 = min(n, p0 + kChunk);
   float acc = 0.f;
   for (int p = p0; p < p1; ++p) {
-    const int j = perm[base + p];
+    const int j = checked_id(perm, base + p, N, status);
     acc += DT<T>::to_f(K[((size_t)bh * rows + j) * D + threadIdx.x]);
   }
   atomicAdd(&sums[(size_t)blockIdx.x * D + threadIdx.x], acc);
@@ -107,7 +118,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128)
     power_kernel(const T *__restrict__ K, const int *__restrict__ perm, int n, int N, int rows,
                  const float *__restrict__ sums, const float *__restrict__ v_in, int first,
-                 float *__restrict__ acc_out, float *__restrict__ proj) {
+                 float *__restrict__ acc_out, float *__restrict__ proj, uint32_t *status) {
   constexpr int EPL = D / 32;
   __shared__ float red[4][D];
   const int seg = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -130,7 +141,7 @@ __global__ void __launch_bounds__(128)
   for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
   const int p0 = blockIdx.y * kChunk, p1 = min(n, p0 + kChunk);
   for (int p = p0 + warp; p < p1; p += 4) {
-    const int j = perm[base + p];
+    const int j = checked_id(perm, base + p, N, status);
     float x[EPL];
     load_elems<T, EPL>(K + ((size_t)bh * rows + j) * D + lane * EPL, x);
     float y = 0.f;
@@ -198,14 +209,16 @@ __global__ void __launch_bounds__(kLvThreads)
 // perm[bh][p]; one thread per 16-byte piece.
 template <typename T, int D>
 __global__ void gather_keys_kernel(const T *__restrict__ K, const int *__restrict__ perm, int N,
-                                   int rows, long long total_rows, T *__restrict__ keys) {
+                                   int rows, long long total_rows, T *__restrict__ keys,
+                                   uint32_t *status) {
   constexpr int CPR = D * (int)sizeof(T) / 16;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= total_rows * CPR) return;
   const long long row = i / CPR;
   const int part = (int)(i % CPR);
   const long long bh = row / N;
-  const uint4 *src = reinterpret_cast<const uint4 *>(K + ((size_t)bh * rows + perm[row]) * D);
+  const int j = checked_id(perm, row, N, status);
+  const uint4 *src = reinterpret_cast<const uint4 *>(K + ((size_t)bh * rows + j) * D);
   reinterpret_cast<uint4 *>(keys + (size_t)row * D)[part] = src[part];
 }
 
@@ -214,7 +227,8 @@ __global__ void gather_keys_kernel(const T *__restrict__ K, const int *__restric
 template <typename T, int D>
 __global__ void __launch_bounds__(128)
     bounds_kernel(const T *__restrict__ K, const int *__restrict__ perm, int r, int N, int rows,
-                  long long nclusters, float *__restrict__ centres, float *__restrict__ radii) {
+                  long long nclusters, float *__restrict__ centres, float *__restrict__ radii,
+                  uint32_t *status) {
   constexpr int EPL = D / 32;
   const long long cl = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -226,7 +240,8 @@ __global__ void __launch_bounds__(128)
   for (int e = 0; e < EPL; ++e) c[e] = 0.f;
   for (int p = 0; p < r; ++p) {
     float x[EPL];
-    load_elems<T, EPL>(K + ((size_t)bh * rows + perm[base + p]) * D + lane * EPL, x);
+    load_elems<T, EPL>(K + ((size_t)bh * rows + checked_id(perm, base + p, N, status)) * D +
+                           lane * EPL, x);
 #pragma unroll
     for (int e = 0; e < EPL; ++e) c[e] += x[e];
   }
@@ -235,7 +250,8 @@ __global__ void __launch_bounds__(128)
   float dmax = 0.f;
   for (int p = 0; p < r; ++p) {
     float x[EPL];
-    load_elems<T, EPL>(K + ((size_t)bh * rows + perm[base + p]) * D + lane * EPL, x);
+    load_elems<T, EPL>(K + ((size_t)bh * rows + checked_id(perm, base + p, N, status)) * D +
+                           lane * EPL, x);
     float d2 = 0.f;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) d2 += (x[e] - c[e]) * (x[e] - c[e]);
@@ -252,7 +268,10 @@ __global__ void __launch_bounds__(128)
 //  1. ball test of the owned clusters, eight lanes per cluster (64 clusters
 //     per round with all their loads in flight; the first round's before
 //     q's); survivors listed in shared memory;
-//  2. exact check of the survivors' keys in items of 32 keys, each warp
+//  1b. the 32-key leaves of the surviving clusters (the tree continues below
+//     the clusters down to leaves of 32 keys, each with its own ball) get
+//     the same ball test, and only the leaves that pass are checked;
+//  2. exact check of the surviving leaves' keys (32 per item), each warp
 //     taking every kQWarps-th item through its own ring of nb shared-memory
 //     slots: an item's rows are contiguous in the index's cluster-ordered key
 //     copy, so one bulk copy (TMA, completion on the slot's mbarrier) brings
@@ -329,10 +348,11 @@ __device__ uint32_t compact_slice(const uint32_t *__restrict__ bm, int s0, int s
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kQThreads)
+__global__ void __launch_bounds__(kQThreads, 1)
     louver_query_kernel(const T *__restrict__ q, int Hq, int Hkv, int N, float scale,
                         const int *__restrict__ perm, const float *__restrict__ centres,
-                        const float *__restrict__ radii, const T *__restrict__ keys, int r,
+                        const float *__restrict__ radii, const float *__restrict__ sub_centres,
+                        const float *__restrict__ sub_radii, const T *__restrict__ keys, int r,
                         int nc, const float *__restrict__ tau, int nb, int cap,
                         uint32_t *__restrict__ bitmap, uint32_t *__restrict__ parity,
                         int *__restrict__ nsurv, uint32_t *__restrict__ done,
@@ -346,7 +366,7 @@ __global__ void __launch_bounds__(kQThreads)
   __shared__ __align__(16) float qb[D];
   __shared__ __align__(8) uint64_t bars[kQWarps][kQMaxSlots];
   __shared__ float qn_s;
-  __shared__ int nlist, ready;
+  __shared__ int nlist, nitem, ready;
   __shared__ uint32_t wbuf[kQWarps];
   const int bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int splits = gridDim.x;
@@ -434,21 +454,74 @@ __global__ void __launch_bounds__(kQThreads)
   }
   __syncthreads();
   const int ns = nlist;
-  if (tid == 0 && ns) atomicAdd(&nsurv[bh], ns);
+  if (tid == 0 && ns) atomicAdd(&nsurv[2 * bh], ns);
+
+  // ---- 1b. the 32-key leaves of the surviving clusters: their own balls,
+  // the same test; the leaves that pass are the exact check's items (with
+  // r = 32 the clusters are the leaves)
+  const int ipc = r / 32;  // leaves per cluster
+  int *items = list + mc;  // leaf ids within the head
+  if (ipc == 1) {
+    items = list;
+  } else {
+    if (tid == 0) nitem = 0;
+    __syncthreads();
+    const int ntest = ns * ipc;
+    float qv[EPG];
+#pragma unroll
+    for (int e = 0; e < EPG; ++e) qv[e] = qb[gl * EPG + e];
+    for (int m0 = 0; m0 < ntest; m0 += 2 * kQGroupsPerRound) {
+      float4 sv[2][EPG / 4];
+      float srho[2];
+      int leaf[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int m = m0 + u * kQGroupsPerRound + grp;
+        leaf[u] = m < ntest ? list[m / ipc] * ipc + m % ipc : -1;
+        const size_t g = (size_t)bh * nc * ipc + (leaf[u] < 0 ? 0 : leaf[u]);
+        const float4 *c = reinterpret_cast<const float4 *>(sub_centres + g * D + gl * EPG);
+#pragma unroll
+        for (int v = 0; v < EPG / 4; ++v)
+          sv[u][v] = leaf[u] < 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(c + v);
+        srho[u] = leaf[u] < 0 ? 0.f : __ldg(sub_radii + g);
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float dot = 0.f, cc = 0.f;
+#pragma unroll
+        for (int v = 0; v < EPG / 4; ++v) {
+          const float4 c4 = sv[u][v];
+          dot = fmaf(qv[4 * v + 0], c4.x, dot);
+          dot = fmaf(qv[4 * v + 1], c4.y, dot);
+          dot = fmaf(qv[4 * v + 2], c4.z, dot);
+          dot = fmaf(qv[4 * v + 3], c4.w, dot);
+          cc = fmaf(c4.x, c4.x, fmaf(c4.y, c4.y, fmaf(c4.z, c4.z, fmaf(c4.w, c4.w, cc))));
+        }
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) {
+          dot += __shfl_xor_sync(0xffffffffu, dot, o);
+          cc += __shfl_xor_sync(0xffffffffu, cc, o);
+        }
+        const float ub = dot + qn * srho[u];
+        const float slack = 1e-5f * qn * (sqrtf(cc) + srho[u]);
+        if (gl == 0 && leaf[u] >= 0 && (ub >= lim - slack || !(ub == ub)))
+          items[atomicAdd(&nitem, 1)] = leaf[u];
+      }
+    }
+    __syncthreads();
+  }
+  const int nitems = ipc == 1 ? ns : nitem;
+  if (tid == 0 && nitems) atomicAdd(&nsurv[2 * bh + 1], nitems);
 
   // ---- 2. exact check, 32 keys per item, a private ring of slots per warp
   float qs[C::kEpl];
 #pragma unroll
   for (int e = 0; e < C::kEpl; ++e) qs[e] = qb[(lane % C::kLpk) * C::kEpl + e];
   const uint32_t tkey = order_key(t);
-  const int ipc = r / 32;  // items per cluster
-  const int nitems = ns * ipc;
   unsigned char *wb = lv_smem + (size_t)warp * nb * kSlotBytes;
   const size_t head0 = (size_t)bh * nc * r;  // the head's first cluster-ordered row
   // cluster-ordered row of row 0 of item it
-  auto item_row = [&](int it) -> size_t {
-    return head0 + (size_t)list[it / ipc] * r + (it % ipc) * 32;
-  };
+  auto item_row = [&](int it) -> size_t { return head0 + (size_t)items[it] * 32; };
   // key id of row `lane` of item it (0 past the end)
   auto load_id = [&](int it) -> int { return it < nitems ? __ldg(perm + item_row(it) + lane) : 0; };
   // item it's rows into slot `slot` (its key ids j, one per lane)
@@ -487,7 +560,11 @@ __global__ void __launch_bounds__(kQThreads)
     const float score = warp_tile_scores<T, D>(sp, 0, qs, lane);
     const int row = (lane % C::kLpk) * C::kKpr + lane / C::kLpk;
     const int jk = reinterpret_cast<const int *>(sp + kItemBytes)[row];
-    if (order_key(score) >= tkey) atomicOr(&bm[jk >> 5], 1u << (jk & 31));
+    if ((unsigned)jk >= (unsigned)N) {  // only with a corrupted index (flagged)
+      raise_flag(status, FLAG_INTERNAL);
+    } else if (order_key(score) >= tkey) {
+      atomicOr(&bm[jk >> 5], 1u << (jk & 31));
+    }
     if (__any_sync(0xffffffffu, !isfinite(score)) && lane == 0)
       raise_flag(status, FLAG_NONFINITE);
     __syncwarp();  // the slot is read before it is refilled
@@ -525,9 +602,12 @@ __global__ void __launch_bounds__(kQThreads)
     }
     // the last CTA to leave resets the head's counters and flips its bitmaps
     if (atomicAdd(done + 2 * bh + 1, 1u) == (uint32_t)splits - 1) {
-      const int sv = __ldcg(nsurv + bh);
-      if (survivors_out) survivors_out[bh] = sv;
-      nsurv[bh] = 0;
+      if (survivors_out) {
+        survivors_out[2 * bh] = __ldcg(nsurv + 2 * bh);
+        survivors_out[2 * bh + 1] = __ldcg(nsurv + 2 * bh + 1);
+      }
+      nsurv[2 * bh] = 0;
+      nsurv[2 * bh + 1] = 0;
       parity[bh] = par ^ 1u;
       done[2 * bh] = 0u;
       done[2 * bh + 1] = 0u;
@@ -538,7 +618,7 @@ __global__ void __launch_bounds__(kQThreads)
 // ---- host side ----------------------------------------------------------------
 
 struct LvLayout {
-  size_t perm, centres, radii, keys, index_total;                      // index
+  size_t perm, centres, radii, keys, sub_centres, sub_radii, index_total;  // index
   size_t sums, va, vb, proj, perm2, sel, bitmap, parity, nsurv, done, ws_total;  // workspace
 };
 
@@ -558,8 +638,12 @@ LvLayout lv_layout(const Shape &s, int r) {
   l.centres = lv_align(BH * N * 4);
   l.radii = l.centres + lv_align(BH * nc * d * 4);
   l.keys = l.radii + lv_align(BH * nc * 4);
-  l.index_total = l.keys + lv_align(BH * N * d * (size_t)s.esize());
-  const size_t nseg = BH * N / r;  // bound on the segments of any level
+  l.sub_centres = l.keys + lv_align(BH * N * d * (size_t)s.esize());
+  l.sub_radii = l.sub_centres + lv_align(BH * (N / 32) * d * 4);
+  l.index_total = l.sub_radii + lv_align(BH * (N / 32) * 4);
+  // the deepest split level has nodes of 64 keys (leaves of 32): the most
+  // segments any level has
+  const size_t nseg = BH * N / 64;
   l.sums = kLvHeader;
   l.va = l.sums + lv_align(nseg * d * 4);
   l.vb = l.va + lv_align(nseg * d * 4);
@@ -569,7 +653,7 @@ LvLayout lv_layout(const Shape &s, int r) {
   l.bitmap = l.sel + lv_align(BH * N / 2 * 4 + 4);  // two per head (double-buffered)
   l.parity = l.bitmap + lv_align(2 * BH * N / 32 * 4);
   l.nsurv = l.parity + lv_align(BH * 4);
-  l.done = l.nsurv + lv_align(BH * 4);
+  l.done = l.nsurv + lv_align(2 * BH * 4);  // surviving clusters and leaves per head
   l.ws_total = l.done + lv_align(2 * BH * 4);
   return l;
 }
@@ -591,24 +675,25 @@ cudaError_t lv_build_t(const Shape &s, const void *Kv, int r, char *index, char 
   identity_perm_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(perm, s.N, total);
   cudaError_t e = cudaGetLastError();
   int *cur = perm, *nxt = perm2;
-  for (int n = s.N; n > r && e == cudaSuccess; n /= 2) {
+  for (int n = s.N; n > 32 && e == cudaSuccess; n /= 2) {  // down to 32-key leaves
     const int nseg = (int)(total / n);
     const dim3 grid((unsigned)nseg, (unsigned)((n + kChunk - 1) / kChunk));
     e = cudaMemsetAsync(sums, 0, (size_t)nseg * D * 4, st);
     if (e != cudaSuccess) break;
-    seg_sum_kernel<T, D><<<grid, D, 0, st>>>(K, cur, n, s.N, s.Ncap, sums);
+    seg_sum_kernel<T, D><<<grid, D, 0, st>>>(K, cur, n, s.N, s.Ncap, sums, status);
     float *vin = va, *vout = vb;
     for (int it = 0; it < kPowerIters && e == cudaSuccess; ++it) {
       e = cudaMemsetAsync(vout, 0, (size_t)nseg * D * 4, st);
       if (e != cudaSuccess) break;
       power_kernel<T, D><<<grid, 128, 0, st>>>(K, cur, n, s.N, s.Ncap, sums, vin, it == 0, vout,
-                                                nullptr);
+                                                nullptr, status);
       float *t = vin;
       vin = vout;
       vout = t;
     }
     if (e != cudaSuccess) break;
-    power_kernel<T, D><<<grid, 128, 0, st>>>(K, cur, n, s.N, s.Ncap, sums, vin, 0, nullptr, proj);
+    power_kernel<T, D><<<grid, 128, 0, st>>>(K, cur, n, s.N, s.Ncap, sums, vin, 0, nullptr, proj,
+                                             status);
     e = cudaGetLastError();
     if (e != cudaSuccess) break;
     // the n/2 largest projections of every segment (ties to the lower position)
@@ -633,13 +718,17 @@ cudaError_t lv_build_t(const Shape &s, const void *Kv, int r, char *index, char 
   if (e != cudaSuccess) return e;
   constexpr int CPR = D * (int)sizeof(T) / 16;
   gather_keys_kernel<T, D><<<(unsigned)((total * CPR + 255) / 256), 256, 0, st>>>(
-      K, perm, s.N, s.Ncap, total, reinterpret_cast<T *>(index + l.keys));
+      K, perm, s.N, s.Ncap, total, reinterpret_cast<T *>(index + l.keys), status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long ncl = total / r;
   bounds_kernel<T, D><<<(unsigned)((ncl + 3) / 4), 128, 0, st>>>(
       K, perm, r, s.N, s.Ncap, ncl, reinterpret_cast<float *>(index + l.centres),
-      reinterpret_cast<float *>(index + l.radii));
+      reinterpret_cast<float *>(index + l.radii), status);
+  const long long nleaf = total / 32;
+  bounds_kernel<T, D><<<(unsigned)((nleaf + 3) / 4), 128, 0, st>>>(
+      K, perm, 32, s.N, s.Ncap, nleaf, reinterpret_cast<float *>(index + l.sub_centres),
+      reinterpret_cast<float *>(index + l.sub_radii), status);
   return cudaGetLastError();
 }
 
@@ -660,7 +749,7 @@ cudaError_t lv_query_t(const Shape &s, const void *qv, int r, const char *index,
   splits = splits < 1 ? 1 : (splits > nc ? nc : splits);
   const int mc = (nc + splits - 1) / splits;
   const size_t slot = 32 * (size_t)C::kRowBytes + 32 * 4;
-  const size_t list_bytes = (size_t)mc * sizeof(int);
+  const size_t list_bytes = (size_t)mc * (1 + r / 32) * sizeof(int);  // clusters, leaves
   // as many slots per warp as fit next to the static shared memory, up to 4
   const size_t static_smem = 2048;
   int nb = (int)(((size_t)di.max_smem_optin - static_smem - list_bytes) / (kQWarps * slot));
@@ -685,6 +774,8 @@ cudaError_t lv_query_t(const Shape &s, const void *qv, int r, const char *index,
                          reinterpret_cast<const int *>(index + l.perm),
                          reinterpret_cast<const float *>(index + l.centres),
                          reinterpret_cast<const float *>(index + l.radii),
+                         reinterpret_cast<const float *>(index + l.sub_centres),
+                         reinterpret_cast<const float *>(index + l.sub_radii),
                          reinterpret_cast<const T *>(index + l.keys), r, nc, tau, nb, cap,
                          reinterpret_cast<uint32_t *>(ws + l.bitmap),
                          reinterpret_cast<uint32_t *>(ws + l.parity),
