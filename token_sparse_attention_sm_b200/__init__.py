@@ -500,66 +500,59 @@ class LouverIndex:
         _check(load().sparse_louver_sizes(ctypes.byref(sh), self.r, ctypes.byref(ib),
                                           ctypes.byref(wb)), "louver_sizes")
         self.index = torch.empty(int(ib.value), dtype=torch.uint8, device=K.device)
+        last = self._parts()["leaf_radii"]
+        if last[0] + last[3] > self.index.numel():
+            raise RuntimeError("index layout does not match the library's")
         self.ws = Workspace(K.device)
         self.ws_bytes = int(wb.value)
         self.ws.get(self.ws_bytes)
 
-    def perm(self):
-        """Key ids in cluster order, [B,Hkv,N] int32."""
-        n = self.B * self.Hkv * self.N
-        return self.index[:4 * n].view(torch.int32).view(self.B, self.Hkv, self.N)
+    def _parts(self):
+        """(offset, dtype, shape) of each part of the index buffer, in the
+        library's layout: each part at the next 256-byte boundary."""
+        BH, N, d, nc = self.B * self.Hkv, self.N, self.d, self.N // self.r
+        shapes = [("perm", torch.int32, (self.B, self.Hkv, N)),
+                  ("centres", torch.float32, (self.B, self.Hkv, nc, d)),
+                  ("radii", torch.float32, (self.B, self.Hkv, nc)),
+                  ("keys", self.dtype, (self.B, self.Hkv, N, d)),
+                  ("leaf_centres", torch.float32, (self.B, self.Hkv, N // 32, d)),
+                  ("leaf_radii", torch.float32, (self.B, self.Hkv, N // 32))]
+        parts, off = {}, 0
+        for name, dt, shape in shapes:
+            size = int(np.prod(shape)) * torch.tensor([], dtype=dt).element_size()
+            parts[name] = (off, dt, shape, size)
+            off += (size + 255) // 256 * 256
+        return parts
 
-    def _offsets(self):
-        al = lambda x: (x + 255) // 256 * 256
-        BH, nc = self.B * self.Hkv, self.N // self.r
-        c0 = al(BH * self.N * 4)
-        r0 = c0 + al(BH * nc * self.d * 4)
-        return c0, r0
+    def _view(self, name):
+        off, dt, shape, size = self._parts()[name]
+        return self.index[off:off + size].view(dt).view(shape)
+
+    def perm(self):
+        """Key ids in cluster order, [B,Hkv,N] int32 (cluster c of head bh is
+        perm[bh][c*r .. c*r+r), leaf l is perm[bh][32*l .. 32*l+32))."""
+        return self._view("perm")
 
     def centres(self):
         """Cluster centres, [B,Hkv,N/r,d] fp32."""
-        c0, _ = self._offsets()
-        nc = self.N // self.r
-        n = self.B * self.Hkv * nc * self.d
-        return self.index[c0:c0 + 4 * n].view(torch.float32).view(self.B, self.Hkv, nc, self.d)
+        return self._view("centres")
 
-    def _leaf_offsets(self):
-        al = lambda x: (x + 255) // 256 * 256
-        _, r0 = self._offsets()
-        k0 = r0 + al(self.B * self.Hkv * (self.N // self.r) * 4)
-        es = 4 if self.dtype == torch.float32 else 2
-        c0 = k0 + al(self.B * self.Hkv * self.N * self.d * es)
-        return c0, c0 + al(self.B * self.Hkv * (self.N // 32) * self.d * 4)
-
-    def leaf_centres(self):
-        """Centres of the 32-key leaves, [B,Hkv,N/32,d] fp32."""
-        c0, _ = self._leaf_offsets()
-        n = self.B * self.Hkv * (self.N // 32) * self.d
-        return self.index[c0:c0 + 4 * n].view(torch.float32).view(
-            self.B, self.Hkv, self.N // 32, self.d)
-
-    def leaf_radii(self):
-        """Radii of the 32-key leaves, [B,Hkv,N/32] fp32."""
-        _, r0 = self._leaf_offsets()
-        n = self.B * self.Hkv * (self.N // 32)
-        return self.index[r0:r0 + 4 * n].view(torch.float32).view(self.B, self.Hkv, self.N // 32)
+    def radii(self):
+        """Cluster radii, [B,Hkv,N/r] fp32."""
+        return self._view("radii")
 
     def keys(self):
         """Cluster-ordered key rows, [B,Hkv,N,d] (row p of head bh is key
         perm[bh][p])."""
-        _, r0 = self._offsets()
-        al = lambda x: (x + 255) // 256 * 256
-        k0 = r0 + al(self.B * self.Hkv * (self.N // self.r) * 4)
-        es = 4 if self.dtype == torch.float32 else 2
-        n = self.B * self.Hkv * self.N * self.d
-        return self.index[k0:k0 + es * n].view(self.dtype).view(self.B, self.Hkv, self.N, self.d)
+        return self._view("keys")
 
-    def radii(self):
-        """Cluster radii, [B,Hkv,N/r] fp32."""
-        _, r0 = self._offsets()
-        nc = self.N // self.r
-        n = self.B * self.Hkv * nc
-        return self.index[r0:r0 + 4 * n].view(torch.float32).view(self.B, self.Hkv, nc)
+    def leaf_centres(self):
+        """Centres of the 32-key leaves, [B,Hkv,N/32,d] fp32."""
+        return self._view("leaf_centres")
+
+    def leaf_radii(self):
+        """Radii of the 32-key leaves, [B,Hkv,N/32] fp32."""
+        return self._view("leaf_radii")
 
 
 def louver_build(K, r: int, n: int | None = None, check: bool = True) -> LouverIndex:
