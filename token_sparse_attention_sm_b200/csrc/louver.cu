@@ -222,6 +222,65 @@ __global__ void gather_keys_kernel(const T *__restrict__ K, const int *__restric
   reinterpret_cast<uint4 *>(keys + (size_t)row * D)[part] = src[part];
 }
 
+// Median split of a small node in one kernel (n a power of two, 64 <= n <=
+// kSmallSplit; one CTA per node): the node's projections are sorted by
+// (value descending, position ascending) in shared memory with a bitonic
+// network, the first n/2 positions of that order are the upper half (the
+// n/2 largest, ties to the lower position, exactly as the radix select takes
+// them), and a stable partition writes the other half, then the upper half,
+// each in position order -- what the select and partition kernels produce
+// for large nodes, without a cluster per node.
+constexpr int kSmallSplit = 2048;
+constexpr int kSmallThreads = 256;
+
+__global__ void __launch_bounds__(kSmallThreads)
+    split_small_kernel(const float *__restrict__ proj, const int *__restrict__ perm, int n,
+                       int *__restrict__ perm_out, uint32_t *status) {
+  __shared__ unsigned long long kv[kSmallSplit];
+  __shared__ unsigned char upper[kSmallSplit];
+  __shared__ uint32_t wbuf[kSmallThreads / 32];
+  const long long base = (long long)blockIdx.x * n;
+  const int tid = threadIdx.x;
+  bool bad = false;
+  for (int i = tid; i < n; i += kSmallThreads) {
+    const float f = proj[base + i];
+    bad |= !isfinite(f);
+    kv[i] = ((unsigned long long)(~order_key(f)) << 32) | (unsigned)i;
+  }
+  if (__syncthreads_or(bad) && tid == 0) raise_flag(status, FLAG_NONFINITE);
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < n; i += kSmallThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long a = kv[i], b = kv[ixj];
+          if ((a > b) == ((i & k) == 0)) {
+            kv[i] = b;
+            kv[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < n; i += kSmallThreads)
+    upper[(unsigned)(kv[i] & 0xffffffffull)] = i < n / 2 ? 1 : 0;
+  __syncthreads();
+  // thread tid owns positions [p0, p1)
+  const int per = (n + kSmallThreads - 1) / kSmallThreads;
+  const int p0 = min(n, tid * per), p1 = min(n, p0 + per);
+  uint32_t nlow = 0;
+  for (int p = p0; p < p1; ++p) nlow += upper[p] ? 0u : 1u;
+  uint32_t total;
+  uint32_t lo = lv_block_scan<kSmallThreads>(nlow, wbuf, &total);
+  uint32_t hi = (uint32_t)(n / 2) + ((uint32_t)p0 - lo);
+  for (int p = p0; p < p1; ++p) {
+    const int key = perm[base + p];
+    if (upper[p]) perm_out[base + hi++] = key;
+    else perm_out[base + lo++] = key;
+  }
+}
+
 // Centre (mean) and radius (largest distance from it, inflated) of each leaf
 // cluster of r keys; one warp per cluster.
 template <typename T, int D>
@@ -696,19 +755,25 @@ cudaError_t lv_build_t(const Shape &s, const void *Kv, int r, char *index, char 
                                              status);
     e = cudaGetLastError();
     if (e != cudaSuccess) break;
-    // the n/2 largest projections of every segment (ties to the lower position)
-    Shape ss{1, n, nseg, nseg, 64, 0, n};
-    e = launch_select(ss, proj, n / 2, nullptr, 0, sel, nullptr, n / 2, nullptr, status, st);
-    if (e != cudaSuccess) break;
-    const int psmem = (n / 32) * 4;
-    if (psmem > 48 * 1024) {
-      e = cudaFuncSetAttribute(partition_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               psmem);
+    if (n <= kSmallSplit) {
+      // small nodes: sort-based split, one CTA per node
+      split_small_kernel<<<(unsigned)nseg, kSmallThreads, 0, st>>>(proj, cur, n, nxt, status);
+      e = cudaGetLastError();
+    } else {
+      // the n/2 largest projections of every segment (ties to the lower position)
+      Shape ss{1, n, nseg, nseg, 64, 0, n};
+      e = launch_select(ss, proj, n / 2, nullptr, 0, sel, nullptr, n / 2, nullptr, status, st);
       if (e != cudaSuccess) break;
+      const int psmem = (n / 32) * 4;
+      if (psmem > 48 * 1024) {
+        e = cudaFuncSetAttribute(partition_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 psmem);
+        if (e != cudaSuccess) break;
+      }
+      partition_kernel<<<(unsigned)nseg, kLvThreads, (size_t)psmem, st>>>(cur, sel, n, nxt,
+                                                                         status);
+      e = cudaGetLastError();
     }
-    partition_kernel<<<(unsigned)nseg, kLvThreads, (size_t)psmem, st>>>(cur, sel, n, nxt,
-                                                                       status);
-    e = cudaGetLastError();
     int *t = cur;
     cur = nxt;
     nxt = t;
