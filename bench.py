@@ -512,9 +512,10 @@ def run_e2e(sd, w, variants, K, V, ws, stream, dev, args, world):
     return {"value": round(world * steps / sec, 2), "unit": "steps/s",
             "h2d_bytes_per_step": g0.h2d_bytes, "d2h_bytes_per_step": g0.d2h_bytes,
             "steps": steps,
-            "api": "token_sparse_attention_sm_b200.DecodeStepGraph (the decode step with one "
-                   "packed host-to-device and one device-to-host transfer, one CUDA graph; "
-                   "synchronised every step)"}
+            "api": "token_sparse_attention_sm_b200.DecodeStepGraph (routing and the layers' "
+                   "attention in one CUDA graph with the host transfers; the layers' queries "
+                   "and the index set cross PCIe on a second stream while routing and "
+                   "attention run; synchronised every step)"}
 
 
 # ---------------------------------------------------------------------------
@@ -923,14 +924,14 @@ def run_e2e_threshold(sd, w, variants, K, V, taus, ws, stream, dev, args, world)
     from pinned memory, outputs, set and counts back, per-step sync):
     DecodeStepGraph, one per query set."""
     return _e2e_graphs(sd, w, variants, K, V, taus, ws, stream, args, world, None,
-                       "decode_step threshold mode")
+                       "route_threshold (full scan)")
 
 
 def run_e2e_louver(sd, w, variants, K, V, ix, taus, ws, stream, dev, args, world):
     """The Louver step through the public API with host buffers:
     DecodeStepGraph over the index, one per query set."""
     return _e2e_graphs(sd, w, variants, K, V, taus, ws, stream, args, world, ix,
-                       "louver_decode_step")
+                       "louver_route_threshold (through the index)")
 
 
 def _e2e_graphs(sd, w, variants, K, V, taus, ws, stream, args, world, index, what):
@@ -958,9 +959,10 @@ def _e2e_graphs(sd, w, variants, K, V, taus, ws, stream, args, world, index, wha
     return {"value": round(world * steps / sec, 2), "unit": "steps/s",
             "h2d_bytes_per_step": g0.h2d_bytes, "d2h_bytes_per_step": g0.d2h_bytes,
             "steps": steps,
-            "api": "token_sparse_attention_sm_b200.DecodeStepGraph (%s with one packed "
-                   "host-to-device and one device-to-host transfer, one CUDA graph; "
-                   "synchronised every step)" % what}
+            "api": "token_sparse_attention_sm_b200.DecodeStepGraph (%s and the layers' "
+                   "attention in one CUDA graph with the host transfers; the layers' queries "
+                   "and the index set cross PCIe on a second stream while routing and "
+                   "attention run; synchronised every step)" % what}
 
 
 def cpu_baseline_threshold(w, x, budget_s: float = 10.0):

@@ -38,7 +38,11 @@
  *    idx [B,Hkv,stride] int32 out [L,B,Hq,d]           lse [L,B,Hq] fp32
  * q/K/V/out share one dtype (fp32 or bf16).  All pointers are device
  * pointers owned by the caller; the library allocates nothing and keeps no
- * per-call state.  q, K, V, S and out must be 16-byte aligned.
+ * per-call state.  q, K, V, S and out must be 16-byte aligned.  out may also
+ * be pinned host memory that kernels reach at its own address (checked with
+ * sparse_pointer_device_usable): the attention then writes the results
+ * straight to the host, and they are there once the stream has passed the
+ * call.
  *
  * Supported: d in {64, 128}; dtype fp32 or bf16; 1 <= G <= 16; N >= 1;
  * B*Hkv <= 65535; L*G <= 1024.
@@ -362,6 +366,14 @@ sparse_status_t sparse_route_topk_static(const sparse_shape_t *shape,
  * receives the raw bit set. */
 sparse_status_t sparse_read_device_status(void *ws, void *stream,
                                           uint32_t *flags);
+
+/* *usable = 1 when kernels can read and write p at its own address: device
+ * memory, managed memory, or pinned host memory mapped into the device's
+ * address space (cudaHostAlloc memory under unified addressing); 0 for
+ * anything else, including pageable host memory and pointers the CUDA
+ * runtime does not know.  Returns SPARSE_ERR_INVALID_ARG for NULL arguments,
+ * else SPARSE_OK.  Enqueues nothing. */
+sparse_status_t sparse_pointer_device_usable(const void *p, int32_t *usable);
 
 #ifdef __cplusplus
 }

@@ -178,3 +178,24 @@ def test_selftest_arguments_rejected(lib):
     assert lib.sparse_selftest_bounded_wait(ctypes.c_void_p(0x100010), 1 << 20, 1000, None) == 1
     assert lib.sparse_selftest_bounded_wait(fake, 1024, 1000, None) == 1
 
+
+
+def test_pointer_device_usable_on_host_memory(lib):
+    """NULL arguments are rejected; ordinary (pageable) host memory is never
+    reported usable by kernels."""
+    ok = ctypes.c_int32(7)
+    assert lib.sparse_pointer_device_usable(None, ctypes.byref(ok)) == 1
+    buf = ctypes.create_string_buffer(4096)
+    assert lib.sparse_pointer_device_usable(ctypes.addressof(buf), None) == 1
+    assert lib.sparse_pointer_device_usable(ctypes.addressof(buf), ctypes.byref(ok)) == 0
+    assert ok.value == 0
+
+
+def test_python_binding_refuses_pageable_out(lib):
+    """An out tensor in pageable host memory is refused before any launch."""
+    t = torch.zeros(2, 1, 8, 64, dtype=torch.bfloat16)
+    assert not sd.device_usable(t)
+    with pytest.raises(ValueError):
+        sd._need_out(t, t)
+    with pytest.raises(ValueError):
+        sd._need_out(torch.zeros(2, 1, 8, 32, dtype=torch.bfloat16), t)

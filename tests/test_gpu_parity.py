@@ -615,6 +615,7 @@ def test_decode_step_graph_equals_eager_step(dev, mode):
         tau=torch.from_numpy(oracle.percentile_tau(oracle.scores(_f(x["q_route"]), _f(x["K"])),
                                                    90, 100)).to(dev), cap=w.cap)
     g = sd.DecodeStepGraph(K, V, w.L, w.Hq, ws=sd.Workspace(dev), **kw)
+    assert g.mapped_out       # torch's pinned buffers are mapped under unified addressing
     assert g.h2d_bytes >= (w.B * w.Hq * w.d + w.L * w.B * w.Hq * w.d) * 2
     for qr, ql in variants:
         g.q_route_host.copy_(qr)
@@ -631,6 +632,26 @@ def test_decode_step_graph_equals_eager_step(dev, mode):
                     n = min(int(ref["count"][b, h]), w.cap)
                     assert torch.equal(res[1][b, h, :n], ref["idx"][b, h, :n].cpu())
     sd.read_device_status(g.ws)
+
+
+def test_outputs_written_straight_to_pinned_host_memory(dev):
+    """attn_gather and decode_step given a pinned host out write there the
+    same bytes they write to device memory."""
+    w = synth.custom(B=1, N=3000, Hq=8, Hkv=2, d=128, L=2, k=64, dtype="bf16", seed=23)
+    x = synth.generate(w)
+    t = {n: x[n].to(dev) for n in ("q_route", "q_layers", "K", "V")}
+    ref = sd.decode_step(t["q_route"], t["q_layers"], t["K"], t["V"], k=w.k)
+    host = torch.full(tuple(t["q_layers"].shape), float("nan"),
+                      dtype=torch.bfloat16).pin_memory()
+    assert sd.device_usable(host)
+    res = sd.decode_step(t["q_route"], t["q_layers"], t["K"], t["V"], k=w.k, out=host)
+    torch.cuda.synchronize()
+    assert res["out"].data_ptr() == host.data_ptr()
+    assert torch.equal(host, ref["out"].cpu())
+    host.fill_(float("nan"))
+    sd.attn_gather(t["q_layers"], t["K"], t["V"], ref["idx"], out=host)
+    torch.cuda.synchronize()
+    assert torch.equal(host, ref["out"].cpu())
 
 
 def test_bounded_wait_expires_and_context_stays_usable(dev):

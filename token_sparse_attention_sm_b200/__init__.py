@@ -28,7 +28,8 @@ __all__ = ["SparseDecodeError", "lib_path", "load", "score", "select_topk",
            "decode_step", "read_device_status", "workspace_bytes",
            "Workspace", "STATUS_NAMES", "EXPORTED_SYMBOLS", "decode_step_grouped",
            "kv_append", "LouverIndex", "louver_build", "louver_route_threshold",
-           "DecodeStepGraph", "selftest_bounded_wait", "louver_decode_step"]
+           "DecodeStepGraph", "selftest_bounded_wait", "louver_decode_step",
+           "device_usable"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_PKG, "libsparse_decode.so")
@@ -48,6 +49,7 @@ EXPORTED_SYMBOLS = (
     "sparse_route_topk_static", "sparse_decode_step_grouped", "sparse_kv_append",
     "sparse_louver_sizes", "sparse_louver_build", "sparse_louver_route_threshold",
     "sparse_selftest_bounded_wait", "sparse_louver_decode_step",
+    "sparse_pointer_device_usable",
 )
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
@@ -113,6 +115,7 @@ def load():
             "sparse_louver_build": (I32, [SH, P, I32, P, SZ, P, SZ, P]),
             "sparse_louver_route_threshold": (I32, [SH, P, P, SZ, I32, P, I32, P, P, P, P,
                                                     SZ, P]),
+            "sparse_pointer_device_usable": (I32, [P, ctypes.POINTER(I32)]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -159,6 +162,34 @@ def _need_cuda(*ts):
             raise ValueError("all tensors must be CUDA tensors")
         if not t.is_contiguous():
             raise ValueError("all tensors must be contiguous")
+
+
+def device_usable(t) -> bool:
+    """True when kernels can write t at its own address: a CUDA tensor, or a
+    pinned host tensor mapped into the device's address space."""
+    if t.is_cuda:
+        return True
+    if not t.is_pinned():
+        return False
+    ok = ctypes.c_int32(0)
+    _check(load().sparse_pointer_device_usable(_ptr(t), ctypes.byref(ok)),
+           "pointer_device_usable")
+    return bool(ok.value)
+
+
+def _need_out(out, like):
+    """out (if given) must have like's shape and dtype, be contiguous, and be
+    device memory or mapped pinned host memory (the attention then writes the
+    results straight to the host)."""
+    if out is None:
+        return
+    if out.shape != like.shape or out.dtype != like.dtype:
+        raise ValueError(f"out must be {tuple(like.shape)} {like.dtype}")
+    if not out.is_contiguous():
+        raise ValueError("out must be contiguous")
+    if not device_usable(out):
+        raise ValueError("out must be a CUDA tensor or pinned host memory the device can "
+                         "reach at its own address")
 
 
 def workspace_bytes(B, N, Hq, Hkv, d, dtype, k_or_cap: int, L: int) -> int:
@@ -344,6 +375,7 @@ def attn_gather(q, K, V, idx, count=None, ws: Workspace | None = None,
     [B,Hkv,stride] (first count[b,h] of each row if count is given).
     Returns (out, lse) with out shaped like q."""
     _need_cuda(q, K, V, idx, count)
+    _need_out(out, q)
     single = q.dim() == 3
     q4 = q.unsqueeze(0) if single else q
     L, B, Hq, d = q4.shape
@@ -392,6 +424,7 @@ def decode_step(q_route, q_layers, K, V, k: int | None = None, tau=None,
     L = q_layers.shape[0]
     if q_layers.shape != (L, B, Hq, d) or V.shape != K.shape:
         raise ValueError("q_layers must be [L,B,Hq,d] and V like K")
+    _need_out(out, q_layers)
     topk = k is not None
     if topk == (tau is not None):
         raise ValueError("give exactly one of k or tau")
@@ -441,6 +474,7 @@ def decode_step_grouped(q_routes, q_layers, K, V, R: int, k: int | None = None, 
     ng = (L + R - 1) // R
     if q_routes.shape[0] != ng or q_layers.shape != (L, B, Hq, d) or V.shape != K.shape:
         raise ValueError("q_routes must be [ceil(L/R),B,Hq,d], q_layers [L,B,Hq,d], V like K")
+    _need_out(out, q_layers)
     topk = k is not None
     if topk == (tau is not None):
         raise ValueError("give exactly one of k or tau")
@@ -615,13 +649,16 @@ class DecodeStepGraph:
     its results, with tensor views: ``q_route_host`` [B,Hq,d] and
     ``q_layers_host`` [L,B,Hq,d] (the cache dtype) to write the next step's
     queries into, ``out_host`` [L,B,Hq,d], ``idx_host`` [B,Hkv,k or cap] and,
-    in threshold mode, ``count_host`` [B,Hkv] to read.  Each replay copies
-    the inputs to the device in one transfer, runs one fused decode step (top-k
-    with ``k``, or threshold with a device ``tau`` [B,Hkv] and ``cap``) over
-    the cache K, V, and copies the results back in one transfer: one graph
-    launch and two copies per step instead of a Python call and four copy
-    launches.  With ``index`` (a LouverIndex of K) and threshold mode the
-    step routes through the index (louver_decode_step).  ``replay()`` enqueues a step on ``stream`` (a new stream by
+    in threshold mode, ``count_host`` [B,Hkv] to read.  Each replay runs one
+    decode step (top-k with ``k``, or threshold with a device ``tau`` [B,Hkv]
+    and ``cap``) over the cache K, V as one graph launch: the routing query is
+    copied in and routing starts while the layers' queries travel on a second
+    stream (joined before the attention); the attention writes its outputs
+    straight into ``out_host`` when the pinned buffer is mapped into the
+    device's address space (``mapped_out``), while the set (and counts)
+    travel back on the second stream; otherwise outputs and set are copied
+    back together after the attention.  With ``index`` (a LouverIndex of K) and
+    threshold mode the step routes through the index.  ``replay()`` enqueues a step on ``stream`` (a new stream by
     default; graphs that share a workspace must use one stream),
     ``synchronize()`` waits for it, calling the object does both.  The device
     status is checked once after the warm-up step (use
@@ -677,29 +714,63 @@ class DecodeStepGraph:
         if index is not None:
             if topk:
                 raise ValueError("routing through a Louver index needs tau and cap")
+            n = index.N
 
-            def run_step():
-                louver_decode_step(q_route, q_layers, K, V, index, tau, cap, ws=self.ws,
-                                   check=False, out=out, idx=idx, count=count,
-                                   return_lse=False)
+            def route():
+                louver_route_threshold(q_route, K, index, tau, cap, check=False, idx=idx,
+                                       count=count)
+        elif topk:
+            def route():
+                route_topk(q_route, K, k, ws=self.ws, check=False, idx=idx, n=n)
         else:
-            args = dict(k=k, tau=tau, cap=cap, ws=self.ws, check=False, out=out, idx=idx,
-                        count=count, return_lse=False, n=n)
+            def route():
+                route_threshold(q_route, K, tau, cap, ws=self.ws, check=False, n=n, idx=idx,
+                                count=count)
 
-            def run_step():
-                decode_step(q_route, q_layers, K, V, **args)
+        self.mapped_out = device_usable(self.out_host)
+        out_dst = self.out_host if self.mapped_out else out
+
+        def attend():
+            attn_gather(q_layers, K, V, idx, count=count, ws=self.ws, check=False,
+                        return_lse=False, out=out_dst, n=n)
+
+        # byte ranges of the packed buffers: [q_route | q_layers], [out | idx (| count)]
+        qr_end = in_offs[1]
+        back = out_offs[1] if self.mapped_out else 0
+        self.side = torch.cuda.Stream(device=dev)
+        ev = [torch.cuda.Event() for _ in range(4)]
 
         def body():
-            self.dev_in.copy_(self.host_in, non_blocking=True)
-            run_step()
-            self.host_out.copy_(self.dev_out, non_blocking=True)
+            main = torch.cuda.current_stream(dev)
+            # the routing query first: the two uploads share one copy engine
+            self.dev_in[:qr_end].copy_(self.host_in[:qr_end], non_blocking=True)
+            ev[0].record(main)
+            self.side.wait_event(ev[0])
+            with torch.cuda.stream(self.side):
+                self.dev_in[qr_end:].copy_(self.host_in[qr_end:], non_blocking=True)
+                ev[1].record(self.side)
+            route()
+            if self.mapped_out:
+                ev[2].record(main)
+                self.side.wait_event(ev[2])
+                with torch.cuda.stream(self.side):
+                    self.host_out[back:].copy_(self.dev_out[back:], non_blocking=True)
+                    ev[3].record(self.side)
+            main.wait_event(ev[1])
+            attend()
+            if self.mapped_out:
+                main.wait_event(ev[3])
+            else:
+                self.host_out.copy_(self.dev_out, non_blocking=True)
 
         self.q_route_host.zero_()
         self.q_layers_host.zero_()
         with torch.cuda.stream(self.stream):
-            body()                       # warm-up: sizes the workspace, loads the library
+            body()                       # warm-up: sizes the workspaces, loads the library
             self.stream.synchronize()
             read_device_status(self.ws)
+            if index is not None:
+                read_device_status(index.ws)
             self.graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(self.graph, stream=self.stream):
                 body()
@@ -746,6 +817,7 @@ def louver_decode_step(q_route, q_layers, K, V, index: LouverIndex, tau, cap: in
     L = q_layers.shape[0]
     if q_layers.shape != (L, B, Hq, d) or V.shape != K.shape:
         raise ValueError("q_layers must be [L,B,Hq,d] and V like K")
+    _need_out(out, q_layers)
     dev = q_route.device
     w = _ws(ws, dev)
     N = index.N

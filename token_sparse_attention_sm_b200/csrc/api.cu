@@ -538,4 +538,26 @@ sparse_status_t sparse_read_device_status(void *ws, void *stream,
   return SPARSE_OK;
 }
 
+sparse_status_t sparse_pointer_device_usable(const void *p, int32_t *usable) {
+  if (!p || !usable) return SPARSE_ERR_INVALID_ARG;
+  *usable = 0;
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();  // an unknown pointer is an answer, not a failure
+    return SPARSE_OK;
+  }
+  switch (a.type) {
+    case cudaMemoryTypeDevice:
+    case cudaMemoryTypeHost:
+      *usable = a.devicePointer == p ? 1 : 0;
+      break;
+    case cudaMemoryTypeManaged:
+      *usable = 1;
+      break;
+    default:
+      break;
+  }
+  return SPARSE_OK;
+}
+
 }  // extern "C"

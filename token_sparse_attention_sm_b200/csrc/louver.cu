@@ -46,6 +46,7 @@ namespace {
 
 constexpr int kPowerIters = 8;
 constexpr int kChunk = 256;       // keys per CTA in the per-node passes
+constexpr int kPU = 4;            // keys whose loads a warp has in flight in those passes
 constexpr int kLvThreads = 512;   // partition CTAs
 constexpr size_t kLvHeader = 4096;
 
@@ -92,21 +93,45 @@ __global__ void identity_perm_kernel(int *perm, int N, long long total) {
   if (i < total) perm[i] = (int)(i % N);
 }
 
-// sums[seg][e] += sum of dimension e over the segment's keys (one CTA of D
-// threads per (segment, chunk)).
+// sums[seg][e] += sum of dimension e over the segment's keys.  Four warps
+// per CTA of kChunk keys, a warp per key with D/32 dimensions per lane and
+// kPU keys' loads in flight per warp.
 template <typename T, int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(128)
     seg_sum_kernel(const T *__restrict__ K, const int *__restrict__ perm, int n, int N,
                    int rows, float *__restrict__ sums, uint32_t *status) {
+  constexpr int EPL = D / 32;
+  __shared__ float red[4][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long base = (long long)blockIdx.x * n;
   const int bh = (int)(base / N);
   const int p0 = blockIdx.y * kChunk, p1 = min(n, p0 + kChunk);
-  float acc = 0.f;
-  for (int p = p0; p < p1; ++p) {
-    const int j = checked_id(perm, base + p, N, status);
-    acc += DT<T>::to_f(K[((size_t)bh * rows + j) * D + threadIdx.x]);
+  float acc[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+  for (int pb = p0 + warp; pb < p1; pb += 4 * kPU) {
+    float x[kPU][EPL];
+#pragma unroll
+    for (int u = 0; u < kPU; ++u) {
+      const int p = pb + 4 * u;
+      if (p < p1) {
+        const int j = checked_id(perm, base + p, N, status);
+        load_elems<T, EPL>(K + ((size_t)bh * rows + j) * D + lane * EPL, x[u]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) x[u][e] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPU; ++u)
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) acc[e] += x[u][e];
   }
-  atomicAdd(&sums[(size_t)blockIdx.x * D + threadIdx.x], acc);
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) red[warp][lane * EPL + e] = acc[e];
+  __syncthreads();
+  for (int i = threadIdx.x; i < D; i += 128)
+    atomicAdd(&sums[(size_t)blockIdx.x * D + i], red[0][i] + red[1][i] + red[2][i] + red[3][i]);
 }
 
 // One pass of the power iteration over the segment's keys: with v = v_in /
@@ -140,22 +165,33 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
   for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
   const int p0 = blockIdx.y * kChunk, p1 = min(n, p0 + kChunk);
-  for (int p = p0 + warp; p < p1; p += 4) {
-    const int j = checked_id(perm, base + p, N, status);
-    float x[EPL];
-    load_elems<T, EPL>(K + ((size_t)bh * rows + j) * D + lane * EPL, x);
-    float y = 0.f;
+  for (int pb = p0 + warp; pb < p1; pb += 4 * kPU) {
+    float x[kPU][EPL];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      x[e] -= mu[e];
-      y += x[e] * v[e];
+    for (int u = 0; u < kPU; ++u) {
+      const int p = pb + 4 * u;
+      if (p < p1) {
+        const int j = checked_id(perm, base + p, N, status);
+        load_elems<T, EPL>(K + ((size_t)bh * rows + j) * D + lane * EPL, x[u]);
+      }
     }
-    y = warp_sum(y);
-    if (proj) {
-      if (lane == 0) proj[base + p] = y;
-    } else {
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) acc[e] += y * x[e];
+    for (int u = 0; u < kPU; ++u) {
+      const int p = pb + 4 * u;
+      if (p >= p1) break;
+      float y = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        x[u][e] -= mu[e];
+        y += x[u][e] * v[e];
+      }
+      y = warp_sum(y);
+      if (proj) {
+        if (lane == 0) proj[base + p] = y;
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] += y * x[u][e];
+      }
     }
   }
   if (proj) return;
@@ -739,7 +775,7 @@ cudaError_t lv_build_t(const Shape &s, const void *Kv, int r, char *index, char 
     const dim3 grid((unsigned)nseg, (unsigned)((n + kChunk - 1) / kChunk));
     e = cudaMemsetAsync(sums, 0, (size_t)nseg * D * 4, st);
     if (e != cudaSuccess) break;
-    seg_sum_kernel<T, D><<<grid, D, 0, st>>>(K, cur, n, s.N, s.Ncap, sums, status);
+    seg_sum_kernel<T, D><<<grid, 128, 0, st>>>(K, cur, n, s.N, s.Ncap, sums, status);
     float *vin = va, *vout = vb;
     for (int it = 0; it < kPowerIters && e == cudaSuccess; ++it) {
       e = cudaMemsetAsync(vout, 0, (size_t)nseg * D * 4, st);
