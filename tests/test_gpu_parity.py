@@ -413,6 +413,28 @@ def test_dense_attention_all_keys(dev, dtype, N):
     assert_attn_close(out, lse, o_ref, l_ref, dtype)
 
 
+@pytest.mark.parametrize("B,Hkv,N,k", [(1, 8, 8192, 2048), (2, 8, 6000, 1024),
+                                       (1, 2, 5000, 300), (3, 1, 4000, 700)])
+def test_attention_cluster_merge_equals_global_merge(dev, monkeypatch, B, Hkv, N, k):
+    """The split-k merge inside a thread-block cluster (partials read through
+    distributed shared memory) and the merge through global memory combine
+    the same partials in the same order: bit-identical outputs, both within
+    tolerance of the oracle."""
+    w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=16, k=k, dtype="bf16", seed=31)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    idx = oracle.topk(oracle.scores(_f(x["q_route"]), _f(x["K"])), w.k)
+    idx_t = torch.from_numpy(idx).to(dev)
+    monkeypatch.setenv("SPARSE_DECODE_ATTN_MERGE", "global")
+    o_g, l_g = sd.attn_gather(t["q_layers"], t["K"], t["V"], idx_t)
+    monkeypatch.delenv("SPARSE_DECODE_ATTN_MERGE")
+    o_c, l_c = sd.attn_gather(t["q_layers"], t["K"], t["V"], idx_t)
+    assert torch.equal(o_g, o_c)
+    assert torch.equal(l_g, l_c)
+    o_ref, l_ref = oracle.attn(_f(x["q_layers"]), _f(x["K"]), _f(x["V"]), idx)
+    assert_attn_close(o_c, l_c, o_ref, l_ref, "bf16")
+
+
 def test_attn_gather_mma_sync_variant_matches(dev, monkeypatch):
     """The warp-level mma.sync kernel (kept for comparison) agrees too."""
     monkeypatch.setenv("SPARSE_DECODE_ATTN", "mma")

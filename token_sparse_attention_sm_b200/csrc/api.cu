@@ -20,6 +20,7 @@
 //   [.., ..)              fused routing: published boundary-bin keys
 //   [.., ..)              attention split partials
 #include <stdlib.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -158,6 +159,11 @@ bool cooperative_forced() {
     return v && v[0] == '1';
   }();
   return on;
+}
+
+bool attn_cluster_merge_enabled() {
+  const char *v = getenv("SPARSE_DECODE_ATTN_MERGE");  // read per call
+  return !(v && strcmp(v, "global") == 0);
 }
 
 bool pdl_enabled() {

@@ -30,14 +30,25 @@
 // counter and waits (bounded) for the other splits -- the grid is at most
 // one CTA per SM, so all of them are resident -- then merges its share of the
 // rows by log-sum-exp rescaling; the last split to leave resets the counters.
+// When the splits of a head can run as one thread-block cluster (up to 16
+// CTAs, all clusters resident at once), the partials stay in shared memory
+// instead: one cluster barrier, then each CTA merges its rows reading every
+// split's partial through distributed shared memory, and a second barrier
+// keeps each partial in place until its readers are done.
 //
 // Every wait is bounded; on expiry the kernel raises the TIMEOUT flag, stops
 // issuing work, frees its tensor memory and returns.
+#include <cooperative_groups.h>
+
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace sd {
 namespace {
+
+namespace cg = cooperative_groups;
 
 constexpr int kGroups = 4;          // warps sharing a tensor-memory lane quadrant
 constexpr int kTcThreads = 128 * kGroups;
@@ -48,6 +59,7 @@ constexpr int kChunkTiles = 4;      // tiles per chunk (S uses 256 TMEM columns)
 constexpr int kChunkKeys = kTileN * kChunkTiles;
 constexpr int kTmemCols = 512;
 constexpr int kTcMaxSplits = 16;
+constexpr int kTcMaxDevices = 64;
 
 template <int D>
 struct TcCfg {
@@ -168,7 +180,7 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
 
-template <int D>
+template <int D, bool kCluster>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __nv_bfloat16 *__restrict__ q,
                    const __nv_bfloat16 *__restrict__ K,
@@ -510,7 +522,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         make_float4(have ? mrun : -INFINITY, ls, 0.f, 0.f);
   }
   __syncthreads();
-  {
+  if constexpr (!kCluster) {
     const int n4 = mrows * PR / 4;
     const float4 *src = reinterpret_cast<const float4 *>(stage);
     float4 *dst = reinterpret_cast<float4 *>(mypart);
@@ -524,23 +536,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)
                  : "memory");
-  // arrive, then wait (bounded) until every split of this head block arrived;
-  // the grid (at most one CTA per SM) is resident as a whole
-  uint32_t *arrive = counters + 2 * ((size_t)bh * gridDim.y + qb);
-  uint32_t *depart = arrive + 1;
-  __shared__ int ready;
-  if (tid == 0) {
-    __threadfence();
-    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(arrive) : "memory");
-    ready = wait_counter_geq(arrive, (uint32_t)csize, kWaitLimitNs, status);
-  }
-  __syncthreads();
-  if (ready) {
-    // merge rows lr = rank, rank + csize, ...: thread = (row slot, float4
-    // chunk); every split's values are loaded before any is used
+  // merge rows lr = rank, rank + csize, ...: thread = (row slot, float4
+  // chunk); every split's values are loaded before any is used.  prow(r, lr)
+  // is split r's partial row lr.
+  auto merge = [&](auto prow) {
     constexpr int CH = D / 4;
     constexpr int RPP = kTcThreads / CH;  // rows per pass
-    const float *hp = part + ((size_t)bh * gridDim.y + qb) * csize * kTcRows * PR;
     const int nmine = (mrows - rank + csize - 1) / csize;
     for (int i = tid / CH; i < nmine; i += RPP) {
       const int lr = rank + i * csize;
@@ -550,7 +551,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int r = 0; r < kTcMaxSplits; ++r) {
         if (r < csize) {
-          const float *pr = hp + ((size_t)r * kTcRows + lr) * PR;
+          const float *pr = prow(r, lr);
           ml[r] = *reinterpret_cast<const float2 *>(pr + D);
           v[r] = *reinterpret_cast<const float4 *>(pr + ch * 4);
         } else {
@@ -584,10 +585,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lse && ch == 0)
         lse[orow] = ls > 0.f ? (mx + log2f(ls)) * 0.69314718055994531f : -INFINITY;
     }
+  };
+  if constexpr (kCluster) {
+    // the head's splits are this cluster (cluster rank = blockIdx.x); the
+    // barriers are hardware cluster barriers that every CTA reaches (nothing
+    // above returns early)
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();  // every split's partial is staged in its shared memory
+    merge([&](int r, int lr) -> const float * {
+      return cluster.map_shared_rank(stage, r) + (size_t)lr * PR;
+    });
+    cluster.sync();  // no CTA leaves while another reads its partial
+    return;
+  } else {
+    // arrive, then wait (bounded) until every split of this head block
+    // arrived; the grid (at most one CTA per SM) is resident as a whole
+    uint32_t *arrive = counters + 2 * ((size_t)bh * gridDim.y + qb);
+    __shared__ int ready;
+    if (tid == 0) {
+      __threadfence();
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(arrive) : "memory");
+      ready = wait_counter_geq(arrive, (uint32_t)csize, kWaitLimitNs, status);
+    }
+    __syncthreads();
+    const float *hp = part + ((size_t)bh * gridDim.y + qb) * csize * kTcRows * PR;
+    if (ready)
+      merge([&](int r, int lr) -> const float * {
+        return hp + ((size_t)r * kTcRows + lr) * PR;
+      });
   }
   // the last split to leave resets both counters for the next call
   __syncthreads();
   if (tid == 0) {
+    uint32_t *arrive = counters + 2 * ((size_t)bh * gridDim.y + qb);
+    uint32_t *depart = arrive + 1;
     const uint32_t old = atomicAdd(depart, 1u);
     if (old == (uint32_t)csize - 1) {
       *arrive = 0u;
@@ -602,6 +633,51 @@ size_t tc_part_bytes(const Shape &s, int L) {
   const int M = L * s.G();
   const int qblocks = (M + kTcRows - 1) / kTcRows;
   return (size_t)s.BH() * qblocks * kTcMaxSplits * kTcRows * (D + 4) * sizeof(float);
+}
+
+// Whether `blocks` clusters of `nsplit` attention CTAs can all be resident
+// at once (cudaOccupancyMaxActiveClusters), cached per device and split
+// count; sizes above the portable 8 need the non-portable opt-in.
+template <int D>
+bool tc_clusters_fit(int nsplit, long long blocks) {
+  using C = TcCfg<D>;
+  static std::atomic<int> cache[kTcMaxDevices][kTcMaxSplits + 1];  // 0 unknown, 1 + max
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kTcMaxDevices ||
+      nsplit > kTcMaxSplits) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  int v = cache[dev][nsplit].load(std::memory_order_relaxed);
+  if (v == 0) {
+    auto kern = attn_tc_kernel<D, true>;
+    int n = 0;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e == cudaSuccess && nsplit > 8)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)nsplit, 1, 1);
+      cfg.blockDim = dim3(kTcThreads, 1, 1);
+      cfg.dynamicSmemBytes = C::kSmem;
+      cudaLaunchAttribute a;
+      a.id = cudaLaunchAttributeClusterDimension;
+      a.val.clusterDim.x = (unsigned)nsplit;
+      a.val.clusterDim.y = 1;
+      a.val.clusterDim.z = 1;
+      cfg.attrs = &a;
+      cfg.numAttrs = 1;
+      e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    }
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    v = 1 + n;
+    cache[dev][nsplit].store(v, std::memory_order_relaxed);
+  }
+  return (long long)(v - 1) >= blocks;
 }
 
 template <int D>
@@ -625,9 +701,6 @@ cudaError_t launch_tc_t(const Shape &s, int L, const void *q, const void *K,
   nsplit = nsplit > kTcMaxSplits ? kTcMaxSplits : nsplit;
   nsplit = nsplit < 1 ? 1 : nsplit;
   if (blocks > kAttnMaxCounterBlocks) nsplit = 1;  // counters live in a fixed area
-  auto kern = attn_tc_kernel<D>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-  if (e != cudaSuccess) return e;
   float *part = static_cast<float *>(ws);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)nsplit, (unsigned)qblocks, (unsigned)s.BH());
@@ -635,10 +708,29 @@ cudaError_t launch_tc_t(const Shape &s, int L, const void *q, const void *K,
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  // merge through distributed shared memory when each head block's splits
+  // can form one cluster and all those clusters fit on the device at once
+  bool cluster = nsplit > 1 && !cooperative_forced() && attn_cluster_merge_enabled() &&
+                 tc_clusters_fit<D>(nsplit, blocks);
+  auto kern = cluster ? attn_tc_kernel<D, true> : attn_tc_kernel<D, false>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  if (cluster && nsplit > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  if (cluster) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)nsplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.numAttrs = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.numAttrs = (nsplit > 1 && cooperative_forced()) ? 1 : 0;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = (nsplit > 1 && cooperative_forced()) ? 1 : 0;
   add_pdl_attr(cfg, attr);
   const float scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16 *>(q),

@@ -68,6 +68,10 @@ cudaError_t launch_route_topk_fused(const Shape &s, const void *q, const void *K
 // SPARSE_DECODE_COOPERATIVE=1 launches them cooperatively instead (the driver
 // then guarantees co-residency even next to other work on the device).
 bool cooperative_forced();
+// The split attention merges its partials inside a thread-block cluster
+// (distributed shared memory) when the clusters fit; SPARSE_DECODE_ATTN_MERGE=global
+// selects the merge through global memory and a counter barrier instead.
+bool attn_cluster_merge_enabled();
 
 // A2 / A2': selection from S.  k >= 1: top-k (tau ignored); k == 0:
 // threshold with tau and cap, count written.  idx rows have `stride`
