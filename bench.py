@@ -513,9 +513,10 @@ def run_e2e(sd, w, variants, K, V, ws, stream, dev, args, world):
             "h2d_bytes_per_step": g0.h2d_bytes, "d2h_bytes_per_step": g0.d2h_bytes,
             "steps": steps,
             "api": "token_sparse_attention_sm_b200.DecodeStepGraph (routing and the layers' "
-                   "attention in one CUDA graph with the host transfers; the layers' queries "
+                   "attention in one CUDA graph with the host transfers: the layers' queries "
                    "and the index set cross PCIe on a second stream while routing and "
-                   "attention run; synchronised every step)"}
+                   "attention run, the attention writes its outputs into mapped pinned host "
+                   "memory (mapped_out=%s); synchronised every step)" % g0.mapped_out}
 
 
 # ---------------------------------------------------------------------------
@@ -960,9 +961,10 @@ def _e2e_graphs(sd, w, variants, K, V, taus, ws, stream, args, world, index, wha
             "h2d_bytes_per_step": g0.h2d_bytes, "d2h_bytes_per_step": g0.d2h_bytes,
             "steps": steps,
             "api": "token_sparse_attention_sm_b200.DecodeStepGraph (%s and the layers' "
-                   "attention in one CUDA graph with the host transfers; the layers' queries "
+                   "attention in one CUDA graph with the host transfers: the layers' queries "
                    "and the index set cross PCIe on a second stream while routing and "
-                   "attention run; synchronised every step)" % what}
+                   "attention run, the attention writes its outputs into mapped pinned host "
+                   "memory (mapped_out=%s); synchronised every step)" % (what, g0.mapped_out)}
 
 
 def cpu_baseline_threshold(w, x, budget_s: float = 10.0):
