@@ -656,6 +656,28 @@ def test_decode_step_graph_equals_eager_step(dev, mode):
     sd.read_device_status(g.ws)
 
 
+def test_decode_step_graph_survives_workspace_growth(dev):
+    """A later call that needs a larger workspace replaces the workspace's
+    buffer; a graph captured before keeps the buffer it captured and still
+    returns the eager step's results."""
+    w = synth.custom(B=1, N=4000, Hq=8, Hkv=2, d=128, L=2, k=64, dtype="bf16", seed=41)
+    x = synth.generate(w)
+    K, V = x["K"].to(dev), x["V"].to(dev)
+    ws = sd.Workspace(dev)
+    g = sd.DecodeStepGraph(K, V, w.L, w.Hq, k=w.k, ws=ws)
+    before = ws.buf.data_ptr()
+    big = torch.randn(64, 1, w.Hq, w.d, generator=torch.Generator().manual_seed(3)).to(
+        torch.bfloat16).to(dev)
+    sd.decode_step(x["q_route"].to(dev), big, K, V, k=3000, ws=ws)   # grows ws
+    assert ws.buf.data_ptr() != before
+    g.q_route_host.copy_(x["q_route"])
+    g.q_layers_host.copy_(x["q_layers"])
+    out, idx = g()
+    ref = sd.decode_step(x["q_route"].to(dev), x["q_layers"].to(dev), K, V, k=w.k)
+    assert torch.equal(out, ref["out"].cpu())
+    assert torch.equal(idx, ref["idx"].cpu())
+
+
 def test_outputs_written_straight_to_pinned_host_memory(dev):
     """attn_gather and decode_step given a pinned host out write there the
     same bytes they write to device memory."""

@@ -202,7 +202,10 @@ def workspace_bytes(B, N, Hq, Hkv, d, dtype, k_or_cap: int, L: int) -> int:
 
 class Workspace:
     """A zero-initialised device workspace that grows on demand.  Calls that
-    share one must be ordered on the same stream."""
+    share one must be ordered on the same stream.  Growing replaces the
+    buffer: a CUDA graph captured earlier keeps using the old one, so whoever
+    holds such a graph also holds a reference to the buffer it captured
+    (DecodeStepGraph does)."""
 
     def __init__(self, device=None):
         self.device = torch.device(device) if device is not None else torch.device(
@@ -774,6 +777,10 @@ class DecodeStepGraph:
             self.graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(self.graph, stream=self.stream):
                 body()
+        # the graph holds raw addresses: keep every buffer it touches alive
+        # (a later, larger call may replace a workspace's buffer)
+        self._captured = (self.ws.buf, index.ws.buf if index is not None else None, index,
+                          K, V, tau)
 
     @property
     def h2d_bytes(self) -> int:
