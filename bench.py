@@ -483,12 +483,13 @@ def run_native(args, rank, world, local_rank):
 def run_e2e(sd, w, variants, K, V, ws, stream, dev, args, world):
     """Same metric through the public Python API with host buffers: every
     step copies its queries from pinned host memory to the device, runs the
-    decode step, and copies the outputs and the index set back to pinned
-    host memory, then waits for them -- all inside the timed region.  The
-    step is the library's DecodeStepGraph (the step and its two packed
-    transfers captured once as a CUDA graph), one per query set, as a caller
-    double-buffering its inputs keeps them; its pinned input views hold the
-    set's queries."""
+    decode step, and brings the outputs and the index set back to pinned host
+    memory (the outputs written there by the attention itself when the buffer
+    is mapped), then waits for them -- all inside the timed region.  The step
+    is the library's DecodeStepGraph (routing, attention and the transfers
+    captured once as a CUDA graph, launched by one C call per step), one per
+    query set, as a caller double-buffering its inputs keeps them; its pinned
+    input views hold the set's queries."""
     graphs = []
     for qr, ql in variants:
         g = sd.DecodeStepGraph(K, V, w.L, w.Hq, k=w.k, ws=ws, stream=stream)

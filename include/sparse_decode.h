@@ -367,6 +367,12 @@ sparse_status_t sparse_route_topk_static(const sparse_shape_t *shape,
 sparse_status_t sparse_read_device_status(void *ws, void *stream,
                                           uint32_t *flags);
 
+/* Enqueue an instantiated CUDA graph (a cudaGraphExec_t, e.g. a captured
+ * decode step with its host transfers) on `stream`: one C call per replayed
+ * step.  Returns SPARSE_ERR_INVALID_ARG for a NULL graph, SPARSE_ERR_CUDA if
+ * the launch fails, else SPARSE_OK.  Does not synchronise. */
+sparse_status_t sparse_graph_launch(void *graph_exec, void *stream);
+
 /* *usable = 1 when kernels can read and write p at its own address: device
  * memory, managed memory, or pinned host memory mapped into the device's
  * address space (cudaHostAlloc memory under unified addressing); 0 for

@@ -199,3 +199,7 @@ def test_python_binding_refuses_pageable_out(lib):
         sd._need_out(t, t)
     with pytest.raises(ValueError):
         sd._need_out(torch.zeros(2, 1, 8, 32, dtype=torch.bfloat16), t)
+
+
+def test_graph_launch_rejects_null(lib):
+    assert lib.sparse_graph_launch(None, None) == 1

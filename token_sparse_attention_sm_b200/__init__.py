@@ -49,7 +49,7 @@ EXPORTED_SYMBOLS = (
     "sparse_route_topk_static", "sparse_decode_step_grouped", "sparse_kv_append",
     "sparse_louver_sizes", "sparse_louver_build", "sparse_louver_route_threshold",
     "sparse_selftest_bounded_wait", "sparse_louver_decode_step",
-    "sparse_pointer_device_usable",
+    "sparse_pointer_device_usable", "sparse_graph_launch",
 )
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
@@ -116,6 +116,7 @@ def load():
             "sparse_louver_route_threshold": (I32, [SH, P, P, SZ, I32, P, I32, P, P, P, P,
                                                     SZ, P]),
             "sparse_pointer_device_usable": (I32, [P, ctypes.POINTER(I32)]),
+            "sparse_graph_launch": (I32, [P, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -781,6 +782,9 @@ class DecodeStepGraph:
         # (a later, larger call may replace a workspace's buffer)
         self._captured = (self.ws.buf, index.ws.buf if index is not None else None, index,
                           K, V, tau)
+        self._exec = ctypes.c_void_p(self.graph.raw_cuda_graph_exec())
+        self._st = ctypes.c_void_p(self.stream.cuda_stream)
+        self._launch = load().sparse_graph_launch
 
     @property
     def h2d_bytes(self) -> int:
@@ -791,13 +795,11 @@ class DecodeStepGraph:
         return self.host_out.numel()
 
     def replay(self):
-        """Enqueue one step (inputs from, results to, the pinned host buffers).
-        Cheapest when called with the graph's stream current."""
-        if torch.cuda.current_stream(self.stream.device).cuda_stream == self.stream.cuda_stream:
-            self.graph.replay()
-        else:
-            with torch.cuda.stream(self.stream):
-                self.graph.replay()
+        """Enqueue one step on the object's stream (inputs from, results to,
+        the pinned host buffers): one C call launching the instantiated graph."""
+        rc = self._launch(self._exec, self._st)
+        if rc != 0:
+            raise SparseDecodeError(rc, "graph_launch")
 
     def synchronize(self):
         self.stream.synchronize()
