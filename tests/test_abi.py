@@ -203,3 +203,25 @@ def test_python_binding_refuses_pageable_out(lib):
 
 def test_graph_launch_rejects_null(lib):
     assert lib.sparse_graph_launch(None, None) == 1
+
+
+def test_result_and_tau_checks_reject_bad_tensors(lib):
+    """Caller-given results must match exactly and live where kernels can
+    write them; tau needs one float per row of the sets.  All checked before
+    anything is launched."""
+    sd._need_result(None, (2, 3), torch.int32, "idx")          # nothing given: fine
+    with pytest.raises(ValueError, match="idx"):
+        sd._need_result(torch.zeros(2, 4, dtype=torch.int32), (2, 3), torch.int32, "idx")
+    with pytest.raises(ValueError, match="idx"):
+        sd._need_result(torch.zeros(2, 3, dtype=torch.int64), (2, 3), torch.int32, "idx")
+    with pytest.raises(ValueError, match="contiguous"):
+        sd._need_result(torch.zeros(3, 2, dtype=torch.int32).t(), (2, 3), torch.int32, "idx")
+    with pytest.raises(ValueError, match="CUDA"):                # host memory, right shape
+        sd._need_result(torch.zeros(2, 3, dtype=torch.int32), (2, 3), torch.int32, "idx")
+    with pytest.raises(ValueError, match="pinned"):              # pageable host memory
+        sd._need_result(torch.zeros(2, 3), (2, 3), torch.float32, "lse", host_ok=True)
+    sd._need_tau(torch.zeros(2, 3), (2, 3))
+    with pytest.raises(ValueError, match="tau"):
+        sd._need_tau(torch.zeros(2, 4), (2, 3))
+    with pytest.raises(ValueError, match="tau"):
+        sd._need_tau(torch.zeros(2, 3, dtype=torch.int32), (2, 3))

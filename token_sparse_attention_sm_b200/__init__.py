@@ -178,19 +178,37 @@ def device_usable(t) -> bool:
     return bool(ok.value)
 
 
+def _need_result(t, shape, dtype, name: str, host_ok: bool = False):
+    """A caller-given result tensor (if any) must have exactly this shape and
+    dtype, be contiguous, and be device memory -- or, where host_ok, pinned
+    host memory mapped into the device's address space -- since the kernels
+    write all of it."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.is_cuda or (host_ok and device_usable(t)):
+        return
+    raise ValueError(f"{name} must be a CUDA tensor" +
+                     (" or pinned host memory the device can reach at its own address"
+                      if host_ok else ""))
+
+
+def _need_tau(tau, shape):
+    """tau holds one threshold per row of the sets: exactly this shape, real."""
+    if tuple(tau.shape) != tuple(shape) or not tau.is_floating_point():
+        raise ValueError(f"tau must be a float tensor of shape {tuple(shape)}, "
+                         f"got {tau.dtype} {tuple(tau.shape)}")
+
+
 def _need_out(out, like):
     """out (if given) must have like's shape and dtype, be contiguous, and be
     device memory or mapped pinned host memory (the attention then writes the
     results straight to the host)."""
-    if out is None:
-        return
-    if out.shape != like.shape or out.dtype != like.dtype:
-        raise ValueError(f"out must be {tuple(like.shape)} {like.dtype}")
-    if not out.is_contiguous():
-        raise ValueError("out must be contiguous")
-    if not device_usable(out):
-        raise ValueError("out must be a CUDA tensor or pinned host memory the device can "
-                         "reach at its own address")
+    _need_result(out, like.shape, like.dtype, "out", host_ok=True)
 
 
 def workspace_bytes(B, N, Hq, Hkv, d, dtype, k_or_cap: int, L: int) -> int:
@@ -271,6 +289,7 @@ def score(q, K, ws: Workspace | None = None, check: bool = True, out=None,
     _need_cuda(q, K, out)
     B, Ncap, Hq, Hkv, d = _dims_qk(q, K)
     N = _length(Ncap, n)
+    _need_result(out, (B, Hkv, N), torch.float32, "out")
     w = _ws(ws, q.device)
     sh = _shape(B, N, Hq, Hkv, d, q.dtype, Ncap)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, 1, 1))
@@ -287,6 +306,7 @@ def select_topk(S, k: int, ws: Workspace | None = None, check: bool = True,
     """Top-k of S [B,Hkv,N] fp32 -> idx [B,Hkv,k] int32 ascending."""
     _need_cuda(S, idx)
     B, Hkv, N = S.shape
+    _need_result(idx, (B, Hkv, k), torch.int32, "idx")
     w = _ws(ws, S.device)
     sh = _shape(B, N, Hkv, Hkv, 64, torch.float32)
     buf = w.get(workspace_bytes(B, N, Hkv, Hkv, 64, torch.float32, k, 1))
@@ -319,6 +339,7 @@ def select_threshold(S, tau, cap: int, ws: Workspace | None = None,
     """Threshold sets of S: (idx [B,Hkv,cap], count [B,Hkv])."""
     _need_cuda(S, tau)
     B, Hkv, N = S.shape
+    _need_tau(tau, (B, Hkv))
     w = _ws(ws, S.device)
     sh = _shape(B, N, Hkv, Hkv, 64, torch.float32)
     buf = w.get(workspace_bytes(B, N, Hkv, Hkv, 64, torch.float32, cap, 1))
@@ -339,6 +360,7 @@ def route_topk(q, K, k: int, ws: Workspace | None = None, check: bool = True,
     _need_cuda(q, K, idx)
     B, Ncap, Hq, Hkv, d = _dims_qk(q, K)
     N = _length(Ncap, n)
+    _need_result(idx, (B, Hkv, k), torch.int32, "idx")
     w = _ws(ws, q.device)
     sh = _shape(B, N, Hq, Hkv, d, q.dtype, Ncap)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, k, 1))
@@ -363,6 +385,7 @@ def route_threshold(q, K, tau, cap: int, ws: Workspace | None = None,
     sh = _shape(B, N, Hq, Hkv, d, q.dtype, Ncap)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q.dtype, cap, 1))
     idx, count = _threshold_outputs(idx, count, B, Hkv, cap, q.device)
+    _need_tau(tau, (B, Hkv))
     tau = tau.float().contiguous()
     _check(load().sparse_route_threshold(
         ctypes.byref(sh), _ptr(q), _ptr(K), _ptr(tau), int(cap), _ptr(idx),
@@ -380,6 +403,7 @@ def attn_gather(q, K, V, idx, count=None, ws: Workspace | None = None,
     Returns (out, lse) with out shaped like q."""
     _need_cuda(q, K, V, idx, count)
     _need_out(out, q)
+    _need_result(lse, q.shape[:-1], torch.float32, "lse", host_ok=True)
     single = q.dim() == 3
     q4 = q.unsqueeze(0) if single else q
     L, B, Hq, d = q4.shape
@@ -389,6 +413,7 @@ def attn_gather(q, K, V, idx, count=None, ws: Workspace | None = None,
         raise ValueError("shape mismatch between q, K and V")
     if idx.dtype != torch.int32 or idx.dim() != 3 or idx.shape[:2] != (B, Hkv):
         raise ValueError("idx must be int32 [B,Hkv,stride]")
+    _need_result(count, (B, Hkv), torch.int32, "count")
     stride = idx.shape[2]
     w = _ws(ws, q.device)
     sh = _shape(B, N, Hq, Hkv, d, q.dtype, Ncap)
@@ -433,6 +458,12 @@ def decode_step(q_route, q_layers, K, V, k: int | None = None, tau=None,
     if topk == (tau is not None):
         raise ValueError("give exactly one of k or tau")
     stride = int(k) if topk else int(cap)
+    _need_result(idx, (B, Hkv, stride), torch.int32, "idx")
+    if not topk:
+        _need_result(count, (B, Hkv), torch.int32, "count")
+    _need_result(lse, (L, B, Hq), torch.float32, "lse", host_ok=True)
+    if not topk:
+        _need_tau(tau, (B, Hkv))
     dev = q_route.device
     w = _ws(ws, dev)
     sh = _shape(B, N, Hq, Hkv, d, q_route.dtype, Ncap)
@@ -483,6 +514,12 @@ def decode_step_grouped(q_routes, q_layers, K, V, R: int, k: int | None = None, 
     if topk == (tau is not None):
         raise ValueError("give exactly one of k or tau")
     stride = int(k) if topk else int(cap)
+    _need_result(idx, (ng, B, Hkv, stride), torch.int32, "idx")
+    if not topk:
+        _need_result(count, (ng, B, Hkv), torch.int32, "count")
+    _need_result(lse, (L, B, Hq), torch.float32, "lse", host_ok=True)
+    if not topk:
+        _need_tau(tau, (ng, B, Hkv))
     dev = q_routes.device
     w = _ws(ws, dev)
     sh = _shape(B, N, Hq, Hkv, d, q_routes.dtype, Ncap)
@@ -624,15 +661,12 @@ def louver_route_threshold(q, K, index: LouverIndex, tau, cap: int, check: bool 
     if (B, Hkv, Ncap, d, K.dtype) != (index.B, index.Hkv, index.Ncap, index.d, index.dtype):
         raise ValueError("the index was built for another K")
     sh = _shape(B, index.N, Hq, Hkv, d, q.dtype, Ncap)
-    if idx is None:
-        idx = torch.empty((B, Hkv, cap), dtype=torch.int32, device=q.device)
-    if count is None:
-        count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    idx, count = _threshold_outputs(idx, count, B, Hkv, cap, q.device)
+    _need_result(survivors, (B, Hkv, 2), torch.int32, "survivors")
     surv = survivors
     if return_survivors and surv is None:
         surv = torch.empty((B, Hkv, 2), dtype=torch.int32, device=q.device)
-    if idx.shape != (B, Hkv, cap) or count.shape != (B, Hkv):
-        raise ValueError("idx must be [B,Hkv,cap] and count [B,Hkv]")
+    _need_tau(tau, (B, Hkv))
     tau = tau.float().contiguous()
     buf = index.ws.get(index.ws_bytes)
     _check(load().sparse_louver_route_threshold(
@@ -833,6 +867,8 @@ def louver_decode_step(q_route, q_layers, K, V, index: LouverIndex, tau, cap: in
     sh = _shape(B, N, Hq, Hkv, d, q_route.dtype, Ncap)
     buf = w.get(workspace_bytes(B, N, Hq, Hkv, d, q_route.dtype, cap, L))
     idx, count = _threshold_outputs(idx, count, B, Hkv, cap, dev)
+    _need_result(lse, (L, B, Hq), torch.float32, "lse", host_ok=True)
+    _need_tau(tau, (B, Hkv))
     if out is None:
         out = torch.empty_like(q_layers)
     if lse is None and return_lse:
