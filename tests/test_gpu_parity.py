@@ -625,7 +625,7 @@ def test_kv_append_then_decode(dev, dtype, d):
 
 @pytest.mark.parametrize("mode", ["topk", "threshold"])
 def test_decode_step_graph_equals_eager_step(dev, mode):
-    """The captured step with its packed host transfers returns, for each new
+    """The captured step with its host transfers returns, for each new
     query written into its pinned input views, exactly what the eager step
     returns."""
     w = synth.custom(B=2, N=5000, Hq=8, Hkv=2, d=128, L=3, k=100, dtype="bf16", seed=17,
