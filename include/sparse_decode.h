@@ -69,7 +69,10 @@
  * ordinary kernels so that each can start while its predecessor drains.  A
  * caller that runs other kernels on the same device at the same time (other
  * streams, other processes) sets SPARSE_DECODE_COOPERATIVE=1: they are then
- * launched cooperatively and the driver guarantees co-residency.
+ * launched cooperatively and the driver guarantees co-residency.  Where all
+ * of a launch's heads fit at once as thread-block clusters, the attention's
+ * splits of a head run as one cluster instead and merge through distributed
+ * shared memory behind hardware cluster barriers.
  *
  * Environment variables read by the library:
  *   SPARSE_DECODE_PDL=0           no programmatic dependent launch
@@ -77,6 +80,8 @@
  *   SPARSE_DECODE_FUSED_ROUTE=1   top-k routing as one fused scan+select kernel
  *                                 where the shape allows (results identical)
  *   SPARSE_DECODE_ATTN=mma        bf16 attention on the mma.sync kernel
+ *   SPARSE_DECODE_ATTN_MERGE=global  the attention's split merge through
+ *                                 global memory even where clusters would fit
  */
 #ifndef SPARSE_DECODE_H_
 #define SPARSE_DECODE_H_
