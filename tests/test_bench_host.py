@@ -1,0 +1,89 @@
+"""bench.py's host-side contract, on the CPU: the reference arm (the CPU
+oracle on bounded samples) prints one JSON line with the required keys and
+only on rank 0, and the figures the native arm reports are derived from the
+workload as stated (no GPU involved)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from token_sparse_attention_sm_b200 import synth  # noqa: E402
+
+
+def _run(args, env_extra=None, timeout=300):
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT,
+                       env=env, capture_output=True, text=True, timeout=timeout)
+    return r
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = _run(["--impl", "reference", "--workload", "tiny_f32", "--steps", "2",
+              "--warmup", "3"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
+    assert d["unit"] == "steps/s" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["n_gpus"] == 1 and d["steps"] == 2 and d["warmup"] == 3
+    assert abs(d["ms_per_step"] - 1e3 / d["value"]) <= 1e-3 * d["ms_per_step"] + 1e-3
+    assert d["config"]["workload"] == "tiny_f32"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
+    assert cb["unit"] == "steps/s" and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "steps/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    r = _run(["--impl", "reference", "--workload", "tiny_f32", "--steps", "1",
+              "--warmup", "3"], {"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
+
+
+def test_warmup_below_three_is_refused():
+    r = _run(["--impl", "reference", "--workload", "tiny_f32", "--steps", "1",
+              "--warmup", "2"])
+    assert r.returncode != 0
+
+
+def test_algorithmic_bytes_of_the_headline_step():
+    """The K cache once plus the selected K and V rows once: 268,435,456 +
+    8,388,608 = 276,824,064 bytes per step at 128K, k = 2048, bf16."""
+    scan, gathered = bench.algorithmic_bytes(synth.WORKLOADS["decode_128k"])
+    assert scan == 268_435_456 and gathered == 8_388_608
+
+
+def test_kernels_per_step(monkeypatch):
+    monkeypatch.delenv("SPARSE_DECODE_FUSED_ROUTE", raising=False)
+    w = synth.WORKLOADS["decode_128k"]
+    assert bench.kernels_per_step(w) == 3                     # scan, select, attention
+    assert bench.kernels_per_step(w, reroute=1) == 3 * w.L     # per-layer routing
+    assert bench.kernels_per_step(w, reroute=5) == 3 * 4       # ceil(16 / 5) groups
+    assert bench.kernels_per_step(synth.WORKLOADS["tiny_f32"]) == 4  # fp32: partial + merge
+    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "1")
+    assert bench.kernels_per_step(w) == 2
+
+
+def test_peak_denominator_is_the_measured_copy_bandwidth():
+    gbs, src = bench.load_peaks()
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            assert gbs == pytest.approx(float(json.load(f)["hbm_gbs"]))
+        assert src.startswith("measured")
+    else:
+        assert gbs == bench.FALLBACK_HBM_GBS and src.startswith("fallback")
