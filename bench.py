@@ -128,22 +128,30 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
             return None
-        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) == len(_SMI_FIELDS)]
-        try:
-            if self.t0 is not None and self.t1 is not None:
-                rows = [r for r in rows if self.t0 - 0.05 <= _smi_time(r[0]) <= self.t1 + 0.05]
-        except Exception:
-            pass
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4)
-                          if r[5 + i].strip().lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+        return summarize_clocks(out, self.t0, self.t1)
+
+
+def summarize_clocks(out: str, t0=None, t1=None):
+    """The clocks record of one timed region from nvidia-smi's CSV rows
+    (_SMI_FIELDS, no header, no units): the median SM clock, the largest max
+    clock and every throttle reason seen Active, over the rows stamped inside
+    [t0, t1] (with 50 ms of slack); None when no row qualifies."""
+    rows = [r for r in csv.reader(io.StringIO(out)) if len(r) == len(_SMI_FIELDS)]
+    try:
+        if t0 is not None and t1 is not None:
+            rows = [r for r in rows if t0 - 0.05 <= _smi_time(r[0]) <= t1 + 0.05]
+    except Exception:
+        pass
+    if not rows:
+        return None
+    sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+    mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in rows for i in range(4)
+                      if r[5 + i].strip().lower() == "active"})
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+            "samples": len(rows)}
 
 
 # ---------------------------------------------------------------------------

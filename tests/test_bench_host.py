@@ -87,3 +87,28 @@ def test_peak_denominator_is_the_measured_copy_bandwidth():
         assert src.startswith("measured")
     else:
         assert gbs == bench.FALLBACK_HBM_GBS and src.startswith("fallback")
+
+
+def _smi_row(t, sm, mx=1965, hw="Not Active", thermal="Not Active", cap="Not Active"):
+    from datetime import datetime
+    stamp = datetime.fromtimestamp(t).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+    return f"{stamp}, {sm}, {mx}, 700.5, 0x0000000000000000, {hw}, {thermal}, Not Active, {cap}"
+
+
+def test_clock_summary_of_the_timed_region():
+    """Only rows stamped inside the timed region count; the SM clock is their
+    median, the max clock the largest seen, and a reason is reported when any
+    row shows it Active."""
+    t0 = 1_700_000_000.0
+    rows = [_smi_row(t0 - 1.0, 345, cap="Active"),          # before the region
+            _smi_row(t0 + 0.1, 1965),
+            _smi_row(t0 + 0.2, 1900, cap="Active"),
+            _smi_row(t0 + 0.3, 1950),
+            _smi_row(t0 + 2.0, 210, hw="Active")]           # after it
+    c = bench.summarize_clocks("\n".join(rows), t0, t0 + 0.5)
+    assert c == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                 "samples": 3}
+    c = bench.summarize_clocks("\n".join(rows))              # no region: every row
+    assert c["samples"] == 5 and c["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    assert bench.summarize_clocks("", t0, t0 + 1) is None
+    assert bench.summarize_clocks("garbage,row\n", t0, t0 + 1) is None
