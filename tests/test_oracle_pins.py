@@ -17,6 +17,7 @@ import numpy as np
 import pytest
 import scipy.special
 import torch
+import torch.nn.attention
 
 import oracle
 
@@ -241,7 +242,7 @@ def test_percentile_tau_matches_numpy_inverted_cdf():
 # --------------------------------------------------------------------------
 
 def _sdpa_f64(q, K, V):
-    """torch scaled_dot_product_attention in fp64 with GQA repetition.
+    """torch scaled_dot_product_attention (math backend) in fp64 with GQA repetition.
     q [B,Hq,d] (one query per head), K,V [B,Hkv,n,d]."""
     qt = torch.from_numpy(q.astype(np.float64))[:, :, None, :]
     Kt = torch.from_numpy(K.astype(np.float64))
@@ -249,7 +250,9 @@ def _sdpa_f64(q, K, V):
     G = q.shape[1] // K.shape[1]
     Kt = Kt.repeat_interleave(G, dim=1)
     Vt = Vt.repeat_interleave(G, dim=1)
-    o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt)
+    # the plain math backend: one fixed evaluation order, whatever the thread pool
+    with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.MATH):
+        o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt)
     logits = (qt @ Kt.transpose(-1, -2))[:, :, 0, :] / math.sqrt(q.shape[-1])
     return o[:, :, 0, :].numpy(), torch.logsumexp(logits, dim=-1).numpy()
 
