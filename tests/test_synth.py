@@ -56,3 +56,31 @@ def test_named_workloads_shapes():
     assert t.mode == "threshold" and t.cap == 8192 and t.stride == 8192
     bt = synth.WORKLOADS["batched_16x64k"]
     assert bt.seeds == tuple(range(1, 17))
+
+
+def test_clustered_keys_recipe():
+    """blobs > 0: every key of a head is its centre (one of `blobs`, drawn
+    2 * N(0,1)) plus blob_spread * N(0,1) noise, so keys lie close to their
+    nearest centre, far from the others, with about blob_spread per axis."""
+    w = synth.custom(B=1, N=2000, Hq=8, Hkv=2, d=64, L=1, dtype="f32", seed=3,
+                     mode="threshold", cap=64, blobs=6, blob_spread=0.1)
+    x = synth.generate(w)
+    K = synth.f32(x["K"])[0].astype(np.float64)               # [Hkv, N, d]
+    for h in range(2):
+        X = K[h]
+        # recover the centres: centres sit ~2*sqrt(2d) ~ 23 apart and keys
+        # within ~0.1*sqrt(d) ~ 0.8 of theirs, so farthest-point picks give
+        # one key per blob and one nearest-pick pass gives the groups
+        pick = [0]
+        for _ in range(5):
+            dmin = np.min(((X[:, None, :] - X[pick][None]) ** 2).sum(-1), axis=1)
+            pick.append(int(np.argmax(dmin)))
+        lab = np.argmin(((X[:, None, :] - X[pick][None]) ** 2).sum(-1), axis=1)
+        cent = np.stack([X[lab == c].mean(0) for c in range(6)])
+        resid = X - cent[lab]
+        assert 0.08 < resid.std() < 0.12                     # blob_spread per axis
+        assert np.sqrt((resid ** 2).sum(1)).max() < 0.1 * 8 + 0.5
+    lw = synth.WORKLOADS["louver_128k"]
+    assert (lw.N, lw.Hq, lw.Hkv, lw.d, lw.L, lw.cap, lw.blobs) == (131072, 32, 8, 128, 16,
+                                                                  8192, 64)
+    assert lw.mode == "threshold" and lw.blob_spread == 0.1
