@@ -44,6 +44,13 @@ METRIC = ("128K-context sparse decode steps/s (16 layers, k=2048); "
           "HBM GB/s vs roofline")
 FALLBACK_HBM_GBS = 6650.0
 QUERY_SETS = 8
+TIMING = ("the K timed decode steps replayed back to back as one CUDA graph (query set "
+          "i %% 8 at step i; %d kernels per step, programmatic dependent launch between "
+          "them; for K > 256 a 64-step graph replayed plus a remainder graph), after the W "
+          "warm-up steps; CUDA events on the launch stream; max over ranks")
+TIMING_OTHER = ("the K timed steps replayed back to back as one CUDA graph (query set i %% 8 at "
+                "step i; for K > 256 a 64-step graph replayed plus a remainder graph), after the "
+                "W warm-up steps; CUDA events on the launch stream; max over ranks") % ()
 
 
 def load_peaks():
@@ -183,22 +190,31 @@ def time_graphs(graphs, steps: int, warmup: int, stream, sampler=None) -> float:
     return start.elapsed_time(end)
 
 
-def time_steps(g_loop, g_one, steps: int, warmup: int, stream, sampler=None) -> float:
-    """Run warmup + steps decode steps: whole replays of g_loop (one graph of
-    len(g_one) consecutive steps, query set i at step i) and single-step
-    graphs g_one[i] for the remainder; return the CUDA-event time (ms) of the
-    last `steps` steps, bracketed by a barrier and device synchronisation."""
-    n = len(g_one)
+def step_graphs(step_fns, count: int, stream, max_one: int = 256, chunk: int = 64):
+    """CUDA graphs that together run `count` consecutive decode steps
+    (step_fns[i % n] at step i): [(graph, replays)].  One graph of all the
+    steps when count <= max_one, else a chunk-step graph replayed and one
+    graph for the remainder (n must divide chunk so the cycle lines up)."""
+    n = len(step_fns)
+    if count <= max_one:
+        return [(capture_loop([step_fns[i % n] for i in range(count)], stream), 1)]
+    assert chunk % n == 0
+    plan = [(capture_loop([step_fns[i % n] for i in range(chunk)], stream), count // chunk)]
+    if count % chunk:
+        plan.append((capture_loop([step_fns[i % n] for i in range(count % chunk)], stream), 1))
+    return plan
 
-    def run(count):
-        done = 0
-        while count - done >= n:
-            g_loop.replay()
-            done += n
-        for i in range(count - done):
-            g_one[i].replay()
 
-    run(warmup)
+def time_steps(step_fns, steps: int, warmup: int, stream, sampler=None) -> float:
+    """Run warmup + steps decode steps, each phase as whole CUDA graph
+    replays (step_graphs: the timed steps back to back in one graph when
+    there are at most 256 of them); return the CUDA-event time (ms) of the
+    `steps` timed steps, bracketed by a barrier and device synchronisation."""
+    warm = step_graphs(step_fns, warmup, stream)
+    timed = step_graphs(step_fns, steps, stream)
+    for g, reps in warm:
+        for _ in range(reps):
+            g.replay()
     torch.cuda.synchronize()
     sdist.barrier()
     torch.cuda.synchronize()
@@ -207,7 +223,9 @@ def time_steps(g_loop, g_one, steps: int, warmup: int, stream, sampler=None) -> 
     if sampler:
         sampler.mark_start()
     start.record(stream)
-    run(steps)
+    for g, reps in timed:
+        for _ in range(reps):
+            g.replay()
     end.record(stream)
     torch.cuda.synchronize()
     if sampler:
@@ -255,14 +273,19 @@ def capture_loop(fn_list, stream):
 
 
 def kernels_per_step(w, reroute: int = 0) -> int:
-    """Kernels one decode step launches: the routing scan and the select (one
-    fused kernel when SPARSE_DECODE_FUSED_ROUTE=1 applies), then the
-    attention (one kernel for bf16, a partial and a merge kernel for fp32);
-    once per group of `reroute` layers when routing is re-computed."""
-    route = 1 if os.environ.get("SPARSE_DECODE_FUSED_ROUTE") == "1" and w.mode == "topk" else 2
-    attn = 1 if w.dtype == "bf16" else 2
+    """Kernels one decode step launches: the routing scan, then -- for bf16
+    steps whose shape lets the attention kernel finish the routing (L*G <=
+    128 query vectors per head, N <= 131072, k or cap <= 16384) -- that one
+    kernel, else the select (or threshold compaction) and the attention (one
+    kernel for bf16, a partial and a merge kernel for fp32); once per group of
+    `reroute` layers when routing is re-computed."""
+    lg = min(reroute, w.L) if reroute else w.L
+    stride = w.k if w.mode == "topk" else w.cap
+    fused = (w.dtype == "bf16" and lg * (w.Hq // w.Hkv) <= 128 and w.N <= 131072
+             and stride <= 16384)
+    per_group = 2 if fused else 2 + (1 if w.dtype == "bf16" else 2)
     groups = -(-w.L // reroute) if reroute else 1
-    return (route + attn) * groups
+    return per_group * groups
 
 
 def capture(fn_list, stream):
@@ -346,10 +369,10 @@ def run_native(args, rank, world, local_rank):
         for i in range(len(qs)):          # warm the workspace and the library
             step_fn(i)()
         sd.read_device_status(ws)
-        graphs = capture([step_fn(i) for i in range(len(qs))], stream)
         loop = capture_loop([step_fn(i) for i in range(len(qs))], stream)
         with ClockSampler(local_rank) as cs:
-            ms = time_steps(loop, graphs, args.steps, args.warmup, stream, cs)
+            ms = time_steps([step_fn(i) for i in range(len(qs))], args.steps, args.warmup,
+                            stream, cs)
         clocks = cs.result()
         dist = step_distribution(loop, len(qs), stream)
         sd.read_device_status(ws)         # no device-side condition in the run
@@ -449,11 +472,7 @@ def run_native(args, rank, world, local_rank):
             "l2": "inputs larger than L2 (K+V = %.0f MB per replica); the query "
                   "rotates over %d sets so the selected rows change every step"
                   % (2 * scan_b / 1e6, QUERY_SETS),
-            "timing": "decode steps replayed as CUDA graphs of %d consecutive steps "
-                      "(query set i at step i; %d kernels per step, programmatic "
-                      "dependent launch between them), single-step graphs for a "
-                      "remainder; CUDA events on the launch stream; max over ranks"
-                      % (QUERY_SETS, kernels_per_step(w, args.reroute)),
+            "timing": TIMING % kernels_per_step(w, args.reroute),
             **({"reroute": args.reroute,
                 "routing": "re-computed every %d layers (group g routes with its first "
                            "layer's query)" % args.reroute} if args.reroute else {}),
@@ -472,11 +491,16 @@ def run_native(args, rank, world, local_rank):
             "achieved_gbs": round((scan_b + gath_b) / (ms_per_step * 1e-3) / 1e9, 1),
             "frac_of_measured_peak": round((scan_b + gath_b) / (ms_per_step * 1e-3) / 1e9 / peak, 4),
         },
-        "kernels_us": {"score": round(t_score * 1e3, 2), "select": round(t_sel * 1e3, 2),
+        "kernels_us": {"score": round(t_score * 1e3, 2),
+                       "select_and_attention_in_step": round(ms_per_step * 1e3 - t_score * 1e3, 2),
+                       "select_kernel": round(t_sel * 1e3, 2),
                        "attn_gather_all_layers": round(t_attn * 1e3, 2),
-                       "note": "score and attention timed alone in back-to-back graph "
-                               "launches (attention alone may find its rows in L2); select "
-                               "= route (score + select) minus score"},
+                       "note": "score (the routing scan) and attn_gather (attention over given "
+                               "sets) timed alone in back-to-back graph launches (attention "
+                               "alone may find its rows in L2); in the step the select runs "
+                               "inside the attention kernel, whose share is the step time minus "
+                               "the scan; select_kernel = route_topk (scan + the select as its "
+                               "own kernel) minus the scan"},
         **({"dense_attention": dense} if dense else {}),
         "e2e": e2e,
         "gpu_launches": kernels_per_step(w, args.reroute) * args.steps,
@@ -707,10 +731,10 @@ def run_native_louver(args, rank, world, local_rank):
             full_fn(i)()
         sd.read_device_status(ws)
         sd.read_device_status(ix.ws)
-        graphs = capture([step_fn(i) for i in range(len(qs))], stream)
         loop = capture_loop([step_fn(i) for i in range(len(qs))], stream)
         with ClockSampler(local_rank) as cs:
-            ms = time_steps(loop, graphs, args.steps, args.warmup, stream, cs)
+            ms = time_steps([step_fn(i) for i in range(len(qs))], args.steps, args.warmup,
+                            stream, cs)
         clocks = cs.result()
         dist = step_distribution(loop, len(qs), stream)
         sd.read_device_status(ws)
@@ -721,9 +745,7 @@ def run_native_louver(args, rank, world, local_rank):
                               stream) / n_k
         t_attn = time_graphs(capture([attn_fn(i) for i in range(len(qs))], stream), n_k, wk,
                              stream) / n_k
-        full_one = capture([full_fn(i) for i in range(len(qs))], stream)
-        full_loop = capture_loop([full_fn(i) for i in range(len(qs))], stream)
-        ms_full = time_steps(full_loop, full_one, n_k, wk, stream) / n_k
+        ms_full = time_steps([full_fn(i) for i in range(len(qs))], n_k, wk, stream) / n_k
         full_route = capture([lambda i=i: sd.route_threshold(qs[i][0], K, taus[i], cap, ws=ws,
                                                              check=False)
                               for i in range(len(qs))], stream)
@@ -769,8 +791,7 @@ def run_native_louver(args, rank, world, local_rank):
             "l2": "inputs larger than L2 (K+V = %.0f MB, index keys %.0f MB per replica); the "
                   "query rotates over %d sets" % (2 * BH * w.N * w.d * w.esize / 1e6,
                                                     BH * w.N * w.d * w.esize / 1e6, QUERY_SETS),
-            "timing": "steps replayed as CUDA graphs of %d consecutive steps; CUDA events on "
-                      "the launch stream; max over ranks" % QUERY_SETS,
+            "timing": TIMING_OTHER,
             "index_build_ms": round(build_ms, 3),
             "surviving_clusters_per_query": round(mean_surv, 1),
             "surviving_leaves_per_query": round(mean_leaves, 1),
@@ -856,10 +877,10 @@ def run_native_threshold(args, rank, world, local_rank):
             step_fn(i)()
             counts.append(outs[i]["count"].cpu())
         sd.read_device_status(ws)
-        graphs = capture([step_fn(i) for i in range(len(qs))], stream)
         loop = capture_loop([step_fn(i) for i in range(len(qs))], stream)
         with ClockSampler(local_rank) as cs:
-            ms = time_steps(loop, graphs, args.steps, args.warmup, stream, cs)
+            ms = time_steps([step_fn(i) for i in range(len(qs))], args.steps, args.warmup,
+                            stream, cs)
         clocks = cs.result()
         dist = step_distribution(loop, len(qs), stream)
         sd.read_device_status(ws)
@@ -900,8 +921,7 @@ def run_native_threshold(args, rank, world, local_rank):
             "parallelism": f"replicas x{world}", "query_sets": QUERY_SETS,
             "l2": "inputs larger than L2 (K+V = %.0f MB per replica); the query rotates over "
                   "%d sets" % (2 * scan_b / 1e6, QUERY_SETS),
-            "timing": "steps replayed as CUDA graphs of %d consecutive steps; CUDA events on "
-                      "the launch stream; max over ranks" % QUERY_SETS,
+            "timing": TIMING_OTHER,
             "mean_set_size_per_query": round(mean_count, 1),
         },
         "roofline": {

@@ -67,15 +67,15 @@ def test_algorithmic_bytes_of_the_headline_step():
     assert scan == 268_435_456 and gathered == 8_388_608
 
 
-def test_kernels_per_step(monkeypatch):
-    monkeypatch.delenv("SPARSE_DECODE_FUSED_ROUTE", raising=False)
+def test_kernels_per_step():
     w = synth.WORKLOADS["decode_128k"]
-    assert bench.kernels_per_step(w) == 3                     # scan, select, attention
-    assert bench.kernels_per_step(w, reroute=1) == 3 * w.L     # per-layer routing
-    assert bench.kernels_per_step(w, reroute=5) == 3 * 4       # ceil(16 / 5) groups
-    assert bench.kernels_per_step(synth.WORKLOADS["tiny_f32"]) == 4  # fp32: partial + merge
-    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "1")
-    assert bench.kernels_per_step(w) == 2
+    assert bench.kernels_per_step(w) == 2                     # scan, select + attention
+    assert bench.kernels_per_step(w, reroute=1) == 2 * w.L     # per-layer routing
+    assert bench.kernels_per_step(w, reroute=5) == 2 * 4       # ceil(16 / 5) groups
+    assert bench.kernels_per_step(synth.WORKLOADS["tiny_f32"]) == 4  # fp32: select, partial, merge
+    assert bench.kernels_per_step(synth.WORKLOADS["threshold_128k"]) == 2
+    big = w.with_(N=262144)
+    assert bench.kernels_per_step(big) == 3                   # select as a kernel of its own
 
 
 def test_peak_denominator_is_the_measured_copy_bandwidth():

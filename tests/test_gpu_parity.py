@@ -236,13 +236,31 @@ def test_attn_gather_bad_index_flags_without_fault(dev):
 # Routing end to end and the fused step
 # ---------------------------------------------------------------------------
 
-@pytest.fixture(params=["fused", "scan_then_select"])
-def route_path(request, monkeypatch):
-    """Routing runs as one fused scan+select kernel when the shape allows it,
-    else as the scan kernel followed by the select kernel; every routing test
-    runs both ways."""
-    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "1" if request.param == "fused" else "0")
+@pytest.fixture(params=["select_kernel", "fused_step"])
+def route_path(request):
+    """Top-k routing ends in the select kernel (sparse_route_topk) or, in a
+    decode step, inside the attention kernel; every routing test runs both
+    ways and reads the index set either call returns."""
     return request.param
+
+
+def _route(path, t, K, k, ws=None, L=1):
+    """The top-k set of routing with t["q_route"] over K, by `path` (the
+    device status is left for the caller to read)."""
+    if path == "select_kernel":
+        return sd.route_topk(t["q_route"], K, k, ws=ws, check=False)
+    res = sd.decode_step(t["q_route"], t["q_layers"][:L], K, torch.zeros_like(K), k=k, ws=ws,
+                         check=False)
+    return res["idx"]
+
+
+def _sample_tiles(N, d=128, esize=2, want=32):
+    """Key ranges [j0, j1) of the routing scan's sample tiles of a head (tile
+    u of a head is sampled when u % stride == 0)."""
+    per = 32768 // (d * esize)
+    tph = -(-N // per)
+    stride = max(1, tph // want)
+    return [(u * per, min(N, (u + 1) * per)) for u in range(0, tph, stride)]
 
 
 ROUTE_CASES = [
@@ -258,10 +276,10 @@ def test_route_topk_matches_oracle(dev, c, route_path):
     w = synth.custom(L=1, seed=c["N"], **c)
     x = synth.generate(w)
     t = _to(dev, x)
-    gidx = sd.route_topk(t["q_route"], t["K"], w.k).cpu().numpy()
+    gidx = _route(route_path, t, t["K"], w.k).cpu().numpy()
     S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
     assert_topk_within_band(gidx, S, w.k)
-    again = sd.route_topk(t["q_route"], t["K"], w.k).cpu().numpy()
+    again = _route(route_path, t, t["K"], w.k).cpu().numpy()
     np.testing.assert_array_equal(gidx, again)   # deterministic
 
 
@@ -299,16 +317,19 @@ def _check_decode(dev, w, x, batches_checked=None):
 
 
 @pytest.mark.parametrize("name", ["tiny_f32", "decode_32k", "decode_128k"])
-def test_decode_step_named_workloads(dev, name, route_path):
+def test_decode_step_named_workloads(dev, name):
     w = synth.WORKLOADS[name]
     x = synth.generate(w)
     _check_decode(dev, w, x)
 
 
-def test_decode_step_batched_16x64k_sampled(dev):
+def test_decode_step_batched_16x64k(dev):
+    """The batched workload, every one of its 16 sequences checked: index
+    sets within the band of the oracle's, the step's set equal to the routing
+    call's, and attention on the oracle's sets within tolerance."""
     w = synth.WORKLOADS["batched_16x64k"]
     x = synth.generate(w)
-    _check_decode(dev, w, x, batches_checked=[0, 7, 15])
+    _check_decode(dev, w, x)
 
 
 @pytest.mark.parametrize("name,cap", [("threshold_128k", 8192), ("threshold_128k", 2000)])
@@ -362,25 +383,32 @@ def test_route_topk_all_equal_keys_takes_lowest_indices(dev, route_path):
     t = _to(dev, x)
     K = t["K"].clone()
     K[:] = K[:, :, :1, :]
-    idx = sd.route_topk(t["q_route"], K, 300).cpu().numpy()
+    idx = _route(route_path, t, K, 300).cpu().numpy()
     np.testing.assert_array_equal(idx, np.tile(np.arange(300), (1, 2, 1)))
 
 
 def test_route_topk_recovers_from_dirty_workspace(dev, route_path):
-    """A workspace whose histogram area holds garbage (not zero-filled) is
-    detected (the counts do not sum to N) and the result is still exact; the
-    call leaves the workspace clean for the next one."""
+    """A workspace whose histogram and sample areas hold garbage (not
+    zero-filled) is detected (the counts do not sum to N; the candidate lists
+    come out short) and the result is still exact; the call leaves those
+    areas clean for the next one."""
     w = synth.custom(B=2, N=5000, Hq=8, Hkv=2, d=128, L=1, k=100, dtype="bf16", seed=6)
     x = synth.generate(w)
     t = _to(dev, x)
     S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
     ws = sd.Workspace(dev)
     ws.get(sd.workspace_bytes(2, 5000, 8, 2, 128, torch.bfloat16, 100, 1))
-    ws.buf[4096:4096 + 4 * 2048 * 4] = 7  # the histogram area (after the 4 KB header)
+    # header 4 KB | histogram [256][2048] | sample histogram [256][2048] | sample counts
+    hist, smp = 4096, 4096 + 256 * 2048 * 4
+    cnt = smp + 256 * 2048 * 4
+    areas = [(hist, hist + 4 * 2048 * 4), (smp, smp + 4 * 2048 * 4), (cnt, cnt + 4 * 4)]
+    for a, b in areas:
+        ws.buf[a:b] = 7
     for _ in range(2):
-        gidx = sd.route_topk(t["q_route"], t["K"], 100, ws=ws).cpu().numpy()
+        gidx = _route(route_path, t, t["K"], 100, ws=ws).cpu().numpy()
         assert_topk_within_band(gidx, S, 100)
-    assert int(ws.buf[4096:4096 + 4 * 2048 * 4].sum()) == 0
+    for a, b in areas:
+        assert int(ws.buf[a:b].sum()) == 0
 
 
 @pytest.mark.parametrize("k,count", [(4096, None), (8192, [3933, 4100, 100, 0, 8192, 2, 3000, 7000])])
@@ -413,46 +441,11 @@ def test_dense_attention_all_keys(dev, dtype, N):
     assert_attn_close(out, lse, o_ref, l_ref, dtype)
 
 
-@pytest.mark.parametrize("B,Hkv,N,k", [(1, 8, 8192, 2048), (2, 8, 6000, 1024),
-                                       (1, 2, 5000, 300), (3, 1, 4000, 700)])
-def test_attention_cluster_merge_equals_global_merge(dev, monkeypatch, B, Hkv, N, k):
-    """The split-k merge inside a thread-block cluster (partials read through
-    distributed shared memory) and the merge through global memory combine
-    the same partials in the same order: bit-identical outputs, both within
-    tolerance of the oracle."""
-    w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=16, k=k, dtype="bf16", seed=31)
-    x = synth.generate(w)
-    t = _to(dev, x)
-    idx = oracle.topk(oracle.scores(_f(x["q_route"]), _f(x["K"])), w.k)
-    idx_t = torch.from_numpy(idx).to(dev)
-    monkeypatch.setenv("SPARSE_DECODE_ATTN_MERGE", "global")
-    o_g, l_g = sd.attn_gather(t["q_layers"], t["K"], t["V"], idx_t)
-    monkeypatch.delenv("SPARSE_DECODE_ATTN_MERGE")
-    o_c, l_c = sd.attn_gather(t["q_layers"], t["K"], t["V"], idx_t)
-    assert torch.equal(o_g, o_c)
-    assert torch.equal(l_g, l_c)
-    o_ref, l_ref = oracle.attn(_f(x["q_layers"]), _f(x["K"]), _f(x["V"]), idx)
-    assert_attn_close(o_c, l_c, o_ref, l_ref, "bf16")
-
-
-def test_attn_gather_mma_sync_variant_matches(dev, monkeypatch):
-    """The warp-level mma.sync kernel (kept for comparison) agrees too."""
-    monkeypatch.setenv("SPARSE_DECODE_ATTN", "mma")
-    w = synth.custom(B=2, N=3000, Hq=32, Hkv=8, d=128, L=16, k=2048, dtype="bf16", seed=77)
-    x = synth.generate(w)
-    t = _to(dev, x)
-    S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
-    idx = oracle.topk(S, w.k)
-    out, lse = sd.attn_gather(t["q_layers"], t["K"], t["V"], torch.from_numpy(idx).to(dev))
-    o_ref, l_ref = oracle.attn(_f(x["q_layers"]), _f(x["K"]), _f(x["V"]), idx)
-    assert_attn_close(out, lse, o_ref, l_ref, "bf16")
-
-
 @pytest.mark.parametrize("kind", ["random", "duplicated_rows", "few_values", "heavy"])
 def test_route_topk_bit_exact_on_its_own_scores(dev, kind, route_path):
-    """Routing (scan + histogram fast-path select) against the oracle's top-k
-    of the very scores the scan produced: identical fp32 scores, so the index
-    sets must be identical, ties included."""
+    """Routing (scan + exact select) against the oracle's top-k of the very
+    scores the scan produced: identical fp32 scores, so the index sets must
+    be identical, ties included."""
     w = synth.custom(B=2, N=40000, Hq=32, Hkv=8, d=128, L=1, k=2048, dtype="bf16",
                      heavy=64 if kind == "heavy" else 0, seed=17)
     x = synth.generate(w)
@@ -466,49 +459,71 @@ def test_route_topk_bit_exact_on_its_own_scores(dev, kind, route_path):
         K = torch.randint(-2, 3, K.shape, device=dev).to(K.dtype)
     ws = sd.Workspace(dev)
     S = sd.score(t["q_route"], K, ws=ws).cpu().numpy()
-    idx = sd.route_topk(t["q_route"], K, w.k, ws=ws).cpu().numpy()
+    idx = _route(route_path, t, K, w.k, ws=ws).cpu().numpy()
     np.testing.assert_array_equal(idx, oracle.topk(S, w.k))
 
 
 @pytest.mark.parametrize("B,N,Hkv,k", [(1, 131072, 8, 2048), (3, 20000, 2, 1), (4, 8192, 4, 8000),
-                                       (1, 65536, 1, 700), (2, 2048, 8, 64)])
-def test_fused_route_equals_scan_then_select(dev, monkeypatch, B, N, Hkv, k):
-    """The fused scan+select kernel and the two-kernel path give the same
-    index sets, bit for bit (same scan arithmetic, exact selection), over
-    shapes where CTAs span two heads, a head spans one CTA or many, k = 1 and
-    k close to N."""
+                                       (1, 65536, 1, 700), (2, 2048, 8, 64),
+                                       (16, 65536, 8, 2048), (1, 262144, 2, 2048)])
+def test_fused_select_equals_select_kernel(dev, B, N, Hkv, k):
+    """The select inside the attention kernel (decode step) and the select
+    kernel (routing call) give the same index sets, bit for bit, over shapes
+    where scan CTAs span two heads, a head spans one CTA or many, k = 1, k
+    close to N, the batched decode shape, and a cache too long for the fused
+    select (the step then runs the select kernel itself)."""
     w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=1, k=k, dtype="bf16", seed=N + k)
     x = synth.generate(w)
     t = _to(dev, x)
-    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "1")
-    a = sd.route_topk(t["q_route"], t["K"], k).cpu().numpy()
-    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "0")
-    b = sd.route_topk(t["q_route"], t["K"], k).cpu().numpy()
+    ws = sd.Workspace(dev)
+    a = _route("fused_step", t, t["K"], k, ws=ws).cpu().numpy()
+    assert sd.read_device_flags(ws) & ~sd.FLAG_SLOW_SELECT == 0
+    b = _route("select_kernel", t, t["K"], k, ws=ws).cpu().numpy()
     np.testing.assert_array_equal(a, b)
     S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
     assert_topk_within_band(a, S, k)
 
 
-@pytest.mark.parametrize("B,N,Hkv,hot", [(1, 65536, 1, 4096), (2, 131072, 2, 20000)])
-def test_fused_route_concentrated_top_k(dev, monkeypatch, B, N, Hkv, hot):
-    """Most of the top k lies in the first `hot` keys of each head, far more
-    than any CTA's proportional share: the fused kernel's local threshold
-    estimate is too high there and its second (histogram) round must give
-    the same exact sets as the two-kernel path."""
+@pytest.mark.parametrize("route", ["select_kernel", "fused_step"])
+@pytest.mark.parametrize("B,N,Hkv", [(1, 131072, 8), (2, 65536, 4)])
+def test_select_when_the_sample_misleads(dev, route, B, N, Hkv):
+    """The routing scan estimates each head's candidate bound from its sample
+    tiles.  Here the sample tiles hold scaled-up keys, so the bound lands
+    above the k-th score and the candidate lists miss keys of the top k: the
+    select must notice (its count check), take the exact streaming path
+    (flagged FLAG_SLOW_SELECT, not an error) and still return the exact set."""
     k = 2048
-    w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=1, k=k, dtype="bf16", seed=hot)
+    w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=1, k=k, dtype="bf16", seed=N + 3)
     x = synth.generate(w)
     t = _to(dev, x)
     K = t["K"].clone()
-    K[:, :, :hot] *= 4
-    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "1")
-    a = sd.route_topk(t["q_route"], K, k).cpu().numpy()
-    monkeypatch.setenv("SPARSE_DECODE_FUSED_ROUTE", "0")
-    b = sd.route_topk(t["q_route"], K, k).cpu().numpy()
-    np.testing.assert_array_equal(a, b)
-    S = oracle.scores(_f(x["q_route"]), _f(K.cpu()))
-    assert_topk_within_band(a, S, k)
-    assert (a < hot).mean() > 0.3   # far above the hot keys' proportional share
+    for j0, j1 in _sample_tiles(N):
+        K[:, :, j0:j1] *= 3
+    ws = sd.Workspace(dev)
+    S = sd.score(t["q_route"], K, ws=ws).cpu().numpy()
+    sd.read_device_flags(ws)
+    a = _route(route, t, K, k, ws=ws).cpu().numpy()
+    flags = sd.read_device_flags(ws)
+    assert flags == sd.FLAG_SLOW_SELECT
+    np.testing.assert_array_equal(a, oracle.topk(S, k))
+    # the next call on the same workspace (state cleared) takes the fast path
+    b = _route(route, t, t["K"], k, ws=ws).cpu().numpy()
+    assert sd.read_device_flags(ws) == 0
+    S2 = oracle.scores(_f(x["q_route"]), _f(x["K"]))
+    assert_topk_within_band(b, S2, k)
+
+
+@pytest.mark.parametrize("route", ["select_kernel", "fused_step"])
+def test_select_fast_path_on_the_decode_workloads(dev, route):
+    """On the decode workloads' distributions the sample bound holds: no head
+    falls back to the streaming select."""
+    for name in ("decode_32k", "decode_128k"):
+        w = synth.WORKLOADS[name]
+        x = synth.generate(w)
+        t = _to(dev, x)
+        ws = sd.Workspace(dev)
+        _route(route, t, t["K"], w.k, ws=ws, L=w.L)
+        assert sd.read_device_flags(ws) == 0, name
 
 
 # ---------------------------------------------------------------------------
@@ -666,9 +681,8 @@ def test_decode_step_graph_survives_workspace_growth(dev):
     ws = sd.Workspace(dev)
     g = sd.DecodeStepGraph(K, V, w.L, w.Hq, k=w.k, ws=ws)
     before = ws.buf.data_ptr()
-    big = torch.randn(64, 1, w.Hq, w.d, generator=torch.Generator().manual_seed(3)).to(
-        torch.bfloat16).to(dev)
-    sd.decode_step(x["q_route"].to(dev), big, K, V, k=3000, ws=ws)   # grows ws
+    long_k = torch.zeros((1, w.Hkv, 400_000, w.d), dtype=torch.bfloat16, device=dev)
+    sd.score(x["q_route"].to(dev), long_k, ws=ws)   # a longer cache: grows ws
     assert ws.buf.data_ptr() != before
     g.q_route_host.copy_(x["q_route"])
     g.q_layers_host.copy_(x["q_layers"])

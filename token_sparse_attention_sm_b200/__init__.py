@@ -29,7 +29,7 @@ __all__ = ["SparseDecodeError", "lib_path", "load", "score", "select_topk",
            "Workspace", "STATUS_NAMES", "EXPORTED_SYMBOLS", "decode_step_grouped",
            "kv_append", "LouverIndex", "louver_build", "louver_route_threshold",
            "DecodeStepGraph", "selftest_bounded_wait", "louver_decode_step",
-           "device_usable"]
+           "device_usable", "read_device_flags", "FLAG_SLOW_SELECT"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_FILE = os.path.join(_PKG, "libsparse_decode.so")
@@ -248,6 +248,19 @@ def _ws(ws: Workspace | None, device) -> Workspace:
     if key not in _default_ws:
         _default_ws[key] = Workspace(device)
     return _default_ws[key]
+
+
+FLAG_SLOW_SELECT = 1 << 8  # informational: a top-k select took its exact streaming path
+
+
+def read_device_flags(ws: Workspace) -> int:
+    """Synchronise the current stream, read (and reset) the device status
+    word of ``ws`` and return its raw bits without raising: the error flags
+    (NONFINITE 1, CAPACITY 2, TIMEOUT 4, INDEX 8, INTERNAL 16) and the
+    informational FLAG_SLOW_SELECT."""
+    flags = ctypes.c_uint32(0)
+    load().sparse_read_device_status(_ptr(ws.buf), _stream(), ctypes.byref(flags))
+    return int(flags.value)
 
 
 def read_device_status(ws: Workspace, raise_on_error: bool = True) -> int:

@@ -4,21 +4,24 @@
 // before anything is enqueued; then it enqueues the kernels on the caller's
 // stream and returns.  The library allocates nothing: scratch lives in the
 // caller's workspace, whose layout is
-//   [0, 4096)             header: device status word (uint32) at offset 0;
-//                         offset 64: a word no kernel writes (the bounded
-//                         wait self-test waits on it);
-//                         [256, 1024) attention split-merge counters;
-//                         [1024, 4096) fused-routing barrier counters, one
-//                         per head (fixed, shape-independent areas, zero
-//                         between calls: the kernels reset them)
-//   [4096, ..)            radix histogram [max(B*Hkv, 256)][2048] uint32 (scan ->
-//                         select; cleared after use).  At least 256 rows, so
-//                         that calls of different shapes (up to 256 heads)
-//                         sharing one workspace never put other data there.
-//   [.., ..)              fp32 scores S [B,Hkv,N]; threshold routing keeps
-//                         its per-head bitmaps [B*Hkv][ceil(N/32)] here
-//   [.., ..)              fused routing: published boundary-bin keys
-//   [.., ..)              attention split partials
+//   [0, 4096)      header: device status word (uint32) at offset 0; offset
+//                  64: a word no kernel writes (the bounded-wait self-test
+//                  waits on it)
+//   hist           radix histogram [max(B*Hkv, 256)][2048] uint32 (scan ->
+//                  select; cleared after use)
+//   sample hist    [max(B*Hkv, 256)][2048] uint32 and sample counts
+//                  [max(B*Hkv, 256)] uint32 (the routing scan's sample;
+//                  cleared after use)
+//                  -- these three must be zero between calls; they sit at
+//                  fixed offsets for up to 256 heads, so calls of different
+//                  shapes sharing one workspace never put other data there
+//   cand counts    list lengths [B*Hkv][head_ctas] uint32, then the scan
+//                  CTAs covering each head [max(B*Hkv, 256)] (rewritten by
+//                  every top-k scan; head_ctas: the CTAs a head can span)
+//   cand lists     [B*Hkv][head_ctas][4096] (key, index) pairs
+//   scores         fp32 S [B,Hkv,N]; threshold routing keeps its per-head
+//                  bitmaps [B*Hkv][ceil(N/32)] here
+//   attn           fp32 attention split partials (fp32 inputs only)
 #include <stdlib.h>
 #include <string.h>
 
@@ -40,33 +43,32 @@ cudaError_t g_info_err[kMaxDevices];
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 constexpr size_t kHeader = 4096;
-constexpr size_t kCountersOff = 256;
 constexpr size_t kSelftestOff = 64;  // a header word no kernel writes
-constexpr size_t kRouteCountersOff = 1024;
 constexpr int kHistMinRows = 256;
 
 struct Layout {
-  size_t hist_off, hist_bytes, scores_off, scores_bytes, seg_off, seg_bytes, attn_off,
-      attn_bytes, total;
+  size_t hist_off, smp_off, smp_cnt_off, cnt_off, list_off, scores_off, attn_off, total;
 };
 
 Layout layout(const Shape &s, int stride, int L) {
+  const size_t rows = (size_t)(s.BH() > kHistMinRows ? s.BH() : kHistMinRows);
   Layout l;
   l.hist_off = kHeader;
-  l.hist_bytes = (size_t)(s.BH() > kHistMinRows ? s.BH() : kHistMinRows) * 2048 * sizeof(uint32_t);
-  l.scores_off = l.hist_off + l.hist_bytes;
-  l.scores_bytes = align_up((size_t)s.BH() * s.N * sizeof(float), 256);
-  l.seg_off = l.scores_off + l.scores_bytes;
-  l.seg_bytes = align_up(kFusedSegAreaBytes, 256);
-  l.attn_off = l.seg_off + l.seg_bytes;
-  l.attn_bytes = align_up(attn_workspace_bytes(s, L, stride), 256);
-  l.total = l.attn_off + l.attn_bytes;
+  l.smp_off = l.hist_off + rows * kHistBins * sizeof(uint32_t);
+  l.smp_cnt_off = l.smp_off + rows * kHistBins * sizeof(uint32_t);
+  l.cnt_off = l.smp_cnt_off + align_up(rows * sizeof(uint32_t), 256);
+  l.list_off = l.cnt_off + align_up(cand_count_bytes(s) + rows * 4, 256);
+  l.scores_off = l.list_off + align_up(cand_list_bytes(s), 256);
+  l.attn_off = l.scores_off + align_up((size_t)s.BH() * s.N * sizeof(float), 256);
+  l.total = l.attn_off + align_up(attn_workspace_bytes(s, L, stride), 256);
   return l;
 }
 
 bool aligned(const void *p, size_t a) {
   return (reinterpret_cast<uintptr_t>(p) % a) == 0;
 }
+
+}  // namespace
 
 sparse_status_t check_shape(const sparse_shape_t *shape, Shape *s) {
   if (!shape) return SPARSE_ERR_INVALID_ARG;
@@ -89,6 +91,8 @@ sparse_status_t check_shape(const sparse_shape_t *shape, Shape *s) {
   return SPARSE_OK;
 }
 
+namespace {
+
 sparse_status_t check_ws(const Shape &s, int stride, int L, void *ws,
                          size_t ws_bytes) {
   if (!ws || !aligned(ws, 256)) return SPARSE_ERR_INVALID_ARG;
@@ -101,41 +105,39 @@ sparse_status_t from_cuda(cudaError_t e) {
 }
 
 uint32_t *status_word(void *ws) { return static_cast<uint32_t *>(ws); }
-uint32_t *attn_counters(void *ws) {
-  return reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + kCountersOff);
-}
-static_assert(kCountersOff + 2 * sizeof(uint32_t) * kAttnMaxCounterBlocks <= kRouteCountersOff,
-              "attention counters fit in their area");
-static_assert(kRouteCountersOff + sizeof(uint32_t) * kFusedMaxHeads <= kHeader,
-              "routing counters fit in the header");
-uint32_t *route_counters(void *ws) {
-  return reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + kRouteCountersOff);
-}
-void *seg_ptr(void *ws, const Layout &l) { return static_cast<char *>(ws) + l.seg_off; }
 
-uint32_t *hist_ptr(void *ws, const Layout &l) {
-  return reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + l.hist_off);
+template <typename T>
+T *at(void *ws, size_t off) {
+  return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
 }
-float *scores_ptr(void *ws, const Layout &l) {
-  return reinterpret_cast<float *>(static_cast<char *>(ws) + l.scores_off);
-}
-void *attn_ptr(void *ws, const Layout &l) {
-  return static_cast<char *>(ws) + l.attn_off;
+uint32_t *hist_ptr(void *ws, const Layout &l) { return at<uint32_t>(ws, l.hist_off); }
+float *scores_ptr(void *ws, const Layout &l) { return at<float>(ws, l.scores_off); }
+void *attn_ptr(void *ws, const Layout &l) { return at<char>(ws, l.attn_off); }
+
+// The candidate-list plan of a top-k routing call (false: no lists).
+bool cand_for(const Shape &s, int k, void *ws, const Layout &l, CandArgs *cand) {
+  DeviceInfo di;
+  if (device_info(&di) != cudaSuccess) return false;
+  if (!plan_cand(s, k, di.sm_count, cand)) return false;
+  cand->lists = at<uint64_t>(ws, l.list_off);
+  cand->counts = at<uint32_t>(ws, l.cnt_off);
+  cand->nspan = at<uint32_t>(ws, l.cnt_off + cand_count_bytes(s));
+  cand->smp_hist = at<uint32_t>(ws, l.smp_off);
+  cand->smp_cnt = at<uint32_t>(ws, l.smp_cnt_off);
+  return true;
 }
 
-// A1 + A2 (top-k): the fused kernel when the shape allows it, else the scan
-// followed by the select kernel.
+// A1 + A2 (top-k): the scan (with candidate lists where they apply), then the
+// select kernel.
 cudaError_t route_topk_any(const Shape &s, const void *q, const void *K, int k, int *idx,
                            void *ws, const Layout &l, cudaStream_t st) {
   float *S = scores_ptr(ws, l);
   uint32_t *hist = hist_ptr(ws, l);
-  cudaError_t e = launch_route_topk_fused(s, q, K, k, S, hist, route_counters(ws),
-                                          seg_ptr(ws, l), idx, status_word(ws), st);
-  if (e != cudaErrorNotSupported) return e;
-  cudaGetLastError();
-  e = launch_score(s, q, K, S, hist, status_word(ws), st);
+  CandArgs cand{};
+  const bool lists = cand_for(s, k, ws, l, &cand);
+  cudaError_t e = launch_score(s, q, K, S, hist, lists ? &cand : nullptr, status_word(ws), st);
   if (e == cudaSuccess)
-    e = launch_select(s, S, k, nullptr, 0, idx, nullptr, k, hist, status_word(ws), st);
+    e = launch_select_cand(s, S, k, idx, hist, lists ? &cand : nullptr, status_word(ws), st);
   return e;
 }
 
@@ -152,19 +154,6 @@ cudaError_t route_threshold_any(const Shape &s, const void *q, const void *K, co
 }
 
 }  // namespace
-
-bool cooperative_forced() {
-  static const bool on = [] {
-    const char *v = getenv("SPARSE_DECODE_COOPERATIVE");
-    return v && v[0] == '1';
-  }();
-  return on;
-}
-
-bool attn_cluster_merge_enabled() {
-  const char *v = getenv("SPARSE_DECODE_ATTN_MERGE");  // read per call
-  return !(v && strcmp(v, "global") == 0);
-}
 
 bool pdl_enabled() {
   static const bool on = [] {
@@ -218,7 +207,10 @@ sparse_status_t check_decode_args(const Shape &s, int32_t L, const void *q_route
 }
 
 // Route once with q_route, then attend L layers over that set (arguments
-// checked by the caller; the workspace layout l fits L layers).
+// checked by the caller; the workspace layout l fits L layers).  bf16 steps
+// whose shape allows it finish the routing inside the attention kernel (the
+// scan, then one kernel); the others run the select (or the threshold
+// compaction) as a kernel of its own before the attention.
 cudaError_t decode_step_enqueue(const Shape &s, int L, const void *q_route,
                                 const void *q_layers, const void *K, const void *V, int k,
                                 const float *tau, int cap, int *idx, int *count, void *out,
@@ -226,7 +218,27 @@ cudaError_t decode_step_enqueue(const Shape &s, int L, const void *q_route,
   const bool topk = k > 0;
   const int stride = topk ? k : cap;
   uint32_t *status = status_word(ws);
+  const bool fused = fused_route_ok(s, L, stride);
   cudaError_t e;
+  if (topk && fused) {
+    float *S = scores_ptr(ws, l);
+    uint32_t *hist = hist_ptr(ws, l);
+    CandArgs cand{};
+    const bool lists = cand_for(s, k, ws, l, &cand);
+    e = launch_score(s, q_route, K, S, hist, lists ? &cand : nullptr, status, st);
+    if (e == cudaSuccess)
+      e = launch_route_attn_topk(s, L, q_layers, K, V, k, S, hist, lists ? &cand : nullptr, idx,
+                                 out, lse, status, st);
+    return e;
+  }
+  if (!topk && fused) {
+    uint32_t *bits = reinterpret_cast<uint32_t *>(scores_ptr(ws, l));
+    e = launch_threshold_mark(s, q_route, K, tau, bits, status, st);
+    if (e == cudaSuccess)
+      e = launch_route_attn_threshold(s, L, q_layers, K, V, bits, cap, idx, count, out, lse,
+                                      status, st);
+    return e;
+  }
   if (topk) {
     e = route_topk_any(s, q_route, K, k, idx, ws, l, st);
   } else {
@@ -234,7 +246,7 @@ cudaError_t decode_step_enqueue(const Shape &s, int L, const void *q_route,
   }
   if (e == cudaSuccess)
     e = launch_attn(s, L, q_layers, K, V, idx, stride, topk ? nullptr : count, stride, out,
-                    lse, attn_ptr(ws, l), attn_counters(ws), status, st);
+                    lse, attn_ptr(ws, l), status, st);
   return e;
 }
 
@@ -290,7 +302,7 @@ sparse_status_t sparse_score(const sparse_shape_t *shape, const void *q,
   if (!sd::aligned(q, 16) || !sd::aligned(K, 16) || !sd::aligned(S, 16))
     return SPARSE_ERR_INVALID_ARG;
   if ((r = sd::check_ws(s, 1, 1, ws, ws_bytes)) != SPARSE_OK) return r;
-  return sd::from_cuda(sd::launch_score(s, q, K, S, nullptr, sd::status_word(ws),
+  return sd::from_cuda(sd::launch_score(s, q, K, S, nullptr, nullptr, sd::status_word(ws),
                                         static_cast<cudaStream_t>(stream)));
 }
 
@@ -378,9 +390,9 @@ sparse_status_t sparse_attn_gather(const sparse_shape_t *shape, int32_t L,
     return SPARSE_ERR_INVALID_ARG;
   if ((r = sd::check_ws(s, stride, L, ws, ws_bytes)) != SPARSE_OK) return r;
   const sd::Layout l = sd::layout(s, stride, L);
-  return sd::from_cuda(sd::launch_attn(
-      s, L, q, K, V, idx, stride, count, stride, out, lse, sd::attn_ptr(ws, l),
-      sd::attn_counters(ws), sd::status_word(ws), static_cast<cudaStream_t>(stream)));
+  return sd::from_cuda(sd::launch_attn(s, L, q, K, V, idx, stride, count, stride, out, lse,
+                                       sd::attn_ptr(ws, l), sd::status_word(ws),
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
@@ -512,7 +524,7 @@ sparse_status_t sparse_louver_decode_step(const sparse_shape_t *shape, int32_t L
                                    louver_ws, sd::status_word(ws), st);
   if (e == cudaSuccess)
     e = sd::launch_attn(s, L, q_layers, K, V, idx, cap, count, cap, out, lse, sd::attn_ptr(ws, l),
-                        sd::attn_counters(ws), sd::status_word(ws), st);
+                        sd::status_word(ws), st);
   return sd::from_cuda(e);
 }
 

@@ -1,4 +1,4 @@
-// attn.cu -- A3 + A4 for fp32 inputs (bf16 inputs take attn_mma.cu).
+// attn.cu -- A3 + A4 for fp32 inputs (bf16 inputs take attn_fused.cu).
 //
 // Every query vector of every layer attends over the same selected rows of
 // its KV head (CLSA article, section CLSAの仕組み: the routing set is reused
@@ -244,7 +244,7 @@ cudaError_t launch_attn_t(const Shape &s, int L, const void *q, const void *K,
 }  // namespace
 
 size_t attn_workspace_bytes(const Shape &s, int L, int stride) {
-  if (s.dtype == 1) return attn_tc_workspace_bytes(s, L);
+  if (s.dtype == 1) return 0;  // the tcgen05 kernel merges its splits on chip
   const int Mtot = L * s.G();
   const int qblocks = (Mtot + kQPerCta - 1) / kQPerCta;
   const int nsplit = num_splits(s.BH(), qblocks, stride);
@@ -254,17 +254,9 @@ size_t attn_workspace_bytes(const Shape &s, int L, int stride) {
 cudaError_t launch_attn(const Shape &s, int L, const void *q, const void *K,
                         const void *V, const int *idx, int stride,
                         const int *count, int count_cap, void *out, float *lse,
-                        void *ws, uint32_t *counters, uint32_t *status,
-                        cudaStream_t st) {
-  if (s.dtype == 1) {
-    // bf16: tcgen05 tensor cores by default; SPARSE_DECODE_ATTN=mma selects
-    // the warp-level mma.sync kernel instead (kept for comparison).
-    const char *impl = getenv("SPARSE_DECODE_ATTN");
-    if (impl && strcmp(impl, "mma") == 0)
-      return launch_attn_mma(s, L, q, K, V, idx, stride, count, out, lse, status, st);
-    return launch_attn_tc(s, L, q, K, V, idx, stride, count, out, lse, ws, counters,
-                          status, st);
-  }
+                        void *ws, uint32_t *status, cudaStream_t st) {
+  if (s.dtype == 1)
+    return launch_attn_fused(s, L, q, K, V, idx, stride, count, out, lse, status, st);
   if (s.d == 128)
     return launch_attn_t<float, 128>(s, L, q, K, V, idx, stride, count, count_cap,
                                      out, lse, ws, status, st);

@@ -16,6 +16,9 @@ enum : uint32_t {
   FLAG_TIMEOUT = 1u << 2,
   FLAG_INDEX = 1u << 3,
   FLAG_INTERNAL = 1u << 4,
+  // informational, not an error: a top-k select took its exact streaming
+  // path (its fast path's preconditions did not hold for some head)
+  FLAG_SLOW_SELECT = 1u << 8,
 };
 
 __device__ __forceinline__ void raise_flag(uint32_t *status, uint32_t f) {
@@ -115,6 +118,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     }
   }
   return true;
+}
+
+// ---- shared-memory atomics addressed in the shared window -----------------
+// (explicit .shared forms: no generic-address resolution on a hot path)
+__device__ __forceinline__ void sh_red_or(uint32_t *p, uint32_t v) {
+  asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sh_red_add(uint32_t *p, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t sh_atom_add(uint32_t *p, uint32_t v) {
+  uint32_t r;
+  asm volatile("atom.shared.add.u32 %0, [%1], %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(v)
+               : "memory");
+  return r;
 }
 
 // ---- 1-D bulk copy global -> shared (TMA, no tensor map) ------------------

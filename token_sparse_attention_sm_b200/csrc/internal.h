@@ -6,6 +6,9 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "route_cand.cuh"
+#include "sparse_decode.h"
+
 namespace sd {
 
 struct Shape {
@@ -15,6 +18,9 @@ struct Shape {
   int BH() const { return B * Hkv; }
   int esize() const { return dtype == 0 ? 4 : 2; }
 };
+
+// Reads and checks a caller's shape (the checks every entry point shares).
+sparse_status_t check_shape(const sparse_shape_t *shape, Shape *s);
 
 // Device properties cached per device (SM count, cluster support).
 struct DeviceInfo {
@@ -37,41 +43,28 @@ inline void add_pdl_attr(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attrs) {
 
 // A1: S[b,h,j] for every key; one streaming pass over K.  hist (nullable):
 // [B*Hkv][2048] counts of the top 11 key bits, accumulated (must start zero).
-cudaError_t launch_score(const Shape &s, const void *q, const void *K,
-                         float *S, uint32_t *hist, uint32_t *status,
-                         cudaStream_t st);
+// cand (nullable): a plan from plan_cand with its list pointers -- the scan
+// then also draws the sample and fills the candidate lists (top-k routing).
+cudaError_t launch_score(const Shape &s, const void *q, const void *K, float *S, uint32_t *hist,
+                         const CandArgs *cand, uint32_t *status, cudaStream_t st);
+// Keys per scan tile, and the scan's grid (one CTA per SM, at most one per tile).
+int scan_stage_keys(const Shape &s);
+int scan_grid(const Shape &s, int sm_count);
+// Fills the plan fields of cand (not the pointers) for top-k routing with
+// candidate lists; false when the lists do not apply to this shape and k.
+bool plan_cand(const Shape &s, int k, int sm_count, CandArgs *cand);
+// The workspace areas of the candidate lists and their lengths for a shape
+// (0 when lists never apply to it), and the CTAs a head can span.
+constexpr size_t kCandMaxListBytes = (size_t)512 << 20;
+int cand_head_ctas_of(const Shape &s);
+size_t cand_list_bytes(const Shape &s);
+size_t cand_count_bytes(const Shape &s);
 
-// A1 + A2 fused (route_fused.cu): the scan and the exact top-k in one
-// persistent kernel whose CTAs synchronise per head through counters in
-// global memory.  ctr: one uint32 per head, zero between calls (the kernel
-// resets them); seg_area: kFusedSegAreaBytes of scratch.  Returns
-// cudaErrorNotSupported, launching nothing, when the shape does not fit (a
-// CTA's keys must fit on chip) or unless SPARSE_DECODE_FUSED_ROUTE=1 (the
-// scan followed by the select kernel is the default: at the 128K decode
-// shapes the two are on par and the two-kernel path leaves SMs free for the
-// attention kernel to start early).
-constexpr int kFusedMaxCtas = 256;
-constexpr int kFusedMaxHeads = 768;
-constexpr int kFusedSegCap = 1024;  // boundary-bin keys a CTA publishes per head
-constexpr size_t kFusedMetaBytes = (size_t)kFusedMaxCtas * 2 * 8;
-constexpr size_t kFusedSegAreaBytes =
-    kFusedMetaBytes + (size_t)kFusedMaxCtas * 2 * kFusedSegCap * sizeof(uint32_t);
-bool fused_route_enabled();
-cudaError_t launch_route_topk_fused(const Shape &s, const void *q, const void *K, int k,
-                                    float *S, uint32_t *hist, uint32_t *ctr, void *seg_area,
-                                    int *idx, uint32_t *status, cudaStream_t st);
-
-// Kernels whose CTAs wait for one another (the fused routing kernel, the
-// split merge of the tcgen05 attention) rely on the whole grid being resident
-// at once -- at most one CTA per SM.  They are launched as ordinary kernels so
-// that programmatic dependent launch can overlap them with their predecessor;
-// SPARSE_DECODE_COOPERATIVE=1 launches them cooperatively instead (the driver
-// then guarantees co-residency even next to other work on the device).
-bool cooperative_forced();
-// The split attention merges its partials inside a thread-block cluster
-// (distributed shared memory) when the clusters fit; SPARSE_DECODE_ATTN_MERGE=global
-// selects the merge through global memory and a counter barrier instead.
-bool attn_cluster_merge_enabled();
+// A2 after the scan: one CTA per head selects the exact top-k from the
+// scan's histogram and candidate lists (cand nullable: from the score rows)
+// and clears what it consumed.
+cudaError_t launch_select_cand(const Shape &s, const float *S, int k, int *idx, uint32_t *hist,
+                               const CandArgs *cand, uint32_t *status, cudaStream_t st);
 
 // A2 / A2': selection from S.  k >= 1: top-k (tau ignored); k == 0:
 // threshold with tau and cap, count written.  idx rows have `stride`
@@ -83,28 +76,30 @@ cudaError_t launch_select(const Shape &s, const float *S, int k,
                           cudaStream_t st);
 
 // A3 + A4: L query sets over the same index rows.  bf16 runs on the tcgen05
-// tensor cores (split partials in the workspace) or, on request, the mma.sync
-// kernel (split merge in distributed shared memory); fp32 runs on the CUDA
-// cores with split partials in the workspace.
+// tensor cores (attn_fused.cu, no workspace); fp32 on the CUDA cores with
+// split partials in the workspace (attn.cu).
 size_t attn_workspace_bytes(const Shape &s, int L, int stride);
-cudaError_t launch_attn_mma(const Shape &s, int L, const void *q, const void *K,
-                            const void *V, const int *idx, int stride,
-                            const int *count, void *out, float *lse,
-                            uint32_t *status, cudaStream_t st);
-size_t attn_tc_workspace_bytes(const Shape &s, int L);
-// Split-merge counters of the tcgen05 attention: two per (head, query block)
-// in a fixed, shape-independent area of the workspace header (zero between
-// calls: the kernel resets them).  More blocks than this run unsplit.
-constexpr int kAttnMaxCounterBlocks = 96;
-cudaError_t launch_attn_tc(const Shape &s, int L, const void *q, const void *K,
-                           const void *V, const int *idx, int stride,
-                           const int *count, void *out, float *lse, void *ws,
-                           uint32_t *counters, uint32_t *status, cudaStream_t st);
 cudaError_t launch_attn(const Shape &s, int L, const void *q, const void *K,
                         const void *V, const int *idx, int stride,
                         const int *count, int count_cap, void *out, float *lse,
-                        void *ws, uint32_t *counters, uint32_t *status,
-                        cudaStream_t st);
+                        void *ws, uint32_t *status, cudaStream_t st);
+cudaError_t launch_attn_fused(const Shape &s, int L, const void *q, const void *K, const void *V,
+                              const int *idx, int stride, const int *count, void *out, float *lse,
+                              uint32_t *status, cudaStream_t st);
+// The tail of routing fused into the attention kernel (bf16, L*G <= 128,
+// N <= 131072, every split's keys on chip): top-k from the scan's
+// by-products (writes idx [B*Hkv][k], clears hist and the sample state), or
+// the threshold sets from the marking scan's bitmaps (writes idx rows of
+// `cap` and count).
+bool fused_route_ok(const Shape &s, int L, int k_or_cap);
+cudaError_t launch_route_attn_topk(const Shape &s, int L, const void *q_layers, const void *K,
+                                   const void *V, int k, const float *S, uint32_t *hist,
+                                   const CandArgs *cand, int *idx, void *out, float *lse,
+                                   uint32_t *status, cudaStream_t st);
+cudaError_t launch_route_attn_threshold(const Shape &s, int L, const void *q_layers,
+                                        const void *K, const void *V, const uint32_t *bits,
+                                        int cap, int *idx, int *count, void *out, float *lse,
+                                        uint32_t *status, cudaStream_t st);
 
 // Louver index (louver.cu).  louver_shape_ok: r and N fit the balanced tree.
 bool louver_shape_ok(const Shape &s, int r);

@@ -869,8 +869,11 @@ cudaError_t lv_query_t(const Shape &s, const void *qv, int r, const char *index,
   cfg.gridDim = dim3((unsigned)splits, (unsigned)s.BH(), 1);
   cfg.blockDim = dim3(kQThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
-  cfg.numAttrs = (splits > 1 && cooperative_forced()) ? 1 : 0;
-  add_pdl_attr(cfg, attrs);
+  // the CTAs of a head meet at a counter barrier: a cooperative launch makes
+  // the driver guarantee that they are all resident (at the price of not
+  // overlapping with the previous kernel); a single CTA per head needs neither
+  cfg.numAttrs = splits > 1 ? 1 : 0;
+  if (splits == 1) add_pdl_attr(cfg, attrs);
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(qv), s.Hq, s.Hkv, s.N, scale,
                          reinterpret_cast<const int *>(index + l.perm),
                          reinterpret_cast<const float *>(index + l.centres),

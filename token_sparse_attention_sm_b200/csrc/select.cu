@@ -16,11 +16,12 @@
 //    needed) 11 more bits, then the last 10 bits.  The result is either a key
 //    threshold T (take every key >= T) or the exact k-th key value v plus the
 //    number t of keys equal to v to take, which go to the lowest indices.
-//  * This file holds the general path: each level builds a shared-memory
-//    histogram per CTA, one cluster barrier, and every CTA sums the C
-//    histograms through distributed shared memory.  When the score scan has
-//    already counted the top 11 bits (route and decode calls), the top-k
-//    fast path in select_topk.cu runs instead.
+//  * Each level builds a shared-memory histogram per CTA, one cluster
+//    barrier, and every CTA sums the C histograms through distributed shared
+//    memory.  (Routing calls, where the score scan has already counted the
+//    top 11 bits and kept candidate lists, select in select_cand.cu or in
+//    the fused attention kernel instead; this kernel serves selections from
+//    given scores and the Louver index build.)
 //  * Compaction is order preserving: each warp owns a contiguous run of its
 //    CTA's slice and walks it 32 keys at a time; warp ballots and popcounts
 //    give positions, one more cluster barrier exchanges the per-CTA totals,
@@ -128,17 +129,10 @@ static cudaError_t plan_select(const Shape &s, SelectPlan *plan) {
 
 cudaError_t select_cluster_size(int sm_count, int smem_optin, int *out);
 
-cudaError_t launch_select_topk_fast(const Shape &s, const float *S, int k, int *idx,
-                                    uint32_t *hist, uint32_t *status, cudaStream_t st);
-
 cudaError_t launch_select(const Shape &s, const float *S, int k,
                           const float *tau, int cap, int *idx, int *count,
                           int stride, uint32_t *hist, uint32_t *status,
                           cudaStream_t st) {
-  if (k > 0 && hist && stride == k) {
-    const cudaError_t ef = launch_select_topk_fast(s, S, k, idx, hist, status, st);
-    if (ef != cudaErrorNotSupported) return ef;
-  }
   SelectPlan plan;
   cudaError_t e = plan_select(s, &plan);
   if (e != cudaSuccess) return e;

@@ -1,5 +1,5 @@
-// select_common.cuh -- pieces shared by the two selection kernels
-// (select.cu: general top-k and threshold; select_topk.cu: top-k fast path).
+// select_common.cuh -- the cluster radix select of select.cu (general top-k
+// and threshold selection from given scores).
 #pragma once
 #include <cooperative_groups.h>
 
@@ -14,35 +14,18 @@ constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kBinsPerThread = kBins / kSelThreads;
-constexpr int kCandLocal = 2048;  // boundary-bin keys one CTA may hold
-constexpr int kCandAll = 8192;    // boundary-bin keys of a whole head
 constexpr int kMaxCluster = 16;
-constexpr int kFinMax = 64;       // keys ranked pairwise after two levels
-constexpr int kWarpList = 128;    // fast path: keys >= the boundary bin per warp
-constexpr int kSelFixedSmem =
-    2 * kBins * 4 + kCandLocal * 8 + kCandAll * 4 + 2 * kSelWarps * kWarpList * 4 + 1024;
+constexpr int kSelFixedSmem = 2 * kBins * 4 + 1024;
 
 struct SelShared {
   uint32_t hist[2][kBins];
-  uint2 cand_local[kCandLocal];     // (key, slice index); read remotely
-  uint32_t cand_all[kCandAll];
   uint32_t warp_buf[33];
   alignas(8) uint32_t pub[2];  // this CTA's (>= T, == v) counts, read remotely
-  uint32_t bnd[3];        // boundary bin, count above it, count in it
-  uint32_t ncand;         // candidates in cand_local (may exceed kCandLocal)
-  uint32_t cinfo[2];      // total candidates, overflow flag
-  uint32_t wge[kSelWarps];  // per-warp counts of keys >= threshold
-  uint32_t weq[kSelWarps];  // per-warp counts of keys == tie value
-  uint32_t rcnt[kMaxCluster];  // candidates held by each CTA of the cluster
+  uint32_t bnd[3];             // boundary bin, count above it, count in it
+  uint32_t wge[kSelWarps];     // per-warp counts of keys >= threshold
+  uint32_t weq[kSelWarps];     // per-warp counts of keys == tie value
   uint32_t rge[kMaxCluster];   // per-CTA counts, copied from remote pub[]
   uint32_t req[kMaxCluster];
-  uint32_t wdef[kSelWarps];    // fast path: keys above the boundary bin, per warp
-  uint32_t wpass[kSelWarps];   // fast path: boundary-bin keys that pass, per warp
-  int seg4[kSelWarps + 1];     // fast path: warp segment bounds in float4 units
-  uint32_t nfin;               // fast path: keys left after two levels
-  uint32_t fin[kFinMax];
-  uint32_t wl_key[kSelWarps][kWarpList];  // fast path: per-warp key lists
-  uint32_t wl_idx[kSelWarps][kWarpList];
 };
 static_assert(sizeof(SelShared) <= kSelFixedSmem, "fixed select smem");
 
