@@ -273,16 +273,17 @@ def capture_loop(fn_list, stream):
 
 
 def kernels_per_step(w, reroute: int = 0) -> int:
-    """Kernels one decode step launches: the routing scan, then -- for bf16
-    steps whose shape lets the attention kernel finish the routing (L*G <=
-    128 query vectors per head, N <= 131072, k or cap <= 16384) -- that one
+    """Kernels one decode step launches: the routing scan, then -- where the
+    library says the step runs fused (bf16, L*G <= 128 query vectors per
+    head, N <= 131072, k or cap <= 32768) -- the one select + attention
     kernel, else the select (or threshold compaction) and the attention (one
     kernel for bf16, a partial and a merge kernel for fp32); once per group of
     `reroute` layers when routing is re-computed."""
+    import token_sparse_attention_sm_b200 as sd
     lg = min(reroute, w.L) if reroute else w.L
-    stride = w.k if w.mode == "topk" else w.cap
-    fused = (w.dtype == "bf16" and lg * (w.Hq // w.Hkv) <= 128 and w.N <= 131072
-             and stride <= 16384)
+    fused = sd.decode_step_fused(w.B, w.N, w.Hq, w.Hkv, w.d, w.torch_dtype, lg,
+                                 k=w.k if w.mode == "topk" else None,
+                                 cap=w.cap if w.mode != "topk" else None)
     per_group = 2 if fused else 2 + (1 if w.dtype == "bf16" else 2)
     groups = -(-w.L // reroute) if reroute else 1
     return per_group * groups
@@ -546,10 +547,12 @@ def run_e2e(sd, w, variants, K, V, ws, stream, dev, args, world):
             "h2d_bytes_per_step": g0.h2d_bytes, "d2h_bytes_per_step": g0.d2h_bytes,
             "steps": steps,
             "api": "token_sparse_attention_sm_b200.DecodeStepGraph (routing and the layers' "
-                   "attention in one CUDA graph with the host transfers: the layers' queries "
-                   "and the index set cross PCIe on a second stream while routing and "
-                   "attention run, the attention writes its outputs into mapped pinned host "
-                   "memory (mapped_out=%s); synchronised every step)" % g0.mapped_out}
+                   "attention in one CUDA graph with the host transfers: the routing query "
+                   "crosses PCIe first, the layers' queries on a second stream while the "
+                   "routing scan runs; fused=%s: the select + attention kernel writes the "
+                   "outputs and the index set into mapped pinned host memory "
+                   "(results_direct=%s); synchronised every step)" % (g0.fused,
+                                                                      g0.results_direct)}
 
 
 # ---------------------------------------------------------------------------

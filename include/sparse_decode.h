@@ -62,26 +62,21 @@
  * Asynchrony: every compute entry point enqueues its kernels on `stream`
  * and returns without synchronising.
  *
- * Co-residency: the bf16 attention kernel, the Louver query kernel (and the
- * optional fused routing kernel) split one head's work over several CTAs
- * that wait for one another (bounded waits).  Their grid is at most one CTA per SM, so it is resident
- * as a whole while the device runs nothing else; they are launched as
- * ordinary kernels so that each can start while its predecessor drains.  A
- * caller that runs other kernels on the same device at the same time (other
- * streams, other processes) sets SPARSE_DECODE_COOPERATIVE=1: they are then
- * launched cooperatively and the driver guarantees co-residency.  Where all
- * of a launch's heads fit at once as thread-block clusters, the attention's
- * splits of a head run as one cluster instead and merge through distributed
- * shared memory behind hardware cluster barriers.
+ * Co-residency: no kernel of the library waits for a CTA that is not
+ * already running.  The bf16 attention splits each head over up to 16 CTAs
+ * that form one thread-block cluster (the hardware schedules a cluster's
+ * CTAs together) and meet only at cluster barriers.  The routing scan's CTAs
+ * never wait for one another: a CTA that finds a head's sample incomplete
+ * when its own tiles are done marks that head's keys without a bound (every
+ * key a candidate).  The Louver query, whose CTAs of a head meet at a
+ * counter barrier in global memory, is launched cooperatively (the driver
+ * then guarantees that the whole grid is resident) whenever a head spans
+ * several CTAs.  So another kernel or process sharing the device can slow a
+ * call down but cannot stall it.
  *
  * Environment variables read by the library:
- *   SPARSE_DECODE_PDL=0           no programmatic dependent launch
- *   SPARSE_DECODE_COOPERATIVE=1   cooperative launches (see Co-residency)
- *   SPARSE_DECODE_FUSED_ROUTE=1   top-k routing as one fused scan+select kernel
- *                                 where the shape allows (results identical)
- *   SPARSE_DECODE_ATTN=mma        bf16 attention on the mma.sync kernel
- *   SPARSE_DECODE_ATTN_MERGE=global  the attention's split merge through
- *                                 global memory even where clusters would fit
+ *   SPARSE_DECODE_PDL=0           no programmatic dependent launch between
+ *                                 the library's kernels
  */
 #ifndef SPARSE_DECODE_H_
 #define SPARSE_DECODE_H_
@@ -210,6 +205,32 @@ sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
                                    float *lse, void *ws, size_t ws_bytes,
                                    void *stream);
 
+/* sparse_decode_step with the layers' queries arriving late: the routing
+ * (which reads only q_route) is enqueued first, then the stream waits on
+ * layers_ready (a cudaEvent_t recorded after q_layers was written, e.g. by a
+ * copy on another stream; NULL: no wait), then the attention is enqueued.
+ * The same arguments, checks and results as sparse_decode_step otherwise.
+ * When the step runs on the fused kernels (sparse_decode_step_fused), idx,
+ * count and out are only written, never read back, so they may point into
+ * mapped pinned host memory (sparse_pointer_device_usable); on the other
+ * path the attention reads idx and count, which then belong in device
+ * memory. */
+sparse_status_t sparse_decode_step_join(const sparse_shape_t *shape, int32_t L,
+                                        const void *q_route, const void *q_layers,
+                                        const void *K, const void *V, int32_t k,
+                                        const float *tau, int32_t cap, int32_t *idx,
+                                        int32_t *count, void *out, float *lse, void *ws,
+                                        size_t ws_bytes, void *stream, void *layers_ready);
+
+/* Whether sparse_decode_step on this shape (k >= 1: top-k; k == 0: threshold
+ * with cap >= 1) takes the fused kernels -- the routing scan, then one
+ * kernel that selects and attends -- (*fused = 1) or routes and attends in
+ * separate kernels (*fused = 0).  Fused: bf16, L * Hq / Hkv <= 128, N <=
+ * 131072 and k (or cap) <= 32768.  Pure shape logic: no device call.
+ * Returns SPARSE_ERR_INVALID_ARG for a null fused or invalid L, k, cap. */
+sparse_status_t sparse_decode_step_fused(const sparse_shape_t *shape, int32_t L, int32_t k,
+                                         int32_t cap, int32_t *fused);
+
 /* Decode step that re-routes every R layers (CLSA article, section
  * 計算コストの削減効果: token-sparse attention with per-layer routing (DSA)
  * scores the context once per layer, CLSA once per step; section
@@ -329,8 +350,8 @@ sparse_status_t sparse_louver_decode_step(const sparse_shape_t *shape, int32_t L
 
 /* Self-test of failure detection, with no fault: one device thread waits,
  * through the bounded wait that every counter barrier of the library uses
- * (the split attention's merge, the Louver query's per-head barrier, the
- * fused routing kernel), on a workspace word that nothing ever increments.
+ * (the Louver query's per-head barrier), on a workspace word that nothing
+ * ever increments.
  * After limit_ns of the GPU's global timer (capped at the library's own 2 s
  * limit) the wait gives up and raises the TIMEOUT flag in the status word,
  * so sparse_read_device_status then returns SPARSE_ERR_TIMEOUT and the

@@ -225,3 +225,38 @@ def test_result_and_tau_checks_reject_bad_tensors(lib):
         sd._need_tau(torch.zeros(2, 4), (2, 3))
     with pytest.raises(ValueError, match="tau"):
         sd._need_tau(torch.zeros(2, 3, dtype=torch.int32), (2, 3))
+
+
+def test_decode_step_fused_is_shape_logic(lib):
+    """Which decode steps run on the fused select + attention kernel: bf16
+    with at most 128 query rows per KV head over all layers and a cache the
+    select's on-chip bitmap covers; the answer needs no device."""
+    def fused(sh, L, k, cap=0):
+        f = ctypes.c_int32(-1)
+        rc = lib.sparse_decode_step_fused(ctypes.byref(sh), L, k, cap, ctypes.byref(f))
+        return rc, f.value
+    big = _shape(N=131072, Hq=32, Hkv=8, d=128)
+    assert fused(big, 16, 2048) == (0, 1)
+    assert fused(big, 16, 0, 8192) == (0, 1)                      # threshold
+    assert fused(_shape(N=131072, Hq=32, Hkv=8, d=128, dtype=0), 16, 2048) == (0, 0)
+    assert fused(_shape(N=262144, Hq=32, Hkv=8, d=128), 16, 2048) == (0, 0)
+    assert fused(big, 64, 2048) == (0, 0)                         # 256 query rows
+    assert fused(big, 0, 2048)[0] == 1
+    assert fused(big, 16, 0, 0)[0] == 1
+    assert lib.sparse_decode_step_fused(ctypes.byref(big), 16, 2048, 0, None) == 1
+    assert lib.sparse_decode_step_fused(ctypes.byref(_shape(d=96)), 2, 16, 0,
+                                        ctypes.byref(ctypes.c_int32())) == 2
+
+
+def test_decode_step_join_checks_like_decode_step(lib):
+    sh = _shape()
+    fake = ctypes.c_void_p(1 << 20)
+    ws_ok = ctypes.c_void_p(1 << 24)
+    rc, need = _ws_size(lib, sh, k=16, L=2)
+    # both k and tau; then a workspace one byte short
+    assert lib.sparse_decode_step_join(ctypes.byref(sh), 2, fake, fake, fake, fake, 16, fake,
+                                       0, fake, fake, fake, None, ws_ok, need, None,
+                                       None) == 1
+    assert lib.sparse_decode_step_join(ctypes.byref(sh), 2, fake, fake, fake, fake, 16, None,
+                                       0, fake, None, fake, None, ws_ok, need - 1, None,
+                                       None) == 3

@@ -377,3 +377,66 @@ def test_louver_nonfinite_inputs_are_flagged(dev):
     tau = torch.tensor([[0.5, 0.5]], device=dev)
     a = sd.louver_route_threshold(qd, Kc, ix, tau, 2048)
     _assert_same_set(a, sd.route_threshold(qd, Kc, tau, 2048), 2048)
+
+
+def _keys_on_a_line(rng, N, d, torch_dtype):
+    """Keys t_i * s (one head): t a permutation of N distinct values, s a
+    fixed direction.  fp32: s a random unit vector plus 1e-3 noise per key;
+    bf16: s with entries in {+-1, +-1/2, +-1/4} and t integers in [-N/2, N/2),
+    so every key is exact in bf16 (N <= 256) and the keys are collinear."""
+    t = rng.permutation(N).astype(np.float64) - N // 2
+    if torch_dtype == torch.float32:
+        s = rng.standard_normal(d)
+        s /= np.linalg.norm(s)
+        Kh = t[:, None] * s[None, :] + 1e-3 * rng.standard_normal((N, d))
+    else:
+        s = rng.choice([-1.0, -0.5, -0.25, 0.25, 0.5, 1.0], size=d)
+        Kh = t[:, None] * s[None, :]
+    return t, Kh.astype(np.float32)
+
+
+@pytest.mark.parametrize("dtype,d,N,r", [("f32", 64, 4096, 64), ("bf16", 128, 256, 32),
+                                         ("f32", 128, 2048, 256)])
+def test_louver_tree_splits_keys_on_a_line_by_their_coordinate(dev, dtype, d, N, r):
+    """Louver summary, section 2. Louver インデックス (balanced tree of
+    principal-direction splits at the median): for keys spread along one
+    direction the principal direction of every node is that direction, so
+    every node of the tree -- each run of N / 2^L consecutive entries of the
+    cluster order, down to the 32-key leaves -- holds the keys whose
+    coordinates along it have ranks in one aligned block [j N/2^L, (j+1)
+    N/2^L).  The GPU tree must have this form at every level, and its node
+    sets must equal the oracle's (fp64 eigendecomposition) at every level.
+    """
+    torch_dtype = torch.float32 if dtype == "f32" else torch.bfloat16
+    rng = np.random.default_rng(4242)
+    B, Hkv = 1, 2
+    ts, K32 = [], np.zeros((B, Hkv, N, d), np.float32)
+    for h in range(Hkv):
+        t, Kh = _keys_on_a_line(rng, N, d, torch_dtype)
+        ts.append(t)
+        K32[0, h] = Kh
+    K = torch.from_numpy(K32).to(dev, torch_dtype)
+    assert torch.equal(K.float().cpu(), torch.from_numpy(K32)), "keys not exact in this dtype"
+    ix = sd.louver_build(K, r)
+    torch.cuda.synchronize()
+    _check_index(ix, K32, r)
+    perm = ix.perm().cpu().numpy()
+    for h in range(Hkv):
+        rank = np.empty(N, np.int64)
+        rank[np.argsort(ts[h], kind="stable")] = np.arange(N)
+        oix = olouver.build_index(K32[0, h], r)
+        operm = np.asarray(oix["perm"])
+        size = N // 2
+        while size >= 32:
+            for j in range(N // size):
+                blk = rank[perm[0, h, j * size:(j + 1) * size]]
+                lo = blk.min()
+                assert lo % size == 0 and blk.max() == lo + size - 1, \
+                    f"head {h}: node of {size} keys is not one block of coordinate ranks"
+            if size >= r:  # the oracle's tree stops at the clusters
+                g = sorted(tuple(sorted(perm[0, h, j * size:(j + 1) * size].tolist()))
+                           for j in range(N // size))
+                o = sorted(tuple(sorted(operm[j * size:(j + 1) * size].tolist()))
+                           for j in range(N // size))
+                assert g == o, f"head {h}: nodes of {size} keys differ from the oracle's"
+            size //= 2

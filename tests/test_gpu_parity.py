@@ -1,8 +1,9 @@
 """Parity of the CUDA library (through its C ABI) with the CPU oracle.
 
 Comparison rules (fixed before any kernel ran):
-* Scores: |S_gpu - S_exact| within the fp32 summation bound
-  (G*d + 2) * 2^-24 * sum|q_i k_i| / sqrt(d), with S_exact in fp64.
+* Scores: |S_gpu - S_exact| within the fp32 rounding bound of the kernel's
+  order of operations, gamma_{G+d+1} * sum|q_i k_i| / sqrt(d) with
+  gamma_n = n 2^-24 / (1 - n 2^-24), S_exact in fp64.
 * Selection on the SAME fp32 scores (the GPU's own, fed to the oracle):
   bit-exact index sets, ties included (the decision is taken in the same
   precision on both sides).
@@ -101,7 +102,16 @@ def test_scores_match_oracle(dev, c):
     Krep = np.repeat(np.abs(K.astype(np.float64)), G, axis=1)
     mag = np.einsum("bgd,bgnd->bgn", np.abs(q.astype(np.float64)), Krep)
     mag = mag.reshape(w.B, w.Hkv, G, w.N).sum(axis=2) / np.sqrt(w.d)
-    bound = (G * w.d + 2) * 2.0 ** -24 * mag * 2 + 1e-30
+    # The kernel sums the G query rows (G-1 fp32 additions), multiplies by
+    # fl(1/sqrt(d)) (two roundings: the constant and the product), then takes
+    # one d-long dot product with fused multiply-adds (at most d-1 rounded
+    # additions in any order).  Every rounding is relative to a partial sum
+    # bounded by the magnitudes above, so with u = 2^-24 and
+    # gamma_n = n u / (1 - n u) the error is at most gamma_{G+d} * mag; one
+    # more u covers the fp64 arbiter's own rounding (about 2^-53 * G d * mag).
+    u = 2.0 ** -24
+    n = G + w.d + 1
+    bound = n * u / (1 - n * u) * mag + 1e-30
     assert np.all(np.abs(S - S64) <= bound)
 
 
@@ -254,15 +264,6 @@ def _route(path, t, K, k, ws=None, L=1):
     return res["idx"]
 
 
-def _sample_tiles(N, d=128, esize=2, want=32):
-    """Key ranges [j0, j1) of the routing scan's sample tiles of a head (tile
-    u of a head is sampled when u % stride == 0)."""
-    per = 32768 // (d * esize)
-    tph = -(-N // per)
-    stride = max(1, tph // want)
-    return [(u * per, min(N, (u + 1) * per)) for u in range(0, tph, stride)]
-
-
 ROUTE_CASES = [
     dict(B=1, N=4096, Hq=8, Hkv=2, d=64, k=256, dtype="f32"),
     dict(B=2, N=10007, Hq=32, Hkv=8, d=128, k=333, dtype="bf16", heavy=16),
@@ -304,8 +305,9 @@ def _check_decode(dev, w, x, batches_checked=None):
     assert_topk_within_band(gidx[bsel], S, w.k)
     # shared routing: the fused step's set is the routing call's set, bitwise
     np.testing.assert_array_equal(gidx, sd.route_topk(t["q_route"], t["K"], w.k).cpu().numpy())
-    # every layer's output equals the gather call on that set, and matches the
-    # oracle on the oracle's own set
+    # every layer's output equals the gather call on that set (both split the
+    # set into the same equal shares), and matches the oracle on the oracle's
+    # own set
     out2, lse2 = sd.attn_gather(t["q_layers"], t["K"], t["V"], res["idx"])
     assert torch.equal(out2, res["out"]) and torch.equal(lse2, res["lse"])
     ridx = oracle.topk(S, w.k)
@@ -377,7 +379,7 @@ def test_decode_step_threshold_empty_set(dev):
 
 def test_route_topk_all_equal_keys_takes_lowest_indices(dev, route_path):
     """Every score equal: the boundary bin holds all N keys, more than the
-    candidate buffers, so the select takes its general path."""
+    select lists on chip, so the select takes its streaming path."""
     w = synth.custom(B=1, N=20000, Hq=8, Hkv=2, d=128, L=1, k=300, dtype="bf16", seed=4)
     x = synth.generate(w)
     t = _to(dev, x)
@@ -388,20 +390,18 @@ def test_route_topk_all_equal_keys_takes_lowest_indices(dev, route_path):
 
 
 def test_route_topk_recovers_from_dirty_workspace(dev, route_path):
-    """A workspace whose histogram and sample areas hold garbage (not
-    zero-filled) is detected (the counts do not sum to N; the candidate lists
-    come out short) and the result is still exact; the call leaves those
-    areas clean for the next one."""
+    """A workspace whose histogram area holds garbage (not zero-filled) is
+    detected (the counts do not sum to N) and the result is still exact; the
+    call leaves the area clean for the next one."""
     w = synth.custom(B=2, N=5000, Hq=8, Hkv=2, d=128, L=1, k=100, dtype="bf16", seed=6)
     x = synth.generate(w)
     t = _to(dev, x)
     S = oracle.scores(_f(x["q_route"]), _f(x["K"]))
     ws = sd.Workspace(dev)
     ws.get(sd.workspace_bytes(2, 5000, 8, 2, 128, torch.bfloat16, 100, 1))
-    # header 4 KB | histogram [256][2048] | sample histogram [256][2048] | sample counts
-    hist, smp = 4096, 4096 + 256 * 2048 * 4
-    cnt = smp + 256 * 2048 * 4
-    areas = [(hist, hist + 4 * 2048 * 4), (smp, smp + 4 * 2048 * 4), (cnt, cnt + 4 * 4)]
+    # header 4 KB | histogram [256][2048] | scores
+    hist = 4096
+    areas = [(hist, hist + 4 * 2048 * 4)]
     for a, b in areas:
         ws.buf[a:b] = 7
     for _ in range(2):
@@ -484,40 +484,93 @@ def test_fused_select_equals_select_kernel(dev, B, N, Hkv, k):
     assert_topk_within_band(a, S, k)
 
 
+def _plant(K, rows, v):
+    """K [B,Hkv,N,d] with the given rows of every head set to the vector v."""
+    K = K.clone()
+    K[:, :, rows] = v.to(K.dtype)
+    return K
+
+
+def _qbar_dir(t, Hkv):
+    """Unit vector along head 0's summed routing query (its keys' score
+    direction)."""
+    q = t["q_route"][0].float()
+    qbar = q.reshape(Hkv, q.shape[0] // Hkv, -1).sum(1)[0]
+    return qbar / qbar.norm()
+
+
 @pytest.mark.parametrize("route", ["select_kernel", "fused_step"])
-@pytest.mark.parametrize("B,N,Hkv", [(1, 131072, 8), (2, 65536, 4)])
-def test_select_when_the_sample_misleads(dev, route, B, N, Hkv):
-    """The routing scan estimates each head's candidate bound from its sample
-    tiles.  Here the sample tiles hold scaled-up keys, so the bound lands
-    above the k-th score and the candidate lists miss keys of the top k: the
-    select must notice (its count check), take the exact streaming path
-    (flagged FLAG_SLOW_SELECT, not an error) and still return the exact set."""
-    k = 2048
-    w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=1, k=k, dtype="bf16", seed=N + 3)
+def test_select_ties_split_across_ctas(dev, route):
+    """40 keys with one identical top score, spread over the runs of the
+    head's CTAs, and k = 19: the k-th value is shared, so the set is the 19
+    lowest-index keys of the 40 -- a run holding the 18th..20th takes only
+    part of its tied keys.  The split select does this on its fast path."""
+    B, N, Hkv, k = 1, 131072, 2, 19
+    w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=1, k=k, dtype="bf16", seed=77)
     x = synth.generate(w)
     t = _to(dev, x)
-    K = t["K"].clone()
-    for j0, j1 in _sample_tiles(N):
-        K[:, :, j0:j1] *= 3
+    rows = torch.arange(40) * 3000 + 7
+    K = _plant(t["K"], rows, 8 * _qbar_dir(t, Hkv))
     ws = sd.Workspace(dev)
     S = sd.score(t["q_route"], K, ws=ws).cpu().numpy()
-    sd.read_device_flags(ws)
     a = _route(route, t, K, k, ws=ws).cpu().numpy()
-    flags = sd.read_device_flags(ws)
-    assert flags == sd.FLAG_SLOW_SELECT
+    assert sd.read_device_flags(ws) == 0
+    ref = oracle.topk(S, k)
+    np.testing.assert_array_equal(a, ref)
+    np.testing.assert_array_equal(ref[0, 0], rows[:k].numpy())
+
+
+@pytest.mark.parametrize("route", ["select_kernel", "fused_step"])
+def test_select_boundary_bin_over_capacity(dev, route):
+    """4096 identical keys in one CTA's run score above every other key and
+    k = 2048 of them are taken: the boundary bin overflows that CTA's list,
+    so every CTA takes the exact streaming path (FLAG_SLOW_SELECT, not an
+    error), which returns the 2048 lowest indices; the next call on the same
+    workspace is back on the fast path."""
+    B, N, Hkv, k = 1, 131072, 2, 2048
+    w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=1, k=k, dtype="bf16", seed=78)
+    x = synth.generate(w)
+    t = _to(dev, x)
+    rows = torch.arange(4096) + 100
+    K = _plant(t["K"], rows, 8 * _qbar_dir(t, Hkv))
+    ws = sd.Workspace(dev)
+    S = sd.score(t["q_route"], K, ws=ws).cpu().numpy()
+    a = _route(route, t, K, k, ws=ws).cpu().numpy()
+    assert sd.read_device_flags(ws) == sd.FLAG_SLOW_SELECT
     np.testing.assert_array_equal(a, oracle.topk(S, k))
-    # the next call on the same workspace (state cleared) takes the fast path
     b = _route(route, t, t["K"], k, ws=ws).cpu().numpy()
     assert sd.read_device_flags(ws) == 0
-    S2 = oracle.scores(_f(x["q_route"]), _f(x["K"]))
-    assert_topk_within_band(b, S2, k)
+    assert_topk_within_band(b, oracle.scores(_f(x["q_route"]), _f(x["K"])), k)
+
+
+@pytest.mark.parametrize("route", ["select_kernel", "fused_step"])
+def test_select_whole_set_in_one_run(dev, route):
+    """Every key of head 0's top k lies in one CTA's run (a block of keys
+    shifted along the head's query direction): the select kernel keeps its
+    fast path with one CTA writing the whole set; the attention kernel,
+    which holds at most 2048 keys per CTA on chip, takes the streaming path
+    with equal shares once the run holds more.  Both return the exact set."""
+    B, N, Hkv = 1, 131072, 2
+    for k, slow in ((1500, False), (3000, True)):
+        w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=1, k=k, dtype="bf16",
+                         seed=79)
+        x = synth.generate(w)
+        t = _to(dev, x)
+        K = t["K"].clone()
+        K[:, :, 300:300 + 4000] += (10 * _qbar_dir(t, Hkv)).to(K.dtype)
+        ws = sd.Workspace(dev)
+        S = sd.score(t["q_route"], K, ws=ws).cpu().numpy()
+        a = _route(route, t, K, k, ws=ws).cpu().numpy()
+        want = sd.FLAG_SLOW_SELECT if (slow and route == "fused_step") else 0
+        assert sd.read_device_flags(ws) == want, (k, route)
+        np.testing.assert_array_equal(a, oracle.topk(S, k))
 
 
 @pytest.mark.parametrize("route", ["select_kernel", "fused_step"])
 def test_select_fast_path_on_the_decode_workloads(dev, route):
-    """On the decode workloads' distributions the sample bound holds: no head
-    falls back to the streaming select."""
-    for name in ("decode_32k", "decode_128k"):
+    """On the decode workloads' distributions no head falls back to the
+    streaming select."""
+    for name in ("decode_32k", "decode_128k", "batched_16x64k"):
         w = synth.WORKLOADS[name]
         x = synth.generate(w)
         t = _to(dev, x)
@@ -638,12 +691,15 @@ def test_kv_append_then_decode(dev, dtype, d):
         assert_attn_close(o_gpu, l_gpu, o_ref, l_ref, dtype)
 
 
-@pytest.mark.parametrize("mode", ["topk", "threshold"])
-def test_decode_step_graph_equals_eager_step(dev, mode):
+@pytest.mark.parametrize("mode,dtype", [("topk", "bf16"), ("threshold", "bf16"),
+                                        ("topk", "f32")])
+def test_decode_step_graph_equals_eager_step(dev, mode, dtype):
     """The captured step with its host transfers returns, for each new
     query written into its pinned input views, exactly what the eager step
-    returns."""
-    w = synth.custom(B=2, N=5000, Hq=8, Hkv=2, d=128, L=3, k=100, dtype="bf16", seed=17,
+    returns: on the fused kernels with every result written straight into
+    the mapped host buffer (bf16), and on separate routing and attention
+    kernels (fp32)."""
+    w = synth.custom(B=2, N=5000, Hq=8, Hkv=2, d=128, L=3, k=100, dtype=dtype, seed=17,
                      heavy=8, mode=mode, cap=5000)
     x = synth.generate(w)
     K, V = x["K"].to(dev), x["V"].to(dev)
@@ -653,6 +709,7 @@ def test_decode_step_graph_equals_eager_step(dev, mode):
                                                    90, 100)).to(dev), cap=w.cap)
     g = sd.DecodeStepGraph(K, V, w.L, w.Hq, ws=sd.Workspace(dev), **kw)
     assert g.mapped_out       # torch's pinned buffers are mapped under unified addressing
+    assert g.fused == (dtype == "bf16") and g.results_direct == g.fused
     assert g.h2d_bytes >= (w.B * w.Hq * w.d + w.L * w.B * w.Hq * w.d) * 2
     for qr, ql in variants:
         g.q_route_host.copy_(qr)

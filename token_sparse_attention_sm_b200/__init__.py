@@ -49,7 +49,8 @@ EXPORTED_SYMBOLS = (
     "sparse_route_topk_static", "sparse_decode_step_grouped", "sparse_kv_append",
     "sparse_louver_sizes", "sparse_louver_build", "sparse_louver_route_threshold",
     "sparse_selftest_bounded_wait", "sparse_louver_decode_step",
-    "sparse_pointer_device_usable", "sparse_graph_launch",
+    "sparse_pointer_device_usable", "sparse_graph_launch", "sparse_decode_step_join",
+    "sparse_decode_step_fused",
 )
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
@@ -103,6 +104,9 @@ def load():
                                          SZ, P]),
             "sparse_decode_step": (I32, [SH, I32, P, P, P, P, I32, P, I32, P, P,
                                          P, P, P, SZ, P]),
+            "sparse_decode_step_join": (I32, [SH, I32, P, P, P, P, I32, P, I32, P, P,
+                                              P, P, P, SZ, P, P]),
+            "sparse_decode_step_fused": (I32, [SH, I32, I32, I32, ctypes.POINTER(I32)]),
             "sparse_read_device_status": (I32, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
             "sparse_route_topk_static": (I32, [SH, P, P, I32, P, P]),
             "sparse_decode_step_grouped": (I32, [SH, I32, I32, P, P, P, P, I32, P, I32,
@@ -450,16 +454,34 @@ def attn_gather(q, K, V, idx, count=None, ws: Workspace | None = None,
     return out, lse
 
 
+def decode_step_fused(B: int, N: int, Hq: int, Hkv: int, d: int, dtype, L: int,
+                      k: int | None = None, cap: int | None = None) -> bool:
+    """Whether decode_step on this shape (top-k with ``k``, threshold with
+    ``cap``) runs on the fused kernels (the routing scan, then one kernel
+    that selects and attends), where idx, count and out are write-only."""
+    topk = k is not None
+    sh = _shape(B, N, Hq, Hkv, d, dtype)
+    f = ctypes.c_int32(0)
+    _check(load().sparse_decode_step_fused(ctypes.byref(sh), int(L), int(k) if topk else 0,
+                                           0 if topk else int(cap), ctypes.byref(f)),
+           "decode_step_fused")
+    return bool(f.value)
+
+
 def decode_step(q_route, q_layers, K, V, k: int | None = None, tau=None,
                 cap: int | None = None, ws: Workspace | None = None,
                 check: bool = True, out=None, idx=None, count=None, lse=None,
-                return_lse: bool = True, n: int | None = None):
+                return_lse: bool = True, n: int | None = None, layers_ready=None):
     """One fused decode step: route once, attend L layers over that set.
 
     Top-k mode with ``k``; threshold mode with ``tau`` [B,Hkv] and ``cap``.
     The cache is the first n rows of K and V (default: all rows).
     Returns dict(idx, count, out, lse).  Preallocated outputs may be passed
-    to keep a timing loop free of allocations."""
+    to keep a timing loop free of allocations.  ``layers_ready`` (a
+    torch.cuda.Event): the attention waits for it, the routing does not --
+    for q_layers still being copied on another stream.  When the step runs
+    on the fused kernels (decode_step_fused), idx and count may also be
+    mapped pinned host memory (they are only written)."""
     _need_cuda(q_route, q_layers, K, V, tau)
     B, Ncap, Hq, Hkv, d = _dims_qk(q_route, K)
     N = _length(Ncap, n)
@@ -471,9 +493,11 @@ def decode_step(q_route, q_layers, K, V, k: int | None = None, tau=None,
     if topk == (tau is not None):
         raise ValueError("give exactly one of k or tau")
     stride = int(k) if topk else int(cap)
-    _need_result(idx, (B, Hkv, stride), torch.int32, "idx")
+    fused = decode_step_fused(B, N, Hq, Hkv, d, q_route.dtype, L, k=k if topk else None,
+                              cap=None if topk else cap)
+    _need_result(idx, (B, Hkv, stride), torch.int32, "idx", host_ok=fused)
     if not topk:
-        _need_result(count, (B, Hkv), torch.int32, "count")
+        _need_result(count, (B, Hkv), torch.int32, "count", host_ok=fused)
     _need_result(lse, (L, B, Hq), torch.float32, "lse", host_ok=True)
     if not topk:
         _need_tau(tau, (B, Hkv))
@@ -490,10 +514,11 @@ def decode_step(q_route, q_layers, K, V, k: int | None = None, tau=None,
     if lse is None and return_lse:
         lse = torch.empty((L, B, Hq), dtype=torch.float32, device=dev)
     tau_t = None if topk else tau.float().contiguous()
-    _check(load().sparse_decode_step(
+    ev = None if layers_ready is None else ctypes.c_void_p(layers_ready.cuda_event)
+    _check(load().sparse_decode_step_join(
         ctypes.byref(sh), L, _ptr(q_route), _ptr(q_layers), _ptr(K), _ptr(V),
         int(k) if topk else 0, _ptr(tau_t), 0 if topk else int(cap), _ptr(idx),
-        _ptr(count), _ptr(out), _ptr(lse), _ptr(buf), buf.numel(), _stream()),
+        _ptr(count), _ptr(out), _ptr(lse), _ptr(buf), buf.numel(), _stream(), ev),
         "decode_step")
     if check:
         read_device_status(w)
@@ -704,12 +729,15 @@ class DecodeStepGraph:
     decode step (top-k with ``k``, or threshold with a device ``tau`` [B,Hkv]
     and ``cap``) over the cache K, V as one graph launch: the routing query is
     copied in and routing starts while the layers' queries travel on a second
-    stream (joined before the attention); the attention writes its outputs
-    straight into ``out_host`` when the pinned buffer is mapped into the
-    device's address space (``mapped_out``), while the set (and counts)
-    travel back on the second stream; otherwise outputs and set are copied
-    back together after the attention.  With ``index`` (a LouverIndex of K) and
-    threshold mode the step routes through the index.  ``replay()`` enqueues a step on ``stream`` (a new stream by
+    stream (joined before the attention).  When the pinned buffer is mapped
+    into the device's address space (``mapped_out``) the attention writes its
+    outputs straight into ``out_host``; on the fused kernels (``fused``: the
+    routing scan, then one select + attention kernel) it writes the set (and
+    counts) there too (``results_direct``), so nothing is copied back; on
+    separate routing and attention kernels the set travels back on the second
+    stream while the attention runs.  Without a mapping, outputs and set are
+    copied back together after the attention.  With ``index`` (a LouverIndex
+    of K) and threshold mode the step routes through the index.  ``replay()`` enqueues a step on ``stream`` (a new stream by
     default; graphs that share a workspace must use one stream),
     ``synchronize()`` waits for it, calling the object does both.  The device
     status is checked once after the warm-up step (use
@@ -780,10 +808,24 @@ class DecodeStepGraph:
 
         self.mapped_out = device_usable(self.out_host)
         out_dst = self.out_host if self.mapped_out else out
+        # on the fused kernels the step only writes its set, counts and
+        # outputs: with mapped host buffers all of them go straight to the host
+        self.fused = index is None and decode_step_fused(
+            B, _length(K.shape[2], n), Hq, Hkv, d, dt, L, k=k if topk else None,
+            cap=None if topk else cap)
+        direct = self.fused and self.mapped_out
+        self.results_direct = direct
 
         def attend():
             attn_gather(q_layers, K, V, idx, count=count, ws=self.ws, check=False,
                         return_lse=False, out=out_dst, n=n)
+
+        def fused_step(layers_ready):
+            decode_step(q_route, q_layers, K, V, k=k if topk else None,
+                        tau=None if topk else tau, cap=None if topk else cap, ws=self.ws,
+                        check=False, out=out_dst, idx=self.idx_host if direct else idx,
+                        count=(self.count_host if direct else count) if not topk else None,
+                        return_lse=False, n=n, layers_ready=layers_ready)
 
         # byte ranges of the packed buffers: [q_route | q_layers], [out | idx (| count)]
         qr_end = in_offs[1]
@@ -800,6 +842,14 @@ class DecodeStepGraph:
             with torch.cuda.stream(self.side):
                 self.dev_in[qr_end:].copy_(self.host_in[qr_end:], non_blocking=True)
                 ev[1].record(self.side)
+            if self.fused:
+                # routing, then (once the layers' queries are in) the fused
+                # select + attention; results back after it unless written
+                # to the host directly
+                fused_step(ev[1])
+                if not direct:
+                    self.host_out[back:].copy_(self.dev_out[back:], non_blocking=True)
+                return
             route()
             if self.mapped_out:
                 ev[2].record(main)

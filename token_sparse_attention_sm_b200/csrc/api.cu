@@ -15,10 +15,8 @@
 //                  -- these three must be zero between calls; they sit at
 //                  fixed offsets for up to 256 heads, so calls of different
 //                  shapes sharing one workspace never put other data there
-//   cand counts    list lengths [B*Hkv][head_ctas] uint32, then the scan
-//                  CTAs covering each head [max(B*Hkv, 256)] (rewritten by
-//                  every top-k scan; head_ctas: the CTAs a head can span)
-//   cand lists     [B*Hkv][head_ctas][4096] (key, index) pairs
+//   cand bits      [B*Hkv][ceil(N/32)] uint32: the routing scan's candidate
+//                  bitmap (rewritten by every top-k scan)
 //   scores         fp32 S [B,Hkv,N]; threshold routing keeps its per-head
 //                  bitmaps [B*Hkv][ceil(N/32)] here
 //   attn           fp32 attention split partials (fp32 inputs only)
@@ -47,18 +45,14 @@ constexpr size_t kSelftestOff = 64;  // a header word no kernel writes
 constexpr int kHistMinRows = 256;
 
 struct Layout {
-  size_t hist_off, smp_off, smp_cnt_off, cnt_off, list_off, scores_off, attn_off, total;
+  size_t hist_off, scores_off, attn_off, total;
 };
 
 Layout layout(const Shape &s, int stride, int L) {
   const size_t rows = (size_t)(s.BH() > kHistMinRows ? s.BH() : kHistMinRows);
   Layout l;
   l.hist_off = kHeader;
-  l.smp_off = l.hist_off + rows * kHistBins * sizeof(uint32_t);
-  l.smp_cnt_off = l.smp_off + rows * kHistBins * sizeof(uint32_t);
-  l.cnt_off = l.smp_cnt_off + align_up(rows * sizeof(uint32_t), 256);
-  l.list_off = l.cnt_off + align_up(cand_count_bytes(s) + rows * 4, 256);
-  l.scores_off = l.list_off + align_up(cand_list_bytes(s), 256);
+  l.scores_off = l.hist_off + rows * kHistBins * sizeof(uint32_t);
   l.attn_off = l.scores_off + align_up((size_t)s.BH() * s.N * sizeof(float), 256);
   l.total = l.attn_off + align_up(attn_workspace_bytes(s, L, stride), 256);
   return l;
@@ -114,30 +108,13 @@ uint32_t *hist_ptr(void *ws, const Layout &l) { return at<uint32_t>(ws, l.hist_o
 float *scores_ptr(void *ws, const Layout &l) { return at<float>(ws, l.scores_off); }
 void *attn_ptr(void *ws, const Layout &l) { return at<char>(ws, l.attn_off); }
 
-// The candidate-list plan of a top-k routing call (false: no lists).
-bool cand_for(const Shape &s, int k, void *ws, const Layout &l, CandArgs *cand) {
-  DeviceInfo di;
-  if (device_info(&di) != cudaSuccess) return false;
-  if (!plan_cand(s, k, di.sm_count, cand)) return false;
-  cand->lists = at<uint64_t>(ws, l.list_off);
-  cand->counts = at<uint32_t>(ws, l.cnt_off);
-  cand->nspan = at<uint32_t>(ws, l.cnt_off + cand_count_bytes(s));
-  cand->smp_hist = at<uint32_t>(ws, l.smp_off);
-  cand->smp_cnt = at<uint32_t>(ws, l.smp_cnt_off);
-  return true;
-}
-
-// A1 + A2 (top-k): the scan (with candidate lists where they apply), then the
-// select kernel.
+// A1 + A2 (top-k): the scan (scores and histogram), then the split select.
 cudaError_t route_topk_any(const Shape &s, const void *q, const void *K, int k, int *idx,
                            void *ws, const Layout &l, cudaStream_t st) {
   float *S = scores_ptr(ws, l);
   uint32_t *hist = hist_ptr(ws, l);
-  CandArgs cand{};
-  const bool lists = cand_for(s, k, ws, l, &cand);
-  cudaError_t e = launch_score(s, q, K, S, hist, lists ? &cand : nullptr, status_word(ws), st);
-  if (e == cudaSuccess)
-    e = launch_select_cand(s, S, k, idx, hist, lists ? &cand : nullptr, status_word(ws), st);
+  cudaError_t e = launch_score(s, q, K, S, hist, status_word(ws), st);
+  if (e == cudaSuccess) e = launch_select_split(s, S, k, idx, hist, status_word(ws), st);
   return e;
 }
 
@@ -211,29 +188,35 @@ sparse_status_t check_decode_args(const Shape &s, int32_t L, const void *q_route
 // whose shape allows it finish the routing inside the attention kernel (the
 // scan, then one kernel); the others run the select (or the threshold
 // compaction) as a kernel of its own before the attention.
+// layers_ready (may be null): an event the attention waits on after the
+// routing is enqueued, so the layers' queries may still be in flight while
+// the routing runs.
 cudaError_t decode_step_enqueue(const Shape &s, int L, const void *q_route,
                                 const void *q_layers, const void *K, const void *V, int k,
                                 const float *tau, int cap, int *idx, int *count, void *out,
-                                float *lse, void *ws, const Layout &l, cudaStream_t st) {
+                                float *lse, void *ws, const Layout &l, cudaStream_t st,
+                                cudaEvent_t layers_ready) {
   const bool topk = k > 0;
   const int stride = topk ? k : cap;
   uint32_t *status = status_word(ws);
   const bool fused = fused_route_ok(s, L, stride);
+  auto join = [&]() {
+    return layers_ready ? cudaStreamWaitEvent(st, layers_ready, 0) : cudaSuccess;
+  };
   cudaError_t e;
   if (topk && fused) {
     float *S = scores_ptr(ws, l);
     uint32_t *hist = hist_ptr(ws, l);
-    CandArgs cand{};
-    const bool lists = cand_for(s, k, ws, l, &cand);
-    e = launch_score(s, q_route, K, S, hist, lists ? &cand : nullptr, status, st);
+    e = launch_score(s, q_route, K, S, hist, status, st);
+    if (e == cudaSuccess) e = join();
     if (e == cudaSuccess)
-      e = launch_route_attn_topk(s, L, q_layers, K, V, k, S, hist, lists ? &cand : nullptr, idx,
-                                 out, lse, status, st);
+      e = launch_route_attn_topk(s, L, q_layers, K, V, k, S, hist, idx, out, lse, status, st);
     return e;
   }
   if (!topk && fused) {
     uint32_t *bits = reinterpret_cast<uint32_t *>(scores_ptr(ws, l));
     e = launch_threshold_mark(s, q_route, K, tau, bits, status, st);
+    if (e == cudaSuccess) e = join();
     if (e == cudaSuccess)
       e = launch_route_attn_threshold(s, L, q_layers, K, V, bits, cap, idx, count, out, lse,
                                       status, st);
@@ -244,6 +227,7 @@ cudaError_t decode_step_enqueue(const Shape &s, int L, const void *q_route,
   } else {
     e = route_threshold_any(s, q_route, K, tau, cap, idx, count, ws, l, st);
   }
+  if (e == cudaSuccess) e = join();
   if (e == cudaSuccess)
     e = launch_attn(s, L, q_layers, K, V, idx, stride, topk ? nullptr : count, stride, out,
                     lse, attn_ptr(ws, l), status, st);
@@ -302,8 +286,8 @@ sparse_status_t sparse_score(const sparse_shape_t *shape, const void *q,
   if (!sd::aligned(q, 16) || !sd::aligned(K, 16) || !sd::aligned(S, 16))
     return SPARSE_ERR_INVALID_ARG;
   if ((r = sd::check_ws(s, 1, 1, ws, ws_bytes)) != SPARSE_OK) return r;
-  return sd::from_cuda(sd::launch_score(s, q, K, S, nullptr, nullptr, sd::status_word(ws),
-                                        static_cast<cudaStream_t>(stream)));
+  return sd::from_cuda(
+      sd::launch_score(s, q, K, S, nullptr, sd::status_word(ws), static_cast<cudaStream_t>(stream)));
 }
 
 sparse_status_t sparse_select_topk(const sparse_shape_t *shape,
@@ -402,6 +386,16 @@ sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
                                    int32_t *idx, int32_t *count, void *out,
                                    float *lse, void *ws, size_t ws_bytes,
                                    void *stream) {
+  return sparse_decode_step_join(shape, L, q_route, q_layers, K, V, k, tau, cap, idx, count, out,
+                                 lse, ws, ws_bytes, stream, nullptr);
+}
+
+sparse_status_t sparse_decode_step_join(const sparse_shape_t *shape, int32_t L,
+                                        const void *q_route, const void *q_layers,
+                                        const void *K, const void *V, int32_t k,
+                                        const float *tau, int32_t cap, int32_t *idx,
+                                        int32_t *count, void *out, float *lse, void *ws,
+                                        size_t ws_bytes, void *stream, void *layers_ready) {
   Shape s;
   sparse_status_t r = sd::check_shape(shape, &s);
   if (r != SPARSE_OK) return r;
@@ -412,7 +406,19 @@ sparse_status_t sparse_decode_step(const sparse_shape_t *shape, int32_t L,
   if ((r = sd::check_ws(s, stride, L, ws, ws_bytes)) != SPARSE_OK) return r;
   return sd::from_cuda(sd::decode_step_enqueue(s, L, q_route, q_layers, K, V, k, tau, cap, idx,
                                                count, out, lse, ws, sd::layout(s, stride, L),
-                                               static_cast<cudaStream_t>(stream)));
+                                               static_cast<cudaStream_t>(stream),
+                                               static_cast<cudaEvent_t>(layers_ready)));
+}
+
+sparse_status_t sparse_decode_step_fused(const sparse_shape_t *shape, int32_t L, int32_t k,
+                                         int32_t cap, int32_t *fused) {
+  Shape s;
+  sparse_status_t r = sd::check_shape(shape, &s);
+  if (r != SPARSE_OK) return r;
+  if (!fused || L < 1 || k < 0 || (k == 0 && cap < 1) || (k > 0 && k > s.N))
+    return SPARSE_ERR_INVALID_ARG;
+  *fused = sd::fused_route_ok(s, L, k > 0 ? k : cap) ? 1 : 0;
+  return SPARSE_OK;
 }
 
 sparse_status_t sparse_decode_step_grouped(const sparse_shape_t *shape, int32_t L, int32_t R,
@@ -444,7 +450,7 @@ sparse_status_t sparse_decode_step_grouped(const sparse_shape_t *shape, int32_t 
         static_cast<const char *>(q_layers) + (size_t)l0 * qsz, K, V, k,
         tau ? tau + (size_t)g * s.BH() : nullptr, cap, idx + (size_t)g * s.BH() * stride,
         count ? count + (size_t)g * s.BH() : nullptr, static_cast<char *>(out) + (size_t)l0 * qsz,
-        lse ? lse + (size_t)l0 * s.B * s.Hq : nullptr, ws, l, st);
+        lse ? lse + (size_t)l0 * s.B * s.Hq : nullptr, ws, l, st, nullptr);
   }
   return sd::from_cuda(e);
 }

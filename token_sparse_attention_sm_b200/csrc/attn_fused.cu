@@ -13,15 +13,20 @@
 // key order), in one of three ways:
 //  * given sets (sparse_attn_gather): from the caller's idx rows, a chunk at
 //    a time;
-//  * top-k routing (sparse_decode_step): every CTA of the head runs the exact
-//    select of topk_cand.cuh on the routing scan's histogram and candidate
-//    lists, keeps its own run on chip and writes it to the caller's idx row;
+//  * top-k routing (sparse_decode_step): the head's CTAs run the split
+//    select of topk_split.cuh on the routing scan's histogram and score row
+//    -- each classifies its own run of the row, the boundary bin's keys are
+//    exchanged through distributed shared memory -- and each keeps the
+//    selected keys of its own run on chip (their positions in the set come
+//    with them) and writes them to the caller's idx row; after one more
+//    cluster barrier each CTA takes an equal share of the set's positions,
+//    reading the indices from their owners' lists, so the CTAs run equal
+//    numbers of chunks and split the set exactly as the gather call does;
 //  * threshold routing: every CTA counts the marking scan's bitmap of keys
 //    with score >= tau (Louver summary, 1. 半空間範囲検索への帰着) and keeps
-//    its run of the ascending set; rank 0 writes the count.
-// The select is repeated by every CTA of the head instead of being shared:
-// it reads a few tens of KB from L2, and the repetition saves a kernel
-// boundary and a round trip of the set through global memory.
+//    an equal share of the ascending set; rank 0 writes the count.
+// Either way the set never makes a round trip through global memory before
+// the attention, and no kernel boundary separates the select from it.
 //
 // Then, per chunk of up to 128 keys:
 //  1. 16-byte async copies gather the chunk's K and V rows straight into
@@ -57,7 +62,7 @@
 
 #include "common.cuh"
 #include "internal.h"
-#include "topk_cand.cuh"
+#include "topk_split.cuh"
 
 namespace sd {
 namespace {
@@ -72,8 +77,8 @@ constexpr int kChunkTiles = 2;
 constexpr int kChunkKeys = kTileN * kChunkTiles;
 constexpr int kTmemCols = 256;          // S (128 columns) + O (d <= 128 columns)
 constexpr int kMaxSplits = 16;
-constexpr int kMaxPer = 1024;           // keys of one split held on chip (routing modes)
-constexpr int kSelBitmapWords = 4096;   // the fused select's bitmap: N <= 131072
+constexpr int kMaxPer = 2048;           // keys of one split held on chip (routing modes)
+static_assert(kMaxSplits == kTsMaxSplits, "a head's cluster is the select's cluster");
 constexpr int kMaxDevices = 64;
 
 constexpr int cmax_i(int a, int b) { return a > b ? a : b; }
@@ -91,19 +96,22 @@ struct FuCfg {
   static constexpr int kKPOff = kQBytes;
   static constexpr int kVOff = kKPOff + kKPBytes;
   static constexpr int kAttnBytes = kVOff + kVBytes;
-  static constexpr int kSelBytes = (int)tk_scratch_bytes(kSelBitmapWords);
+  static constexpr int kSelBytes = (int)ts_scratch_bytes();
   static constexpr int kBigBytes = cmax_i(kAttnBytes, kSelBytes);
   static constexpr int kStageBytes = kRows * (D + 4) * 4;  // merge partials
   static_assert(kStageBytes <= kBigBytes, "merge staging fits");
   // small area: barriers, TMEM slot, select bookkeeping, row reductions,
-  // validity flags, chunk indices, the split's indices
+  // validity flags, chunk indices, the split's indices, the partial (max,
+  // sum) pairs from the peers, and what the select shows its peers
   static constexpr int kSmallOff = (kBigBytes + 1023) / 1024 * 1024;
   static constexpr int kBarsOff = 0, kTmemSlotOff = 64, kTkOff = 128, kXredOff = 512;
   static constexpr int kKvalOff = kXredOff + kGroups * 128 * 4;
   static constexpr int kCidxOff = kKvalOff + kChunkKeys;
   static constexpr int kSidxOff = kCidxOff + kChunkKeys * 4;
   static constexpr int kMlOff = kSidxOff + kMaxPer * 4;  // [kMaxSplits][kRows] float2 from peers
-  static constexpr int kSmallBytes = kMlOff + kMaxSplits * kRows * 8;
+  static constexpr int kShowOff = kMlOff + kMaxSplits * kRows * 8;
+  static constexpr int kBookOff = kShowOff + (int)sizeof(TsShow);
+  static constexpr int kSmallBytes = kBookOff + (int)sizeof(TsBook);
   // merge scratch after the staged partials: [kFuThreads] float4 + [kFuThreads] float
   static constexpr int kRedOff = (kStageBytes + 15) / 16 * 16;
   static_assert(kRedOff + kFuThreads * 20 <= kBigBytes, "merge scratch fits");
@@ -194,26 +202,6 @@ __device__ __forceinline__ void l2_prefetch(const void *p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// Shared-memory address of `p` in the CTA of the cluster with rank `rank`,
-// and loads and stores through such an address.
-__device__ __forceinline__ uint32_t cl_addr(const void *p, int rank) {
-  uint32_t a;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
-  return a;
-}
-__device__ __forceinline__ float4 cl_ld4(uint32_t a) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(a)
-               : "memory");
-  return v;
-}
-__device__ __forceinline__ void cl_st2(uint32_t a, float2 v) {
-  asm volatile("st.shared::cluster.v2.f32 [%0], {%1,%2};" ::"r"(a), "f"(v.x), "f"(v.y)
-               : "memory");
-}
-
 // 2^x with the hardware approximation (ex2.approx.ftz: relative error about
 // 2^-22, results below 2^-126 flush to zero -- harmless for softmax weights).
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -249,8 +237,6 @@ struct FuArgs {
   uint32_t *hist;        // top-k: the scan's histograms (cleared here)
   const uint32_t *bits;  // threshold: the marking scan's bitmaps
   int k_or_cap;
-  int use_lists;
-  CandArgs cand;
 };
 
 enum : int { kModeIdx = 0, kModeTopk = 1, kModeThresh = 2 };
@@ -287,6 +273,8 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
   unsigned char *kval = small + C::kKvalOff;                      // [128] valid flags
   int *cidx = reinterpret_cast<int *>(small + C::kCidxOff);       // [128] chunk indices
   int *sidx = reinterpret_cast<int *>(small + C::kSidxOff);       // [kMaxPer] this split's keys
+  TsShow *show = reinterpret_cast<TsShow *>(small + C::kShowOff);
+  TsBook *book = reinterpret_cast<TsBook *>(small + C::kBookOff);
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -308,73 +296,80 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
   const uint32_t t_O = tmem + kChunkKeys;  // columns [128, 128 + D)
   const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
 
-  // ---- this split's share [lo, hi) of the head's set --------------------------
-  int cnt = 0;
+  // ---- this split's part [lo, lo + nmine) of the head's set ---------------------
+  int lo = 0, nmine = 0;
+  bool from_peers = false;  // the split's keys are read from their owners' lists
   int *orow = a.idx + (size_t)bh * a.stride;
-  if constexpr (kMode == kModeIdx) {
-    cnt = a.count ? min(max(a.count[bh], 0), a.stride) : a.stride;
-  } else if constexpr (kMode == kModeTopk) {
-    cnt = a.k_or_cap;
-  } else {
-    // threshold: the set is the marking scan's bitmap of the head
-    const int nw = (N + 31) / 32;
-    const uint32_t *words = a.bits + (size_t)bh * nw;
-    uint32_t n = 0;
-    for (int w = tid; w < nw; w += kFuThreads) n += __popc(words[w]);
-    uint32_t total;
-    tk_scan(n, tks, &total);
-    cnt = (int)min(total, (uint32_t)a.k_or_cap);
-    if (rank == 0 && qb == 0 && tid == 0) {
-      a.count[bh] = (int)total;
-      if (total > (uint32_t)a.k_or_cap) raise_flag(a.status, FLAG_CAPACITY);
-    }
-  }
-  const int per = (cnt + nsplit - 1) / nsplit;
-  const int lo = min(cnt, rank * per), hi = min(cnt, lo + per);
-  if constexpr (kMode != kModeIdx) {
-    auto emit = [&](uint32_t pos, uint32_t j) {
-      if (pos >= (uint32_t)lo && pos < (uint32_t)hi) {
-        sidx[pos - lo] = (int)j;
-        if (qb == 0) orow[pos] = (int)j;
-      }
+  if constexpr (kMode == kModeTopk) {
+    // keys known to be in the set early are prefetched into L2 by the CTA
+    // that will gather them, so the gather below finds its rows there
+    const size_t head_rows = (size_t)bh * a.kv_rows * D;
+    auto sure = [&](uint32_t j) {
+      l2_prefetch(a.K + head_rows + (size_t)j * D, D * 2);
+      l2_prefetch(a.V + head_rows + (size_t)j * D, D * 2);
     };
-    if constexpr (kMode == kModeTopk) {
-      // keys known to be in the set early are prefetched into L2, each split
-      // taking every nsplit-th of them, so the gather below finds its rows
-      // there
-      const size_t head_rows = (size_t)bh * a.kv_rows * D;
-      auto sure = [&](uint32_t j) {
-        if ((int)(j % (uint32_t)nsplit) == rank) {
-          l2_prefetch(a.K + head_rows + (size_t)j * D, D * 2);
-          l2_prefetch(a.V + head_rows + (size_t)j * D, D * 2);
+    auto emit = [&](uint32_t i, uint32_t pos, uint32_t j) {
+      sidx[i] = (int)j;
+      if (qb == 0) orow[pos] = (int)j;
+    };
+    const TsOut part = ts_select(a.S + (size_t)bh * N, N, (uint32_t)a.k_or_cap,
+                                 a.hist + (size_t)bh * kHistBins, rank, nsplit, kMaxPer, base,
+                                 show, book, tks, a.status, emit, sure);
+    __syncthreads();  // the split's indices are on chip; the select's scratch is free
+    if (part.split && nsplit > 1) {
+      // the runs hold unequal parts of the set: every CTA attends over an
+      // equal share instead (so each runs the same number of chunks), its
+      // indices read from their owners' lists chunk by chunk once every
+      // list is complete; the owners keep their lists until the merge's
+      // first cluster barrier
+      cluster_sync_all();
+      const int per = (a.k_or_cap + nsplit - 1) / nsplit;
+      lo = min(a.k_or_cap, rank * per);
+      nmine = min(a.k_or_cap, lo + per) - lo;
+      from_peers = true;
+    } else {
+      lo = (int)part.lo;
+      nmine = (int)part.n;
+    }
+    // with one split this CTA was the head's only reader: clear the scan's
+    // histogram for the next call now (with several, after the merge's first
+    // cluster barrier)
+    if (nsplit == 1)
+      for (int i = tid; i < kHistBins; i += kFuThreads) a.hist[(size_t)bh * kHistBins + i] = 0u;
+  } else {
+    int cnt = 0;
+    if constexpr (kMode == kModeIdx) {
+      cnt = a.count ? min(max(a.count[bh], 0), a.stride) : a.stride;
+    } else {
+      // threshold: the set is the marking scan's bitmap of the head
+      const int nw = (N + 31) / 32;
+      const uint32_t *words = a.bits + (size_t)bh * nw;
+      uint32_t n = 0;
+      for (int w = tid; w < nw; w += kFuThreads) n += __popc(words[w]);
+      uint32_t total;
+      tk_scan(n, tks, &total);
+      cnt = (int)min(total, (uint32_t)a.k_or_cap);
+      if (rank == 0 && qb == 0 && tid == 0) {
+        a.count[bh] = (int)total;
+        if (total > (uint32_t)a.k_or_cap) raise_flag(a.status, FLAG_CAPACITY);
+      }
+    }
+    const int per = (cnt + nsplit - 1) / nsplit;
+    lo = min(cnt, rank * per);
+    const int hi = min(cnt, lo + per);
+    nmine = hi - lo;
+    if constexpr (kMode == kModeThresh) {
+      auto emit = [&](uint32_t pos, uint32_t j) {
+        if (pos >= (uint32_t)lo && pos < (uint32_t)hi) {
+          sidx[pos - lo] = (int)j;
+          if (qb == 0) orow[pos] = (int)j;
         }
       };
-      const uint32_t n = tk_select(a.S + (size_t)bh * N, N, (uint32_t)cnt,
-                                   a.hist + (size_t)bh * kHistBins, a.cand, a.use_lists != 0,
-                                   bh, base, kSelBitmapWords, tks, a.status, emit, sure,
-                                   (uint32_t)lo, (uint32_t)hi);
-      if (rank == 0 && qb == 0 && tid == 0 && n != (uint32_t)cnt)
-        raise_flag(a.status, FLAG_INTERNAL);
-    } else {
       const int nw = (N + 31) / 32;
       tk_bitmap_emit(a.bits + (size_t)bh * nw, nw, tks, emit, (uint32_t)lo, (uint32_t)hi);
-    }
-    __syncthreads();  // the split's indices are on chip; the select's scratch is free
-    if constexpr (kMode == kModeTopk) {
-      // with one split this CTA was the head's only reader: clear the scan's
-      // by-products for the next call now (with several, after the merge's
-      // first cluster barrier)
-      if (nsplit == 1) {
-        for (int i = tid; i < kHistBins; i += kFuThreads) a.hist[(size_t)bh * kHistBins + i] = 0u;
-        if (a.use_lists) {
-          for (int i = tid; i < kHistBins; i += kFuThreads)
-            a.cand.smp_hist[(size_t)bh * kHistBins + i] = 0u;
-          if (tid == 0) a.cand.smp_cnt[bh] = 0u;
-        }
-      }
+      __syncthreads();  // the split's indices are on chip
     }
   }
-  const int nmine = hi - lo;
   const size_t head_off = (size_t)bh * a.kv_rows * D;
 
   bool failed = false;
@@ -392,6 +387,26 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
       if (tid < kChunkKeys) cidx[tid] = tid < nk ? orow[lo + c0 + tid] : -1;
       __syncthreads();
       cix = cidx;
+    } else if constexpr (kMode == kModeTopk) {
+      if (from_peers) {
+        if (tid < kChunkKeys) {
+          int j = -1;
+          if (tid < nk) {
+            const uint32_t pos = (uint32_t)(lo + c0 + tid);
+            int o = 0, hi2 = nsplit - 1;  // the last CTA whose part starts at or before pos
+            while (o < hi2) {
+              const int mid = (o + hi2 + 1) >> 1;
+              if (book->part_lo[mid] <= pos) o = mid;
+              else hi2 = mid - 1;
+            }
+            const uint32_t i = pos - book->part_lo[o];
+            j = o == rank ? sidx[i] : (int)cl_ld_u32(cl_addr(sidx + i, o));
+          }
+          cidx[tid] = j;
+        }
+        __syncthreads();
+        cix = cidx;
+      }
     }
     if (c0 == 0) {
       // the query block (rows beyond M zero), in the same copy group as K
@@ -669,14 +684,8 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
   }
   cluster.sync();  // every split's partial is staged and its (max, sum) delivered
   if constexpr (kMode == kModeTopk) {
-    if (rank == 0) {
+    if (rank == 0)
       for (int i = tid; i < kHistBins; i += kFuThreads) a.hist[(size_t)bh * kHistBins + i] = 0u;
-      if (a.use_lists) {
-        for (int i = tid; i < kHistBins; i += kFuThreads)
-          a.cand.smp_hist[(size_t)bh * kHistBins + i] = 0u;
-        if (tid == 0) a.cand.smp_cnt[bh] = 0u;
-      }
-    }
   }
   // merge rows lr = rank, rank + nsplit, ...: thread = (peer group q, row
   // slot, float4 chunk); the weights come from the (max, sum) pairs on chip,
@@ -714,7 +723,7 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
               const int r = r0 + u * qg;
               if (r < nsplit) {
                 const float2 ml = ml_recv[r * C::kRows + lr];
-                const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - mx);
+                const float w = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - mx);
                 ls += ml.y * w;
                 acc.x += w * v[u].x;
                 acc.y += w * v[u].y;
@@ -934,20 +943,18 @@ cudaError_t launch_attn_fused(const Shape &s, int L, const void *q, const void *
 }
 
 bool fused_route_ok(const Shape &s, int L, int k_or_cap) {
-  return s.dtype == 1 && L * s.G() <= 128 && s.N <= kSelBitmapWords * 32 &&
+  return s.dtype == 1 && L * s.G() <= 128 && s.N <= kTsMaxWords * 32 &&
          (k_or_cap + kMaxPer - 1) / kMaxPer <= kMaxSplits;
 }
 
 cudaError_t launch_route_attn_topk(const Shape &s, int L, const void *q_layers, const void *K,
                                    const void *V, int k, const float *S, uint32_t *hist,
-                                   const CandArgs *cand, int *idx, void *out, float *lse,
-                                   uint32_t *status, cudaStream_t st) {
+                                   int *idx, void *out, float *lse, uint32_t *status,
+                                   cudaStream_t st) {
   FuArgs a = fu_base(s, L, q_layers, K, V, idx, k, nullptr, out, lse, status);
   a.S = S;
   a.hist = hist;
   a.k_or_cap = k;
-  a.use_lists = cand && cand->lists ? 1 : 0;
-  if (a.use_lists) a.cand = *cand;
   return launch_fu<kModeTopk>(a, s, k, st);
 }
 

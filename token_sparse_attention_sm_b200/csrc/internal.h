@@ -6,10 +6,13 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "route_cand.cuh"
 #include "sparse_decode.h"
 
 namespace sd {
+
+// Routing histogram rows: counts of the top 11 bits of the order-preserving
+// score key, per (sequence, KV head).
+constexpr int kHistBins = 2048;
 
 struct Shape {
   int B, N, Hq, Hkv, d, dtype;  // dtype: 0 = fp32, 1 = bf16
@@ -42,29 +45,18 @@ inline void add_pdl_attr(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attrs) {
 }
 
 // A1: S[b,h,j] for every key; one streaming pass over K.  hist (nullable):
-// [B*Hkv][2048] counts of the top 11 key bits, accumulated (must start zero).
-// cand (nullable): a plan from plan_cand with its list pointers -- the scan
-// then also draws the sample and fills the candidate lists (top-k routing).
+// [B*Hkv][kHistBins] counts of the top 11 key bits, accumulated (must start
+// zero).
 cudaError_t launch_score(const Shape &s, const void *q, const void *K, float *S, uint32_t *hist,
-                         const CandArgs *cand, uint32_t *status, cudaStream_t st);
+                         uint32_t *status, cudaStream_t st);
 // Keys per scan tile, and the scan's grid (one CTA per SM, at most one per tile).
 int scan_stage_keys(const Shape &s);
 int scan_grid(const Shape &s, int sm_count);
-// Fills the plan fields of cand (not the pointers) for top-k routing with
-// candidate lists; false when the lists do not apply to this shape and k.
-bool plan_cand(const Shape &s, int k, int sm_count, CandArgs *cand);
-// The workspace areas of the candidate lists and their lengths for a shape
-// (0 when lists never apply to it), and the CTAs a head can span.
-constexpr size_t kCandMaxListBytes = (size_t)512 << 20;
-int cand_head_ctas_of(const Shape &s);
-size_t cand_list_bytes(const Shape &s);
-size_t cand_count_bytes(const Shape &s);
-
-// A2 after the scan: one CTA per head selects the exact top-k from the
-// scan's histogram and candidate lists (cand nullable: from the score rows)
-// and clears what it consumed.
-cudaError_t launch_select_cand(const Shape &s, const float *S, int k, int *idx, uint32_t *hist,
-                               const CandArgs *cand, uint32_t *status, cudaStream_t st);
+// A2 after the scan: one cluster per head selects the exact top-k from the
+// scan's score rows S and histogram hist (complete), writes idx
+// [B*Hkv][k] and clears hist.
+cudaError_t launch_select_split(const Shape &s, const float *S, int k, int *idx, uint32_t *hist,
+                                uint32_t *status, cudaStream_t st);
 
 // A2 / A2': selection from S.  k >= 1: top-k (tau ignored); k == 0:
 // threshold with tau and cap, count written.  idx rows have `stride`
@@ -87,15 +79,14 @@ cudaError_t launch_attn_fused(const Shape &s, int L, const void *q, const void *
                               const int *idx, int stride, const int *count, void *out, float *lse,
                               uint32_t *status, cudaStream_t st);
 // The tail of routing fused into the attention kernel (bf16, L*G <= 128,
-// N <= 131072, every split's keys on chip): top-k from the scan's
-// by-products (writes idx [B*Hkv][k], clears hist and the sample state), or
-// the threshold sets from the marking scan's bitmaps (writes idx rows of
-// `cap` and count).
+// N <= 131072, every split's keys on chip): top-k from the scan's score rows
+// and histogram (writes idx [B*Hkv][k], clears hist), or the threshold sets
+// from the marking scan's bitmaps (writes idx rows of `cap` and count).
 bool fused_route_ok(const Shape &s, int L, int k_or_cap);
 cudaError_t launch_route_attn_topk(const Shape &s, int L, const void *q_layers, const void *K,
                                    const void *V, int k, const float *S, uint32_t *hist,
-                                   const CandArgs *cand, int *idx, void *out, float *lse,
-                                   uint32_t *status, cudaStream_t st);
+                                   int *idx, void *out, float *lse, uint32_t *status,
+                                   cudaStream_t st);
 cudaError_t launch_route_attn_threshold(const Shape &s, int L, const void *q_layers,
                                         const void *K, const void *V, const uint32_t *bits,
                                         int cap, int *idx, int *count, void *out, float *lse,

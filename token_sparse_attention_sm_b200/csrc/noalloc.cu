@@ -94,7 +94,7 @@ extern "C" sparse_status_t sparse_route_topk_static(const sparse_shape_t *shape,
   // status word and this call's histogram rows must start at zero
   cudaError_t e = cudaMemsetAsync(
       base, 0, sd::kStaticHeader + (size_t)s.BH() * 2048 * sizeof(uint32_t), st);
-  if (e == cudaSuccess) e = sd::launch_score(s, q, K, S, hist, nullptr, status, st);
-  if (e == cudaSuccess) e = sd::launch_select_cand(s, S, k, idx, hist, nullptr, status, st);
+  if (e == cudaSuccess) e = sd::launch_score(s, q, K, S, hist, status, st);
+  if (e == cudaSuccess) e = sd::launch_select_split(s, S, k, idx, hist, status, st);
   return e == cudaSuccess ? SPARSE_OK : SPARSE_ERR_CUDA;
 }

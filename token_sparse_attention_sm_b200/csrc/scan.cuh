@@ -5,8 +5,9 @@
 // (CLSA article, section CLSAの仕組み).  A CTA owns a contiguous run of 32 KB
 // key tiles (tiles never straddle heads).  One producer thread streams them
 // into a shared-memory ring with 1-D bulk copies (cp.async.bulk + mbarrier
-// transaction counts, L2 evict-first: K is read once); four consumer warps
-// read them back with conflict-free 128-bit shared loads.  A warp handles 32
+// transaction counts, L2 evict-first: K is read once); two groups of four
+// consumer warps take alternate stages and read them back with
+// conflict-free 128-bit shared loads.  A warp handles 32
 // keys at a time: each lane loads 16 bytes of a row per round (rows are split
 // over LPK lanes), keeps one partial dot per round, and a transposing shuffle
 // reduction leaves one finished score per lane, stored as one coalesced
@@ -16,7 +17,6 @@
 #pragma once
 
 #include "common.cuh"
-#include "route_cand.cuh"
 
 namespace sd {
 namespace {
@@ -32,6 +32,11 @@ static_assert(kScanStages % kScanGroups == 0, "a stage belongs to one consumer g
 constexpr int kScanStageBytes = 32768;
 constexpr int kScanThreads = (kScanConsumerWarps + 1) * 32;  // + the copy-issuing warp
 constexpr int kScanBins = 2048;  // top 11 bits of the order-preserving key
+
+// First tile of scan CTA c (tiles are dealt in contiguous runs).
+__host__ __device__ inline long long scan_tile_begin(int c, long long total, int grid) {
+  return (long long)c * total / grid;
+}
 
 template <typename T, int D>
 struct ScoreCfg {
@@ -137,90 +142,24 @@ struct ScanOut {
   const float *tau;
 };
 
-// Shared-memory state of the candidate machinery (scan_tiles<..., kCand>).
-constexpr int kDeferCap = 16;  // tiles a consumer warp may scan before its head's bound is known
-struct CandShared {
-  volatile uint32_t bound[kCandSlots];  // 1 + bound bin of the head in slot s; 0 while unknown
-  volatile uint32_t consumers_done;     // consumer warps past their tile loop
-  int jpos[kCandSlots];                 // this CTA's place among the CTAs covering that head
-  uint32_t lcount[kCandSlots];          // entries appended to this CTA's list of that head
-  long long deferred[kScanConsumerWarps][kDeferCap];
-};
-
-// The order in which a CTA takes its tiles [t_begin, t_end): with sampling
-// on (stride > 0), first the sample tiles (tile u of a head with
-// u % stride == 0), then the others, each group ascending; otherwise plain
-// ascending order.  Producer and consumers walk identical sequences.  The
-// position is kept as (head, tile of the head) and stepped without any
-// division: the walk runs once per tile in the copy-issuing thread, where a
-// 64-bit division per tile is enough to slow the stream down.
-struct TileSeq {
-  int bh, u, us;        // current tile: head, tile of the head, u % stride
-  int bh0, u0, us0, n;  // the run's first tile and its length
-  int step, tph, stride, phase;
-  __device__ bool sample() const { return stride > 0 && us == 0; }
-  __device__ void move() {
-    ++u;
-    if (stride > 0 && ++us == stride) us = 0;
-    if (u == tph) {
+// A CTA's walk over its tiles [t_begin, t_end) in ascending order, kept as
+// (head, tile of the head) and stepped without any division: the walk runs
+// once per tile in the copy-issuing thread, where a 64-bit division per tile
+// is enough to slow the stream down.
+struct TileWalk {
+  int bh, u, tph;
+  __device__ void init(long long b, int tiles_per_head) {
+    tph = tiles_per_head;
+    bh = (int)(b / tph);
+    u = (int)(b - (long long)bh * tph);
+  }
+  __device__ void next() {
+    if (++u == tph) {
       u = 0;
-      us = 0;
       ++bh;
     }
   }
-  __device__ void restart() {
-    bh = bh0;
-    u = u0;
-    us = us0;
-    step = 0;
-  }
-  // to the next tile of the walk (the first one when called after restart
-  // with step == -1 semantics handled by init)
-  __device__ void advance() {
-    while (true) {
-      if (step + 1 >= n) {
-        if (phase == 0) {
-          phase = 1;
-          restart();
-          if (!sample()) return;
-          continue;
-        }
-        step = n;  // past the end
-        return;
-      }
-      ++step;
-      move();
-      if (phase == 0 ? sample() : !sample()) return;
-    }
-  }
-  __device__ void init(long long b, long long e, int tiles_per_head, int smp_stride) {
-    tph = tiles_per_head;
-    stride = smp_stride;
-    n = (int)(e - b);
-    bh0 = (int)(b / tph);
-    u0 = (int)(b - (long long)bh0 * tph);
-    us0 = stride > 0 ? u0 % stride : 0;
-    phase = stride > 0 ? 0 : 1;
-    restart();
-    if (n <= 0) return;
-    if (phase == 0 ? !sample() : sample()) advance();
-  }
 };
-
-// Append the keys of one 32-key warp tile that reach the bound bin to this
-// CTA's list of the head (one shared-memory counter update per warp; *cnt
-// counts every passing key, also those past the list's capacity).
-__device__ __forceinline__ void cand_append(uint64_t *list, uint32_t *cnt, bool pass,
-                                            uint32_t key, uint32_t j, int lane) {
-  const uint32_t m = __ballot_sync(0xffffffffu, pass);
-  if (m) {
-    uint32_t base = 0;
-    if (lane == 0) base = atomicAdd(cnt, (uint32_t)__popc(m));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    const uint32_t pos = base + __popc(m & ((1u << lane) - 1u));
-    if (pass && pos < (uint32_t)kCandListCap) list[pos] = ((uint64_t)key << 32) | j;
-  }
-}
 
 // One CTA's share of the scan: tiles [t_begin, t_end).  K holds kv_rows rows
 // per (sequence, KV head), the first N of them scanned.  Warps 0..7 consume
@@ -228,34 +167,26 @@ __device__ __forceinline__ void cand_append(uint64_t *list, uint32_t *cnt, bool 
 // warp 8 produces: its lane 0 issues the copies and waits for the last ones
 // to land, its other lanes (and any further warps) return at once.  Barriers
 // full/empty must be initialised (count 1 / kScanGroupWarps).
-//
-// kCand (top-k routing): sample tiles come first; their keys are counted in
-// the head's sample histogram (cand.smp_hist, then cand.smp_cnt with release
-// order).  On every other tile a consumer warp appends the keys whose top 11
-// bits reach its head's bound bin (cs->bound, published by the sample warp,
-// see score.cu) to its own list; a tile scanned while the bound is still
-// unknown is remembered and checked again from S at the end (cand_deferred).
-template <typename T, int D, int kSlots, bool kMark = false, bool kCand = false>
+template <typename T, int D, int kSlots, bool kMark = false>
 __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__restrict__ K,
                                            int N, int kv_rows, int Hq, int Hkv,
                                            int tiles_per_head, long long t_begin, long long t_end,
                                            int bh_first, float scale, unsigned char *ring,
                                            uint64_t *full, uint64_t *empty, ScanOut o,
-                                           const CandArgs &cand, CandShared *cs, int &ndef,
                                            uint32_t *status) {
+  const int nw = (N + 31) / 32;
   using C = ScoreCfg<T, D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = (int)(t_end - t_begin);
-  const int stride = kCand ? cand.smp_stride : 0;
   if (warp > kScanConsumerWarps) return;  // extra warps of a larger CTA idle here
   if (warp == kScanConsumerWarps) {
     // ---- producer: one thread issues the bulk copies -------------------------
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy();
-      TileSeq seq;
-      seq.init(t_begin, t_end, tiles_per_head, stride);
+      TileWalk seq;
+      seq.init(t_begin, tiles_per_head);
       int issued = 0;
-      for (int i = 0; i < ntiles; ++i, seq.advance()) {
+      for (int i = 0; i < ntiles; ++i, seq.next()) {
         const int s = i % kScanStages;
         if (i >= kScanStages &&
             !mbar_wait(&empty[s], ((i / kScanStages) - 1) & 1, status))
@@ -281,11 +212,10 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
   const int sub = lane % C::kLpk;  // which 16-byte slice of the row
   int cur_bh = -1;
   uint32_t tkey = 0;  // threshold marking: order key of the head's tau
-  const int nw = (N + 31) / 32;
   float qs[C::kEpl];
-  TileSeq seq;
-  seq.init(t_begin, t_end, tiles_per_head, stride);
-  for (int i = 0; i < ntiles; ++i, seq.advance()) {
+  TileWalk seq;
+  seq.init(t_begin, tiles_per_head);
+  for (int i = 0; i < ntiles; ++i, seq.next()) {
     const int s = i % kScanStages;
     if (s % kScanGroups != grp) continue;  // the other group's stage
     const int bh = seq.bh;
@@ -304,23 +234,6 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
     const unsigned char *stage = ring + (size_t)s * kScanStageBytes;
     float *Srow = kMark ? nullptr : o.S + (size_t)bh * N + j0;
     const int slot = bh - bh_first;
-    // candidate handling of this tile: sample, append with a known bound, or defer
-    bool sample = false;
-    uint32_t bound = 0;  // 1 + bound bin; 0: unknown
-    uint64_t *list = nullptr;
-    if constexpr (kCand) {
-      sample = seq.sample();
-      if (!sample && slot < kCandSlots) {
-        bound = cs->bound[slot];
-        if (bound) {
-          list = cand_list(cand, bh, cs->jpos[slot]);
-        } else if (lane == 0) {
-          if (ndef < kDeferCap) cs->deferred[warp][ndef] = (long long)bh * tiles_per_head + seq.u;
-        }
-        if (!bound) ++ndef;  // past kDeferCap the tile is simply not kept
-      }
-    }
-    uint32_t nsample = 0;
     for (int wt = wq; wt < C::kWarpTiles; wt += kScanGroupWarps) {
       const int key0 = wt * 32;
       if (key0 >= nk) break;
@@ -344,66 +257,12 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
               atomicAdd(&o.hist[(size_t)bh * kScanBins + bin], 1u);
           }
         }
-        if constexpr (kCand) {
-          if (sample) {
-            if (valid)
-              asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(
-                               cand.smp_hist + (size_t)bh * kScanBins + (key >> 21))
-                           : "memory");
-            nsample += __popc(__ballot_sync(0xffffffffu, valid));
-          } else if (list) {
-            cand_append(list, &cs->lcount[slot], valid && (key >> 21) + 1 >= bound, key,
-                        (uint32_t)(j0 + kk), lane);
-          }
-        }
       }
       if (__any_sync(0xffffffffu, valid && !isfinite(score)) && lane == 0)
         raise_flag(status, FLAG_NONFINITE);
     }
-    if constexpr (kCand) {
-      if (sample) {
-        // this warp's sample keys of the tile are counted: publish them
-        __threadfence();
-        __syncwarp();
-        if (lane == 0 && nsample)
-          asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(cand.smp_cnt + bh),
-                       "r"(nsample)
-                       : "memory");
-      }
-    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-  }
-}
-
-// Tiles a consumer warp scanned before its head's bound was known: check
-// their keys again from S (this warp's own earlier writes) once the bound is
-// there.  Tiles whose bound never became known are left out; the select then
-// finds the lists incomplete and reads the full score rows.
-template <typename T, int D>
-__device__ __forceinline__ void cand_deferred(const float *__restrict__ S, int N,
-                                              int tiles_per_head, int bh_first,
-                                              const CandArgs &cand, CandShared *cs, int ndef) {
-  using C = ScoreCfg<T, D>;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = 0; i < min(ndef, kDeferCap); ++i) {
-    const long long t = cs->deferred[warp][i];
-    const int bh = (int)(t / tiles_per_head);
-    const int slot = bh - bh_first;
-    const uint32_t bound = cs->bound[slot];
-    if (!bound) continue;
-    const int j0 = (int)(t % tiles_per_head) * C::kStageKeys;
-    const int nk = min(C::kStageKeys, N - j0);
-    uint64_t *list = cand_list(cand, bh, cs->jpos[slot]);
-    for (int wt = warp % kScanGroupWarps; wt < C::kWarpTiles; wt += kScanGroupWarps) {
-      const int key0 = wt * 32;
-      if (key0 >= nk) break;
-      const int kk = key0 + lane;
-      const bool valid = kk < nk;
-      const uint32_t key = valid ? order_key(S[(size_t)bh * N + j0 + kk]) : 0u;
-      cand_append(list, &cs->lcount[slot], valid && (key >> 21) + 1 >= bound, key,
-                  (uint32_t)(j0 + kk), lane);
-    }
   }
 }
 

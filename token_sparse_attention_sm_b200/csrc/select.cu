@@ -19,9 +19,9 @@
 //  * Each level builds a shared-memory histogram per CTA, one cluster
 //    barrier, and every CTA sums the C histograms through distributed shared
 //    memory.  (Routing calls, where the score scan has already counted the
-//    top 11 bits and kept candidate lists, select in select_cand.cu or in
-//    the fused attention kernel instead; this kernel serves selections from
-//    given scores and the Louver index build.)
+//    top 11 bits, select in select_split.cu or in the fused attention kernel
+//    instead; this kernel serves selections from given scores and the Louver
+//    index build.)
 //  * Compaction is order preserving: each warp owns a contiguous run of its
 //    CTA's slice and walks it 32 keys at a time; warp ballots and popcounts
 //    give positions, one more cluster barrier exchanges the per-CTA totals,
