@@ -6,17 +6,13 @@
 // caller's workspace, whose layout is
 //   [0, 4096)      header: device status word (uint32) at offset 0; offset
 //                  64: a word no kernel writes (the bounded-wait self-test
-//                  waits on it)
+//                  waits on it); [1024, 3072): the routing scan's tile claim
+//                  counters (zero between calls; the scan leaves them zero)
 //   hist           radix histogram [max(B*Hkv, 256)][2048] uint32 (scan ->
-//                  select; cleared after use)
-//   sample hist    [max(B*Hkv, 256)][2048] uint32 and sample counts
-//                  [max(B*Hkv, 256)] uint32 (the routing scan's sample;
-//                  cleared after use)
-//                  -- these three must be zero between calls; they sit at
-//                  fixed offsets for up to 256 heads, so calls of different
-//                  shapes sharing one workspace never put other data there
-//   cand bits      [B*Hkv][ceil(N/32)] uint32: the routing scan's candidate
-//                  bitmap (rewritten by every top-k scan)
+//                  select; cleared after use) -- it must be zero between
+//                  calls and sits at a fixed offset for up to 256 heads, so
+//                  calls of different shapes sharing one workspace never put
+//                  other data there
 //   scores         fp32 S [B,Hkv,N]; threshold routing keeps its per-head
 //                  bitmaps [B*Hkv][ceil(N/32)] here
 //   attn           fp32 attention split partials (fp32 inputs only)

@@ -44,6 +44,12 @@ inline void add_pdl_attr(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attrs) {
   ++cfg.numAttrs;
 }
 
+// The routing scan's tile claim counters live in the workspace header, at a
+// fixed word offset from the status word (which is the header's first word):
+// kScanCtrWord .. kScanCtrWord + 512, zero between calls.
+constexpr int kScanCtrWord = 256;  // byte offset 1024
+inline uint32_t *scan_counters(uint32_t *status) { return status + kScanCtrWord; }
+
 // A1: S[b,h,j] for every key; one streaming pass over K.  hist (nullable):
 // [B*Hkv][kHistBins] counts of the top 11 key bits, accumulated (must start
 // zero).

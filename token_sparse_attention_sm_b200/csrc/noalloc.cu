@@ -22,7 +22,7 @@
 namespace sd {
 namespace {
 
-constexpr size_t kStaticHeader = 256;
+constexpr size_t kStaticHeader = 4096;  // the workspace header's layout (status, scan counters)
 constexpr int kStaticMaxHeads = 64;                 // B * Hkv
 constexpr long long kStaticMaxScores = 1LL << 20;   // B * Hkv * N
 constexpr size_t kStaticHistBytes = (size_t)kStaticMaxHeads * 2048 * sizeof(uint32_t);

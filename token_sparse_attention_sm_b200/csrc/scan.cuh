@@ -33,10 +33,24 @@ constexpr int kScanStageBytes = 32768;
 constexpr int kScanThreads = (kScanConsumerWarps + 1) * 32;  // + the copy-issuing warp
 constexpr int kScanBins = 2048;  // top 11 bits of the order-preserving key
 
-// First tile of scan CTA c (tiles are dealt in contiguous runs).
+// The scan's tiles are dealt to its CTAs in contiguous runs: CTA c's run
+// starts at scan_tile_begin(c) (q = total / grid tiles each, the first
+// total % grid runs one more).
 __host__ __device__ inline long long scan_tile_begin(int c, long long total, int grid) {
-  return (long long)c * total / grid;
+  const long long q = total / grid, r = total % grid;
+  return (long long)c * q + (c < r ? c : r);
 }
+
+// Dynamic claiming of the runs' tiles.  Some SMs stream K measurably slower
+// than others (the same ones from call to call), so a static split leaves
+// the whole scan waiting for its slowest CTAs.  Each run has a claim counter
+// (the next tile of the run is run_begin + atomicAdd(counter, 1)); a CTA
+// claims from its own run first, then from the runs of the next
+// kScanStealSpan CTAs, always the one with the most tiles left.  The last CTA
+// to finish zeroes the counters for the next call.
+constexpr int kScanMaxCtas = 511;     // counters: [kScanMaxCtas + 1] words
+constexpr int kScanStealSpan = 8;     // runs a CTA may take tiles from after its own
+constexpr int kScanStealRounds = 4;   // probe rounds before a CTA gives up
 
 template <typename T, int D>
 struct ScoreCfg {
@@ -142,59 +156,89 @@ struct ScanOut {
   const float *tau;
 };
 
-// A CTA's walk over its tiles [t_begin, t_end) in ascending order, kept as
-// (head, tile of the head) and stepped without any division: the walk runs
-// once per tile in the copy-issuing thread, where a 64-bit division per tile
-// is enough to slow the stream down.
-struct TileWalk {
-  int bh, u, tph;
-  __device__ void init(long long b, int tiles_per_head) {
-    tph = tiles_per_head;
-    bh = (int)(b / tph);
-    u = (int)(b - (long long)bh * tph);
-  }
-  __device__ void next() {
-    if (++u == tph) {
-      u = 0;
-      ++bh;
-    }
-  }
-};
-
-// One CTA's share of the scan: tiles [t_begin, t_end).  K holds kv_rows rows
+// One CTA's share of the scan: its run of tiles [t_begin, t_end), then tiles
+// claimed from the runs after it (see kScanStealSpan).  K holds kv_rows rows
 // per (sequence, KV head), the first N of them scanned.  Warps 0..7 consume
 // (warp w in group w / 4, which takes the tiles in stages of its parity),
-// warp 8 produces: its lane 0 issues the copies and waits for the last ones
-// to land, its other lanes (and any further warps) return at once.  Barriers
-// full/empty must be initialised (count 1 / kScanGroupWarps).
+// warp 8 produces: its lane 0 claims the tiles, tells the consumers which
+// tile each stage holds (sinfo: head, tile of the head; head -1 ends a
+// group's loop) and issues the copies; its other lanes (and any further
+// warps) return at once.  ctr: the claim counters of the grid's runs, zero
+// on entry and left zero.  Barriers full/empty must be initialised (count 1
+// / kScanGroupWarps).
 template <typename T, int D, int kSlots, bool kMark = false>
 __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__restrict__ K,
                                            int N, int kv_rows, int Hq, int Hkv,
-                                           int tiles_per_head, long long t_begin, long long t_end,
-                                           int bh_first, float scale, unsigned char *ring,
-                                           uint64_t *full, uint64_t *empty, ScanOut o,
-                                           uint32_t *status) {
+                                           int tiles_per_head, long long total_tiles,
+                                           long long t_begin, long long t_end, int bh_first,
+                                           float scale, unsigned char *ring, uint64_t *full,
+                                           uint64_t *empty, int2 *sinfo, uint32_t *ctr,
+                                           ScanOut o, uint32_t *status) {
   const int nw = (N + 31) / 32;
   using C = ScoreCfg<T, D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntiles = (int)(t_end - t_begin);
   if (warp > kScanConsumerWarps) return;  // extra warps of a larger CTA idle here
   if (warp == kScanConsumerWarps) {
-    // ---- producer: one thread issues the bulk copies -------------------------
+    // ---- producer: one thread claims tiles and issues the bulk copies -------
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy();
-      TileWalk seq;
-      seq.init(t_begin, tiles_per_head);
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i, seq.next()) {
-        const int s = i % kScanStages;
-        if (i >= kScanStages &&
-            !mbar_wait(&empty[s], ((i / kScanStages) - 1) & 1, status))
+      const int grid = (int)gridDim.x, me = (int)blockIdx.x;
+      const long long rq = total_tiles / grid, rr = total_tiles % grid;
+      int victim = me;
+      long long vb = t_begin, vlen = t_end - t_begin;
+      uint32_t pend = atomicAdd(&ctr[victim], 1u);
+      int issued = 0, rounds = 0;
+      bool ok = true;
+      while (true) {
+        long long t = -1;
+        while (true) {
+          if ((long long)pend < vlen) {
+            t = vb + pend;
+            break;
+          }
+          // this run is exhausted: the next kScanStealSpan runs' counters,
+          // read all at once; claim from the one with the most tiles left
+          if (++rounds > kScanStealRounds) break;
+          uint32_t seen[kScanStealSpan];
+#pragma unroll
+          for (int j = 0; j < kScanStealSpan; ++j) {
+            const int v = (me + 1 + j) % grid;
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(seen[j]) : "l"(ctr + v)
+                         : "memory");
+          }
+          long long best_left = 0;
+          int best = -1;
+#pragma unroll
+          for (int j = 0; j < kScanStealSpan; ++j) {
+            const int v = (me + 1 + j) % grid;
+            if (v == me) continue;
+            const long long len = rq + (v < rr ? 1 : 0);
+            const long long left = len - (long long)seen[j];
+            if (left > best_left) {
+              best_left = left;
+              best = v;
+            }
+          }
+          if (best < 0) break;
+          victim = best;
+          vb = (long long)victim * rq + (victim < rr ? victim : rr);
+          vlen = rq + (victim < rr ? 1 : 0);
+          pend = atomicAdd(&ctr[victim], 1u);
+        }
+        if (t < 0) break;
+        pend = atomicAdd(&ctr[victim], 1u);  // the next claim, in flight while this tile is issued
+        const int s = issued % kScanStages;
+        if (issued >= kScanStages &&
+            !mbar_wait(&empty[s], ((issued / kScanStages) - 1) & 1, status)) {
+          ok = false;
           break;
-        const int bh = seq.bh;
-        const int j0 = seq.u * C::kStageKeys;
+        }
+        const int bh = (int)((unsigned long long)t / (unsigned)tiles_per_head);
+        const int u = (int)(t - (long long)bh * tiles_per_head);
+        const int j0 = u * C::kStageKeys;
         const int nk = min(C::kStageKeys, N - j0);
         const uint32_t bytes = (uint32_t)nk * C::kRowBytes;
+        sinfo[s] = make_int2(bh, u);
         mbar_arrive_expect_tx(&full[s], bytes);
         bulk_g2s(ring + (size_t)s * kScanStageBytes, K + ((size_t)bh * kv_rows + j0) * D,
                  bytes, &full[s], pol);
@@ -203,6 +247,17 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
       // Do not leave while copies may still be landing in shared memory.
       for (int i = max(0, issued - kScanStages); i < issued; ++i)
         mbar_wait(&full[i % kScanStages], (i / kScanStages) & 1, status);
+      // one end marker per consumer group
+      for (int e = 0, i = issued; e < kScanGroups && ok; ++e, ++i) {
+        const int s = i % kScanStages;
+        if (i >= kScanStages && !mbar_wait(&empty[s], ((i / kScanStages) - 1) & 1, status))
+          break;
+        sinfo[s] = make_int2(-1, 0);
+        mbar_arrive(&full[s]);
+      }
+      // every claim of this CTA has returned; the last CTA out resets the counters
+      if (atomicAdd(&ctr[grid], 1u) == (uint32_t)grid - 1u)
+        for (int v = 0; v <= grid; ++v) ctr[v] = 0u;
     }
     return;
   }
@@ -213,13 +268,14 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
   int cur_bh = -1;
   uint32_t tkey = 0;  // threshold marking: order key of the head's tau
   float qs[C::kEpl];
-  TileWalk seq;
-  seq.init(t_begin, tiles_per_head);
-  for (int i = 0; i < ntiles; ++i, seq.next()) {
+  for (int i = 0;; ++i) {
     const int s = i % kScanStages;
     if (s % kScanGroups != grp) continue;  // the other group's stage
-    const int bh = seq.bh;
-    const int j0 = seq.u * C::kStageKeys;
+    if (!mbar_wait(&full[s], (i / kScanStages) & 1, status)) break;
+    const int2 tile = sinfo[s];
+    if (tile.x < 0) break;  // the producer's end marker
+    const int bh = tile.x;
+    const int j0 = tile.y * C::kStageKeys;
     const int nk = min(C::kStageKeys, N - j0);
     if (bh != cur_bh) {
       cur_bh = bh;
@@ -230,7 +286,6 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
         if (!isfinite(tv) && lane == 0 && warp == 0) raise_flag(status, FLAG_NONFINITE);
       }
     }
-    if (!mbar_wait(&full[s], (i / kScanStages) & 1, status)) break;
     const unsigned char *stage = ring + (size_t)s * kScanStageBytes;
     float *Srow = kMark ? nullptr : o.S + (size_t)bh * N + j0;
     const int slot = bh - bh_first;
@@ -251,7 +306,7 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
           Srow[kk] = score;
           if (o.hist) {
             const uint32_t bin = key >> 21;
-            if (slot < kSlots)
+            if ((unsigned)slot < (unsigned)kSlots)
               atomicAdd(&o.shist[slot * kScanBins + bin], 1u);
             else
               atomicAdd(&o.hist[(size_t)bh * kScanBins + bin], 1u);

@@ -35,26 +35,25 @@ namespace sd {
 namespace {
 
 constexpr int kHistSlots = 2;  // heads a CTA can count in shared memory (later ones: global)
-constexpr int kScoreSmem =
-    kScanStages * kScanStageBytes + kHistSlots * kScanBins * 4 + 2 * kScanStages * 8;
+constexpr int kScoreSmem = kScanStages * kScanStageBytes + kHistSlots * kScanBins * 4 +
+                           2 * kScanStages * 8 + kScanStages * 8;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kScanThreads, 1)
     score_kernel(const T *__restrict__ q, const T *__restrict__ K,
                  float *__restrict__ S, int N, int kv_rows, int Hq, int Hkv,
                  int tiles_per_head, long long total_tiles, float scale,
-                 uint32_t *__restrict__ hist, uint32_t *status) {
+                 uint32_t *__restrict__ hist, uint32_t *ctr, uint32_t *status) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t *shist = reinterpret_cast<uint32_t *>(smem + kScanStages * kScanStageBytes);
   uint64_t *full = reinterpret_cast<uint64_t *>(
       smem + kScanStages * kScanStageBytes + kHistSlots * kScanBins * 4);
   uint64_t *empty = full + kScanStages;
+  int2 *sinfo = reinterpret_cast<int2 *>(empty + kScanStages);
 
   const long long t_begin = scan_tile_begin(blockIdx.x, total_tiles, gridDim.x);
   const long long t_end = scan_tile_begin(blockIdx.x + 1, total_tiles, gridDim.x);
-  const int ntiles = (int)(t_end - t_begin);
   const int bh_first = (int)(t_begin / tiles_per_head);
-  const int bh_last = ntiles > 0 ? (int)((t_end - 1) / tiles_per_head) : bh_first - 1;
 
   if (hist) {
     for (int i = threadIdx.x; i < kHistSlots * kScanBins; i += blockDim.x) shist[i] = 0u;
@@ -76,13 +75,17 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   o.shist = shist;
   o.bits = nullptr;
   o.tau = nullptr;
-  scan_tiles<T, D, kHistSlots, false>(q, K, N, kv_rows, Hq, Hkv, tiles_per_head, t_begin, t_end,
-                                      bh_first, scale, smem, full, empty, o, status);
+  scan_tiles<T, D, kHistSlots, false>(q, K, N, kv_rows, Hq, Hkv, tiles_per_head, total_tiles,
+                                      t_begin, t_end, bh_first, scale, smem, full, empty, sinfo,
+                                      ctr, o, status);
   if (threadIdx.x >= kScanConsumerWarps * 32) return;  // producer warp
   if (hist) {
     // consumer warps only (named barrier 1): every count is in shared memory
     asm volatile("bar.sync 1, %0;" ::"r"(kScanConsumerWarps * 32) : "memory");
-    const int nslots = min(kHistSlots, bh_last - bh_first + 1);
+    // every slot that names a head may hold counts: tiles of the head after
+    // this CTA's own run can be claimed from a neighbour's run
+    const int nheads = (int)(total_tiles / tiles_per_head);
+    const int nslots = min(kHistSlots, nheads - bh_first);
     for (int i = threadIdx.x; i < nslots * kScanBins; i += kScanConsumerWarps * 32) {
       const uint32_t c = shist[i];
       if (c) atomicAdd(&hist[(size_t)(bh_first + i / kScanBins) * kScanBins + (i % kScanBins)], c);
@@ -99,10 +102,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     threshold_mark_kernel(const T *__restrict__ q, const T *__restrict__ K,
                           const float *__restrict__ tau, uint32_t *__restrict__ bits, int N,
                           int kv_rows, int Hq, int Hkv, int tiles_per_head, long long total_tiles,
-                          float scale, uint32_t *status) {
+                          float scale, uint32_t *ctr, uint32_t *status) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kScanStages * kScanStageBytes);
   uint64_t *empty = full + kScanStages;
+  int2 *sinfo = reinterpret_cast<int2 *>(empty + kScanStages);
   const long long t_begin = scan_tile_begin(blockIdx.x, total_tiles, gridDim.x);
   const long long t_end = scan_tile_begin(blockIdx.x + 1, total_tiles, gridDim.x);
   if (threadIdx.x == 0) {
@@ -121,9 +125,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   o.shist = nullptr;
   o.bits = bits;
   o.tau = tau;
-  scan_tiles<T, D, kHistSlots, true>(q, K, N, kv_rows, Hq, Hkv, tiles_per_head, t_begin, t_end,
-                                     (int)(t_begin / tiles_per_head), scale, smem, full, empty, o,
-                                     status);
+  scan_tiles<T, D, kHistSlots, true>(q, K, N, kv_rows, Hq, Hkv, tiles_per_head, total_tiles,
+                                     t_begin, t_end, (int)(t_begin / tiles_per_head), scale, smem,
+                                     full, empty, sinfo, ctr, o, status);
 }
 
 template <typename T, int D>
@@ -133,13 +137,13 @@ cudaError_t launch_mark_t(const Shape &s, const void *q, const void *K, const fl
   DeviceInfo di;
   cudaError_t e = device_info(&di);
   if (e != cudaSuccess) return e;
-  constexpr int kSmem = kScanStages * kScanStageBytes + 2 * kScanStages * 8;
+  constexpr int kSmem = kScanStages * kScanStageBytes + 2 * kScanStages * 8 + kScanStages * 8;
   auto kern = threshold_mark_kernel<T, D>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   const int tiles_per_head = (s.N + C::kStageKeys - 1) / C::kStageKeys;
   const long long total = (long long)s.BH() * tiles_per_head;
-  const int grid = (int)(total < di.sm_count ? total : di.sm_count);
+  const int grid = scan_grid(s, di.sm_count);
   const float scale = (float)(1.0 / __builtin_sqrt((double)D));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
@@ -151,7 +155,8 @@ cudaError_t launch_mark_t(const Shape &s, const void *q, const void *K, const fl
   cfg.numAttrs = 0;
   add_pdl_attr(cfg, attrs);
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(q), static_cast<const T *>(K), tau,
-                         bits, s.N, s.Ncap, s.Hq, s.Hkv, tiles_per_head, total, scale, status);
+                         bits, s.N, s.Ncap, s.Hq, s.Hkv, tiles_per_head, total, scale,
+                         scan_counters(status), status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -180,7 +185,8 @@ cudaError_t launch_score_t(const Shape &s, const void *q, const void *K, float *
   cfg.numAttrs = 0;
   add_pdl_attr(cfg, attrs);
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(q), static_cast<const T *>(K), S,
-                         s.N, s.Ncap, s.Hq, s.Hkv, tiles_per_head, total, scale, hist, status);
+                         s.N, s.Ncap, s.Hq, s.Hkv, tiles_per_head, total, scale, hist,
+                         scan_counters(status), status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -214,7 +220,8 @@ int scan_grid(const Shape &s, int sm_count) {
   const int stage_keys = scan_stage_keys(s);
   const long long tph = (s.N + stage_keys - 1) / stage_keys;
   const long long total = (long long)s.BH() * tph;
-  return (int)(total < sm_count ? total : sm_count);
+  const int cap = sm_count < kScanMaxCtas ? sm_count : kScanMaxCtas;
+  return (int)(total < cap ? total : cap);
 }
 
 }  // namespace sd

@@ -315,16 +315,33 @@ __device__ __forceinline__ TsOut ts_select(const float *__restrict__ S, int N, u
   const int w_hi = (int)((long long)(rank + 1) * nw / nsplit);
   const int ow = w_hi - w_lo;
 
-  // the first words of the run are loaded before the histogram is read (the
-  // two latencies overlap)
-  constexpr int U = 16;  // words a warp has in flight
-  float sc[U];
+  // The run is read in blocks of 128 keys, lane l of a warp taking keys
+  // 4l .. 4l+3 of a block (one 16-byte load when the row is 16-byte aligned,
+  // which N % 4 == 0 makes true of every row).  The first blocks are loaded
+  // before the histogram is read (the two latencies overlap).
+  const int j_lo = 32 * w_lo, j_end = min(N, 32 * w_hi);
+  const int nblk = (ow + 3) / 4;
+  const bool vec = (N & 3) == 0;
+  constexpr int U = 4;  // blocks a warp has in flight
+  float sc[U][4];
+  auto load_blocks = [&](int b0) {
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int w = w_lo + warp + u * kTkWarps;
-    const int j = 32 * w + lane;
-    sc[u] = (w < w_hi && j < N) ? S[j] : 0.f;
-  }
+    for (int u = 0; u < U; ++u) {
+      const int j0 = j_lo + 128 * (b0 + u * kTkWarps) + 4 * lane;
+      if (vec) {
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j0 < j_end) f = *reinterpret_cast<const float4 *>(S + j0);
+        sc[u][0] = f.x;
+        sc[u][1] = f.y;
+        sc[u][2] = f.z;
+        sc[u][3] = f.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[u][e] = j0 + e < j_end ? S[j0 + e] : 0.f;
+      }
+    }
+  };
+  load_blocks(warp);
 
   // ---- 1. the boundary bin ------------------------------------------------------
   uint32_t tot;
@@ -333,6 +350,7 @@ __device__ __forceinline__ TsOut ts_select(const float *__restrict__ S, int N, u
   bool hist_ok = tot == (uint32_t)N && b1 != ~0u;
   bool fast = hist_ok && (nw + nsplit - 1) / nsplit <= kTsMaxWords;
   for (int i = tid; i < 2048 + 1024; i += kTkThreads) h2[i] = 0u;  // h3 follows h2
+  for (int i = tid; i < ow && fast; i += kTkThreads) bits[i] = 0u;
   if (tid == 0) {
     bk->nab = 0u;
     bk->nlist = 0u;
@@ -342,37 +360,51 @@ __device__ __forceinline__ TsOut ts_select(const float *__restrict__ S, int N, u
   if (fast) {
     // ---- 2. classify the run ----------------------------------------------------
     uint32_t nab = 0;
-    for (int w0 = w_lo + warp; w0 < w_hi; w0 += U * kTkWarps) {
-      if (w0 != w_lo + warp) {
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int w = w0 + u * kTkWarps;
-          const int j = 32 * w + lane;
-          sc[u] = (w < w_hi && j < N) ? S[j] : 0.f;
-        }
-      }
+    for (int b0 = warp; b0 < nblk; b0 += U * kTkWarps) {
+      if (b0 != warp) load_blocks(b0);
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const int w = w0 + u * kTkWarps;
-        if (w >= w_hi) break;  // warp-uniform
-        const int j = 32 * w + lane;
-        const bool valid = j < N;
-        const uint32_t key = order_key(sc[u]);
-        const uint32_t bin = key >> 21;
-        const bool up = valid && bin > b1;
-        const bool inb = valid && bin == b1;
-        const uint32_t upm = __ballot_sync(0xffffffffu, up);
-        const uint32_t inm = __ballot_sync(0xffffffffu, inb);
-        if (lane == 0) bits[w - w_lo] = upm;
-        if (up) sure((uint32_t)j);
-        nab += up ? 1u : 0u;
-        if (inm) {
+        const int blk = b0 + u * kTkWarps;
+        if (blk >= nblk) break;  // warp-uniform
+        const int j0 = j_lo + 128 * blk + 4 * lane;
+        uint32_t key[4], un = 0, inn = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          key[e] = order_key(sc[u][e]);
+          const bool valid = j0 + e < j_end;
+          const uint32_t bin = key[e] >> 21;
+          un |= (valid && bin > b1) ? 1u << e : 0u;
+          inn |= (valid && bin == b1) ? 1u << e : 0u;
+        }
+        if (un) {
+          // this lane's keys above the boundary bin: a nibble of the run's bitmap
+          sh_red_or(&bits[(j0 - j_lo) >> 5], un << (j0 & 31));
+          nab += (uint32_t)__popc(un);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if ((un >> e) & 1u) sure((uint32_t)(j0 + e));
+        }
+        const uint32_t c = (uint32_t)__popc(inn);
+        if (__any_sync(0xffffffffu, c != 0)) {
+          // boundary-bin keys join the list: one shared counter update per warp
+          uint32_t inc = c;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+          }
           uint32_t slot = 0;
-          if (lane == 0) slot = sh_atom_add(&bk->nlist, (uint32_t)__popc(inm));
-          slot = __shfl_sync(0xffffffffu, slot, 0) + (uint32_t)__popc(inm & ((1u << lane) - 1u));
-          if (inb && slot < (uint32_t)kTsOwnCap) {
-            show->lkey[slot] = key;
-            lidx[slot] = (uint32_t)j;
+          if (lane == 31) slot = sh_atom_add(&bk->nlist, inc);
+          slot = __shfl_sync(0xffffffffu, slot, 31) + inc - c;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if ((inn >> e) & 1u) {
+              if (slot < (uint32_t)kTsOwnCap) {
+                show->lkey[slot] = key[e];
+                lidx[slot] = (uint32_t)(j0 + e);
+              }
+              ++slot;
+            }
           }
         }
       }
