@@ -63,16 +63,15 @@
  * and returns without synchronising.
  *
  * Co-residency: no kernel of the library waits for a CTA that is not
- * already running.  The bf16 attention splits each head over up to 16 CTAs
- * that form one thread-block cluster (the hardware schedules a cluster's
- * CTAs together) and meet only at cluster barriers.  The routing scan's CTAs
- * never wait for one another: a CTA that finds a head's sample incomplete
- * when its own tiles are done marks that head's keys without a bound (every
- * key a candidate).  The Louver query, whose CTAs of a head meet at a
- * counter barrier in global memory, is launched cooperatively (the driver
- * then guarantees that the whole grid is resident) whenever a head spans
- * several CTAs.  So another kernel or process sharing the device can slow a
- * call down but cannot stall it.
+ * already running.  The top-k select and the bf16 attention split each head
+ * over up to 16 CTAs that form one thread-block cluster (the hardware
+ * schedules a cluster's CTAs together) and meet only at cluster barriers.
+ * The routing scan's CTAs never wait for one another: they claim tiles
+ * through counters (a CTA whose claims fail simply stops).  The Louver
+ * query, whose CTAs of a head meet at a counter barrier in global memory, is
+ * launched cooperatively (the driver then guarantees that the whole grid is
+ * resident) whenever a head spans several CTAs.  So another kernel or
+ * process sharing the device can slow a call down but cannot stall it.
  *
  * Environment variables read by the library:
  *   SPARSE_DECODE_PDL=0           no programmatic dependent launch between
@@ -398,6 +397,12 @@ sparse_status_t sparse_read_device_status(void *ws, void *stream,
  * step.  Returns SPARSE_ERR_INVALID_ARG for a NULL graph, SPARSE_ERR_CUDA if
  * the launch fails, else SPARSE_OK.  Does not synchronise. */
 sparse_status_t sparse_graph_launch(void *graph_exec, void *stream);
+
+/* Upload an instantiated CUDA graph's work to the device ahead of its first
+ * launch (cudaGraphUpload on `stream`), so that launch does not pay for it.
+ * Returns SPARSE_ERR_INVALID_ARG for a NULL graph, SPARSE_ERR_CUDA if the
+ * upload fails, else SPARSE_OK.  Runs nothing of the graph. */
+sparse_status_t sparse_graph_upload(void *graph_exec, void *stream);
 
 /* *usable = 1 when kernels can read and write p at its own address: device
  * memory, managed memory, or pinned host memory mapped into the device's

@@ -50,7 +50,7 @@ EXPORTED_SYMBOLS = (
     "sparse_louver_sizes", "sparse_louver_build", "sparse_louver_route_threshold",
     "sparse_selftest_bounded_wait", "sparse_louver_decode_step",
     "sparse_pointer_device_usable", "sparse_graph_launch", "sparse_decode_step_join",
-    "sparse_decode_step_fused",
+    "sparse_decode_step_fused", "sparse_graph_upload",
 )
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
@@ -121,6 +121,7 @@ def load():
                                                     SZ, P]),
             "sparse_pointer_device_usable": (I32, [P, ctypes.POINTER(I32)]),
             "sparse_graph_launch": (I32, [P, P]),
+            "sparse_graph_upload": (I32, [P, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -908,6 +909,14 @@ class DecodeStepGraph:
         if self.count_host is None:
             return self.out_host, self.idx_host
         return self.out_host, self.idx_host, self.count_host
+
+
+def graph_upload(graph, stream=None):
+    """Upload a captured torch.cuda.CUDAGraph's work to the device before its
+    first replay (sparse_graph_upload), on `stream` (default: current)."""
+    st = stream if stream is not None else torch.cuda.current_stream()
+    _check(load().sparse_graph_upload(ctypes.c_void_p(graph.raw_cuda_graph_exec()),
+                                      ctypes.c_void_p(st.cuda_stream)), "graph_upload")
 
 
 def louver_decode_step(q_route, q_layers, K, V, index: LouverIndex, tau, cap: int,

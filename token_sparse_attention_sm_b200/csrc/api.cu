@@ -564,6 +564,12 @@ sparse_status_t sparse_graph_launch(void *graph_exec, void *stream) {
                                        static_cast<cudaStream_t>(stream)));
 }
 
+sparse_status_t sparse_graph_upload(void *graph_exec, void *stream) {
+  if (!graph_exec) return SPARSE_ERR_INVALID_ARG;
+  return sd::from_cuda(cudaGraphUpload(static_cast<cudaGraphExec_t>(graph_exec),
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 sparse_status_t sparse_pointer_device_usable(const void *p, int32_t *usable) {
   if (!p || !usable) return SPARSE_ERR_INVALID_ARG;
   *usable = 0;

@@ -45,11 +45,13 @@ __host__ __device__ inline long long scan_tile_begin(int c, long long total, int
 // than others (the same ones from call to call), so a static split leaves
 // the whole scan waiting for its slowest CTAs.  Each run has a claim counter
 // (the next tile of the run is run_begin + atomicAdd(counter, 1)); a CTA
-// claims from its own run first, then from the runs of the next
-// kScanStealSpan CTAs, always the one with the most tiles left.  The last CTA
-// to finish zeroes the counters for the next call.
+// claims from its own run first, then from other runs: each probe round
+// reads the counters of kScanStealSpan runs spread evenly over the grid
+// (the slow CTAs come in blocks of neighbouring indices, so nearby runs are
+// the wrong place to look) and claims from the one with the most tiles
+// left.  The last CTA to finish zeroes the counters for the next call.
 constexpr int kScanMaxCtas = 511;     // counters: [kScanMaxCtas + 1] words
-constexpr int kScanStealSpan = 8;     // runs a CTA may take tiles from after its own
+constexpr int kScanStealSpan = 16;    // runs probed per round
 constexpr int kScanStealRounds = 4;   // probe rounds before a CTA gives up
 
 template <typename T, int D>
@@ -157,7 +159,7 @@ struct ScanOut {
 };
 
 // One CTA's share of the scan: its run of tiles [t_begin, t_end), then tiles
-// claimed from the runs after it (see kScanStealSpan).  K holds kv_rows rows
+// claimed from other runs (see kScanStealSpan).  K holds kv_rows rows
 // per (sequence, KV head), the first N of them scanned.  Warps 0..7 consume
 // (warp w in group w / 4, which takes the tiles in stages of its parity),
 // warp 8 produces: its lane 0 claims the tiles, tells the consumers which
@@ -196,21 +198,23 @@ __device__ __forceinline__ void scan_tiles(const T *__restrict__ q, const T *__r
             t = vb + pend;
             break;
           }
-          // this run is exhausted: the next kScanStealSpan runs' counters,
-          // read all at once; claim from the one with the most tiles left
+          // this run is exhausted: kScanStealSpan runs spread over the grid
+          // (shifted each round), their counters read all at once; claim
+          // from the one with the most tiles left
           if (++rounds > kScanStealRounds) break;
           uint32_t seen[kScanStealSpan];
+          int pv[kScanStealSpan];
 #pragma unroll
           for (int j = 0; j < kScanStealSpan; ++j) {
-            const int v = (me + 1 + j) % grid;
-            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(seen[j]) : "l"(ctr + v)
+            pv[j] = (me + rounds + j * grid / kScanStealSpan) % grid;
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(seen[j]) : "l"(ctr + pv[j])
                          : "memory");
           }
           long long best_left = 0;
           int best = -1;
 #pragma unroll
           for (int j = 0; j < kScanStealSpan; ++j) {
-            const int v = (me + 1 + j) % grid;
+            const int v = pv[j];
             if (v == me) continue;
             const long long len = rq + (v < rr ? 1 : 0);
             const long long left = len - (long long)seen[j];
