@@ -459,9 +459,13 @@ def run_native(args, rank, world, local_rank):
     achieved = scan_b / (t_score_max * 1e-3) / 1e9
     trec = traffic_record(SCORE_SOURCES)
     line = {
-        "metric": METRIC,
+        "metric": METRIC if w.name == "decode_128k" else (
+            "sparse decode steps/s on %s (B=%d, N=%d, %d layers, k=%d); HBM GB/s vs roofline"
+            % (w.name, w.B, w.N, w.L, w.k)),
         "value": round(value, 2),
         "unit": "steps/s",
+        # a step decodes one token of each of the B sequences
+        **({"tokens_per_s": round(value * w.B, 2)} if w.B > 1 else {}),
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,

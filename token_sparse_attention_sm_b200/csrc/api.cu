@@ -206,7 +206,8 @@ cudaError_t decode_step_enqueue(const Shape &s, int L, const void *q_route,
     e = launch_score(s, q_route, K, S, hist, status, st);
     if (e == cudaSuccess) e = join();
     if (e == cudaSuccess)
-      e = launch_route_attn_topk(s, L, q_layers, K, V, k, S, hist, idx, out, lse, status, st);
+      e = launch_route_attn_topk(s, L, q_layers, K, V, k, S, hist, idx, out, lse, attn_ptr(ws, l),
+                                 status, st);
     return e;
   }
   if (!topk && fused) {
@@ -215,7 +216,7 @@ cudaError_t decode_step_enqueue(const Shape &s, int L, const void *q_route,
     if (e == cudaSuccess) e = join();
     if (e == cudaSuccess)
       e = launch_route_attn_threshold(s, L, q_layers, K, V, bits, cap, idx, count, out, lse,
-                                      status, st);
+                                      attn_ptr(ws, l), status, st);
     return e;
   }
   if (topk) {

@@ -244,7 +244,7 @@ cudaError_t launch_attn_t(const Shape &s, int L, const void *q, const void *K,
 }  // namespace
 
 size_t attn_workspace_bytes(const Shape &s, int L, int stride) {
-  if (s.dtype == 1) return 0;  // the tcgen05 kernel merges its splits on chip
+  if (s.dtype == 1) return attn_fused_workspace_bytes(s, L, stride);
   const int Mtot = L * s.G();
   const int qblocks = (Mtot + kQPerCta - 1) / kQPerCta;
   const int nsplit = num_splits(s.BH(), qblocks, stride);
@@ -256,7 +256,7 @@ cudaError_t launch_attn(const Shape &s, int L, const void *q, const void *K,
                         const int *count, int count_cap, void *out, float *lse,
                         void *ws, uint32_t *status, cudaStream_t st) {
   if (s.dtype == 1)
-    return launch_attn_fused(s, L, q, K, V, idx, stride, count, out, lse, status, st);
+    return launch_attn_fused(s, L, q, K, V, idx, stride, count, out, lse, ws, status, st);
   if (s.d == 128)
     return launch_attn_t<float, 128>(s, L, q, K, V, idx, stride, count, count_cap,
                                      out, lse, ws, status, st);

@@ -56,8 +56,6 @@
 // Every mbarrier wait is bounded; on expiry the kernel raises the TIMEOUT
 // flag, stops issuing work, still meets its cluster barriers, frees its
 // tensor memory and returns.
-#include <cooperative_groups.h>
-
 #include <atomic>
 
 #include "common.cuh"
@@ -66,8 +64,6 @@
 
 namespace sd {
 namespace {
-
-namespace cg = cooperative_groups;
 
 constexpr int kFuThreads = kTkThreads;  // 512: 16 warps, 4 per TMEM lane quadrant
 constexpr int kGroups = 4;              // warps sharing a tensor-memory lane quadrant
@@ -78,6 +74,7 @@ constexpr int kChunkKeys = kTileN * kChunkTiles;
 constexpr int kTmemCols = 256;          // S (128 columns) + O (d <= 128 columns)
 constexpr int kMaxSplits = 16;
 constexpr int kMaxPer = 2048;           // keys of one split held on chip (routing modes)
+constexpr int kFuSlotBound = 512;       // CTA slots the split count may spread a head block over
 static_assert(kMaxSplits == kTsMaxSplits, "a head's cluster is the select's cluster");
 constexpr int kMaxDevices = 64;
 
@@ -98,23 +95,19 @@ struct FuCfg {
   static constexpr int kAttnBytes = kVOff + kVBytes;
   static constexpr int kSelBytes = (int)ts_scratch_bytes();
   static constexpr int kBigBytes = cmax_i(kAttnBytes, kSelBytes);
-  static constexpr int kStageBytes = kRows * (D + 4) * 4;  // merge partials
-  static_assert(kStageBytes <= kBigBytes, "merge staging fits");
   // small area: barriers, TMEM slot, select bookkeeping, row reductions,
-  // validity flags, chunk indices, the split's indices, the partial (max,
-  // sum) pairs from the peers, and what the select shows its peers
+  // validity flags, chunk indices, the split's indices, and what the select
+  // shows its peers
   static constexpr int kSmallOff = (kBigBytes + 1023) / 1024 * 1024;
   static constexpr int kBarsOff = 0, kTmemSlotOff = 64, kTkOff = 128, kXredOff = 512;
   static constexpr int kKvalOff = kXredOff + kGroups * 128 * 4;
   static constexpr int kCidxOff = kKvalOff + kChunkKeys;
   static constexpr int kSidxOff = kCidxOff + kChunkKeys * 4;
-  static constexpr int kMlOff = kSidxOff + kMaxPer * 4;  // [kMaxSplits][kRows] float2 from peers
-  static constexpr int kShowOff = kMlOff + kMaxSplits * kRows * 8;
+  static constexpr int kShowOff = kSidxOff + kMaxPer * 4;
   static constexpr int kBookOff = kShowOff + (int)sizeof(TsShow);
   static constexpr int kSmallBytes = kBookOff + (int)sizeof(TsBook);
-  // merge scratch after the staged partials: [kFuThreads] float4 + [kFuThreads] float
-  static constexpr int kRedOff = (kStageBytes + 15) / 16 * 16;
-  static_assert(kRedOff + kFuThreads * 20 <= kBigBytes, "merge scratch fits");
+  // merge scratch in the (then free) tile buffers: [kFuThreads] float4 + [kFuThreads] float
+  static_assert(kFuThreads * 20 <= kBigBytes, "merge scratch fits");
   static constexpr int kSmem = kSmallOff + kSmallBytes + 1024;  // + alignment slack
   static_assert(sizeof(TkSmall) <= kXredOff - kTkOff, "select bookkeeping fits");
 };
@@ -197,11 +190,6 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Prefetch `bytes` (a multiple of 16, 16-byte aligned) into L2.
-__device__ __forceinline__ void l2_prefetch(const void *p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // 2^x with the hardware approximation (ex2.approx.ftz: relative error about
 // 2^-22, results below 2^-126 flush to zero -- harmless for softmax weights).
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -237,6 +225,7 @@ struct FuArgs {
   uint32_t *hist;        // top-k: the scan's histograms (cleared here)
   const uint32_t *bits;  // threshold: the marking scan's bitmaps
   int k_or_cap;
+  float *part;           // several splits: their partials, fu_workspace_bytes()
 };
 
 enum : int { kModeIdx = 0, kModeTopk = 1, kModeThresh = 2 };
@@ -301,20 +290,13 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
   bool from_peers = false;  // the split's keys are read from their owners' lists
   int *orow = a.idx + (size_t)bh * a.stride;
   if constexpr (kMode == kModeTopk) {
-    // keys known to be in the set early are prefetched into L2 by the CTA
-    // that will gather them, so the gather below finds its rows there
-    const size_t head_rows = (size_t)bh * a.kv_rows * D;
-    auto sure = [&](uint32_t j) {
-      l2_prefetch(a.K + head_rows + (size_t)j * D, D * 2);
-      l2_prefetch(a.V + head_rows + (size_t)j * D, D * 2);
-    };
     auto emit = [&](uint32_t i, uint32_t pos, uint32_t j) {
       sidx[i] = (int)j;
       if (qb == 0) orow[pos] = (int)j;
     };
     const TsOut part = ts_select(a.S + (size_t)bh * N, N, (uint32_t)a.k_or_cap,
                                  a.hist + (size_t)bh * kHistBins, rank, nsplit, kMaxPer, base,
-                                 show, book, tks, a.status, emit, sure);
+                                 show, book, tks, a.status, emit);
     __syncthreads();  // the split's indices are on chip; the select's scratch is free
     if (part.split && nsplit > 1) {
       // the runs hold unequal parts of the set: every CTA attends over an
@@ -636,13 +618,18 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
     return;
   }
 
-  // Several splits: stage (O, max, sum) of the real rows in shared memory
-  // (the tile buffers are free now), [row][D + 4] fp32, and give every peer
-  // this split's (max, sum) of every row before the cluster barrier.
-  constexpr int PR = D + 4;
-  float *stage = reinterpret_cast<float *>(base);
-  float2 *ml_recv = reinterpret_cast<float2 *>(small + C::kMlOff);  // [split][row]
+  // Several splits: each writes its partial (O, max, sum) of the real rows
+  // to the workspace -- [split][row][D] fp32, then [split][row] (max, sum)
+  // -- one cluster barrier (release / acquire at cluster scope) makes them
+  // visible to the head's CTAs, and each CTA merges a share of the rows by
+  // log-sum-exp, reading the partials from L2.  No CTA reads another's
+  // shared memory after the barrier, so none waits for another to finish.
+  float *pbase = a.part + (size_t)(bh * gridDim.y + qb) * nsplit * C::kRows * (D + 2);
+  const float2 *pml = reinterpret_cast<const float2 *>(pbase + (size_t)nsplit * C::kRows * D);
   if (live) {
+    // tcgen05.ld is warp-collective: every lane of a live warp loads (have
+    // and live are warp-uniform); only the stores depend on the lane's row
+    float *dst = pbase + ((size_t)rank * C::kRows + row) * D + grp * (D / kGroups);
 #pragma unroll
     for (int cb = 0; cb < D / kGroups / 16; ++cb) {
       uint32_t r[16];
@@ -651,10 +638,9 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
         tmem_wait_ld();
       }
       if (row < mrows) {
-        float *dst = stage + row * PR + grp * (D / kGroups) + cb * 16;
 #pragma unroll
         for (int i = 0; i < 16; i += 4)
-          *reinterpret_cast<float4 *>(dst + i) =
+          *reinterpret_cast<float4 *>(dst + cb * 16 + i) =
               have ? make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
                                  __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]))
                    : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -666,7 +652,8 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
     float ls = 0.f;
 #pragma unroll
     for (int g = 0; g < kGroups; ++g) ls += xsum[g * 128 + row];
-    *reinterpret_cast<float2 *>(stage + row * PR + D) = make_float2(have ? mrun : -INFINITY, ls);
+    reinterpret_cast<float2 *>(pbase + (size_t)nsplit * C::kRows * D)[rank * C::kRows + row] =
+        make_float2(have ? mrun : -INFINITY, ls);
   }
   // tensor memory is no longer needed
   tc_fence_before();
@@ -676,22 +663,16 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)
                  : "memory");
-  cg::cluster_group cluster = cg::this_cluster();
-  for (int t = tid; t < nsplit * mrows; t += kFuThreads) {
-    const int peer = t / mrows, r = t % mrows;
-    cl_st2(cl_addr(ml_recv + rank * C::kRows + r, peer),
-           *reinterpret_cast<const float2 *>(stage + r * PR + D));
-  }
-  cluster.sync();  // every split's partial is staged and its (max, sum) delivered
+  cluster_sync_all();  // every split's partial is in the workspace
   if constexpr (kMode == kModeTopk) {
     if (rank == 0)
       for (int i = tid; i < kHistBins; i += kFuThreads) a.hist[(size_t)bh * kHistBins + i] = 0u;
   }
   // merge rows lr = rank, rank + nsplit, ...: thread = (peer group q, row
-  // slot, float4 chunk); the weights come from the (max, sum) pairs on chip,
-  // each thread reads its peers' partial O through distributed shared
-  // memory (all loads in flight), and with several peer groups the group
-  // partials are added in shared memory.
+  // slot, float4 chunk); every (max, sum) pair and the thread's peers'
+  // partial O are loaded at once (L2 only: they were written by other SMs
+  // during this kernel), and with several peer groups the group partials
+  // are added in shared memory (the tile buffers are free now).
   {
     constexpr int CH = D / 4;
     const int nrows = (mrows - rank + nsplit - 1) / nsplit;
@@ -699,38 +680,53 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
     while (qg < 4 && qg * 2 <= nsplit && nrows * CH * qg * 2 <= kFuThreads) qg *= 2;
     const int rpq = kFuThreads / (CH * qg);  // row slots per pass
     const int ch = tid % CH, slot = (tid / CH) % rpq, q = tid / (CH * rpq);
-    float4 *red = reinterpret_cast<float4 *>(base + C::kRedOff);
-    float *red_ls = reinterpret_cast<float *>(base + C::kRedOff + kFuThreads * 16);
+    float4 *red = reinterpret_cast<float4 *>(base);
+    float *red_ls = reinterpret_cast<float *>(base + kFuThreads * 16);
     for (int i0 = 0; i0 < nrows; i0 += rpq) {
       const int i = i0 + slot;
       const int lr = rank + i * nsplit;
       const bool mine = i < nrows;
       float mx = -INFINITY, ls = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (mine) {
-        for (int r = 0; r < nsplit; ++r) mx = fmaxf(mx, ml_recv[r * C::kRows + lr].x);
-        if (mx != -INFINITY) {
-          // this thread's peers q, q + qg, ..., four loads in flight at a time
-          for (int r0 = q; r0 < nsplit; r0 += 4 * qg) {
-            float4 v[4];
+      // the CH lanes of a row slot (CH >= kMaxSplits) each load one split's
+      // (max, sum) pair and share them by shuffles
+      float2 mlv = make_float2(-INFINITY, 0.f);
+      if (mine && ch < nsplit) mlv = __ldcg(pml + ch * C::kRows + lr);
+      float4 v[4];  // this thread's first peers' partial O, in flight with the pairs
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int r = r0 + u * qg;
-              if (r < nsplit) v[u] = cl_ld4(cl_addr(stage + lr * PR + ch * 4, r));
-            }
+      for (int u = 0; u < 4; ++u) {
+        const int r = q + u * qg;
+        if (mine && r < nsplit)
+          v[u] = __ldcg(reinterpret_cast<const float4 *>(
+              pbase + ((size_t)r * C::kRows + lr) * D + ch * 4));
+      }
+      mx = mlv.x;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int r = r0 + u * qg;
-              if (r < nsplit) {
-                const float2 ml = ml_recv[r * C::kRows + lr];
-                const float w = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - mx);
-                ls += ml.y * w;
-                acc.x += w * v[u].x;
-                acc.y += w * v[u].y;
-                acc.z += w * v[u].z;
-                acc.w += w * v[u].w;
-              }
-            }
+      for (int o = CH / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o, CH));
+      // this thread's peers q, q + qg, ..., four loads in flight at a time
+      for (int r0 = q; r0 < nsplit; r0 += 4 * qg) {
+        if (r0 != q) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int r = r0 + u * qg;
+            if (mine && r < nsplit)
+              v[u] = __ldcg(reinterpret_cast<const float4 *>(
+                  pbase + ((size_t)r * C::kRows + lr) * D + ch * 4));
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = r0 + u * qg;
+          // every lane of the row slot takes part in the shuffles
+          const float mr = __shfl_sync(0xffffffffu, mlv.x, r & (CH - 1), CH);
+          const float lr_sum = __shfl_sync(0xffffffffu, mlv.y, r & (CH - 1), CH);
+          if (mine && r < nsplit && mx != -INFINITY) {
+            const float w = mr == -INFINITY ? 0.f : fast_exp2(mr - mx);
+            ls += lr_sum * w;
+            acc.x += w * v[u].x;
+            acc.y += w * v[u].y;
+            acc.z += w * v[u].z;
+            acc.w += w * v[u].w;
           }
         }
       }
@@ -763,7 +759,6 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
       }
     }
   }
-  cluster.sync();  // no CTA leaves while another reads its partial
 }
 
 // The kernel's dynamic shared memory, with the whole unified L1/shared
@@ -842,6 +837,7 @@ template <int D, bool kHalf>
 int fu_splits(long long blocks, int max_keys, bool routed, int sm_count) {
   const int slots = sm_count * (kHalf ? 2 : 1);
   long long want = slots / blocks;
+  if (want > (kFuSlotBound + blocks - 1) / blocks) want = (kFuSlotBound + blocks - 1) / blocks;
   const int by_keys = (max_keys + kTileN - 1) / kTileN;
   if (want > by_keys) want = by_keys;
   if (want > kMaxSplits) want = kMaxSplits;
@@ -911,7 +907,7 @@ cudaError_t launch_fu(const FuArgs &a, const Shape &s, int max_keys, cudaStream_
 }
 
 FuArgs fu_base(const Shape &s, int L, const void *q, const void *K, const void *V, int *idx,
-               int stride, int *count, void *out, float *lse, uint32_t *status) {
+               int stride, int *count, void *out, float *lse, uint32_t *status, void *part) {
   FuArgs a{};
   a.q = static_cast<const __nv_bfloat16 *>(q);
   a.K = static_cast<const __nv_bfloat16 *>(K);
@@ -929,16 +925,35 @@ FuArgs fu_base(const Shape &s, int L, const void *q, const void *K, const void *
   a.out = static_cast<__nv_bfloat16 *>(out);
   a.lse = lse;
   a.status = status;
+  a.part = static_cast<float *>(part);
   return a;
 }
 
 }  // namespace
 
+size_t attn_fused_workspace_bytes(const Shape &s, int L, int stride) {
+  // the split count is at most kMaxSplits, one split per kTileN keys and,
+  // beyond what the on-chip capacity forces, kFuSlotBound slots over the
+  // head blocks (fu_splits keeps to the same bound)
+  const int M = L * s.G();
+  const int qblocks = M <= 64 ? 1 : (M + 127) / 128;
+  const int rows = M <= 64 ? 64 : 128;
+  const long long blocks = (long long)s.BH() * qblocks;
+  long long ns = (kFuSlotBound + blocks - 1) / blocks;
+  const long long by_keys = (stride + kTileN - 1) / kTileN;
+  if (ns > by_keys) ns = by_keys;
+  const long long need = (stride + kMaxPer - 1) / kMaxPer;
+  if (ns < need) ns = need;
+  if (ns > kMaxSplits) ns = kMaxSplits;
+  if (ns < 2) return 0;  // one split: no partials
+  return (size_t)blocks * ns * rows * (s.d + 2) * sizeof(float);
+}
+
 cudaError_t launch_attn_fused(const Shape &s, int L, const void *q, const void *K, const void *V,
                               const int *idx, int stride, const int *count, void *out, float *lse,
-                              uint32_t *status, cudaStream_t st) {
+                              void *part, uint32_t *status, cudaStream_t st) {
   FuArgs a = fu_base(s, L, q, K, V, const_cast<int *>(idx), stride, const_cast<int *>(count), out,
-                     lse, status);
+                     lse, status, part);
   return launch_fu<kModeIdx>(a, s, stride, st);
 }
 
@@ -949,9 +964,9 @@ bool fused_route_ok(const Shape &s, int L, int k_or_cap) {
 
 cudaError_t launch_route_attn_topk(const Shape &s, int L, const void *q_layers, const void *K,
                                    const void *V, int k, const float *S, uint32_t *hist,
-                                   int *idx, void *out, float *lse, uint32_t *status,
-                                   cudaStream_t st) {
-  FuArgs a = fu_base(s, L, q_layers, K, V, idx, k, nullptr, out, lse, status);
+                                   int *idx, void *out, float *lse, void *part,
+                                   uint32_t *status, cudaStream_t st) {
+  FuArgs a = fu_base(s, L, q_layers, K, V, idx, k, nullptr, out, lse, status, part);
   a.S = S;
   a.hist = hist;
   a.k_or_cap = k;
@@ -961,8 +976,8 @@ cudaError_t launch_route_attn_topk(const Shape &s, int L, const void *q_layers, 
 cudaError_t launch_route_attn_threshold(const Shape &s, int L, const void *q_layers,
                                         const void *K, const void *V, const uint32_t *bits,
                                         int cap, int *idx, int *count, void *out, float *lse,
-                                        uint32_t *status, cudaStream_t st) {
-  FuArgs a = fu_base(s, L, q_layers, K, V, idx, cap, count, out, lse, status);
+                                        void *part, uint32_t *status, cudaStream_t st) {
+  FuArgs a = fu_base(s, L, q_layers, K, V, idx, cap, count, out, lse, status, part);
   a.bits = bits;
   a.k_or_cap = cap;
   return launch_fu<kModeThresh>(a, s, cap, st);

@@ -74,29 +74,31 @@ cudaError_t launch_select(const Shape &s, const float *S, int k,
                           cudaStream_t st);
 
 // A3 + A4: L query sets over the same index rows.  bf16 runs on the tcgen05
-// tensor cores (attn_fused.cu, no workspace); fp32 on the CUDA cores with
-// split partials in the workspace (attn.cu).
+// tensor cores (attn_fused.cu), fp32 on the CUDA cores (attn.cu); both keep
+// their split partials in the workspace (attn_workspace_bytes).
 size_t attn_workspace_bytes(const Shape &s, int L, int stride);
+size_t attn_fused_workspace_bytes(const Shape &s, int L, int stride);
 cudaError_t launch_attn(const Shape &s, int L, const void *q, const void *K,
                         const void *V, const int *idx, int stride,
                         const int *count, int count_cap, void *out, float *lse,
                         void *ws, uint32_t *status, cudaStream_t st);
 cudaError_t launch_attn_fused(const Shape &s, int L, const void *q, const void *K, const void *V,
                               const int *idx, int stride, const int *count, void *out, float *lse,
-                              uint32_t *status, cudaStream_t st);
+                              void *part, uint32_t *status, cudaStream_t st);
 // The tail of routing fused into the attention kernel (bf16, L*G <= 128,
 // N <= 131072, every split's keys on chip): top-k from the scan's score rows
 // and histogram (writes idx [B*Hkv][k], clears hist), or the threshold sets
 // from the marking scan's bitmaps (writes idx rows of `cap` and count).
 bool fused_route_ok(const Shape &s, int L, int k_or_cap);
+// part: the workspace's attention area (attn_workspace_bytes).
 cudaError_t launch_route_attn_topk(const Shape &s, int L, const void *q_layers, const void *K,
                                    const void *V, int k, const float *S, uint32_t *hist,
-                                   int *idx, void *out, float *lse, uint32_t *status,
+                                   int *idx, void *out, float *lse, void *part, uint32_t *status,
                                    cudaStream_t st);
 cudaError_t launch_route_attn_threshold(const Shape &s, int L, const void *q_layers,
                                         const void *K, const void *V, const uint32_t *bits,
                                         int cap, int *idx, int *count, void *out, float *lse,
-                                        uint32_t *status, cudaStream_t st);
+                                        void *part, uint32_t *status, cudaStream_t st);
 
 // Louver index (louver.cu).  louver_shape_ok: r and N fit the balanced tree.
 bool louver_shape_ok(const Shape &s, int r);

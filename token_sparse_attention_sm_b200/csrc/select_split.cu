@@ -33,10 +33,9 @@ __global__ void __launch_bounds__(kTkThreads, 1)
   auto emit = [&](uint32_t, uint32_t pos, uint32_t j) {
     if (pos < (uint32_t)k) out[pos] = (int)j;
   };
-  TkNoSure no_hook;
   uint32_t *h = hist + (size_t)bh * kHistBins;
   ts_select(S + (size_t)bh * N, N, (uint32_t)k, h, rank, nsplit, (uint32_t)k, smem_raw, show,
-            book, sm, status, emit, no_hook);
+            book, sm, status, emit);
   // no CTA leaves while a peer may still read its list, and the histogram
   // is cleared only after every CTA is done with it
   if (nsplit > 1)

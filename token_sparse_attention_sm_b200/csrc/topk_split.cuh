@@ -12,10 +12,9 @@
 //  1. The histogram gives the boundary bin b1 where the descending count
 //     reaches k: every key above b1 is in, every key below it out.  Every
 //     CTA reads it.
-//  2. Each CTA reads its run once (one coalesced 128-byte load per warp and
-//     word): the keys above b1 go into an on-chip bitmap of the run (and to
-//     the `sure` hook, e.g. to prefetch their rows), the keys in b1 onto an
-//     on-chip list whose order keys the peers may read.
+//  2. Each CTA reads its run once (16-byte loads, four keys per lane): the
+//     keys above b1 go into an on-chip bitmap of the run, the keys in b1 onto
+//     an on-chip list whose order keys the peers may read.
 //  3. One cluster barrier.  Every CTA reads the peers' counts and copies all
 //     of their lists through distributed shared memory: the whole boundary
 //     bin, a few thousand keys, lands in every CTA.
@@ -274,11 +273,6 @@ __device__ __forceinline__ uint32_t tk_bitmap_emit(const uint32_t *bits, int nwo
   return total;
 }
 
-// A no-op for ts_select's `sure` hook.
-struct TkNoSure {
-  __device__ void operator()(uint32_t) const {}
-};
-
 // This CTA's part of the set: positions [lo, lo + n).
 struct TsOut {
   uint32_t lo, n;
@@ -292,18 +286,17 @@ struct TsOut {
 // shared memory; show, bk, sm: this CTA's shared structures.  max_own: the
 // most keys the caller can take in one CTA on the fast path (the fallback's
 // equal share, ceil(k / nsplit), must not exceed it).  Calls emit(i, pos, j)
-// for the CTA's i-th key j at position pos of the set (i = pos - lo), and
-// sure(j) for keys known to be selected as soon as that is known.  On the
+// for the CTA's i-th key j at position pos of the set (i = pos - lo).  On the
 // fast path (split) the CTA's part is its run's keys and bk->part_lo holds
 // every CTA's first position (and k after the last).  Every
 // thread of every CTA of the cluster must call it; it contains one cluster
 // barrier (on the fast path, which the whole cluster takes or leaves).
-template <typename Emit, typename Sure>
+template <typename Emit>
 __device__ __forceinline__ TsOut ts_select(const float *__restrict__ S, int N, uint32_t k,
                                            const uint32_t *__restrict__ hist, int rank,
                                            int nsplit, uint32_t max_own, unsigned char *scratch,
                                            TsShow *show, TsBook *bk, TkSmall *sm,
-                                           uint32_t *status, Emit &emit, Sure &sure) {
+                                           uint32_t *status, Emit &emit) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t *bits = reinterpret_cast<uint32_t *>(scratch);  // the run's words
   uint32_t *lidx = bits + kTsMaxWords;                     // own list: key indices
@@ -350,7 +343,6 @@ __device__ __forceinline__ TsOut ts_select(const float *__restrict__ S, int N, u
   bool hist_ok = tot == (uint32_t)N && b1 != ~0u;
   bool fast = hist_ok && (nw + nsplit - 1) / nsplit <= kTsMaxWords;
   for (int i = tid; i < 2048 + 1024; i += kTkThreads) h2[i] = 0u;  // h3 follows h2
-  for (int i = tid; i < ow && fast; i += kTkThreads) bits[i] = 0u;
   if (tid == 0) {
     bk->nab = 0u;
     bk->nlist = 0u;
@@ -376,35 +368,37 @@ __device__ __forceinline__ TsOut ts_select(const float *__restrict__ S, int N, u
           un |= (valid && bin > b1) ? 1u << e : 0u;
           inn |= (valid && bin == b1) ? 1u << e : 0u;
         }
-        if (un) {
-          // this lane's keys above the boundary bin: a nibble of the run's bitmap
-          sh_red_or(&bits[(j0 - j_lo) >> 5], un << (j0 & 31));
-          nab += (uint32_t)__popc(un);
+        // the run's bitmap word of keys 32 g .. 32 g + 31 of the block is the
+        // nibbles of lanes 8 g .. 8 g + 7: one reduction per group of 8 lanes,
+        // one plain store
+        const uint32_t grp8 = 0xffu << (lane & 24);
+        const uint32_t word = __reduce_or_sync(grp8, un << (j0 & 31));
+        if ((lane & 7) == 0 && j0 < j_end) bits[(j0 - j_lo) >> 5] = word;
+        nab += (uint32_t)__popc(un);
+        // boundary-bin keys join the list, ordered by nibble bit then lane:
+        // four ballots give every entry its slot, one shared counter update
+        // per warp gives the warp's base
+        uint32_t m[4], tot4 = 0;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if ((un >> e) & 1u) sure((uint32_t)(j0 + e));
+        for (int e = 0; e < 4; ++e) {
+          m[e] = __ballot_sync(0xffffffffu, (inn >> e) & 1u);
+          tot4 += (uint32_t)__popc(m[e]);
         }
-        const uint32_t c = (uint32_t)__popc(inn);
-        if (__any_sync(0xffffffffu, c != 0)) {
-          // boundary-bin keys join the list: one shared counter update per warp
-          uint32_t inc = c;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += y;
-          }
-          uint32_t slot = 0;
-          if (lane == 31) slot = sh_atom_add(&bk->nlist, inc);
-          slot = __shfl_sync(0xffffffffu, slot, 31) + inc - c;
+        if (tot4) {
+          uint32_t base = 0;
+          if (lane == 0) base = sh_atom_add(&bk->nlist, tot4);
+          base = __shfl_sync(0xffffffffu, base, 0);
+          const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            if ((inn >> e) & 1u) {
+            if ((m[e] >> lane) & 1u) {
+              const uint32_t slot = base + (uint32_t)__popc(m[e] & lt);
               if (slot < (uint32_t)kTsOwnCap) {
                 show->lkey[slot] = key[e];
                 lidx[slot] = (uint32_t)(j0 + e);
               }
-              ++slot;
             }
+            base += (uint32_t)__popc(m[e]);
           }
         }
       }
