@@ -93,8 +93,10 @@ struct FuCfg {
   static constexpr int kKPOff = kQBytes;
   static constexpr int kVOff = kKPOff + kKPBytes;
   static constexpr int kAttnBytes = kVOff + kVBytes;
+  // the select's scratch sits after Q (whose copy starts before the select)
+  static constexpr int kSelOff = kQBytes;
   static constexpr int kSelBytes = (int)ts_scratch_bytes();
-  static constexpr int kBigBytes = cmax_i(kAttnBytes, kSelBytes);
+  static constexpr int kBigBytes = cmax_i(kAttnBytes, kSelOff + kSelBytes);
   // small area: barriers, TMEM slot, select bookkeeping, row reductions,
   // validity flags, chunk indices, the split's indices, and what the select
   // shows its peers
@@ -278,6 +280,25 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The query block (rows beyond M zero) into its swizzled tile.  In the
+  // routing modes the kernel before this one on the stream is the routing
+  // scan, which never writes the queries and released this launch only once
+  // every kernel before it had finished: the copy starts before the wait for
+  // the scan, in a copy group of its own.
+  auto issue_q = [&]() {
+    for (int p = tid; p < C::kRows * CPR; p += kFuThreads) {
+      const int r = p / CPR, c = p % CPR;
+      const int m = qb * 128 + r;
+      const __nv_bfloat16 *qr = nullptr;
+      if (m < M) qr = a.q + (((size_t)(m / G) * B + b) * Hq + (size_t)h * G + m % G) * D;
+      const uint32_t dst = q_s + (c >> 3) * C::kQCb + swz(r, c & 7);
+      cp_async16(dst, qr ? qr + c * 8 : a.q, qr != nullptr);
+    }
+  };
+  if constexpr (kMode != kModeIdx) {
+    issue_q();
+    cp_async_commit();
+  }
   grid_dep_wait();  // sets, scores, bitmaps and queries come from earlier kernels
   grid_dep_launch();
   const uint32_t tmem = *tmem_slot;
@@ -295,8 +316,8 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
       if (qb == 0) orow[pos] = (int)j;
     };
     const TsOut part = ts_select(a.S + (size_t)bh * N, N, (uint32_t)a.k_or_cap,
-                                 a.hist + (size_t)bh * kHistBins, rank, nsplit, kMaxPer, base,
-                                 show, book, tks, a.status, emit);
+                                 a.hist + (size_t)bh * kHistBins, rank, nsplit, kMaxPer,
+                                 base + C::kSelOff, show, book, tks, a.status, emit);
     __syncthreads();  // the split's indices are on chip; the select's scratch is free
     if (part.split && nsplit > 1) {
       // the runs hold unequal parts of the set: every CTA attends over an
@@ -390,17 +411,7 @@ __global__ void __launch_bounds__(kFuThreads, kHalf ? 2 : 1)
         cix = cidx;
       }
     }
-    if (c0 == 0) {
-      // the query block (rows beyond M zero), in the same copy group as K
-      for (int p = tid; p < C::kRows * CPR; p += kFuThreads) {
-        const int r = p / CPR, c = p % CPR;
-        const int m = qb * 128 + r;
-        const __nv_bfloat16 *qr = nullptr;
-        if (m < M) qr = a.q + (((size_t)(m / G) * B + b) * Hq + (size_t)h * G + m % G) * D;
-        const uint32_t dst = q_s + (c >> 3) * C::kQCb + swz(r, c & 7);
-        cp_async16(dst, qr ? qr + c * 8 : a.q, qr != nullptr);
-      }
-    }
+    if (c0 == 0 && kMode == kModeIdx) issue_q();  // in the same copy group as K
     // gather the chunk's K rows, then its V rows (two async-copy groups)
     for (int p = tid; p < ntile * kTileN * CPR; p += kFuThreads) {
       const int r = p / CPR, c = p % CPR;

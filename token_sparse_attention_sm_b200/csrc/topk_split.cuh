@@ -108,19 +108,19 @@ __device__ __forceinline__ uint32_t tk_scan(uint32_t x, TkSmall *sm, uint32_t *t
   return r;
 }
 
-// The bin of histogram h (NB bins, read highest first) where the descending
-// count reaches need: sm->bnd = {bin, keys above it, keys in it}, or bnd[0] =
-// ~0 when the histogram holds fewer than need keys.  *total = its sum.
+// The bin of a histogram of NB bins, read highest first, where the
+// descending count reaches need: sm->bnd = {bin, keys above it, keys in it},
+// or bnd[0] = ~0 when the histogram holds fewer than need keys; *total = its
+// sum.  This thread's bins come already loaded: c[e] = bin NB - 1 -
+// (NB / 512 * t + e) (so the loads can be issued ahead of other work).
 template <int NB>
-__device__ __forceinline__ void tk_boundary(const uint32_t *h, uint32_t need, TkSmall *sm, uint32_t *total) {
+__device__ __forceinline__ void tk_boundary_of(const uint32_t (&c)[NB / kTkThreads], uint32_t need,
+                                               TkSmall *sm, uint32_t *total) {
   constexpr int BPT = NB / kTkThreads;
   const int t = threadIdx.x;
-  uint32_t c[BPT], sum = 0;
+  uint32_t sum = 0;
 #pragma unroll
-  for (int e = 0; e < BPT; ++e) {
-    c[e] = h[NB - 1 - (BPT * t + e)];
-    sum += c[e];
-  }
+  for (int e = 0; e < BPT; ++e) sum += c[e];
   if (t == 0) sm->bnd[0] = ~0u;
   uint32_t above = tk_scan(sum, sm, total);  // its barriers order the write above
   if (above < need && above + sum >= need) {
@@ -136,6 +136,16 @@ __device__ __forceinline__ void tk_boundary(const uint32_t *h, uint32_t need, Tk
     }
   }
   __syncthreads();
+}
+
+// The same, reading histogram h.
+template <int NB>
+__device__ __forceinline__ void tk_boundary(const uint32_t *h, uint32_t need, TkSmall *sm, uint32_t *total) {
+  constexpr int BPT = NB / kTkThreads;
+  uint32_t c[BPT];
+#pragma unroll
+  for (int e = 0; e < BPT; ++e) c[e] = h[NB - 1 - (BPT * threadIdx.x + e)];
+  tk_boundary_of<NB>(c, need, sm, total);
 }
 
 // Where the k-th key lies: every key with key >= t_ge is selected, plus the
@@ -334,11 +344,16 @@ __device__ __forceinline__ TsOut ts_select(const float *__restrict__ S, int N, u
       }
     }
   };
+  // the histogram's bins first (the boundary needs them first), then the
+  // run's first blocks
+  uint32_t hb[2048 / kTkThreads];
+#pragma unroll
+  for (int e = 0; e < 2048 / kTkThreads; ++e) hb[e] = hist[2047 - (2048 / kTkThreads * tid + e)];
   load_blocks(warp);
 
   // ---- 1. the boundary bin ------------------------------------------------------
   uint32_t tot;
-  tk_boundary<2048>(hist, k, sm, &tot);
+  tk_boundary_of<2048>(hb, k, sm, &tot);
   const uint32_t b1 = sm->bnd[0], above1 = sm->bnd[1], cb1 = sm->bnd[2];
   bool hist_ok = tot == (uint32_t)N && b1 != ~0u;
   bool fast = hist_ok && (nw + nsplit - 1) / nsplit <= kTsMaxWords;
