@@ -317,14 +317,16 @@ SCORE_SOURCES = [os.path.join(ROOT, "token_sparse_attention_sm_b200", "csrc", n)
                  for n in ("score.cu", "scan.cuh")]
 
 
-def traffic_record(files):
+def traffic_record(files, workload: str = "decode_128k"):
     """ncu DRAM bytes per launch of the dominant kernel, valid only while the
-    kernel source is unchanged since the capture."""
+    kernel source is unchanged since the capture and for the workload it was
+    captured on."""
     path = os.path.join(ROOT, "profiles", "score_kernel_traffic.txt")
     try:
         with open(path) as f:
             rec = json.load(f)
-        if rec.get("source_sha256") == kernel_source_sha(files):
+        if (rec.get("source_sha256") == kernel_source_sha(files)
+                and rec.get("workload", "").split(" ")[0] == workload):
             return rec
     except Exception:
         pass
@@ -457,7 +459,7 @@ def run_native(args, rank, world, local_rank):
     peak, peak_src = load_peaks()
     scan_b, gath_b = algorithmic_bytes(w)
     achieved = scan_b / (t_score_max * 1e-3) / 1e9
-    trec = traffic_record(SCORE_SOURCES)
+    trec = traffic_record(SCORE_SOURCES, w.name)
     line = {
         "metric": METRIC if w.name == "decode_128k" else (
             "sparse decode steps/s on %s (B=%d, N=%d, %d layers, k=%d); HBM GB/s vs roofline"

@@ -736,8 +736,9 @@ class DecodeStepGraph:
     routing scan, then one select + attention kernel) it writes the set (and
     counts) there too (``results_direct``), so nothing is copied back; on
     separate routing and attention kernels the set travels back on the second
-    stream while the attention runs.  Without a mapping, outputs and set are
-    copied back together after the attention.  With ``index`` (a LouverIndex
+    stream while the attention runs.  Without a mapping (or with
+    ``host_writes=False``), outputs and set are copied back together after
+    the attention.  With ``index`` (a LouverIndex
     of K) and threshold mode the step routes through the index.  ``replay()`` enqueues a step on ``stream`` (a new stream by
     default; graphs that share a workspace must use one stream),
     ``synchronize()`` waits for it, calling the object does both.  The device
@@ -756,7 +757,8 @@ class DecodeStepGraph:
 
     def __init__(self, K, V, L: int, Hq: int, k: int | None = None, tau=None,
                  cap: int | None = None, ws: Workspace | None = None, n: int | None = None,
-                 stream=None, index: "LouverIndex | None" = None):
+                 stream=None, index: "LouverIndex | None" = None,
+                 host_writes: bool = True):
         _need_cuda(K, V, tau)
         dev = K.device
         B, Hkv, _, d = K.shape
@@ -807,7 +809,9 @@ class DecodeStepGraph:
                 route_threshold(q_route, K, tau, cap, ws=self.ws, check=False, n=n, idx=idx,
                                 count=count)
 
-        self.mapped_out = device_usable(self.out_host)
+        # host_writes=False: kernels write only device memory, and every
+        # result comes back by one copy after the step
+        self.mapped_out = host_writes and device_usable(self.out_host)
         out_dst = self.out_host if self.mapped_out else out
         # on the fused kernels the step only writes its set, counts and
         # outputs: with mapped host buffers all of them go straight to the host
