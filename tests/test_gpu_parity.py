@@ -411,6 +411,29 @@ def test_route_topk_recovers_from_dirty_workspace(dev, route_path):
         assert int(ws.buf[a:b].sum()) == 0
 
 
+def test_scan_claim_counters_left_zero(dev):
+    """The routing scan claims its tiles through counters in the workspace
+    header ([1024, 3072)); every scan, top-k or threshold marking, long or
+    short, leaves them zero for the next call, and the next call still sees
+    every tile (its scores equal a fresh workspace's)."""
+    ws = sd.Workspace(dev)
+    for N, B, Hkv in ((131072, 1, 8), (5000, 2, 2), (300, 3, 8), (70000, 1, 1)):
+        w = synth.custom(B=B, N=N, Hq=4 * Hkv, Hkv=Hkv, d=128, L=1, k=min(100, N), dtype="bf16",
+                         seed=N)
+        x = synth.generate(w)
+        t = _to(dev, x)
+        idx = sd.route_topk(t["q_route"], t["K"], w.k, ws=ws)
+        torch.cuda.synchronize()
+        assert int(ws.buf[1024:3072].view(torch.int32).abs().sum()) == 0, N
+        tau = torch.zeros((B, Hkv), device=dev)
+        sd.route_threshold(t["q_route"], t["K"], tau, N, ws=ws)
+        torch.cuda.synchronize()
+        assert int(ws.buf[1024:3072].view(torch.int32).abs().sum()) == 0, N
+        again = sd.route_topk(t["q_route"], t["K"], w.k, ws=ws)
+        fresh = sd.route_topk(t["q_route"], t["K"], w.k, ws=sd.Workspace(dev))
+        assert torch.equal(again, idx) and torch.equal(again, fresh)
+
+
 @pytest.mark.parametrize("k,count", [(4096, None), (8192, [3933, 4100, 100, 0, 8192, 2, 3000, 7000])])
 def test_attn_gather_many_keys_per_cta(dev, k, count):
     """More selected keys than one on-chip chunk per CTA: the running max is

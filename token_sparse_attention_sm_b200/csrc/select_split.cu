@@ -19,7 +19,9 @@ constexpr size_t kSelSmallOff = kSelBookOff + sizeof(TsBook);
 constexpr size_t kSelSmem = kSelSmallOff + sizeof(TkSmall);
 constexpr int kSelMaxDevices = 64;
 
-__global__ void __launch_bounds__(kTkThreads, 1)
+// Two CTAs per SM (64 registers a thread): with one, only 7 clusters of 16
+// are resident at once, and an 8th head waits for a second wave.
+__global__ void __launch_bounds__(kTkThreads, 2)
     select_split_kernel(const float *__restrict__ S, int N, int k, int *__restrict__ idx,
                         uint32_t *__restrict__ hist, uint32_t *status) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
