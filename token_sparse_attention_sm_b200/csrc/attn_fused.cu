@@ -41,11 +41,11 @@
 //     significant bits) into swizzled shared memory over the dead K tiles.
 //  4. One thread issues O += P_hi V + P_lo V into tensor memory.
 // A running maximum rescales O between chunks.  With one split the CTA
-// normalises O and writes the output; with several, each CTA leaves its
-// partial (O, max, sum) in its shared memory, and after a cluster barrier
-// each merges a share of the rows by log-sum-exp, reading every split's
-// partial through distributed shared memory.  Only hardware cluster barriers
-// join the CTAs, so no CTA ever waits for one that is not resident.
+// normalises O and writes the output; with several, each CTA writes its
+// partial (O, max, sum) to the workspace, and after a cluster barrier each
+// merges a share of the rows by log-sum-exp, reading every split's partial
+// from L2.  Only hardware cluster barriers join the CTAs, so no CTA ever
+// waits for one that is not resident.
 //
 // Query blocks of at most 64 rows (L*G <= 64, the usual decode shape) keep
 // only the 64 real rows of Q and P on chip: the MMA still reads 128 rows, and
