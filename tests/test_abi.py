@@ -205,6 +205,10 @@ def test_graph_launch_rejects_null(lib):
     assert lib.sparse_graph_launch(None, None) == 1
 
 
+def test_graph_upload_rejects_null(lib):
+    assert lib.sparse_graph_upload(None, None) == 1
+
+
 def test_result_and_tau_checks_reject_bad_tensors(lib):
     """Caller-given results must match exactly and live where kernels can
     write them; tau needs one float per row of the sets.  All checked before
